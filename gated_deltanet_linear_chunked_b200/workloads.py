@@ -1,0 +1,178 @@
+"""Seeded synthetic workloads for the GDN scan (numpy only).
+
+This module only draws random inputs; it holds none of the scan's arithmetic
+and imports nothing from the library or from the oracle, so tests, the
+benchmark and the oracle can all take their inputs from it.
+
+Shapes follow the pages' streaming workload: 1280x704 frames under a 32x
+spatial latent give 40 x 22 = 880 tokens per latent frame (DCAE-V, F32T4C32:
+SANA-Video blog "SANA-Video视频生成领域的效率革命", 3.2 多分辨率VAE设计), and a
+streaming chunk is three
+latent frames ("SANA-Streaming：基于混合扩散Transformer的实时流式视频编辑系统",
+方法步骤详情, second step), i.e. 2640 tokens; the DiT has 15 GDN blocks
+(same page, 核心方法).  Heads are 112 wide (SANA-Video-2B, same blog,
+3.1 模型架构配置); 20 heads is the workload's stated head count.
+
+Every (batch, head) pair draws from its own generator, seeded with
+``[seed, b, h]``, in the fixed order q, k, v, gate, beta, so any single head
+can be regenerated without drawing the rest.  Values are drawn in fp32 and,
+for bf16 workloads, rounded to the nearest bf16 (ties to even) so that the
+fp32 arrays returned hold exactly the values a bf16 tensor stores.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Iterator
+
+import numpy as np
+
+TOKENS_PER_LATENT_FRAME = 40 * 22  # 1280/32 x 704/32
+FRAMES_PER_CHUNK = 3
+CHUNK_TOKENS = FRAMES_PER_CHUNK * TOKENS_PER_LATENT_FRAME  # 2640
+GDN_LAYERS = 15
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """One scan call's shape and input distributions."""
+    name: str
+    B: int
+    T: int
+    H: int
+    Dk: int
+    Dv: int
+    dtype: str            # "f32" or "bf16": dtype of q, k, v and out
+    chunk: int            # sub-chunk length handed to the library
+    mode: str             # "fwd" or "bidir"
+    gate: tuple           # ("neg_softplus",) or ("uniform", lo, hi): g = log decay
+    beta: tuple           # ("sigmoid",) or ("const", value)
+    state: tuple          # ("zero",) or ("normal", std)
+    seed: int
+
+    @property
+    def head_tokens(self) -> int:
+        return self.B * self.H * self.T
+
+
+def tiny() -> Workload:
+    """Tiny causal scan, fp32: B1 H2 d16 T64, sub-chunk 16, zero state."""
+    return Workload("tiny_causal_f32", 1, 64, 2, 16, 16, "f32", 16, "fwd",
+                    ("neg_softplus",), ("sigmoid",), ("zero",), 1)
+
+
+def stream_chunk(mode: str = "fwd", seed: int | None = None) -> Workload:
+    """One 1280x704 streaming chunk: B1 H20 d112 T2640 bf16, sub-chunk 64,
+    g ~ U[-0.5, 0], beta = sigmoid(N(0,1)), state_in ~ N(0, 0.02^2)."""
+    if seed is None:
+        seed = 2 if mode == "fwd" else 3
+    name = "stream_chunk_causal" if mode == "fwd" else "stream_chunk_bidir"
+    return Workload(name, 1, CHUNK_TOKENS, 20, 112, 112, "bf16", 64, mode,
+                    ("uniform", -0.5, 0.0), ("sigmoid",), ("normal", 0.02), seed)
+
+
+def stack_call(layer: int, chunk_index: int, mode: str = "bidir") -> Workload:
+    """Chunk `chunk_index` of GDN layer `layer` in the 32-chunk x 15-layer
+    stream; the state is carried per layer (zero before chunk 0)."""
+    w = stream_chunk(mode, seed=1000 + 37 * layer + chunk_index)
+    return dataclasses.replace(w, name=f"stack_l{layer}_c{chunk_index}", state=("zero",))
+
+
+STRESS_DIMS = (64, 128)
+STRESS_LENGTHS = (256, 4096, 65536)
+STRESS_GATES = (("uniform", -1e-4, 0.0), ("uniform", -8.0, -4.0))
+STRESS_BETAS = (0.01, 0.99)
+
+
+def stress_cases() -> list[Workload]:
+    """24 stress cases: B4 H16, d in {64,128}, T in {256,4096,65536}, bf16,
+    near-identity (g in [-1e-4,0]) or fast (g in [-8,-4]) decay, constant
+    beta in {0.01, 0.99}, state_in ~ N(0, 0.02^2)."""
+    cases = []
+    i = 0
+    for d in STRESS_DIMS:
+        for T in STRESS_LENGTHS:
+            for gate in STRESS_GATES:
+                for b in STRESS_BETAS:
+                    tag = "slow" if gate[1] > -1.0 else "fast"
+                    cases.append(Workload(f"stress_d{d}_T{T}_{tag}_b{b}", 4, T, 16, d, d,
+                                          "bf16", 64, "fwd", gate, ("const", b),
+                                          ("normal", 0.02), 5000 + i))
+                    i += 1
+    return cases
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round fp32 values to the nearest bf16 (ties to even); returns fp32."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    u = x.view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
+    return u.astype(np.uint32).view(np.float32)
+
+
+def _l2_rows(x: np.ndarray) -> np.ndarray:
+    # Part of the input recipe ("q, k ~ N(0,1), then L2-normalised"); the
+    # library normalises again itself, so this only shapes the stored values.
+    return (x / np.linalg.norm(x, axis=-1, keepdims=True)).astype(np.float32)
+
+
+def make_head(w: Workload, b: int, h: int) -> dict:
+    """Inputs of one (batch, head) pair: q, k [T,Dk]; v [T,Dv]; g, beta [T]."""
+    rng = np.random.default_rng([w.seed, b, h])
+    q = _l2_rows(rng.standard_normal((w.T, w.Dk), dtype=np.float32))
+    k = _l2_rows(rng.standard_normal((w.T, w.Dk), dtype=np.float32))
+    v = rng.standard_normal((w.T, w.Dv), dtype=np.float32)
+    if w.gate[0] == "neg_softplus":
+        z = rng.standard_normal(w.T, dtype=np.float32).astype(np.float64)
+        g = -np.logaddexp(0.0, z)
+    elif w.gate[0] == "uniform":
+        lo, hi = w.gate[1], w.gate[2]
+        g = lo + (hi - lo) * rng.random(w.T, dtype=np.float64)
+    else:
+        raise ValueError(w.gate)
+    g = np.minimum(g.astype(np.float32), np.float32(0.0))
+    if w.beta[0] == "sigmoid":
+        z = rng.standard_normal(w.T, dtype=np.float32).astype(np.float64)
+        beta = (1.0 / (1.0 + np.exp(-z))).astype(np.float32)
+    elif w.beta[0] == "const":
+        beta = np.full(w.T, w.beta[1], dtype=np.float32)
+    else:
+        raise ValueError(w.beta)
+    if w.dtype == "bf16":
+        q, k, v = round_bf16(q), round_bf16(k), round_bf16(v)
+    return {"q": q, "k": k, "v": v, "g": g, "beta": beta}
+
+
+def make_state(w: Workload) -> np.ndarray | None:
+    """state_in [B,H,Dk,Dv] fp32, or None for a zero state."""
+    if w.state[0] == "zero":
+        return None
+    rng = np.random.default_rng([w.seed, 0x57A7E])
+    return (w.state[1] * rng.standard_normal((w.B, w.H, w.Dk, w.Dv))).astype(np.float32)
+
+
+def iter_heads(w: Workload) -> Iterator[tuple[int, int, dict]]:
+    for b in range(w.B):
+        for h in range(w.H):
+            yield b, h, make_head(w, b, h)
+
+
+def make_inputs(w: Workload) -> dict:
+    """All inputs in the library's layouts, fp32 numpy (bf16-exact for bf16
+    workloads): q, k [B,T,H,Dk]; v [B,T,H,Dv]; g, beta [B,T,H]; state_in."""
+    q = np.empty((w.B, w.T, w.H, w.Dk), np.float32)
+    k = np.empty_like(q)
+    v = np.empty((w.B, w.T, w.H, w.Dv), np.float32)
+    g = np.empty((w.B, w.T, w.H), np.float32)
+    beta = np.empty_like(g)
+    for b, h, d in iter_heads(w):
+        q[b, :, h], k[b, :, h], v[b, :, h] = d["q"], d["k"], d["v"]
+        g[b, :, h], beta[b, :, h] = d["g"], d["beta"]
+    return {"q": q, "k": k, "v": v, "g": g, "beta": beta, "state_in": make_state(w)}
+
+
+def slice_head(inputs: dict, b: int, h: int) -> dict:
+    """One head of `make_inputs` output, shaped [1,T,1,D] for a B=H=1 call."""
+    out = {n: np.ascontiguousarray(inputs[n][b:b + 1, :, h:h + 1]) for n in ("q", "k", "v", "g", "beta")}
+    s = inputs.get("state_in")
+    out["state_in"] = None if s is None else np.ascontiguousarray(s[b:b + 1, h:h + 1])
+    return out

@@ -1,0 +1,131 @@
+/*
+ * gdn.h -- C ABI of libgdn.so: the chunked Gated DeltaNet (GDN) scan of the
+ * GDN blocks of SANA-Streaming's hybrid diffusion Transformer, on sm_100a.
+ *
+ * The operation.  Per batch row b and head h the scan carries a state
+ * S (Dk x Dv, fp32) through the gated delta rule
+ *
+ *     q^_t = q_t / sqrt(max(|q_t|^2, 1e-12)),   k^_t likewise
+ *     S_t  = a_t (I - beta_t k^_t k^_t^T) S_{t-1} + beta_t k^_t v_t^T,
+ *     o_t  = S_t^T q^_t,                        a_t = exp(g_t), g_t <= 0.
+ *
+ * The pages describe GDN only in words: a fixed-size memory updated
+ * recursively from the previous state ("[논문리뷰] SANA-Streaming: Real-time
+ * Streaming Video Editing with Hybrid Diffusion Transformer", 1. Key Terms &
+ * Definitions).  Streaming runs a forward scan that starts from the previous
+ * chunk's cache, and the streaming model adds a backward scan inside the chunk
+ * ("SANA-Streaming：基于混合扩散Transformer的实时流式视频编辑系统",
+ * 方法步骤详情, second and fourth steps; the fourth names the fused kernel's
+ * three stages: frame summaries, recurrent scan, state application).
+ *
+ * Layouts (row-major, contiguous, element strides implied by the sizes):
+ *   q, k       [B, T, H, Dk]   dtype (GDN_F32: float, GDN_BF16: bf16)
+ *   v, out     [B, T, H, Dv]   dtype
+ *   g, beta    [B, T, H]       float   (g <= 0 is the log of the decay a_t;
+ *                                       beta in [0, 1])
+ *   state      [B, H, Dk, Dv]  float
+ *
+ * Ownership.  The caller owns every buffer; all pointers are device (or
+ * managed) pointers.  The library keeps no pointer after a call returns.
+ * Internal scratch, when a path needs it, is allocated and freed
+ * stream-ordered on `stream` (cudaMallocAsync / cudaFreeAsync).
+ *
+ * Execution.  Work is enqueued on `stream` (a cudaStream_t; NULL is the
+ * legacy default stream) and the call returns without synchronising;
+ * results are stream-ordered.  No call throws, aborts or prints.
+ *
+ * Errors.  Arguments are validated on the host before anything is enqueued;
+ * on any error nothing is launched and a status is returned:
+ *   GDN_ERR_INVALID_ARG  null pointer where data is needed, negative size,
+ *                        pointer not 16-byte aligned, host (pageable or
+ *                        pinned) pointer, unknown dtype, bad chunk value
+ *   GDN_ERR_UNSUPPORTED  Dk or Dv not a multiple of 16 in [16, 128]
+ *   GDN_ERR_ALIAS        out overlaps an input or the state; state_out
+ *                        overlaps an input or partially overlaps state_in
+ *   GDN_ERR_CUDA         a CUDA runtime call or a launch failed
+ *   GDN_ERR_TIMEOUT      a kernel's bounded wait expired (reported by
+ *                        gdn_device_error, or by the calls themselves when
+ *                        the environment sets GDN_DEBUG_SYNC=1)
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GDN_OK = 0,
+  GDN_ERR_INVALID_ARG = 1,
+  GDN_ERR_UNSUPPORTED = 2,
+  GDN_ERR_ALIAS = 3,
+  GDN_ERR_CUDA = 4,
+  GDN_ERR_TIMEOUT = 5
+} gdn_status;
+
+typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
+
+/*
+ * Causal (forward) scan of one streaming chunk with a carried state.
+ *
+ * state_in   previous chunk's final state, or NULL for a zero state.
+ * state_out  receives the final state; may equal state_in (in place);
+ *            may be NULL when the caller does not need it.
+ * out        receives o_t for every token, in `dtype`.
+ * chunk      sub-chunk length the kernels tile time with: 0 (default, 64),
+ *            16, 32 or 64.  It changes rounding only, never the result's
+ *            definition.  The fp32 path scans token by token and ignores it.
+ * T == 0     is allowed: state_out = state_in (or zero), out is untouched.
+ * B == 0 or H == 0 is allowed and does nothing.
+ */
+gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v,
+                         const float* g, const float* beta,
+                         const float* state_in, float* state_out, void* out,
+                         int B, int T, int H, int Dk, int Dv, gdn_dtype dtype,
+                         int chunk, void* stream);
+
+/*
+ * Bidirectional scan of one chunk: out = (forward scan from state_in) +
+ * (the same recurrence over the time-reversed chunk from a zero state, each
+ * token keeping its own g_t and beta_t), summed per token.  state_out is the
+ * forward scan's final state.  Arguments as for gdn_chunk_fwd.
+ */
+gdn_status gdn_chunk_bidir(const void* q, const void* k, const void* v,
+                           const float* g, const float* beta,
+                           const float* state_in, float* state_out, void* out,
+                           int B, int T, int H, int Dk, int Dv,
+                           gdn_dtype dtype, int chunk, void* stream);
+
+/*
+ * Zero a state [B, H, Dk, Dv] (streaming restart: the state is the only thing
+ * a stream keeps, "SANA-Streaming：基于混合扩散Transformer的实时流式视频编辑系统",
+ * 前置知识, 流式生成).  Any positive Dk, Dv are accepted here.
+ */
+gdn_status gdn_state_reset(float* state, int B, int H, int Dk, int Dv,
+                           void* stream);
+
+/*
+ * Synchronise `stream`, then read and clear the device error word that
+ * kernels set when a bounded wait expires.  Returns GDN_OK, GDN_ERR_TIMEOUT
+ * or GDN_ERR_CUDA.
+ */
+gdn_status gdn_device_error(void* stream);
+
+/*
+ * Test hook: the number of polls a kernel's bounded wait makes before it
+ * gives up (0 restores the default).  Affects launches enqueued after the
+ * call, on every device.  Returns the previous value.
+ */
+long long gdn_set_wait_limit(long long polls);
+
+/* Static, human-readable name of a status; never NULL. */
+const char* gdn_status_string(gdn_status status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

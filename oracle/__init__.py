@@ -1,0 +1,28 @@
+"""CPU oracle for the chunked Gated DeltaNet (GDN) scan.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+the CPU-baseline leg of ``bench.py`` may import, call, link or run anything
+in this package.  The product path (``gated_deltanet_linear_chunked_b200``)
+never does, and the two share no code: they meet only through the seeded
+input generators, which hold none of the method's arithmetic.
+
+Contents
+  * ``cpu``        -- ctypes front end of ``gdn_oracle.c``: the token-by-token
+                      recurrence in double (and long double), threaded over
+                      (batch, head).  The reference for every parity test.
+  * ``numpy_ref``  -- the same recurrence in numpy (a second, independent
+                      transcription for tiny cases) and the chunked (WY / UT)
+                      form of the scan in fp64, used only to pin that the
+                      chunked algebra reaches the recurrence exactly.
+
+Parity is pinned, not assumed: ``tests/test_oracle_pins.py`` checks these
+functions against closed forms, invariants, a hand-derived example and brute
+force (see each test's docstring).
+"""
+from .cpu import build, online_cores, oracle_bidir, oracle_fwd  # noqa: F401
+from .numpy_ref import (  # noqa: F401
+    chunked_bidir,
+    chunked_fwd,
+    recurrence_bidir,
+    recurrence_fwd,
+)

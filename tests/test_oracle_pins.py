@@ -1,0 +1,392 @@
+"""Pins for the CPU oracle (no GPU).
+
+The pages print no numeric example of the scan, so the oracle is pinned to
+things other than itself: a hand-derived example, closed forms for special
+gates, invariants of the delta rule, and brute force (the chunked WY form, an
+independent algorithm, must reach the token recurrence).  Each pin is chosen
+so that a plausible slip in the oracle (a dropped term, a wrong sign, the
+decay on the wrong factor, a transposed state, the projection on the wrong
+side, a missing normalisation) fails at least one of them.
+
+Both transcriptions of the definition are pinned: the C oracle (double and
+long double) and the numpy recurrence.
+"""
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from gated_deltanet_linear_chunked_b200 import workloads as wl
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def c_fwd(q, k, v, g, beta, s=None):
+    return oracle.oracle_fwd(q, k, v, g, beta, s, nthreads=2)
+
+
+def c_bidir(q, k, v, g, beta, s=None):
+    return oracle.oracle_bidir(q, k, v, g, beta, s, nthreads=2)
+
+
+FWD = {"c": c_fwd, "numpy": oracle.recurrence_fwd}
+BIDIR = {"c": c_bidir, "numpy": oracle.recurrence_bidir}
+
+
+def rand_inputs(rng, B=2, T=23, H=3, Dk=8, Dv=6, g_lo=-1.0, unit=False):
+    q = rng.standard_normal((B, T, H, Dk)).astype(np.float32)
+    k = rng.standard_normal((B, T, H, Dk)).astype(np.float32)
+    if unit:
+        q /= np.linalg.norm(q, axis=-1, keepdims=True)
+        k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((B, T, H, Dv)).astype(np.float32)
+    g = rng.uniform(g_lo, 0.0, (B, T, H)).astype(np.float32)
+    beta = rng.uniform(0.0, 1.0, (B, T, H)).astype(np.float32)
+    s = (0.3 * rng.standard_normal((B, H, Dk, Dv))).astype(np.float64)
+    return q, k, v, g, beta, s
+
+
+def unit(x):
+    x = np.asarray(x, np.float64)
+    return x / np.linalg.norm(x, axis=-1, keepdims=True)
+
+
+def rel(a, b):
+    return np.max(np.abs(np.asarray(a, np.float64) - np.asarray(b, np.float64))) / max(
+        np.max(np.abs(np.asarray(b, np.float64))), 1e-300)
+
+
+def load_golden(name):
+    vals = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, rhs = line.split("=", 1)
+            rows = [[float(x) for x in r.split()] for r in rhs.split(";")]
+            vals[key.strip()] = np.array(rows)
+    return vals
+
+
+# --------------------------------------------------------------- hand example
+@pytest.mark.parametrize("impl", ["c", "numpy"])
+def test_hand_derived_example(impl):
+    """Pin: the worked example in tests/golden/hand_d2_t2.txt, derived on
+    paper from the definition (decay, unit-gate projection, normalisation of
+    q and k, reverse scan and the bidirectional sum all exercised)."""
+    G = load_golden("hand_d2_t2.txt")
+    q = G["q"].reshape(1, 2, 1, 2).astype(np.float32)
+    k = G["k"].reshape(1, 2, 1, 2).astype(np.float32)
+    v = G["v"].reshape(1, 2, 1, 2).astype(np.float32)
+    g = G["g"].reshape(1, 2, 1).astype(np.float32)
+    beta = G["beta"].reshape(1, 2, 1).astype(np.float32)
+    out, S = FWD[impl](q, k, v, g, beta)
+    # g is stored in fp32, so a_1 = exp(fp32(ln 0.5)) differs from 0.5 by ~2e-9
+    np.testing.assert_allclose(out[0, :, 0], G["out_fwd"], rtol=0, atol=1e-8)
+    np.testing.assert_allclose(S[0, 0], G["state_fwd"], rtol=0, atol=1e-8)
+    out_b, S_b = BIDIR[impl](q, k, v, g, beta)
+    np.testing.assert_allclose(out_b[0, :, 0], G["out_bidir"], rtol=0, atol=1e-8)
+    np.testing.assert_allclose(S_b[0, 0], G["state_fwd"], rtol=0, atol=1e-8)
+
+
+# ------------------------------------------------------------- closed forms
+@pytest.mark.parametrize("impl", ["c", "numpy"])
+def test_p1_identity_gate_zero_beta_keeps_state(impl):
+    """Pin p1: a = 1, beta = 0 -> S never changes and o_t = S_in^T q^_t."""
+    rng = np.random.default_rng(11)
+    q, k, v, g, beta, s = rand_inputs(rng)
+    g[:] = 0
+    beta[:] = 0
+    out, S = FWD[impl](q, k, v, g, beta, s)
+    np.testing.assert_allclose(S, s, rtol=0, atol=1e-14)
+    expect = np.einsum("bthi,bhij->bthj", unit(q), s)
+    np.testing.assert_allclose(out, expect, rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("impl", ["c", "numpy"])
+def test_p2_unit_gate_writes_value_exactly(impl):
+    """Pin p2: a = 1, beta = 1, orthonormal keys k_t = e_{pi(t)} -> the state
+    is S_in with row pi(t) replaced by v_t (the last write wins), so
+    S^T e_{pi(t)} = v_t; every output follows from those row replacements."""
+    rng = np.random.default_rng(12)
+    B, T, H, Dk, Dv = 1, 6, 2, 8, 5
+    q, k, v, g, beta, s = rand_inputs(rng, B, T, H, Dk, Dv)
+    g[:] = 0
+    beta[:] = 1
+    perm = [3, 0, 6, 3, 1, 7]           # key 3 written twice
+    k[:] = 0
+    for t, i in enumerate(perm):
+        k[:, t, :, i] = 2.5              # not unit: normalisation must fix it
+    out, S = FWD[impl](q, k, v, g, beta, s)
+    expect = s.copy()
+    for t, i in enumerate(perm):
+        expect[:, :, i, :] = v[:, t, :, :]
+        np.testing.assert_allclose(out[:, t], np.einsum("bhi,bhij->bhj", unit(q[:, t]), expect),
+                                   rtol=0, atol=1e-13)
+    np.testing.assert_allclose(S, expect, rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("impl", ["c", "numpy"])
+def test_p2b_general_unit_key_projection(impl):
+    """Pin p2 (general key): a = 1, beta = 1 -> after the update S^T k^ = v
+    for any key direction, and S is unchanged on the complement of k^."""
+    rng = np.random.default_rng(13)
+    q, k, v, g, beta, s = rand_inputs(rng, 2, 1, 3, 16, 9)
+    g[:] = 0
+    beta[:] = 1
+    out, S = FWD[impl](q, k, v, g, beta, s)
+    kh = unit(k[:, 0])
+    np.testing.assert_allclose(np.einsum("bhi,bhij->bhj", kh, S), v[:, 0], rtol=0, atol=1e-13)
+    z = unit(rng.standard_normal(kh.shape))
+    z = z - np.sum(z * kh, -1, keepdims=True) * kh          # orthogonal to k^
+    np.testing.assert_allclose(np.einsum("bhi,bhij->bhj", z, S),
+                               np.einsum("bhi,bhij->bhj", z, s), rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("impl", ["c", "numpy"])
+def test_p3_pure_decay(impl):
+    """Pin p3: beta = 0 -> S_t = exp(sum_{s<=t} g_s) S_in and
+    o_t = exp(sum_{s<=t} g_s) S_in^T q^_t."""
+    rng = np.random.default_rng(14)
+    q, k, v, g, beta, s = rand_inputs(rng, g_lo=-2.0)
+    beta[:] = 0
+    out, S = FWD[impl](q, k, v, g, beta, s)
+    G = np.cumsum(g.astype(np.float64), axis=1)                 # [B,T,H]
+    np.testing.assert_allclose(S, np.exp(G[:, -1])[..., None, None] * s, rtol=1e-13, atol=1e-300)
+    expect = np.exp(G)[..., None] * np.einsum("bthi,bhij->bthj", unit(q), s)
+    np.testing.assert_allclose(out, expect, rtol=1e-12, atol=1e-15)
+
+
+@pytest.mark.parametrize("impl", ["c", "numpy"])
+def test_p9_single_token_formula(impl):
+    """Pin p9a: T = 1 written out by hand:
+    S1 = a S0 - a beta k^ (k^^T S0) + beta k^ v^T,  o = S1^T q^."""
+    rng = np.random.default_rng(15)
+    q, k, v, g, beta, s = rand_inputs(rng, 2, 1, 3, 12, 7)
+    out, S = FWD[impl](q, k, v, g, beta, s)
+    a = np.exp(g[:, 0].astype(np.float64))[..., None, None]
+    b = beta[:, 0].astype(np.float64)[..., None, None]
+    kh, qh = unit(k[:, 0]), unit(q[:, 0])
+    kS = np.einsum("bhi,bhij->bhj", kh, s)
+    S1 = a * s - a * b * kh[..., :, None] * kS[..., None, :] + b * kh[..., :, None] * v[:, 0][..., None, :]
+    np.testing.assert_allclose(S, S1, rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(out[:, 0], np.einsum("bhi,bhij->bhj", qh, S1), rtol=1e-13, atol=1e-15)
+
+
+@pytest.mark.parametrize("impl", ["c", "numpy"])
+def test_p9_scalar_state(impl):
+    """Pin p9b: Dk = Dv = 1 reduces to the scalar recurrence
+    s_t = a_t (1 - beta_t) s_{t-1} + beta_t sign(k_t) v_t, o_t = sign(q_t) s_t."""
+    rng = np.random.default_rng(16)
+    q, k, v, g, beta, s = rand_inputs(rng, 1, 40, 2, 1, 1)
+    out, S = FWD[impl](q, k, v, g, beta, s)
+    for h in range(2):
+        st = s[0, h, 0, 0]
+        for t in range(40):
+            a = np.exp(np.float64(g[0, t, h]))
+            b = np.float64(beta[0, t, h])
+            st = a * (1.0 - b) * st + b * np.sign(k[0, t, h, 0]) * v[0, t, h, 0]
+            assert abs(out[0, t, h, 0] - np.sign(q[0, t, h, 0]) * st) <= 1e-13 * max(1.0, abs(st))
+        assert abs(S[0, h, 0, 0] - st) <= 1e-13 * max(1.0, abs(st))
+
+
+@pytest.mark.parametrize("impl", ["c", "numpy"])
+def test_p10_bidir_single_token(impl):
+    """Pin p10: T = 1 bidirectional -> out = forward + beta (q^ . k^) v (the
+    reverse scan from zero state sees only the token itself)."""
+    rng = np.random.default_rng(17)
+    q, k, v, g, beta, s = rand_inputs(rng, 2, 1, 3, 10, 4)
+    out_f, S_f = FWD[impl](q, k, v, g, beta, s)
+    out_b, S_b = BIDIR[impl](q, k, v, g, beta, s)
+    qk = np.sum(unit(q[:, 0]) * unit(k[:, 0]), -1)
+    expect = out_f[:, 0] + beta[:, 0, :, None] * qk[..., None] * v[:, 0]
+    np.testing.assert_allclose(out_b[:, 0], expect, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(S_b, S_f, rtol=0, atol=0)
+
+
+# ---------------------------------------------------------------- invariants
+@pytest.mark.parametrize("impl", ["c", "numpy"])
+def test_p5_streaming_equals_one_scan(impl):
+    """Pin p5: chunks scanned one after another with the state carried equal
+    one scan over their concatenation (outputs and state)."""
+    rng = np.random.default_rng(18)
+    q, k, v, g, beta, s = rand_inputs(rng, 2, 37, 2, 8, 8)
+    out, S = FWD[impl](q, k, v, g, beta, s)
+    cuts = [0, 5, 6, 20, 37]
+    St = s
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        o, St = FWD[impl](q[:, a:b], k[:, a:b], v[:, a:b], g[:, a:b], beta[:, a:b], St)
+        np.testing.assert_allclose(o, out[:, a:b], rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(St, S, rtol=1e-13, atol=1e-14)
+
+
+@pytest.mark.parametrize("impl", ["c", "numpy"])
+def test_p6_linearity_in_values_and_state(impl):
+    """Pin p6: for fixed q, k, g, beta the map (V, S_in) -> (out, S_out) is
+    linear."""
+    rng = np.random.default_rng(19)
+    q, k, v1, g, beta, s1 = rand_inputs(rng)
+    # values on a 1/64 grid so the combination below is exact in fp32 inputs
+    v1 = (np.round(v1 * 64) / 64).astype(np.float32)
+    v2 = (np.round(rng.standard_normal(v1.shape) * 64) / 64).astype(np.float32)
+    s2 = rng.standard_normal(s1.shape)
+    al, be = np.float32(0.75), np.float32(-1.5)
+    o1, S1 = FWD[impl](q, k, v1, g, beta, s1)
+    o2, S2 = FWD[impl](q, k, v2, g, beta, s2)
+    o3, S3 = FWD[impl](q, k, al * v1 + be * v2, g, beta, al * s1 + be * s2)
+    np.testing.assert_allclose(o3, al * o1 + be * o2, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(S3, al * S1 + be * S2, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("impl", ["c", "numpy"])
+def test_p7_columns_are_independent(impl):
+    """Pin p7: column j of out and of S depends only on v[..., j] and
+    S_in[..., j]; perturbing column 2 leaves every other column bit-equal."""
+    rng = np.random.default_rng(20)
+    q, k, v, g, beta, s = rand_inputs(rng, Dv=6)
+    o1, S1 = FWD[impl](q, k, v, g, beta, s)
+    v2, s2 = v.copy(), s.copy()
+    v2[..., 2] += 1.0
+    s2[..., 2] -= 0.5
+    o2, S2 = FWD[impl](q, k, v2, g, beta, s2)
+    keep = [0, 1, 3, 4, 5]
+    assert np.array_equal(o1[..., keep], o2[..., keep])
+    assert np.array_equal(S1[..., keep], S2[..., keep])
+    assert np.max(np.abs(o1[..., 2] - o2[..., 2])) > 1e-3
+
+
+@pytest.mark.parametrize("impl", ["c", "numpy"])
+def test_p8_state_norm_bound(impl):
+    """Pin p8: |I - b k^k^T|_2 = 1 for b in [0,1], so
+    |S_t|_2 <= a_t |S_{t-1}|_2 + beta_t |v_t|.  Checked token by token."""
+    rng = np.random.default_rng(21)
+    q, k, v, g, beta, s = rand_inputs(rng, 1, 30, 2, 8, 8, g_lo=-0.3)
+    St = s
+    for t in range(30):
+        _, Sn = FWD[impl](q[:, t:t + 1], k[:, t:t + 1], v[:, t:t + 1], g[:, t:t + 1],
+                          beta[:, t:t + 1], St)
+        for h in range(2):
+            lhs = np.linalg.norm(Sn[0, h], 2)
+            rhs = (np.exp(np.float64(g[0, t, h])) * np.linalg.norm(St[0, h], 2)
+                   + np.float64(beta[0, t, h]) * np.linalg.norm(v[0, t, h].astype(np.float64)))
+            assert lhs <= rhs * (1 + 1e-12)
+        St = Sn
+
+
+def test_bidir_is_forward_plus_flipped_forward():
+    """Reading of the bidirectional mode: out = fwd(state_in) + flip(fwd(flip(x),
+    0)); the state comes from the forward scan only (C oracle vs its own
+    forward entry point run on the flipped sequence)."""
+    rng = np.random.default_rng(22)
+    q, k, v, g, beta, s = rand_inputs(rng)
+    out_b, S_b = c_bidir(q, k, v, g, beta, s)
+    out_f, S_f = c_fwd(q, k, v, g, beta, s)
+    fl = lambda x: np.ascontiguousarray(x[:, ::-1])  # noqa: E731
+    out_r, _ = c_fwd(fl(q), fl(k), fl(v), fl(g), fl(beta), None)
+    np.testing.assert_allclose(out_b, out_f + out_r[:, ::-1], rtol=1e-14, atol=1e-14)
+    np.testing.assert_array_equal(S_b, S_f)
+
+
+# --------------------------------------------------------------- brute force
+@pytest.mark.parametrize("chunk", [1, 3, 16, 64])
+@pytest.mark.parametrize("T", [1, 37, 100])
+def test_p4_chunked_form_equals_recurrence(chunk, T):
+    """Pin p4: the chunked WY/UT form (an independent algorithm) reaches the
+    token recurrence to ~1e-13 for every sub-chunk length, ragged tails
+    included."""
+    rng = np.random.default_rng(100 + T + chunk)
+    q, k, v, g, beta, s = rand_inputs(rng, 1, T, 2, 16, 12, g_lo=-1.0)
+    o_c, S_c = oracle.chunked_fwd(q, k, v, g, beta, s, chunk)
+    o_r, S_r = c_fwd(q, k, v, g, beta, s)
+    assert rel(o_c, o_r) < 1e-12
+    assert rel(S_c, S_r) < 1e-12
+    ob_c, _ = oracle.chunked_bidir(q, k, v, g, beta, s, chunk)
+    ob_r, _ = c_bidir(q, k, v, g, beta, s)
+    assert rel(ob_c, ob_r) < 1e-12
+
+
+def test_p4_chunked_form_fast_decay_does_not_overflow():
+    """Pin p4 (fast decay): g in [-8,-4] over a 64-token sub-chunk drives
+    exp(gamma) to ~e^-400; the chunked form must still equal the recurrence."""
+    rng = np.random.default_rng(31)
+    q, k, v, g, beta, s = rand_inputs(rng, 1, 130, 2, 16, 16)
+    g[:] = rng.uniform(-8, -4, g.shape)
+    with np.errstate(under="ignore"):
+        o_c, S_c = oracle.chunked_fwd(q, k, v, g, beta, s, 64)
+    o_r, S_r = c_fwd(q, k, v, g, beta, s)
+    assert np.all(np.isfinite(o_c))
+    assert rel(o_c, o_r) < 1e-12
+
+
+def test_c_and_numpy_recurrences_agree_on_tiny_workload():
+    """The two transcriptions agree on the tiny fp32 workload (fwd + bidir)."""
+    w = wl.tiny()
+    x = wl.make_inputs(w)
+    args = (x["q"], x["k"], x["v"], x["g"], x["beta"], x["state_in"])
+    o1, S1 = c_fwd(*args)
+    o2, S2 = oracle.recurrence_fwd(*args)
+    assert rel(o1, o2) < 1e-13 and rel(S1, S2) < 1e-13
+    o1, _ = c_bidir(*args)
+    o2, _ = oracle.recurrence_bidir(*args)
+    assert rel(o1, o2) < 1e-13
+
+
+def test_p11_double_vs_long_double_error_floor():
+    """Pin p11: on the stress gate extremes (near-identity and fast decay,
+    beta 0.01 / 0.99) the double oracle agrees with a long-double rerun to
+    far below the parity tolerances, so its own rounding is negligible."""
+    rng = np.random.default_rng(41)
+    for lo, hi in ((-1e-4, 0.0), (-8.0, -4.0)):
+        for b in (0.01, 0.99):
+            q, k, v, g, beta, s = rand_inputs(rng, 1, 512, 2, 32, 32, unit=True)
+            g[:] = rng.uniform(lo, hi, g.shape)
+            beta[:] = b
+            o64, S64 = oracle.oracle_fwd(q, k, v, g, beta, s, nthreads=2)
+            oLD, SLD = oracle.oracle_fwd(q, k, v, g, beta, s, nthreads=2, precision="long double")
+            assert rel(o64, oLD.astype(np.float64)) < 1e-11
+            assert rel(S64, SLD.astype(np.float64)) < 1e-11
+
+
+def test_empty_sequence_passes_state_through():
+    """T = 0: nothing to scan, state_out = state_in (or zero)."""
+    rng = np.random.default_rng(5)
+    q, k, v, g, beta, s = rand_inputs(rng, 1, 0, 2, 4, 4)
+    out, S = c_fwd(q, k, v, g, beta, s)
+    assert out.shape == (1, 0, 2, 4)
+    np.testing.assert_array_equal(S, s)
+    _, S0 = c_fwd(q, k, v, g, beta, None)
+    assert not S0.any()
+
+
+def test_oracle_planted_sign_error_is_caught():
+    """The pins have teeth: an oracle with the decay applied after the delta
+    correction instead of before (a plausible slip) fails pin p2's exact
+    write-back once a < 1.  Planted in a CPU copy of the numpy recurrence."""
+    def wrong_fwd(q, k, v, g, beta, s):
+        q, k, v, g, beta = [np.asarray(x, np.float64) for x in (q, k, v, g, beta)]
+        S = np.array(s, copy=True)
+        out = np.zeros(v.shape)
+        for t in range(q.shape[1]):
+            kh = unit(k[:, t])
+            a = np.exp(g[:, t])[..., None, None]
+            b = beta[:, t][..., None, None]
+            S = a * S
+            S = S - b * kh[..., :, None] * np.einsum("bhi,bhij->bhj", kh, S)[..., None, :] \
+                + a * b * kh[..., :, None] * v[:, t][..., None, :]
+            out[:, t] = np.einsum("bhi,bhij->bhj", unit(q[:, t]), S)
+        return out, S
+
+    rng = np.random.default_rng(6)
+    q, k, v, g, beta, s = rand_inputs(rng, 1, 3, 1, 4, 3)
+    g[:] = -0.5
+    beta[:] = 1.0
+    _, S_ok = c_fwd(q, k, v, g, beta, s)
+    _, S_bad = wrong_fwd(q, k, v, g, beta, s)
+    kh = unit(k[:, -1])
+    ok = np.einsum("bhi,bhij->bhj", kh, S_ok)
+    bad = np.einsum("bhi,bhij->bhj", kh, S_bad)
+    # with beta = 1 the right ordering gives S^T k^ = v for any a; the slip gives a v
+    np.testing.assert_allclose(ok, v[:, -1], atol=1e-12)
+    assert np.max(np.abs(bad - v[:, -1])) > 1e-2
