@@ -1,0 +1,465 @@
+#!/usr/bin/env python
+"""Throughput of the chunked GDN scan on B200: head-tokens/s and latent
+frames/s on the 1280x704 streaming chunk, with the roofline fraction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+A step is one library call on one streaming chunk: B1 x H20 x T2640 tokens
+(3 latent frames of 40x22), d_k = d_v = 112, bf16 q/k/v/out, fp32 g, beta and
+carried state -- the causal scan with the previous chunk's state.  Inputs are
+resident in HBM before timing starts and rotate over enough buffer sets that
+their total exceeds L2 (so every step reads from HBM).  Steps are timed with
+CUDA events on the launching stream, K steps between a barrier + synchronize
+on both sides, max over ranks.  With N > 1 (torchrun) every rank scans its own
+chunk stream: the work partitions over independent chunks with no exchange,
+so scaling is weak and no collective sits on the data path.
+
+``--impl reference`` times the fp64 CPU oracle (token recurrence) on the same
+workload on this host's cores instead (rank 0 only).
+
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "GDN head-tokens/s and latent frames/s at 2640-tok chunk; % of B200 roofline"
+UNIT = "head-tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+N_SETS = 8                      # rotating input sets (8 x 49.7 MB > 126 MB L2)
+DOMINANT_KERNEL_SOURCE = "gated_deltanet_linear_chunked_b200/csrc/scan_serial.cu"
+DOMINANT_KERNEL_NAME = "gdn_scan_serial_kernel"
+
+
+def parse():
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=400)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["native", "reference"], default="native")
+    p.add_argument("--mode", choices=["fwd", "bidir"], default="fwd",
+                   help="causal chunk (the headline workload) or the bidirectional chunk")
+    p.add_argument("--no-graph", action="store_true", help="time direct calls instead of CUDA-graph replays")
+    p.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle CPU baseline")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-extras", action="store_true", help="skip the bidir / stacked-stream side figures")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except OSError:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def algorithmic_bytes(w) -> int:
+    """q, k, v, out (dtype) + g, beta (fp32) per token-head, plus the fp32
+    state read and written once per (b, h)."""
+    es = 2 if w.dtype == "bf16" else 4
+    per_tok = (2 * w.Dk + 2 * w.Dv) * es + 8
+    return w.head_tokens * per_tok + 2 * w.B * w.H * w.Dk * w.Dv * 4
+
+
+def algorithmic_flops(w, bidir=False) -> int:
+    """Chunked-form work per token-head: 6 d^2 + 8 C d (doubled for bidir)."""
+    d = w.Dk
+    f = w.head_tokens * (6 * d * d + 8 * w.chunk * d)
+    return 2 * f if bidir else f
+
+
+def recorded_traffic():
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, if it was taken on the current source of that kernel."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    kv = dict(l.split(":", 1) for l in lines if ":" in l and not l.startswith("#"))
+    kv = {k.strip(): v.strip() for k, v in kv.items()}
+    try:
+        src = open(os.path.join(ROOT, DOMINANT_KERNEL_SOURCE), "rb").read()
+    except OSError:
+        return None
+    if kv.get("kernel") != DOMINANT_KERNEL_NAME or kv.get("source_sha256") != hashlib.sha256(src).hexdigest():
+        return None
+    try:
+        return int(float(kv["dram_bytes_per_launch"]))
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML every ~20 ms."""
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._thr = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    _REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def _sample(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        mask = get(self.h)
+        for bit, name in self._REASONS.items():
+            if mask & bit:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                pass
+            self._stop.wait(0.02)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thr is not None:
+            self._thr.join()
+            try:
+                self._sample()
+            except Exception:
+                pass
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+def cpu_baseline(w, budget_s: float):
+    """The fp64 oracle (as it stands) on this host's cores, on the full
+    streaming chunk, repeated until `budget_s` seconds have been spent."""
+    import oracle
+    from gated_deltanet_linear_chunked_b200 import workloads as wl
+    x = wl.make_inputs(w)
+    fn = oracle.oracle_bidir if w.mode == "bidir" else oracle.oracle_fwd
+    cores = min(oracle.online_cores(), w.B * w.H)   # the pool never exceeds one thread per head
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        fn(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state_in"], nthreads=cores)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or reps >= 1000:
+            break
+    return {"value": w.head_tokens * reps / el, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"full {w.name} chunk (B{w.B} H{w.H} T{w.T} d{w.Dk}, fp64 token recurrence), "
+                      f"{reps} repetitions in {el:.1f} s"}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    from gated_deltanet_linear_chunked_b200 import workloads as wl
+    x = wl.make_inputs(w)
+    fn = oracle.oracle_bidir if w.mode == "bidir" else oracle.oracle_fwd
+    cores = min(oracle.online_cores(), w.B * w.H)   # the pool never exceeds one thread per head
+    # size one step so the whole run stays within a few minutes
+    t0 = time.perf_counter()
+    fn(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state_in"], nthreads=cores)
+    one = time.perf_counter() - t0
+    heads = w.H
+    budget_per_step = 120.0 / max(1, args.steps + args.warmup)
+    if one > budget_per_step:
+        heads = max(1, int(w.H * budget_per_step / one))
+    xs = {n: x[n][:, :, :heads].copy() for n in ("q", "k", "v", "g", "beta")}
+    s_in = None if x["state_in"] is None else x["state_in"][:, :heads].copy()
+    for _ in range(args.warmup):
+        fn(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], s_in, nthreads=cores)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        fn(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], s_in, nthreads=cores)
+    el = time.perf_counter() - t0
+    ht = w.B * heads * w.T * args.steps
+    value = ht / el
+    sample = (f"{heads} of {w.H} heads of the {w.name} chunk (T{w.T}, d{w.Dk}) per step, "
+              f"fp64 token recurrence")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000 * el / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": heads, "T": w.T, "Dk": w.Dk, "Dv": w.Dv,
+                   "mode": w.mode, "latent_frames_per_chunk": w.T / 880},
+        "latent_frames_per_s": value / (w.B * heads * 880),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    from gated_deltanet_linear_chunked_b200 import workloads as wl
+    w = wl.stream_chunk(args.mode)
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+    import gated_deltanet_linear_chunked_b200 as gdn
+    from gated_deltanet_linear_chunked_b200 import _lib
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    lib = _lib.load()
+    stream = torch.cuda.Stream(device=dev)
+    fn = gdn.chunk_bidir if w.mode == "bidir" else gdn.chunk_fwd
+
+    # ---- inputs: one seeded chunk per rank, copied into N_SETS rotating sets
+    w_r = wl.stream_chunk(w.mode, seed=w.seed + 7919 * rank)
+    xh = wl.make_inputs(w_r)
+    dt = torch.bfloat16
+    base = {n: torch.from_numpy(xh[n]).to(dev) for n in ("q", "k", "v", "g", "beta")}
+    for n in ("q", "k", "v"):
+        base[n] = base[n].to(dt)
+    base["state_in"] = torch.from_numpy(xh["state_in"]).to(dev)
+    sets = []
+    for _ in range(N_SETS):
+        s = {n: t.clone() for n, t in base.items()}
+        s["out"] = torch.empty((w.B, w.T, w.H, w.Dv), dtype=dt, device=dev)
+        s["state_out"] = torch.empty_like(s["state_in"])
+        sets.append(s)
+    torch.cuda.synchronize()
+
+    def step(i):
+        s = sets[i % N_SETS]
+        fn(s["q"], s["k"], s["v"], s["g"], s["beta"], s["state_in"], state_out=s["state_out"],
+           out=s["out"], chunk=w.chunk, stream=stream)
+
+    # launches per step (counted on a direct call)
+    c0 = lib.gdn_launch_count()
+    with torch.cuda.stream(stream):
+        step(0)
+    launches_per_step = lib.gdn_launch_count() - c0
+    torch.cuda.synchronize()
+
+    use_graph = not args.no_graph
+    graphs = []
+    if use_graph:
+        for i in range(N_SETS):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step(i)
+            graphs.append(g)
+        torch.cuda.synchronize()
+
+    def run_steps(n, offset=0):
+        with torch.cuda.stream(stream):
+            for i in range(n):
+                if use_graph:
+                    graphs[(i + offset) % N_SETS].replay()
+                else:
+                    step(i + offset)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+        torch.cuda.synchronize()
+
+    run_steps(max(3, args.warmup))
+    barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    try:
+        nvml_index = torch.cuda._get_nvml_device_index(local)
+    except Exception:
+        nvml_index = local
+    with ClockSampler(nvml_index) as clocks:
+        barrier()
+        ev0.record(stream)
+        run_steps(args.steps)
+        ev1.record(stream)
+        barrier()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = world * args.steps * w.head_tokens / (ms / 1000.0)
+
+    # ---- end to end through the public API: pinned host -> device, call, device -> host
+    e2e_steps = max(3, min(args.steps, 200))
+    host = {n: (t.cpu().pin_memory()) for n, t in base.items()}
+    host_out = torch.empty((w.B, w.T, w.H, w.Dv), dtype=dt).pin_memory()
+    host_state = torch.empty_like(host["state_in"]).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = host_out.numel() * host_out.element_size() + host_state.numel() * host_state.element_size()
+
+    def e2e_step(i):
+        s = sets[i % N_SETS]
+        for n in ("q", "k", "v", "g", "beta", "state_in"):
+            s[n].copy_(host[n], non_blocking=True)
+        fn(s["q"], s["k"], s["v"], s["g"], s["beta"], s["state_in"], state_out=s["state_out"],
+           out=s["out"], chunk=w.chunk, stream=stream)
+        host_out.copy_(s["out"], non_blocking=True)
+        host_state.copy_(s["state_out"], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            e2e_step(i)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(e2e_steps):
+            e2e_step(i)
+        e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * e2e_steps * w.head_tokens / (e2e_ms / 1000.0)
+
+    # ---- side figures: the other mode, and the 15-layer stacked stream
+    extras = {}
+    if not args.no_extras:
+        other = "bidir" if w.mode == "fwd" else "fwd"
+        fo = gdn.chunk_bidir if other == "bidir" else gdn.chunk_fwd
+        n_side = max(3, min(args.steps, 200))
+
+        def side_run(n):
+            with torch.cuda.stream(stream):
+                for i in range(n):
+                    s = sets[i % N_SETS]
+                    fo(s["q"], s["k"], s["v"], s["g"], s["beta"], s["state_in"],
+                       state_out=s["state_out"], out=s["out"], chunk=w.chunk, stream=stream)
+        side_run(3)
+        barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        side_run(n_side)
+        a1.record(stream)
+        barrier()
+        other_ms = a0.elapsed_time(a1) / n_side
+        extras[f"{other}_chunk"] = {"ms_per_call": other_ms,
+                                    "head_tokens_per_s": w.head_tokens / (other_ms / 1000.0),
+                                    "timing": "direct calls"}
+        # 32 chunks x 15 layers in model order (chunk-major), bidirectional,
+        # one state per layer carried in place, inputs rotating over the sets
+        states = [torch.zeros_like(base["state_in"]) for _ in range(wl.GDN_LAYERS)]
+        n_chunks = 32
+
+        def stack_run():
+            with torch.cuda.stream(stream):
+                i = 0
+                for _c in range(n_chunks):
+                    for l in range(wl.GDN_LAYERS):
+                        s = sets[i % N_SETS]
+                        gdn.chunk_bidir(s["q"], s["k"], s["v"], s["g"], s["beta"], states[l],
+                                        state_out=states[l], out=s["out"], chunk=w.chunk,
+                                        stream=stream)
+                        i += 1
+        stack_run()
+        barrier()
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        stack_run()
+        b1.record(stream)
+        barrier()
+        stack_ms = b0.elapsed_time(b1)
+        frames = n_chunks * 3
+        extras["stack_32x15_bidir"] = {"ms": stack_ms, "latent_frames_per_s": frames / (stack_ms / 1000.0),
+                                       "calls": n_chunks * wl.GDN_LAYERS, "timing": "direct calls"}
+
+    # ---- roofline of the dominant kernel (the one launch per step)
+    peaks, peak_kind = load_peaks()
+    bytes_step = algorithmic_bytes(w)
+    flops_step = algorithmic_flops(w, w.mode == "bidir")
+    achieved = bytes_step / (ms_per_step / 1000.0) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": recorded_traffic(),
+                "peak_source": f"{peak_kind} hbm_gbs", "algorithmic_bytes": bytes_step,
+                "kernel": DOMINANT_KERNEL_NAME,
+                "tensor_frac_of_sustained": (flops_step / (ms_per_step / 1000.0) / 1e12)
+                / peaks["bf16_tflops_sustained"]}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.cpu_seconds)
+
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        graphs.clear()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "Dk": w.Dk, "Dv": w.Dv,
+                   "chunk": w.chunk, "mode": w.mode, "io": "bf16 q/k/v/out, fp32 g/beta/state",
+                   "l2": f"inputs rotate over {N_SETS} sets of "
+                         f"{bytes_step / 1e6:.1f} MB ({N_SETS * bytes_step / 1e6:.0f} MB > 126 MB L2)",
+                   "graph": use_graph, "parallelism": f"replicas x{world} (independent chunk streams)"},
+        "latent_frames_per_s": value / (w.B * w.H * 880),
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": int(launches_per_step * args.steps),
+        "launches_per_step": int(launches_per_step),
+        "clocks": clocks.summary(),
+        "extras": extras,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,1 +1,21 @@
-"""B200-native chunked Gated DeltaNet (GDN) scan."""
+"""B200-native chunked Gated DeltaNet (GDN) scan.
+
+The scan runs in ``libgdn.so`` (hand-written CUDA for sm_100a, C ABI in
+``include/gdn.h``); this package is its thin torch binding plus the seeded
+workload generators.  Importing the package does not load CUDA; the library
+is loaded on the first call.
+"""
+from . import workloads  # noqa: F401
+
+__all__ = ["chunk_fwd", "chunk_bidir", "state_reset", "device_error",
+           "set_wait_limit", "GDNError", "workloads"]
+
+
+def __getattr__(name):
+    if name in ("chunk_fwd", "chunk_bidir", "state_reset", "device_error", "set_wait_limit"):
+        from . import api
+        return getattr(api, name)
+    if name == "GDNError":
+        from ._lib import GDNError
+        return GDNError
+    raise AttributeError(name)

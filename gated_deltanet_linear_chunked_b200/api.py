@@ -1,0 +1,107 @@
+"""Thin torch-facing binding of the C ABI (include/gdn.h).
+
+Argument marshalling only: each function checks that it was handed CUDA
+tensors of the expected shapes and dtypes, allocates outputs the caller did
+not supply, and passes raw pointers, sizes and the current CUDA stream to
+libgdn.so.  Every step of the scan runs in the library's kernels; there is
+no CPU or PyTorch fallback.
+
+Layouts: q, k [B,T,H,Dk]; v, out [B,T,H,Dv] (bf16 or fp32); g, beta [B,T,H]
+fp32; state [B,H,Dk,Dv] fp32.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib
+
+_DTYPES = {torch.float32: _lib.GDN_F32, torch.bfloat16: _lib.GDN_BF16}
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _check_tensor(t, name, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _scan(entry, q, k, v, g, beta, state_in, state_out, out, chunk, stream):
+    if q.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k must be [B,T,H,Dk] and v [B,T,H,Dv]")
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    if q.dtype not in _DTYPES:
+        raise TypeError(f"q/k/v must be bfloat16 or float32, got {q.dtype}")
+    dt = q.dtype
+    _check_tensor(q, "q", dt)
+    _check_tensor(k, "k", dt, (B, T, H, Dk))
+    _check_tensor(v, "v", dt, (B, T, H, Dv))
+    _check_tensor(g, "g", torch.float32, (B, T, H))
+    _check_tensor(beta, "beta", torch.float32, (B, T, H))
+    if state_in is not None:
+        _check_tensor(state_in, "state_in", torch.float32, (B, H, Dk, Dv))
+    if state_out is None:
+        state_out = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=q.device)
+    else:
+        _check_tensor(state_out, "state_out", torch.float32, (B, H, Dk, Dv))
+    if out is None:
+        out = torch.empty((B, T, H, Dv), dtype=dt, device=q.device)
+    else:
+        _check_tensor(out, "out", dt, (B, T, H, Dv))
+    lib = _lib.load()
+    st = getattr(lib, entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                             _ptr(state_in), _ptr(state_out), _ptr(out),
+                             B, T, H, Dk, Dv, _DTYPES[dt], int(chunk), _stream(stream))
+    _lib.check(st, entry)
+    return out, state_out
+
+
+def chunk_fwd(q, k, v, g, beta, state_in=None, state_out=None, out=None, chunk=0,
+              stream=None):
+    """Causal scan of one chunk from ``state_in`` (None = zero state).
+    Returns ``(out, state_out)``; ``state_out`` may be ``state_in`` (in place)."""
+    return _scan("gdn_chunk_fwd", q, k, v, g, beta, state_in, state_out, out, chunk, stream)
+
+
+def chunk_bidir(q, k, v, g, beta, state_in=None, state_out=None, out=None, chunk=0,
+                stream=None):
+    """Forward scan from ``state_in`` plus the in-chunk reverse scan from zero,
+    summed.  ``state_out`` is the forward scan's final state."""
+    return _scan("gdn_chunk_bidir", q, k, v, g, beta, state_in, state_out, out, chunk, stream)
+
+
+def state_reset(state, stream=None):
+    """Zero a state tensor [B,H,Dk,Dv] in place (streaming restart)."""
+    _check_tensor(state, "state", torch.float32)
+    if state.dim() != 4:
+        raise ValueError("state must be [B,H,Dk,Dv]")
+    B, H, Dk, Dv = state.shape
+    st = _lib.load().gdn_state_reset(_ptr(state), B, H, Dk, Dv, _stream(stream))
+    _lib.check(st, "gdn_state_reset")
+    return state
+
+
+def device_error(stream=None) -> int:
+    """Synchronise and read/clear the device error word (0 = none)."""
+    return int(_lib.load().gdn_device_error(_stream(stream)))
+
+
+def set_wait_limit(polls: int) -> int:
+    """Polls a kernel's bounded wait makes before giving up (0 = default)."""
+    return int(_lib.load().gdn_set_wait_limit(int(polls)))

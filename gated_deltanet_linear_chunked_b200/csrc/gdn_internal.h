@@ -1,0 +1,43 @@
+// Internal interface between the C-ABI front end (gdn_api.cu) and the kernel
+// translation units.  Not installed; callers use include/gdn.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gdn.h"
+
+namespace gdn {
+
+// One scan call, after validation.  Pointers are device pointers.
+struct ScanArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* g;
+  const float* beta;
+  const float* state_in;   // nullptr => zero state
+  float* state_out;        // nullptr => not written
+  void* out;
+  int B, T, H, Dk, Dv;
+  gdn_dtype dtype;
+  int chunk;               // sub-chunk length (already defaulted)
+  bool bidir;
+  cudaStream_t stream;
+  unsigned int* err;       // device error word (bounded waits report here)
+  long long wait_limit;    // polls before a bounded wait gives up
+};
+
+// Adds n to the process-wide count of kernels the library has enqueued.
+void count_launches(unsigned n);
+
+// Token-serial SIMT scan (fp32 arithmetic, fp32 or bf16 I/O).
+cudaError_t launch_scan_serial(const ScanArgs& a);
+
+// Device error word values.
+enum : unsigned int {
+  kErrNone = 0,
+  kErrTimeout = 1,
+};
+
+}  // namespace gdn

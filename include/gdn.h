@@ -50,6 +50,12 @@
 #ifndef GDN_H_
 #define GDN_H_
 
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -78,7 +84,7 @@ typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
  * T == 0     is allowed: state_out = state_in (or zero), out is untouched.
  * B == 0 or H == 0 is allowed and does nothing.
  */
-gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v,
+GDN_API gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v,
                          const float* g, const float* beta,
                          const float* state_in, float* state_out, void* out,
                          int B, int T, int H, int Dk, int Dv, gdn_dtype dtype,
@@ -90,7 +96,7 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v,
  * token keeping its own g_t and beta_t), summed per token.  state_out is the
  * forward scan's final state.  Arguments as for gdn_chunk_fwd.
  */
-gdn_status gdn_chunk_bidir(const void* q, const void* k, const void* v,
+GDN_API gdn_status gdn_chunk_bidir(const void* q, const void* k, const void* v,
                            const float* g, const float* beta,
                            const float* state_in, float* state_out, void* out,
                            int B, int T, int H, int Dk, int Dv,
@@ -101,7 +107,7 @@ gdn_status gdn_chunk_bidir(const void* q, const void* k, const void* v,
  * a stream keeps, "SANA-Streaming：基于混合扩散Transformer的实时流式视频编辑系统",
  * 前置知识, 流式生成).  Any positive Dk, Dv are accepted here.
  */
-gdn_status gdn_state_reset(float* state, int B, int H, int Dk, int Dv,
+GDN_API gdn_status gdn_state_reset(float* state, int B, int H, int Dk, int Dv,
                            void* stream);
 
 /*
@@ -109,20 +115,27 @@ gdn_status gdn_state_reset(float* state, int B, int H, int Dk, int Dv,
  * kernels set when a bounded wait expires.  Returns GDN_OK, GDN_ERR_TIMEOUT
  * or GDN_ERR_CUDA.
  */
-gdn_status gdn_device_error(void* stream);
+GDN_API gdn_status gdn_device_error(void* stream);
 
 /*
  * Test hook: the number of polls a kernel's bounded wait makes before it
  * gives up (0 restores the default).  Affects launches enqueued after the
  * call, on every device.  Returns the previous value.
  */
-long long gdn_set_wait_limit(long long polls);
+GDN_API long long gdn_set_wait_limit(long long polls);
+
+/*
+ * Instrumentation (no counterpart on the pages): the number of kernels this
+ * process has enqueued through the library so far, on all devices and
+ * streams (launches captured into a CUDA graph count once, at capture).
+ */
+GDN_API unsigned long long gdn_launch_count(void);
 
 /* Static, human-readable name of a status; never NULL. */
-const char* gdn_status_string(gdn_status status);
+GDN_API const char* gdn_status_string(gdn_status status);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
-int gdn_version(void);
+GDN_API int gdn_version(void);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,125 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, and rejects bad arguments on the host before any CUDA call.
+
+Pointers below are fake integers: every rejection tested here happens in the
+library's pure host checks (null, sizes, dims, dtype, chunk, alignment,
+overlap), so nothing is dereferenced and no device is touched.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_deltanet_linear_chunked_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+
+def header_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"GDN_API\s+[\w\s\*]+?\b(gdn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    syms = header_symbols()
+    for name in ("gdn_chunk_fwd", "gdn_chunk_bidir", "gdn_state_reset", "gdn_status_string"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.load()
+    for name in header_symbols():
+        assert hasattr(lib, name), name
+    assert set(header_symbols()) == set(_lib.SIGNATURES)
+
+
+def test_status_strings_and_version():
+    lib = _lib.load()
+    names = [lib.gdn_status_string(i).decode() for i in range(6)]
+    assert names == ["GDN_OK", "GDN_ERR_INVALID_ARG", "GDN_ERR_UNSUPPORTED",
+                     "GDN_ERR_ALIAS", "GDN_ERR_CUDA", "GDN_ERR_TIMEOUT"]
+    assert lib.gdn_status_string(99).decode() == "GDN_ERR_UNKNOWN"
+    assert lib.gdn_version() >= 100
+
+
+# Fake, 16-byte aligned, non-overlapping "device" addresses.
+MB = 1 << 20
+BASE = 0x7F0000000000
+
+
+def fake(i):
+    return BASE + i * 256 * MB
+
+
+def call(entry="gdn_chunk_fwd", q=fake(0), k=fake(1), v=fake(2), g=fake(3), beta=fake(4),
+         s_in=fake(5), s_out=fake(6), out=fake(7), B=1, T=64, H=2, Dk=64, Dv=64,
+         dtype=_lib.GDN_BF16, chunk=0):
+    lib = _lib.load()
+    return getattr(lib, entry)(q, k, v, g, beta, s_in, s_out, out, B, T, H, Dk, Dv,
+                               dtype, chunk, None)
+
+
+@pytest.mark.parametrize("entry", ["gdn_chunk_fwd", "gdn_chunk_bidir"])
+def test_null_pointers_rejected(entry):
+    for name in ("q", "k", "v", "g", "beta", "out"):
+        assert call(entry, **{name: None}) == _lib.GDN_ERR_INVALID_ARG, name
+
+
+@pytest.mark.parametrize("entry", ["gdn_chunk_fwd", "gdn_chunk_bidir"])
+def test_bad_sizes_and_dims(entry):
+    assert call(entry, B=-1) == _lib.GDN_ERR_INVALID_ARG
+    assert call(entry, T=-5) == _lib.GDN_ERR_INVALID_ARG
+    assert call(entry, H=-2) == _lib.GDN_ERR_INVALID_ARG
+    for d in (0, 8, 24, 100, 144, 256):
+        assert call(entry, Dk=d) == _lib.GDN_ERR_UNSUPPORTED, d
+        assert call(entry, Dv=d) == _lib.GDN_ERR_UNSUPPORTED, d
+    assert call(entry, dtype=7) == _lib.GDN_ERR_INVALID_ARG
+    for c in (-1, 8, 48, 128):
+        assert call(entry, chunk=c) == _lib.GDN_ERR_INVALID_ARG, c
+
+
+def test_empty_batch_is_a_no_op():
+    # nothing to do: returns before touching any pointer or device
+    assert call(B=0, q=None, k=None, v=None, g=None, beta=None, out=None) == _lib.GDN_OK
+    assert call(H=0, q=None, k=None, v=None, g=None, beta=None, out=None) == _lib.GDN_OK
+
+
+def test_misaligned_pointers_rejected():
+    for name in ("q", "k", "v", "g", "beta", "s_in", "s_out", "out"):
+        assert call(**{name: fake(0 if name != "q" else 9) + 8}) == _lib.GDN_ERR_INVALID_ARG, name
+
+
+def test_overlaps_rejected():
+    # out overlapping any input or the state
+    for name in ("q", "k", "v", "g", "beta", "s_in", "s_out"):
+        assert call(**{name: fake(7) + 1024}) == _lib.GDN_ERR_ALIAS, name
+    # state_out overlapping an input
+    for name in ("q", "k", "v", "g", "beta"):
+        assert call(**{name: fake(6)}) == _lib.GDN_ERR_ALIAS, name
+    # state_out partially overlapping state_in (exact equality is allowed)
+    assert call(s_out=fake(5) + 4096) == _lib.GDN_ERR_ALIAS
+
+
+def test_valid_arguments_reach_the_device_checks_without_a_gpu():
+    # All host checks pass; with no usable device the call reports a CUDA
+    # error instead of crashing (on a GPU machine the fake pointers are rejected
+    # as not device memory).  Either way nothing is launched.
+    st = call()
+    assert st in (_lib.GDN_ERR_CUDA, _lib.GDN_ERR_INVALID_ARG)
+
+
+def test_state_reset_host_checks():
+    lib = _lib.load()
+    assert lib.gdn_state_reset(None, 0, 4, 16, 16, None) == _lib.GDN_OK
+    assert lib.gdn_state_reset(None, 1, 4, 16, 16, None) == _lib.GDN_ERR_INVALID_ARG
+    assert lib.gdn_state_reset(fake(1) + 4, 1, 4, 16, 16, None) == _lib.GDN_ERR_INVALID_ARG
+    assert lib.gdn_state_reset(fake(1), -1, 4, 16, 16, None) == _lib.GDN_ERR_INVALID_ARG
+
+
+def test_wait_limit_hook_round_trips():
+    lib = _lib.load()
+    old = lib.gdn_set_wait_limit(1234)
+    assert lib.gdn_set_wait_limit(0) == 1234
+    assert lib.gdn_set_wait_limit(old) > 0
