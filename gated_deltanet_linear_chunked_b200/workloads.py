@@ -103,10 +103,12 @@ def stress_cases() -> list[Workload]:
 
 def round_bf16(x: np.ndarray) -> np.ndarray:
     """Round fp32 values to the nearest bf16 (ties to even); returns fp32."""
-    x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
-    return u.astype(np.uint32).view(np.float32)
+    u = np.array(x, dtype=np.float32, copy=True).view(np.uint32)
+    lsb = (u >> 16) & 1
+    u += np.uint32(0x7FFF)          # finite inputs: no wrap-around
+    u += lsb
+    u &= np.uint32(0xFFFF0000)
+    return u.view(np.float32)
 
 
 def _l2_rows(x: np.ndarray) -> np.ndarray:

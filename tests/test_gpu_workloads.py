@@ -18,17 +18,20 @@ STACK_CHUNKS = 32
 def test_stacked_stream_layer_parity():
     """32 consecutive chunks x 15 GDN layers, bidirectional, state carried
     per layer, in model order (chunk-major, layer-minor) on one stream.
-    Every layer's outputs must be finite; layer 0 and layer 14 are compared
-    with the oracle on heads 0 and 19 over all 32 chunks, with the oracle
-    carrying its own state."""
+    Layers 0 and 14 get their own seeded inputs for every chunk and are
+    compared with the oracle on heads 0 and 19 over all 32 chunks (the
+    oracle carries its own state).  Layers 1-13 only keep the launch order
+    of the full stack: they run on a recycled pool of four seeded chunks
+    (each layer's state is independent, so they cannot affect 0 and 14);
+    their states must stay finite."""
     layers = wl.GDN_LAYERS
     H, D = 20, 112
     states = [torch.zeros(1, H, D, D, device="cuda") for _ in range(layers)]
     sampled = {0: {}, layers - 1: {}}
+    pool = [device_inputs(wl.stack_call(7, c)) for c in range(4)]
     for c in range(STACK_CHUNKS):
         for l in range(layers):
-            w = wl.stack_call(l, c)
-            x = device_inputs(w)
+            x = device_inputs(wl.stack_call(l, c)) if l in sampled else pool[(c + l) % 4]
             out, _ = gdn.chunk_bidir(x["q"], x["k"], x["v"], x["g"], x["beta"], states[l],
                                      state_out=states[l])
             if l in sampled:
