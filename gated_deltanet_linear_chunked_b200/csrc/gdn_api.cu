@@ -170,7 +170,20 @@ gdn_status scan(const void* q, const void* k, const void* v, const float* g,
   a.dtype = dtype; a.chunk = chunk; a.bidir = bidir; a.stream = s;
   a.err = err; a.wait_limit = g_wait_limit.load();
 
-  const cudaError_t e = launch_scan_serial(a);
+  cudaError_t e;
+  if (dtype == GDN_F32) {
+    e = launch_scan_serial(a);
+  } else {
+    // bf16: chunked tensor-core path with stream-ordered scratch
+    void* ws = nullptr;
+    const size_t bytes = chunk_tc_workspace_bytes(B, T, H, Dk, Dv, bidir);
+    e = cudaMallocAsync(&ws, bytes, s);
+    if (e == cudaSuccess) {
+      e = launch_chunk_tc(a, ws);
+      const cudaError_t f = cudaFreeAsync(ws, s);
+      if (e == cudaSuccess) e = f;
+    }
+  }
   return finish(s, e, err);
 }
 

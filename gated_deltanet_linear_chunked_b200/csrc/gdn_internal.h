@@ -34,6 +34,11 @@ void count_launches(unsigned n);
 // Token-serial SIMT scan (fp32 arithmetic, fp32 or bf16 I/O).
 cudaError_t launch_scan_serial(const ScanArgs& a);
 
+// Chunked tcgen05 path (bf16 I/O): stage A prep, stage B recurrence, stage C
+// output.  `workspace` must hold chunk_tc_workspace_bytes(...) bytes.
+size_t chunk_tc_workspace_bytes(int B, int T, int H, int Dk, int Dv, bool bidir);
+cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace);
+
 // Device error word values.
 enum : unsigned int {
   kErrNone = 0,
