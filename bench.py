@@ -38,8 +38,12 @@ METRIC = "GDN head-tokens/s and latent frames/s at 2640-tok chunk; % of B200 roo
 UNIT = "head-tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 N_SETS = 8                      # rotating input sets (8 x 49.7 MB > 126 MB L2)
-DOMINANT_KERNEL_SOURCE = "gated_deltanet_linear_chunked_b200/csrc/scan_serial.cu"
-DOMINANT_KERNEL_NAME = "gdn_scan_serial_kernel"
+KERNEL_SOURCES = {
+    "gdn_scan_serial_kernel": "gated_deltanet_linear_chunked_b200/csrc/scan_serial.cu",
+    "gdn_prep_kernel": "gated_deltanet_linear_chunked_b200/csrc/chunk_tc.cu",
+    "gdn_recur_kernel": "gated_deltanet_linear_chunked_b200/csrc/chunk_tc.cu",
+    "gdn_output_kernel": "gated_deltanet_linear_chunked_b200/csrc/chunk_tc.cu",
+}
 
 
 def parse():
@@ -82,26 +86,49 @@ def algorithmic_flops(w, bidir=False) -> int:
     return 2 * f if bidir else f
 
 
-def recorded_traffic():
-    """DRAM bytes per launch of the dominant kernel from the committed ncu
-    summary, if it was taken on the current source of that kernel."""
+def kernel_algorithmic_bytes(name, w) -> int:
+    """Each kernel's share of the path's algorithmic bytes: stage A reads k, v,
+    g, beta; stage B reads and writes the state; stage C reads q (and g) and
+    writes out.  The token-serial kernel does all of it.  The shares sum to
+    the path's bytes (q, k, v, out, g, beta + state)."""
+    es = 2 if w.dtype == "bf16" else 4
+    state = 2 * w.B * w.H * w.Dk * w.Dv * 4
+    if name == "gdn_prep_kernel":
+        return w.head_tokens * ((w.Dk + w.Dv) * es + 8)
+    if name == "gdn_recur_kernel":
+        return state
+    if name == "gdn_output_kernel":
+        return w.head_tokens * ((w.Dk + w.Dv) * es)
+    return algorithmic_bytes(w)
+
+
+def recorded_traffic(kernel):
+    """DRAM bytes per launch of `kernel` on this workload from the committed
+    ncu summary (profiles/dram_traffic.txt), if the summary was taken on the
+    kernel's current source; else None."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     try:
         lines = open(path).read().splitlines()
     except OSError:
         return None
-    kv = dict(l.split(":", 1) for l in lines if ":" in l and not l.startswith("#"))
-    kv = {k.strip(): v.strip() for k, v in kv.items()}
+    src_path = KERNEL_SOURCES.get(kernel)
+    if src_path is None:
+        return None
     try:
-        src = open(os.path.join(ROOT, DOMINANT_KERNEL_SOURCE), "rb").read()
+        digest = hashlib.sha256(open(os.path.join(ROOT, src_path), "rb").read()).hexdigest()
     except OSError:
         return None
-    if kv.get("kernel") != DOMINANT_KERNEL_NAME or kv.get("source_sha256") != hashlib.sha256(src).hexdigest():
-        return None
-    try:
-        return int(float(kv["dram_bytes_per_launch"]))
-    except (KeyError, ValueError):
-        return None
+    for line in lines:
+        if line.startswith("#") or not line.strip():
+            continue
+        parts = line.split()
+        # kernel  source_sha256  dram_bytes_per_launch
+        if len(parts) >= 3 and parts[0] == kernel and parts[1] == digest:
+            try:
+                return int(float(parts[2]))
+            except ValueError:
+                return None
+    return None
 
 
 class ClockSampler:
@@ -416,17 +443,44 @@ def main():
         extras["stack_32x15_bidir"] = {"ms": stack_ms, "latent_frames_per_s": frames / (stack_ms / 1000.0),
                                        "calls": n_chunks * wl.GDN_LAYERS, "timing": "direct calls"}
 
-    # ---- roofline of the dominant kernel (the one launch per step)
+    # ---- per-kernel device times (CUDA events on the launching stream,
+    # recorded by the library around each launch over a loop of direct calls)
+    n_prof = max(3, min(args.steps, 100))
+    import ctypes
+    _lib.check(lib.gdn_profile_begin(int(n_prof * max(1, launches_per_step) + 8)), "gdn_profile_begin")
+    with torch.cuda.stream(stream):
+        for i in range(n_prof):
+            step(i)
+    kms = (ctypes.c_float * 4)()
+    kn = (ctypes.c_int * 4)()
+    _lib.check(lib.gdn_profile_end(ctypes.addressof(kms), ctypes.addressof(kn), 4), "gdn_profile_end")
+    kernels = {}
+    for i in range(4):
+        if kn[i]:
+            name = lib.gdn_kernel_name(i).decode()
+            kernels[name] = {"launches": kn[i], "ms_per_launch": kms[i] / kn[i]}
+    tot = sum(v["ms_per_launch"] for v in kernels.values())
+    for v in kernels.values():
+        v["share"] = v["ms_per_launch"] / tot if tot else None
+
+    # ---- roofline of the dominant kernel
     peaks, peak_kind = load_peaks()
     bytes_step = algorithmic_bytes(w)
     flops_step = algorithmic_flops(w, w.mode == "bidir")
-    achieved = bytes_step / (ms_per_step / 1000.0) / 1e9
+    dom = max(kernels, key=lambda k: kernels[k]["ms_per_launch"])
+    dom_bytes = kernel_algorithmic_bytes(dom, w)
+    dom_ms = kernels[dom]["ms_per_launch"]
+    achieved = dom_bytes / (dom_ms / 1000.0) / 1e9
+    path_achieved = bytes_step / (ms_per_step / 1000.0) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": recorded_traffic(),
-                "peak_source": f"{peak_kind} hbm_gbs", "algorithmic_bytes": bytes_step,
-                "kernel": DOMINANT_KERNEL_NAME,
-                "tensor_frac_of_sustained": (flops_step / (ms_per_step / 1000.0) / 1e12)
-                / peaks["bf16_tflops_sustained"]}
+                "frac": achieved / peaks["hbm_gbs"], "traffic": recorded_traffic(dom),
+                "peak_source": f"{peak_kind} hbm_gbs", "kernel": dom,
+                "algorithmic_bytes_per_launch": dom_bytes, "ms_per_launch": dom_ms,
+                "kernels": kernels,
+                "path": {"algorithmic_bytes": bytes_step, "achieved": path_achieved,
+                         "frac": path_achieved / peaks["hbm_gbs"],
+                         "tensor_frac_of_sustained": (flops_step / (ms_per_step / 1000.0) / 1e12)
+                         / peaks["bf16_tflops_sustained"]}}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -34,6 +34,9 @@ SIGNATURES = {
     "gdn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "gdn_version": (ctypes.c_int, []),
     "gdn_launch_count": (ctypes.c_ulonglong, []),
+    "gdn_profile_begin": (ctypes.c_int, [ctypes.c_int]),
+    "gdn_profile_end": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]),
+    "gdn_kernel_name": (ctypes.c_char_p, [ctypes.c_int]),
 }
 
 _lock = threading.Lock()

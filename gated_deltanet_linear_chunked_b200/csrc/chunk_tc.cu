@@ -51,17 +51,17 @@ using namespace sm100;
 constexpr int kC = 64;            // tokens per chunk
 constexpr int kThreads = 128;
 constexpr int kSlab64 = kC * 16;  // bytes of one 8-column slab of a 64-row tile
-constexpr int kRecStages = 3;
+constexpr int kRecStages = 4;
 constexpr long long kDrainPolls = 1LL << 40;  // drains are bounded by the 2 s timer
 
 // ----------------------------------------------------------------- workspace
 struct Workspace {
   __nv_bfloat16* W;    // [dir][bh][chunk] [Dk/8][64][8]
   __nv_bfloat16* Ut;   // [dir][bh][chunk] [Dv/8][64][8]
-  __nv_bfloat16* Qc;   // [dir][bh][chunk] [Dk/8][128][8]
+  __nv_bfloat16* Qc;   // [dir][bh][chunk] [Dk/8][Dk][8]
   __nv_bfloat16* Rc;   // [dir][bh][chunk] [Dv/16][Dk][16]
   __nv_bfloat16* S;    // [dir][bh][chunk] [Dv/8][Dk][8]  state at chunk start
-  float* decay;        // [dir][bh][chunk] e^{gamma_C}
+  float* decay;        // [dir][bh][chunk] {e^{gamma_C}, 0, 0, 0} (16 B per chunk)
   int NBH, nC, Dk, Dv;
 
   __device__ size_t tile(int dir, int bh, int j) const {
@@ -351,18 +351,16 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
     const int r = tid;  // TMEM lane = feature row of Qc / Rc
     const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
     const size_t tile = ws.tile(dir, bh, j);
-    uint4* Qg = reinterpret_cast<uint4*>(ws.Qc + tile * 128 * Dk);
+    uint4* Qg = reinterpret_cast<uint4*>(ws.Qc + tile * (size_t)Dk * Dk);
     uint4* Rg = reinterpret_cast<uint4*>(ws.Rc + tile * (size_t)Dk * Dv);
     for (int c = 0; c < Dk / 16; ++c) {
       float v[16];
       tmem_ld16(tm + lane_base + 320 + 16 * c, v);
       tmem_wait_ld();
-      if (r >= Dk) {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) v[e] = 0.f;
+      if (r < Dk) {
+        Qg[(2 * c) * Dk + r] = pack8_bf16(v);
+        Qg[(2 * c + 1) * Dk + r] = pack8_bf16(v + 8);
       }
-      Qg[(2 * c) * 128 + r] = pack8_bf16(v);
-      Qg[(2 * c + 1) * 128 + r] = pack8_bf16(v + 8);
     }
     for (int c = 0; c < Dv / 16; ++c) {
       float v[16];
@@ -373,7 +371,8 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
         Rg[(c * Dk + r) * 2 + 1] = pack8_bf16(v + 8);
       }
     }
-    if (tid == 0) ws.decay[tile] = expf(gamC);
+    if (tid == 0)
+      reinterpret_cast<float4*>(ws.decay)[tile] = make_float4(expf(gamC), 0.f, 0.f, 0.f);
   }
   return true;
 }
@@ -411,7 +410,9 @@ struct RecSmemHead {
   uint64_t mma_bar;
   uint32_t tmem;
 };
-// dynamic layout: [head (128 B)] [S operand 4 KB] [stages: Qc tile | Rc slice]
+// dynamic layout: [head (128 B)] [S operand 4 KB] [stages: Qc | Rc slice | decay]
+// [2 KB tail pad: the M = 128 MMA reads up to 128 rows of Qc's last slab;
+//  rows past Dk are don't-care rows of D but must lie in shared memory]
 constexpr int kRecHeadBytes = 128;
 constexpr int kRecSBytes = 2 * 128 * 16;
 
@@ -421,8 +422,8 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
   uint8_t* Ssm = smem + kRecHeadBytes;
   uint8_t* stage0 = Ssm + kRecSBytes;
   const int Dk = ws.Dk, Dv = ws.Dv, nC = ws.nC;
-  const uint32_t qbytes = 128u * Dk * 2, rbytes = (uint32_t)Dk * 32;
-  const uint32_t stage_bytes = (qbytes + rbytes + 127) & ~127u;
+  const uint32_t qbytes = (uint32_t)Dk * Dk * 2, rbytes = (uint32_t)Dk * 32;
+  const uint32_t stage_bytes = (qbytes + rbytes + 16 + 127) & ~127u;
   const int tid = threadIdx.x, warp = tid >> 5;
   const int slice = blockIdx.x, bh = blockIdx.y, dir = blockIdx.z;
   const int r = tid;
@@ -443,10 +444,11 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
     const int jt = dir ? nC - 1 - c : c;
     const size_t tile = ws.tile(dir, bh, jt);
     uint8_t* st = stage0 + (c % kRecStages) * stage_bytes;
-    mbar_arrive_expect_tx(&hd.full[c % kRecStages], qbytes + rbytes);
-    bulk_load(st, ws.Qc + tile * 128 * Dk, qbytes, &hd.full[c % kRecStages]);
+    mbar_arrive_expect_tx(&hd.full[c % kRecStages], qbytes + rbytes + 16);
+    bulk_load(st, ws.Qc + tile * (size_t)Dk * Dk, qbytes, &hd.full[c % kRecStages]);
     bulk_load(st + qbytes, ws.Rc + tile * (size_t)Dk * Dv + (size_t)slice * Dk * 16, rbytes,
               &hd.full[c % kRecStages]);
+    bulk_load(st + qbytes + rbytes, ws.decay + 4 * tile, 16, &hd.full[c % kRecStages]);
   };
   int issued = 0;
   if (tid == 0)
@@ -480,7 +482,7 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
     if (tid == 0) {
       tc_fence_after_sync();
       for (int ks = 0; ks < Dk / 16; ++ks) {
-        const uint64_t a = sdesc(smem_u32(Qst) + ks * 2 * 2048, 2048, 128);
+        const uint64_t a = sdesc(smem_u32(Qst) + ks * 2 * Dk * 16, Dk * 16, 128);
         const uint64_t bd = sdesc(smem_u32(Ssm) + ks * 256, 128, 2048);
         mma_bf16(tm, a, bd, id, ks > 0);
       }
@@ -500,7 +502,7 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
       const uint4* Rs = reinterpret_cast<const uint4*>(Qst + qbytes);
       unpack8_bf16(Rs[2 * r], R);
       unpack8_bf16(Rs[2 * r + 1], R + 8);
-      const float a = __ldg(ws.decay + tile);
+      const float a = *reinterpret_cast<const float*>(Qst + qbytes + rbytes);
 #pragma unroll
       for (int e = 0; e < 16; ++e) S[e] = fmaf(a, S[e], R[e] - D[e]);
     }
@@ -749,8 +751,8 @@ bool make_map(CUtensorMap* m, const void* base, int B, int T, int H, int D) {
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 int recur_smem_bytes(int Dk) {
-  const int stage = ((128 * Dk * 2 + Dk * 32) + 127) & ~127;
-  return kRecHeadBytes + kRecSBytes + kRecStages * stage;
+  const int stage = ((Dk * Dk * 2 + Dk * 32 + 16) + 127) & ~127;
+  return kRecHeadBytes + kRecSBytes + kRecStages * stage + 2048;
 }
 
 // Opt the kernels into their dynamic shared memory, once per device.
@@ -781,8 +783,8 @@ cudaError_t set_smem_attrs() {
 size_t chunk_tc_workspace_bytes(int B, int T, int H, int Dk, int Dv, bool bidir) {
   const size_t tiles = (size_t)(bidir ? 2 : 1) * B * H * ((T + kC - 1) / kC);
   return align256(tiles * kC * Dk * 2) + align256(tiles * kC * Dv * 2) +
-         align256(tiles * 128 * Dk * 2) + align256(tiles * (size_t)Dk * Dv * 2) +
-         align256(tiles * (size_t)Dk * Dv * 2) + align256(tiles * 4);
+         align256(tiles * (size_t)Dk * Dk * 2) + align256(tiles * (size_t)Dk * Dv * 2) +
+         align256(tiles * (size_t)Dk * Dv * 2) + align256(tiles * 16);
 }
 
 cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
@@ -796,7 +798,7 @@ cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
   uint8_t* p = static_cast<uint8_t*>(workspace);
   ws.W = reinterpret_cast<__nv_bfloat16*>(p);  p += align256(tiles * kC * a.Dk * 2);
   ws.Ut = reinterpret_cast<__nv_bfloat16*>(p); p += align256(tiles * kC * a.Dv * 2);
-  ws.Qc = reinterpret_cast<__nv_bfloat16*>(p); p += align256(tiles * 128 * a.Dk * 2);
+  ws.Qc = reinterpret_cast<__nv_bfloat16*>(p); p += align256(tiles * (size_t)a.Dk * a.Dk * 2);
   ws.Rc = reinterpret_cast<__nv_bfloat16*>(p); p += align256(tiles * (size_t)a.Dk * a.Dv * 2);
   ws.S = reinterpret_cast<__nv_bfloat16*>(p);  p += align256(tiles * (size_t)a.Dk * a.Dv * 2);
   ws.decay = reinterpret_cast<float*>(p);
@@ -807,16 +809,25 @@ cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
       !make_map(&mv, a.v, a.B, a.T, a.H, a.Dv))
     return cudaErrorInvalidValue;
 
-  gdn_prep_kernel<<<dim3(nC, NBH, ndir), kThreads, sizeof(PrepSmem), a.stream>>>(
-      mk, mv, a.g, a.beta, ws, a.T, a.H, a.wait_limit, a.err);
+  {
+    ProfileScope ps(a.stream, kKernPrep);
+    gdn_prep_kernel<<<dim3(nC, NBH, ndir), kThreads, sizeof(PrepSmem), a.stream>>>(
+        mk, mv, a.g, a.beta, ws, a.T, a.H, a.wait_limit, a.err);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  gdn_recur_kernel<<<dim3(a.Dv / 16, NBH, ndir), kThreads, recur_smem_bytes(a.Dk), a.stream>>>(
-      a.state_in, a.state_out, ws, a.wait_limit, a.err);
+  {
+    ProfileScope ps(a.stream, kKernRecur);
+    gdn_recur_kernel<<<dim3(a.Dv / 16, NBH, ndir), kThreads, recur_smem_bytes(a.Dk), a.stream>>>(
+        a.state_in, a.state_out, ws, a.wait_limit, a.err);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  gdn_output_kernel<<<dim3(nC, NBH), kThreads, sizeof(OutSmem), a.stream>>>(
-      mq, mk, a.g, static_cast<__nv_bfloat16*>(a.out), ws, a.T, a.H, ndir, a.wait_limit, a.err);
+  {
+    ProfileScope ps(a.stream, kKernOutput);
+    gdn_output_kernel<<<dim3(nC, NBH), kThreads, sizeof(OutSmem), a.stream>>>(
+        mq, mk, a.g, static_cast<__nv_bfloat16*>(a.out), ws, a.T, a.H, ndir, a.wait_limit, a.err);
+  }
   e = cudaGetLastError();
   if (e == cudaSuccess) count_launches(3);
   return e;

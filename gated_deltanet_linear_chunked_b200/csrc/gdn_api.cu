@@ -10,6 +10,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <new>
 
 #include "gdn_internal.h"
 
@@ -191,6 +192,31 @@ gdn_status scan(const void* q, const void* k, const void* v, const float* g,
 
 void count_launches(unsigned n) { g_launches.fetch_add(n); }
 
+// ------------------------------------------------------------- profiling
+namespace {
+struct Profile {
+  std::mutex mu;
+  bool armed = false;
+  int capacity = 0, used = 0;
+  cudaEvent_t* ev = nullptr;  // 2 per launch
+  int* ids = nullptr;
+};
+Profile g_prof;
+}  // namespace
+
+ProfileScope::ProfileScope(cudaStream_t s, int kernel_id) : stream_(s), slot_(-1) {
+  std::lock_guard<std::mutex> lock(g_prof.mu);
+  if (!g_prof.armed || g_prof.used >= g_prof.capacity) return;
+  slot_ = g_prof.used++;
+  g_prof.ids[slot_] = kernel_id;
+  cudaEventRecord(g_prof.ev[2 * slot_], stream_);
+}
+
+ProfileScope::~ProfileScope() {
+  if (slot_ < 0) return;
+  cudaEventRecord(g_prof.ev[2 * slot_ + 1], stream_);
+}
+
 }  // namespace gdn
 
 extern "C" {
@@ -265,5 +291,73 @@ const char* gdn_status_string(gdn_status status) {
 int gdn_version(void) { return 100; }
 
 unsigned long long gdn_launch_count(void) { return gdn::g_launches.load(); }
+
+gdn_status gdn_profile_begin(int max_launches) {
+  using gdn::g_prof;
+  if (max_launches < 1) return GDN_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_prof.mu);
+  if (g_prof.armed) return GDN_ERR_INVALID_ARG;
+  g_prof.ev = new (std::nothrow) cudaEvent_t[2 * (size_t)max_launches];
+  g_prof.ids = new (std::nothrow) int[max_launches];
+  if (!g_prof.ev || !g_prof.ids) {
+    delete[] g_prof.ev; delete[] g_prof.ids;
+    g_prof.ev = nullptr; g_prof.ids = nullptr;
+    return GDN_ERR_INVALID_ARG;
+  }
+  for (int i = 0; i < 2 * max_launches; ++i) {
+    if (cudaEventCreate(&g_prof.ev[i]) != cudaSuccess) {
+      for (int j = 0; j < i; ++j) cudaEventDestroy(g_prof.ev[j]);
+      delete[] g_prof.ev; delete[] g_prof.ids;
+      g_prof.ev = nullptr; g_prof.ids = nullptr;
+      cudaGetLastError();
+      return GDN_ERR_CUDA;
+    }
+  }
+  g_prof.capacity = max_launches;
+  g_prof.used = 0;
+  g_prof.armed = true;
+  return GDN_OK;
+}
+
+gdn_status gdn_profile_end(float* ms, int* n, int nids) {
+  using gdn::g_prof;
+  std::lock_guard<std::mutex> lock(g_prof.mu);
+  if (!g_prof.armed) return GDN_ERR_INVALID_ARG;
+  for (int i = 0; i < nids; ++i) {
+    if (ms) ms[i] = 0.f;
+    if (n) n[i] = 0;
+  }
+  gdn_status st = GDN_OK;
+  for (int i = 0; i < g_prof.used; ++i) {
+    float t = 0.f;
+    if (cudaEventSynchronize(g_prof.ev[2 * i + 1]) != cudaSuccess ||
+        cudaEventElapsedTime(&t, g_prof.ev[2 * i], g_prof.ev[2 * i + 1]) != cudaSuccess) {
+      st = GDN_ERR_CUDA;
+      cudaGetLastError();
+      continue;
+    }
+    const int id = g_prof.ids[i];
+    if (id >= 0 && id < nids) {
+      if (ms) ms[id] += t;
+      if (n) n[id] += 1;
+    }
+  }
+  for (int i = 0; i < 2 * g_prof.capacity; ++i) cudaEventDestroy(g_prof.ev[i]);
+  delete[] g_prof.ev; delete[] g_prof.ids;
+  g_prof.ev = nullptr; g_prof.ids = nullptr;
+  g_prof.capacity = g_prof.used = 0;
+  g_prof.armed = false;
+  return st;
+}
+
+const char* gdn_kernel_name(int id) {
+  switch (id) {
+    case gdn::kKernSerial: return "gdn_scan_serial_kernel";
+    case gdn::kKernPrep: return "gdn_prep_kernel";
+    case gdn::kKernRecur: return "gdn_recur_kernel";
+    case gdn::kKernOutput: return "gdn_output_kernel";
+  }
+  return "unknown";
+}
 
 }  // extern "C"

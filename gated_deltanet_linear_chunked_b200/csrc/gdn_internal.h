@@ -28,6 +28,25 @@ struct ScanArgs {
   long long wait_limit;    // polls before a bounded wait gives up
 };
 
+// Kernel ids for the profiling hook.
+enum KernelId : int {
+  kKernSerial = 0,
+  kKernPrep = 1,
+  kKernRecur = 2,
+  kKernOutput = 3,
+  kNumKernelIds = 4,
+};
+
+// While profiling is armed, records CUDA events around one launch.
+class ProfileScope {
+ public:
+  ProfileScope(cudaStream_t s, int kernel_id);
+  ~ProfileScope();
+ private:
+  cudaStream_t stream_;
+  int slot_;
+};
+
 // Adds n to the process-wide count of kernels the library has enqueued.
 void count_launches(unsigned n);
 

@@ -235,6 +235,7 @@ cudaError_t launch_scan_serial(const ScanArgs& a) {
     e = cudaMallocAsync(reinterpret_cast<void**>(&acc), bytes, a.stream);
     if (e != cudaSuccess) return e;
   }
+  ProfileScope ps(a.stream, kKernSerial);
   if (a.dtype == GDN_F32) {
     gdn_scan_serial_kernel<float><<<grid, kThreads, 0, a.stream>>>(
         static_cast<const float*>(a.q), static_cast<const float*>(a.k),

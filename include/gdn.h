@@ -131,6 +131,21 @@ GDN_API long long gdn_set_wait_limit(long long polls);
  */
 GDN_API unsigned long long gdn_launch_count(void);
 
+/*
+ * Instrumentation (no counterpart on the pages): per-kernel device times.
+ * gdn_profile_begin arms CUDA-event timing of every kernel the library
+ * launches from then on (on the launching stream, up to `max_launches`
+ * launches, current device); gdn_profile_end synchronises the recorded
+ * events, disarms, and writes for each kernel id i < nids the total
+ * milliseconds ms[i] and launch count n[i].  Kernel ids: 0 token-serial scan,
+ * 1 stage A (prep), 2 stage B (recurrence), 3 stage C (output); names from
+ * gdn_kernel_name.  Not thread-safe against concurrent calls on other
+ * threads; meant for benchmarks.
+ */
+GDN_API gdn_status gdn_profile_begin(int max_launches);
+GDN_API gdn_status gdn_profile_end(float* ms, int* n, int nids);
+GDN_API const char* gdn_kernel_name(int id);
+
 /* Static, human-readable name of a status; never NULL. */
 GDN_API const char* gdn_status_string(gdn_status status);
 
