@@ -54,6 +54,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return done != 0;
 }
 
+// Non-blocking probe of the same phase.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -61,9 +74,12 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 // Wait for phase `parity` of `bar` to complete.  Gives up (returns false)
-// after `limit` polls or about two seconds, whichever comes first.
+// after `limit` polls or about two seconds, whichever comes first.  The first
+// poll never blocks, so a limit of 1 fails whenever the phase is not already
+// complete; later polls use try_wait, which may suspend the thread briefly.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_test_wait(bar, parity)) return true;
+  if (limit <= 1) return false;
   const uint64_t t0 = globaltimer_ns();
   for (long long i = 1; i < limit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
