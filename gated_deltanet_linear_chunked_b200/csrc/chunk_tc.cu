@@ -122,80 +122,128 @@ __device__ float row_rnorm(const uint8_t* tile, int r, int D) {
 }
 
 // ============================================================ stage A: prep
+// Shared memory: K and V tiles stay for the whole tile; the solve's fp32
+// scratch and the bf16 A operands TW/TU are dead once W and U~ are in TMEM,
+// so the scaled B operands Wp/Up reuse their space.  ~102 KB: two CTAs/SM.
+constexpr int kLd = 68;  // fp32 row stride of the 64 x 64 scratch (16 B aligned rows)
 struct PrepSmem {
   alignas(128) uint8_t K[16 * kSlab64];   // [16 slabs][64][8]; slabs >= Dk/8 zero
   alignas(128) uint8_t V[16 * kSlab64];
-  alignas(128) uint8_t TW[8 * kSlab64];   // Tm diag(beta e^g / |k|), K-major A
-  alignas(128) uint8_t TU[8 * kSlab64];   // Tm diag(beta), K-major A
-  alignas(128) uint8_t Wp[16 * kSlab64];  // diag(e^{gC-g}/|k|) W, MN-major B
-  alignas(128) uint8_t Up[16 * kSlab64];  // diag(e^{gC-g}/|k|) U~, MN-major B
-  float A[64][65];                         // strictly triangular A, then scratch
-  float T[64][65];                         // (I + A)^-1
-  float X[3][16][17];
-  float g[64], beta[64], gam[64], rn[64], csW[64], csU[64];
+  union alignas(128) U {
+    struct {
+      uint8_t TW[8 * kSlab64];             // Tm diag(beta e^g / |k|), K-major A
+      uint8_t TU[8 * kSlab64];             // Tm diag(beta), K-major A
+      float A[64][kLd];                    // strictly lower A in scan order
+      float T[64][kLd];                    // (I + A)^-1 in scan order
+      float Y[64][kLd];                    // product scratch
+    } a;
+    struct {
+      uint8_t Wp[16 * kSlab64];            // diag(e^{gC-g}/|k|) W, MN-major B
+      uint8_t Up[16 * kSlab64];            // diag(e^{gC-g}/|k|) U~, MN-major B
+    } b;
+  } u;
+  float g[64], beta[64], gam[64], g2[64], rn[64], csW[64], csU[64];
   uint64_t tma_bar, mma_bar;
   uint32_t tmem;
 };
 
-// Blocked inverse of the unit triangular 64 x 64 matrix I + A (A in s.A,
-// strictly lower in "scan index" p = map(r)), written to s.T.  Diagonal
-// 16 x 16 blocks by forward substitution (one warp per block, one lane per
-// column), then the off-diagonal blocks in order of distance from the
-// diagonal: T_ij = -T_ii sum_{j<=k<i} A_ik T_kj.
-__device__ void unit_triangular_inverse(PrepSmem& s, int reverse) {
+constexpr float kLog2e = 1.4426950408889634f;
+
+// In-place blocked inverse of the unit lower-triangular 64 x 64 matrix
+// I + A (A strictly lower, scan order) into T:
+//   16 x 16 diagonal blocks by right-looking forward substitution (one lane
+//   per column: the dependent chain is one FMA per row);
+//   16 -> 32:  T_hl = -T_hh (A_hl T_ll) for the two 32 x 32 diagonal halves;
+//   32 -> 64:  T_HL = -T_HH (A_HL T_LL) for the lower-left 32 x 32 block.
+__device__ void unit_lower_inverse(PrepSmem::U& u) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  auto M = [reverse](int p) { return reverse ? 63 - p : p; };  // scan index -> row
-  // zero T
-  for (int i = tid; i < 64 * 64; i += kThreads) s.T[i >> 6][i & 63] = 0.f;
+  float (*A)[kLd] = u.a.A;
+  float (*T)[kLd] = u.a.T;
+  float (*Y)[kLd] = u.a.Y;
+  for (int i = tid; i < 64 * 64; i += kThreads) T[i >> 6][i & 63] = 0.f;
   __syncthreads();
-  // diagonal blocks
+  if (lane < 16) {
+    const int b0 = 16 * warp, j = lane;
+    float acc[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) acc[t] = (t == j) ? 1.f : 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float x = acc[i];
+#pragma unroll
+      for (int t = i + 1; t < 16; ++t) acc[t] = fmaf(-A[b0 + t][b0 + i], x, acc[t]);
+    }
+#pragma unroll
+    for (int t = 0; t < 16; ++t) T[b0 + t][b0 + j] = acc[t];
+  }
+  __syncthreads();
+  // 16 -> 32: pairs (blocks 1,0) and (3,2); thread: 1 x 4 strip of a 16 x 16 block
   {
-    const int blk = warp, j = lane & 15;
-    if (lane < 16) {
-      float x[16];
+    const int pr = tid >> 6, idx = tid & 63, r = idx >> 2, c0 = (idx & 3) * 4;
+    const int hb = 32 * pr + 16, lb = 32 * pr;  // row offset of the high block, col offset of the low
+    float y[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int t = 0; t < 16; ++t) {
-        float acc = (t == j) ? 1.f : 0.f;
-#pragma unroll
-        for (int i = 0; i < t; ++i) acc = fmaf(-s.A[M(16 * blk + t)][M(16 * blk + i)], x[i], acc);
-        x[t] = (t < j) ? 0.f : acc;
-      }
-#pragma unroll
-      for (int t = 0; t < 16; ++t) s.T[M(16 * blk + t)][M(16 * blk + j)] = x[t];
+    for (int k = 0; k < 16; ++k) {
+      const float a = A[hb + r][lb + k];
+      const float4 t = *reinterpret_cast<const float4*>(&T[lb + k][lb + c0]);
+      y[0] = fmaf(a, t.x, y[0]); y[1] = fmaf(a, t.y, y[1]);
+      y[2] = fmaf(a, t.z, y[2]); y[3] = fmaf(a, t.w, y[3]);
     }
+    *reinterpret_cast<float4*>(&Y[hb + r][lb + c0]) = make_float4(y[0], y[1], y[2], y[3]);
+    __syncthreads();
+    float z[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const float a = T[hb + r][hb + k];
+      const float4 t = *reinterpret_cast<const float4*>(&Y[hb + k][lb + c0]);
+      z[0] = fmaf(a, t.x, z[0]); z[1] = fmaf(a, t.y, z[1]);
+      z[2] = fmaf(a, t.z, z[2]); z[3] = fmaf(a, t.w, z[3]);
+    }
+    *reinterpret_cast<float4*>(&T[hb + r][lb + c0]) = make_float4(-z[0], -z[1], -z[2], -z[3]);
   }
   __syncthreads();
-  // off-diagonal blocks by distance d = 1, 2, 3
-  for (int d = 1; d <= 3; ++d) {
-    const int nb = 4 - d;  // blocks (j + d, j), j = 0 .. nb-1
-    for (int idx = tid; idx < nb * 256; idx += kThreads) {
-      const int jb = idx >> 8, e = idx & 255, r = e >> 4, c = e & 15;
-      const int ib = jb + d;
-      float acc = 0.f;
-      for (int kb = jb; kb < ib; ++kb)
-#pragma unroll
-        for (int k = 0; k < 16; ++k)
-          acc = fmaf(s.A[M(16 * ib + r)][M(16 * kb + k)], s.T[M(16 * kb + k)][M(16 * jb + c)], acc);
-      s.X[jb][r][c] = acc;
+  // 32 -> 64: thread: 2 x 4 tile of the 32 x 32 block
+  {
+    const int r0 = (tid >> 3) * 2, c0 = (tid & 7) * 4;
+    float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+    for (int k = 0; k < 32; ++k) {
+      const float a0 = A[32 + r0][k], a1 = A[33 + r0][k];
+      const float4 t = *reinterpret_cast<const float4*>(&T[k][c0]);
+      y0[0] = fmaf(a0, t.x, y0[0]); y0[1] = fmaf(a0, t.y, y0[1]);
+      y0[2] = fmaf(a0, t.z, y0[2]); y0[3] = fmaf(a0, t.w, y0[3]);
+      y1[0] = fmaf(a1, t.x, y1[0]); y1[1] = fmaf(a1, t.y, y1[1]);
+      y1[2] = fmaf(a1, t.z, y1[2]); y1[3] = fmaf(a1, t.w, y1[3]);
     }
+    *reinterpret_cast<float4*>(&Y[32 + r0][c0]) = make_float4(y0[0], y0[1], y0[2], y0[3]);
+    *reinterpret_cast<float4*>(&Y[33 + r0][c0]) = make_float4(y1[0], y1[1], y1[2], y1[3]);
     __syncthreads();
-    for (int idx = tid; idx < nb * 256; idx += kThreads) {
-      const int jb = idx >> 8, e = idx & 255, r = e >> 4, c = e & 15;
-      const int ib = jb + d;
-      float acc = 0.f;
-#pragma unroll
-      for (int k = 0; k < 16; ++k) acc = fmaf(s.T[M(16 * ib + r)][M(16 * ib + k)], s.X[jb][k][c], acc);
-      s.T[M(16 * ib + r)][M(16 * jb + c)] = -acc;
+    float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+    for (int k = 0; k < 32; ++k) {
+      const float a0 = T[32 + r0][32 + k], a1 = T[33 + r0][32 + k];
+      const float4 t = *reinterpret_cast<const float4*>(&Y[32 + k][c0]);
+      z0[0] = fmaf(a0, t.x, z0[0]); z0[1] = fmaf(a0, t.y, z0[1]);
+      z0[2] = fmaf(a0, t.z, z0[2]); z0[3] = fmaf(a0, t.w, z0[3]);
+      z1[0] = fmaf(a1, t.x, z1[0]); z1[1] = fmaf(a1, t.y, z1[1]);
+      z1[2] = fmaf(a1, t.z, z1[2]); z1[3] = fmaf(a1, t.w, z1[3]);
     }
-    __syncthreads();
+    *reinterpret_cast<float4*>(&T[32 + r0][c0]) = make_float4(-z0[0], -z0[1], -z0[2], -z0[3]);
+    *reinterpret_cast<float4*>(&T[33 + r0][c0]) = make_float4(-z1[0], -z1[1], -z1[2], -z1[3]);
   }
+  __syncthreads();
 }
 
+// Scan position of memory row r within a tile.
+template <int REV>
+__device__ __forceinline__ int scan_pos(int r) { return REV ? 63 - r : r; }
+
+template <int REV>
 __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                           const float* __restrict__ g, const float* __restrict__ beta,
                           const Workspace& ws, int T, int H, long long limit, unsigned* err) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int j = blockIdx.x, bh = blockIdx.y, dir = blockIdx.z;
+  const int j = blockIdx.x, bh = blockIdx.y, dir = REV;
   const int b = bh / H, h = bh - b * H;
   const int Dk = ws.Dk, Dv = ws.Dv;
   const int t0 = j * kC;
@@ -218,7 +266,7 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
     s.beta[tid] = bv;
   }
   __syncthreads();
-  if (warp == 0) warp_gamma(s.g, s.gam, dir);
+  if (warp == 0) warp_gamma(s.g, s.gam, REV);
   if (!block_wait(&s.tma_bar, 0, limit, err)) return false;
 
   if (tid < kC) s.rn[tid] = row_rnorm(s.K, tid, Dk);
@@ -233,61 +281,73 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
     mma_commit(&s.mma_bar);
   }
   __syncthreads();
-  const float gamC = dir ? s.gam[0] : s.gam[63];
+  const float gamC = REV ? s.gam[0] : s.gam[63];
   if (tid < kC) {
-    const float eg = expf(s.gam[tid]);
-    s.csW[tid] = s.beta[tid] * eg * s.rn[tid];
+    s.g2[tid] = s.gam[tid] * kLog2e;
+    s.csW[tid] = s.beta[tid] * expf(s.gam[tid]) * s.rn[tid];
     s.csU[tid] = s.beta[tid];
   }
   if (!block_wait(&s.mma_bar, 0, limit, err)) return false;
   tc_fence_after_sync();
 
-  // A_ri = beta_r e^{gam_r - gam_i} G_ri / (|k_r| |k_i|) for i before r
+  // A[p][q] = beta_r e^{gam_r - gam_i} G_ri / (|k_r| |k_i|), p = pos(r) > q = pos(i)
   {
     const int r = 16 * warp + (lane & 15);
+    const int p = scan_pos<REV>(r);
     const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
-    for (int c = 0; c < 4; ++c) {
-      float v[16];
-      tmem_ld16(tm + lane_base + 16 * c, v);
-      tmem_wait_ld();
-      if (lane < 16) {
-        const float br = s.beta[r] * s.rn[r], gr = s.gam[r];
+    float v[64];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int i = 16 * c + e;
-          const bool before = dir ? (i > r) : (i < r);
-          s.A[r][i] = before ? br * expf(gr - s.gam[i]) * v[e] * s.rn[i] : 0.f;
+    for (int c = 0; c < 4; ++c) {
+      float* vc = v + 16 * c;
+      tmem_ld16(tm + lane_base + 16 * c, *reinterpret_cast<float(*)[16]>(vc));
+    }
+    tmem_wait_ld();
+    if (lane < 16) {
+      const float br = s.beta[r] * s.rn[r], g2r = s.g2[r];
+      float* Arow = s.u.a.A[p];
+#pragma unroll
+      for (int q4 = 0; q4 < 16; ++q4) {
+        float o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int q = 4 * q4 + e;
+          const int i = scan_pos<REV>(q);
+          o[e] = (q < p) ? br * exp2f(g2r - s.g2[i]) * v[i] * s.rn[i] : 0.f;
         }
+        *reinterpret_cast<float4*>(Arow + 4 * q4) = make_float4(o[0], o[1], o[2], o[3]);
       }
     }
   }
   __syncthreads();
-  unit_triangular_inverse(s, dir);
+  unit_lower_inverse(s.u);
 
-  // TW = Tm diag(beta e^gam / |k|), TU = Tm diag(beta) as bf16 K-major A operands
+  // TW[r][i] = T[pos r][pos i] beta_i e^{gam_i} / |k_i|, TU[r][i] = T[..] beta_i,
+  // as bf16 K-major A operands in memory order
   for (int idx = tid; idx < 64 * 8; idx += kThreads) {
     const int r = idx & 63, ks = idx >> 6;
-    float w[8], u[8];
+    const float* Trow = s.u.a.T[scan_pos<REV>(r)];
+    float w[8], uu[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      const float t = s.T[r][8 * ks + e];
-      w[e] = t * s.csW[8 * ks + e];
-      u[e] = t * s.csU[8 * ks + e];
+      const int i = 8 * ks + e;
+      const float t = Trow[scan_pos<REV>(i)];
+      w[e] = t * s.csW[i];
+      uu[e] = t * s.csU[i];
     }
-    reinterpret_cast<uint4*>(s.TW + ks * kSlab64)[r] = pack8_bf16(w);
-    reinterpret_cast<uint4*>(s.TU + ks * kSlab64)[r] = pack8_bf16(u);
+    reinterpret_cast<uint4*>(s.u.a.TW + ks * kSlab64)[r] = pack8_bf16(w);
+    reinterpret_cast<uint4*>(s.u.a.TU + ks * kSlab64)[r] = pack8_bf16(uu);
   }
   block_sync_async();
   // W = TW K (N = Dk), U~ = TU V (N = Dv); K and V read MN-major (N = feature)
   if (tid == 0) {
     const uint32_t idW = idesc_bf16(64, Dk, 0, 1), idU = idesc_bf16(64, Dv, 0, 1);
     for (int ks = 0; ks < kC / 16; ++ks) {
-      const uint64_t aw = sdesc(smem_u32(s.TW) + ks * 2 * kSlab64, kSlab64, 128);
-      const uint64_t au = sdesc(smem_u32(s.TU) + ks * 2 * kSlab64, kSlab64, 128);
+      const uint64_t aw = sdesc(smem_u32(s.u.a.TW) + ks * 2 * kSlab64, kSlab64, 128);
+      const uint64_t au = sdesc(smem_u32(s.u.a.TU) + ks * 2 * kSlab64, kSlab64, 128);
       const uint64_t bk = sdesc(smem_u32(s.K) + ks * 256, 128, kSlab64);
       const uint64_t bv = sdesc(smem_u32(s.V) + ks * 256, 128, kSlab64);
-      mma_bf16(tm + 64, aw, bk, idW, ks > 0);
-      mma_bf16(tm + 192, au, bv, idU, ks > 0);
+      mma_bf16(tm, aw, bk, idW, ks > 0);
+      mma_bf16(tm + 128, au, bv, idU, ks > 0);
     }
     mma_commit(&s.mma_bar);
   }
@@ -304,7 +364,7 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
     uint4* Ug = reinterpret_cast<uint4*>(ws.Ut + tile * kC * Dv);
     for (int c = 0; c < Dk / 16; ++c) {
       float v[16];
-      tmem_ld16(tm + lane_base + 64 + 16 * c, v);
+      tmem_ld16(tm + lane_base + 16 * c, v);
       tmem_wait_ld();
       if (lane < 16) {
         float sv[16];
@@ -312,13 +372,13 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
         for (int e = 0; e < 16; ++e) sv[e] = v[e] * sc;
         Wg[(2 * c) * kC + r] = pack8_bf16(v);
         Wg[(2 * c + 1) * kC + r] = pack8_bf16(v + 8);
-        reinterpret_cast<uint4*>(s.Wp + (2 * c) * kSlab64)[r] = pack8_bf16(sv);
-        reinterpret_cast<uint4*>(s.Wp + (2 * c + 1) * kSlab64)[r] = pack8_bf16(sv + 8);
+        reinterpret_cast<uint4*>(s.u.b.Wp + (2 * c) * kSlab64)[r] = pack8_bf16(sv);
+        reinterpret_cast<uint4*>(s.u.b.Wp + (2 * c + 1) * kSlab64)[r] = pack8_bf16(sv + 8);
       }
     }
     for (int c = 0; c < Dv / 16; ++c) {
       float v[16];
-      tmem_ld16(tm + lane_base + 192 + 16 * c, v);
+      tmem_ld16(tm + lane_base + 128 + 16 * c, v);
       tmem_wait_ld();
       if (lane < 16) {
         float sv[16];
@@ -326,8 +386,8 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
         for (int e = 0; e < 16; ++e) sv[e] = v[e] * sc;
         Ug[(2 * c) * kC + r] = pack8_bf16(v);
         Ug[(2 * c + 1) * kC + r] = pack8_bf16(v + 8);
-        reinterpret_cast<uint4*>(s.Up + (2 * c) * kSlab64)[r] = pack8_bf16(sv);
-        reinterpret_cast<uint4*>(s.Up + (2 * c + 1) * kSlab64)[r] = pack8_bf16(sv + 8);
+        reinterpret_cast<uint4*>(s.u.b.Up + (2 * c) * kSlab64)[r] = pack8_bf16(sv);
+        reinterpret_cast<uint4*>(s.u.b.Up + (2 * c + 1) * kSlab64)[r] = pack8_bf16(sv + 8);
       }
     }
   }
@@ -338,10 +398,10 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
     const uint32_t idQ = idesc_bf16(128, Dk, 1, 1), idR = idesc_bf16(128, Dv, 1, 1);
     for (int ks = 0; ks < kC / 16; ++ks) {
       const uint64_t a = sdesc(smem_u32(s.K) + ks * 256, 128, kSlab64);
-      const uint64_t bw = sdesc(smem_u32(s.Wp) + ks * 256, 128, kSlab64);
-      const uint64_t bu = sdesc(smem_u32(s.Up) + ks * 256, 128, kSlab64);
-      mma_bf16(tm + 320, a, bw, idQ, ks > 0);
-      mma_bf16(tm + 0, a, bu, idR, ks > 0);
+      const uint64_t bw = sdesc(smem_u32(s.u.b.Wp) + ks * 256, 128, kSlab64);
+      const uint64_t bu = sdesc(smem_u32(s.u.b.Up) + ks * 256, 128, kSlab64);
+      mma_bf16(tm, a, bw, idQ, ks > 0);
+      mma_bf16(tm + 128, a, bu, idR, ks > 0);
     }
     mma_commit(&s.mma_bar);
   }
@@ -355,7 +415,7 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
     uint4* Rg = reinterpret_cast<uint4*>(ws.Rc + tile * (size_t)Dk * Dv);
     for (int c = 0; c < Dk / 16; ++c) {
       float v[16];
-      tmem_ld16(tm + lane_base + 320 + 16 * c, v);
+      tmem_ld16(tm + lane_base + 16 * c, v);
       tmem_wait_ld();
       if (r < Dk) {
         Qg[(2 * c) * Dk + r] = pack8_bf16(v);
@@ -364,7 +424,7 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
     }
     for (int c = 0; c < Dv / 16; ++c) {
       float v[16];
-      tmem_ld16(tm + lane_base + 16 * c, v);
+      tmem_ld16(tm + lane_base + 128 + 16 * c, v);
       tmem_wait_ld();
       if (r < Dk) {
         Rg[(c * Dk + r) * 2] = pack8_bf16(v);
@@ -377,7 +437,7 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
   return true;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const float* __restrict__ g, const float* __restrict__ beta, Workspace ws, int T,
                 int H, long long limit, unsigned* err) {
@@ -390,7 +450,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     fence_mbar_init();
   }
   if ((tid >> 5) == 0) {
-    tmem_alloc(&s.tmem, 512);
+    tmem_alloc(&s.tmem, 256);
     tmem_relinquish();
   }
   {  // zero the feature slabs past Dk (rows of the M = 128 products)
@@ -398,10 +458,13 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     for (int i = tid; i < (16 - ws.Dk / 8) * kSlab64 / 16; i += kThreads) z[i] = make_uint4(0, 0, 0, 0);
   }
   block_sync_async();
-  prep_body(s, &tm_k, &tm_v, g, beta, ws, T, H, limit, err);
+  if (blockIdx.z == 0)
+    prep_body<0>(s, &tm_k, &tm_v, g, beta, ws, T, H, limit, err);
+  else
+    prep_body<1>(s, &tm_k, &tm_v, g, beta, ws, T, H, limit, err);
   tc_fence_before_sync();
   __syncthreads();
-  if ((tid >> 5) == 0) tmem_dealloc(s.tmem, 512);
+  if ((tid >> 5) == 0) tmem_dealloc(s.tmem, 256);
 }
 
 // ======================================================= stage B: recurrence
@@ -538,21 +601,36 @@ gdn_recur_kernel(const float* state_in, float* state_out, Workspace ws, long lon
 }
 
 // ========================================================== stage C: output
-struct OutSmem {
-  alignas(128) uint8_t Q[16 * kSlab64];   // raw q tile [slab][64][8]
-  alignas(128) uint8_t K[16 * kSlab64];   // raw k tile
-  alignas(128) uint8_t W[16 * kSlab64];   // W of this direction
-  alignas(128) uint8_t Ut[16 * kSlab64];  // U~ of this direction
-  alignas(128) uint8_t S[16 * 128 * 16];  // state at chunk start [Dv/8][Dk][8]
-  alignas(128) uint8_t P[8 * kSlab64];    // masked, gated Q K^T, K-major A
-  alignas(128) uint8_t U[16 * kSlab64];   // U, MN-major B
-  alignas(128) uint8_t Qs[16 * kSlab64];  // diag(e^gamma) Q, K-major A
+// Dynamic shared-memory layout (offsets from Dk, Dv, 128 B aligned):
+//   Q   [Dk/8][64][8]  raw q tile (TMA)
+//   K   [Dk/8][64][8]  raw k tile (TMA); after P = Q K^T it holds Qs = diag(e^g) Q
+//   W   [max(Dk,Dv)/8][64][8]  W of the current direction; after W S it holds
+//                  U [Dv/8][64][8] (B operand)
+//   Ut  [Dv/8][64][8]  U~ of the current direction
+//   S   [Dv/8][Dk][8]  state at the chunk's start (MN-major B operand)
+//   P   [8][64][8]     masked, gated Q K^T (K-major A operand)
+// ~90 KB at Dk = Dv = 112: two CTAs per SM.
+struct OutLayout {
+  uint32_t q, k, w, ut, s, p, small, total;
+  __host__ __device__ OutLayout(int Dk, int Dv) {
+    auto al = [](uint32_t x) { return (x + 127u) & ~127u; };
+    q = 0;
+    k = al(q + 64u * Dk * 2);
+    w = al(k + 64u * Dk * 2);
+    ut = al(w + 64u * (Dk > Dv ? Dk : Dv) * 2);  // W, later U: room for either
+    s = al(ut + 64u * Dv * 2);
+    p = al(s + (uint32_t)Dk * Dv * 2);
+    small = al(p + 8u * kSlab64);
+    total = small + 1024;
+  }
+};
+struct OutSmall {
   float g[64], gam[64], rnq[64], rnk[64];
   uint64_t tma_bar, ld_bar, mma_bar;
   uint32_t tmem;
 };
 
-__device__ bool output_body(OutSmem& s, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
+__device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                             const float* __restrict__ g, __nv_bfloat16* __restrict__ out,
                             const Workspace& ws, int T, int H, int ndir, long long limit,
                             unsigned* err) {
@@ -560,73 +638,86 @@ __device__ bool output_body(OutSmem& s, const CUtensorMap* tm_q, const CUtensorM
   const int j = blockIdx.x, bh = blockIdx.y;
   const int b = bh / H, h = bh - b * H;
   const int Dk = ws.Dk, Dv = ws.Dv;
+  const OutLayout L(Dk, Dv);
+  uint8_t* sQ = smem + L.q;
+  uint8_t* sK = smem + L.k;   // then Qs
+  uint8_t* sW = smem + L.w;   // then U
+  uint8_t* sUt = smem + L.ut;
+  uint8_t* sS = smem + L.s;
+  uint8_t* sP = smem + L.p;
+  OutSmall& sm = *reinterpret_cast<OutSmall*>(smem + L.small);
   const int t0 = j * kC;
   const int nvalid = min(kC, T - t0);
-  const uint32_t tm = s.tmem;
-  const uint32_t tmO = tm, tmU = tm + 128, tmP = tm + 256;
+  const uint32_t tm = sm.tmem;
+  // TMEM: P = Q K^T [0,64); D_O [64,192); D_U see below
+  const uint32_t tmP = tm, tmO = tm + 64;
   const uint32_t wbytes = kC * Dk * 2, ubytes = kC * Dv * 2, sbytes = Dk * Dv * 2;
   auto issue_dir = [&](int dir) {
     const size_t tile = ws.tile(dir, bh, j);
-    mbar_arrive_expect_tx(&s.ld_bar, wbytes + ubytes + sbytes);
-    bulk_load(s.W, ws.W + tile * kC * Dk, wbytes, &s.ld_bar);
-    bulk_load(s.Ut, ws.Ut + tile * kC * Dv, ubytes, &s.ld_bar);
-    bulk_load(s.S, ws.S + tile * (size_t)Dk * Dv, sbytes, &s.ld_bar);
+    mbar_arrive_expect_tx(&sm.ld_bar, wbytes + ubytes + sbytes);
+    bulk_load(sW, ws.W + tile * kC * Dk, wbytes, &sm.ld_bar);
+    bulk_load(sUt, ws.Ut + tile * kC * Dv, ubytes, &sm.ld_bar);
+    bulk_load(sS, ws.S + tile * (size_t)Dk * Dv, sbytes, &sm.ld_bar);
   };
   if (tid == 0) {
-    mbar_arrive_expect_tx(&s.tma_bar, 2 * (Dk / 8) * kSlab64);
+    mbar_arrive_expect_tx(&sm.tma_bar, 2 * (Dk / 8) * kSlab64);
     for (int sl = 0; sl < Dk / 8; ++sl) {
-      tma_load_4d(s.Q + sl * kSlab64, tm_q, &s.tma_bar, 8 * sl, h, t0, b);
-      tma_load_4d(s.K + sl * kSlab64, tm_k, &s.tma_bar, 8 * sl, h, t0, b);
+      tma_load_4d(sQ + sl * kSlab64, tm_q, &sm.tma_bar, 8 * sl, h, t0, b);
+      tma_load_4d(sK + sl * kSlab64, tm_k, &sm.tma_bar, 8 * sl, h, t0, b);
     }
     issue_dir(0);
   }
-  if (tid < kC) s.g[tid] = (tid < nvalid) ? __ldg(g + ((size_t)b * T + t0 + tid) * H + h) : 0.f;
-  if (!block_wait(&s.tma_bar, 0, limit, err)) {
-    mbar_wait(&s.ld_bar, 0, kDrainPolls);
+  if (tid < kC) sm.g[tid] = (tid < nvalid) ? __ldg(g + ((size_t)b * T + t0 + tid) * H + h) : 0.f;
+  if (!block_wait(&sm.tma_bar, 0, limit, err)) {
+    mbar_wait(&sm.ld_bar, 0, kDrainPolls);
     return false;
   }
   if (tid < kC) {
-    s.rnq[tid] = row_rnorm(s.Q, tid, Dk);
-    s.rnk[tid] = row_rnorm(s.K, tid, Dk);
+    sm.rnq[tid] = row_rnorm(sQ, tid, Dk);
+    sm.rnk[tid] = row_rnorm(sK, tid, Dk);
   }
   uint32_t mma_phase = 0;
   const int r = 16 * warp + (lane & 15);
   const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
   for (int dir = 0; dir < ndir; ++dir) {
+    // D_U: direction 0 borrows D_O's columns (D_O is first written after D_U
+    // is consumed); direction 1 needs its own, [192, 320) of a 512-column
+    // allocation, because D_O then holds direction 0's sum.
+    const uint32_t tmU = tm + (dir == 0 ? 64u : 192u);
     __syncthreads();
-    if (warp == 0) warp_gamma(s.g, s.gam, dir);
-    if (!block_wait(&s.ld_bar, dir & 1, limit, err)) return false;
+    if (warp == 0) warp_gamma(sm.g, sm.gam, dir);
+    if (!block_wait(&sm.ld_bar, dir & 1, limit, err)) return false;
     if (tid == 0) {
       tc_fence_after_sync();
       if (dir == 0) {  // P = Q K^T, shared by both directions
         const uint32_t idP = idesc_bf16(64, 64, 0, 0);
         for (int ks = 0; ks < Dk / 16; ++ks)
-          mma_bf16(tmP, sdesc(smem_u32(s.Q) + ks * 2 * kSlab64, kSlab64, 128),
-                   sdesc(smem_u32(s.K) + ks * 2 * kSlab64, kSlab64, 128), idP, ks > 0);
+          mma_bf16(tmP, sdesc(smem_u32(sQ) + ks * 2 * kSlab64, kSlab64, 128),
+                   sdesc(smem_u32(sK) + ks * 2 * kSlab64, kSlab64, 128), idP, ks > 0);
       }
       // D_U = W S  (M = 64, N = Dv, K = Dk); S read MN-major (N = value column)
       const uint32_t idU = idesc_bf16(64, Dv, 0, 1);
       for (int ks = 0; ks < Dk / 16; ++ks)
-        mma_bf16(tmU, sdesc(smem_u32(s.W) + ks * 2 * kSlab64, kSlab64, 128),
-                 sdesc(smem_u32(s.S) + ks * 256, 128, Dk * 16), idU, ks > 0);
-      mma_commit(&s.mma_bar);
+        mma_bf16(tmU, sdesc(smem_u32(sW) + ks * 2 * kSlab64, kSlab64, 128),
+                 sdesc(smem_u32(sS) + ks * 256, 128, Dk * 16), idU, ks > 0);
+      mma_commit(&sm.mma_bar);
     }
-    if (!block_wait(&s.mma_bar, mma_phase & 1, limit, err)) return false;
+    if (!block_wait(&sm.mma_bar, mma_phase & 1, limit, err)) return false;
     ++mma_phase;
     tc_fence_after_sync();
-    // U = U~ - W S  -> s.U (MN-major B: [slab][64 tokens][8])
+    // U = U~ - W S  -> sW (MN-major B: [slab][64 tokens][8])
     for (int c = 0; c < Dv / 16; ++c) {
       float v[16];
       tmem_ld16(tmU + lane_base + 16 * c, v);
       tmem_wait_ld();
       if (lane < 16) {
         float ut[16];
-        unpack8_bf16(reinterpret_cast<const uint4*>(s.Ut + (2 * c) * kSlab64)[r], ut);
-        unpack8_bf16(reinterpret_cast<const uint4*>(s.Ut + (2 * c + 1) * kSlab64)[r], ut + 8);
+        unpack8_bf16(reinterpret_cast<const uint4*>(sUt + (2 * c) * kSlab64)[r], ut);
+        unpack8_bf16(reinterpret_cast<const uint4*>(sUt + (2 * c + 1) * kSlab64)[r], ut + 8);
 #pragma unroll
         for (int e = 0; e < 16; ++e) ut[e] -= v[e];
-        reinterpret_cast<uint4*>(s.U + (2 * c) * kSlab64)[r] = pack8_bf16(ut);
-        reinterpret_cast<uint4*>(s.U + (2 * c + 1) * kSlab64)[r] = pack8_bf16(ut + 8);
+        reinterpret_cast<uint4*>(sW + (2 * c) * kSlab64)[r] = pack8_bf16(ut);
+        reinterpret_cast<uint4*>(sW + (2 * c + 1) * kSlab64)[r] = pack8_bf16(ut + 8);
       }
     }
     // P'_ri = (q_r . k_i) / |k_i| * e^{gam_r - gam_i} for i at or before r
@@ -635,47 +726,47 @@ __device__ bool output_body(OutSmem& s, const CUtensorMap* tm_q, const CUtensorM
       tmem_ld16(tmP + lane_base + 16 * c, v);
       tmem_wait_ld();
       if (lane < 16) {
-        const float gr = s.gam[r];
+        const float g2r = sm.gam[r] * kLog2e;
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int i = 16 * c + e;
           const bool incl = dir ? (i >= r) : (i <= r);
-          v[e] = incl ? v[e] * s.rnk[i] * expf(gr - s.gam[i]) : 0.f;
+          v[e] = incl ? v[e] * sm.rnk[i] * exp2f(g2r - sm.gam[i] * kLog2e) : 0.f;
         }
-        reinterpret_cast<uint4*>(s.P + (2 * c) * kSlab64)[r] = pack8_bf16(v);
-        reinterpret_cast<uint4*>(s.P + (2 * c + 1) * kSlab64)[r] = pack8_bf16(v + 8);
+        reinterpret_cast<uint4*>(sP + (2 * c) * kSlab64)[r] = pack8_bf16(v);
+        reinterpret_cast<uint4*>(sP + (2 * c + 1) * kSlab64)[r] = pack8_bf16(v + 8);
       }
     }
-    // Qs = diag(e^gam) Q
+    // Qs = diag(e^gam) Q -> sK (K is dead once P is in TMEM)
     if (lane < 16) {
-      const float eg = expf(s.gam[r]);
+      const float eg = expf(sm.gam[r]);
       for (int sl = 0; sl < Dk / 8; ++sl) {
         float x[8];
-        unpack8_bf16(reinterpret_cast<const uint4*>(s.Q + sl * kSlab64)[r], x);
+        unpack8_bf16(reinterpret_cast<const uint4*>(sQ + sl * kSlab64)[r], x);
 #pragma unroll
         for (int e = 0; e < 8; ++e) x[e] *= eg;
-        reinterpret_cast<uint4*>(s.Qs + sl * kSlab64)[r] = pack8_bf16(x);
+        reinterpret_cast<uint4*>(sK + sl * kSlab64)[r] = pack8_bf16(x);
       }
     }
     block_sync_async();
     if (tid == 0) {
       const uint32_t idO = idesc_bf16(64, Dv, 0, 1);
       for (int ks = 0; ks < Dk / 16; ++ks)
-        mma_bf16(tmO, sdesc(smem_u32(s.Qs) + ks * 2 * kSlab64, kSlab64, 128),
-                 sdesc(smem_u32(s.S) + ks * 256, 128, Dk * 16), idO, (dir > 0) || (ks > 0));
+        mma_bf16(tmO, sdesc(smem_u32(sK) + ks * 2 * kSlab64, kSlab64, 128),
+                 sdesc(smem_u32(sS) + ks * 256, 128, Dk * 16), idO, (dir > 0) || (ks > 0));
       for (int ks = 0; ks < kC / 16; ++ks)
-        mma_bf16(tmO, sdesc(smem_u32(s.P) + ks * 2 * kSlab64, kSlab64, 128),
-                 sdesc(smem_u32(s.U) + ks * 256, 128, kSlab64), idO, 1);
-      mma_commit(&s.mma_bar);
+        mma_bf16(tmO, sdesc(smem_u32(sP) + ks * 2 * kSlab64, kSlab64, 128),
+                 sdesc(smem_u32(sW) + ks * 256, 128, kSlab64), idO, 1);
+      mma_commit(&sm.mma_bar);
     }
-    if (!block_wait(&s.mma_bar, mma_phase & 1, limit, err)) return false;
+    if (!block_wait(&sm.mma_bar, mma_phase & 1, limit, err)) return false;
     ++mma_phase;
     if (dir + 1 < ndir && tid == 0) issue_dir(dir + 1);
   }
   tc_fence_after_sync();
   // O = diag(1/|q|) D_O -> out (rows of this chunk that exist)
   {
-    const float rq = s.rnq[r];
+    const float rq = sm.rnq[r];
     for (int c = 0; c < Dv / 16; ++c) {
       float v[16];
       tmem_ld16(tmO + lane_base + 16 * c, v);
@@ -692,28 +783,30 @@ __device__ bool output_body(OutSmem& s, const CUtensorMap* tm_q, const CUtensorM
   return true;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 gdn_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const float* __restrict__ g, __nv_bfloat16* __restrict__ out, Workspace ws, int T,
                   int H, int ndir, long long limit, unsigned* err) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  OutSmem& s = *reinterpret_cast<OutSmem*>(smem_raw);
+  const OutLayout L(ws.Dk, ws.Dv);
+  OutSmall& sm = *reinterpret_cast<OutSmall*>(smem_raw + L.small);
   const int tid = threadIdx.x;
+  const uint32_t ncols = ndir > 1 ? 512u : 256u;
   if (tid == 0) {
-    mbar_init(&s.tma_bar, 1);
-    mbar_init(&s.ld_bar, 1);
-    mbar_init(&s.mma_bar, 1);
+    mbar_init(&sm.tma_bar, 1);
+    mbar_init(&sm.ld_bar, 1);
+    mbar_init(&sm.mma_bar, 1);
     fence_mbar_init();
   }
   if ((tid >> 5) == 0) {
-    tmem_alloc(&s.tmem, 512);
+    tmem_alloc(&sm.tmem, ncols);
     tmem_relinquish();
   }
   block_sync_async();
-  output_body(s, &tm_q, &tm_k, g, out, ws, T, H, ndir, limit, err);
+  output_body(smem_raw, &tm_q, &tm_k, g, out, ws, T, H, ndir, limit, err);
   tc_fence_before_sync();
   __syncthreads();
-  if ((tid >> 5) == 0) tmem_dealloc(s.tmem, 512);
+  if ((tid >> 5) == 0) tmem_dealloc(sm.tmem, ncols);
 }
 
 // ===================================================================== host
@@ -773,7 +866,7 @@ cudaError_t set_smem_attrs() {
                              recur_smem_bytes(128));
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(gdn_output_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sizeof(OutSmem));
+                             (int)OutLayout(128, 128).total);
   if (e == cudaSuccess) done[dev] = true;
   return e;
 }
@@ -825,7 +918,7 @@ cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
   if (e != cudaSuccess) return e;
   {
     ProfileScope ps(a.stream, kKernOutput);
-    gdn_output_kernel<<<dim3(nC, NBH), kThreads, sizeof(OutSmem), a.stream>>>(
+    gdn_output_kernel<<<dim3(nC, NBH), kThreads, OutLayout(a.Dk, a.Dv).total, a.stream>>>(
         mq, mk, a.g, static_cast<__nv_bfloat16*>(a.out), ws, a.T, a.H, ndir, a.wait_limit, a.err);
   }
   e = cudaGetLastError();
