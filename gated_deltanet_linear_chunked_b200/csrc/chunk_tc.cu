@@ -610,6 +610,11 @@ gdn_recur_kernel(const float* state_in, float* state_out, Workspace ws, long lon
 //   S   [Dv/8][Dk][8]  state at the chunk's start (MN-major B operand)
 //   P   [8][64][8]     masked, gated Q K^T (K-major A operand)
 // ~90 KB at Dk = Dv = 112: two CTAs per SM.
+struct OutSmall {
+  float g[64], gam[64], rnq[64], rnk[64];
+  uint64_t tma_bar, ld_bar, mma_bar;
+  uint32_t tmem;
+};
 struct OutLayout {
   uint32_t q, k, w, ut, s, p, small, total;
   __host__ __device__ OutLayout(int Dk, int Dv) {
@@ -621,13 +626,8 @@ struct OutLayout {
     s = al(ut + 64u * Dv * 2);
     p = al(s + (uint32_t)Dk * Dv * 2);
     small = al(p + 8u * kSlab64);
-    total = small + 1024;
+    total = al(small + (uint32_t)sizeof(OutSmall));
   }
-};
-struct OutSmall {
-  float g[64], gam[64], rnq[64], rnk[64];
-  uint64_t tma_bar, ld_bar, mma_bar;
-  uint32_t tmem;
 };
 
 __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
