@@ -49,7 +49,8 @@ namespace {
 using namespace sm100;
 
 constexpr int kC = 64;            // tokens per chunk
-constexpr int kThreads = 128;
+constexpr int kThreads = 128;     // stage B
+constexpr int kWideThreads = 256; // stages A and C: two warps per TMEM lane quadrant
 constexpr int kSlab64 = kC * 16;  // bytes of one 8-column slab of a 64-row tile
 constexpr int kRecStages = 4;
 constexpr long long kDrainPolls = 1LL << 40;  // drains are bounded by the 2 s timer
@@ -142,7 +143,9 @@ struct PrepSmem {
       uint8_t Up[16 * kSlab64];            // diag(e^{gC-g}/|k|) U~, MN-major B
     } b;
   } u;
-  float g[64], beta[64], gam[64], g2[64], rn[64], csW[64], csU[64];
+  float g[64], beta[64], gam[64], rn[64], csW[64], csU[64];
+  float arow[64];      // beta_r |k_r|^-1 e^{gam_r - m_b(r)}       (scan order)
+  float bcol[8][64];   // |k_q|^-1 e^{m_b - gam_q}, b = 8-row block (scan order)
   uint64_t tma_bar, mma_bar;
   uint32_t tmem;
 };
@@ -160,9 +163,10 @@ __device__ void unit_lower_inverse(PrepSmem::U& u) {
   float (*A)[kLd] = u.a.A;
   float (*T)[kLd] = u.a.T;
   float (*Y)[kLd] = u.a.Y;
-  for (int i = tid; i < 64 * 64; i += kThreads) T[i >> 6][i & 63] = 0.f;
+  for (int i = tid; i < 64 * 16; i += kWideThreads)
+    reinterpret_cast<float4*>(T[i >> 4])[i & 15] = make_float4(0.f, 0.f, 0.f, 0.f);
   __syncthreads();
-  if (lane < 16) {
+  if (warp < 4 && lane < 16) {
     const int b0 = 16 * warp, j = lane;
     float acc[16];
 #pragma unroll
@@ -177,59 +181,53 @@ __device__ void unit_lower_inverse(PrepSmem::U& u) {
     for (int t = 0; t < 16; ++t) T[b0 + t][b0 + j] = acc[t];
   }
   __syncthreads();
-  // 16 -> 32: pairs (blocks 1,0) and (3,2); thread: 1 x 4 strip of a 16 x 16 block
+  // 16 -> 32: pairs (blocks 1,0) and (3,2); thread: 1 x 2 strip of a 16 x 16 block
   {
-    const int pr = tid >> 6, idx = tid & 63, r = idx >> 2, c0 = (idx & 3) * 4;
-    const int hb = 32 * pr + 16, lb = 32 * pr;  // row offset of the high block, col offset of the low
-    float y[4] = {0.f, 0.f, 0.f, 0.f};
+    const int pr = tid >> 7, idx = tid & 127, r = idx >> 3, c0 = (idx & 7) * 2;
+    const int hb = 32 * pr + 16, lb = 32 * pr;
+    float y0 = 0.f, y1 = 0.f;
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
       const float a = A[hb + r][lb + k];
-      const float4 t = *reinterpret_cast<const float4*>(&T[lb + k][lb + c0]);
-      y[0] = fmaf(a, t.x, y[0]); y[1] = fmaf(a, t.y, y[1]);
-      y[2] = fmaf(a, t.z, y[2]); y[3] = fmaf(a, t.w, y[3]);
+      const float2 t = *reinterpret_cast<const float2*>(&T[lb + k][lb + c0]);
+      y0 = fmaf(a, t.x, y0);
+      y1 = fmaf(a, t.y, y1);
     }
-    *reinterpret_cast<float4*>(&Y[hb + r][lb + c0]) = make_float4(y[0], y[1], y[2], y[3]);
+    *reinterpret_cast<float2*>(&Y[hb + r][lb + c0]) = make_float2(y0, y1);
     __syncthreads();
-    float z[4] = {0.f, 0.f, 0.f, 0.f};
+    float z0 = 0.f, z1 = 0.f;
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
       const float a = T[hb + r][hb + k];
-      const float4 t = *reinterpret_cast<const float4*>(&Y[hb + k][lb + c0]);
+      const float2 t = *reinterpret_cast<const float2*>(&Y[hb + k][lb + c0]);
+      z0 = fmaf(a, t.x, z0);
+      z1 = fmaf(a, t.y, z1);
+    }
+    *reinterpret_cast<float2*>(&T[hb + r][lb + c0]) = make_float2(-z0, -z1);
+  }
+  __syncthreads();
+  // 32 -> 64: thread: 1 x 4 strip of the 32 x 32 block
+  {
+    const int r = tid >> 3, c0 = (tid & 7) * 4;
+    float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+    for (int k = 0; k < 32; ++k) {
+      const float a = A[32 + r][k];
+      const float4 t = *reinterpret_cast<const float4*>(&T[k][c0]);
+      y[0] = fmaf(a, t.x, y[0]); y[1] = fmaf(a, t.y, y[1]);
+      y[2] = fmaf(a, t.z, y[2]); y[3] = fmaf(a, t.w, y[3]);
+    }
+    *reinterpret_cast<float4*>(&Y[32 + r][c0]) = make_float4(y[0], y[1], y[2], y[3]);
+    __syncthreads();
+    float z[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+    for (int k = 0; k < 32; ++k) {
+      const float a = T[32 + r][32 + k];
+      const float4 t = *reinterpret_cast<const float4*>(&Y[32 + k][c0]);
       z[0] = fmaf(a, t.x, z[0]); z[1] = fmaf(a, t.y, z[1]);
       z[2] = fmaf(a, t.z, z[2]); z[3] = fmaf(a, t.w, z[3]);
     }
-    *reinterpret_cast<float4*>(&T[hb + r][lb + c0]) = make_float4(-z[0], -z[1], -z[2], -z[3]);
-  }
-  __syncthreads();
-  // 32 -> 64: thread: 2 x 4 tile of the 32 x 32 block
-  {
-    const int r0 = (tid >> 3) * 2, c0 = (tid & 7) * 4;
-    float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-    for (int k = 0; k < 32; ++k) {
-      const float a0 = A[32 + r0][k], a1 = A[33 + r0][k];
-      const float4 t = *reinterpret_cast<const float4*>(&T[k][c0]);
-      y0[0] = fmaf(a0, t.x, y0[0]); y0[1] = fmaf(a0, t.y, y0[1]);
-      y0[2] = fmaf(a0, t.z, y0[2]); y0[3] = fmaf(a0, t.w, y0[3]);
-      y1[0] = fmaf(a1, t.x, y1[0]); y1[1] = fmaf(a1, t.y, y1[1]);
-      y1[2] = fmaf(a1, t.z, y1[2]); y1[3] = fmaf(a1, t.w, y1[3]);
-    }
-    *reinterpret_cast<float4*>(&Y[32 + r0][c0]) = make_float4(y0[0], y0[1], y0[2], y0[3]);
-    *reinterpret_cast<float4*>(&Y[33 + r0][c0]) = make_float4(y1[0], y1[1], y1[2], y1[3]);
-    __syncthreads();
-    float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-    for (int k = 0; k < 32; ++k) {
-      const float a0 = T[32 + r0][32 + k], a1 = T[33 + r0][32 + k];
-      const float4 t = *reinterpret_cast<const float4*>(&Y[32 + k][c0]);
-      z0[0] = fmaf(a0, t.x, z0[0]); z0[1] = fmaf(a0, t.y, z0[1]);
-      z0[2] = fmaf(a0, t.z, z0[2]); z0[3] = fmaf(a0, t.w, z0[3]);
-      z1[0] = fmaf(a1, t.x, z1[0]); z1[1] = fmaf(a1, t.y, z1[1]);
-      z1[2] = fmaf(a1, t.z, z1[2]); z1[3] = fmaf(a1, t.w, z1[3]);
-    }
-    *reinterpret_cast<float4*>(&T[32 + r0][c0]) = make_float4(-z0[0], -z0[1], -z0[2], -z0[3]);
-    *reinterpret_cast<float4*>(&T[33 + r0][c0]) = make_float4(-z1[0], -z1[1], -z1[2], -z1[3]);
+    *reinterpret_cast<float4*>(&T[32 + r][c0]) = make_float4(-z[0], -z[1], -z[2], -z[3]);
   }
   __syncthreads();
 }
@@ -283,38 +281,58 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
   __syncthreads();
   const float gamC = REV ? s.gam[0] : s.gam[63];
   if (tid < kC) {
-    s.g2[tid] = s.gam[tid] * kLog2e;
     s.csW[tid] = s.beta[tid] * expf(s.gam[tid]) * s.rn[tid];
     s.csU[tid] = s.beta[tid];
   }
   if (!block_wait(&s.mma_bar, 0, limit, err)) return false;
   tc_fence_after_sync();
 
-  // A[p][q] = beta_r e^{gam_r - gam_i} G_ri / (|k_r| |k_i|), p = pos(r) > q = pos(i)
+  // A[p][q] = beta_r e^{gam_r - gam_i} G_ri / (|k_r| |k_i|) for scan positions
+  // q < p, formed as arow[p] G bcol[b(p)][q]: the gate factor is split at
+  // m_b = gam at the first scan position of p's 8-row block b, so both factors
+  // are bounded (|gam_r - m_b| and, inside the block, |m_b - gam_i| span at
+  // most 7 tokens) and only 8 x 64 + 64 exponentials are taken per tile.
   {
-    const int r = 16 * warp + (lane & 15);
-    const int p = scan_pos<REV>(r);
-    const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
-    float v[64];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float* vc = v + 16 * c;
-      tmem_ld16(tm + lane_base + 16 * c, *reinterpret_cast<float(*)[16]>(vc));
+    for (int e = tid; e < 8 * 64; e += kWideThreads) {
+      const int blk = e >> 6, q = e & 63;
+      const int i = REV ? 63 - q : q;
+      const float mb = s.gam[REV ? 63 - 8 * blk : 8 * blk];
+      s.bcol[blk][q] = (q < 8 * blk + 8) ? s.rn[i] * exp2f((mb - s.gam[i]) * kLog2e) : 0.f;
     }
+    if (tid < 64) {
+      const int p = tid, r = REV ? 63 - p : p;
+      const float mb = s.gam[REV ? 63 - 8 * (p >> 3) : 8 * (p >> 3)];
+      s.arow[p] = s.beta[r] * s.rn[r] * exp2f((s.gam[r] - mb) * kLog2e);
+    }
+    __syncthreads();
+    const int quad = warp & 3, half = warp >> 2;
+    const int r = 16 * quad + (lane & 15);
+    const int p = scan_pos<REV>(r);
+    const uint32_t lane_base = static_cast<uint32_t>(32 * quad) << 16;
+    // this warp half covers scan columns q in [32 half, 32 half + 32); the
+    // matching memory columns i = pos(q) form one contiguous 32-column range
+    const int i0 = REV ? 32 - 32 * half : 32 * half;
+    float v[32];
+    tmem_ld16(tm + lane_base + i0, *reinterpret_cast<float(*)[16]>(v));
+    tmem_ld16(tm + lane_base + i0 + 16, *reinterpret_cast<float(*)[16]>(v + 16));
     tmem_wait_ld();
     if (lane < 16) {
-      const float br = s.beta[r] * s.rn[r], g2r = s.g2[r];
+      const float ap = s.arow[p];
+      const float* bc = s.bcol[p >> 3];
       float* Arow = s.u.a.A[p];
 #pragma unroll
-      for (int q4 = 0; q4 < 16; ++q4) {
+      for (int q4 = 0; q4 < 8; ++q4) {
+        const int qb = 32 * half + 4 * q4;
+        const float4 b4 = *reinterpret_cast<const float4*>(bc + qb);
+        const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
         float o[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int q = 4 * q4 + e;
-          const int i = scan_pos<REV>(q);
-          o[e] = (q < p) ? br * exp2f(g2r - s.g2[i]) * v[i] * s.rn[i] : 0.f;
+          const int q = qb + e;
+          const int iv = REV ? 31 - (4 * q4 + e) : 4 * q4 + e;  // index into v
+          o[e] = (q < p) ? ap * v[iv] * bb[e] : 0.f;
         }
-        *reinterpret_cast<float4*>(Arow + 4 * q4) = make_float4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<float4*>(Arow + qb) = make_float4(o[0], o[1], o[2], o[3]);
       }
     }
   }
@@ -323,7 +341,7 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
 
   // TW[r][i] = T[pos r][pos i] beta_i e^{gam_i} / |k_i|, TU[r][i] = T[..] beta_i,
   // as bf16 K-major A operands in memory order
-  for (int idx = tid; idx < 64 * 8; idx += kThreads) {
+  for (int idx = tid; idx < 64 * 8; idx += kWideThreads) {
     const int r = idx & 63, ks = idx >> 6;
     const float* Trow = s.u.a.T[scan_pos<REV>(r)];
     float w[8], uu[8];
@@ -354,15 +372,17 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
   if (!block_wait(&s.mma_bar, 1, limit, err)) return false;
   tc_fence_after_sync();
 
-  // W, U~ -> workspace (bf16 [slab][64][8]); scaled copies -> Wp, Up
+  // W, U~ -> workspace (bf16 [slab][64][8]); scaled copies -> Wp, Up.
+  // Warps w and w + 4 share a TMEM lane quadrant and split the column blocks.
   {
-    const int r = 16 * warp + (lane & 15);
-    const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
+    const int quad = warp & 3, half = warp >> 2;
+    const int r = 16 * quad + (lane & 15);
+    const uint32_t lane_base = static_cast<uint32_t>(32 * quad) << 16;
     const size_t tile = ws.tile(dir, bh, j);
     const float sc = expf(gamC - s.gam[r]) * s.rn[r];
     uint4* Wg = reinterpret_cast<uint4*>(ws.W + tile * kC * Dk);
     uint4* Ug = reinterpret_cast<uint4*>(ws.Ut + tile * kC * Dv);
-    for (int c = 0; c < Dk / 16; ++c) {
+    for (int c = half; c < Dk / 16; c += 2) {
       float v[16];
       tmem_ld16(tm + lane_base + 16 * c, v);
       tmem_wait_ld();
@@ -376,7 +396,7 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
         reinterpret_cast<uint4*>(s.u.b.Wp + (2 * c + 1) * kSlab64)[r] = pack8_bf16(sv + 8);
       }
     }
-    for (int c = 0; c < Dv / 16; ++c) {
+    for (int c = half; c < Dv / 16; c += 2) {
       float v[16];
       tmem_ld16(tm + lane_base + 128 + 16 * c, v);
       tmem_wait_ld();
@@ -408,12 +428,13 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
   if (!block_wait(&s.mma_bar, 0, limit, err)) return false;
   tc_fence_after_sync();
   {
-    const int r = tid;  // TMEM lane = feature row of Qc / Rc
-    const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
+    const int quad = warp & 3, half = warp >> 2;
+    const int r = 32 * quad + lane;  // TMEM lane = feature row of Qc / Rc
+    const uint32_t lane_base = static_cast<uint32_t>(32 * quad) << 16;
     const size_t tile = ws.tile(dir, bh, j);
     uint4* Qg = reinterpret_cast<uint4*>(ws.Qc + tile * (size_t)Dk * Dk);
     uint4* Rg = reinterpret_cast<uint4*>(ws.Rc + tile * (size_t)Dk * Dv);
-    for (int c = 0; c < Dk / 16; ++c) {
+    for (int c = half; c < Dk / 16; c += 2) {
       float v[16];
       tmem_ld16(tm + lane_base + 16 * c, v);
       tmem_wait_ld();
@@ -422,7 +443,7 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
         Qg[(2 * c + 1) * Dk + r] = pack8_bf16(v + 8);
       }
     }
-    for (int c = 0; c < Dv / 16; ++c) {
+    for (int c = half; c < Dv / 16; c += 2) {
       float v[16];
       tmem_ld16(tm + lane_base + 128 + 16 * c, v);
       tmem_wait_ld();
@@ -437,7 +458,7 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
   return true;
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kWideThreads, 2)
 gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const float* __restrict__ g, const float* __restrict__ beta, Workspace ws, int T,
                 int H, long long limit, unsigned* err) {
@@ -455,7 +476,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
   }
   {  // zero the feature slabs past Dk (rows of the M = 128 products)
     uint4* z = reinterpret_cast<uint4*>(s.K + (ws.Dk / 8) * kSlab64);
-    for (int i = tid; i < (16 - ws.Dk / 8) * kSlab64 / 16; i += kThreads) z[i] = make_uint4(0, 0, 0, 0);
+    for (int i = tid; i < (16 - ws.Dk / 8) * kSlab64 / 16; i += kWideThreads) z[i] = make_uint4(0, 0, 0, 0);
   }
   block_sync_async();
   if (blockIdx.z == 0)
@@ -507,68 +528,81 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
     const int jt = dir ? nC - 1 - c : c;
     const size_t tile = ws.tile(dir, bh, jt);
     uint8_t* st = stage0 + (c % kRecStages) * stage_bytes;
-    mbar_arrive_expect_tx(&hd.full[c % kRecStages], qbytes + rbytes + 16);
-    bulk_load(st, ws.Qc + tile * (size_t)Dk * Dk, qbytes, &hd.full[c % kRecStages]);
-    bulk_load(st + qbytes, ws.Rc + tile * (size_t)Dk * Dv + (size_t)slice * Dk * 16, rbytes,
-              &hd.full[c % kRecStages]);
-    bulk_load(st + qbytes + rbytes, ws.decay + 4 * tile, 16, &hd.full[c % kRecStages]);
+    uint64_t* bar = &hd.full[c % kRecStages];
+    mbar_arrive_expect_tx(bar, qbytes + rbytes + 16);
+    bulk_load(st, ws.Qc + tile * (size_t)Dk * Dk, qbytes, bar);
+    bulk_load(st + qbytes, ws.Rc + tile * (size_t)Dk * Dv + (size_t)slice * Dk * 16, rbytes, bar);
+    bulk_load(st + qbytes + rbytes, ws.decay + 4 * tile, 16, bar);
   };
-  int issued = 0;
+  int issued = min(kRecStages, nC);
   if (tid == 0)
-    for (; issued < kRecStages && issued < nC; ++issued) issue(issued);
-  issued = min(kRecStages, nC);
+    for (int c = 0; c < issued; ++c) issue(c);
 
+  // Descriptors: A = the chunk's Qc (K-major, Dk rows per slab), B = S (MN-major)
   const uint32_t id = idesc_bf16(128, 16, 0, 1);
+  const uint64_t bdesc0 = sdesc(smem_u32(Ssm), 128, 2048);
   const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
-  for (int c = 0; c < nC; ++c) {
+  uint4* Sg_base = reinterpret_cast<uint4*>(ws.S);
+  bool good = true;
+  int c = 0;
+  for (; c < nC; ++c) {
     const int jt = dir ? nC - 1 - c : c;
     const size_t tile = ws.tile(dir, bh, jt);
-    // publish S at the start of this chunk: MMA operand + workspace for stage C
+    const int st = c % kRecStages;
+    const uint8_t* Qst = stage0 + st * stage_bytes;
+    // S at the start of this chunk -> MMA operand and workspace (for stage C)
     if (r < Dk) {
       const uint4 lo = pack8_bf16(S), hi = pack8_bf16(S + 8);
       reinterpret_cast<uint4*>(Ssm)[r] = lo;
       reinterpret_cast<uint4*>(Ssm + 2048)[r] = hi;
-      uint4* Sg = reinterpret_cast<uint4*>(ws.S + tile * (size_t)Dk * Dv);
+      uint4* Sg = Sg_base + tile * (size_t)Dk * Dv / 8;
       Sg[(2 * slice) * Dk + r] = lo;
       Sg[(2 * slice + 1) * Dk + r] = hi;
     }
-    block_sync_async();
-    if (tid == 0 && c >= 1 && c - 1 + kRecStages < nC) issue(c - 1 + kRecStages);
-    if (c >= 1 && c - 1 + kRecStages < nC) issued = c - 1 + kRecStages + 1;
-    const int st = c % kRecStages;
-    if (!block_wait(&hd.full[st], (c / kRecStages) & 1, limit, err)) {
-      for (int p = c + 1; p < issued; ++p)
-        mbar_wait(&hd.full[p % kRecStages], (p / kRecStages) & 1, kDrainPolls);
-      return false;
-    }
-    const uint8_t* Qst = stage0 + st * stage_bytes;
+    bool ok = good;
+    if (tid == 0 && ok) ok = mbar_wait(&hd.full[st], (c / kRecStages) & 1, limit);
+    fence_proxy_async_smem();
+    tc_fence_before_sync();
+    if (!__syncthreads_and(ok)) break;  // operand and stage data visible to all
+    tc_fence_after_sync();
     if (tid == 0) {
-      tc_fence_after_sync();
-      for (int ks = 0; ks < Dk / 16; ++ks) {
-        const uint64_t a = sdesc(smem_u32(Qst) + ks * 2 * Dk * 16, Dk * 16, 128);
-        const uint64_t bd = sdesc(smem_u32(Ssm) + ks * 256, 128, 2048);
-        mma_bf16(tm, a, bd, id, ks > 0);
-      }
+      const uint64_t adesc0 = sdesc(smem_u32(Qst), Dk * 16, 128);
+      for (int ks = 0; ks < Dk / 16; ++ks)
+        mma_bf16(tm, adesc0 + (uint64_t)((ks * 2 * Dk * 16) >> 4), bdesc0 + (uint64_t)((ks * 256) >> 4),
+                 id, ks > 0);
       mma_commit(&hd.mma_bar);
+      if (c >= 1 && c - 1 + kRecStages < nC) issue(c - 1 + kRecStages);  // stage of chunk c-1
     }
-    if (!block_wait(&hd.mma_bar, c & 1, limit, err)) {
-      for (int p = c + 1; p < issued; ++p)
-        mbar_wait(&hd.full[p % kRecStages], (p / kRecStages) & 1, kDrainPolls);
-      return false;
+    if (c >= 1 && c - 1 + kRecStages < nC) issued = c - 1 + kRecStages + 1;
+    float R[16];
+    float a = 0.f;
+    if (r < Dk) {
+      const uint4* Rs = reinterpret_cast<const uint4*>(Qst + qbytes);
+      unpack8_bf16(Rs[2 * r], R);
+      unpack8_bf16(Rs[2 * r + 1], R + 8);
+      a = *reinterpret_cast<const float*>(Qst + qbytes + rbytes);
     }
+    good = mbar_wait(&hd.mma_bar, c & 1, limit);
+    if (!good) continue;  // the next barrier (or the final check) ends the walk
     tc_fence_after_sync();
     float D[16];
     tmem_ld16(tm + lane_base, D);
     tmem_wait_ld();
     if (r < Dk) {
-      float R[16];
-      const uint4* Rs = reinterpret_cast<const uint4*>(Qst + qbytes);
-      unpack8_bf16(Rs[2 * r], R);
-      unpack8_bf16(Rs[2 * r + 1], R + 8);
-      const float a = *reinterpret_cast<const float*>(Qst + qbytes + rbytes);
 #pragma unroll
       for (int e = 0; e < 16; ++e) S[e] = fmaf(a, S[e], R[e] - D[e]);
     }
+  }
+  const bool all_good = __syncthreads_and(good) && c == nC;
+  if (!all_good) {
+    if (tid == 0) atomicOr(err, kErrTimeout);
+    // drain: the last committed MMA and every load still in flight
+    const int last = (c == nC ? nC : c) - 1;
+    if (last >= 0) mbar_wait(&hd.mma_bar, last & 1, kDrainPolls);
+    for (int p = (c < nC ? c : nC); p < issued; ++p)
+      mbar_wait(&hd.full[p % kRecStages], (p / kRecStages) & 1, kDrainPolls);
+    __syncthreads();
+    return false;
   }
   if (dir == 0 && state_out && r < Dk) {
     float4* p = reinterpret_cast<float4*>(state_out + ((size_t)bh * Dk + r) * Dv + 16 * slice);
@@ -672,13 +706,13 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
     mbar_wait(&sm.ld_bar, 0, kDrainPolls);
     return false;
   }
-  if (tid < kC) {
-    sm.rnq[tid] = row_rnorm(sQ, tid, Dk);
-    sm.rnk[tid] = row_rnorm(sK, tid, Dk);
-  }
+  if (tid < kC) sm.rnq[tid] = row_rnorm(sQ, tid, Dk);
+  else if (tid < 2 * kC) sm.rnk[tid - kC] = row_rnorm(sK, tid - kC, Dk);
   uint32_t mma_phase = 0;
-  const int r = 16 * warp + (lane & 15);
-  const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
+  // warps w and w + 4 share TMEM lane quadrant w % 4 and split column blocks
+  const int quad = warp & 3, half = warp >> 2;
+  const int r = 16 * quad + (lane & 15);
+  const uint32_t lane_base = static_cast<uint32_t>(32 * quad) << 16;
   for (int dir = 0; dir < ndir; ++dir) {
     // D_U: direction 0 borrows D_O's columns (D_O is first written after D_U
     // is consumed); direction 1 needs its own, [192, 320) of a 512-column
@@ -706,7 +740,7 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
     ++mma_phase;
     tc_fence_after_sync();
     // U = U~ - W S  -> sW (MN-major B: [slab][64 tokens][8])
-    for (int c = 0; c < Dv / 16; ++c) {
+    for (int c = half; c < Dv / 16; c += 2) {
       float v[16];
       tmem_ld16(tmU + lane_base + 16 * c, v);
       tmem_wait_ld();
@@ -721,7 +755,7 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
       }
     }
     // P'_ri = (q_r . k_i) / |k_i| * e^{gam_r - gam_i} for i at or before r
-    for (int c = 0; c < 4; ++c) {
+    for (int c = half; c < 4; c += 2) {
       float v[16];
       tmem_ld16(tmP + lane_base + 16 * c, v);
       tmem_wait_ld();
@@ -740,7 +774,7 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
     // Qs = diag(e^gam) Q -> sK (K is dead once P is in TMEM)
     if (lane < 16) {
       const float eg = expf(sm.gam[r]);
-      for (int sl = 0; sl < Dk / 8; ++sl) {
+      for (int sl = half; sl < Dk / 8; sl += 2) {
         float x[8];
         unpack8_bf16(reinterpret_cast<const uint4*>(sQ + sl * kSlab64)[r], x);
 #pragma unroll
@@ -767,7 +801,7 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
   // O = diag(1/|q|) D_O -> out (rows of this chunk that exist)
   {
     const float rq = sm.rnq[r];
-    for (int c = 0; c < Dv / 16; ++c) {
+    for (int c = half; c < Dv / 16; c += 2) {
       float v[16];
       tmem_ld16(tmO + lane_base + 16 * c, v);
       tmem_wait_ld();
@@ -783,7 +817,7 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
   return true;
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kWideThreads, 2)
 gdn_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const float* __restrict__ g, __nv_bfloat16* __restrict__ out, Workspace ws, int T,
                   int H, int ndir, long long limit, unsigned* err) {
@@ -904,7 +938,7 @@ cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
 
   {
     ProfileScope ps(a.stream, kKernPrep);
-    gdn_prep_kernel<<<dim3(nC, NBH, ndir), kThreads, sizeof(PrepSmem), a.stream>>>(
+    gdn_prep_kernel<<<dim3(nC, NBH, ndir), kWideThreads, sizeof(PrepSmem), a.stream>>>(
         mk, mv, a.g, a.beta, ws, a.T, a.H, a.wait_limit, a.err);
   }
   e = cudaGetLastError();
@@ -918,7 +952,7 @@ cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
   if (e != cudaSuccess) return e;
   {
     ProfileScope ps(a.stream, kKernOutput);
-    gdn_output_kernel<<<dim3(nC, NBH), kThreads, OutLayout(a.Dk, a.Dv).total, a.stream>>>(
+    gdn_output_kernel<<<dim3(nC, NBH), kWideThreads, OutLayout(a.Dk, a.Dv).total, a.stream>>>(
         mq, mk, a.g, static_cast<__nv_bfloat16*>(a.out), ws, a.T, a.H, ndir, a.wait_limit, a.err);
   }
   e = cudaGetLastError();
