@@ -49,7 +49,6 @@ namespace {
 using namespace sm100;
 
 constexpr int kC = 64;            // tokens per chunk
-constexpr int kThreads = 128;     // stage B
 constexpr int kWideThreads = 256; // stages A and C: two warps per TMEM lane quadrant
 constexpr int kSlab64 = kC * 16;  // bytes of one 8-column slab of a 64-row tile
 constexpr int kRecStages = 4;
@@ -489,42 +488,72 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 }
 
 // ======================================================= stage B: recurrence
+// One CTA per (16 state columns, b*h, direction), Dk/16 warps; warp w owns
+// state rows [16w, 16w + 16).  Per chunk the product Qc S (Dk x Dk times
+// Dk x 16) is a dependent chain across chunks and is latency-bound: a
+// tcgen05 round trip (issue 7 MMAs, commit, mbarrier, TMEM load) costs
+// ~1.2k cycles per chunk here, so this stage uses warp-level
+// mma.sync.m16n8k16 (bf16 in, fp32 accumulate) with the fp32 state held in
+// the accumulator registers and the bf16 copy of S exchanged through a
+// double-buffered shared-memory operand: one barrier per chunk.
+// Dynamic layout: [head 128 B] [S operand x 2: [2 n-slabs][Dk][8] bf16]
+//                 [stages: Qc [Dk/8][Dk][8] | Rc slice [Dk][16] | decay 16 B]
 struct RecSmemHead {
   uint64_t full[kRecStages];
-  uint64_t mma_bar;
-  uint32_t tmem;
 };
-// dynamic layout: [head (128 B)] [S operand 4 KB] [stages: Qc | Rc slice | decay]
-// [2 KB tail pad: the M = 128 MMA reads up to 128 rows of Qc's last slab;
-//  rows past Dk are don't-care rows of D but must lie in shared memory]
 constexpr int kRecHeadBytes = 128;
-constexpr int kRecSBytes = 2 * 128 * 16;
+constexpr int kRecSBytes = 2 * 128 * 16;  // one S operand buffer at Dk = 128
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+// D += A B, m16n8k16, bf16 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
 
 __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_out,
                            const Workspace& ws, long long limit, unsigned* err) {
   RecSmemHead& hd = *reinterpret_cast<RecSmemHead*>(smem);
-  uint8_t* Ssm = smem + kRecHeadBytes;
-  uint8_t* stage0 = Ssm + kRecSBytes;
   const int Dk = ws.Dk, Dv = ws.Dv, nC = ws.nC;
+  uint8_t* Sop0 = smem + kRecHeadBytes;
+  const uint32_t nslab_bytes = (uint32_t)Dk * 16;  // one n-slab [Dk][8] bf16 of the operand
+  uint8_t* stage0 = Sop0 + 2 * kRecSBytes;
   const uint32_t qbytes = (uint32_t)Dk * Dk * 2, rbytes = (uint32_t)Dk * 32;
   const uint32_t stage_bytes = (qbytes + rbytes + 16 + 127) & ~127u;
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int slice = blockIdx.x, bh = blockIdx.y, dir = blockIdx.z;
-  const int r = tid;
-  const uint32_t tm = hd.tmem;
+  const int nks = Dk / 16;
+  // accumulator coordinates of this thread: rows rA, rA + 8; columns cA, cA + 1 (+ 8 nt)
+  const int rA = 16 * warp + (lane >> 2), cA = 2 * (lane & 3);
 
-  float S[16];
+  float S[2][4];  // [n-tile][c0..c3], fp32 state
 #pragma unroll
-  for (int e = 0; e < 16; ++e) S[e] = 0.f;
-  if (dir == 0 && state_in && r < Dk) {
-    const float4* p = reinterpret_cast<const float4*>(state_in + ((size_t)bh * Dk + r) * Dv + 16 * slice);
+  for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float4 v = p[q];
-      S[4 * q] = v.x; S[4 * q + 1] = v.y; S[4 * q + 2] = v.z; S[4 * q + 3] = v.w;
+    for (int i = 0; i < 4; ++i) S[nt][i] = 0.f;
+  if (dir == 0 && state_in) {
+    const float* base = state_in + (size_t)bh * Dk * Dv + 16 * slice;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const float2 lo = *reinterpret_cast<const float2*>(base + (size_t)rA * Dv + 8 * nt + cA);
+      const float2 hi = *reinterpret_cast<const float2*>(base + (size_t)(rA + 8) * Dv + 8 * nt + cA);
+      S[nt][0] = lo.x; S[nt][1] = lo.y; S[nt][2] = hi.x; S[nt][3] = hi.y;
     }
   }
-  auto issue = [&](int c) {  // thread 0: load chunk c (scan order) into its stage
+  auto issue = [&](int c) {  // one thread: load chunk c (scan order) into its stage
     const int jt = dir ? nC - 1 - c : c;
     const size_t tile = ws.tile(dir, bh, jt);
     uint8_t* st = stage0 + (c % kRecStages) * stage_bytes;
@@ -538,100 +567,100 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
   if (tid == 0)
     for (int c = 0; c < issued; ++c) issue(c);
 
-  // Descriptors: A = the chunk's Qc (K-major, Dk rows per slab), B = S (MN-major)
-  const uint32_t id = idesc_bf16(128, 16, 0, 1);
-  const uint64_t bdesc0 = sdesc(smem_u32(Ssm), 128, 2048);
-  const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
-  uint4* Sg_base = reinterpret_cast<uint4*>(ws.S);
-  bool good = true;
+  // S (bf16) of this thread's accumulator positions -> operand buffer `buf`
+  // ([n-slab][Dk rows][8]) and, for stage C, the workspace copy of the state
+  // at the start of chunk `jt` ([Dv/8][Dk][8]).
+  auto publish = [&](int buf, size_t tile) {
+    uint8_t* Sop = Sop0 + buf * kRecSBytes;
+    __nv_bfloat16* Sg = ws.S + tile * (size_t)Dk * Dv;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const uint32_t lo = pack_bf16x2(S[nt][0], S[nt][1]);
+      const uint32_t hi = pack_bf16x2(S[nt][2], S[nt][3]);
+      *reinterpret_cast<uint32_t*>(Sop + nt * nslab_bytes + rA * 16 + cA * 2) = lo;
+      *reinterpret_cast<uint32_t*>(Sop + nt * nslab_bytes + (rA + 8) * 16 + cA * 2) = hi;
+      const size_t slab = (size_t)(2 * slice + nt) * Dk;
+      *reinterpret_cast<uint32_t*>(Sg + (slab + rA) * 8 + cA) = lo;
+      *reinterpret_cast<uint32_t*>(Sg + (slab + rA + 8) * 8 + cA) = hi;
+    }
+  };
+  publish(0, ws.tile(dir, bh, dir ? nC - 1 : 0));
+
+  // ldmatrix row addresses (bytes in shared space) for this thread
+  const int mi = lane >> 3, mr = lane & 7;
+  // A: matrices (rows 0-7 | 8-15) x (k 0-7 | 8-15) of this warp's 16 rows
+  const uint32_t a_off = (uint32_t)((mi >> 1) * Dk * 16 + (16 * warp + (mi & 1) * 8 + mr) * 16);
+  // B (trans): matrices (k 0-7 | 8-15) x (n-slab 0 | 1)
+  const uint32_t b_off = (uint32_t)((mi >> 1) * nslab_bytes + ((mi & 1) * 8 + mr) * 16);
+  const uint32_t sop_u32 = smem_u32(Sop0), stage_u32 = smem_u32(stage0);
+
+  bool ok = true;
   int c = 0;
   for (; c < nC; ++c) {
-    const int jt = dir ? nC - 1 - c : c;
-    const size_t tile = ws.tile(dir, bh, jt);
     const int st = c % kRecStages;
-    const uint8_t* Qst = stage0 + st * stage_bytes;
-    // S at the start of this chunk -> MMA operand and workspace (for stage C)
-    if (r < Dk) {
-      const uint4 lo = pack8_bf16(S), hi = pack8_bf16(S + 8);
-      reinterpret_cast<uint4*>(Ssm)[r] = lo;
-      reinterpret_cast<uint4*>(Ssm + 2048)[r] = hi;
-      uint4* Sg = Sg_base + tile * (size_t)Dk * Dv / 8;
-      Sg[(2 * slice) * Dk + r] = lo;
-      Sg[(2 * slice + 1) * Dk + r] = hi;
-    }
-    bool ok = good;
-    if (tid == 0 && ok) ok = mbar_wait(&hd.full[st], (c / kRecStages) & 1, limit);
-    fence_proxy_async_smem();
-    tc_fence_before_sync();
-    if (!__syncthreads_and(ok)) break;  // operand and stage data visible to all
-    tc_fence_after_sync();
-    if (tid == 0) {
-      const uint64_t adesc0 = sdesc(smem_u32(Qst), Dk * 16, 128);
-      for (int ks = 0; ks < Dk / 16; ++ks)
-        mma_bf16(tm, adesc0 + (uint64_t)((ks * 2 * Dk * 16) >> 4), bdesc0 + (uint64_t)((ks * 256) >> 4),
-                 id, ks > 0);
-      mma_commit(&hd.mma_bar);
-      if (c >= 1 && c - 1 + kRecStages < nC) issue(c - 1 + kRecStages);  // stage of chunk c-1
-    }
+    if (tid == 0) ok = mbar_wait(&hd.full[st], (c / kRecStages) & 1, limit);
+    if (!__syncthreads_and(ok)) break;  // S operand written, stage data visible
+    if (tid == 32 % blockDim.x && c >= 1 && c - 1 + kRecStages < nC) issue(c - 1 + kRecStages);
     if (c >= 1 && c - 1 + kRecStages < nC) issued = c - 1 + kRecStages + 1;
-    float R[16];
-    float a = 0.f;
-    if (r < Dk) {
-      const uint4* Rs = reinterpret_cast<const uint4*>(Qst + qbytes);
-      unpack8_bf16(Rs[2 * r], R);
-      unpack8_bf16(Rs[2 * r + 1], R + 8);
-      a = *reinterpret_cast<const float*>(Qst + qbytes + rbytes);
-    }
-    good = mbar_wait(&hd.mma_bar, c & 1, limit);
-    if (!good) continue;  // the next barrier (or the final check) ends the walk
-    tc_fence_after_sync();
-    float D[16];
-    tmem_ld16(tm + lane_base, D);
-    tmem_wait_ld();
-    if (r < Dk) {
+    const uint32_t qa = stage_u32 + st * stage_bytes + a_off;
+    const uint32_t sb = sop_u32 + (c & 1) * kRecSBytes + b_off;
+    float acc[2][4];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) S[e] = fmaf(a, S[e], R[e] - D[e]);
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
+#pragma unroll 8
+    for (int ks = 0; ks < nks; ++ks) {
+      uint32_t af[4], bf[4];
+      ldmatrix_x4(qa + ks * 2 * Dk * 16, af);
+      ldmatrix_x4_trans(sb + ks * 256, bf);
+      mma_16816(acc[0], af, bf[0], bf[1]);
+      mma_16816(acc[1], af, bf[2], bf[3]);
     }
+    // S <- e^{gamma_C} S - Qc S + Rc
+    const uint8_t* stp = stage0 + st * stage_bytes;
+    const float a = *reinterpret_cast<const float*>(stp + qbytes + rbytes);
+    const __nv_bfloat16* R = reinterpret_cast<const __nv_bfloat16*>(stp + qbytes);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const __nv_bfloat162 r0 = *reinterpret_cast<const __nv_bfloat162*>(R + rA * 16 + 8 * nt + cA);
+      const __nv_bfloat162 r1 = *reinterpret_cast<const __nv_bfloat162*>(R + (rA + 8) * 16 + 8 * nt + cA);
+      S[nt][0] = fmaf(a, S[nt][0], __low2float(r0) - acc[nt][0]);
+      S[nt][1] = fmaf(a, S[nt][1], __high2float(r0) - acc[nt][1]);
+      S[nt][2] = fmaf(a, S[nt][2], __low2float(r1) - acc[nt][2]);
+      S[nt][3] = fmaf(a, S[nt][3], __high2float(r1) - acc[nt][3]);
+    }
+    if (c + 1 < nC) publish((c + 1) & 1, ws.tile(dir, bh, dir ? nC - 2 - c : c + 1));
   }
-  const bool all_good = __syncthreads_and(good) && c == nC;
-  if (!all_good) {
+  if (c < nC) {  // a bounded wait expired: drain every load still in flight
     if (tid == 0) atomicOr(err, kErrTimeout);
-    // drain: the last committed MMA and every load still in flight
-    const int last = (c == nC ? nC : c) - 1;
-    if (last >= 0) mbar_wait(&hd.mma_bar, last & 1, kDrainPolls);
-    for (int p = (c < nC ? c : nC); p < issued; ++p)
+    for (int p = c; p < issued; ++p)
       mbar_wait(&hd.full[p % kRecStages], (p / kRecStages) & 1, kDrainPolls);
     __syncthreads();
     return false;
   }
-  if (dir == 0 && state_out && r < Dk) {
-    float4* p = reinterpret_cast<float4*>(state_out + ((size_t)bh * Dk + r) * Dv + 16 * slice);
+  if (dir == 0 && state_out) {
+    float* base = state_out + (size_t)bh * Dk * Dv + 16 * slice;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) p[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
+    for (int nt = 0; nt < 2; ++nt) {
+      *reinterpret_cast<float2*>(base + (size_t)rA * Dv + 8 * nt + cA) = make_float2(S[nt][0], S[nt][1]);
+      *reinterpret_cast<float2*>(base + (size_t)(rA + 8) * Dv + 8 * nt + cA) = make_float2(S[nt][2], S[nt][3]);
+    }
   }
   return true;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(256, 1)
 gdn_recur_kernel(const float* state_in, float* state_out, Workspace ws, long long limit,
                  unsigned* err) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   RecSmemHead& hd = *reinterpret_cast<RecSmemHead*>(smem_raw);
-  const int tid = threadIdx.x;
-  if (tid == 0) {
+  if (threadIdx.x == 0) {
     for (int i = 0; i < kRecStages; ++i) mbar_init(&hd.full[i], 1);
-    mbar_init(&hd.mma_bar, 1);
     fence_mbar_init();
   }
-  if ((tid >> 5) == 0) {
-    tmem_alloc(&hd.tmem, 32);
-    tmem_relinquish();
-  }
-  block_sync_async();
-  recur_body(smem_raw, state_in, state_out, ws, limit, err);
-  tc_fence_before_sync();
   __syncthreads();
-  if ((tid >> 5) == 0) tmem_dealloc(hd.tmem, 32);
+  recur_body(smem_raw, state_in, state_out, ws, limit, err);
 }
 
 // ========================================================== stage C: output
@@ -879,7 +908,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 int recur_smem_bytes(int Dk) {
   const int stage = ((Dk * Dk * 2 + Dk * 32 + 16) + 127) & ~127;
-  return kRecHeadBytes + kRecSBytes + kRecStages * stage + 2048;
+  return kRecHeadBytes + 2 * kRecSBytes + kRecStages * stage;
 }
 
 // Opt the kernels into their dynamic shared memory, once per device.
@@ -945,7 +974,7 @@ cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
   if (e != cudaSuccess) return e;
   {
     ProfileScope ps(a.stream, kKernRecur);
-    gdn_recur_kernel<<<dim3(a.Dv / 16, NBH, ndir), kThreads, recur_smem_bytes(a.Dk), a.stream>>>(
+    gdn_recur_kernel<<<dim3(a.Dv / 16, NBH, ndir), 32 * (a.Dk / 16), recur_smem_bytes(a.Dk), a.stream>>>(
         a.state_in, a.state_out, ws, a.wait_limit, a.err);
   }
   e = cudaGetLastError();
