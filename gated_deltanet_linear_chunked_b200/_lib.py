@@ -18,6 +18,7 @@ GDN_ERR_UNSUPPORTED = 2
 GDN_ERR_ALIAS = 3
 GDN_ERR_CUDA = 4
 GDN_ERR_TIMEOUT = 5
+GDN_ERR_SCRATCH_LIMIT = 6
 
 GDN_F32 = 0
 GDN_BF16 = 1
@@ -28,6 +29,7 @@ _SCAN_ARGS = [_vp, _vp, _vp, _fp, _fp, _fp, _fp, _vp] + [_i] * 5 + [_i, _i, _vp]
 SIGNATURES = {
     "gdn_chunk_fwd": (ctypes.c_int, _SCAN_ARGS),
     "gdn_chunk_bidir": (ctypes.c_int, _SCAN_ARGS),
+    "gdn_chunk_fwd_noalloc": (ctypes.c_int, _SCAN_ARGS),
     "gdn_state_reset": (ctypes.c_int, [_fp, _i, _i, _i, _i, _vp]),
     "gdn_device_error": (ctypes.c_int, [_vp]),
     "gdn_set_wait_limit": (ctypes.c_longlong, [_ll]),

@@ -192,6 +192,9 @@ gdn_status scan(const void* q, const void* k, const void* v, const float* g,
 
 void count_launches(unsigned n) { g_launches.fetch_add(n); }
 
+cudaError_t current_error_word(unsigned int** out) { return error_word(out); }
+long long current_wait_limit() { return g_wait_limit.load(); }
+
 // ------------------------------------------------------------- profiling
 namespace {
 struct Profile {
@@ -284,6 +287,7 @@ const char* gdn_status_string(gdn_status status) {
     case GDN_ERR_ALIAS: return "GDN_ERR_ALIAS";
     case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
     case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+    case GDN_ERR_SCRATCH_LIMIT: return "GDN_ERR_SCRATCH_LIMIT";
   }
   return "GDN_ERR_UNKNOWN";
 }

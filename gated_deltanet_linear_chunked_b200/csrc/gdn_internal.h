@@ -47,6 +47,11 @@ class ProfileScope {
   int slot_;
 };
 
+// Device address of the error word on the current device, and the poll
+// limit handed to bounded waits.
+cudaError_t current_error_word(unsigned int** out);
+long long current_wait_limit();
+
 // Adds n to the process-wide count of kernels the library has enqueued.
 void count_launches(unsigned n);
 

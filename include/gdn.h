@@ -46,6 +46,8 @@
  *   GDN_ERR_TIMEOUT      a kernel's bounded wait expired (reported by
  *                        gdn_device_error, or by the calls themselves when
  *                        the environment sets GDN_DEBUG_SYNC=1)
+ *   GDN_ERR_SCRATCH_LIMIT  (gdn_chunk_fwd_noalloc only) the problem needs more
+ *                        scratch than its fixed device array holds
  */
 #ifndef GDN_H_
 #define GDN_H_
@@ -66,7 +68,8 @@ typedef enum {
   GDN_ERR_UNSUPPORTED = 2,
   GDN_ERR_ALIAS = 3,
   GDN_ERR_CUDA = 4,
-  GDN_ERR_TIMEOUT = 5
+  GDN_ERR_TIMEOUT = 5,
+  GDN_ERR_SCRATCH_LIMIT = 6
 } gdn_status;
 
 typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
@@ -101,6 +104,41 @@ GDN_API gdn_status gdn_chunk_bidir(const void* q, const void* k, const void* v,
                            const float* state_in, float* state_out, void* out,
                            int B, int T, int H, int Dk, int Dv,
                            gdn_dtype dtype, int chunk, void* stream);
+
+/*
+ * gdn_chunk_fwd for callers that cannot allocate device memory (no
+ * counterpart on the pages).  Some callers cannot let a library allocate: a
+ * streaming server that has already handed all remaining HBM to its caches
+ * (an allocation in the middle of a stream can fail or stall on the memory
+ * pool), or a process whose CUDA memory-pool API is unavailable or turned
+ * off.  This entry point runs the same bf16 tensor-core kernels as
+ * gdn_chunk_fwd but takes their scratch from one fixed array of
+ * GDN_NOALLOC_SCRATCH_BYTES (96 MiB) that the library declares in device
+ * memory; every GPU that loads the library holds that array until the process
+ * exits.  It calls no cudaMalloc, cudaMallocAsync, cudaFree or other
+ * allocating routine.
+ *
+ * Arguments and layouts are those of gdn_chunk_fwd, with dtype GDN_BF16
+ * only (other dtypes: GDN_ERR_UNSUPPORTED).  A problem whose scratch exceeds
+ * the array returns GDN_ERR_SCRATCH_LIMIT and launches nothing.  The scratch
+ * is about 104 KB per 64-token chunk of one head at Dk = Dv = 112, so about
+ * 960 chunk-heads (B * H * ceil(T / 64)) fit: the 2640-token x 20-head
+ * streaming chunk (840) does, two of them in one call do not.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, once per device, with that device current); make
+ * that first call before any stream capture.  All calls share the one array
+ * and it keeps the last call's contents (every scratch byte a call reads was
+ * written earlier in the same call, so nothing needs clearing); calls whose
+ * work overlaps on the GPU -- two streams, or two host threads -- race on it,
+ * so order them on one stream.
+ */
+#define GDN_NOALLOC_SCRATCH_BYTES (96ull << 20)
+GDN_API gdn_status gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
+                                         const float* g, const float* beta,
+                                         const float* state_in, float* state_out,
+                                         void* out, int B, int T, int H, int Dk, int Dv,
+                                         gdn_dtype dtype, int chunk, void* stream);
 
 /*
  * Zero a state [B, H, Dk, Dv] (streaming restart: the state is the only thing
