@@ -38,6 +38,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "gdn_internal.h"
@@ -664,22 +665,24 @@ gdn_recur_kernel(const float* state_in, float* state_out, Workspace ws, long lon
 }
 
 // ========================================================== stage C: output
-// Dynamic shared-memory layout (offsets from Dk, Dv, 128 B aligned):
+// Persistent: one CTA per SM walks tiles t = blockIdx.x, + gridDim.x, ...
+// with two input sets in shared memory, so the next tile's TMA / bulk loads
+// land while the current tile computes.  Per set (offsets from Dk, Dv):
 //   Q   [Dk/8][64][8]  raw q tile (TMA)
 //   K   [Dk/8][64][8]  raw k tile (TMA); after P = Q K^T it holds Qs = diag(e^g) Q
-//   W   [max(Dk,Dv)/8][64][8]  W of the current direction; after W S it holds
-//                  U [Dv/8][64][8] (B operand)
+//   W   [max(Dk,Dv)/8][64][8]  W of the current direction; after W S it holds U
 //   Ut  [Dv/8][64][8]  U~ of the current direction
 //   S   [Dv/8][Dk][8]  state at the chunk's start (MN-major B operand)
-//   P   [8][64][8]     masked, gated Q K^T (K-major A operand)
-// ~90 KB at Dk = Dv = 112: two CTAs per SM.
+// then P [8][64][8] (masked, gated Q K^T, K-major A) and the scalar block.
 struct OutSmall {
-  float g[64], gam[64], rnq[64], rnk[64];
-  uint64_t tma_bar, ld_bar, mma_bar;
+  float g[2][64];
+  float gam[64], rnq[64], rnk[64], arow[64];
+  float bcol[8][64];
+  uint64_t tma_bar[2], ld_bar[2], mma_bar;
   uint32_t tmem;
 };
 struct OutLayout {
-  uint32_t q, k, w, ut, s, p, small, total;
+  uint32_t q, k, w, ut, s, set_bytes, p, small, total;
   __host__ __device__ OutLayout(int Dk, int Dv) {
     auto al = [](uint32_t x) { return (x + 127u) & ~127u; };
     q = 0;
@@ -687,166 +690,239 @@ struct OutLayout {
     w = al(k + 64u * Dk * 2);
     ut = al(w + 64u * (Dk > Dv ? Dk : Dv) * 2);  // W, later U: room for either
     s = al(ut + 64u * Dv * 2);
-    p = al(s + (uint32_t)Dk * Dv * 2);
+    set_bytes = al(s + (uint32_t)Dk * Dv * 2);
+    p = 2 * set_bytes;
     small = al(p + 8u * kSlab64);
     total = al(small + (uint32_t)sizeof(OutSmall));
   }
 };
+
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                             const float* __restrict__ g, __nv_bfloat16* __restrict__ out,
                             const Workspace& ws, int T, int H, int ndir, long long limit,
                             unsigned* err) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int j = blockIdx.x, bh = blockIdx.y;
-  const int b = bh / H, h = bh - b * H;
-  const int Dk = ws.Dk, Dv = ws.Dv;
+  const int Dk = ws.Dk, Dv = ws.Dv, nC = ws.nC;
+  const int ntiles = nC * ws.NBH;
   const OutLayout L(Dk, Dv);
-  uint8_t* sQ = smem + L.q;
-  uint8_t* sK = smem + L.k;   // then Qs
-  uint8_t* sW = smem + L.w;   // then U
-  uint8_t* sUt = smem + L.ut;
-  uint8_t* sS = smem + L.s;
-  uint8_t* sP = smem + L.p;
   OutSmall& sm = *reinterpret_cast<OutSmall*>(smem + L.small);
-  const int t0 = j * kC;
-  const int nvalid = min(kC, T - t0);
+  uint8_t* sP = smem + L.p;
   const uint32_t tm = sm.tmem;
-  // TMEM: P = Q K^T [0,64); D_O [64,192); D_U see below
   const uint32_t tmP = tm, tmO = tm + 64;
   const uint32_t wbytes = kC * Dk * 2, ubytes = kC * Dv * 2, sbytes = Dk * Dv * 2;
-  auto issue_dir = [&](int dir) {
-    const size_t tile = ws.tile(dir, bh, j);
-    mbar_arrive_expect_tx(&sm.ld_bar, wbytes + ubytes + sbytes);
-    bulk_load(sW, ws.W + tile * kC * Dk, wbytes, &sm.ld_bar);
-    bulk_load(sUt, ws.Ut + tile * kC * Dv, ubytes, &sm.ld_bar);
-    bulk_load(sS, ws.S + tile * (size_t)Dk * Dv, sbytes, &sm.ld_bar);
-  };
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&sm.tma_bar, 2 * (Dk / 8) * kSlab64);
-    for (int sl = 0; sl < Dk / 8; ++sl) {
-      tma_load_4d(sQ + sl * kSlab64, tm_q, &sm.tma_bar, 8 * sl, h, t0, b);
-      tma_load_4d(sK + sl * kSlab64, tm_k, &sm.tma_bar, 8 * sl, h, t0, b);
-    }
-    issue_dir(0);
-  }
-  if (tid < kC) sm.g[tid] = (tid < nvalid) ? __ldg(g + ((size_t)b * T + t0 + tid) * H + h) : 0.f;
-  if (!block_wait(&sm.tma_bar, 0, limit, err)) {
-    mbar_wait(&sm.ld_bar, 0, kDrainPolls);
-    return false;
-  }
-  if (tid < kC) sm.rnq[tid] = row_rnorm(sQ, tid, Dk);
-  else if (tid < 2 * kC) sm.rnk[tid - kC] = row_rnorm(sK, tid - kC, Dk);
-  uint32_t mma_phase = 0;
   // warps w and w + 4 share TMEM lane quadrant w % 4 and split column blocks
   const int quad = warp & 3, half = warp >> 2;
   const int r = 16 * quad + (lane & 15);
   const uint32_t lane_base = static_cast<uint32_t>(32 * quad) << 16;
-  for (int dir = 0; dir < ndir; ++dir) {
-    // D_U: direction 0 borrows D_O's columns (D_O is first written after D_U
-    // is consumed); direction 1 needs its own, [192, 320) of a 512-column
-    // allocation, because D_O then holds direction 0's sum.
-    const uint32_t tmU = tm + (dir == 0 ? 64u : 192u);
-    __syncthreads();
-    if (warp == 0) warp_gamma(sm.g, sm.gam, dir);
-    if (!block_wait(&sm.ld_bar, dir & 1, limit, err)) return false;
+
+  auto issue_dir = [&](int set, int tile_t, int dir) {  // thread 0
+    uint8_t* base = smem + set * L.set_bytes;
+    const int bh = tile_t / nC, j = tile_t - bh * nC;
+    const size_t tile = ws.tile(dir, bh, j);
+    mbar_arrive_expect_tx(&sm.ld_bar[set], wbytes + ubytes + sbytes);
+    bulk_load(base + L.w, ws.W + tile * kC * Dk, wbytes, &sm.ld_bar[set]);
+    bulk_load(base + L.ut, ws.Ut + tile * kC * Dv, ubytes, &sm.ld_bar[set]);
+    bulk_load(base + L.s, ws.S + tile * (size_t)Dk * Dv, sbytes, &sm.ld_bar[set]);
+  };
+  // all threads: start loading tile `tile_t` into `set`
+  auto issue_tile = [&](int set, int tile_t) {
+    const int bh = tile_t / nC, j = tile_t - bh * nC;
+    const int b = bh / H, h = bh - b * H, t0 = j * kC;
     if (tid == 0) {
-      tc_fence_after_sync();
-      if (dir == 0) {  // P = Q K^T, shared by both directions
-        const uint32_t idP = idesc_bf16(64, 64, 0, 0);
-        for (int ks = 0; ks < Dk / 16; ++ks)
-          mma_bf16(tmP, sdesc(smem_u32(sQ) + ks * 2 * kSlab64, kSlab64, 128),
-                   sdesc(smem_u32(sK) + ks * 2 * kSlab64, kSlab64, 128), idP, ks > 0);
+      uint8_t* base = smem + set * L.set_bytes;
+      mbar_arrive_expect_tx(&sm.tma_bar[set], 2 * (Dk / 8) * kSlab64);
+      for (int sl = 0; sl < Dk / 8; ++sl) {
+        tma_load_4d(base + L.q + sl * kSlab64, tm_q, &sm.tma_bar[set], 8 * sl, h, t0, b);
+        tma_load_4d(base + L.k + sl * kSlab64, tm_k, &sm.tma_bar[set], 8 * sl, h, t0, b);
       }
-      // D_U = W S  (M = 64, N = Dv, K = Dk); S read MN-major (N = value column)
-      const uint32_t idU = idesc_bf16(64, Dv, 0, 1);
-      for (int ks = 0; ks < Dk / 16; ++ks)
-        mma_bf16(tmU, sdesc(smem_u32(sW) + ks * 2 * kSlab64, kSlab64, 128),
-                 sdesc(smem_u32(sS) + ks * 256, 128, Dk * 16), idU, ks > 0);
-      mma_commit(&sm.mma_bar);
+      issue_dir(set, tile_t, 0);
     }
-    if (!block_wait(&sm.mma_bar, mma_phase & 1, limit, err)) return false;
-    ++mma_phase;
-    tc_fence_after_sync();
-    // U = U~ - W S  -> sW (MN-major B: [slab][64 tokens][8])
-    for (int c = half; c < Dv / 16; c += 2) {
-      float v[16];
-      tmem_ld16(tmU + lane_base + 16 * c, v);
-      tmem_wait_ld();
-      if (lane < 16) {
-        float ut[16];
-        unpack8_bf16(reinterpret_cast<const uint4*>(sUt + (2 * c) * kSlab64)[r], ut);
-        unpack8_bf16(reinterpret_cast<const uint4*>(sUt + (2 * c + 1) * kSlab64)[r], ut + 8);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) ut[e] -= v[e];
-        reinterpret_cast<uint4*>(sW + (2 * c) * kSlab64)[r] = pack8_bf16(ut);
-        reinterpret_cast<uint4*>(sW + (2 * c + 1) * kSlab64)[r] = pack8_bf16(ut + 8);
+    if (tid < kC) {
+      if (tid < T - t0) cp_async4(&sm.g[set][tid], g + ((size_t)b * T + t0 + tid) * H + h);
+      else sm.g[set][tid] = 0.f;
+      cp_async_commit();
+    }
+  };
+
+  int k = 0;
+  if (blockIdx.x < ntiles) issue_tile(0, blockIdx.x);
+  if (blockIdx.x + gridDim.x < ntiles) issue_tile(1, blockIdx.x + gridDim.x);
+  // mbarrier phase parities: bit `set` of tma_ph / ld_ph
+  uint32_t tma_ph = 0, ld_ph = 0, mma_ph = 0;
+  for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++k) {
+    const int set = k & 1;
+    const bool next_issued = t + gridDim.x < ntiles;
+    // on a failed wait: drain the other set's loads (the caller drained its own)
+    auto drain_other = [&]() {
+      if (next_issued) {
+        mbar_wait(&sm.tma_bar[set ^ 1], (tma_ph >> (set ^ 1)) & 1, kDrainPolls);
+        mbar_wait(&sm.ld_bar[set ^ 1], (ld_ph >> (set ^ 1)) & 1, kDrainPolls);
       }
+    };
+    uint8_t* base = smem + set * L.set_bytes;
+    uint8_t* sQ = base + L.q;
+    uint8_t* sK = base + L.k;   // then Qs
+    uint8_t* sW = base + L.w;   // then U
+    uint8_t* sUt = base + L.ut;
+    uint8_t* sS = base + L.s;
+    const int bh = t / nC, j = t - bh * nC;
+    const int b = bh / H, h = bh - b * H, t0 = j * kC;
+    const int nvalid = min(kC, T - t0);
+
+    if (tid < kC) {
+      if (next_issued) cp_async_wait<1>();
+      else cp_async_wait<0>();
     }
-    // P'_ri = (q_r . k_i) / |k_i| * e^{gam_r - gam_i} for i at or before r
-    for (int c = half; c < 4; c += 2) {
-      float v[16];
-      tmem_ld16(tmP + lane_base + 16 * c, v);
-      tmem_wait_ld();
-      if (lane < 16) {
-        const float g2r = sm.gam[r] * kLog2e;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int i = 16 * c + e;
-          const bool incl = dir ? (i >= r) : (i <= r);
-          v[e] = incl ? v[e] * sm.rnk[i] * exp2f(g2r - sm.gam[i] * kLog2e) : 0.f;
+    if (!block_wait(&sm.tma_bar[set], (tma_ph >> set) & 1, limit, err)) {
+      mbar_wait(&sm.ld_bar[set], (ld_ph >> set) & 1, kDrainPolls);
+      drain_other();
+      return false;
+    }
+    tma_ph ^= 1u << set;
+    if (tid < kC) sm.rnq[tid] = row_rnorm(sQ, tid, Dk);
+    else if (tid < 2 * kC) sm.rnk[tid - kC] = row_rnorm(sK, tid - kC, Dk);
+    for (int dir = 0; dir < ndir; ++dir) {
+      // D_U: direction 0 borrows D_O's columns (D_O is first written after
+      // D_U is consumed); direction 1 needs its own, [192, 320) of a
+      // 512-column allocation, because D_O then holds direction 0's sum.
+      const uint32_t tmU = tm + (dir == 0 ? 64u : 192u);
+      __syncthreads();
+      if (warp == 0) warp_gamma(sm.g[set], sm.gam, dir);
+      __syncthreads();
+      // Gate factors split at m_b = gam at the first scan position of each
+      // 8-row block (as in stage A): P'_ri = arow_r P_ri bcol[b(r)][i].
+      for (int e = tid; e < 8 * 64; e += kWideThreads) {
+        const int blk = e >> 6, i = e & 63;
+        const int qpos = dir ? 63 - i : i;
+        const float mb = sm.gam[dir ? 63 - 8 * blk : 8 * blk];
+        sm.bcol[blk][i] = (qpos < 8 * blk + 8) ? sm.rnk[i] * exp2f((mb - sm.gam[i]) * kLog2e) : 0.f;
+      }
+      if (tid < 64) {
+        const int p = dir ? 63 - tid : tid;
+        const float mb = sm.gam[dir ? 63 - 8 * (p >> 3) : 8 * (p >> 3)];
+        sm.arow[tid] = exp2f((sm.gam[tid] - mb) * kLog2e);
+      }
+      if (!block_wait(&sm.ld_bar[set], (ld_ph >> set) & 1, limit, err)) {
+        drain_other();
+        return false;
+      }
+      ld_ph ^= 1u << set;
+      if (tid == 0) {
+        tc_fence_after_sync();
+        if (dir == 0) {  // P = Q K^T, shared by both directions
+          const uint32_t idP = idesc_bf16(64, 64, 0, 0);
+          for (int ks = 0; ks < Dk / 16; ++ks)
+            mma_bf16(tmP, sdesc(smem_u32(sQ) + ks * 2 * kSlab64, kSlab64, 128),
+                     sdesc(smem_u32(sK) + ks * 2 * kSlab64, kSlab64, 128), idP, ks > 0);
         }
-        reinterpret_cast<uint4*>(sP + (2 * c) * kSlab64)[r] = pack8_bf16(v);
-        reinterpret_cast<uint4*>(sP + (2 * c + 1) * kSlab64)[r] = pack8_bf16(v + 8);
+        // D_U = W S  (M = 64, N = Dv, K = Dk); S read MN-major (N = value column)
+        const uint32_t idU = idesc_bf16(64, Dv, 0, 1);
+        for (int ks = 0; ks < Dk / 16; ++ks)
+          mma_bf16(tmU, sdesc(smem_u32(sW) + ks * 2 * kSlab64, kSlab64, 128),
+                   sdesc(smem_u32(sS) + ks * 256, 128, Dk * 16), idU, ks > 0);
+        mma_commit(&sm.mma_bar);
       }
-    }
-    // Qs = diag(e^gam) Q -> sK (K is dead once P is in TMEM)
-    if (lane < 16) {
-      const float eg = expf(sm.gam[r]);
-      for (int sl = half; sl < Dk / 8; sl += 2) {
-        float x[8];
-        unpack8_bf16(reinterpret_cast<const uint4*>(sQ + sl * kSlab64)[r], x);
+      if (!block_wait(&sm.mma_bar, mma_ph, limit, err)) {
+        drain_other();
+        return false;
+      }
+      mma_ph ^= 1;
+      tc_fence_after_sync();
+      // U = U~ - W S  -> sW (MN-major B: [slab][64 tokens][8])
+      for (int c = half; c < Dv / 16; c += 2) {
+        float v[16];
+        tmem_ld16(tmU + lane_base + 16 * c, v);
+        tmem_wait_ld();
+        if (lane < 16) {
+          float ut[16];
+          unpack8_bf16(reinterpret_cast<const uint4*>(sUt + (2 * c) * kSlab64)[r], ut);
+          unpack8_bf16(reinterpret_cast<const uint4*>(sUt + (2 * c + 1) * kSlab64)[r], ut + 8);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] *= eg;
-        reinterpret_cast<uint4*>(sK + sl * kSlab64)[r] = pack8_bf16(x);
+          for (int e = 0; e < 16; ++e) ut[e] -= v[e];
+          reinterpret_cast<uint4*>(sW + (2 * c) * kSlab64)[r] = pack8_bf16(ut);
+          reinterpret_cast<uint4*>(sW + (2 * c + 1) * kSlab64)[r] = pack8_bf16(ut + 8);
+        }
       }
-    }
-    block_sync_async();
-    if (tid == 0) {
-      const uint32_t idO = idesc_bf16(64, Dv, 0, 1);
-      for (int ks = 0; ks < Dk / 16; ++ks)
-        mma_bf16(tmO, sdesc(smem_u32(sK) + ks * 2 * kSlab64, kSlab64, 128),
-                 sdesc(smem_u32(sS) + ks * 256, 128, Dk * 16), idO, (dir > 0) || (ks > 0));
-      for (int ks = 0; ks < kC / 16; ++ks)
-        mma_bf16(tmO, sdesc(smem_u32(sP) + ks * 2 * kSlab64, kSlab64, 128),
-                 sdesc(smem_u32(sW) + ks * 256, 128, kSlab64), idO, 1);
-      mma_commit(&sm.mma_bar);
-    }
-    if (!block_wait(&sm.mma_bar, mma_phase & 1, limit, err)) return false;
-    ++mma_phase;
-    if (dir + 1 < ndir && tid == 0) issue_dir(dir + 1);
-  }
-  tc_fence_after_sync();
-  // O = diag(1/|q|) D_O -> out (rows of this chunk that exist)
-  {
-    const float rq = sm.rnq[r];
-    for (int c = half; c < Dv / 16; c += 2) {
-      float v[16];
-      tmem_ld16(tmO + lane_base + 16 * c, v);
-      tmem_wait_ld();
-      if (lane < 16 && r < nvalid) {
+      // P'_ri = (q_r . k_i) / |k_i| * e^{gam_r - gam_i} for i at or before r
+      for (int c = half; c < 4; c += 2) {
+        float v[16];
+        tmem_ld16(tmP + lane_base + 16 * c, v);
+        tmem_wait_ld();
+        if (lane < 16) {
+          const float ar = sm.arow[r];
+          const float* bc = sm.bcol[(dir ? 63 - r : r) >> 3];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) v[e] *= rq;
-        uint4* o = reinterpret_cast<uint4*>(out + (((size_t)b * T + t0 + r) * H + h) * Dv + 16 * c);
-        o[0] = pack8_bf16(v);
-        o[1] = pack8_bf16(v + 8);
+          for (int e = 0; e < 16; ++e) {
+            const int i = 16 * c + e;
+            const bool incl = dir ? (i >= r) : (i <= r);
+            v[e] = incl ? ar * v[e] * bc[i] : 0.f;
+          }
+          reinterpret_cast<uint4*>(sP + (2 * c) * kSlab64)[r] = pack8_bf16(v);
+          reinterpret_cast<uint4*>(sP + (2 * c + 1) * kSlab64)[r] = pack8_bf16(v + 8);
+        }
+      }
+      // Qs = diag(e^gam) Q -> sK (K is dead once P is in TMEM)
+      if (lane < 16) {
+        const float eg = expf(sm.gam[r]);
+        for (int sl = half; sl < Dk / 8; sl += 2) {
+          float x[8];
+          unpack8_bf16(reinterpret_cast<const uint4*>(sQ + sl * kSlab64)[r], x);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] *= eg;
+          reinterpret_cast<uint4*>(sK + sl * kSlab64)[r] = pack8_bf16(x);
+        }
+      }
+      block_sync_async();
+      if (tid == 0) {
+        const uint32_t idO = idesc_bf16(64, Dv, 0, 1);
+        for (int ks = 0; ks < Dk / 16; ++ks)
+          mma_bf16(tmO, sdesc(smem_u32(sK) + ks * 2 * kSlab64, kSlab64, 128),
+                   sdesc(smem_u32(sS) + ks * 256, 128, Dk * 16), idO, (dir > 0) || (ks > 0));
+        for (int ks = 0; ks < kC / 16; ++ks)
+          mma_bf16(tmO, sdesc(smem_u32(sP) + ks * 2 * kSlab64, kSlab64, 128),
+                   sdesc(smem_u32(sW) + ks * 256, 128, kSlab64), idO, 1);
+        mma_commit(&sm.mma_bar);
+      }
+      if (!block_wait(&sm.mma_bar, mma_ph, limit, err)) {
+        drain_other();
+        return false;
+      }
+      mma_ph ^= 1;
+      if (dir + 1 < ndir && tid == 0) issue_dir(set, t, dir + 1);
+    }
+    tc_fence_after_sync();
+    // O = diag(1/|q|) D_O -> out (rows of this chunk that exist)
+    {
+      const float rq = sm.rnq[r];
+      for (int c = half; c < Dv / 16; c += 2) {
+        float v[16];
+        tmem_ld16(tmO + lane_base + 16 * c, v);
+        tmem_wait_ld();
+        if (lane < 16 && r < nvalid) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[e] *= rq;
+          uint4* o = reinterpret_cast<uint4*>(out + (((size_t)b * T + t0 + r) * H + h) * Dv + 16 * c);
+          o[0] = pack8_bf16(v);
+          o[1] = pack8_bf16(v + 8);
+        }
       }
     }
+    tc_fence_before_sync();
+    __syncthreads();  // this set's buffers and the TMEM accumulators are free
+    tc_fence_after_sync();
+    if (t + 2 * gridDim.x < ntiles) issue_tile(set, t + 2 * gridDim.x);
   }
   return true;
 }
 
-__global__ void __launch_bounds__(kWideThreads, 2)
+__global__ void __launch_bounds__(kWideThreads, 1)
 gdn_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const float* __restrict__ g, __nv_bfloat16* __restrict__ out, Workspace ws, int T,
                   int H, int ndir, long long limit, unsigned* err) {
@@ -856,8 +932,10 @@ gdn_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const int tid = threadIdx.x;
   const uint32_t ncols = ndir > 1 ? 512u : 256u;
   if (tid == 0) {
-    mbar_init(&sm.tma_bar, 1);
-    mbar_init(&sm.ld_bar, 1);
+    mbar_init(&sm.tma_bar[0], 1);
+    mbar_init(&sm.tma_bar[1], 1);
+    mbar_init(&sm.ld_bar[0], 1);
+    mbar_init(&sm.ld_bar[1], 1);
     mbar_init(&sm.mma_bar, 1);
     fence_mbar_init();
   }
@@ -905,6 +983,20 @@ bool make_map(CUtensorMap* m, const void* base, int B, int T, int H, int D) {
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Streaming multiprocessors of the current device (persistent grids).
+int num_sms() {
+  constexpr int kMaxDev = 64;
+  static int cached[kMaxDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
 
 int recur_smem_bytes(int Dk) {
   const int stage = ((Dk * Dk * 2 + Dk * 32 + 16) + 127) & ~127;
@@ -981,7 +1073,8 @@ cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
   if (e != cudaSuccess) return e;
   {
     ProfileScope ps(a.stream, kKernOutput);
-    gdn_output_kernel<<<dim3(nC, NBH), kWideThreads, OutLayout(a.Dk, a.Dv).total, a.stream>>>(
+    gdn_output_kernel<<<dim3(std::min(nC * NBH, num_sms())), kWideThreads,
+                        OutLayout(a.Dk, a.Dv).total, a.stream>>>(
         mq, mk, a.g, static_cast<__nv_bfloat16*>(a.out), ws, a.T, a.H, ndir, a.wait_limit, a.err);
   }
   e = cudaGetLastError();
