@@ -50,7 +50,8 @@ namespace {
 using namespace sm100;
 
 constexpr int kC = 64;            // tokens per chunk
-constexpr int kWideThreads = 256; // stages A and C: two warps per TMEM lane quadrant
+constexpr int kWideThreads = 256; // stage A: two warps per TMEM lane quadrant
+constexpr int kOutThreads = 512;  // stage C: four warps per TMEM lane quadrant
 constexpr int kSlab64 = kC * 16;  // bytes of one 8-column slab of a 64-row tile
 constexpr int kRecStages = 4;
 constexpr long long kDrainPolls = 1LL << 40;  // drains are bounded by the 2 s timer
@@ -717,8 +718,9 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
   const uint32_t tm = sm.tmem;
   const uint32_t tmP = tm, tmO = tm + 64;
   const uint32_t wbytes = kC * Dk * 2, ubytes = kC * Dv * 2, sbytes = Dk * Dv * 2;
-  // warps w and w + 4 share TMEM lane quadrant w % 4 and split column blocks
-  const int quad = warp & 3, half = warp >> 2;
+  // warps w, w + 4, w + 8, w + 12 share TMEM lane quadrant w % 4 and split
+  // the column blocks four ways
+  const int quad = warp & 3, part = warp >> 2;
   const int r = 16 * quad + (lane & 15);
   const uint32_t lane_base = static_cast<uint32_t>(32 * quad) << 16;
 
@@ -798,7 +800,7 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
       __syncthreads();
       // Gate factors split at m_b = gam at the first scan position of each
       // 8-row block (as in stage A): P'_ri = arow_r P_ri bcol[b(r)][i].
-      for (int e = tid; e < 8 * 64; e += kWideThreads) {
+      for (int e = tid; e < 8 * 64; e += kOutThreads) {
         const int blk = e >> 6, i = e & 63;
         const int qpos = dir ? 63 - i : i;
         const float mb = sm.gam[dir ? 63 - 8 * blk : 8 * blk];
@@ -836,7 +838,7 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
       mma_ph ^= 1;
       tc_fence_after_sync();
       // U = U~ - W S  -> sW (MN-major B: [slab][64 tokens][8])
-      for (int c = half; c < Dv / 16; c += 2) {
+      for (int c = part; c < Dv / 16; c += 4) {
         float v[16];
         tmem_ld16(tmU + lane_base + 16 * c, v);
         tmem_wait_ld();
@@ -851,7 +853,8 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
         }
       }
       // P'_ri = (q_r . k_i) / |k_i| * e^{gam_r - gam_i} for i at or before r
-      for (int c = half; c < 4; c += 2) {
+      {
+        const int c = part;
         float v[16];
         tmem_ld16(tmP + lane_base + 16 * c, v);
         tmem_wait_ld();
@@ -871,7 +874,7 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
       // Qs = diag(e^gam) Q -> sK (K is dead once P is in TMEM)
       if (lane < 16) {
         const float eg = expf(sm.gam[r]);
-        for (int sl = half; sl < Dk / 8; sl += 2) {
+        for (int sl = part; sl < Dk / 8; sl += 4) {
           float x[8];
           unpack8_bf16(reinterpret_cast<const uint4*>(sQ + sl * kSlab64)[r], x);
 #pragma unroll
@@ -901,7 +904,7 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
     // O = diag(1/|q|) D_O -> out (rows of this chunk that exist)
     {
       const float rq = sm.rnq[r];
-      for (int c = half; c < Dv / 16; c += 2) {
+      for (int c = part; c < Dv / 16; c += 4) {
         float v[16];
         tmem_ld16(tmO + lane_base + 16 * c, v);
         tmem_wait_ld();
@@ -922,7 +925,7 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
   return true;
 }
 
-__global__ void __launch_bounds__(kWideThreads, 1)
+__global__ void __launch_bounds__(kOutThreads, 1)
 gdn_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const float* __restrict__ g, __nv_bfloat16* __restrict__ out, Workspace ws, int T,
                   int H, int ndir, long long limit, unsigned* err) {
@@ -1073,7 +1076,7 @@ cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
   if (e != cudaSuccess) return e;
   {
     ProfileScope ps(a.stream, kKernOutput);
-    gdn_output_kernel<<<dim3(std::min(nC * NBH, num_sms())), kWideThreads,
+    gdn_output_kernel<<<dim3(std::min(nC * NBH, num_sms())), kOutThreads,
                         OutLayout(a.Dk, a.Dv).total, a.stream>>>(
         mq, mk, a.g, static_cast<__nv_bfloat16*>(a.out), ws, a.T, a.H, ndir, a.wait_limit, a.err);
   }
