@@ -57,18 +57,34 @@ constexpr int kRecStages = 4;
 constexpr long long kDrainPolls = 1LL << 40;  // drains are bounded by the 2 s timer
 
 // ----------------------------------------------------------------- workspace
+// One contiguous block per (direction, b*h, chunk), in the order the stages
+// read them so that each read is a single bulk copy:
+//   Qc    [Dk/8][Dk][8]   bf16  chunk summary K~^T W          (stage B)
+//   decay {e^{gamma_C}, 0, 0, 0} fp32                        (stage B)
+//   Rc    [Dv/16][Dk][16] bf16  chunk summary K~^T U~ by slice (stage B)
+//   W     [Dk/8][64][8]   bf16                                (stage C)
+//   Ut    [Dv/8][64][8]   bf16  U~                            (stage C)
+//   S     [Dv/8][Dk][8]   bf16  state at the chunk's start    (stage C)
 struct Workspace {
-  __nv_bfloat16* W;    // [dir][bh][chunk] [Dk/8][64][8]
-  __nv_bfloat16* Ut;   // [dir][bh][chunk] [Dv/8][64][8]
-  __nv_bfloat16* Qc;   // [dir][bh][chunk] [Dk/8][Dk][8]
-  __nv_bfloat16* Rc;   // [dir][bh][chunk] [Dv/16][Dk][16]
-  __nv_bfloat16* S;    // [dir][bh][chunk] [Dv/8][Dk][8]  state at chunk start
-  float* decay;        // [dir][bh][chunk] {e^{gamma_C}, 0, 0, 0} (16 B per chunk)
+  uint8_t* base;
+  size_t block_bytes;
+  uint32_t off_decay, off_rc, off_w, off_ut, off_s;
   int NBH, nC, Dk, Dv;
 
+  __host__ __device__ void layout(int dk, int dv) {
+    Dk = dk;
+    Dv = dv;
+    off_decay = (uint32_t)Dk * Dk * 2;
+    off_rc = off_decay + 16;
+    off_w = off_rc + (uint32_t)Dk * Dv * 2;
+    off_ut = off_w + 64u * Dk * 2;
+    off_s = off_ut + 64u * Dv * 2;
+    block_bytes = ((size_t)off_s + (size_t)Dk * Dv * 2 + 255) & ~size_t(255);
+  }
   __device__ size_t tile(int dir, int bh, int j) const {
     return ((size_t)dir * NBH + bh) * nC + j;
   }
+  __device__ uint8_t* blk(size_t tile_index) const { return base + tile_index * block_bytes; }
 };
 
 // Block-wide bounded wait: every thread polls, then all agree.  On failure
@@ -251,8 +267,8 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
 
   if (tid == 0) {
     mbar_arrive_expect_tx(&s.tma_bar, (Dk / 8 + Dv / 8) * kSlab64);
-    for (int sl = 0; sl < Dk / 8; ++sl) tma_load_4d(s.K + sl * kSlab64, tm_k, &s.tma_bar, 8 * sl, h, t0, b);
-    for (int sl = 0; sl < Dv / 8; ++sl) tma_load_4d(s.V + sl * kSlab64, tm_v, &s.tma_bar, 8 * sl, h, t0, b);
+    tma_load_tile(s.K, tm_k, &s.tma_bar, t0, h, b);
+    tma_load_tile(s.V, tm_v, &s.tma_bar, t0, h, b);
   }
   if (tid < kC) {
     float gv = 0.f, bv = 0.f;  // padding rows: a = 1, beta = 0 (no effect)
@@ -381,8 +397,8 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
     const uint32_t lane_base = static_cast<uint32_t>(32 * quad) << 16;
     const size_t tile = ws.tile(dir, bh, j);
     const float sc = expf(gamC - s.gam[r]) * s.rn[r];
-    uint4* Wg = reinterpret_cast<uint4*>(ws.W + tile * kC * Dk);
-    uint4* Ug = reinterpret_cast<uint4*>(ws.Ut + tile * kC * Dv);
+    uint4* Wg = reinterpret_cast<uint4*>(ws.blk(tile) + ws.off_w);
+    uint4* Ug = reinterpret_cast<uint4*>(ws.blk(tile) + ws.off_ut);
     for (int c = half; c < Dk / 16; c += 2) {
       float v[16];
       tmem_ld16(tm + lane_base + 16 * c, v);
@@ -433,8 +449,8 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
     const int r = 32 * quad + lane;  // TMEM lane = feature row of Qc / Rc
     const uint32_t lane_base = static_cast<uint32_t>(32 * quad) << 16;
     const size_t tile = ws.tile(dir, bh, j);
-    uint4* Qg = reinterpret_cast<uint4*>(ws.Qc + tile * (size_t)Dk * Dk);
-    uint4* Rg = reinterpret_cast<uint4*>(ws.Rc + tile * (size_t)Dk * Dv);
+    uint4* Qg = reinterpret_cast<uint4*>(ws.blk(tile));
+    uint4* Rg = reinterpret_cast<uint4*>(ws.blk(tile) + ws.off_rc);
     for (int c = half; c < Dk / 16; c += 2) {
       float v[16];
       tmem_ld16(tm + lane_base + 16 * c, v);
@@ -454,7 +470,7 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
       }
     }
     if (tid == 0)
-      reinterpret_cast<float4*>(ws.decay)[tile] = make_float4(expf(gamC), 0.f, 0.f, 0.f);
+      *reinterpret_cast<float4*>(ws.blk(tile) + ws.off_decay) = make_float4(expf(gamC), 0.f, 0.f, 0.f);
   }
   return true;
 }
@@ -499,7 +515,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 // the accumulator registers and the bf16 copy of S exchanged through a
 // double-buffered shared-memory operand: one barrier per chunk.
 // Dynamic layout: [head 128 B] [S operand x 2: [2 n-slabs][Dk][8] bf16]
-//                 [stages: Qc [Dk/8][Dk][8] | Rc slice [Dk][16] | decay 16 B]
+//                 [stages: Qc [Dk/8][Dk][8] | decay 16 B | Rc slice [Dk][16]]
 struct RecSmemHead {
   uint64_t full[kRecStages];
 };
@@ -560,10 +576,9 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
     const size_t tile = ws.tile(dir, bh, jt);
     uint8_t* st = stage0 + (c % kRecStages) * stage_bytes;
     uint64_t* bar = &hd.full[c % kRecStages];
-    mbar_arrive_expect_tx(bar, qbytes + rbytes + 16);
-    bulk_load(st, ws.Qc + tile * (size_t)Dk * Dk, qbytes, bar);
-    bulk_load(st + qbytes, ws.Rc + tile * (size_t)Dk * Dv + (size_t)slice * Dk * 16, rbytes, bar);
-    bulk_load(st + qbytes + rbytes, ws.decay + 4 * tile, 16, bar);
+    mbar_arrive_expect_tx(bar, qbytes + 16 + rbytes);
+    bulk_load(st, ws.blk(tile), qbytes + 16, bar);  // Qc and decay
+    bulk_load(st + qbytes + 16, ws.blk(tile) + ws.off_rc + (size_t)slice * Dk * 32, rbytes, bar);
   };
   int issued = min(kRecStages, nC);
   if (tid == 0)
@@ -574,7 +589,7 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
   // at the start of chunk `jt` ([Dv/8][Dk][8]).
   auto publish = [&](int buf, size_t tile) {
     uint8_t* Sop = Sop0 + buf * kRecSBytes;
-    __nv_bfloat16* Sg = ws.S + tile * (size_t)Dk * Dv;
+    __nv_bfloat16* Sg = reinterpret_cast<__nv_bfloat16*>(ws.blk(tile) + ws.off_s);
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
       const uint32_t lo = pack_bf16x2(S[nt][0], S[nt][1]);
@@ -621,8 +636,8 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
     }
     // S <- e^{gamma_C} S - Qc S + Rc
     const uint8_t* stp = stage0 + st * stage_bytes;
-    const float a = *reinterpret_cast<const float*>(stp + qbytes + rbytes);
-    const __nv_bfloat16* R = reinterpret_cast<const __nv_bfloat16*>(stp + qbytes);
+    const float a = *reinterpret_cast<const float*>(stp + qbytes);
+    const __nv_bfloat16* R = reinterpret_cast<const __nv_bfloat16*>(stp + qbytes + 16);
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
       const __nv_bfloat162 r0 = *reinterpret_cast<const __nv_bfloat162*>(R + rA * 16 + 8 * nt + cA);
@@ -671,9 +686,9 @@ gdn_recur_kernel(const float* state_in, float* state_out, Workspace ws, long lon
 // land while the current tile computes.  Per set (offsets from Dk, Dv):
 //   Q   [Dk/8][64][8]  raw q tile (TMA)
 //   K   [Dk/8][64][8]  raw k tile (TMA); after P = Q K^T it holds Qs = diag(e^g) Q
-//   W   [max(Dk,Dv)/8][64][8]  W of the current direction; after W S it holds U
-//   Ut  [Dv/8][64][8]  U~ of the current direction
-//   S   [Dv/8][Dk][8]  state at the chunk's start (MN-major B operand)
+//   W   [Dk/8][64][8]  W of the current direction     } one contiguous block,
+//   Ut  [Dv/8][64][8]  U~, then U in place            } as in the workspace:
+//   S   [Dv/8][Dk][8]  state at the chunk's start     } a single bulk copy
 // then P [8][64][8] (masked, gated Q K^T, K-major A) and the scalar block.
 struct OutSmall {
   float g[2][64];
@@ -689,8 +704,8 @@ struct OutLayout {
     q = 0;
     k = al(q + 64u * Dk * 2);
     w = al(k + 64u * Dk * 2);
-    ut = al(w + 64u * (Dk > Dv ? Dk : Dv) * 2);  // W, later U: room for either
-    s = al(ut + 64u * Dv * 2);
+    ut = w + 64u * Dk * 2;
+    s = ut + 64u * Dv * 2;
     set_bytes = al(s + (uint32_t)Dk * Dv * 2);
     p = 2 * set_bytes;
     small = al(p + 8u * kSlab64);
@@ -724,14 +739,12 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
   const int r = 16 * quad + (lane & 15);
   const uint32_t lane_base = static_cast<uint32_t>(32 * quad) << 16;
 
-  auto issue_dir = [&](int set, int tile_t, int dir) {  // thread 0
+  auto issue_dir = [&](int set, int tile_t, int dir) {  // thread 0: W | U~ | S
     uint8_t* base = smem + set * L.set_bytes;
     const int bh = tile_t / nC, j = tile_t - bh * nC;
     const size_t tile = ws.tile(dir, bh, j);
     mbar_arrive_expect_tx(&sm.ld_bar[set], wbytes + ubytes + sbytes);
-    bulk_load(base + L.w, ws.W + tile * kC * Dk, wbytes, &sm.ld_bar[set]);
-    bulk_load(base + L.ut, ws.Ut + tile * kC * Dv, ubytes, &sm.ld_bar[set]);
-    bulk_load(base + L.s, ws.S + tile * (size_t)Dk * Dv, sbytes, &sm.ld_bar[set]);
+    bulk_load(base + L.w, ws.blk(tile) + ws.off_w, wbytes + ubytes + sbytes, &sm.ld_bar[set]);
   };
   // all threads: start loading tile `tile_t` into `set`
   auto issue_tile = [&](int set, int tile_t) {
@@ -740,10 +753,8 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
     if (tid == 0) {
       uint8_t* base = smem + set * L.set_bytes;
       mbar_arrive_expect_tx(&sm.tma_bar[set], 2 * (Dk / 8) * kSlab64);
-      for (int sl = 0; sl < Dk / 8; ++sl) {
-        tma_load_4d(base + L.q + sl * kSlab64, tm_q, &sm.tma_bar[set], 8 * sl, h, t0, b);
-        tma_load_4d(base + L.k + sl * kSlab64, tm_k, &sm.tma_bar[set], 8 * sl, h, t0, b);
-      }
+      tma_load_tile(base + L.q, tm_q, &sm.tma_bar[set], t0, h, b);
+      tma_load_tile(base + L.k, tm_k, &sm.tma_bar[set], t0, h, b);
       issue_dir(set, tile_t, 0);
     }
     if (tid < kC) {
@@ -771,8 +782,8 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
     uint8_t* base = smem + set * L.set_bytes;
     uint8_t* sQ = base + L.q;
     uint8_t* sK = base + L.k;   // then Qs
-    uint8_t* sW = base + L.w;   // then U
-    uint8_t* sUt = base + L.ut;
+    uint8_t* sW = base + L.w;
+    uint8_t* sUt = base + L.ut;  // then U
     uint8_t* sS = base + L.s;
     const int bh = t / nC, j = t - bh * nC;
     const int b = bh / H, h = bh - b * H, t0 = j * kC;
@@ -837,7 +848,7 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
       }
       mma_ph ^= 1;
       tc_fence_after_sync();
-      // U = U~ - W S  -> sW (MN-major B: [slab][64 tokens][8])
+      // U = U~ - W S, in place of U~ (MN-major B: [slab][64 tokens][8])
       for (int c = part; c < Dv / 16; c += 4) {
         float v[16];
         tmem_ld16(tmU + lane_base + 16 * c, v);
@@ -848,8 +859,8 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
           unpack8_bf16(reinterpret_cast<const uint4*>(sUt + (2 * c + 1) * kSlab64)[r], ut + 8);
 #pragma unroll
           for (int e = 0; e < 16; ++e) ut[e] -= v[e];
-          reinterpret_cast<uint4*>(sW + (2 * c) * kSlab64)[r] = pack8_bf16(ut);
-          reinterpret_cast<uint4*>(sW + (2 * c + 1) * kSlab64)[r] = pack8_bf16(ut + 8);
+          reinterpret_cast<uint4*>(sUt + (2 * c) * kSlab64)[r] = pack8_bf16(ut);
+          reinterpret_cast<uint4*>(sUt + (2 * c + 1) * kSlab64)[r] = pack8_bf16(ut + 8);
         }
       }
       // P'_ri = (q_r . k_i) / |k_i| * e^{gam_r - gam_i} for i at or before r
@@ -890,7 +901,7 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
                    sdesc(smem_u32(sS) + ks * 256, 128, Dk * 16), idO, (dir > 0) || (ks > 0));
         for (int ks = 0; ks < kC / 16; ++ks)
           mma_bf16(tmO, sdesc(smem_u32(sP) + ks * 2 * kSlab64, kSlab64, 128),
-                   sdesc(smem_u32(sW) + ks * 256, 128, kSlab64), idO, 1);
+                   sdesc(smem_u32(sUt) + ks * 256, 128, kSlab64), idO, 1);
         mma_commit(&sm.mma_bar);
       }
       if (!block_wait(&sm.mma_bar, mma_ph, limit, err)) {
@@ -972,20 +983,21 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [B, T, H, D] bf16 tensor; box = 8 features x 1 head x 64 tokens x 1 batch.
+// A [B, T, H, D] bf16 tensor viewed as 5-D (8 features, T, D/8 feature slabs,
+// H, B) so that one box (8 x 64 tokens x D/8 slabs x 1 x 1) lands in shared
+// memory exactly in the [slab][token][8] core-matrix layout of a tile.
 bool make_map(CUtensorMap* m, const void* base, int B, int T, int H, int D) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-  const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
-  const cuuint32_t box[4] = {8, 1, (cuuint32_t)kC, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+  const cuuint64_t dims[5] = {8, (cuuint64_t)T, (cuuint64_t)(D / 8), (cuuint64_t)H, (cuuint64_t)B};
+  const cuuint64_t strides[4] = {(cuuint64_t)H * D * 2, 16, (cuuint64_t)D * 2,
+                                 (cuuint64_t)T * H * D * 2};
+  const cuuint32_t box[5] = {8, (cuuint32_t)kC, (cuuint32_t)(D / 8), 1, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-
-size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Streaming multiprocessors of the current device (persistent grids).
 int num_sms() {
@@ -1033,9 +1045,9 @@ cudaError_t set_smem_attrs() {
 
 size_t chunk_tc_workspace_bytes(int B, int T, int H, int Dk, int Dv, bool bidir) {
   const size_t tiles = (size_t)(bidir ? 2 : 1) * B * H * ((T + kC - 1) / kC);
-  return align256(tiles * kC * Dk * 2) + align256(tiles * kC * Dv * 2) +
-         align256(tiles * (size_t)Dk * Dk * 2) + align256(tiles * (size_t)Dk * Dv * 2) +
-         align256(tiles * (size_t)Dk * Dv * 2) + align256(tiles * 16);
+  Workspace ws;
+  ws.layout(Dk, Dv);
+  return tiles * ws.block_bytes;
 }
 
 cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
@@ -1044,16 +1056,11 @@ cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
   const int ndir = a.bidir ? 2 : 1;
   const int nC = (a.T + kC - 1) / kC;
   const int NBH = a.B * a.H;
-  const size_t tiles = (size_t)ndir * NBH * nC;
   Workspace ws;
-  uint8_t* p = static_cast<uint8_t*>(workspace);
-  ws.W = reinterpret_cast<__nv_bfloat16*>(p);  p += align256(tiles * kC * a.Dk * 2);
-  ws.Ut = reinterpret_cast<__nv_bfloat16*>(p); p += align256(tiles * kC * a.Dv * 2);
-  ws.Qc = reinterpret_cast<__nv_bfloat16*>(p); p += align256(tiles * (size_t)a.Dk * a.Dk * 2);
-  ws.Rc = reinterpret_cast<__nv_bfloat16*>(p); p += align256(tiles * (size_t)a.Dk * a.Dv * 2);
-  ws.S = reinterpret_cast<__nv_bfloat16*>(p);  p += align256(tiles * (size_t)a.Dk * a.Dv * 2);
-  ws.decay = reinterpret_cast<float*>(p);
-  ws.NBH = NBH; ws.nC = nC; ws.Dk = a.Dk; ws.Dv = a.Dv;
+  ws.base = static_cast<uint8_t*>(workspace);
+  ws.layout(a.Dk, a.Dv);
+  ws.NBH = NBH;
+  ws.nC = nC;
 
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, a.q, a.B, a.T, a.H, a.Dk) || !make_map(&mk, a.k, a.B, a.T, a.H, a.Dk) ||
