@@ -169,12 +169,49 @@ struct PrepSmem {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// tf32 tensor-core product on fp32 shared-memory tiles (row stride kLd):
+// D(16 x 8) = sum_k A[ar + i][ac + k] * B[br + k][bc + j], k < 8 * ksteps,
+// one warp, mma.sync.m16n8k8 (tf32 inputs rounded to nearest, fp32 accumulate).
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ void warp_mma_tf32(const float (*A)[kLd], int ar, int ac,
+                                              const float (*B)[kLd], int br, int bc, int ksteps,
+                                              float (&d)[4]) {
+  const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+  d[0] = d[1] = d[2] = d[3] = 0.f;
+  for (int ks = 0; ks < ksteps; ++ks) {
+    const int k0 = 8 * ks;
+    const uint32_t a0 = to_tf32(A[ar + gq][ac + k0 + tq]);
+    const uint32_t a1 = to_tf32(A[ar + gq + 8][ac + k0 + tq]);
+    const uint32_t a2 = to_tf32(A[ar + gq][ac + k0 + tq + 4]);
+    const uint32_t a3 = to_tf32(A[ar + gq + 8][ac + k0 + tq + 4]);
+    const uint32_t b0 = to_tf32(B[br + k0 + tq][bc + gq]);
+    const uint32_t b1 = to_tf32(B[br + k0 + tq + 4][bc + gq]);
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
+}
+// Store a 16 x 8 accumulator tile (times `sign`) at C[cr .. cr+15][cc .. cc+7].
+__device__ __forceinline__ void warp_store_tile(float (*C)[kLd], int cr, int cc, const float (&d)[4],
+                                                float sign) {
+  const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+  *reinterpret_cast<float2*>(&C[cr + gq][cc + 2 * tq]) = make_float2(sign * d[0], sign * d[1]);
+  *reinterpret_cast<float2*>(&C[cr + gq + 8][cc + 2 * tq]) = make_float2(sign * d[2], sign * d[3]);
+}
+
 // In-place blocked inverse of the unit lower-triangular 64 x 64 matrix
 // I + A (A strictly lower, scan order) into T:
-//   16 x 16 diagonal blocks by right-looking forward substitution (one lane
-//   per column: the dependent chain is one FMA per row);
+//   16 x 16 diagonal blocks by right-looking forward substitution in fp32
+//   (one lane per column: the dependent chain is one FMA per row);
 //   16 -> 32:  T_hl = -T_hh (A_hl T_ll) for the two 32 x 32 diagonal halves;
-//   32 -> 64:  T_HL = -T_HH (A_HL T_LL) for the lower-left 32 x 32 block.
+//   32 -> 64:  T_HL = -T_HH (A_HL T_LL) for the lower-left 32 x 32 block;
+// the block products on tf32 tensor cores (T is rounded to bf16 right after).
 __device__ void unit_lower_inverse(PrepSmem::U& u) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   float (*A)[kLd] = u.a.A;
@@ -198,53 +235,32 @@ __device__ void unit_lower_inverse(PrepSmem::U& u) {
     for (int t = 0; t < 16; ++t) T[b0 + t][b0 + j] = acc[t];
   }
   __syncthreads();
-  // 16 -> 32: pairs (blocks 1,0) and (3,2); thread: 1 x 2 strip of a 16 x 16 block
-  {
-    const int pr = tid >> 7, idx = tid & 127, r = idx >> 3, c0 = (idx & 7) * 2;
+  // 16 -> 32: pair p = warp >> 1 (blocks (32p+16, 32p)), n-tile = warp & 1
+  if (warp < 4) {
+    const int pr = warp >> 1, nt = warp & 1;
     const int hb = 32 * pr + 16, lb = 32 * pr;
-    float y0 = 0.f, y1 = 0.f;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const float a = A[hb + r][lb + k];
-      const float2 t = *reinterpret_cast<const float2*>(&T[lb + k][lb + c0]);
-      y0 = fmaf(a, t.x, y0);
-      y1 = fmaf(a, t.y, y1);
-    }
-    *reinterpret_cast<float2*>(&Y[hb + r][lb + c0]) = make_float2(y0, y1);
-    __syncthreads();
-    float z0 = 0.f, z1 = 0.f;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const float a = T[hb + r][hb + k];
-      const float2 t = *reinterpret_cast<const float2*>(&Y[hb + k][lb + c0]);
-      z0 = fmaf(a, t.x, z0);
-      z1 = fmaf(a, t.y, z1);
-    }
-    *reinterpret_cast<float2*>(&T[hb + r][lb + c0]) = make_float2(-z0, -z1);
+    float d[4];
+    warp_mma_tf32(A, hb, lb, T, lb, lb + 8 * nt, 2, d);
+    warp_store_tile(Y, hb, lb + 8 * nt, d, 1.f);
   }
   __syncthreads();
-  // 32 -> 64: thread: 1 x 4 strip of the 32 x 32 block
+  if (warp < 4) {
+    const int pr = warp >> 1, nt = warp & 1;
+    const int hb = 32 * pr + 16, lb = 32 * pr;
+    float d[4];
+    warp_mma_tf32(T, hb, hb, Y, hb, lb + 8 * nt, 2, d);
+    warp_store_tile(T, hb, lb + 8 * nt, d, -1.f);
+  }
+  __syncthreads();
+  // 32 -> 64: the 32 x 32 block as 2 x 4 tiles of 16 x 8, one per warp
   {
-    const int r = tid >> 3, c0 = (tid & 7) * 4;
-    float y[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-    for (int k = 0; k < 32; ++k) {
-      const float a = A[32 + r][k];
-      const float4 t = *reinterpret_cast<const float4*>(&T[k][c0]);
-      y[0] = fmaf(a, t.x, y[0]); y[1] = fmaf(a, t.y, y[1]);
-      y[2] = fmaf(a, t.z, y[2]); y[3] = fmaf(a, t.w, y[3]);
-    }
-    *reinterpret_cast<float4*>(&Y[32 + r][c0]) = make_float4(y[0], y[1], y[2], y[3]);
+    const int mt = warp >> 2, nt = warp & 3;
+    float d[4];
+    warp_mma_tf32(A, 32 + 16 * mt, 0, T, 0, 8 * nt, 4, d);
+    warp_store_tile(Y, 32 + 16 * mt, 8 * nt, d, 1.f);
     __syncthreads();
-    float z[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-    for (int k = 0; k < 32; ++k) {
-      const float a = T[32 + r][32 + k];
-      const float4 t = *reinterpret_cast<const float4*>(&Y[32 + k][c0]);
-      z[0] = fmaf(a, t.x, z[0]); z[1] = fmaf(a, t.y, z[1]);
-      z[2] = fmaf(a, t.z, z[2]); z[3] = fmaf(a, t.w, z[3]);
-    }
-    *reinterpret_cast<float4*>(&T[32 + r][c0]) = make_float4(-z[0], -z[1], -z[2], -z[3]);
+    warp_mma_tf32(T, 32 + 16 * mt, 32, Y, 32, 8 * nt, 4, d);
+    warp_store_tile(T, 32 + 16 * mt, 8 * nt, d, -1.f);
   }
   __syncthreads();
 }
