@@ -34,7 +34,8 @@ enum KernelId : int {
   kKernPrep = 1,
   kKernRecur = 2,
   kKernOutput = 3,
-  kNumKernelIds = 4,
+  kKernCompose = 4,
+  kNumKernelIds = 5,
 };
 
 // While profiling is armed, records CUDA events around one launch.
