@@ -43,7 +43,6 @@ KERNEL_SOURCES = {
     "gdn_prep_kernel": "gated_deltanet_linear_chunked_b200/csrc/chunk_tc.cu",
     "gdn_recur_kernel": "gated_deltanet_linear_chunked_b200/csrc/chunk_tc.cu",
     "gdn_output_kernel": "gated_deltanet_linear_chunked_b200/csrc/chunk_tc.cu",
-    "gdn_compose_kernel": "gated_deltanet_linear_chunked_b200/csrc/chunk_tc.cu",
 }
 
 
@@ -100,8 +99,6 @@ def kernel_algorithmic_bytes(name, w) -> int:
         return state
     if name == "gdn_output_kernel":
         return w.head_tokens * ((w.Dk + w.Dv) * es)
-    if name == "gdn_compose_kernel":
-        return 0  # works on scratch only
     return algorithmic_bytes(w)
 
 
@@ -454,11 +451,11 @@ def main():
     with torch.cuda.stream(stream):
         for i in range(n_prof):
             step(i)
-    kms = (ctypes.c_float * 8)()
-    kn = (ctypes.c_int * 8)()
-    _lib.check(lib.gdn_profile_end(ctypes.addressof(kms), ctypes.addressof(kn), 8), "gdn_profile_end")
+    kms = (ctypes.c_float * 4)()
+    kn = (ctypes.c_int * 4)()
+    _lib.check(lib.gdn_profile_end(ctypes.addressof(kms), ctypes.addressof(kn), 4), "gdn_profile_end")
     kernels = {}
-    for i in range(8):
+    for i in range(4):
         if kn[i]:
             name = lib.gdn_kernel_name(i).decode()
             kernels[name] = {"launches": kn[i], "ms_per_launch": kms[i] / kn[i]}

@@ -53,6 +53,7 @@ constexpr int kC = 64;            // tokens per chunk
 constexpr int kWideThreads = 256; // stage A: two warps per TMEM lane quadrant
 constexpr int kOutThreads = 512;  // stage C: four warps per TMEM lane quadrant
 constexpr int kSlab64 = kC * 16;  // bytes of one 8-column slab of a 64-row tile
+constexpr int kRecStages = 4;
 constexpr long long kDrainPolls = 1LL << 40;  // drains are bounded by the 2 s timer
 
 // ----------------------------------------------------------------- workspace
@@ -60,20 +61,15 @@ constexpr long long kDrainPolls = 1LL << 40;  // drains are bounded by the 2 s t
 // read them so that each read is a single bulk copy:
 //   Qc    [Dk/8][Dk][8]   bf16  chunk summary K~^T W          (stage B)
 //   decay {e^{gamma_C}, 0, 0, 0} fp32                        (stage B)
-//   Rc    [Dv/8][Dk][8]   bf16  chunk summary K~^T U~           (stage B)
+//   Rc    [Dv/16][Dk][16] bf16  chunk summary K~^T U~ by slice (stage B)
 //   W     [Dk/8][64][8]   bf16                                (stage C)
 //   Ut    [Dv/8][64][8]   bf16  U~                            (stage C)
 //   S     [Dv/8][Dk][8]   bf16  state at the chunk's start    (stage C)
-// After the chunk blocks, one block per (direction, b*h, pair of consecutive
-// chunks in scan order) holds the pair's composed summary, same layout as the
-// chunk blocks' first three fields: Qp [Dk/8][Dk][8] | decay_p | Rp [Dv/8][Dk][8].
 struct Workspace {
   uint8_t* base;
   size_t block_bytes;
-  size_t pair_bytes;   // bytes of one pair block
-  size_t pairs_off;    // byte offset of the first pair block
   uint32_t off_decay, off_rc, off_w, off_ut, off_s;
-  int NBH, nC, nP, Dk, Dv;
+  int NBH, nC, Dk, Dv;
 
   __host__ __device__ void layout(int dk, int dv) {
     Dk = dk;
@@ -84,15 +80,11 @@ struct Workspace {
     off_ut = off_w + 64u * Dk * 2;
     off_s = off_ut + 64u * Dv * 2;
     block_bytes = ((size_t)off_s + (size_t)Dk * Dv * 2 + 255) & ~size_t(255);
-    pair_bytes = ((size_t)off_w + 255) & ~size_t(255);
   }
   __device__ size_t tile(int dir, int bh, int j) const {
     return ((size_t)dir * NBH + bh) * nC + j;
   }
   __device__ uint8_t* blk(size_t tile_index) const { return base + tile_index * block_bytes; }
-  __device__ uint8_t* pair_blk(int dir, int bh, int pi) const {
-    return base + pairs_off + (((size_t)dir * NBH + bh) * nP + pi) * pair_bytes;
-  }
 };
 
 // Block-wide bounded wait: every thread polls, then all agree.  On failure
@@ -489,8 +481,8 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
       tmem_ld16(tm + lane_base + 128 + 16 * c, v);
       tmem_wait_ld();
       if (r < Dk) {
-        Rg[(2 * c) * Dk + r] = pack8_bf16(v);
-        Rg[(2 * c + 1) * Dk + r] = pack8_bf16(v + 8);
+        Rg[(c * Dk + r) * 2] = pack8_bf16(v);
+        Rg[(c * Dk + r) * 2 + 1] = pack8_bf16(v + 8);
       }
     }
     if (tid == 0)
@@ -529,140 +521,19 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
   if ((tid >> 5) == 0) tmem_dealloc(s.tmem, 256);
 }
 
-// ================================================== stage B0: chunk pairs
-// Two consecutive chunks (scan order 2p, 2p+1) act on the state as one affine
-// map: with P_k = e^{gamma_k} I - Qc_k,
-//   S_{2p+2} = P_2 P_1 S_{2p} + P_2 Rc_1 + Rc_2
-//            = e^{gamma_1 + gamma_2} S - Qp S + Rp,
-//   Qp = e^{gamma_1} Qc_2 + e^{gamma_2} Qc_1 - Qc_2 Qc_1,
-//   Rp = e^{gamma_2} Rc_1 - Qc_2 Rc_1 + Rc_2,
-// so the dependent walk of stage B takes ceil(nC / 2) steps.  One CTA per
-// (pair, b*h, direction): two tcgen05 products (M = 128 >= Dk rows of Qc_2)
-// and an epilogue; a trailing single chunk is copied through.
-struct PairSmemHead {
-  uint64_t ld_bar, mma_bar;
-  uint32_t tmem;
-};
-
-__device__ bool compose_body(uint8_t* smem, const Workspace& ws, long long limit, unsigned* err) {
-  PairSmemHead& hd = *reinterpret_cast<PairSmemHead*>(smem);
-  const int Dk = ws.Dk, Dv = ws.Dv, nC = ws.nC;
-  const int pi = blockIdx.x, bh = blockIdx.y, dir = blockIdx.z;
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const uint32_t head_bytes = (uint32_t)ws.off_w;  // Qc | decay | Rc of one chunk
-  uint8_t* blk1 = smem + 128;                      // chunk 2p
-  uint8_t* blk2 = blk1 + ((head_bytes + 127) & ~127u);  // chunk 2p + 1
-  const int c1 = 2 * pi, c2 = 2 * pi + 1;
-  const size_t t1 = ws.tile(dir, bh, dir ? nC - 1 - c1 : c1);
-  uint8_t* out = ws.pair_blk(dir, bh, pi);
-  if (c2 >= nC) {  // trailing single chunk: its own summary
-    const uint4* src = reinterpret_cast<const uint4*>(ws.blk(t1));
-    uint4* dst = reinterpret_cast<uint4*>(out);
-    for (uint32_t i = tid; i < head_bytes / 16; i += blockDim.x) dst[i] = src[i];
-    return true;
-  }
-  const size_t t2 = ws.tile(dir, bh, dir ? nC - 1 - c2 : c2);
-  const uint32_t tm = hd.tmem;
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&hd.ld_bar, 2 * head_bytes);
-    bulk_load(blk1, ws.blk(t1), head_bytes, &hd.ld_bar);
-    bulk_load(blk2, ws.blk(t2), head_bytes, &hd.ld_bar);
-  }
-  if (!block_wait(&hd.ld_bar, 0, limit, err)) return false;
-  // D1 = Qc_2 Qc_1 (N = Dk), D2 = Qc_2 Rc_1 (N = Dv); Qc_2 K-major A (its rows
-  // past Dk are don't-care), Qc_1 / Rc_1 MN-major B (rows = K)
-  if (tid == 0) {
-    tc_fence_after_sync();
-    const uint32_t idQ = idesc_bf16(128, Dk, 0, 1), idR = idesc_bf16(128, Dv, 0, 1);
-    for (int ks = 0; ks < Dk / 16; ++ks) {
-      const uint64_t a = sdesc(smem_u32(blk2) + ks * 2 * Dk * 16, Dk * 16, 128);
-      mma_bf16(tm, a, sdesc(smem_u32(blk1) + ks * 256, 128, Dk * 16), idQ, ks > 0);
-      mma_bf16(tm + 128, a, sdesc(smem_u32(blk1 + ws.off_rc) + ks * 256, 128, Dk * 16), idR, ks > 0);
-    }
-    mma_commit(&hd.mma_bar);
-  }
-  if (!block_wait(&hd.mma_bar, 0, limit, err)) return false;
-  tc_fence_after_sync();
-  const float e1 = *reinterpret_cast<const float*>(blk1 + ws.off_decay);
-  const float e2 = *reinterpret_cast<const float*>(blk2 + ws.off_decay);
-  const int r = tid;  // TMEM lane = row of Qp / Rp
-  const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
-  for (int c = 0; c < Dk / 16; ++c) {
-    float v[16];
-    tmem_ld16(tm + lane_base + 16 * c, v);
-    tmem_wait_ld();
-    if (r < Dk) {
-#pragma unroll
-      for (int hsl = 0; hsl < 2; ++hsl) {
-        const int sl = 2 * c + hsl;
-        float q1[8], q2[8], o[8];
-        unpack8_bf16(reinterpret_cast<const uint4*>(blk1 + sl * Dk * 16)[r], q1);
-        unpack8_bf16(reinterpret_cast<const uint4*>(blk2 + sl * Dk * 16)[r], q2);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] = e1 * q2[e] + e2 * q1[e] - v[8 * hsl + e];
-        reinterpret_cast<uint4*>(out + sl * Dk * 16)[r] = pack8_bf16(o);
-      }
-    }
-  }
-  for (int c = 0; c < Dv / 16; ++c) {
-    float v[16];
-    tmem_ld16(tm + lane_base + 128 + 16 * c, v);
-    tmem_wait_ld();
-    if (r < Dk) {
-#pragma unroll
-      for (int hsl = 0; hsl < 2; ++hsl) {
-        const int sl = 2 * c + hsl;
-        float r1[8], r2[8], o[8];
-        unpack8_bf16(reinterpret_cast<const uint4*>(blk1 + ws.off_rc + sl * Dk * 16)[r], r1);
-        unpack8_bf16(reinterpret_cast<const uint4*>(blk2 + ws.off_rc + sl * Dk * 16)[r], r2);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] = e2 * r1[e] - v[8 * hsl + e] + r2[e];
-        reinterpret_cast<uint4*>(out + ws.off_rc + sl * Dk * 16)[r] = pack8_bf16(o);
-      }
-    }
-  }
-  if (tid == 0)
-    *reinterpret_cast<float4*>(out + ws.off_decay) = make_float4(e1 * e2, 0.f, 0.f, 0.f);
-  return true;
-}
-
-__global__ void __launch_bounds__(128, 2)
-gdn_compose_kernel(Workspace ws, long long limit, unsigned* err) {
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  PairSmemHead& hd = *reinterpret_cast<PairSmemHead*>(smem_raw);
-  const int tid = threadIdx.x;
-  if (tid == 0) {
-    mbar_init(&hd.ld_bar, 1);
-    mbar_init(&hd.mma_bar, 1);
-    fence_mbar_init();
-  }
-  if ((tid >> 5) == 0) {
-    tmem_alloc(&hd.tmem, 256);
-    tmem_relinquish();
-  }
-  block_sync_async();
-  compose_body(smem_raw, ws, limit, err);
-  tc_fence_before_sync();
-  __syncthreads();
-  if ((tid >> 5) == 0) tmem_dealloc(hd.tmem, 256);
-}
-
 // ======================================================= stage B: recurrence
-// One CTA per (16 state columns, b*h, direction).  The walk steps over chunk
-// pairs: warps [0, Dk/16) own state rows [16w, 16w + 16) and compute
-// S_{2p+2} = d_p S_{2p} - Qp S_{2p} + Rp (the dependent chain; fp32 state in
-// the accumulator registers), while warps [Dk/16, 2 Dk/16) compute the odd
-// chunk's start state S_{2p+1} = d_1 S_{2p} - Qc_1 S_{2p} + Rc_1 from the same
-// operand, off the chain, for stage C.  The per-step product (Dk x Dk times
-// Dk x 16) is latency-bound: a tcgen05 round trip (issue, commit, mbarrier,
-// TMEM load) measured ~1.2k cycles per step here, so this stage uses
-// warp-level mma.sync.m16n8k16 (bf16 in, fp32 accumulate) with a
-// double-buffered bf16 copy of S in shared memory and one barrier per step.
+// One CTA per (16 state columns, b*h, direction), Dk/16 warps; warp w owns
+// state rows [16w, 16w + 16).  Per chunk the product Qc S (Dk x Dk times
+// Dk x 16) is a dependent chain across chunks and is latency-bound: a
+// tcgen05 round trip (issue 7 MMAs, commit, mbarrier, TMEM load) costs
+// ~1.2k cycles per chunk here, so this stage uses warp-level
+// mma.sync.m16n8k16 (bf16 in, fp32 accumulate) with the fp32 state held in
+// the accumulator registers and the bf16 copy of S exchanged through a
+// double-buffered shared-memory operand: one barrier per chunk.
 // Dynamic layout: [head 128 B] [S operand x 2: [2 n-slabs][Dk][8] bf16]
-//   [stages: Qp | d_p | Rp slice [2][Dk][8] | Qc_1 | d_1 | Rc_1 slice [2][Dk][8]]
-constexpr int kRecMaxStages = 4;
+//                 [stages: Qc [Dk/8][Dk][8] | decay 16 B | Rc slice [Dk][16]]
 struct RecSmemHead {
-  uint64_t full[kRecMaxStages];
+  uint64_t full[kRecStages];
 };
 constexpr int kRecHeadBytes = 128;
 constexpr int kRecSBytes = 2 * 128 * 16;  // one S operand buffer at Dk = 128
@@ -687,38 +558,27 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__host__ __device__ inline uint32_t rec_half_bytes(int Dk) {  // one summary in a stage
-  return (uint32_t)Dk * Dk * 2 + 16 + (uint32_t)Dk * 32;
-}
-__host__ __device__ inline uint32_t rec_stage_bytes(int Dk) {
-  return (2 * rec_half_bytes(Dk) + 127) & ~127u;
-}
-
 __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_out,
-                           const Workspace& ws, int nstages, long long limit, unsigned* err) {
+                           const Workspace& ws, long long limit, unsigned* err) {
   RecSmemHead& hd = *reinterpret_cast<RecSmemHead*>(smem);
-  const int Dk = ws.Dk, Dv = ws.Dv, nC = ws.nC, nP = ws.nP;
+  const int Dk = ws.Dk, Dv = ws.Dv, nC = ws.nC;
   uint8_t* Sop0 = smem + kRecHeadBytes;
   const uint32_t nslab_bytes = (uint32_t)Dk * 16;  // one n-slab [Dk][8] bf16 of the operand
   uint8_t* stage0 = Sop0 + 2 * kRecSBytes;
   const uint32_t qbytes = (uint32_t)Dk * Dk * 2, rbytes = (uint32_t)Dk * 32;
-  const uint32_t half_bytes = rec_half_bytes(Dk);
-  const uint32_t stage_bytes = rec_stage_bytes(Dk);
+  const uint32_t stage_bytes = (qbytes + rbytes + 16 + 127) & ~127u;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int slice = blockIdx.x, bh = blockIdx.y, dir = blockIdx.z;
-  const int nks = Dk / 16, nrw = Dk / 16;
-  const bool odd = warp >= nrw;              // computes the odd chunk's state
-  const int rw = odd ? warp - nrw : warp;    // row slab of this warp
-  const uint32_t sub = odd ? half_bytes : 0; // which summary of the stage
+  const int nks = Dk / 16;
   // accumulator coordinates of this thread: rows rA, rA + 8; columns cA, cA + 1 (+ 8 nt)
-  const int rA = 16 * rw + (lane >> 2), cA = 2 * (lane & 3);
+  const int rA = 16 * warp + (lane >> 2), cA = 2 * (lane & 3);
 
-  float S[2][4];  // [n-tile][c0..c3], fp32 state (chain warps)
+  float S[2][4];  // [n-tile][c0..c3], fp32 state
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
     for (int i = 0; i < 4; ++i) S[nt][i] = 0.f;
-  if (!odd && dir == 0 && state_in) {
+  if (dir == 0 && state_in) {
     const float* base = state_in + (size_t)bh * Dk * Dv + 16 * slice;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
@@ -727,62 +587,56 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
       S[nt][0] = lo.x; S[nt][1] = lo.y; S[nt][2] = hi.x; S[nt][3] = hi.y;
     }
   }
-  auto chunk_tile = [&](int c) { return ws.tile(dir, bh, dir ? nC - 1 - c : c); };
-  auto issue = [&](int pi) {  // one thread: load pair pi's summaries into its stage
-    uint8_t* st = stage0 + (pi % nstages) * stage_bytes;
-    uint64_t* bar = &hd.full[pi % nstages];
-    const uint8_t* pb = ws.pair_blk(dir, bh, pi);
-    const uint8_t* cb = ws.blk(chunk_tile(2 * pi));
-    mbar_arrive_expect_tx(bar, 2 * half_bytes);
-    bulk_load(st, pb, qbytes + 16, bar);  // Qp and d_p
-    bulk_load(st + qbytes + 16, pb + ws.off_rc + (size_t)slice * rbytes, rbytes, bar);
-    bulk_load(st + half_bytes, cb, qbytes + 16, bar);  // Qc_1 and d_1
-    bulk_load(st + half_bytes + qbytes + 16, cb + ws.off_rc + (size_t)slice * rbytes, rbytes, bar);
+  auto issue = [&](int c) {  // one thread: load chunk c (scan order) into its stage
+    const int jt = dir ? nC - 1 - c : c;
+    const size_t tile = ws.tile(dir, bh, jt);
+    uint8_t* st = stage0 + (c % kRecStages) * stage_bytes;
+    uint64_t* bar = &hd.full[c % kRecStages];
+    mbar_arrive_expect_tx(bar, qbytes + 16 + rbytes);
+    bulk_load(st, ws.blk(tile), qbytes + 16, bar);  // Qc and decay
+    bulk_load(st + qbytes + 16, ws.blk(tile) + ws.off_rc + (size_t)slice * Dk * 32, rbytes, bar);
   };
-  int issued = min(nstages, nP);
+  int issued = min(kRecStages, nC);
   if (tid == 0)
-    for (int pi = 0; pi < issued; ++pi) issue(pi);
+    for (int c = 0; c < issued; ++c) issue(c);
 
-  // bf16 state at this thread's accumulator positions -> operand buffer
-  // `buf` (chain warps) and the workspace copy for stage C (chunk tile `tile`)
-  auto store_state = [&](const float (&X)[2][4], int buf, bool to_operand, size_t tile) {
+  // S (bf16) of this thread's accumulator positions -> operand buffer `buf`
+  // ([n-slab][Dk rows][8]) and, for stage C, the workspace copy of the state
+  // at the start of chunk `jt` ([Dv/8][Dk][8]).
+  auto publish = [&](int buf, size_t tile) {
     uint8_t* Sop = Sop0 + buf * kRecSBytes;
     __nv_bfloat16* Sg = reinterpret_cast<__nv_bfloat16*>(ws.blk(tile) + ws.off_s);
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
-      const uint32_t lo = pack_bf16x2(X[nt][0], X[nt][1]);
-      const uint32_t hi = pack_bf16x2(X[nt][2], X[nt][3]);
-      if (to_operand) {
-        *reinterpret_cast<uint32_t*>(Sop + nt * nslab_bytes + rA * 16 + cA * 2) = lo;
-        *reinterpret_cast<uint32_t*>(Sop + nt * nslab_bytes + (rA + 8) * 16 + cA * 2) = hi;
-      }
+      const uint32_t lo = pack_bf16x2(S[nt][0], S[nt][1]);
+      const uint32_t hi = pack_bf16x2(S[nt][2], S[nt][3]);
+      *reinterpret_cast<uint32_t*>(Sop + nt * nslab_bytes + rA * 16 + cA * 2) = lo;
+      *reinterpret_cast<uint32_t*>(Sop + nt * nslab_bytes + (rA + 8) * 16 + cA * 2) = hi;
       const size_t slab = (size_t)(2 * slice + nt) * Dk;
       *reinterpret_cast<uint32_t*>(Sg + (slab + rA) * 8 + cA) = lo;
       *reinterpret_cast<uint32_t*>(Sg + (slab + rA + 8) * 8 + cA) = hi;
     }
   };
-  if (!odd) store_state(S, 0, true, chunk_tile(0));
+  publish(0, ws.tile(dir, bh, dir ? nC - 1 : 0));
 
   // ldmatrix row addresses (bytes in shared space) for this thread
   const int mi = lane >> 3, mr = lane & 7;
   // A: matrices (rows 0-7 | 8-15) x (k 0-7 | 8-15) of this warp's 16 rows
-  const uint32_t a_off = (uint32_t)((mi >> 1) * Dk * 16 + (16 * rw + (mi & 1) * 8 + mr) * 16);
+  const uint32_t a_off = (uint32_t)((mi >> 1) * Dk * 16 + (16 * warp + (mi & 1) * 8 + mr) * 16);
   // B (trans): matrices (k 0-7 | 8-15) x (n-slab 0 | 1)
   const uint32_t b_off = (uint32_t)((mi >> 1) * nslab_bytes + ((mi & 1) * 8 + mr) * 16);
   const uint32_t sop_u32 = smem_u32(Sop0), stage_u32 = smem_u32(stage0);
 
   bool ok = true;
-  int pi = 0;
-  for (; pi < nP; ++pi) {
-    const int st = pi % nstages;
-    if (tid == 0) ok = mbar_wait(&hd.full[st], (pi / nstages) & 1, limit);
+  int c = 0;
+  for (; c < nC; ++c) {
+    const int st = c % kRecStages;
+    if (tid == 0) ok = mbar_wait(&hd.full[st], (c / kRecStages) & 1, limit);
     if (!__syncthreads_and(ok)) break;  // S operand written, stage data visible
-    if (tid == 32 % blockDim.x && pi >= 1 && pi - 1 + nstages < nP) issue(pi - 1 + nstages);
-    if (pi >= 1 && pi - 1 + nstages < nP) issued = pi - 1 + nstages + 1;
-    const bool has_odd = 2 * pi + 1 < nC;
-    if (odd && !has_odd) continue;
-    const uint32_t qa = stage_u32 + st * stage_bytes + sub + a_off;
-    const uint32_t sb = sop_u32 + (pi & 1) * kRecSBytes + b_off;
+    if (tid == 32 % blockDim.x && c >= 1 && c - 1 + kRecStages < nC) issue(c - 1 + kRecStages);
+    if (c >= 1 && c - 1 + kRecStages < nC) issued = c - 1 + kRecStages + 1;
+    const uint32_t qa = stage_u32 + st * stage_bytes + a_off;
+    const uint32_t sb = sop_u32 + (c & 1) * kRecSBytes + b_off;
     float acc[2][4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
@@ -796,44 +650,29 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
       mma_16816(acc[0], af, bf[0], bf[1]);
       mma_16816(acc[1], af, bf[2], bf[3]);
     }
-    const uint8_t* stp = stage0 + st * stage_bytes + sub;
+    // S <- e^{gamma_C} S - Qc S + Rc
+    const uint8_t* stp = stage0 + st * stage_bytes;
     const float a = *reinterpret_cast<const float*>(stp + qbytes);
     const __nv_bfloat16* R = reinterpret_cast<const __nv_bfloat16*>(stp + qbytes + 16);
-    float X[2][4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
-      const __nv_bfloat162 r0 = *reinterpret_cast<const __nv_bfloat162*>(R + nt * Dk * 8 + rA * 8 + cA);
-      const __nv_bfloat162 r1 = *reinterpret_cast<const __nv_bfloat162*>(R + nt * Dk * 8 + (rA + 8) * 8 + cA);
-      float s0 = S[nt][0], s1 = S[nt][1], s2 = S[nt][2], s3 = S[nt][3];
-      if (odd) {  // the state S_{2p} from the bf16 operand
-        const uint8_t* Sop = Sop0 + (pi & 1) * kRecSBytes + nt * nslab_bytes;
-        const __nv_bfloat162 p0 = *reinterpret_cast<const __nv_bfloat162*>(Sop + rA * 16 + cA * 2);
-        const __nv_bfloat162 p1 = *reinterpret_cast<const __nv_bfloat162*>(Sop + (rA + 8) * 16 + cA * 2);
-        s0 = __low2float(p0); s1 = __high2float(p0); s2 = __low2float(p1); s3 = __high2float(p1);
-      }
-      X[nt][0] = fmaf(a, s0, __low2float(r0) - acc[nt][0]);
-      X[nt][1] = fmaf(a, s1, __high2float(r0) - acc[nt][1]);
-      X[nt][2] = fmaf(a, s2, __low2float(r1) - acc[nt][2]);
-      X[nt][3] = fmaf(a, s3, __high2float(r1) - acc[nt][3]);
+      const __nv_bfloat162 r0 = *reinterpret_cast<const __nv_bfloat162*>(R + rA * 16 + 8 * nt + cA);
+      const __nv_bfloat162 r1 = *reinterpret_cast<const __nv_bfloat162*>(R + (rA + 8) * 16 + 8 * nt + cA);
+      S[nt][0] = fmaf(a, S[nt][0], __low2float(r0) - acc[nt][0]);
+      S[nt][1] = fmaf(a, S[nt][1], __high2float(r0) - acc[nt][1]);
+      S[nt][2] = fmaf(a, S[nt][2], __low2float(r1) - acc[nt][2]);
+      S[nt][3] = fmaf(a, S[nt][3], __high2float(r1) - acc[nt][3]);
     }
-    if (odd) {
-      store_state(X, 0, false, chunk_tile(2 * pi + 1));
-    } else {
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) S[nt][i] = X[nt][i];
-      if (2 * pi + 2 < nC) store_state(S, (pi + 1) & 1, true, chunk_tile(2 * pi + 2));
-    }
+    if (c + 1 < nC) publish((c + 1) & 1, ws.tile(dir, bh, dir ? nC - 2 - c : c + 1));
   }
-  if (pi < nP) {  // a bounded wait expired: drain every load still in flight
+  if (c < nC) {  // a bounded wait expired: drain every load still in flight
     if (tid == 0) atomicOr(err, kErrTimeout);
-    for (int p2 = pi; p2 < issued; ++p2)
-      mbar_wait(&hd.full[p2 % nstages], (p2 / nstages) & 1, kDrainPolls);
+    for (int p = c; p < issued; ++p)
+      mbar_wait(&hd.full[p % kRecStages], (p / kRecStages) & 1, kDrainPolls);
     __syncthreads();
     return false;
   }
-  if (!odd && dir == 0 && state_out) {
+  if (dir == 0 && state_out) {
     float* base = state_out + (size_t)bh * Dk * Dv + 16 * slice;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
@@ -844,17 +683,17 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
   return true;
 }
 
-__global__ void __launch_bounds__(512, 1)
-gdn_recur_kernel(const float* state_in, float* state_out, Workspace ws, int nstages,
-                 long long limit, unsigned* err) {
+__global__ void __launch_bounds__(256, 1)
+gdn_recur_kernel(const float* state_in, float* state_out, Workspace ws, long long limit,
+                 unsigned* err) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   RecSmemHead& hd = *reinterpret_cast<RecSmemHead*>(smem_raw);
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kRecMaxStages; ++i) mbar_init(&hd.full[i], 1);
+    for (int i = 0; i < kRecStages; ++i) mbar_init(&hd.full[i], 1);
     fence_mbar_init();
   }
   __syncthreads();
-  recur_body(smem_raw, state_in, state_out, ws, nstages, limit, err);
+  recur_body(smem_raw, state_in, state_out, ws, limit, err);
 }
 
 // ========================================================== stage C: output
@@ -1190,20 +1029,9 @@ int num_sms() {
   return cached[dev];
 }
 
-constexpr int kMaxDynSmem = 227 * 1024;
-
-// Ring depth of stage B: as many stages (<= 4) as fit in shared memory.
-int recur_stages(int Dk) {
-  const int room = kMaxDynSmem - kRecHeadBytes - 2 * kRecSBytes;
-  return std::max(1, std::min(kRecMaxStages, room / (int)rec_stage_bytes(Dk)));
-}
 int recur_smem_bytes(int Dk) {
-  return kRecHeadBytes + 2 * kRecSBytes + recur_stages(Dk) * (int)rec_stage_bytes(Dk);
-}
-// Stage B0: head, two chunk summaries, and 2 KB so that the M = 128 product's
-// don't-care rows past Dk stay inside shared memory.
-int compose_smem_bytes(const Workspace& ws) {
-  return 128 + 2 * (int)((ws.off_w + 127) & ~127u) + 2048;
+  const int stage = ((Dk * Dk * 2 + Dk * 32 + 16) + 127) & ~127;
+  return kRecHeadBytes + 2 * kRecSBytes + kRecStages * stage;
 }
 
 // Opt the kernels into their dynamic shared memory, once per device.
@@ -1221,10 +1049,7 @@ cudaError_t set_smem_attrs() {
                            (int)sizeof(PrepSmem));
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(gdn_recur_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kMaxDynSmem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(gdn_compose_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kMaxDynSmem);
+                             recur_smem_bytes(128));
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(gdn_output_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)OutLayout(128, 128).total);
@@ -1235,11 +1060,10 @@ cudaError_t set_smem_attrs() {
 }  // namespace
 
 size_t chunk_tc_workspace_bytes(int B, int T, int H, int Dk, int Dv, bool bidir) {
-  const size_t nC = (T + kC - 1) / kC;
-  const size_t heads = (size_t)(bidir ? 2 : 1) * B * H;
+  const size_t tiles = (size_t)(bidir ? 2 : 1) * B * H * ((T + kC - 1) / kC);
   Workspace ws;
   ws.layout(Dk, Dv);
-  return heads * (nC * ws.block_bytes + ((nC + 1) / 2) * ws.pair_bytes);
+  return tiles * ws.block_bytes;
 }
 
 cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
@@ -1253,8 +1077,6 @@ cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
   ws.layout(a.Dk, a.Dv);
   ws.NBH = NBH;
   ws.nC = nC;
-  ws.nP = (nC + 1) / 2;
-  ws.pairs_off = (size_t)ndir * NBH * nC * ws.block_bytes;
 
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, a.q, a.B, a.T, a.H, a.Dk) || !make_map(&mk, a.k, a.B, a.T, a.H, a.Dk) ||
@@ -1269,17 +1091,9 @@ cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   {
-    ProfileScope ps(a.stream, kKernCompose);
-    gdn_compose_kernel<<<dim3(ws.nP, NBH, ndir), 128, compose_smem_bytes(ws), a.stream>>>(
-        ws, a.wait_limit, a.err);
-  }
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  {
     ProfileScope ps(a.stream, kKernRecur);
-    gdn_recur_kernel<<<dim3(a.Dv / 16, NBH, ndir), 2 * 32 * (a.Dk / 16), recur_smem_bytes(a.Dk),
-                       a.stream>>>(a.state_in, a.state_out, ws, recur_stages(a.Dk), a.wait_limit,
-                                   a.err);
+    gdn_recur_kernel<<<dim3(a.Dv / 16, NBH, ndir), 32 * (a.Dk / 16), recur_smem_bytes(a.Dk), a.stream>>>(
+        a.state_in, a.state_out, ws, a.wait_limit, a.err);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -1290,7 +1104,7 @@ cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
         mq, mk, a.g, static_cast<__nv_bfloat16*>(a.out), ws, a.T, a.H, ndir, a.wait_limit, a.err);
   }
   e = cudaGetLastError();
-  if (e == cudaSuccess) count_launches(4);
+  if (e == cudaSuccess) count_launches(3);
   return e;
 }
 

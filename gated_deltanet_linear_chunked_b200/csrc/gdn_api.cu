@@ -360,7 +360,6 @@ const char* gdn_kernel_name(int id) {
     case gdn::kKernPrep: return "gdn_prep_kernel";
     case gdn::kKernRecur: return "gdn_recur_kernel";
     case gdn::kKernOutput: return "gdn_output_kernel";
-    case gdn::kKernCompose: return "gdn_compose_kernel";
   }
   return "unknown";
 }

@@ -34,8 +34,7 @@ enum KernelId : int {
   kKernPrep = 1,
   kKernRecur = 2,
   kKernOutput = 3,
-  kKernCompose = 4,
-  kNumKernelIds = 5,
+  kNumKernelIds = 4,
 };
 
 // While profiling is armed, records CUDA events around one launch.

@@ -113,7 +113,7 @@ GDN_API gdn_status gdn_chunk_bidir(const void* q, const void* k, const void* v,
  * pool), or a process whose CUDA memory-pool API is unavailable or turned
  * off.  This entry point runs the same bf16 tensor-core kernels as
  * gdn_chunk_fwd but takes their scratch from one fixed array of
- * GDN_NOALLOC_SCRATCH_BYTES (128 MiB) that the library declares in device
+ * GDN_NOALLOC_SCRATCH_BYTES (96 MiB) that the library declares in device
  * memory; every GPU that loads the library holds that array until the process
  * exits.  It calls no cudaMalloc, cudaMallocAsync, cudaFree or other
  * allocating routine.
@@ -121,8 +121,8 @@ GDN_API gdn_status gdn_chunk_bidir(const void* q, const void* k, const void* v,
  * Arguments and layouts are those of gdn_chunk_fwd, with dtype GDN_BF16
  * only (other dtypes: GDN_ERR_UNSUPPORTED).  A problem whose scratch exceeds
  * the array returns GDN_ERR_SCRATCH_LIMIT and launches nothing.  The scratch
- * is about 130 KB per 64-token chunk of one head at Dk = Dv = 112, so about
- * 1030 chunk-heads (B * H * ceil(T / 64)) fit: the 2640-token x 20-head
+ * is about 104 KB per 64-token chunk of one head at Dk = Dv = 112, so about
+ * 960 chunk-heads (B * H * ceil(T / 64)) fit: the 2640-token x 20-head
  * streaming chunk (840) does, two of them in one call do not.
  *
  * The first call on a device looks up the array's device address
@@ -133,7 +133,7 @@ GDN_API gdn_status gdn_chunk_bidir(const void* q, const void* k, const void* v,
  * work overlaps on the GPU -- two streams, or two host threads -- race on it,
  * so order them on one stream.
  */
-#define GDN_NOALLOC_SCRATCH_BYTES (128ull << 20)
+#define GDN_NOALLOC_SCRATCH_BYTES (96ull << 20)
 GDN_API gdn_status gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
                                          const float* g, const float* beta,
                                          const float* state_in, float* state_out,
@@ -176,8 +176,8 @@ GDN_API unsigned long long gdn_launch_count(void);
  * launches, current device); gdn_profile_end synchronises the recorded
  * events, disarms, and writes for each kernel id i < nids the total
  * milliseconds ms[i] and launch count n[i].  Kernel ids: 0 token-serial scan,
- * 1 stage A (prep), 2 stage B (recurrence), 3 stage C (output), 4 chunk-pair
- * composition; names from gdn_kernel_name.  Not thread-safe against concurrent calls on other
+ * 1 stage A (prep), 2 stage B (recurrence), 3 stage C (output); names from
+ * gdn_kernel_name.  Not thread-safe against concurrent calls on other
  * threads; meant for benchmarks.
  */
 GDN_API gdn_status gdn_profile_begin(int max_launches);

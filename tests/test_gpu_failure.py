@@ -53,9 +53,9 @@ def test_profile_hook_counts_each_kernel():
     assert lib.gdn_profile_begin(16) == _lib.GDN_OK
     for _ in range(2):
         gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state_in"])
-    ms = (ctypes.c_float * 5)()
-    n = (ctypes.c_int * 5)()
-    assert lib.gdn_profile_end(ctypes.addressof(ms), ctypes.addressof(n), 5) == _lib.GDN_OK
-    assert list(n) == [0, 2, 2, 2, 2]
-    assert all(ms[i] > 0 for i in (1, 2, 3, 4))
+    ms = (ctypes.c_float * 4)()
+    n = (ctypes.c_int * 4)()
+    assert lib.gdn_profile_end(ctypes.addressof(ms), ctypes.addressof(n), 4) == _lib.GDN_OK
+    assert list(n) == [0, 2, 2, 2]
+    assert all(ms[i] > 0 for i in (1, 2, 3))
     assert lib.gdn_kernel_name(1).decode() == "gdn_prep_kernel"
