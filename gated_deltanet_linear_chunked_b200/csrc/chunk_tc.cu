@@ -40,6 +40,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <utility>
 
 #include "gdn_internal.h"
 #include "sm100.cuh"
@@ -413,34 +414,32 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
     const uint32_t lane_base = static_cast<uint32_t>(32 * quad) << 16;
     const size_t tile = ws.tile(dir, bh, j);
     const float sc = expf(gamC - s.gam[r]) * s.rn[r];
-    uint4* Wg = reinterpret_cast<uint4*>(ws.blk(tile) + ws.off_w);
-    uint4* Ug = reinterpret_cast<uint4*>(ws.blk(tile) + ws.off_ut);
-    for (int c = half; c < Dk / 16; c += 2) {
-      float v[16];
-      tmem_ld16(tm + lane_base + 16 * c, v);
+    // column block cb: W's blocks [0, Dk/16) at TMEM column 16 cb, then
+    // U~'s at 128 + 16 (cb - Dk/16); two TMEM loads in flight per wait
+    const int nkb = Dk / 16, nb = nkb + Dv / 16;
+    auto col = [&](int cb) { return cb < nkb ? 16u * cb : 128u + 16u * (cb - nkb); };
+    auto put = [&](int cb, const float* v) {
+      const bool isw = cb < nkb;
+      const int c = isw ? cb : cb - nkb;
+      uint4* G = reinterpret_cast<uint4*>(ws.blk(tile) + (isw ? ws.off_w : ws.off_ut));
+      uint8_t* Sp = isw ? s.u.b.Wp : s.u.b.Up;
+      float sv[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) sv[e] = v[e] * sc;
+      G[(2 * c) * kC + r] = pack8_bf16(v);
+      G[(2 * c + 1) * kC + r] = pack8_bf16(v + 8);
+      reinterpret_cast<uint4*>(Sp + (2 * c) * kSlab64)[r] = pack8_bf16(sv);
+      reinterpret_cast<uint4*>(Sp + (2 * c + 1) * kSlab64)[r] = pack8_bf16(sv + 8);
+    };
+    for (int cb = half; cb < nb; cb += 4) {
+      float v0[16], v1[16];
+      const bool two = cb + 2 < nb;
+      tmem_ld16(tm + lane_base + col(cb), v0);
+      if (two) tmem_ld16(tm + lane_base + col(cb + 2), v1);
       tmem_wait_ld();
       if (lane < 16) {
-        float sv[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) sv[e] = v[e] * sc;
-        Wg[(2 * c) * kC + r] = pack8_bf16(v);
-        Wg[(2 * c + 1) * kC + r] = pack8_bf16(v + 8);
-        reinterpret_cast<uint4*>(s.u.b.Wp + (2 * c) * kSlab64)[r] = pack8_bf16(sv);
-        reinterpret_cast<uint4*>(s.u.b.Wp + (2 * c + 1) * kSlab64)[r] = pack8_bf16(sv + 8);
-      }
-    }
-    for (int c = half; c < Dv / 16; c += 2) {
-      float v[16];
-      tmem_ld16(tm + lane_base + 128 + 16 * c, v);
-      tmem_wait_ld();
-      if (lane < 16) {
-        float sv[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) sv[e] = v[e] * sc;
-        Ug[(2 * c) * kC + r] = pack8_bf16(v);
-        Ug[(2 * c + 1) * kC + r] = pack8_bf16(v + 8);
-        reinterpret_cast<uint4*>(s.u.b.Up + (2 * c) * kSlab64)[r] = pack8_bf16(sv);
-        reinterpret_cast<uint4*>(s.u.b.Up + (2 * c + 1) * kSlab64)[r] = pack8_bf16(sv + 8);
+        put(cb, v0);
+        if (two) put(cb + 2, v1);
       }
     }
   }
@@ -467,22 +466,28 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
     const size_t tile = ws.tile(dir, bh, j);
     uint4* Qg = reinterpret_cast<uint4*>(ws.blk(tile));
     uint4* Rg = reinterpret_cast<uint4*>(ws.blk(tile) + ws.off_rc);
-    for (int c = half; c < Dk / 16; c += 2) {
-      float v[16];
-      tmem_ld16(tm + lane_base + 16 * c, v);
-      tmem_wait_ld();
-      if (r < Dk) {
-        Qg[(2 * c) * Dk + r] = pack8_bf16(v);
-        Qg[(2 * c + 1) * Dk + r] = pack8_bf16(v + 8);
-      }
-    }
-    for (int c = half; c < Dv / 16; c += 2) {
-      float v[16];
-      tmem_ld16(tm + lane_base + 128 + 16 * c, v);
-      tmem_wait_ld();
-      if (r < Dk) {
+    // column block cb: Qc's [0, Dk/16) at 16 cb, Rc's at 128 + 16 (cb - Dk/16)
+    const int nkb = Dk / 16, nb = nkb + Dv / 16;
+    auto col = [&](int cb) { return cb < nkb ? 16u * cb : 128u + 16u * (cb - nkb); };
+    auto put = [&](int cb, const float* v) {
+      if (cb < nkb) {
+        Qg[(2 * cb) * Dk + r] = pack8_bf16(v);
+        Qg[(2 * cb + 1) * Dk + r] = pack8_bf16(v + 8);
+      } else {
+        const int c = cb - nkb;
         Rg[(c * Dk + r) * 2] = pack8_bf16(v);
         Rg[(c * Dk + r) * 2 + 1] = pack8_bf16(v + 8);
+      }
+    };
+    for (int cb = half; cb < nb; cb += 4) {
+      float v0[16], v1[16];
+      const bool two = cb + 2 < nb;
+      tmem_ld16(tm + lane_base + col(cb), v0);
+      if (two) tmem_ld16(tm + lane_base + col(cb + 2), v1);
+      tmem_wait_ld();
+      if (r < Dk) {
+        put(cb, v0);
+        if (two) put(cb + 2, v1);
       }
     }
     if (tid == 0)
@@ -512,6 +517,10 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     for (int i = tid; i < (16 - ws.Dk / 8) * kSlab64 / 16; i += kWideThreads) z[i] = make_uint4(0, 0, 0, 0);
   }
   block_sync_async();
+  // Programmatic dependent launch: everything above overlaps the previous
+  // kernel in the stream; nothing in global memory is touched before this.
+  pdl_wait();
+  pdl_trigger();
   if (blockIdx.z == 0)
     prep_body<0>(s, &tm_k, &tm_v, g, beta, ws, T, H, limit, err);
   else
@@ -601,23 +610,21 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
     for (int c = 0; c < issued; ++c) issue(c);
 
   // S (bf16) of this thread's accumulator positions -> operand buffer `buf`
-  // ([n-slab][Dk rows][8]) and, for stage C, the workspace copy of the state
-  // at the start of chunk `jt` ([Dv/8][Dk][8]).
-  auto publish = [&](int buf, size_t tile) {
+  // ([n-slab][Dk rows][8]).  Its two n-slabs are exactly this slice's part of
+  // the workspace copy of the chunk-start state ([Dv/8][Dk][8]), which one
+  // thread then writes with a single bulk store after the next barrier.
+  auto publish = [&](int buf) {
     uint8_t* Sop = Sop0 + buf * kRecSBytes;
-    __nv_bfloat16* Sg = reinterpret_cast<__nv_bfloat16*>(ws.blk(tile) + ws.off_s);
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
-      const uint32_t lo = pack_bf16x2(S[nt][0], S[nt][1]);
-      const uint32_t hi = pack_bf16x2(S[nt][2], S[nt][3]);
-      *reinterpret_cast<uint32_t*>(Sop + nt * nslab_bytes + rA * 16 + cA * 2) = lo;
-      *reinterpret_cast<uint32_t*>(Sop + nt * nslab_bytes + (rA + 8) * 16 + cA * 2) = hi;
-      const size_t slab = (size_t)(2 * slice + nt) * Dk;
-      *reinterpret_cast<uint32_t*>(Sg + (slab + rA) * 8 + cA) = lo;
-      *reinterpret_cast<uint32_t*>(Sg + (slab + rA + 8) * 8 + cA) = hi;
+      *reinterpret_cast<uint32_t*>(Sop + nt * nslab_bytes + rA * 16 + cA * 2) =
+          pack_bf16x2(S[nt][0], S[nt][1]);
+      *reinterpret_cast<uint32_t*>(Sop + nt * nslab_bytes + (rA + 8) * 16 + cA * 2) =
+          pack_bf16x2(S[nt][2], S[nt][3]);
     }
   };
-  publish(0, ws.tile(dir, bh, dir ? nC - 1 : 0));
+  const int storer = blockDim.x > 64 ? 64 : 0;
+  publish(0);
 
   // ldmatrix row addresses (bytes in shared space) for this thread
   const int mi = lane >> 3, mr = lane & 7;
@@ -632,7 +639,13 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
   for (; c < nC; ++c) {
     const int st = c % kRecStages;
     if (tid == 0) ok = mbar_wait(&hd.full[st], (c / kRecStages) & 1, limit);
+    if (tid == storer) bulk_wait_read();  // last store done reading the buffer we reuse
+    fence_proxy_async_smem();             // operand writes -> the bulk store
     if (!__syncthreads_and(ok)) break;  // S operand written, stage data visible
+    if (tid == storer)
+      bulk_store(ws.blk(ws.tile(dir, bh, dir ? nC - 1 - c : c)) + ws.off_s +
+                     (size_t)slice * 2 * nslab_bytes,
+                 Sop0 + (c & 1) * kRecSBytes, 2 * nslab_bytes);
     if (tid == 32 % blockDim.x && c >= 1 && c - 1 + kRecStages < nC) issue(c - 1 + kRecStages);
     if (c >= 1 && c - 1 + kRecStages < nC) issued = c - 1 + kRecStages + 1;
     const uint32_t qa = stage_u32 + st * stage_bytes + a_off;
@@ -663,8 +676,9 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
       S[nt][2] = fmaf(a, S[nt][2], __low2float(r1) - acc[nt][2]);
       S[nt][3] = fmaf(a, S[nt][3], __high2float(r1) - acc[nt][3]);
     }
-    if (c + 1 < nC) publish((c + 1) & 1, ws.tile(dir, bh, dir ? nC - 2 - c : c + 1));
+    if (c + 1 < nC) publish((c + 1) & 1);
   }
+  if (tid == storer) bulk_wait_all();
   if (c < nC) {  // a bounded wait expired: drain every load still in flight
     if (tid == 0) atomicOr(err, kErrTimeout);
     for (int p = c; p < issued; ++p)
@@ -693,6 +707,8 @@ gdn_recur_kernel(const float* state_in, float* state_out, Workspace ws, long lon
     fence_mbar_init();
   }
   __syncthreads();
+  pdl_wait();  // stage A's summaries are complete and visible
+  pdl_trigger();
   recur_body(smem_raw, state_in, state_out, ws, limit, err);
 }
 
@@ -864,27 +880,31 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
       }
       mma_ph ^= 1;
       tc_fence_after_sync();
-      // U = U~ - W S, in place of U~ (MN-major B: [slab][64 tokens][8])
-      for (int c = part; c < Dv / 16; c += 4) {
-        float v[16];
-        tmem_ld16(tmU + lane_base + 16 * c, v);
+      // U = U~ - W S, in place of U~ (MN-major B: [slab][64 tokens][8]);
+      // column blocks part and part + 4 of D_U and block part of P are
+      // loaded from TMEM together
+      {
+        float u0[16], u1[16], v[16];
+        const bool has1 = part + 4 < Dv / 16;
+        if (part < Dv / 16) tmem_ld16(tmU + lane_base + 16 * part, u0);
+        if (has1) tmem_ld16(tmU + lane_base + 16 * (part + 4), u1);
+        tmem_ld16(tmP + lane_base + 16 * part, v);
         tmem_wait_ld();
-        if (lane < 16) {
+        auto sub = [&](int c, const float* d) {
           float ut[16];
           unpack8_bf16(reinterpret_cast<const uint4*>(sUt + (2 * c) * kSlab64)[r], ut);
           unpack8_bf16(reinterpret_cast<const uint4*>(sUt + (2 * c + 1) * kSlab64)[r], ut + 8);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) ut[e] -= v[e];
+          for (int e = 0; e < 16; ++e) ut[e] -= d[e];
           reinterpret_cast<uint4*>(sUt + (2 * c) * kSlab64)[r] = pack8_bf16(ut);
           reinterpret_cast<uint4*>(sUt + (2 * c + 1) * kSlab64)[r] = pack8_bf16(ut + 8);
+        };
+        if (lane < 16) {
+          if (part < Dv / 16) sub(part, u0);
+          if (has1) sub(part + 4, u1);
         }
-      }
-      // P'_ri = (q_r . k_i) / |k_i| * e^{gam_r - gam_i} for i at or before r
-      {
+        // P'_ri = (q_r . k_i) / |k_i| * e^{gam_r - gam_i} for i at or before r
         const int c = part;
-        float v[16];
-        tmem_ld16(tmP + lane_base + 16 * c, v);
-        tmem_wait_ld();
         if (lane < 16) {
           const float ar = sm.arow[r];
           const float* bc = sm.bcol[(dir ? 63 - r : r) >> 3];
@@ -931,17 +951,21 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
     // O = diag(1/|q|) D_O -> out (rows of this chunk that exist)
     {
       const float rq = sm.rnq[r];
-      for (int c = part; c < Dv / 16; c += 4) {
-        float v[16];
-        tmem_ld16(tmO + lane_base + 16 * c, v);
-        tmem_wait_ld();
-        if (lane < 16 && r < nvalid) {
+      float v0[16], v1[16];
+      const bool has1 = part + 4 < Dv / 16;
+      if (part < Dv / 16) tmem_ld16(tmO + lane_base + 16 * part, v0);
+      if (has1) tmem_ld16(tmO + lane_base + 16 * (part + 4), v1);
+      tmem_wait_ld();
+      auto put = [&](int c, float* v) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) v[e] *= rq;
-          uint4* o = reinterpret_cast<uint4*>(out + (((size_t)b * T + t0 + r) * H + h) * Dv + 16 * c);
-          o[0] = pack8_bf16(v);
-          o[1] = pack8_bf16(v + 8);
-        }
+        for (int e = 0; e < 16; ++e) v[e] *= rq;
+        uint4* o = reinterpret_cast<uint4*>(out + (((size_t)b * T + t0 + r) * H + h) * Dv + 16 * c);
+        o[0] = pack8_bf16(v);
+        o[1] = pack8_bf16(v + 8);
+      };
+      if (lane < 16 && r < nvalid) {
+        if (part < Dv / 16) put(part, v0);
+        if (has1) put(part + 4, v1);
       }
     }
     tc_fence_before_sync();
@@ -974,6 +998,8 @@ gdn_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     tmem_relinquish();
   }
   block_sync_async();
+  pdl_wait();  // stage B's chunk-start states are complete and visible
+  pdl_trigger();
   output_body(smem_raw, &tm_q, &tm_k, g, out, ws, T, H, ndir, limit, err);
   tc_fence_before_sync();
   __syncthreads();
@@ -1057,6 +1083,25 @@ cudaError_t set_smem_attrs() {
   return e;
 }
 
+// Launch with programmatic stream serialisation: the kernel may start while
+// the previous kernel in the stream drains; each kernel of this path calls
+// griddepcontrol.wait before its first global-memory access.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 }  // namespace
 
 size_t chunk_tc_workspace_bytes(int B, int T, int H, int Dk, int Dv, bool bidir) {
@@ -1085,25 +1130,23 @@ cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
 
   {
     ProfileScope ps(a.stream, kKernPrep);
-    gdn_prep_kernel<<<dim3(nC, NBH, ndir), kWideThreads, sizeof(PrepSmem), a.stream>>>(
-        mk, mv, a.g, a.beta, ws, a.T, a.H, a.wait_limit, a.err);
+    e = launch_pdl(gdn_prep_kernel, dim3(nC, NBH, ndir), kWideThreads, sizeof(PrepSmem), a.stream,
+                   mk, mv, a.g, a.beta, ws, a.T, a.H, a.wait_limit, a.err);
   }
-  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   {
     ProfileScope ps(a.stream, kKernRecur);
-    gdn_recur_kernel<<<dim3(a.Dv / 16, NBH, ndir), 32 * (a.Dk / 16), recur_smem_bytes(a.Dk), a.stream>>>(
-        a.state_in, a.state_out, ws, a.wait_limit, a.err);
+    e = launch_pdl(gdn_recur_kernel, dim3(a.Dv / 16, NBH, ndir), 32 * (a.Dk / 16),
+                   recur_smem_bytes(a.Dk), a.stream, a.state_in, a.state_out, ws, a.wait_limit,
+                   a.err);
   }
-  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   {
     ProfileScope ps(a.stream, kKernOutput);
-    gdn_output_kernel<<<dim3(std::min(nC * NBH, num_sms())), kOutThreads,
-                        OutLayout(a.Dk, a.Dv).total, a.stream>>>(
-        mq, mk, a.g, static_cast<__nv_bfloat16*>(a.out), ws, a.T, a.H, ndir, a.wait_limit, a.err);
+    e = launch_pdl(gdn_output_kernel, dim3(std::min(nC * NBH, num_sms())), kOutThreads,
+                   OutLayout(a.Dk, a.Dv).total, a.stream, mq, mk, a.g,
+                   static_cast<__nv_bfloat16*>(a.out), ws, a.T, a.H, ndir, a.wait_limit, a.err);
   }
-  e = cudaGetLastError();
   if (e == cudaSuccess) count_launches(3);
   return e;
 }
