@@ -567,6 +567,9 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// NKS = Dk / 16, a compile-time constant so that the per-chunk code is
+// straight-line.
+template <int NKS>
 __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_out,
                            const Workspace& ws, long long limit, unsigned* err) {
   RecSmemHead& hd = *reinterpret_cast<RecSmemHead*>(smem);
@@ -578,7 +581,6 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
   const uint32_t stage_bytes = (qbytes + rbytes + 16 + 127) & ~127u;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int slice = blockIdx.x, bh = blockIdx.y, dir = blockIdx.z;
-  const int nks = Dk / 16;
   // accumulator coordinates of this thread: rows rA, rA + 8; columns cA, cA + 1 (+ 8 nt)
   const int rA = 16 * warp + (lane >> 2), cA = 2 * (lane & 3);
 
@@ -634,11 +636,39 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
   const uint32_t b_off = (uint32_t)((mi >> 1) * nslab_bytes + ((mi & 1) * 8 + mr) * 16);
   const uint32_t sop_u32 = smem_u32(Sop0), stage_u32 = smem_u32(stage0);
 
-  bool ok = true;
+  // Software pipeline: the A fragments of Qc, the decay and the Rc slice of
+  // chunk c + 1 are read into registers while chunk c's MMAs run, and
+  // X = e^{gamma_C} S + Rc is formed before the product arrives, so the
+  // dependent path per chunk is: barrier, B fragments, MMA, S = X - Qc S,
+  // operand write.
+  uint32_t af[NKS][4];
+  float X[2][4];
+  // wait for chunk c's stage (every thread), then read its A fragments and
+  // form X from the current S
+  auto prefetch = [&](int cc) -> bool {
+    const int st = cc % kRecStages;
+    const bool okw = mbar_wait(&hd.full[st], (cc / kRecStages) & 1, limit);
+    const uint32_t qa = stage_u32 + st * stage_bytes + a_off;
+#pragma unroll
+    for (int ks = 0; ks < NKS; ++ks) ldmatrix_x4(qa + ks * 2 * Dk * 16, af[ks]);
+    const uint8_t* stp = stage0 + st * stage_bytes;
+    const float a = *reinterpret_cast<const float*>(stp + qbytes);
+    const __nv_bfloat16* R = reinterpret_cast<const __nv_bfloat16*>(stp + qbytes + 16);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const __nv_bfloat162 r0 = *reinterpret_cast<const __nv_bfloat162*>(R + rA * 16 + 8 * nt + cA);
+      const __nv_bfloat162 r1 = *reinterpret_cast<const __nv_bfloat162*>(R + (rA + 8) * 16 + 8 * nt + cA);
+      X[nt][0] = fmaf(a, S[nt][0], __low2float(r0));
+      X[nt][1] = fmaf(a, S[nt][1], __high2float(r0));
+      X[nt][2] = fmaf(a, S[nt][2], __low2float(r1));
+      X[nt][3] = fmaf(a, S[nt][3], __high2float(r1));
+    }
+    return okw;
+  };
+
+  bool ok = prefetch(0);
   int c = 0;
   for (; c < nC; ++c) {
-    const int st = c % kRecStages;
-    if (tid == 0) ok = mbar_wait(&hd.full[st], (c / kRecStages) & 1, limit);
     if (tid == storer) bulk_wait_read();  // last store done reading the buffer we reuse
     fence_proxy_async_smem();             // operand writes -> the bulk store
     if (!__syncthreads_and(ok)) break;  // S operand written, stage data visible
@@ -648,35 +678,32 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
                  Sop0 + (c & 1) * kRecSBytes, 2 * nslab_bytes);
     if (tid == 32 % blockDim.x && c >= 1 && c - 1 + kRecStages < nC) issue(c - 1 + kRecStages);
     if (c >= 1 && c - 1 + kRecStages < nC) issued = c - 1 + kRecStages + 1;
-    const uint32_t qa = stage_u32 + st * stage_bytes + a_off;
     const uint32_t sb = sop_u32 + (c & 1) * kRecSBytes + b_off;
-    float acc[2][4];
+    uint32_t bfr[NKS][4];
+#pragma unroll
+    for (int ks = 0; ks < NKS; ++ks) ldmatrix_x4_trans(sb + ks * 256, bfr[ks]);
+    // two independent accumulator chains per n-tile (even / odd k-steps)
+    float acc[2][2][4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[h][nt][i] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < NKS; ++ks) {
+      mma_16816(acc[ks & 1][0], af[ks], bfr[ks][0], bfr[ks][1]);
+      mma_16816(acc[ks & 1][1], af[ks], bfr[ks][2], bfr[ks][3]);
+    }
+    // S <- (e^{gamma_C} S + Rc) - Qc S
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
-#pragma unroll 8
-    for (int ks = 0; ks < nks; ++ks) {
-      uint32_t af[4], bf[4];
-      ldmatrix_x4(qa + ks * 2 * Dk * 16, af);
-      ldmatrix_x4_trans(sb + ks * 256, bf);
-      mma_16816(acc[0], af, bf[0], bf[1]);
-      mma_16816(acc[1], af, bf[2], bf[3]);
+      for (int i = 0; i < 4; ++i) S[nt][i] = X[nt][i] - (acc[0][nt][i] + acc[1][nt][i]);
+    if (c + 1 < nC) {
+      publish((c + 1) & 1);
+      ok = prefetch(c + 1);
     }
-    // S <- e^{gamma_C} S - Qc S + Rc
-    const uint8_t* stp = stage0 + st * stage_bytes;
-    const float a = *reinterpret_cast<const float*>(stp + qbytes);
-    const __nv_bfloat16* R = reinterpret_cast<const __nv_bfloat16*>(stp + qbytes + 16);
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      const __nv_bfloat162 r0 = *reinterpret_cast<const __nv_bfloat162*>(R + rA * 16 + 8 * nt + cA);
-      const __nv_bfloat162 r1 = *reinterpret_cast<const __nv_bfloat162*>(R + (rA + 8) * 16 + 8 * nt + cA);
-      S[nt][0] = fmaf(a, S[nt][0], __low2float(r0) - acc[nt][0]);
-      S[nt][1] = fmaf(a, S[nt][1], __high2float(r0) - acc[nt][1]);
-      S[nt][2] = fmaf(a, S[nt][2], __low2float(r1) - acc[nt][2]);
-      S[nt][3] = fmaf(a, S[nt][3], __high2float(r1) - acc[nt][3]);
-    }
-    if (c + 1 < nC) publish((c + 1) & 1);
   }
   if (tid == storer) bulk_wait_all();
   if (c < nC) {  // a bounded wait expired: drain every load still in flight
@@ -697,6 +724,7 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
   return true;
 }
 
+template <int NKS>
 __global__ void __launch_bounds__(256, 1)
 gdn_recur_kernel(const float* state_in, float* state_out, Workspace ws, long long limit,
                  unsigned* err) {
@@ -709,7 +737,22 @@ gdn_recur_kernel(const float* state_in, float* state_out, Workspace ws, long lon
   __syncthreads();
   pdl_wait();  // stage A's summaries are complete and visible
   pdl_trigger();
-  recur_body(smem_raw, state_in, state_out, ws, limit, err);
+  recur_body<NKS>(smem_raw, state_in, state_out, ws, limit, err);
+}
+
+// The recurrence kernel for Dk = 16 * nks.
+using RecurKernel = void (*)(const float*, float*, Workspace, long long, unsigned*);
+RecurKernel recur_kernel(int nks) {
+  switch (nks) {
+    case 1: return gdn_recur_kernel<1>;
+    case 2: return gdn_recur_kernel<2>;
+    case 3: return gdn_recur_kernel<3>;
+    case 4: return gdn_recur_kernel<4>;
+    case 5: return gdn_recur_kernel<5>;
+    case 6: return gdn_recur_kernel<6>;
+    case 7: return gdn_recur_kernel<7>;
+    default: return gdn_recur_kernel<8>;
+  }
 }
 
 // ========================================================== stage C: output
@@ -1074,8 +1117,9 @@ cudaError_t set_smem_attrs() {
   e = cudaFuncSetAttribute(gdn_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)sizeof(PrepSmem));
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(gdn_recur_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             recur_smem_bytes(128));
+    for (int nks = 1; nks <= 8 && e == cudaSuccess; ++nks)
+      e = cudaFuncSetAttribute(recur_kernel(nks), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               recur_smem_bytes(128));
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(gdn_output_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)OutLayout(128, 128).total);
@@ -1136,7 +1180,7 @@ cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
   if (e != cudaSuccess) return e;
   {
     ProfileScope ps(a.stream, kKernRecur);
-    e = launch_pdl(gdn_recur_kernel, dim3(a.Dv / 16, NBH, ndir), 32 * (a.Dk / 16),
+    e = launch_pdl(recur_kernel(a.Dk / 16), dim3(a.Dv / 16, NBH, ndir), 32 * (a.Dk / 16),
                    recur_smem_bytes(a.Dk), a.stream, a.state_in, a.state_out, ws, a.wait_limit,
                    a.err);
   }
