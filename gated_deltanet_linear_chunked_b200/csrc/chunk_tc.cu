@@ -128,15 +128,19 @@ __device__ void warp_gamma(const float* g, float* gam, int reverse) {
   gam[r1] = incl;
 }
 
-// 1 / max(|row|, 1e-6) for a 64-row bf16 tile in [slab][64][8] layout.
-__device__ float row_rnorm(const uint8_t* tile, int r, int D) {
+// 1 / max(|row r|, 1e-6) for a 64-row bf16 tile in [slab][64][8] layout,
+// by four consecutive lanes (part = lane & 3 takes slabs part, part + 4, ...);
+// every lane of the four gets the result.
+__device__ float row_rnorm4(const uint8_t* tile, int r, int part, int D) {
   float ss = 0.f;
-  for (int sl = 0; sl < D / 8; ++sl) {
+  for (int sl = part; sl < D / 8; sl += 4) {
     float x[8];
     unpack8_bf16(reinterpret_cast<const uint4*>(tile + sl * kSlab64)[r], x);
 #pragma unroll
     for (int i = 0; i < 8; ++i) ss = fmaf(x[i], x[i], ss);
   }
+  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 2);
   return 1.0f / sqrtf(fmaxf(ss, 1e-12f));
 }
 
@@ -164,7 +168,7 @@ struct PrepSmem {
   float g[64], beta[64], gam[64], rn[64], csW[64], csU[64];
   float arow[64];      // beta_r |k_r|^-1 e^{gam_r - m_b(r)}       (scan order)
   float bcol[8][64];   // |k_q|^-1 e^{m_b - gam_q}, b = 8-row block (scan order)
-  uint64_t tma_bar, mma_bar;
+  uint64_t tma_bar, v_bar, mma_bar;  // K tile, V tile, MMA completion
   uint32_t tmem;
 };
 
@@ -283,9 +287,10 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
   const uint32_t tm = s.tmem;
 
   if (tid == 0) {
-    mbar_arrive_expect_tx(&s.tma_bar, (Dk / 8 + Dv / 8) * kSlab64);
+    mbar_arrive_expect_tx(&s.tma_bar, (Dk / 8) * kSlab64);
+    mbar_arrive_expect_tx(&s.v_bar, (Dv / 8) * kSlab64);
     tma_load_tile(s.K, tm_k, &s.tma_bar, t0, h, b);
-    tma_load_tile(s.V, tm_v, &s.tma_bar, t0, h, b);
+    tma_load_tile(s.V, tm_v, &s.v_bar, t0, h, b);
   }
   if (tid < kC) {
     float gv = 0.f, bv = 0.f;  // padding rows: a = 1, beta = 0 (no effect)
@@ -299,10 +304,15 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
   }
   __syncthreads();
   if (warp == 0) warp_gamma(s.g, s.gam, REV);
-  if (!block_wait(&s.tma_bar, 0, limit, err)) return false;
+  // V is awaited only before W / U~; a failure before that drains it too
+  auto drain_v = [&]() { mbar_wait(&s.v_bar, 0, kDrainPolls); };
+  if (!block_wait(&s.tma_bar, 0, limit, err)) {
+    drain_v();
+    return false;
+  }
 
-  if (tid < kC) s.rn[tid] = row_rnorm(s.K, tid, Dk);
-  // G = K K^T  (M = 64 tokens, N = 64 tokens, K = Dk), raw (unnormalised) keys
+  // G = K K^T  (M = 64 tokens, N = 64 tokens, K = Dk), raw (unnormalised)
+  // keys; the row norms below overlap it
   if (tid == 0) {
     tc_fence_after_sync();
     const uint32_t id = idesc_bf16(64, 64, 0, 0);
@@ -312,13 +322,20 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
     }
     mma_commit(&s.mma_bar);
   }
+  {
+    const float rn = row_rnorm4(s.K, tid >> 2, tid & 3, Dk);
+    if ((tid & 3) == 0) s.rn[tid >> 2] = rn;
+  }
   __syncthreads();
   const float gamC = REV ? s.gam[0] : s.gam[63];
   if (tid < kC) {
     s.csW[tid] = s.beta[tid] * expf(s.gam[tid]) * s.rn[tid];
     s.csU[tid] = s.beta[tid];
   }
-  if (!block_wait(&s.mma_bar, 0, limit, err)) return false;
+  if (!block_wait(&s.mma_bar, 0, limit, err)) {
+    drain_v();
+    return false;
+  }
   tc_fence_after_sync();
 
   // A[p][q] = beta_r e^{gam_r - gam_i} G_ri / (|k_r| |k_i|) for scan positions
@@ -390,6 +407,7 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
     reinterpret_cast<uint4*>(s.u.a.TU + ks * kSlab64)[r] = pack8_bf16(uu);
   }
   block_sync_async();
+  if (!block_wait(&s.v_bar, 0, limit, err)) return false;
   // W = TW K (N = Dk), U~ = TU V (N = Dv); K and V read MN-major (N = feature)
   if (tid == 0) {
     const uint32_t idW = idesc_bf16(64, Dk, 0, 1), idU = idesc_bf16(64, Dv, 0, 1);
@@ -444,6 +462,7 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
     }
   }
   block_sync_async();
+  const size_t tile = ws.tile(dir, bh, j);
   // Qc = K^T Wp (M = 128 >= Dk, N = Dk), Rc = K^T Up (N = Dv); K read MN-major
   // as A (M = feature; slabs >= Dk/8 are zero rows)
   if (tid == 0) {
@@ -463,7 +482,7 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
     const int quad = warp & 3, half = warp >> 2;
     const int r = 32 * quad + lane;  // TMEM lane = feature row of Qc / Rc
     const uint32_t lane_base = static_cast<uint32_t>(32 * quad) << 16;
-    const size_t tile = ws.tile(dir, bh, j);
+    // Qc | decay | Rc staged in the workspace block's own layout
     uint4* Qg = reinterpret_cast<uint4*>(ws.blk(tile));
     uint4* Rg = reinterpret_cast<uint4*>(ws.blk(tile) + ws.off_rc);
     // column block cb: Qc's [0, Dk/16) at 16 cb, Rc's at 128 + 16 (cb - Dk/16)
@@ -505,6 +524,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
   const int tid = threadIdx.x;
   if (tid == 0) {
     mbar_init(&s.tma_bar, 1);
+    mbar_init(&s.v_bar, 1);
     mbar_init(&s.mma_bar, 1);
     fence_mbar_init();
   }
@@ -874,8 +894,19 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
       return false;
     }
     tma_ph ^= 1u << set;
-    if (tid < kC) sm.rnq[tid] = row_rnorm(sQ, tid, Dk);
-    else if (tid < 2 * kC) sm.rnk[tid - kC] = row_rnorm(sK, tid - kC, Dk);
+    if (tid == 0) {  // P = Q K^T, shared by both directions; overlaps the norms
+      tc_fence_after_sync();
+      const uint32_t idP = idesc_bf16(64, 64, 0, 0);
+      for (int ks = 0; ks < Dk / 16; ++ks)
+        mma_bf16(tmP, sdesc(smem_u32(sQ) + ks * 2 * kSlab64, kSlab64, 128),
+                 sdesc(smem_u32(sK) + ks * 2 * kSlab64, kSlab64, 128), idP, ks > 0);
+    }
+    {  // 1 / |q|, 1 / |k| per row: four threads per row and tensor
+      const int row = tid >> 3, part = tid & 3;
+      const bool isk = (tid >> 2) & 1;
+      const float rn = row_rnorm4(isk ? sK : sQ, row, part, Dk);
+      if (part == 0) (isk ? sm.rnk : sm.rnq)[row] = rn;
+    }
     for (int dir = 0; dir < ndir; ++dir) {
       // D_U: direction 0 borrows D_O's columns (D_O is first written after
       // D_U is consumed); direction 1 needs its own, [192, 320) of a
@@ -904,12 +935,6 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
       ld_ph ^= 1u << set;
       if (tid == 0) {
         tc_fence_after_sync();
-        if (dir == 0) {  // P = Q K^T, shared by both directions
-          const uint32_t idP = idesc_bf16(64, 64, 0, 0);
-          for (int ks = 0; ks < Dk / 16; ++ks)
-            mma_bf16(tmP, sdesc(smem_u32(sQ) + ks * 2 * kSlab64, kSlab64, 128),
-                     sdesc(smem_u32(sK) + ks * 2 * kSlab64, kSlab64, 128), idP, ks > 0);
-        }
         // D_U = W S  (M = 64, N = Dv, K = Dk); S read MN-major (N = value column)
         const uint32_t idU = idesc_bf16(64, Dv, 0, 1);
         for (int ks = 0; ks < Dk / 16; ++ks)
