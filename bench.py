@@ -215,6 +215,31 @@ def cpu_baseline(w, budget_s: float):
                       f"{reps} repetitions in {el:.1f} s"}
 
 
+# ---- multi-rank plumbing (one process per GPU; no data-path collective)
+def rank_workload(w, rank: int):
+    """The chunk stream rank `rank` scans: the same shapes and distributions
+    as `w`, its own seed, so ranks process independent streams."""
+    from gated_deltanet_linear_chunked_b200 import workloads as wl
+    return wl.stream_chunk(w.mode, seed=w.seed + 7919 * rank)
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The largest of every rank's `x` (device times are reported as the
+    slowest rank's)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, steps: int, head_tokens: int, ms: float) -> float:
+    """Whole-job head-tokens/s: every rank's units over the slowest rank's time."""
+    return world * steps * head_tokens / (ms / 1000.0)
+
+
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -286,7 +311,7 @@ def main():
     fn = gdn.chunk_bidir if w.mode == "bidir" else gdn.chunk_fwd
 
     # ---- inputs: one seeded chunk per rank, copied into N_SETS rotating sets
-    w_r = wl.stream_chunk(w.mode, seed=w.seed + 7919 * rank)
+    w_r = rank_workload(w, rank)
     xh = wl.make_inputs(w_r)
     dt = torch.bfloat16
     base = {n: torch.from_numpy(xh[n]).to(dev) for n in ("q", "k", "v", "g", "beta")}
@@ -349,13 +374,9 @@ def main():
         run_steps(args.steps)
         ev1.record(stream)
         barrier()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     ms_per_step = ms / args.steps
-    value = world * args.steps * w.head_tokens / (ms / 1000.0)
+    value = job_throughput(world, args.steps, w.head_tokens, ms)
 
     # ---- end to end through the public API: pinned host -> device, call, device -> host
     e2e_steps = max(3, min(args.steps, 200))
@@ -385,12 +406,8 @@ def main():
             e2e_step(i)
         e1.record(stream)
     barrier()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * e2e_steps * w.head_tokens / (e2e_ms / 1000.0)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = job_throughput(world, e2e_steps, w.head_tokens, e2e_ms)
 
     # ---- side figures: the other mode, and the 15-layer stacked stream
     extras = {}
