@@ -378,33 +378,52 @@ def main():
     ms_per_step = ms / args.steps
     value = job_throughput(world, args.steps, w.head_tokens, ms)
 
-    # ---- end to end through the public API: pinned host -> device, call, device -> host
+    # ---- end to end through the public API: pinned host -> device, call, device -> host.
+    # Every step copies its inputs in and its results out.  Three streams
+    # (copy-in, the compute stream, copy-out) over the N_SETS device sets let
+    # step i + 1's inputs load while step i computes and step i - 1's results
+    # return, as a streaming server would; a set is reused only after its
+    # previous results have left.
     e2e_steps = max(3, min(args.steps, 200))
     host = {n: (t.cpu().pin_memory()) for n, t in base.items()}
-    host_out = torch.empty((w.B, w.T, w.H, w.Dv), dtype=dt).pin_memory()
-    host_state = torch.empty_like(host["state_in"]).pin_memory()
+    host_res = [(torch.empty((w.B, w.T, w.H, w.Dv), dtype=dt).pin_memory(),
+                 torch.empty_like(host["state_in"]).pin_memory()) for _ in range(N_SETS)]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = host_out.numel() * host_out.element_size() + host_state.numel() * host_state.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in host_res[0])
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(N_SETS)]
+    ev_done = [torch.cuda.Event() for _ in range(N_SETS)]
+    ev_out = [torch.cuda.Event() for _ in range(N_SETS)]
+    used = [False] * N_SETS
 
     def e2e_step(i):
-        s = sets[i % N_SETS]
-        for n in ("q", "k", "v", "g", "beta", "state_in"):
-            s[n].copy_(host[n], non_blocking=True)
+        k = i % N_SETS
+        s = sets[k]
+        if used[k]:
+            s_in.wait_event(ev_out[k])  # the set's previous results have left
+        with torch.cuda.stream(s_in):
+            for n in ("q", "k", "v", "g", "beta", "state_in"):
+                s[n].copy_(host[n], non_blocking=True)
+            ev_in[k].record(s_in)
+        stream.wait_event(ev_in[k])
         fn(s["q"], s["k"], s["v"], s["g"], s["beta"], s["state_in"], state_out=s["state_out"],
            out=s["out"], chunk=w.chunk, stream=stream)
-        host_out.copy_(s["out"], non_blocking=True)
-        host_state.copy_(s["state_out"], non_blocking=True)
+        ev_done[k].record(stream)
+        s_out.wait_event(ev_done[k])
+        with torch.cuda.stream(s_out):
+            host_res[k][0].copy_(s["out"], non_blocking=True)
+            host_res[k][1].copy_(s["state_out"], non_blocking=True)
+            ev_out[k].record(s_out)
+        used[k] = True
 
-    with torch.cuda.stream(stream):
-        for i in range(3):
-            e2e_step(i)
+    for i in range(3):
+        e2e_step(i)
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for i in range(e2e_steps):
-            e2e_step(i)
-        e1.record(stream)
+    e0.record(s_in)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e1.record(s_out)
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     e2e_value = job_throughput(world, e2e_steps, w.head_tokens, e2e_ms)
@@ -522,7 +541,9 @@ def main():
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "pipelining": "copy-in / compute / copy-out on three streams over the "
+                              f"{N_SETS} device sets"},
         "gpu_launches": int(launches_per_step * args.steps),
         "launches_per_step": int(launches_per_step),
         "clocks": clocks.summary(),
