@@ -54,7 +54,7 @@ constexpr int kC = 64;            // tokens per chunk
 constexpr int kWideThreads = 256; // stage A: two warps per TMEM lane quadrant
 constexpr int kOutThreads = 512;  // stage C: four warps per TMEM lane quadrant
 constexpr int kSlab64 = kC * 16;  // bytes of one 8-column slab of a 64-row tile
-constexpr int kRecStages = 4;
+constexpr int kRecStages = 4;  // deepest stage-B load ring (see recur_stages)
 constexpr long long kDrainPolls = 1LL << 40;  // drains are bounded by the 2 s timer
 
 // ----------------------------------------------------------------- workspace
@@ -587,11 +587,12 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// NKS = Dk / 16, a compile-time constant so that the per-chunk code is
-// straight-line.
-template <int NKS>
+// NKS = Dk / 16 and NST = stages of the load ring, compile-time constants so
+// that the per-chunk code is straight-line.
+template <int NKS, int NST>
 __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_out,
                            const Workspace& ws, long long limit, unsigned* err) {
+  constexpr int nst = NST;
   RecSmemHead& hd = *reinterpret_cast<RecSmemHead*>(smem);
   const int Dk = ws.Dk, Dv = ws.Dv, nC = ws.nC;
   uint8_t* Sop0 = smem + kRecHeadBytes;
@@ -621,13 +622,13 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
   auto issue = [&](int c) {  // one thread: load chunk c (scan order) into its stage
     const int jt = dir ? nC - 1 - c : c;
     const size_t tile = ws.tile(dir, bh, jt);
-    uint8_t* st = stage0 + (c % kRecStages) * stage_bytes;
-    uint64_t* bar = &hd.full[c % kRecStages];
+    uint8_t* st = stage0 + (c % nst) * stage_bytes;
+    uint64_t* bar = &hd.full[c % nst];
     mbar_arrive_expect_tx(bar, qbytes + 16 + rbytes);
     bulk_load(st, ws.blk(tile), qbytes + 16, bar);  // Qc and decay
     bulk_load(st + qbytes + 16, ws.blk(tile) + ws.off_rc + (size_t)slice * Dk * 32, rbytes, bar);
   };
-  int issued = min(kRecStages, nC);
+  int issued = min(nst, nC);
   if (tid == 0)
     for (int c = 0; c < issued; ++c) issue(c);
 
@@ -666,8 +667,8 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
   // wait for chunk c's stage (every thread), then read its A fragments and
   // form X from the current S
   auto prefetch = [&](int cc) -> bool {
-    const int st = cc % kRecStages;
-    const bool okw = mbar_wait(&hd.full[st], (cc / kRecStages) & 1, limit);
+    const int st = cc % nst;
+    const bool okw = mbar_wait(&hd.full[st], (cc / nst) & 1, limit);
     const uint32_t qa = stage_u32 + st * stage_bytes + a_off;
 #pragma unroll
     for (int ks = 0; ks < NKS; ++ks) ldmatrix_x4(qa + ks * 2 * Dk * 16, af[ks]);
@@ -696,8 +697,8 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
       bulk_store(ws.blk(ws.tile(dir, bh, dir ? nC - 1 - c : c)) + ws.off_s +
                      (size_t)slice * 2 * nslab_bytes,
                  Sop0 + (c & 1) * kRecSBytes, 2 * nslab_bytes);
-    if (tid == 32 % blockDim.x && c >= 1 && c - 1 + kRecStages < nC) issue(c - 1 + kRecStages);
-    if (c >= 1 && c - 1 + kRecStages < nC) issued = c - 1 + kRecStages + 1;
+    if (tid == 32 % blockDim.x && c >= 1 && c - 1 + nst < nC) issue(c - 1 + nst);
+    if (c >= 1 && c - 1 + nst < nC) issued = c - 1 + nst + 1;
     const uint32_t sb = sop_u32 + (c & 1) * kRecSBytes + b_off;
     uint32_t bfr[NKS][4];
 #pragma unroll
@@ -729,7 +730,7 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
   if (c < nC) {  // a bounded wait expired: drain every load still in flight
     if (tid == 0) atomicOr(err, kErrTimeout);
     for (int p = c; p < issued; ++p)
-      mbar_wait(&hd.full[p % kRecStages], (p / kRecStages) & 1, kDrainPolls);
+      mbar_wait(&hd.full[p % nst], (p / nst) & 1, kDrainPolls);
     __syncthreads();
     return false;
   }
@@ -744,35 +745,39 @@ __device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_ou
   return true;
 }
 
-template <int NKS>
+template <int NKS, int NST>
 __global__ void __launch_bounds__(256, 1)
 gdn_recur_kernel(const float* state_in, float* state_out, Workspace ws, long long limit,
                  unsigned* err) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   RecSmemHead& hd = *reinterpret_cast<RecSmemHead*>(smem_raw);
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kRecStages; ++i) mbar_init(&hd.full[i], 1);
+    for (int i = 0; i < NST; ++i) mbar_init(&hd.full[i], 1);
     fence_mbar_init();
   }
   __syncthreads();
   pdl_wait();  // stage A's summaries are complete and visible
   pdl_trigger();
-  recur_body<NKS>(smem_raw, state_in, state_out, ws, limit, err);
+  recur_body<NKS, NST>(smem_raw, state_in, state_out, ws, limit, err);
 }
 
-// The recurrence kernel for Dk = 16 * nks.
+// The recurrence kernel for Dk = 16 * nks with an nst-stage load ring.
 using RecurKernel = void (*)(const float*, float*, Workspace, long long, unsigned*);
-RecurKernel recur_kernel(int nks) {
+template <int NST>
+RecurKernel recur_kernel_st(int nks) {
   switch (nks) {
-    case 1: return gdn_recur_kernel<1>;
-    case 2: return gdn_recur_kernel<2>;
-    case 3: return gdn_recur_kernel<3>;
-    case 4: return gdn_recur_kernel<4>;
-    case 5: return gdn_recur_kernel<5>;
-    case 6: return gdn_recur_kernel<6>;
-    case 7: return gdn_recur_kernel<7>;
-    default: return gdn_recur_kernel<8>;
+    case 1: return gdn_recur_kernel<1, NST>;
+    case 2: return gdn_recur_kernel<2, NST>;
+    case 3: return gdn_recur_kernel<3, NST>;
+    case 4: return gdn_recur_kernel<4, NST>;
+    case 5: return gdn_recur_kernel<5, NST>;
+    case 6: return gdn_recur_kernel<6, NST>;
+    case 7: return gdn_recur_kernel<7, NST>;
+    default: return gdn_recur_kernel<8, NST>;
   }
+}
+RecurKernel recur_kernel(int nks, int nst) {
+  return nst >= 4 ? recur_kernel_st<4>(nks) : nst == 3 ? recur_kernel_st<3>(nks) : recur_kernel_st<2>(nks);
 }
 
 // ========================================================== stage C: output
@@ -1123,9 +1128,21 @@ int num_sms() {
   return cached[dev];
 }
 
-int recur_smem_bytes(int Dk) {
+int recur_smem_bytes(int Dk, int nst) {
   const int stage = ((Dk * Dk * 2 + Dk * 32 + 16) + 127) & ~127;
-  return kRecHeadBytes + 2 * kRecSBytes + kRecStages * stage;
+  return kRecHeadBytes + 2 * kRecSBytes + nst * stage;
+}
+
+// Stages of stage B's load ring: the full kRecStages while the grid fits one
+// CTA per SM; otherwise the deepest ring (at least 2) that lets two CTAs
+// share an SM, so a grid of more CTAs than SMs (both directions, many heads)
+// still runs in one wave instead of two chained ones.
+int recur_stages(int Dk, int ctas, int sms) {
+  if (ctas <= sms) return kRecStages;
+  constexpr int kHalfSm = 113 * 1024;  // per-CTA share of an SM's shared memory, two CTAs
+  int nst = kRecStages;
+  while (nst > 2 && recur_smem_bytes(Dk, nst) > kHalfSm) --nst;
+  return nst;
 }
 
 // Opt the kernels into their dynamic shared memory, once per device.
@@ -1143,8 +1160,9 @@ cudaError_t set_smem_attrs() {
                            (int)sizeof(PrepSmem));
   if (e == cudaSuccess)
     for (int nks = 1; nks <= 8 && e == cudaSuccess; ++nks)
-      e = cudaFuncSetAttribute(recur_kernel(nks), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               recur_smem_bytes(128));
+      for (int nst = 2; nst <= kRecStages && e == cudaSuccess; ++nst)
+        e = cudaFuncSetAttribute(recur_kernel(nks, nst), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 recur_smem_bytes(128, nst));
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(gdn_output_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)OutLayout(128, 128).total);
@@ -1205,9 +1223,10 @@ cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
   if (e != cudaSuccess) return e;
   {
     ProfileScope ps(a.stream, kKernRecur);
-    e = launch_pdl(recur_kernel(a.Dk / 16), dim3(a.Dv / 16, NBH, ndir), 32 * (a.Dk / 16),
-                   recur_smem_bytes(a.Dk), a.stream, a.state_in, a.state_out, ws, a.wait_limit,
-                   a.err);
+    const int nst = recur_stages(a.Dk, (a.Dv / 16) * NBH * ndir, num_sms());
+    e = launch_pdl(recur_kernel(a.Dk / 16, nst), dim3(a.Dv / 16, NBH, ndir), 32 * (a.Dk / 16),
+                   recur_smem_bytes(a.Dk, nst), a.stream, a.state_in, a.state_out, ws,
+                   a.wait_limit, a.err);
   }
   if (e != cudaSuccess) return e;
   {
