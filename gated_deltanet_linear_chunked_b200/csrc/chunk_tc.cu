@@ -8,7 +8,9 @@
 //   stage A  gdn_prep_kernel    one CTA per (chunk, b*h, direction), parallel
 //   stage B  gdn_recur_kernel   one CTA per (16 state columns, b*h, direction),
 //                               a dependent walk over the chunks
-//   stage C  gdn_output_kernel  one CTA per (chunk, b*h), both directions
+//   stage C  gdn_output_kernel  persistent, one CTA per SM over the (chunk,
+//                               b*h) tiles, both directions per tile
+// launched back to back with programmatic dependent launch.
 //
 // Algebra (per head; a chunk holds C = 64 tokens in scan order, entered with
 // state S0; gamma_r = sum of g over the chunk's tokens up to r in scan order,
@@ -22,18 +24,22 @@
 //   O     = diag(e^gamma) Q^ S0 + (Mask o Q^ K^^T) U,
 //           Mask_ri = e^{gamma_r - gamma_i} for i at or before r, else 0.
 // Stage A computes Tm, W, U~, Qc, Rc (d x d summaries of the chunk); stage B
-// runs S <- e^{gamma_C} S - Qc S + Rc, one 128 x 16 x d MMA per chunk, and
-// publishes the state at each chunk start; stage C computes U and O.
+// runs S <- e^{gamma_C} S - Qc S + Rc (per 16-column slice, a d x d times
+// d x 16 product on mma.sync per chunk) and publishes the state at each chunk
+// start; stage C computes U and O.
 //
 // The reverse (within-chunk backward) scan of the bidirectional mode uses the
 // same memory tiles visited in the opposite order, with gamma the suffix sums
 // and "before" meaning "later in memory"; both directions' outputs are summed
 // in one fp32 TMEM accumulator before the single bf16 store.
 //
-// Every contraction is a tcgen05.mma (bf16 x bf16 -> fp32 in TMEM) issued by
-// one thread from SWIZZLE_NONE core-matrix shared-memory layouts; q/k/v tiles
-// arrive by TMA tensor loads, workspace tiles by bulk copies.  The 64 x 64
-// triangular inverse is a blocked fp32 forward substitution on CUDA cores.
+// The contractions of stages A and C are tcgen05.mma (bf16 x bf16 -> fp32 in
+// TMEM) issued by one thread from SWIZZLE_NONE core-matrix shared-memory
+// layouts; q/k/v tiles arrive by TMA tensor loads, workspace tiles by bulk
+// copies.  The 64 x 64 triangular inverse is a blocked solve: 16 x 16
+// diagonal blocks by fp32 forward substitution, merges on tf32 mma.sync.
+// Stage B's latency-bound chain uses warp-level mma.sync (bf16, fp32
+// accumulate), its state in registers.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -554,13 +560,14 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 // One CTA per (16 state columns, b*h, direction), Dk/16 warps; warp w owns
 // state rows [16w, 16w + 16).  Per chunk the product Qc S (Dk x Dk times
 // Dk x 16) is a dependent chain across chunks and is latency-bound: a
-// tcgen05 round trip (issue 7 MMAs, commit, mbarrier, TMEM load) costs
-// ~1.2k cycles per chunk here, so this stage uses warp-level
-// mma.sync.m16n8k16 (bf16 in, fp32 accumulate) with the fp32 state held in
-// the accumulator registers and the bf16 copy of S exchanged through a
-// double-buffered shared-memory operand: one barrier per chunk.
+// tcgen05 round trip (issue 7 MMAs, commit, mbarrier, TMEM load) costs about
+// 1.2k cycles for a 16-column slice and over 3k for a whole head, so this
+// stage uses warp-level mma.sync.m16n8k16 (bf16 in, fp32 accumulate) with
+// the fp32 state held in the accumulator registers and the bf16 copy of S
+// exchanged through a double-buffered shared-memory operand: one barrier per
+// chunk.  An NST-stage ring of bulk loads feeds [Qc | decay | Rc slice].
 // Dynamic layout: [head 128 B] [S operand x 2: [2 n-slabs][Dk][8] bf16]
-//                 [stages: Qc [Dk/8][Dk][8] | decay 16 B | Rc slice [Dk][16]]
+//                 [NST stages: Qc [Dk/8][Dk][8] | decay 16 B | Rc slice [Dk][16]]
 struct RecSmemHead {
   uint64_t full[kRecStages];
 };
