@@ -81,9 +81,12 @@ typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
  * state_out  receives the final state; may equal state_in (in place);
  *            may be NULL when the caller does not need it.
  * out        receives o_t for every token, in `dtype`.
- * chunk      sub-chunk length the kernels tile time with: 0 (default, 64),
- *            16, 32 or 64.  It changes rounding only, never the result's
- *            definition.  The fp32 path scans token by token and ignores it.
+ * chunk      sub-chunk length hint: 0 (default), 16, 32 or 64; any other
+ *            value is GDN_ERR_INVALID_ARG.  The chunked form equals the
+ *            recurrence for every sub-chunk length, so the hint can change
+ *            rounding only, never the result's definition.  The bf16
+ *            tensor-core path tiles time with 64 tokens whatever the hint;
+ *            the fp32 path scans token by token.
  * T == 0     is allowed: state_out = state_in (or zero), out is untouched.
  * B == 0 or H == 0 is allowed and does nothing.
  */
