@@ -799,9 +799,10 @@ RecurKernel recur_kernel(int nks, int nst) {
 // then P [8][64][8] (masked, gated Q K^T, K-major A) and the scalar block.
 struct OutSmall {
   float g[2][64];
-  float gam[64], rnq[64], rnk[64], arow[64];
+  float gam[64], rnq[2][64], rnk[2][64], arow[64];  // norms per tile set
   float bcol[8][64];
   uint64_t tma_bar[2], ld_bar[2], mma_bar;
+  uint64_t fin_bar;  // one commit on a failed wait: every MMA issued has landed
   uint32_t tmem;
 };
 struct OutLayout {
@@ -871,20 +872,69 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
     }
   };
 
+  // mbarrier phase parities: bit `set` of tma_ph / ld_ph
+  uint32_t tma_ph = 0, ld_ph = 0, mma_ph = 0;
+  // Head of the tile in `set`: wait for its q/k tile and gates, issue
+  // P = Q K^T (shared by both directions), then the row norms, which overlap
+  // it.  `one_more`: a later tile's gates are in flight too.  The head of
+  // tile t + 1 runs while tile t's last MMA round executes.
+  auto head = [&](int set, bool one_more) -> bool {
+    uint8_t* base = smem + set * L.set_bytes;
+    uint8_t* sQ = base + L.q;
+    uint8_t* sK = base + L.k;
+    if (tid < kC) {
+      if (one_more) cp_async_wait<1>();
+      else cp_async_wait<0>();
+    }
+    if (!block_wait(&sm.tma_bar[set], (tma_ph >> set) & 1, limit, err)) return false;
+    tma_ph ^= 1u << set;
+    if (tid == 0) {
+      tc_fence_after_sync();
+      const uint32_t idP = idesc_bf16(64, 64, 0, 0);
+      for (int ks = 0; ks < Dk / 16; ++ks)
+        mma_bf16(tmP, sdesc(smem_u32(sQ) + ks * 2 * kSlab64, kSlab64, 128),
+                 sdesc(smem_u32(sK) + ks * 2 * kSlab64, kSlab64, 128), idP, ks > 0);
+    }
+    {  // 1 / |q|, 1 / |k| per row: four threads per row and tensor
+      const int row = tid >> 3, part = tid & 3;
+      const bool isk = (tid >> 2) & 1;
+      const float rn = row_rnorm4(isk ? sK : sQ, row, part, Dk);
+      if (part == 0) (isk ? sm.rnk[set] : sm.rnq[set])[row] = rn;
+    }
+    return true;
+  };
+
+  // On a failed wait, before leaving: one commit covering every MMA this
+  // CTA issued (P = Q K^T is issued ahead of its commit), so none is still
+  // writing TMEM when the accumulators are freed.
+  auto drain_mma = [&]() {
+    if (tid == 0) mma_commit(&sm.fin_bar);
+    mbar_wait(&sm.fin_bar, 0, kDrainPolls);
+  };
+
   int k = 0;
   if (blockIdx.x < ntiles) issue_tile(0, blockIdx.x);
   if (blockIdx.x + gridDim.x < ntiles) issue_tile(1, blockIdx.x + gridDim.x);
-  // mbarrier phase parities: bit `set` of tma_ph / ld_ph
-  uint32_t tma_ph = 0, ld_ph = 0, mma_ph = 0;
+  if (blockIdx.x < ntiles && !head(0, blockIdx.x + gridDim.x < ntiles)) {
+    mbar_wait(&sm.ld_bar[0], 0, kDrainPolls);
+    if (blockIdx.x + gridDim.x < ntiles) {
+      mbar_wait(&sm.tma_bar[1], 0, kDrainPolls);
+      mbar_wait(&sm.ld_bar[1], 0, kDrainPolls);
+    }
+    drain_mma();
+    return false;
+  }
   for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++k) {
     const int set = k & 1;
     const bool next_issued = t + gridDim.x < ntiles;
-    // on a failed wait: drain the other set's loads (the caller drained its own)
+    // on a failed wait: drain the next tile's loads (its head has not run;
+    // the caller drained its own barrier)
     auto drain_other = [&]() {
       if (next_issued) {
         mbar_wait(&sm.tma_bar[set ^ 1], (tma_ph >> (set ^ 1)) & 1, kDrainPolls);
         mbar_wait(&sm.ld_bar[set ^ 1], (ld_ph >> (set ^ 1)) & 1, kDrainPolls);
       }
+      drain_mma();
     };
     uint8_t* base = smem + set * L.set_bytes;
     uint8_t* sQ = base + L.q;
@@ -896,29 +946,6 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
     const int b = bh / H, h = bh - b * H, t0 = j * kC;
     const int nvalid = min(kC, T - t0);
 
-    if (tid < kC) {
-      if (next_issued) cp_async_wait<1>();
-      else cp_async_wait<0>();
-    }
-    if (!block_wait(&sm.tma_bar[set], (tma_ph >> set) & 1, limit, err)) {
-      mbar_wait(&sm.ld_bar[set], (ld_ph >> set) & 1, kDrainPolls);
-      drain_other();
-      return false;
-    }
-    tma_ph ^= 1u << set;
-    if (tid == 0) {  // P = Q K^T, shared by both directions; overlaps the norms
-      tc_fence_after_sync();
-      const uint32_t idP = idesc_bf16(64, 64, 0, 0);
-      for (int ks = 0; ks < Dk / 16; ++ks)
-        mma_bf16(tmP, sdesc(smem_u32(sQ) + ks * 2 * kSlab64, kSlab64, 128),
-                 sdesc(smem_u32(sK) + ks * 2 * kSlab64, kSlab64, 128), idP, ks > 0);
-    }
-    {  // 1 / |q|, 1 / |k| per row: four threads per row and tensor
-      const int row = tid >> 3, part = tid & 3;
-      const bool isk = (tid >> 2) & 1;
-      const float rn = row_rnorm4(isk ? sK : sQ, row, part, Dk);
-      if (part == 0) (isk ? sm.rnk : sm.rnq)[row] = rn;
-    }
     for (int dir = 0; dir < ndir; ++dir) {
       // D_U: direction 0 borrows D_O's columns (D_O is first written after
       // D_U is consumed); direction 1 needs its own, [192, 320) of a
@@ -933,7 +960,7 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
         const int blk = e >> 6, i = e & 63;
         const int qpos = dir ? 63 - i : i;
         const float mb = sm.gam[dir ? 63 - 8 * blk : 8 * blk];
-        sm.bcol[blk][i] = (qpos < 8 * blk + 8) ? sm.rnk[i] * exp2f((mb - sm.gam[i]) * kLog2e) : 0.f;
+        sm.bcol[blk][i] = (qpos < 8 * blk + 8) ? sm.rnk[set][i] * exp2f((mb - sm.gam[i]) * kLog2e) : 0.f;
       }
       if (tid < 64) {
         const int p = dir ? 63 - tid : tid;
@@ -1020,17 +1047,33 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
                    sdesc(smem_u32(sUt) + ks * 256, 128, kSlab64), idO, 1);
         mma_commit(&sm.mma_bar);
       }
-      if (!block_wait(&sm.mma_bar, mma_ph, limit, err)) {
-        drain_other();
-        return false;
+      if (dir + 1 < ndir) {
+        if (!block_wait(&sm.mma_bar, mma_ph, limit, err)) {
+          drain_other();
+          return false;
+        }
+        mma_ph ^= 1;
+        if (tid == 0) issue_dir(set, t, dir + 1);
       }
-      mma_ph ^= 1;
-      if (dir + 1 < ndir && tid == 0) issue_dir(set, t, dir + 1);
     }
+    // the last direction's second round is in flight: the next tile's head
+    // (its loads, P = Q K^T and norms) runs meanwhile
+    if (next_issued && !head(set ^ 1, false)) {
+      // head drained the next tile's q/k; its W | U~ | S and this round remain
+      mbar_wait(&sm.ld_bar[set ^ 1], (ld_ph >> (set ^ 1)) & 1, kDrainPolls);
+      drain_mma();
+      return false;
+    }
+    if (!block_wait(&sm.mma_bar, mma_ph, limit, err)) {
+      if (next_issued) mbar_wait(&sm.ld_bar[set ^ 1], (ld_ph >> (set ^ 1)) & 1, kDrainPolls);
+      drain_mma();
+      return false;
+    }
+    mma_ph ^= 1;
     tc_fence_after_sync();
     // O = diag(1/|q|) D_O -> out (rows of this chunk that exist)
     {
-      const float rq = sm.rnq[r];
+      const float rq = sm.rnq[set][r];
       float v0[16], v1[16];
       const bool has1 = part + 4 < Dv / 16;
       if (part < Dv / 16) tmem_ld16(tmO + lane_base + 16 * part, v0);
@@ -1071,6 +1114,7 @@ gdn_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     mbar_init(&sm.ld_bar[0], 1);
     mbar_init(&sm.ld_bar[1], 1);
     mbar_init(&sm.mma_bar, 1);
+    mbar_init(&sm.fin_bar, 1);
     fence_mbar_init();
   }
   if ((tid >> 5) == 0) {
