@@ -210,9 +210,22 @@ def cpu_baseline(w, budget_s: float):
         el = time.perf_counter() - t0
         if el >= budget_s or reps >= 1000:
             break
+    # the same recurrence on one core, over one head of the chunk, for about
+    # a tenth of the budget
+    from gated_deltanet_linear_chunked_b200.workloads import slice_head
+    one = slice_head(x, 0, 0)
+    reps1, t1 = 0, time.perf_counter()
+    while True:
+        fn(one["q"], one["k"], one["v"], one["g"], one["beta"], one["state_in"], nthreads=1)
+        reps1 += 1
+        el1 = time.perf_counter() - t1
+        if el1 >= budget_s / 10 or reps1 >= 1000:
+            break
     return {"value": w.head_tokens * reps / el, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"full {w.name} chunk (B{w.B} H{w.H} T{w.T} d{w.Dk}, fp64 token recurrence), "
-                      f"{reps} repetitions in {el:.1f} s"}
+                      f"{reps} repetitions in {el:.1f} s",
+            "value_1core": w.T * reps1 / el1,
+            "sample_1core": f"one head of the chunk on one thread, {reps1} repetitions in {el1:.1f} s"}
 
 
 # ---- multi-rank plumbing (one process per GPU; no data-path collective)
@@ -430,6 +443,7 @@ def main():
 
     # ---- side figures: the other mode, and the 15-layer stacked stream
     extras = {}
+    graphs.clear()  # the main figure is taken; free its graphs' memory
     if not args.no_extras:
         other = "bidir" if w.mode == "fwd" else "fwd"
         fo = gdn.chunk_bidir if other == "bidir" else gdn.chunk_fwd
@@ -471,32 +485,35 @@ def main():
         extras[f"{other}_chunk"] = {"ms_per_call": other_ms,
                                     "head_tokens_per_s": w.head_tokens / (other_ms / 1000.0),
                                     "timing": "CUDA graph replays" if use_graph else "direct calls"}
-        # 32 chunks x 15 layers in model order (chunk-major), bidirectional,
-        # one state per layer carried in place, inputs rotating over the sets
-        states = [torch.zeros_like(base["state_in"]) for _ in range(wl.GDN_LAYERS)]
+        # 32 chunks x 15 layers in model order (chunk-major), one state per
+        # layer carried in place, inputs rotating over the sets; the pages'
+        # streaming GDN is bidirectional, the causal stack is reported too
         n_chunks = 32
+        for smode, sfn in (("bidir", gdn.chunk_bidir), ("causal", gdn.chunk_fwd)):
+            states = [torch.zeros_like(base["state_in"]) for _ in range(wl.GDN_LAYERS)]
 
-        def stack_run():
-            with torch.cuda.stream(stream):
-                i = 0
-                for _c in range(n_chunks):
-                    for l in range(wl.GDN_LAYERS):
-                        s = sets[i % N_SETS]
-                        gdn.chunk_bidir(s["q"], s["k"], s["v"], s["g"], s["beta"], states[l],
-                                        state_out=states[l], out=s["out"], chunk=w.chunk,
-                                        stream=stream)
-                        i += 1
-        stack_run()
-        barrier()
-        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        b0.record(stream)
-        stack_run()
-        b1.record(stream)
-        barrier()
-        stack_ms = b0.elapsed_time(b1)
-        frames = n_chunks * 3
-        extras["stack_32x15_bidir"] = {"ms": stack_ms, "latent_frames_per_s": frames / (stack_ms / 1000.0),
-                                       "calls": n_chunks * wl.GDN_LAYERS, "timing": "direct calls"}
+            def stack_run():
+                with torch.cuda.stream(stream):
+                    i = 0
+                    for _c in range(n_chunks):
+                        for l in range(wl.GDN_LAYERS):
+                            s = sets[i % N_SETS]
+                            sfn(s["q"], s["k"], s["v"], s["g"], s["beta"], states[l],
+                                state_out=states[l], out=s["out"], chunk=w.chunk, stream=stream)
+                            i += 1
+            stack_run()
+            barrier()
+            b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            b0.record(stream)
+            stack_run()
+            b1.record(stream)
+            barrier()
+            stack_ms = b0.elapsed_time(b1)
+            frames = n_chunks * 3
+            extras[f"stack_32x15_{smode}"] = {"ms": stack_ms,
+                                              "latent_frames_per_s": frames / (stack_ms / 1000.0),
+                                              "calls": n_chunks * wl.GDN_LAYERS,
+                                              "timing": "direct calls"}
 
     # ---- per-kernel device times (CUDA events on the launching stream,
     # recorded by the library around each launch over a loop of direct calls)
@@ -534,6 +551,8 @@ def main():
                 "kernels": kernels,
                 "path": {"algorithmic_bytes": bytes_step, "achieved": path_achieved,
                          "frac": path_achieved / peaks["hbm_gbs"],
+                         "algorithmic_flops": flops_step,
+                         "achieved_tflops": flops_step / (ms_per_step / 1000.0) / 1e12,
                          "tensor_frac_of_sustained": (flops_step / (ms_per_step / 1000.0) / 1e12)
                          / peaks["bf16_tflops_sustained"]}}
 
