@@ -298,6 +298,145 @@ def run_reference(args, w):
     return 0
 
 
+def nvtx(name):
+    """NVTX range around a bench phase (visible in a profiler's timeline)."""
+    import contextlib
+    import torch
+    try:
+        return torch.cuda.nvtx.range(name)
+    except Exception:
+        return contextlib.nullcontext()
+
+
+def make_sets(w, xh, dev, n):
+    """`n` device copies of one chunk's inputs, each with its own out and
+    state_out, so consecutive steps read different buffers."""
+    import torch
+    dt = torch.bfloat16
+    base = {k: torch.from_numpy(xh[k]).to(dev) for k in ("q", "k", "v", "g", "beta")}
+    for k in ("q", "k", "v"):
+        base[k] = base[k].to(dt)
+    base["state_in"] = torch.from_numpy(xh["state_in"]).to(dev)
+    sets = []
+    for _ in range(n):
+        s = {k: t.clone() for k, t in base.items()}
+        s["out"] = torch.empty((w.B, w.T, w.H, w.Dv), dtype=dt, device=dev)
+        s["state_out"] = torch.empty_like(s["state_in"])
+        sets.append(s)
+    return base, sets
+
+
+class Stepper:
+    """One library call per step over rotating input sets, as direct calls or
+    as replays of one captured CUDA graph per set.  A direct call on the
+    stream comes first, so the library's per-stream scratch exists before any
+    capture and the graphs hold kernel nodes only (no memory nodes)."""
+
+    def __init__(self, fn, sets, stream, chunk, use_graph):
+        import torch
+        self.fn, self.sets, self.stream, self.chunk = fn, sets, stream, chunk
+        self.graphs = []
+        with torch.cuda.stream(stream):
+            self.call(0)
+        torch.cuda.synchronize()
+        if use_graph:
+            for i in range(len(sets)):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    self.call(i)
+                self.graphs.append(g)
+            torch.cuda.synchronize()
+
+    def call(self, i):
+        s = self.sets[i % len(self.sets)]
+        self.fn(s["q"], s["k"], s["v"], s["g"], s["beta"], s["state_in"], state_out=s["state_out"],
+                out=s["out"], chunk=self.chunk, stream=self.stream)
+
+    def run(self, n, offset=0):
+        import torch
+        with torch.cuda.stream(self.stream):
+            for i in range(n):
+                if self.graphs:
+                    self.graphs[(i + offset) % len(self.graphs)].replay()
+                else:
+                    self.call(i + offset)
+
+    def warm(self, n):
+        """At least `n` steps, and every graph replayed at least once."""
+        self.run(max(n, len(self.sets)))
+
+    def release(self):
+        self.graphs.clear()
+
+
+def kernel_times(lib, step_fn, n, launches_per_step):
+    """Per-kernel CUDA-event times (the library records events on the
+    launching stream around each launch) over `n` direct calls."""
+    import ctypes
+    from gated_deltanet_linear_chunked_b200 import _lib
+    _lib.check(lib.gdn_profile_begin(int(n * max(1, launches_per_step) + 8)), "gdn_profile_begin")
+    for i in range(n):
+        step_fn(i)
+    kms = (ctypes.c_float * 4)()
+    kn = (ctypes.c_int * 4)()
+    _lib.check(lib.gdn_profile_end(ctypes.addressof(kms), ctypes.addressof(kn), 4), "gdn_profile_end")
+    kernels = {}
+    for i in range(4):
+        if kn[i]:
+            kernels[lib.gdn_kernel_name(i).decode()] = {"launches": kn[i], "ms_per_launch": kms[i] / kn[i]}
+    tot = sum(v["ms_per_launch"] for v in kernels.values())
+    for v in kernels.values():
+        v["share"] = v["ms_per_launch"] / tot if tot else None
+    return kernels
+
+
+def roofline_times(w, bidir, peaks):
+    """Seconds the step would take at the HBM and at the tensor-pipe peak:
+    algorithmic bytes over the measured copy bandwidth, chunked-form FLOPs
+    over the sustained bf16 GEMM rate (the roofline definition the scope
+    table fixes)."""
+    return (algorithmic_bytes(w) / (peaks["hbm_gbs"] * 1e9),
+            algorithmic_flops(w, bidir) / (peaks["bf16_tflops_sustained"] * 1e12))
+
+
+def roofline_of(w, kernels, ms_per_step, peaks, peak_kind, bidir):
+    """The dominant kernel against the path's binding bound: achieved = the
+    path's algorithmic bytes (or FLOPs) per step -- one launch of each kernel
+    processes every unit of the step -- over that kernel's mean launch time.
+    `path` gives the same figure over the whole step's time."""
+    bytes_step = algorithmic_bytes(w)
+    flops_step = algorithmic_flops(w, bidir)
+    dom = max(kernels, key=lambda k: kernels[k]["ms_per_launch"])
+    dom_ms = kernels[dom]["ms_per_launch"]
+    t_hbm, t_tc = roofline_times(w, bidir, peaks)
+    if t_tc > t_hbm:
+        bound, unit, work = "tensor", "TFLOP/s", flops_step / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        src = f"{peak_kind} bf16_tflops_sustained"
+    else:
+        bound, unit, work, peak = "hbm", "GB/s", bytes_step / 1e9, peaks["hbm_gbs"]
+        src = f"{peak_kind} hbm_gbs"
+    achieved = work / (dom_ms / 1000.0)
+    path_achieved = work / (ms_per_step / 1000.0)
+    return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak, "traffic": recorded_traffic(dom),
+            "traffic_source": "committed ncu summary profiles/dram_traffic.txt, valid while the "
+                              "kernel's source hash matches (else null)",
+            "peak_source": src, "kernel": dom,
+            "algorithmic_bytes_per_launch": bytes_step, "algorithmic_flops_per_launch": flops_step,
+            "ms_per_launch": dom_ms, "kernels": kernels,
+            "kernel_share_frac": {k: (kernel_algorithmic_bytes(k, w) / (v["ms_per_launch"] / 1000.0)
+                                      / 1e9 / peaks["hbm_gbs"]) for k, v in kernels.items()},
+            "path": {"ms_per_step": ms_per_step, "achieved": path_achieved, "frac": path_achieved / peak,
+                     "roofline_us": 1e6 * max(t_hbm, t_tc),
+                     "algorithmic_bytes": bytes_step, "algorithmic_flops": flops_step,
+                     "achieved_gbs": bytes_step / (ms_per_step / 1000.0) / 1e9,
+                     "achieved_tflops": flops_step / (ms_per_step / 1000.0) / 1e12,
+                     "hbm_frac": bytes_step / (ms_per_step / 1000.0) / 1e9 / peaks["hbm_gbs"],
+                     "tensor_frac_of_sustained": flops_step / (ms_per_step / 1000.0) / 1e12
+                     / peaks["bf16_tflops_sustained"]}}
+
+
 def main():
     args = parse()
     from gated_deltanet_linear_chunked_b200 import workloads as wl
@@ -322,74 +461,47 @@ def main():
     lib = _lib.load()
     stream = torch.cuda.Stream(device=dev)
     fn = gdn.chunk_bidir if w.mode == "bidir" else gdn.chunk_fwd
+    use_graph = not args.no_graph
 
     # ---- inputs: one seeded chunk per rank, copied into N_SETS rotating sets
     w_r = rank_workload(w, rank)
     xh = wl.make_inputs(w_r)
-    dt = torch.bfloat16
-    base = {n: torch.from_numpy(xh[n]).to(dev) for n in ("q", "k", "v", "g", "beta")}
-    for n in ("q", "k", "v"):
-        base[n] = base[n].to(dt)
-    base["state_in"] = torch.from_numpy(xh["state_in"]).to(dev)
-    sets = []
-    for _ in range(N_SETS):
-        s = {n: t.clone() for n, t in base.items()}
-        s["out"] = torch.empty((w.B, w.T, w.H, w.Dv), dtype=dt, device=dev)
-        s["state_out"] = torch.empty_like(s["state_in"])
-        sets.append(s)
+    base, sets = make_sets(w, xh, dev, N_SETS)
     torch.cuda.synchronize()
-
-    def step(i):
-        s = sets[i % N_SETS]
-        fn(s["q"], s["k"], s["v"], s["g"], s["beta"], s["state_in"], state_out=s["state_out"],
-           out=s["out"], chunk=w.chunk, stream=stream)
 
     # launches per step (counted on a direct call)
     c0 = lib.gdn_launch_count()
     with torch.cuda.stream(stream):
-        step(0)
+        fn(sets[0]["q"], sets[0]["k"], sets[0]["v"], sets[0]["g"], sets[0]["beta"],
+           sets[0]["state_in"], state_out=sets[0]["state_out"], out=sets[0]["out"],
+           chunk=w.chunk, stream=stream)
     launches_per_step = lib.gdn_launch_count() - c0
     torch.cuda.synchronize()
-
-    use_graph = not args.no_graph
-    graphs = []
-    if use_graph:
-        for i in range(N_SETS):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                step(i)
-            graphs.append(g)
-        torch.cuda.synchronize()
-
-    def run_steps(n, offset=0):
-        with torch.cuda.stream(stream):
-            for i in range(n):
-                if use_graph:
-                    graphs[(i + offset) % N_SETS].replay()
-                else:
-                    step(i + offset)
 
     def barrier():
         if world > 1:
             dist.barrier(device_ids=[local])
         torch.cuda.synchronize()
 
-    run_steps(max(3, args.warmup))
+    main_run = Stepper(fn, sets, stream, w.chunk, use_graph)
+    with nvtx("warmup"):
+        main_run.warm(max(3, args.warmup))
     barrier()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     try:
         nvml_index = torch.cuda._get_nvml_device_index(local)
     except Exception:
         nvml_index = local
-    with ClockSampler(nvml_index) as clocks:
+    with ClockSampler(nvml_index) as clocks, nvtx("timed"):
         barrier()
         ev0.record(stream)
-        run_steps(args.steps)
+        main_run.run(args.steps)
         ev1.record(stream)
         barrier()
     ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     ms_per_step = ms / args.steps
     value = job_throughput(world, args.steps, w.head_tokens, ms)
+    main_run.release()
 
     # ---- end to end through the public API: pinned host -> device, call, device -> host.
     # Every step copies its inputs in and its results out.  Three streams
@@ -399,7 +511,7 @@ def main():
     # previous results have left.
     e2e_steps = max(3, min(args.steps, 200))
     host = {n: (t.cpu().pin_memory()) for n, t in base.items()}
-    host_res = [(torch.empty((w.B, w.T, w.H, w.Dv), dtype=dt).pin_memory(),
+    host_res = [(torch.empty((w.B, w.T, w.H, w.Dv), dtype=torch.bfloat16).pin_memory(),
                  torch.empty_like(host["state_in"]).pin_memory()) for _ in range(N_SETS)]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = sum(t.numel() * t.element_size() for t in host_res[0])
@@ -429,62 +541,59 @@ def main():
             ev_out[k].record(s_out)
         used[k] = True
 
-    for i in range(3):
-        e2e_step(i)
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s_in)
-    for i in range(e2e_steps):
-        e2e_step(i)
-    e1.record(s_out)
-    barrier()
+    with nvtx("e2e"):
+        for i in range(max(3, N_SETS)):
+            e2e_step(i)
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s_in)
+        for i in range(e2e_steps):
+            e2e_step(i)
+        e1.record(s_out)
+        barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     e2e_value = job_throughput(world, e2e_steps, w.head_tokens, e2e_ms)
 
-    # ---- side figures: the other mode, and the 15-layer stacked stream
+    # ---- per-kernel device times and the roofline of the dominant kernel
+    peaks, peak_kind = load_peaks()
+    n_prof = max(3, min(args.steps, 100))
+
+    def direct(i):
+        with torch.cuda.stream(stream):
+            main_run.call(i)
+    kernels = kernel_times(lib, direct, n_prof, launches_per_step)
+    roofline = roofline_of(w, kernels, ms_per_step, peaks, peak_kind, w.mode == "bidir")
+
+    # ---- side figures: the other mode (its own roofline), and the 15-layer
+    # stacked stream (direct calls and one captured graph)
     extras = {}
-    graphs.clear()  # the main figure is taken; free its graphs' memory
     if not args.no_extras:
         other = "bidir" if w.mode == "fwd" else "fwd"
         fo = gdn.chunk_bidir if other == "bidir" else gdn.chunk_fwd
         n_side = max(3, min(args.steps, 200))
-
-        def side_call(i):
-            s = sets[i % N_SETS]
-            fo(s["q"], s["k"], s["v"], s["g"], s["beta"], s["state_in"],
-               state_out=s["state_out"], out=s["out"], chunk=w.chunk, stream=stream)
-
-        side_graphs = []
-        if use_graph:  # timed like the main figure: graph replays over the rotating sets
-            with torch.cuda.stream(stream):
-                side_call(0)
-            torch.cuda.synchronize()
-            for i in range(N_SETS):
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=stream):
-                    side_call(i)
-                side_graphs.append(g)
-            torch.cuda.synchronize()
-
-        def side_run(n):
-            with torch.cuda.stream(stream):
-                for i in range(n):
-                    if use_graph:
-                        side_graphs[i % N_SETS].replay()
-                    else:
-                        side_call(i)
-        side_run(3)
-        barrier()
-        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
-        side_run(n_side)
-        a1.record(stream)
-        barrier()
-        side_graphs.clear()
+        with nvtx(f"{other}_chunk"):
+            side = Stepper(fo, sets, stream, w.chunk, use_graph)
+            side.warm(max(3, args.warmup))
+            barrier()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            side.run(n_side)
+            a1.record(stream)
+            barrier()
+            side.release()
         other_ms = a0.elapsed_time(a1) / n_side
-        extras[f"{other}_chunk"] = {"ms_per_call": other_ms,
-                                    "head_tokens_per_s": w.head_tokens / (other_ms / 1000.0),
-                                    "timing": "CUDA graph replays" if use_graph else "direct calls"}
+
+        def side_direct(i):
+            with torch.cuda.stream(stream):
+                side.call(i)
+        side_kernels = kernel_times(lib, side_direct, n_prof, launches_per_step)
+        wo = wl.stream_chunk(other)
+        extras[f"{other}_chunk"] = {
+            "workload": wo.name, "ms_per_step": other_ms,
+            "head_tokens_per_s": w.head_tokens / (other_ms / 1000.0),
+            "latent_frames_per_s": w.B * (w.T / 880) / (other_ms / 1000.0),
+            "steps": n_side, "timing": "CUDA graph replays" if use_graph else "direct calls",
+            "roofline": roofline_of(wo, side_kernels, other_ms, peaks, peak_kind, other == "bidir")}
         # 32 chunks x 15 layers in model order (chunk-major), one state per
         # layer carried in place, inputs rotating over the sets; the pages'
         # streaming GDN is bidirectional, the causal stack is reported too
@@ -492,77 +601,54 @@ def main():
         for smode, sfn in (("bidir", gdn.chunk_bidir), ("causal", gdn.chunk_fwd)):
             states = [torch.zeros_like(base["state_in"]) for _ in range(wl.GDN_LAYERS)]
 
-            def stack_run():
-                with torch.cuda.stream(stream):
-                    i = 0
-                    for _c in range(n_chunks):
-                        for l in range(wl.GDN_LAYERS):
-                            s = sets[i % N_SETS]
-                            sfn(s["q"], s["k"], s["v"], s["g"], s["beta"], states[l],
-                                state_out=states[l], out=s["out"], chunk=w.chunk, stream=stream)
-                            i += 1
-            stack_run()
-            barrier()
-            b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            b0.record(stream)
-            stack_run()
-            b1.record(stream)
-            barrier()
-            stack_ms = b0.elapsed_time(b1)
+            def stack_calls():
+                i = 0
+                for _c in range(n_chunks):
+                    for l in range(wl.GDN_LAYERS):
+                        s = sets[i % N_SETS]
+                        sfn(s["q"], s["k"], s["v"], s["g"], s["beta"], states[l],
+                            state_out=states[l], out=s["out"], chunk=w.chunk, stream=stream)
+                        i += 1
+            res = {"calls": n_chunks * wl.GDN_LAYERS}
             frames = n_chunks * 3
-            extras[f"stack_32x15_{smode}"] = {"ms": stack_ms,
-                                              "latent_frames_per_s": frames / (stack_ms / 1000.0),
-                                              "calls": n_chunks * wl.GDN_LAYERS,
-                                              "timing": "direct calls"}
-
-    # ---- per-kernel device times (CUDA events on the launching stream,
-    # recorded by the library around each launch over a loop of direct calls)
-    n_prof = max(3, min(args.steps, 100))
-    import ctypes
-    _lib.check(lib.gdn_profile_begin(int(n_prof * max(1, launches_per_step) + 8)), "gdn_profile_begin")
-    with torch.cuda.stream(stream):
-        for i in range(n_prof):
-            step(i)
-    kms = (ctypes.c_float * 4)()
-    kn = (ctypes.c_int * 4)()
-    _lib.check(lib.gdn_profile_end(ctypes.addressof(kms), ctypes.addressof(kn), 4), "gdn_profile_end")
-    kernels = {}
-    for i in range(4):
-        if kn[i]:
-            name = lib.gdn_kernel_name(i).decode()
-            kernels[name] = {"launches": kn[i], "ms_per_launch": kms[i] / kn[i]}
-    tot = sum(v["ms_per_launch"] for v in kernels.values())
-    for v in kernels.values():
-        v["share"] = v["ms_per_launch"] / tot if tot else None
-
-    # ---- roofline of the dominant kernel
-    peaks, peak_kind = load_peaks()
-    bytes_step = algorithmic_bytes(w)
-    flops_step = algorithmic_flops(w, w.mode == "bidir")
-    dom = max(kernels, key=lambda k: kernels[k]["ms_per_launch"])
-    dom_bytes = kernel_algorithmic_bytes(dom, w)
-    dom_ms = kernels[dom]["ms_per_launch"]
-    achieved = dom_bytes / (dom_ms / 1000.0) / 1e9
-    path_achieved = bytes_step / (ms_per_step / 1000.0) / 1e9
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": recorded_traffic(dom),
-                "peak_source": f"{peak_kind} hbm_gbs", "kernel": dom,
-                "algorithmic_bytes_per_launch": dom_bytes, "ms_per_launch": dom_ms,
-                "kernels": kernels,
-                "path": {"algorithmic_bytes": bytes_step, "achieved": path_achieved,
-                         "frac": path_achieved / peaks["hbm_gbs"],
-                         "algorithmic_flops": flops_step,
-                         "achieved_tflops": flops_step / (ms_per_step / 1000.0) / 1e12,
-                         "tensor_frac_of_sustained": (flops_step / (ms_per_step / 1000.0) / 1e12)
-                         / peaks["bf16_tflops_sustained"]}}
+            with nvtx(f"stack_{smode}"), torch.cuda.stream(stream):
+                stack_calls()
+                barrier()
+                b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                b0.record(stream)
+                stack_calls()
+                b1.record(stream)
+                barrier()
+                res["direct_ms"] = b0.elapsed_time(b1)
+                res["direct_latent_frames_per_s"] = frames / (res["direct_ms"] / 1000.0)
+                if use_graph:
+                    gs = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(gs, stream=stream):
+                        stack_calls()
+                    for _ in range(2):
+                        gs.replay()
+                    barrier()
+                    b0.record(stream)
+                    reps = 3
+                    for _ in range(reps):
+                        gs.replay()
+                    b1.record(stream)
+                    barrier()
+                    res["graph_ms"] = b0.elapsed_time(b1) / reps
+                    res["graph_latent_frames_per_s"] = frames / (res["graph_ms"] / 1000.0)
+                    del gs
+            ws = wl.stream_chunk("bidir" if smode == "bidir" else "fwd")
+            res["bound_latent_frames_per_s"] = frames / (res["calls"] * max(
+                roofline_times(ws, smode == "bidir", peaks)))
+            extras[f"stack_32x15_{smode}"] = res
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, args.cpu_seconds)
+        with nvtx("cpu_baseline"):
+            cpu = cpu_baseline(w, args.cpu_seconds)
 
     if world > 1:
         dist.barrier(device_ids=[local])
-        graphs.clear()
         dist.destroy_process_group()
     if rank != 0:
         return 0
@@ -573,8 +659,11 @@ def main():
         "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "Dk": w.Dk, "Dv": w.Dv,
                    "chunk": w.chunk, "mode": w.mode, "io": "bf16 q/k/v/out, fp32 g/beta/state",
                    "l2": f"inputs rotate over {N_SETS} sets of "
-                         f"{bytes_step / 1e6:.1f} MB ({N_SETS * bytes_step / 1e6:.0f} MB > 126 MB L2)",
-                   "graph": use_graph, "parallelism": f"replicas x{world} (independent chunk streams)"},
+                         f"{algorithmic_bytes(w) / 1e6:.1f} MB "
+                         f"({N_SETS * algorithmic_bytes(w) / 1e6:.0f} MB > 126 MB L2)",
+                   "graph": use_graph,
+                   "warmup_replays": max(3, args.warmup, N_SETS) if use_graph else max(3, args.warmup),
+                   "parallelism": f"replicas x{world} (independent chunk streams)"},
         "latent_frames_per_s": value / (w.B * w.H * 880),
         "roofline": roofline,
         "cpu_baseline": cpu,

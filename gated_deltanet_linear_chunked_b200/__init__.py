@@ -7,12 +7,13 @@ is loaded on the first call.
 """
 from . import workloads  # noqa: F401
 
-__all__ = ["chunk_fwd", "chunk_bidir", "state_reset", "device_error",
-           "set_wait_limit", "GDNError", "workloads"]
+_API = ("chunk_fwd", "chunk_bidir", "state_reset", "device_error", "set_wait_limit",
+        "workspace_release")
+__all__ = [*_API, "GDNError", "workloads"]
 
 
 def __getattr__(name):
-    if name in ("chunk_fwd", "chunk_bidir", "state_reset", "device_error", "set_wait_limit"):
+    if name in _API:
         from . import api
         return getattr(api, name)
     if name == "GDNError":

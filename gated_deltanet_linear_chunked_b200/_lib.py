@@ -32,6 +32,7 @@ SIGNATURES = {
     "gdn_chunk_fwd_noalloc": (ctypes.c_int, _SCAN_ARGS),
     "gdn_state_reset": (ctypes.c_int, [_fp, _i, _i, _i, _i, _vp]),
     "gdn_device_error": (ctypes.c_int, [_vp]),
+    "gdn_workspace_release": (ctypes.c_int, []),
     "gdn_set_wait_limit": (ctypes.c_longlong, [_ll]),
     "gdn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "gdn_version": (ctypes.c_int, []),

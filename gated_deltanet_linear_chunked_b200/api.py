@@ -102,6 +102,13 @@ def device_error(stream=None) -> int:
     return int(_lib.load().gdn_device_error(_stream(stream)))
 
 
+def workspace_release() -> None:
+    """Free the library's per-stream scratch and error words on the current
+    device (after synchronising it).  No captured graph holding this
+    library's launches may be replayed afterwards."""
+    _lib.check(_lib.load().gdn_workspace_release(), "gdn_workspace_release")
+
+
 def set_wait_limit(polls: int) -> int:
     """Polls a kernel's bounded wait makes before giving up (0 = default)."""
     return int(_lib.load().gdn_set_wait_limit(int(polls)))

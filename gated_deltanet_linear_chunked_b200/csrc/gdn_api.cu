@@ -1,23 +1,41 @@
 // gdn_api.cu -- the C ABI (include/gdn.h): host-side validation and dispatch.
 //
-// Every entry point validates its arguments on the host before enqueueing
+// Every entry point validates its arguments on the host before it enqueues
 // anything, then launches onto the caller's stream and returns without
 // synchronising.  Nothing here throws, aborts or prints.
+//
+// Per-stream context.  The chunked path needs scratch between its kernels,
+// and every bounded wait needs a word to report an expiry in.  Both are kept
+// per (device, stream): the first call on a stream allocates them
+// (cudaMalloc), later calls reuse them, and a larger problem replaces the
+// scratch with a larger one.  Calls on one stream are ordered, so they can
+// share the scratch; calls on different streams never share anything.  A
+// replaced scratch buffer is not freed (a captured CUDA graph may still name
+// it) until gdn_workspace_release.  A call made while its stream is being
+// captured, on a stream with no context yet or with too small a scratch,
+// cannot allocate outside the graph: it falls back to a stream-ordered
+// allocation (captured as graph memory nodes) and to the device-wide error
+// word.
 #include <cuda_runtime.h>
 
 #include <atomic>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <functional>
 #include <mutex>
 #include <new>
+#include <thread>
+#include <vector>
 
 #include "gdn_internal.h"
 
 namespace gdn {
 namespace {
 
-// Device error word set by kernels whose bounded waits expire.
+// Device-wide error word: used by calls without a per-stream context (the
+// allocation-free entry point, and calls captured before their stream had a
+// context).
 __device__ unsigned int g_error_word;
 
 constexpr long long kDefaultWaitLimit = 1LL << 26;
@@ -29,7 +47,7 @@ constexpr int kMaxDevices = 64;
 std::mutex g_err_mu;
 unsigned int* g_err_ptr[kMaxDevices] = {};
 
-// Device address of the error word on the current device.
+// Device address of the device-wide error word on the current device.
 cudaError_t error_word(unsigned int** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -85,20 +103,103 @@ gdn_status check_device_pointer(const void* p, int dev) {
   return GDN_OK;
 }
 
-gdn_status finish(cudaStream_t s, cudaError_t launch_err, unsigned int* err) {
-  if (launch_err != cudaSuccess) return GDN_ERR_CUDA;
-  if (!debug_sync()) return GDN_OK;
-  if (cudaStreamSynchronize(s) != cudaSuccess) return GDN_ERR_CUDA;
-  if (err) {
-    unsigned int word = 0;
-    if (cudaMemcpy(&word, err, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
-      return GDN_ERR_CUDA;
-    if (word != kErrNone) {
-      const unsigned int zero = 0;
-      cudaMemcpy(err, &zero, sizeof(zero), cudaMemcpyHostToDevice);
-      return GDN_ERR_TIMEOUT;
+// Reads and clears one error word; GDN_ERR_TIMEOUT if it was set.
+gdn_status take_error(unsigned int* err) {
+  unsigned int word = 0;
+  if (cudaMemcpy(&word, err, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return GDN_ERR_CUDA;
+  }
+  if (word == kErrNone) return GDN_OK;
+  const unsigned int zero = 0;
+  if (cudaMemcpy(err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) {
+    cudaGetLastError();
+    return GDN_ERR_CUDA;
+  }
+  return GDN_ERR_TIMEOUT;
+}
+
+// ------------------------------------------------------ per-stream contexts
+struct StreamCtx {
+  int dev;
+  cudaStream_t stream;
+  size_t thread;        // owning host thread for the per-thread default stream, else 0
+  unsigned int* err;    // error word of this stream's calls
+  void* ws;             // chunked-path scratch
+  size_t ws_bytes;
+};
+
+std::mutex g_ctx_mu;
+std::vector<StreamCtx*> g_ctx;
+struct Retired {
+  int dev;
+  void* p;
+};
+std::vector<Retired> g_retired;  // scratch buffers replaced by larger ones
+
+size_t thread_key(cudaStream_t s) {
+  if (s != cudaStreamPerThread) return 0;
+  return std::hash<std::thread::id>()(std::this_thread::get_id()) | 1u;
+}
+
+bool capturing(cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  const cudaError_t e = cudaStreamIsCapturing(s, &cs);
+  if (e != cudaSuccess) {  // e.g. the legacy stream while another stream captures
+    cudaGetLastError();
+    return true;
+  }
+  return cs != cudaStreamCaptureStatusNone;
+}
+
+// The error word and scratch of (dev, s), the context created or its scratch
+// grown to at least `bytes` as needed.  Both are copied out under the lock.
+// Sets them to nullptr (and returns GDN_OK) when the stream is being captured
+// and its context cannot serve the call as it is.
+gdn_status stream_context(int dev, cudaStream_t s, size_t bytes, unsigned int** err,
+                          void** ws) {
+  *err = nullptr;
+  *ws = nullptr;
+  const size_t tk = thread_key(s);
+  std::lock_guard<std::mutex> lock(g_ctx_mu);
+  StreamCtx* c = nullptr;
+  for (StreamCtx* x : g_ctx)
+    if (x->dev == dev && x->stream == s && x->thread == tk) c = x;
+  if (!(c && c->ws_bytes >= bytes)) {
+    if (capturing(s)) return GDN_OK;
+    if (!c) {
+      void* p = nullptr;
+      if (cudaMalloc(&p, 256) != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_CUDA;
+      }
+      if (cudaMemsetAsync(p, 0, 256, s) != cudaSuccess) {
+        cudaGetLastError();
+        cudaFree(p);
+        return GDN_ERR_CUDA;
+      }
+      c = new (std::nothrow) StreamCtx{dev, s, tk, static_cast<unsigned int*>(p), nullptr, 0};
+      if (!c) {
+        cudaFree(p);
+        return GDN_ERR_CUDA;
+      }
+      g_ctx.push_back(c);
+    }
+    if (bytes > c->ws_bytes) {
+      const size_t grain = size_t(2) << 20;
+      const size_t nb = (bytes + grain - 1) / grain * grain;
+      void* p = nullptr;
+      if (cudaMalloc(&p, nb) != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_CUDA;
+      }
+      if (c->ws) g_retired.push_back({dev, c->ws});
+      c->ws = p;
+      c->ws_bytes = nb;
     }
   }
+  *err = c->err;
+  *ws = c->ws;
   return GDN_OK;
 }
 
@@ -106,6 +207,49 @@ gdn_status scan(const void* q, const void* k, const void* v, const float* g,
                 const float* beta, const float* state_in, float* state_out,
                 void* out, int B, int T, int H, int Dk, int Dv, gdn_dtype dtype,
                 int chunk, void* stream, bool bidir) {
+  ScanArgs a;
+  int dev = 0;
+  gdn_status st = prepare_scan(q, k, v, g, beta, state_in, state_out, out, B, T, H, Dk, Dv,
+                               dtype, chunk, stream, bidir, &a, &dev);
+  if (st != GDN_OK) return st;
+  if (a.B == 0 || a.H == 0) return GDN_OK;
+  if (a.T == 0) return trivial_state_copy(a);
+
+  const size_t bytes =
+      dtype == GDN_BF16 ? chunk_tc_workspace_bytes(B, T, H, Dk, Dv, bidir) : 0;
+  void* ws = nullptr;
+  st = stream_context(dev, a.stream, bytes, &a.err, &ws);
+  if (st != GDN_OK) return st;
+  if (!a.err && error_word(&a.err) != cudaSuccess) {
+    cudaGetLastError();
+    return GDN_ERR_CUDA;
+  }
+  a.wait_limit = g_wait_limit.load();
+
+  cudaError_t e;
+  if (dtype == GDN_F32) {
+    e = launch_scan_serial(a);
+  } else if (ws) {
+    e = launch_chunk_tc(a, ws);
+  } else {
+    // under capture without a large enough cached scratch: stream-ordered
+    // allocation, captured as graph memory nodes
+    e = cudaMallocAsync(&ws, bytes, a.stream);
+    if (e == cudaSuccess) {
+      e = launch_chunk_tc(a, ws);
+      const cudaError_t f = cudaFreeAsync(ws, a.stream);
+      if (e == cudaSuccess) e = f;
+    }
+  }
+  return finish(a.stream, e, a.err);
+}
+
+}  // namespace
+
+gdn_status prepare_scan(const void* q, const void* k, const void* v, const float* g,
+                        const float* beta, const float* state_in, float* state_out,
+                        void* out, int B, int T, int H, int Dk, int Dv, gdn_dtype dtype,
+                        int chunk, void* stream, bool bidir, ScanArgs* a, int* dev_out) {
   // ---- pure host checks (no CUDA call)
   if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
   if (B < 0 || T < 0 || H < 0 || Dk < 0 || Dv < 0) return GDN_ERR_INVALID_ARG;
@@ -113,6 +257,15 @@ gdn_status scan(const void* q, const void* k, const void* v, const float* g,
   if (chunk != 0 && chunk != 16 && chunk != 32 && chunk != 64)
     return GDN_ERR_INVALID_ARG;
   if (chunk == 0) chunk = 64;
+
+  a->q = q; a->k = k; a->v = v; a->g = g; a->beta = beta;
+  a->state_in = state_in; a->state_out = state_out; a->out = out;
+  a->B = B; a->T = T; a->H = H; a->Dk = Dk; a->Dv = Dv;
+  a->dtype = dtype; a->chunk = chunk; a->bidir = bidir;
+  a->stream = static_cast<cudaStream_t>(stream);
+  a->err = nullptr;
+  a->wait_limit = 0;
+  *dev_out = 0;
   if (B == 0 || H == 0) return GDN_OK;
 
   const size_t es = dtype == GDN_BF16 ? 2 : 4;
@@ -149,46 +302,34 @@ gdn_status scan(const void* q, const void* k, const void* v, const float* g,
     const gdn_status st = check_device_pointer(p, dev);
     if (st != GDN_OK) return st;
   }
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaGetLastError();  // start from a clean launch-error state
-
-  if (T == 0) {
-    if (!state_out) return GDN_OK;
-    cudaError_t e = cudaSuccess;
-    if (!state_in) e = cudaMemsetAsync(state_out, 0, state_bytes, s);
-    else if (state_in != state_out)
-      e = cudaMemcpyAsync(state_out, state_in, state_bytes, cudaMemcpyDeviceToDevice, s);
-    return finish(s, e, nullptr);
-  }
-
-  unsigned int* err = nullptr;
-  if (error_word(&err) != cudaSuccess) return GDN_ERR_CUDA;
-
-  ScanArgs a;
-  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta;
-  a.state_in = state_in; a.state_out = state_out; a.out = out;
-  a.B = B; a.T = T; a.H = H; a.Dk = Dk; a.Dv = Dv;
-  a.dtype = dtype; a.chunk = chunk; a.bidir = bidir; a.stream = s;
-  a.err = err; a.wait_limit = g_wait_limit.load();
-
-  cudaError_t e;
-  if (dtype == GDN_F32) {
-    e = launch_scan_serial(a);
-  } else {
-    // bf16: chunked tensor-core path with stream-ordered scratch
-    void* ws = nullptr;
-    const size_t bytes = chunk_tc_workspace_bytes(B, T, H, Dk, Dv, bidir);
-    e = cudaMallocAsync(&ws, bytes, s);
-    if (e == cudaSuccess) {
-      e = launch_chunk_tc(a, ws);
-      const cudaError_t f = cudaFreeAsync(ws, s);
-      if (e == cudaSuccess) e = f;
-    }
-  }
-  return finish(s, e, err);
+  *dev_out = dev;
+  return GDN_OK;
 }
 
-}  // namespace
+gdn_status trivial_state_copy(const ScanArgs& a) {
+  if (!a.state_out) return GDN_OK;
+  const size_t state_bytes = (size_t)a.B * a.H * a.Dk * a.Dv * sizeof(float);
+  cudaError_t e = cudaSuccess;
+  if (!a.state_in)
+    e = cudaMemsetAsync(a.state_out, 0, state_bytes, a.stream);
+  else if (a.state_in != a.state_out)
+    e = cudaMemcpyAsync(a.state_out, a.state_in, state_bytes, cudaMemcpyDeviceToDevice, a.stream);
+  return finish(a.stream, e, nullptr);
+}
+
+gdn_status finish(cudaStream_t s, cudaError_t launch_err, unsigned int* err) {
+  if (launch_err != cudaSuccess) {
+    cudaGetLastError();
+    return GDN_ERR_CUDA;
+  }
+  if (!debug_sync()) return GDN_OK;
+  if (cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return GDN_ERR_CUDA;
+  }
+  return err ? take_error(err) : GDN_OK;
+}
 
 void count_launches(unsigned n) { g_launches.fetch_add(n); }
 
@@ -261,17 +402,67 @@ gdn_status gdn_state_reset(float* state, int B, int H, int Dk, int Dv,
 
 gdn_status gdn_device_error(void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaStreamSynchronize(s) != cudaSuccess) return GDN_ERR_CUDA;
-  unsigned int* err = nullptr;
-  if (gdn::error_word(&err) != cudaSuccess) return GDN_ERR_CUDA;
-  unsigned int word = 0;
-  if (cudaMemcpy(&word, err, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+  if (cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
     return GDN_ERR_CUDA;
-  if (word == gdn::kErrNone) return GDN_OK;
-  const unsigned int zero = 0;
-  if (cudaMemcpy(err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
     return GDN_ERR_CUDA;
-  return GDN_ERR_TIMEOUT;
+  }
+  unsigned int* own = nullptr;
+  {
+    const size_t tk = gdn::thread_key(s);
+    std::lock_guard<std::mutex> lock(gdn::g_ctx_mu);
+    for (const gdn::StreamCtx* c : gdn::g_ctx)
+      if (c->dev == dev && c->stream == s && c->thread == tk) own = c->err;
+  }
+  unsigned int* shared = nullptr;
+  if (gdn::error_word(&shared) != cudaSuccess) {
+    cudaGetLastError();
+    return GDN_ERR_CUDA;
+  }
+  const gdn_status a = own ? gdn::take_error(own) : GDN_OK;
+  const gdn_status b = gdn::take_error(shared);
+  if (a == GDN_ERR_CUDA || b == GDN_ERR_CUDA) return GDN_ERR_CUDA;
+  return (a == GDN_ERR_TIMEOUT || b == GDN_ERR_TIMEOUT) ? GDN_ERR_TIMEOUT : GDN_OK;
+}
+
+gdn_status gdn_workspace_release(void) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return GDN_ERR_CUDA;
+  }
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    return GDN_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(gdn::g_ctx_mu);
+  gdn_status st = GDN_OK;
+  std::vector<gdn::StreamCtx*> keep;
+  for (gdn::StreamCtx* c : gdn::g_ctx) {
+    if (c->dev != dev) {
+      keep.push_back(c);
+      continue;
+    }
+    if (c->ws && cudaFree(c->ws) != cudaSuccess) st = GDN_ERR_CUDA;
+    if (c->err && cudaFree(c->err) != cudaSuccess) st = GDN_ERR_CUDA;
+    delete c;
+  }
+  gdn::g_ctx.swap(keep);
+  std::vector<gdn::Retired> left;
+  for (const gdn::Retired& r : gdn::g_retired) {
+    if (r.dev != dev) {
+      left.push_back(r);
+      continue;
+    }
+    if (cudaFree(r.p) != cudaSuccess) st = GDN_ERR_CUDA;
+  }
+  gdn::g_retired.swap(left);
+  if (st != GDN_OK) cudaGetLastError();
+  return st;
 }
 
 long long gdn_set_wait_limit(long long polls) {
@@ -292,7 +483,7 @@ const char* gdn_status_string(gdn_status status) {
   return "GDN_ERR_UNKNOWN";
 }
 
-int gdn_version(void) { return 100; }
+int gdn_version(void) { return 200; }
 
 unsigned long long gdn_launch_count(void) { return gdn::g_launches.load(); }
 

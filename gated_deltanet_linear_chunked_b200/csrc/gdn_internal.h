@@ -47,8 +47,27 @@ class ProfileScope {
   int slot_;
 };
 
-// Device address of the error word on the current device, and the poll
-// limit handed to bounded waits.
+// Every check gdn.h lists for a scan call (host checks first, then device
+// residency of each pointer on the current device).  On GDN_OK `a` holds the
+// validated call (chunk defaulted; err and wait_limit not yet set) and `*dev`
+// the current device.  B == 0 or H == 0 returns GDN_OK with a->B or a->H
+// zero: the caller has nothing to do.
+gdn_status prepare_scan(const void* q, const void* k, const void* v, const float* g,
+                        const float* beta, const float* state_in, float* state_out,
+                        void* out, int B, int T, int H, int Dk, int Dv, gdn_dtype dtype,
+                        int chunk, void* stream, bool bidir, ScanArgs* a, int* dev);
+
+// T == 0: state_out = state_in (or zero); out untouched.
+gdn_status trivial_state_copy(const ScanArgs& a);
+
+// Maps a launch result to a status.  With GDN_DEBUG_SYNC set in the
+// environment it also synchronises the stream and reads (and clears) the
+// error word `err`, returning GDN_ERR_TIMEOUT if a bounded wait expired.
+gdn_status finish(cudaStream_t s, cudaError_t launch_err, unsigned int* err);
+
+// Device address of the device-wide error word on the current device (used by
+// calls that have no per-stream context), and the poll limit handed to
+// bounded waits.
 cudaError_t current_error_word(unsigned int** out);
 long long current_wait_limit();
 

@@ -48,6 +48,8 @@ class Workload:
     beta: tuple           # ("sigmoid",) or ("const", value)
     state: tuple          # ("zero",) or ("normal", std)
     seed: int
+    qk: tuple = ("unit",)  # ("unit",): rows L2-normalised; ("raw",): N(0,1) rows;
+                           # ("mixed",): N(0,1) rows with special rows (see qk_rows)
 
     @property
     def head_tokens(self) -> int:
@@ -117,11 +119,45 @@ def _l2_rows(x: np.ndarray) -> np.ndarray:
     return (x / np.linalg.norm(x, axis=-1, keepdims=True)).astype(np.float32)
 
 
+# Row scales of the ("mixed",) q/k recipe, which exercises the library's own
+# L2 normalisation: rows at tiny and huge magnitudes, rows whose squared norm
+# falls under the 1e-12 clamp, and all-zero rows.
+MIXED_SMALL, MIXED_LARGE, MIXED_SUBCLAMP = 1e-3, 1e3, 3e-8
+
+
+def qk_rows(T: int) -> dict:
+    """Token indices of the special rows of the ("mixed",) recipe, the same
+    for every head: q/k rows scaled by 1e-3 and 1e3, rows scaled by 3e-8
+    (squared norm about 1e-13, under the clamp), one all-zero q row and one
+    all-zero k row."""
+    t = np.arange(T)
+    return {"small": t[t % 7 == 3], "large": t[(t % 11 == 5) & (t % 7 != 3)],
+            "subclamp": t[(t % 13 == 8) & (t % 7 != 3) & (t % 11 != 5)],
+            "zero_q": np.array([T // 2]) if T >= 2 else np.array([], int),
+            "zero_k": np.array([T // 3]) if T >= 3 else np.array([], int)}
+
+
+def _shape_qk(x: np.ndarray, recipe: tuple, is_q: bool) -> np.ndarray:
+    if recipe[0] == "unit":
+        return _l2_rows(x)
+    if recipe[0] == "raw":
+        return x
+    if recipe[0] == "mixed":
+        rows = qk_rows(x.shape[0])
+        x = x.copy()
+        x[rows["small"]] *= np.float32(MIXED_SMALL)
+        x[rows["large"]] *= np.float32(MIXED_LARGE)
+        x[rows["subclamp"]] *= np.float32(MIXED_SUBCLAMP)
+        x[rows["zero_q" if is_q else "zero_k"]] = 0.0
+        return x
+    raise ValueError(recipe)
+
+
 def make_head(w: Workload, b: int, h: int) -> dict:
     """Inputs of one (batch, head) pair: q, k [T,Dk]; v [T,Dv]; g, beta [T]."""
     rng = np.random.default_rng([w.seed, b, h])
-    q = _l2_rows(rng.standard_normal((w.T, w.Dk), dtype=np.float32))
-    k = _l2_rows(rng.standard_normal((w.T, w.Dk), dtype=np.float32))
+    q = _shape_qk(rng.standard_normal((w.T, w.Dk), dtype=np.float32), w.qk, True)
+    k = _shape_qk(rng.standard_normal((w.T, w.Dk), dtype=np.float32), w.qk, False)
     v = rng.standard_normal((w.T, w.Dv), dtype=np.float32)
     if w.gate[0] == "neg_softplus":
         z = rng.standard_normal(w.T, dtype=np.float32).astype(np.float64)

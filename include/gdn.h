@@ -26,13 +26,23 @@
  *   state      [B, H, Dk, Dv]  float
  *
  * Ownership.  The caller owns every buffer; all pointers are device (or
- * managed) pointers.  The library keeps no pointer after a call returns.
- * Internal scratch, when a path needs it, is allocated and freed
- * stream-ordered on `stream` (cudaMallocAsync / cudaFreeAsync).
+ * managed) pointers.  The library keeps no pointer to a caller's buffer after
+ * a call returns.  It keeps, per (device, stream), one small context: the
+ * scratch the bf16 path passes between its kernels and an error word.  The
+ * first call on a stream allocates it (cudaMalloc), a larger problem grows
+ * it, and gdn_workspace_release frees it.  Calls on one stream share their
+ * context (they are ordered); calls on different streams share nothing.  A
+ * call made while its stream is being captured into a CUDA graph cannot
+ * allocate outside the graph: if the stream has no context yet, or too small
+ * a scratch, the call allocates stream-ordered (cudaMallocAsync /
+ * cudaFreeAsync, captured as graph memory nodes) and reports through the
+ * device-wide error word.  Make one call on a stream before capturing on it
+ * to keep memory nodes out of the graph.
  *
  * Execution.  Work is enqueued on `stream` (a cudaStream_t; NULL is the
  * legacy default stream) and the call returns without synchronising;
- * results are stream-ordered.  No call throws, aborts or prints.
+ * results are stream-ordered.  No call throws, aborts or prints.  Calls may
+ * come from several host threads at once.
  *
  * Errors.  Arguments are validated on the host before anything is enqueued;
  * on any error nothing is launched and a status is returned:
@@ -44,8 +54,10 @@
  *                        overlaps an input or partially overlaps state_in
  *   GDN_ERR_CUDA         a CUDA runtime call or a launch failed
  *   GDN_ERR_TIMEOUT      a kernel's bounded wait expired (reported by
- *                        gdn_device_error, or by the calls themselves when
- *                        the environment sets GDN_DEBUG_SYNC=1)
+ *                        gdn_device_error for the stream it ran on, or by
+ *                        the calls themselves when the environment sets
+ *                        GDN_DEBUG_SYNC=1: every scan entry point then
+ *                        synchronises its stream before it returns)
  *   GDN_ERR_SCRATCH_LIMIT  (gdn_chunk_fwd_noalloc only) the problem needs more
  *                        scratch than its fixed device array holds
  */
@@ -134,7 +146,10 @@ GDN_API gdn_status gdn_chunk_bidir(const void* q, const void* k, const void* v,
  * and it keeps the last call's contents (every scratch byte a call reads was
  * written earlier in the same call, so nothing needs clearing); calls whose
  * work overlaps on the GPU -- two streams, or two host threads -- race on it,
- * so order them on one stream.
+ * so order them on one stream.  Argument checks and statuses are those of
+ * gdn_chunk_fwd.  A bounded wait that expires is reported through the
+ * device-wide error word (gdn_device_error on any stream of the device), or
+ * by the call itself when GDN_DEBUG_SYNC=1.
  */
 #define GDN_NOALLOC_SCRATCH_BYTES (96ull << 20)
 GDN_API gdn_status gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
@@ -152,16 +167,30 @@ GDN_API gdn_status gdn_state_reset(float* state, int B, int H, int Dk, int Dv,
                            void* stream);
 
 /*
- * Synchronise `stream`, then read and clear the device error word that
- * kernels set when a bounded wait expires.  Returns GDN_OK, GDN_ERR_TIMEOUT
- * or GDN_ERR_CUDA.
+ * Synchronise `stream`, then read and clear the error words that kernels set
+ * when a bounded wait expires: the stream's own word (calls made on this
+ * stream) and the current device's device-wide word (calls of
+ * gdn_chunk_fwd_noalloc and calls captured before the stream had a
+ * context).  Returns GDN_OK, GDN_ERR_TIMEOUT or GDN_ERR_CUDA.  A timeout of
+ * a call on another stream is not reported here.
  */
 GDN_API gdn_status gdn_device_error(void* stream);
 
 /*
+ * Free every per-stream context (scratch and error word) the library holds
+ * on the current device, after synchronising the device.  Call it only when
+ * no captured CUDA graph that contains this library's launches will be
+ * replayed again: such a graph names the freed scratch.  Later calls create
+ * new contexts.  Returns GDN_OK or GDN_ERR_CUDA.
+ */
+GDN_API gdn_status gdn_workspace_release(void);
+
+/*
  * Test hook: the number of polls a kernel's bounded wait makes before it
  * gives up (0 restores the default).  Affects launches enqueued after the
- * call, on every device.  Returns the previous value.
+ * call, on every device and stream: it is one process-wide setting, meant
+ * for fault-injection tests, not for production tuning.  Returns the
+ * previous value.
  */
 GDN_API long long gdn_set_wait_limit(long long polls);
 

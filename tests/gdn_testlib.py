@@ -26,6 +26,39 @@ def max_rel(x, ref) -> float:
     return float(np.max(np.abs(x - ref)) / den)
 
 
+def max_rel_per_head(x, ref, head_axes) -> float:
+    """The largest per-head max relative error: the metric taken separately
+    over each (b, h) slice, so a wrong head of small magnitude cannot hide
+    under another head's maximum.  `head_axes` are the (b, h) axes of the
+    tensor: (0, 2) for outputs [B,T,H,D], (0, 1) for states [B,H,Dk,Dv]."""
+    x = np.asarray(x, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert x.shape == ref.shape, (x.shape, ref.shape)
+    ab, ah = head_axes
+    worst = 0.0
+    for b in range(x.shape[ab]):
+        for h in range(x.shape[ah]):
+            idx = [slice(None)] * x.ndim
+            idx[ab], idx[ah] = b, h
+            worst = max(worst, max_rel(x[tuple(idx)], ref[tuple(idx)]))
+    return worst
+
+
+def max_rel_rows(x, ref, rows) -> float:
+    """Largest error over the given token rows of an output [B,T,H,D],
+    relative to each (b, h, row)'s own largest reference value: rows whose
+    reference is tiny or huge are judged on their own scale."""
+    x = np.asarray(x, np.float64)[:, rows]
+    ref = np.asarray(ref, np.float64)[:, rows]
+    den = np.max(np.abs(ref), axis=-1)
+    num = np.max(np.abs(x - ref), axis=-1)
+    ok = den > 0
+    worst = float(np.max(num[ok] / den[ok])) if ok.any() else 0.0
+    if (~ok).any():
+        worst = max(worst, float(np.max(num[~ok])))
+    return worst
+
+
 def torch_dtype(w: wl.Workload):
     return torch.bfloat16 if w.dtype == "bf16" else torch.float32
 

@@ -46,6 +46,32 @@ def test_wait_expiry_reports_timeout_and_context_survives():
     assert max_rel(to_np(S), ref_S) <= TOL["bf16"]
 
 
+def test_error_words_are_per_stream():
+    """An expired wait on one stream is reported on that stream only: a
+    second stream's calls, before and after, see GDN_OK."""
+    w = small_workload()
+    x = device_inputs(w)
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    for s in (s1, s2):  # give both streams their context before the fault injection
+        gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state_in"], stream=s)
+        assert gdn.device_error(s) == _lib.GDN_OK
+    gdn.set_wait_limit(1)
+    try:
+        gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state_in"], stream=s1)
+        s1.synchronize()
+    finally:
+        gdn.set_wait_limit(0)
+    out2, S2 = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state_in"], stream=s2)
+    assert gdn.device_error(s2) == _lib.GDN_OK
+    assert gdn.device_error(s1) == _lib.GDN_ERR_TIMEOUT
+    assert gdn.device_error(s1) == _lib.GDN_OK
+    torch.cuda.synchronize()
+    ref_o, ref_S = oracle_run(w, host_inputs(w))
+    assert max_rel(to_np(out2), ref_o) <= TOL["bf16"]
+    assert max_rel(to_np(S2), ref_S) <= TOL["bf16"]
+
+
 def test_profile_hook_counts_each_kernel():
     w = small_workload()
     x = device_inputs(w)

@@ -11,7 +11,8 @@ import torch
 import gated_deltanet_linear_chunked_b200 as gdn
 from gated_deltanet_linear_chunked_b200 import workloads as wl
 
-from gdn_testlib import TOL, device_inputs, host_inputs, max_rel, oracle_head, oracle_run, to_np
+from gdn_testlib import (TOL, device_inputs, host_inputs, max_rel, max_rel_per_head, max_rel_rows,
+                         oracle_head, oracle_run, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -35,12 +36,18 @@ def dev_from_host(x, dtype):
     return d
 
 
-def check(w, x_host, out, S, bidir=None):
+def check(w, x_host, out, S, bidir=None, per_head=False):
+    """Element-wise comparison with the oracle at the dtype's tolerance, on
+    the whole tensors and, with per_head, on every (b, h) head alone."""
     ref_o, ref_S = oracle_run(w, x_host, bidir)
-    eo, es = max_rel(to_np(out), ref_o), max_rel(to_np(S), ref_S)
+    o, s = to_np(out), to_np(S)
+    eo, es = max_rel(o, ref_o), max_rel(s, ref_S)
     tol = TOL[w.dtype]
     assert eo <= tol and es <= tol, f"{w.name}: out {eo:.3e} state {es:.3e} tol {tol}"
-    return eo, es
+    if per_head:
+        ho, hs = max_rel_per_head(o, ref_o, (0, 2)), max_rel_per_head(s, ref_S, (0, 1))
+        assert ho <= tol and hs <= tol, f"{w.name}: per head out {ho:.3e} state {hs:.3e} tol {tol}"
+    return ref_o, ref_S
 
 
 @pytest.mark.parametrize("mode", ["fwd", "bidir"])
@@ -71,6 +78,21 @@ def test_small_sweep(T, D, mode, dtype):
     check(w, xh, out, S)
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("mode", ["fwd", "bidir"])
+@pytest.mark.parametrize("D", [16, 112, 128])
+@pytest.mark.parametrize("T", [1, 17, 65, 200])
+def test_small_sweep_unnormalised_qk(T, D, mode, dtype):
+    """Ragged lengths and head-dim classes with the mixed un-normalised q/k
+    recipe (rows at 1e-3 / 1e3 / under the clamp, zero rows)."""
+    w = wl.Workload(f"sweepu_T{T}_D{D}", 2, T, 3, D, D, dtype, 64, mode,
+                    ("uniform", -0.5, 0.0), ("sigmoid",), ("normal", 0.02), 71000 + T * 7 + D,
+                    qk=("mixed",))
+    xh = host_inputs(w)
+    out, S = run(w, dev_from_host(xh, torch.bfloat16 if dtype == "bf16" else torch.float32))
+    check(w, xh, out, S, per_head=True)
+
+
 @pytest.mark.parametrize("Dk,Dv", [(32, 96), (128, 16), (64, 128)])
 def test_rectangular_state(Dk, Dv):
     """Dk != Dv (the state is Dk x Dv; outputs are Dv wide)."""
@@ -84,12 +106,41 @@ def test_rectangular_state(Dk, Dv):
 @pytest.mark.parametrize("mode", ["fwd", "bidir"])
 def test_stream_chunk_full_size(mode):
     """The 1280x704 streaming chunk (B1 H20 d112 T2640 bf16), every head
-    compared with the oracle; bidir adds the in-chunk reverse scan."""
+    compared with the oracle, as a whole and head by head; bidir adds the
+    in-chunk reverse scan."""
     w = wl.stream_chunk(mode)
     xh = host_inputs(w)
     x = device_inputs(w)
     out, S = run(w, x)
-    check(w, xh, out, S)
+    check(w, xh, out, S, per_head=True)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("mode", ["fwd", "bidir"])
+@pytest.mark.parametrize("qk", ["raw", "mixed"])
+def test_stream_chunk_unnormalised_qk(qk, mode, dtype):
+    """The streaming chunk's shapes with q and k NOT pre-normalised, so the
+    library's own L2 normalisation (q/|q|, k/|k|, |.|^2 clamped at 1e-12) is
+    what makes the result right: raw N(0,1) rows (norm about sqrt(112)), and
+    the mixed recipe with rows scaled by 1e-3 and 1e3, rows whose squared
+    norm is under the clamp, and an all-zero q row and k row per head.
+    Compared with the oracle on the whole tensors, head by head, and on the
+    special rows each against its own scale."""
+    import dataclasses
+    w = dataclasses.replace(wl.stream_chunk(mode), qk=(qk,), dtype=dtype,
+                            name=f"stream_{mode}_{qk}_{dtype}")
+    xh = host_inputs(w)
+    x = dev_from_host(xh, torch.bfloat16 if dtype == "bf16" else torch.float32)
+    out, S = run(w, x)
+    ref_o, _ = check(w, xh, out, S, per_head=True)
+    if qk == "mixed":
+        rows = wl.qk_rows(w.T)
+        o = to_np(out)
+        for name in ("small", "large", "subclamp", "zero_k"):
+            e = max_rel_rows(o, ref_o, rows[name])
+            assert e <= TOL[dtype], f"{name} rows: {e:.3e}"
+        # an all-zero q row has an all-zero output (q^ = 0)
+        assert not o[:, rows["zero_q"]].any()
 
 
 def test_streaming_equals_one_scan_on_gpu():

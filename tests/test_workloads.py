@@ -116,3 +116,33 @@ def test_rank_streams_differ(mode):
     a = wl.make_head(wl.stream_chunk(mode, seed=10), 0, 0)
     b = wl.make_head(wl.stream_chunk(mode, seed=11), 0, 0)
     assert not np.array_equal(a["q"], b["q"])
+
+
+def test_raw_and_mixed_qk_recipes():
+    """The un-normalised q/k recipes used to exercise the library's own L2
+    normalisation: raw N(0,1) rows (norm about sqrt(d)), and the mixed recipe
+    with rows at 1e-3 and 1e3, rows under the 1e-12 clamp and zero rows."""
+    import dataclasses
+    base = wl.stream_chunk()
+    raw = wl.make_head(dataclasses.replace(base, qk=("raw",)), 0, 3)
+    for n in ("q", "k"):
+        nrm = np.linalg.norm(raw[n].astype(np.float64), axis=-1)
+        assert abs(np.median(nrm) - np.sqrt(112)) < 0.5
+    w = dataclasses.replace(base, qk=("mixed",))
+    d = wl.make_head(w, 0, 3)
+    rows = wl.qk_rows(w.T)
+    r = np.random.default_rng([w.seed, 0, 3])
+    q0 = r.standard_normal((w.T, w.Dk), dtype=np.float32)
+    for name, scale in (("small", 1e-3), ("large", 1e3), ("subclamp", 3e-8)):
+        t = rows[name]
+        assert len(t) > 10
+        got = d["q"][t].astype(np.float64)
+        want = wl.round_bf16(q0[t] * np.float32(scale)).astype(np.float64)
+        assert np.array_equal(got, want), name
+    sq = np.sum(d["q"][rows["subclamp"]].astype(np.float64) ** 2, axis=-1)
+    assert np.all(sq < 1e-12) and np.all(sq > 0)
+    assert not d["q"][rows["zero_q"]].any() and d["q"][rows["zero_k"]].any()
+    assert not d["k"][rows["zero_k"]].any() and d["k"][rows["zero_q"]].any()
+    # the special row sets are disjoint from one another
+    sets = [set(rows[n].tolist()) for n in ("small", "large", "subclamp")]
+    assert not (sets[0] & sets[1]) and not (sets[0] & sets[2]) and not (sets[1] & sets[2])
