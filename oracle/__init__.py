@@ -10,19 +10,30 @@ Contents
   * ``cpu``        -- ctypes front end of ``gdn_oracle.c``: the token-by-token
                       recurrence in double (and long double), threaded over
                       (batch, head).  The reference for every parity test.
+                      Its ``*_logits`` variants take the gate layer's logits
+                      and form g = -softplus(x), beta = sigmoid(y) themselves.
   * ``numpy_ref``  -- the same recurrence in numpy (a second, independent
                       transcription for tiny cases) and the chunked (WY / UT)
                       form of the scan in fp64, used only to pin that the
-                      chunked algebra reaches the recurrence exactly.
+                      chunked algebra reaches the recurrence exactly; and
+                      ``gates_from_logits``, the gate activations in numpy.
 
 Parity is pinned, not assumed: ``tests/test_oracle_pins.py`` checks these
 functions against closed forms, invariants, a hand-derived example and brute
 force (see each test's docstring).
 """
-from .cpu import build, online_cores, oracle_bidir, oracle_fwd  # noqa: F401
+from .cpu import (  # noqa: F401
+    build,
+    online_cores,
+    oracle_bidir,
+    oracle_bidir_logits,
+    oracle_fwd,
+    oracle_fwd_logits,
+)
 from .numpy_ref import (  # noqa: F401
     chunked_bidir,
     chunked_fwd,
+    gates_from_logits,
     recurrence_bidir,
     recurrence_fwd,
 )

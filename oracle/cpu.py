@@ -47,7 +47,8 @@ def _load():
         fp = ctypes.POINTER(ctypes.c_float)
         for suffix, real in (("", ctypes.c_double), ("_ld", ctypes.c_longdouble)):
             rp = ctypes.POINTER(real)
-            for name in ("gdn_oracle_fwd", "gdn_oracle_bidir"):
+            for name in ("gdn_oracle_fwd", "gdn_oracle_bidir", "gdn_oracle_fwd_logits",
+                         "gdn_oracle_bidir_logits"):
                 fn = getattr(lib, name + suffix)
                 fn.restype = ctypes.c_int
                 fn.argtypes = [fp, fp, fp, fp, fp, rp, rp, rp] + [ctypes.c_int] * 6
@@ -68,7 +69,7 @@ def _f32(x, shape, name):
     return a
 
 
-def _run(bidir, q, k, v, g, beta, state_in, nthreads, precision):
+def _run(bidir, q, k, v, g, beta, state_in, nthreads, precision, logits=False):
     q = np.asarray(q)
     B, T, H, Dk = q.shape
     Dv = np.asarray(v).shape[-1]
@@ -92,7 +93,8 @@ def _run(bidir, q, k, v, g, beta, state_in, nthreads, precision):
     s_out = np.zeros((B, H, Dk, Dv), dtype=real_np)
     out = np.zeros((B, T, H, Dv), dtype=real_np)
     lib = _load()
-    fn = getattr(lib, ("gdn_oracle_bidir" if bidir else "gdn_oracle_fwd") + suffix)
+    name = ("gdn_oracle_bidir" if bidir else "gdn_oracle_fwd") + ("_logits" if logits else "")
+    fn = getattr(lib, name + suffix)
     fp = ctypes.POINTER(ctypes.c_float)
     rp = ctypes.POINTER(real_c)
     rc = fn(q.ctypes.data_as(fp), k.ctypes.data_as(fp), v.ctypes.data_as(fp),
@@ -114,3 +116,17 @@ def oracle_bidir(q, k, v, g, beta, state_in=None, nthreads=0, precision="double"
     """Forward scan from ``state_in`` plus reverse scan from zero, summed;
     the state returned is the forward scan's."""
     return _run(True, q, k, v, g, beta, state_in, nthreads, precision)
+
+
+def oracle_fwd_logits(q, k, v, g_logit, beta_logit, state_in=None, nthreads=0,
+                      precision="double"):
+    """Forward scan whose gates come from the gate layer's logits:
+    g = -softplus(g_logit), beta = sigmoid(beta_logit), both evaluated in the
+    oracle's precision (``gdn_oracle.c``, gate-logit mode)."""
+    return _run(False, q, k, v, g_logit, beta_logit, state_in, nthreads, precision, logits=True)
+
+
+def oracle_bidir_logits(q, k, v, g_logit, beta_logit, state_in=None, nthreads=0,
+                        precision="double"):
+    """Bidirectional scan with gates from logits (as ``oracle_fwd_logits``)."""
+    return _run(True, q, k, v, g_logit, beta_logit, state_in, nthreads, precision, logits=True)

@@ -33,6 +33,13 @@
  * g_t and beta_t, its own term counted in both directions, plain sum);
  * state_out comes from the forward scan only.
  *
+ * Gate-logit mode (the *_logits entry points): the g and beta arrays hold
+ * the gate layer's two logits x_t, y_t instead, and the gates are
+ *   g_t = -softplus(x_t) = -log(1 + e^{x_t}),   beta_t = sigmoid(y_t),
+ * evaluated here in `real`.  The pages name the gate layer (it stays in BF16
+ * under mixed-precision quantisation: same page, 实验结果) but do not write its
+ * activations; these are the plainest maps onto g <= 0 and beta in (0, 1).
+ *
  * Layouts: q, k [B,T,H,Dk]; v, out [B,T,H,Dv]; g, beta [B,T,H];
  * state [B,H,Dk,Dv]; all row-major, contiguous.  Inputs are float (the exact
  * values the device sees, bf16 values are exact in float); outputs are real.
@@ -58,6 +65,7 @@ typedef struct {
   real *state_out, *out;
   int B, T, H, Dk, Dv;
   int bidir;
+  int logits;               /* g, beta hold gate logits */
   int next;                 /* next (b,h) pair to take, guarded by lock */
   pthread_mutex_t lock;
 } job_t;
@@ -69,6 +77,24 @@ static void l2_normalise(const float *x, int n, real *xhat) {
   if (ss < (real)1e-12) ss = (real)1e-12;
   real inv = (real)1 / ORACLE_SQRT(ss);
   for (int i = 0; i < n; ++i) xhat[i] = (real)x[i] * inv;
+}
+
+/* The decay a = e^g and the write strength beta of one token: given
+ * directly, or from the gate logits x, y as a = e^{-softplus(x)}, beta =
+ * sigmoid(y) (each side of the softplus and sigmoid formed without
+ * overflow). */
+static real gate_decay(const job_t *J, size_t row) {
+  const long double x = J->g[row];
+  if (!J->logits) return ORACLE_EXP(x);
+  const long double sp = x > 0 ? x + log1pl(expl(-x)) : log1pl(expl(x));
+  return ORACLE_EXP(-sp);
+}
+static real gate_beta(const job_t *J, size_t row) {
+  const long double y = J->beta[row];
+  if (!J->logits) return (real)y;
+  if (y >= 0) return (real)(1.0L / (1.0L + expl(-y)));
+  const long double e = expl(y);
+  return (real)(e / (1.0L + e));
 }
 
 /* One token of the recurrence: S = a (I - b k k^T) S + b k v^T, then
@@ -117,8 +143,8 @@ static void scan_head(const job_t *J, int b, int h, real *S, real *khat,
     const size_t row = ((size_t)b * T + t) * H + h;
     l2_normalise(J->k + row * Dk, Dk, khat);
     l2_normalise(J->q + row * Dk, Dk, qhat);
-    const real a = ORACLE_EXP(J->g[row]);
-    const real bt = (real)J->beta[row];
+    const real a = gate_decay(J, row);
+    const real bt = gate_beta(J, row);
     token_step(S, khat, qhat, J->v + row * Dv, a, bt, Dk, Dv, x,
                J->out + row * Dv, 0);
   }
@@ -132,8 +158,8 @@ static void scan_head(const job_t *J, int b, int h, real *S, real *khat,
     const size_t row = ((size_t)b * T + t) * H + h;
     l2_normalise(J->k + row * Dk, Dk, khat);
     l2_normalise(J->q + row * Dk, Dk, qhat);
-    const real a = ORACLE_EXP(J->g[row]);
-    const real bt = (real)J->beta[row];
+    const real a = gate_decay(J, row);
+    const real bt = gate_beta(J, row);
     token_step(S, khat, qhat, J->v + row * Dv, a, bt, Dk, Dv, x,
                J->out + row * Dv, 1);
   }
@@ -165,11 +191,11 @@ static void *worker(void *arg) {
 static int run(const float *q, const float *k, const float *v, const float *g,
                const float *beta, const real *state_in, real *state_out,
                real *out, int B, int T, int H, int Dk, int Dv, int bidir,
-               int nthreads) {
+               int logits, int nthreads) {
   if (!q || !k || !v || !g || !beta || !out) return -1;
   if (B < 1 || T < 0 || H < 1 || Dk < 1 || Dv < 1) return -1;
   job_t J = {q, k, v, g, beta, state_in, state_out, out, B, T, H, Dk, Dv,
-             bidir, 0, PTHREAD_MUTEX_INITIALIZER};
+             bidir, logits, 0, PTHREAD_MUTEX_INITIALIZER};
   if (T == 0) {
     if (state_out) {
       const size_t n = (size_t)B * H * Dk * Dv;
@@ -192,23 +218,18 @@ static int run(const float *q, const float *k, const float *v, const float *g,
   return 0;
 }
 
-int ORACLE_SUFFIX(gdn_oracle_fwd)(const float *q, const float *k,
-                                  const float *v, const float *g,
-                                  const float *beta, const real *state_in,
-                                  real *state_out, real *out, int B, int T,
-                                  int H, int Dk, int Dv, int nthreads) {
-  return run(q, k, v, g, beta, state_in, state_out, out, B, T, H, Dk, Dv, 0,
-             nthreads);
-}
-
-int ORACLE_SUFFIX(gdn_oracle_bidir)(const float *q, const float *k,
-                                    const float *v, const float *g,
-                                    const float *beta, const real *state_in,
-                                    real *state_out, real *out, int B, int T,
-                                    int H, int Dk, int Dv, int nthreads) {
-  return run(q, k, v, g, beta, state_in, state_out, out, B, T, H, Dk, Dv, 1,
-             nthreads);
-}
+#define ORACLE_ENTRY(name, bidir, logits)                                      \
+  int ORACLE_SUFFIX(name)(const float *q, const float *k, const float *v,      \
+                          const float *g, const float *beta,                   \
+                          const real *state_in, real *state_out, real *out,    \
+                          int B, int T, int H, int Dk, int Dv, int nthreads) { \
+    return run(q, k, v, g, beta, state_in, state_out, out, B, T, H, Dk, Dv,   \
+               bidir, logits, nthreads);                                       \
+  }
+ORACLE_ENTRY(gdn_oracle_fwd, 0, 0)
+ORACLE_ENTRY(gdn_oracle_bidir, 1, 0)
+ORACLE_ENTRY(gdn_oracle_fwd_logits, 0, 1)
+ORACLE_ENTRY(gdn_oracle_bidir_logits, 1, 1)
 
 int ORACLE_SUFFIX(gdn_oracle_online_cores)(void) {
   return (int)sysconf(_SC_NPROCESSORS_ONLN);

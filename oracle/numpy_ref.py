@@ -43,6 +43,19 @@ from __future__ import annotations
 import numpy as np
 
 
+def gates_from_logits(g_logit, beta_logit):
+    """Gate layer logits -> (g, beta) in fp64: g = -softplus(x) = -log(1 + e^x),
+    beta = sigmoid(y) = 1 / (1 + e^-y).  The pages keep the gate layer in BF16
+    ("SANA-Streaming：基于混合扩散Transformer的实时流式视频编辑系统", 实验结果)
+    without writing its activations; these are the plainest maps onto g <= 0
+    and beta in (0, 1).  A second transcription beside the C oracle's."""
+    x = np.asarray(g_logit, np.float64)
+    y = np.asarray(beta_logit, np.float64)
+    g = -np.logaddexp(0.0, x)
+    beta = np.exp(-np.logaddexp(0.0, -y))
+    return g, beta
+
+
 def _normalise(x):
     ss = np.sum(x * x, axis=-1, keepdims=True)
     return x / np.sqrt(np.maximum(ss, 1e-12))

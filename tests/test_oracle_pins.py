@@ -390,3 +390,140 @@ def test_oracle_planted_sign_error_is_caught():
     # with beta = 1 the right ordering gives S^T k^ = v for any a; the slip gives a v
     np.testing.assert_allclose(ok, v[:, -1], atol=1e-12)
     assert np.max(np.abs(bad - v[:, -1])) > 1e-2
+
+
+# ---------------------------------------------------------------------------
+# Gate activations of the fused prologue (g = -softplus(x), beta = sigmoid(y))
+# ---------------------------------------------------------------------------
+# The pages keep the gate layer in BF16 without writing its activations; the
+# reading taken is g = -softplus(x) (so g <= 0 and a = e^g = 1 / (1 + e^x))
+# and beta = sigmoid(y).  The pins below use only closed forms of those maps.
+
+FWD_LOGITS = {
+    "c": lambda q, k, v, x, y, s=None: oracle.oracle_fwd_logits(q, k, v, x, y, s, nthreads=2),
+    "c_ld": lambda q, k, v, x, y, s=None: oracle.oracle_fwd_logits(q, k, v, x, y, s, nthreads=2,
+                                                                   precision="long double"),
+    "numpy": lambda q, k, v, x, y, s=None: oracle.recurrence_fwd(
+        q, k, v, *oracle.gates_from_logits(x, y), s),
+}
+
+
+def test_gate_maps_closed_forms():
+    """softplus(0) = ln 2 and sigmoid(0) = 1/2; softplus(x) - softplus(-x) = x;
+    sigmoid(y) + sigmoid(-y) = 1; e^{-softplus(x)} = 1 / (1 + e^x); and the
+    limits g -> -x for large x, g -> 0 for very negative x."""
+    x = np.array([-30.0, -3.0, -0.5, 0.0, 0.5, 3.0, 30.0])
+    g, b = oracle.gates_from_logits(x, x)
+    assert g[3] == pytest.approx(-np.log(2.0), abs=1e-16)
+    assert b[3] == pytest.approx(0.5, abs=1e-16)
+    g_neg, b_neg = oracle.gates_from_logits(-x, -x)
+    np.testing.assert_allclose(-g + g_neg, x, atol=1e-14)
+    np.testing.assert_allclose(b + b_neg, 1.0, atol=1e-15)
+    np.testing.assert_allclose(np.exp(g), 1.0 / (1.0 + np.exp(x)), rtol=1e-14)
+    np.testing.assert_allclose(b, 1.0 / (1.0 + np.exp(-x)), rtol=1e-14)
+    assert np.all(g <= 0) and np.all(np.diff(g) < 0) and np.all(np.diff(b) > 0)
+    assert g[-1] == pytest.approx(-30.0, abs=1e-12) and g[0] == pytest.approx(0.0, abs=1e-12)
+
+
+@pytest.mark.parametrize("impl", sorted(FWD_LOGITS))
+def test_gate_logits_pure_decay(impl):
+    """beta logit -800 (beta = 0 in double): the state only decays, by
+    1 / (1 + e^x) per token: S_t = prod_{s<=t} 1/(1 + e^{x_s}) S_in and
+    o_t = S_t^T q^_t."""
+    rng = np.random.default_rng(11)
+    B, T, H, D = 1, 9, 2, 5
+    q = rng.standard_normal((B, T, H, D)).astype(np.float32)
+    k = rng.standard_normal((B, T, H, D)).astype(np.float32)
+    v = rng.standard_normal((B, T, H, D)).astype(np.float32)
+    x = rng.uniform(-3, 3, (B, T, H)).astype(np.float32)
+    y = np.full((B, T, H), -800.0, np.float32)
+    s = rng.standard_normal((B, H, D, D))
+    out, S = FWD_LOGITS[impl](q, k, v, x, y, s)
+    dec = np.cumprod(1.0 / (1.0 + np.exp(x.astype(np.float64))), axis=1)  # [B,T,H]
+    np.testing.assert_allclose(np.asarray(S, np.float64), s * dec[:, -1][:, :, None, None], rtol=1e-13)
+    ref = np.einsum("bth,bthi,bhij->bthj", dec, unit(q), s)
+    np.testing.assert_allclose(np.asarray(out, np.float64), ref, rtol=1e-12, atol=1e-14)
+
+
+@pytest.mark.parametrize("impl", sorted(FWD_LOGITS))
+def test_gate_logits_write_strength(impl):
+    """decay logit -800 (a = 1 in double) and orthonormal keys e_t: token t
+    replaces row t by (1 - sigmoid(y_t)) S_in[t] + sigmoid(y_t) v_t, with
+    sigmoid(y) = 1 / (1 + e^-y)."""
+    rng = np.random.default_rng(12)
+    B, T, H, D = 1, 6, 1, 6
+    k = np.zeros((B, T, H, D), np.float32)
+    for t in range(T):
+        k[0, t, 0, t] = 1.0
+    q = rng.standard_normal((B, T, H, D)).astype(np.float32)
+    v = rng.standard_normal((B, T, H, D)).astype(np.float32)
+    x = np.full((B, T, H), -800.0, np.float32)
+    y = rng.uniform(-4, 4, (B, T, H)).astype(np.float32)
+    s = rng.standard_normal((B, H, D, D))
+    _, S = FWD_LOGITS[impl](q, k, v, x, y, s)
+    bt = 1.0 / (1.0 + np.exp(-y[0, :, 0].astype(np.float64)))
+    want = s[0, 0].copy()
+    for t in range(T):
+        want[t] = (1.0 - bt[t]) * s[0, 0, t] + bt[t] * v[0, t, 0]
+    np.testing.assert_allclose(np.asarray(S, np.float64)[0, 0], want, rtol=1e-13, atol=1e-15)
+
+
+def test_gate_logits_half_gates_scalar():
+    """x = y = 0 gives a = beta = 1/2 exactly; with d = 1 the scan is the
+    scalar recurrence s_t = a (1 - beta) s + beta sign(k_t) v_t = s / 4 +
+    sign(k_t) v_t / 2, o_t = sign(q_t) s_t (forward and bidirectional)."""
+    rng = np.random.default_rng(13)
+    T = 7
+    q = rng.standard_normal((1, T, 1, 1)).astype(np.float32)
+    k = rng.standard_normal((1, T, 1, 1)).astype(np.float32)
+    v = rng.standard_normal((1, T, 1, 1)).astype(np.float32)
+    z = np.zeros((1, T, 1), np.float32)
+    s0 = np.array([[[[0.7]]]])
+    out, S = oracle.oracle_fwd_logits(q, k, v, z, z, s0, nthreads=1)
+    sk, sq, vv = np.sign(k[0, :, 0, 0]), np.sign(q[0, :, 0, 0]), v[0, :, 0, 0].astype(np.float64)
+    s, want = 0.7, []
+    for t in range(T):
+        s = s / 4 + sk[t] * vv[t] / 2
+        want.append(sq[t] * s)
+    np.testing.assert_allclose(out[0, :, 0, 0], want, rtol=1e-14)
+    assert S[0, 0, 0, 0] == pytest.approx(s, rel=1e-14)
+    outb, _ = oracle.oracle_bidir_logits(q, k, v, z, z, s0, nthreads=1)
+    r, rev = 0.0, np.zeros(T)
+    for t in reversed(range(T)):
+        r = r / 4 + sk[t] * vv[t] / 2
+        rev[t] = sq[t] * r
+    np.testing.assert_allclose(outb[0, :, 0, 0], np.array(want) + rev, rtol=1e-13)
+
+
+def test_gate_logits_c_matches_numpy_gates():
+    """Both transcriptions agree: the C oracle's logit mode against the numpy
+    gates fed to the numpy recurrence (all fp64), on random logits, both
+    directions."""
+    rng = np.random.default_rng(14)
+    q, k, v, _, _, s = rand_inputs(rng, T=31)
+    x = rng.standard_normal((2, 31, 3)).astype(np.float32) * 2
+    y = rng.standard_normal((2, 31, 3)).astype(np.float32) * 2
+    o1, S1 = oracle.oracle_fwd_logits(q, k, v, x, y, s, nthreads=2)
+    g, b = oracle.gates_from_logits(x, y)
+    o2, S2 = oracle.recurrence_fwd(q, k, v, g, b, s)
+    assert rel(o1, o2) < 1e-12 and rel(S1, S2) < 1e-12
+    ob1, _ = oracle.oracle_bidir_logits(q, k, v, x, y, s, nthreads=2)
+    ob2, _ = oracle.recurrence_bidir(q, k, v, g, b, s)
+    assert rel(ob1, ob2) < 1e-12
+
+
+def test_planted_gate_slip_fails_the_decay_pin():
+    """A plausible slip -- softplus of -x instead of x, i.e. a = sigmoid(x)
+    instead of 1 - sigmoid(x) -- planted in a copy of the numpy gate map
+    fails the pure-decay closed form."""
+    rng = np.random.default_rng(11)
+    B, T, H, D = 1, 9, 2, 5
+    q = rng.standard_normal((B, T, H, D)).astype(np.float32)
+    k = rng.standard_normal((B, T, H, D)).astype(np.float32)
+    v = rng.standard_normal((B, T, H, D)).astype(np.float32)
+    x = rng.uniform(-3, 3, (B, T, H)).astype(np.float32)
+    s = rng.standard_normal((B, H, D, D))
+    g_wrong = -np.logaddexp(0.0, -x.astype(np.float64))
+    _, S = oracle.recurrence_fwd(q, k, v, g_wrong, np.zeros((B, T, H)), s)
+    dec = np.prod(1.0 / (1.0 + np.exp(x.astype(np.float64))), axis=1)
+    assert not np.allclose(S, s * dec[:, :, None, None], rtol=1e-6)
