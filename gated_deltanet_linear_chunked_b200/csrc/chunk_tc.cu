@@ -6,8 +6,9 @@
 // 系统", 方法步骤详情, fourth step).  Here the three stages are three kernels:
 //
 //   stage A  gdn_prep_kernel    one CTA per (chunk, b*h, direction), parallel
-//   stage B  gdn_recur_kernel   one CTA per (16 state columns, b*h, direction),
-//                               a dependent walk over the chunks
+//   stage B  gdn_recur_kernel   one CTA per (1-4 slices of 16 state columns,
+//                               b*h, direction), a dependent walk over the
+//                               chunks, one warp per slice
 //   stage C  gdn_output_kernel  persistent, one CTA per SM over the (chunk,
 //                               b*h) tiles, both directions per tile
 // launched back to back with programmatic dependent launch.
@@ -20,13 +21,12 @@
 //   W     = Tm diag(beta e^gamma) K^,     U~ = Tm diag(beta) V
 //   U     = U~ - W S0                     (per-token corrected values)
 //   S_out = e^{gamma_C} S0 + K~^T U,      K~ = diag(e^{gamma_C - gamma}) K^
-//         = e^{gamma_C} S0 - Qc S0 + Rc,  Qc = K~^T W,  Rc = K~^T U~
 //   O     = diag(e^gamma) Q^ S0 + (Mask o Q^ K^^T) U,
 //           Mask_ri = e^{gamma_r - gamma_i} for i at or before r, else 0.
-// Stage A computes Tm, W, U~, Qc, Rc (d x d summaries of the chunk); stage B
-// runs S <- e^{gamma_C} S - Qc S + Rc (per 16-column slice, a d x d times
-// d x 16 product on mma.sync per chunk) and publishes the state at each chunk
-// start; stage C computes U and O.
+// Stage A computes Tm, W, U~ and K~ (everything that does not depend on the
+// state); stage B walks the chunks with the state, forming U and the next
+// state (two products per chunk, d x 64 x 16 and 16 x 64 x d per slice) and
+// publishing U and the chunk-start state; stage C computes O.
 //
 // The reverse (within-chunk backward) scan of the bidirectional mode uses the
 // same memory tiles visited in the opposite order, with gamma the suffix sums
@@ -60,32 +60,32 @@ constexpr int kC = 64;            // tokens per chunk
 constexpr int kWideThreads = 256; // stage A: two warps per TMEM lane quadrant
 constexpr int kOutThreads = 512;  // stage C: four warps per TMEM lane quadrant
 constexpr int kSlab64 = kC * 16;  // bytes of one 8-column slab of a 64-row tile
-constexpr int kRecStages = 4;  // deepest stage-B load ring (see recur_stages)
 constexpr long long kDrainPolls = 1LL << 40;  // drains are bounded by the 2 s timer
 
 // ----------------------------------------------------------------- workspace
 // One contiguous block per (direction, b*h, chunk), in the order the stages
 // read them so that each read is a single bulk copy:
-//   Qc    [Dk/8][Dk][8]   bf16  chunk summary K~^T W          (stage B)
-//   decay {e^{gamma_C}, 0, 0, 0} fp32                        (stage B)
-//   Rc    [Dv/16][Dk][16] bf16  chunk summary K~^T U~ by slice (stage B)
-//   W     [Dk/8][64][8]   bf16                                (stage C)
-//   Ut    [Dv/8][64][8]   bf16  U~                            (stage C)
-//   S     [Dv/8][Dk][8]   bf16  state at the chunk's start    (stage C)
+//   W     [Dk/8][64][8]   bf16                        (A writes, B reads)
+//   Kt    [Dk/8][64][8]   bf16  K~                    (A writes, B reads)
+//   decay {e^{gamma_C}, 0, 0, 0} fp32                 (A writes, B reads)
+//   Ut    [Dv/8][64][8]   bf16  U~                    (A writes, B reads)
+//   U     [Dv/8][64][8]   bf16  U = U~ - W S0         (B writes, C reads)
+//   S     [Dv/8][Dk][8]   bf16  state at chunk start  (B writes, C reads)
 struct Workspace {
   uint8_t* base;
   size_t block_bytes;
-  uint32_t off_decay, off_rc, off_w, off_ut, off_s;
+  uint32_t off_w, off_kt, off_decay, off_ut, off_u, off_s;
   int NBH, nC, Dk, Dv;
 
   __host__ __device__ void layout(int dk, int dv) {
     Dk = dk;
     Dv = dv;
-    off_decay = (uint32_t)Dk * Dk * 2;
-    off_rc = off_decay + 16;
-    off_w = off_rc + (uint32_t)Dk * Dv * 2;
-    off_ut = off_w + 64u * Dk * 2;
-    off_s = off_ut + 64u * Dv * 2;
+    off_w = 0;
+    off_kt = off_w + 64u * Dk * 2;
+    off_decay = off_kt + 64u * Dk * 2;
+    off_ut = off_decay + 16;
+    off_u = off_ut + 64u * Dv * 2;
+    off_s = off_u + 64u * Dv * 2;
     block_bytes = ((size_t)off_s + (size_t)Dk * Dv * 2 + 255) & ~size_t(255);
   }
   __device__ size_t tile(int dir, int bh, int j) const {
@@ -152,24 +152,18 @@ __device__ float row_rnorm4(const uint8_t* tile, int r, int part, int D) {
 
 // ============================================================ stage A: prep
 // Shared memory: K and V tiles stay for the whole tile; the solve's fp32
-// scratch and the bf16 A operands TW/TU are dead once W and U~ are in TMEM,
-// so the scaled B operands Wp/Up reuse their space.  ~102 KB: two CTAs/SM.
+// scratch and the bf16 A operands TW/TU live until W and U~ are in TMEM.
+// ~102 KB: two CTAs/SM.
 constexpr int kLd = 68;  // fp32 row stride of the 64 x 64 scratch (16 B aligned rows)
 struct PrepSmem {
-  alignas(128) uint8_t K[16 * kSlab64];   // [16 slabs][64][8]; slabs >= Dk/8 zero
+  alignas(128) uint8_t K[16 * kSlab64];   // [Dk/8 slabs][64][8]
   alignas(128) uint8_t V[16 * kSlab64];
-  union alignas(128) U {
-    struct {
-      uint8_t TW[8 * kSlab64];             // Tm diag(beta e^g / |k|), K-major A
-      uint8_t TU[8 * kSlab64];             // Tm diag(beta), K-major A
-      float A[64][kLd];                    // strictly lower A in scan order
-      float T[64][kLd];                    // (I + A)^-1 in scan order
-      float Y[64][kLd];                    // product scratch
-    } a;
-    struct {
-      uint8_t Wp[16 * kSlab64];            // diag(e^{gC-g}/|k|) W, MN-major B
-      uint8_t Up[16 * kSlab64];            // diag(e^{gC-g}/|k|) U~, MN-major B
-    } b;
+  struct alignas(128) U {
+    uint8_t TW[8 * kSlab64];             // Tm diag(beta e^g / |k|), K-major A
+    uint8_t TU[8 * kSlab64];             // Tm diag(beta), K-major A
+    float A[64][kLd];                    // strictly lower A in scan order
+    float T[64][kLd];                    // (I + A)^-1 in scan order
+    float Y[64][kLd];                    // product scratch
   } u;
   float g[64], beta[64], gam[64], rn[64], csW[64], csU[64];
   float arow[64];      // beta_r |k_r|^-1 e^{gam_r - m_b(r)}       (scan order)
@@ -225,9 +219,9 @@ __device__ __forceinline__ void warp_store_tile(float (*C)[kLd], int cr, int cc,
 // the block products on tf32 tensor cores (T is rounded to bf16 right after).
 __device__ void unit_lower_inverse(PrepSmem::U& u) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  float (*A)[kLd] = u.a.A;
-  float (*T)[kLd] = u.a.T;
-  float (*Y)[kLd] = u.a.Y;
+  float (*A)[kLd] = u.A;
+  float (*T)[kLd] = u.T;
+  float (*Y)[kLd] = u.Y;
   for (int i = tid; i < 64 * 16; i += kWideThreads)
     reinterpret_cast<float4*>(T[i >> 4])[i & 15] = make_float4(0.f, 0.f, 0.f, 0.f);
   __syncthreads();
@@ -376,7 +370,7 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
     if (lane < 16) {
       const float ap = s.arow[p];
       const float* bc = s.bcol[p >> 3];
-      float* Arow = s.u.a.A[p];
+      float* Arow = s.u.A[p];
 #pragma unroll
       for (int q4 = 0; q4 < 8; ++q4) {
         const int qb = 32 * half + 4 * q4;
@@ -400,7 +394,7 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
   // as bf16 K-major A operands in memory order
   for (int idx = tid; idx < 64 * 8; idx += kWideThreads) {
     const int r = idx & 63, ks = idx >> 6;
-    const float* Trow = s.u.a.T[scan_pos<REV>(r)];
+    const float* Trow = s.u.T[scan_pos<REV>(r)];
     float w[8], uu[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
@@ -409,8 +403,8 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
       w[e] = t * s.csW[i];
       uu[e] = t * s.csU[i];
     }
-    reinterpret_cast<uint4*>(s.u.a.TW + ks * kSlab64)[r] = pack8_bf16(w);
-    reinterpret_cast<uint4*>(s.u.a.TU + ks * kSlab64)[r] = pack8_bf16(uu);
+    reinterpret_cast<uint4*>(s.u.TW + ks * kSlab64)[r] = pack8_bf16(w);
+    reinterpret_cast<uint4*>(s.u.TU + ks * kSlab64)[r] = pack8_bf16(uu);
   }
   block_sync_async();
   if (!block_wait(&s.v_bar, 0, limit, err)) return false;
@@ -418,8 +412,8 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
   if (tid == 0) {
     const uint32_t idW = idesc_bf16(64, Dk, 0, 1), idU = idesc_bf16(64, Dv, 0, 1);
     for (int ks = 0; ks < kC / 16; ++ks) {
-      const uint64_t aw = sdesc(smem_u32(s.u.a.TW) + ks * 2 * kSlab64, kSlab64, 128);
-      const uint64_t au = sdesc(smem_u32(s.u.a.TU) + ks * 2 * kSlab64, kSlab64, 128);
+      const uint64_t aw = sdesc(smem_u32(s.u.TW) + ks * 2 * kSlab64, kSlab64, 128);
+      const uint64_t au = sdesc(smem_u32(s.u.TU) + ks * 2 * kSlab64, kSlab64, 128);
       const uint64_t bk = sdesc(smem_u32(s.K) + ks * 256, 128, kSlab64);
       const uint64_t bv = sdesc(smem_u32(s.V) + ks * 256, 128, kSlab64);
       mma_bf16(tm, aw, bk, idW, ks > 0);
@@ -427,17 +421,30 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
     }
     mma_commit(&s.mma_bar);
   }
+  // While W and U~ compute: K~ = diag(e^{gamC - gam} / |k|) K -> workspace,
+  // in the tile's own [slab][64][8] layout, and the chunk decay e^{gamC}
+  const size_t tile = ws.tile(dir, bh, j);
+  uint8_t* blk = ws.blk(tile);
+  for (int idx = tid; idx < (Dk / 8) * kC; idx += kWideThreads) {
+    const int r = idx & 63, sl = idx >> 6;
+    const float sc = expf(gamC - s.gam[r]) * s.rn[r];
+    float x[8];
+    unpack8_bf16(reinterpret_cast<const uint4*>(s.K + sl * kSlab64)[r], x);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] *= sc;
+    reinterpret_cast<uint4*>(blk + ws.off_kt + sl * kSlab64)[r] = pack8_bf16(x);
+  }
+  if (tid == 0)
+    *reinterpret_cast<float4*>(blk + ws.off_decay) = make_float4(expf(gamC), 0.f, 0.f, 0.f);
   if (!block_wait(&s.mma_bar, 1, limit, err)) return false;
   tc_fence_after_sync();
 
-  // W, U~ -> workspace (bf16 [slab][64][8]); scaled copies -> Wp, Up.
-  // Warps w and w + 4 share a TMEM lane quadrant and split the column blocks.
+  // W, U~ -> workspace (bf16 [slab][64][8]).  Warps w and w + 4 share a TMEM
+  // lane quadrant and split the column blocks.
   {
     const int quad = warp & 3, half = warp >> 2;
     const int r = 16 * quad + (lane & 15);
     const uint32_t lane_base = static_cast<uint32_t>(32 * quad) << 16;
-    const size_t tile = ws.tile(dir, bh, j);
-    const float sc = expf(gamC - s.gam[r]) * s.rn[r];
     // column block cb: W's blocks [0, Dk/16) at TMEM column 16 cb, then
     // U~'s at 128 + 16 (cb - Dk/16); two TMEM loads in flight per wait
     const int nkb = Dk / 16, nb = nkb + Dv / 16;
@@ -445,15 +452,9 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
     auto put = [&](int cb, const float* v) {
       const bool isw = cb < nkb;
       const int c = isw ? cb : cb - nkb;
-      uint4* G = reinterpret_cast<uint4*>(ws.blk(tile) + (isw ? ws.off_w : ws.off_ut));
-      uint8_t* Sp = isw ? s.u.b.Wp : s.u.b.Up;
-      float sv[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) sv[e] = v[e] * sc;
+      uint4* G = reinterpret_cast<uint4*>(blk + (isw ? ws.off_w : ws.off_ut));
       G[(2 * c) * kC + r] = pack8_bf16(v);
       G[(2 * c + 1) * kC + r] = pack8_bf16(v + 8);
-      reinterpret_cast<uint4*>(Sp + (2 * c) * kSlab64)[r] = pack8_bf16(sv);
-      reinterpret_cast<uint4*>(Sp + (2 * c + 1) * kSlab64)[r] = pack8_bf16(sv + 8);
     };
     for (int cb = half; cb < nb; cb += 4) {
       float v0[16], v1[16];
@@ -466,57 +467,6 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
         if (two) put(cb + 2, v1);
       }
     }
-  }
-  block_sync_async();
-  const size_t tile = ws.tile(dir, bh, j);
-  // Qc = K^T Wp (M = 128 >= Dk, N = Dk), Rc = K^T Up (N = Dv); K read MN-major
-  // as A (M = feature; slabs >= Dk/8 are zero rows)
-  if (tid == 0) {
-    const uint32_t idQ = idesc_bf16(128, Dk, 1, 1), idR = idesc_bf16(128, Dv, 1, 1);
-    for (int ks = 0; ks < kC / 16; ++ks) {
-      const uint64_t a = sdesc(smem_u32(s.K) + ks * 256, 128, kSlab64);
-      const uint64_t bw = sdesc(smem_u32(s.u.b.Wp) + ks * 256, 128, kSlab64);
-      const uint64_t bu = sdesc(smem_u32(s.u.b.Up) + ks * 256, 128, kSlab64);
-      mma_bf16(tm, a, bw, idQ, ks > 0);
-      mma_bf16(tm + 128, a, bu, idR, ks > 0);
-    }
-    mma_commit(&s.mma_bar);
-  }
-  if (!block_wait(&s.mma_bar, 0, limit, err)) return false;
-  tc_fence_after_sync();
-  {
-    const int quad = warp & 3, half = warp >> 2;
-    const int r = 32 * quad + lane;  // TMEM lane = feature row of Qc / Rc
-    const uint32_t lane_base = static_cast<uint32_t>(32 * quad) << 16;
-    // Qc | decay | Rc staged in the workspace block's own layout
-    uint4* Qg = reinterpret_cast<uint4*>(ws.blk(tile));
-    uint4* Rg = reinterpret_cast<uint4*>(ws.blk(tile) + ws.off_rc);
-    // column block cb: Qc's [0, Dk/16) at 16 cb, Rc's at 128 + 16 (cb - Dk/16)
-    const int nkb = Dk / 16, nb = nkb + Dv / 16;
-    auto col = [&](int cb) { return cb < nkb ? 16u * cb : 128u + 16u * (cb - nkb); };
-    auto put = [&](int cb, const float* v) {
-      if (cb < nkb) {
-        Qg[(2 * cb) * Dk + r] = pack8_bf16(v);
-        Qg[(2 * cb + 1) * Dk + r] = pack8_bf16(v + 8);
-      } else {
-        const int c = cb - nkb;
-        Rg[(c * Dk + r) * 2] = pack8_bf16(v);
-        Rg[(c * Dk + r) * 2 + 1] = pack8_bf16(v + 8);
-      }
-    };
-    for (int cb = half; cb < nb; cb += 4) {
-      float v0[16], v1[16];
-      const bool two = cb + 2 < nb;
-      tmem_ld16(tm + lane_base + col(cb), v0);
-      if (two) tmem_ld16(tm + lane_base + col(cb + 2), v1);
-      tmem_wait_ld();
-      if (r < Dk) {
-        put(cb, v0);
-        if (two) put(cb + 2, v1);
-      }
-    }
-    if (tid == 0)
-      *reinterpret_cast<float4*>(ws.blk(tile) + ws.off_decay) = make_float4(expf(gamC), 0.f, 0.f, 0.f);
   }
   return true;
 }
@@ -538,10 +488,6 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     tmem_alloc(&s.tmem, 256);
     tmem_relinquish();
   }
-  {  // zero the feature slabs past Dk (rows of the M = 128 products)
-    uint4* z = reinterpret_cast<uint4*>(s.K + (ws.Dk / 8) * kSlab64);
-    for (int i = tid; i < (16 - ws.Dk / 8) * kSlab64 / 16; i += kWideThreads) z[i] = make_uint4(0, 0, 0, 0);
-  }
   block_sync_async();
   // Programmatic dependent launch: everything above overlaps the previous
   // kernel in the stream; nothing in global memory is touched before this.
@@ -557,234 +503,381 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 }
 
 // ======================================================= stage B: recurrence
-// One CTA per (16 state columns, b*h, direction), Dk/16 warps; warp w owns
-// state rows [16w, 16w + 16).  Per chunk the product Qc S (Dk x Dk times
-// Dk x 16) is a dependent chain across chunks and is latency-bound: a
-// tcgen05 round trip (issue 7 MMAs, commit, mbarrier, TMEM load) costs about
-// 1.2k cycles for a 16-column slice and over 3k for a whole head, so this
-// stage uses warp-level mma.sync.m16n8k16 (bf16 in, fp32 accumulate) with
-// the fp32 state held in the accumulator registers and the bf16 copy of S
-// exchanged through a double-buffered shared-memory operand: one barrier per
-// chunk.  An NST-stage ring of bulk loads feeds [Qc | decay | Rc slice].
-// Dynamic layout: [head 128 B] [S operand x 2: [2 n-slabs][Dk][8] bf16]
-//                 [NST stages: Qc [Dk/8][Dk][8] | decay 16 B | Rc slice [Dk][16]]
-struct RecSmemHead {
-  uint64_t full[kRecStages];
+// One CTA per (one or two slices of 16 state columns, b*h, direction).  Each
+// slice is walked by a group of P = min(4, Dk/16) warps (one per SM
+// sub-partition); one more warp per CTA, the producer, streams each chunk's
+// [W | K~ | decay] and the CTA's U~ slabs through an nst-stage ring of bulk
+// copies (full / empty mbarriers) and issues the bulk stores that publish the
+// groups' results.  Per chunk, transposed so that the slice's 16 state
+// columns are the M = 16 rows of mma.sync.m16n8k16:
+//   U^T  = U~^T - S^T W^T              (16 x 64 tokens, K = Dk)
+//          warp q of the group takes 64/P of the tokens
+//   S^T <- e^{gamma_C} S^T + U^T K~     (16 x Dk, K = 64 tokens)
+//          warp q takes its share of the Dk state rows and keeps that part
+//          of the fp32 state in its accumulator registers
+// An accumulator tile pair is exactly an A-operand fragment, so between the
+// two products the warps of a group only exchange bf16 fragments through a
+// small shared buffer and a named barrier (U^T after the first product, S^T
+// after the second).  Per-warp mma.sync issue is what bounds this stage, and
+// the split gives every warp about 1/P of each product.  The chunk-start
+// state S and U go to stage C through a triple-buffered staging area
+// (stmatrix.trans): once a chunk's staging is complete the group tells the
+// producer (mbarrier `staged`), which stores it with bulk copies and frees the
+// buffer (mbarrier `freed`) when they have read it, off the chain's path.
+constexpr int kChainMaxGroups = 2;
+constexpr int kChainMaxStages = 6;
+constexpr int kChainHeadBytes = 256;  // mbarriers and the groups' failure flags
+constexpr int kChainBufs = 3;         // staging buffers per group
+
+__host__ __device__ constexpr int chain_group_warps(int nkb) { return nkb >= 4 ? 4 : nkb >= 2 ? 2 : 1; }
+
+struct ChainLayout {
+  uint32_t wk_bytes;  // W | K~ | decay of one chunk (one bulk copy)
+  uint32_t stage;     // stage stride: W | K~ | decay | the CTA's U~ slabs
+  uint32_t stg_s;     // staging of S [2][Dk][8] bf16; U [2][64][8] follows
+  uint32_t stg;       // one staging buffer
+  uint32_t xs;        // exchange: S^T A fragments [Dk/16][32 lanes][16 B]
+  uint32_t group;     // per group: staging buffers | S^T exchange | U^T exchange
+  uint32_t groups;    // offset of group 0
+  uint32_t total;
+  __host__ __device__ ChainLayout(int Dk, int ns, int nst) {
+    wk_bytes = 2u * 64 * Dk * 2 + 16;
+    stage = (wk_bytes + (uint32_t)ns * 2 * kSlab64 + 127) & ~127u;
+    stg_s = 2u * Dk * 16;
+    stg = stg_s + 2u * kSlab64;
+    xs = (uint32_t)(Dk / 16) * 512;
+    group = kChainBufs * stg + xs + 4 * 512;
+    groups = kChainHeadBytes + nst * stage;
+    total = groups + ns * group;
+  }
 };
-constexpr int kRecHeadBytes = 128;
-constexpr int kRecSBytes = 2 * 128 * 16;  // one S operand buffer at Dk = 128
 
-__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
+struct ChainBars {
+  uint64_t full[kChainMaxStages], empty[kChainMaxStages];
+  uint64_t staged[kChainBufs], freed[kChainBufs];  // per staging buffer
+  int fail[kChainMaxGroups];                       // a bounded wait of the group expired
+};
+
+__device__ __forceinline__ void unpack_bf16x2(uint32_t u, float& lo, float& hi) {
+  lo = __uint_as_float(u << 16);
+  hi = __uint_as_float(u & 0xFFFF0000u);
 }
-__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint32_t (&r)[4]) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(r[0]), "r"(r[1]),
+               "r"(r[2]), "r"(r[3])
+               : "memory");
 }
-// D += A B, m16n8k16, bf16 inputs, fp32 accumulators.
-__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                          uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+__device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
 }
 
-// NKS = Dk / 16 and NST = stages of the load ring, compile-time constants so
-// that the per-chunk code is straight-line.
-template <int NKS, int NST>
-__device__ bool recur_body(uint8_t* smem, const float* state_in, float* state_out,
-                           const Workspace& ws, long long limit, unsigned* err) {
-  constexpr int nst = NST;
-  RecSmemHead& hd = *reinterpret_cast<RecSmemHead*>(smem);
+// Warp q of the group walking slice s (16 state columns); gw = group index in
+// the CTA.  NKB = Dk / 16.  Returns false if a bounded wait expired.
+template <int NKB>
+__device__ bool chain_warp(uint8_t* smem, const ChainLayout& L, int nst, int gw, int q, int s,
+                           const float* state_in, float* state_out, const Workspace& ws,
+                           long long limit, unsigned* err) {
+  constexpr int P = chain_group_warps(NKB);
+  constexpr int KPW = (NKB + P - 1) / P;  // most state-row k-blocks of one warp
+  constexpr int TPW = 4 / P;              // 16-token blocks of one warp
+  ChainBars& bars = *reinterpret_cast<ChainBars*>(smem);
+  const int lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+  const int mi = lane >> 3, mr = lane & 7;  // ldmatrix / stmatrix: matrix, row
   const int Dk = ws.Dk, Dv = ws.Dv, nC = ws.nC;
-  uint8_t* Sop0 = smem + kRecHeadBytes;
-  const uint32_t nslab_bytes = (uint32_t)Dk * 16;  // one n-slab [Dk][8] bf16 of the operand
-  uint8_t* stage0 = Sop0 + 2 * kRecSBytes;
-  const uint32_t qbytes = (uint32_t)Dk * Dk * 2, rbytes = (uint32_t)Dk * 32;
-  const uint32_t stage_bytes = (qbytes + rbytes + 16 + 127) & ~127u;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int slice = blockIdx.x, bh = blockIdx.y, dir = blockIdx.z;
-  // accumulator coordinates of this thread: rows rA, rA + 8; columns cA, cA + 1 (+ 8 nt)
-  const int rA = 16 * warp + (lane >> 2), cA = 2 * (lane & 3);
+  const int bh = blockIdx.y, dir = blockIdx.z;
+  const int kb_lo = q * NKB / P, kb_hi = (q + 1) * NKB / P;  // this warp's state rows
+  const int tb0 = q * TPW;                                    // this warp's tokens
+  const int bar_id = 1 + gw, bar_n = 32 * P;
 
-  float S[2][4];  // [n-tile][c0..c3], fp32 state
+  // this warp's part of S^T: rows j = 16 s + g (regs 0, 1) and + 8 (2, 3),
+  // columns i = 8 nt + 2 tq (+1) for n-tiles nt of k-blocks [kb_lo, kb_hi)
+  float S[2 * KPW][4];
 #pragma unroll
-  for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) S[nt][i] = 0.f;
+  for (int k = 0; k < 2 * KPW; ++k) S[k][0] = S[k][1] = S[k][2] = S[k][3] = 0.f;
   if (dir == 0 && state_in) {
-    const float* base = state_in + (size_t)bh * Dk * Dv + 16 * slice;
+    const float* base = state_in + (size_t)bh * Dk * Dv + 16 * s + g;
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      const float2 lo = *reinterpret_cast<const float2*>(base + (size_t)rA * Dv + 8 * nt + cA);
-      const float2 hi = *reinterpret_cast<const float2*>(base + (size_t)(rA + 8) * Dv + 8 * nt + cA);
-      S[nt][0] = lo.x; S[nt][1] = lo.y; S[nt][2] = hi.x; S[nt][3] = hi.y;
+    for (int k = 0; k < 2 * KPW; ++k) {
+      if (kb_lo + k / 2 < kb_hi) {
+        const int i0 = 8 * (2 * kb_lo + k) + 2 * tq;
+        S[k][0] = base[(size_t)i0 * Dv];
+        S[k][1] = base[(size_t)(i0 + 1) * Dv];
+        S[k][2] = base[(size_t)i0 * Dv + 8];
+        S[k][3] = base[(size_t)(i0 + 1) * Dv + 8];
+      }
     }
   }
-  auto issue = [&](int c) {  // one thread: load chunk c (scan order) into its stage
-    const int jt = dir ? nC - 1 - c : c;
-    const size_t tile = ws.tile(dir, bh, jt);
-    uint8_t* st = stage0 + (c % nst) * stage_bytes;
-    uint64_t* bar = &hd.full[c % nst];
-    mbar_arrive_expect_tx(bar, qbytes + 16 + rbytes);
-    bulk_load(st, ws.blk(tile), qbytes + 16, bar);  // Qc and decay
-    bulk_load(st + qbytes + 16, ws.blk(tile) + ws.off_rc + (size_t)slice * Dk * 32, rbytes, bar);
-  };
-  int issued = min(nst, nC);
-  if (tid == 0)
-    for (int c = 0; c < issued; ++c) issue(c);
 
-  // S (bf16) of this thread's accumulator positions -> operand buffer `buf`
-  // ([n-slab][Dk rows][8]).  Its two n-slabs are exactly this slice's part of
-  // the workspace copy of the chunk-start state ([Dv/8][Dk][8]), which one
-  // thread then writes with a single bulk store after the next barrier.
-  auto publish = [&](int buf) {
-    uint8_t* Sop = Sop0 + buf * kRecSBytes;
+  const uint32_t stage0 = smem_u32(smem + kChainHeadBytes);
+  const uint32_t grp_u = smem_u32(smem + L.groups + gw * L.group);
+  const uint32_t xs_u = grp_u + kChainBufs * L.stg, xu_u = xs_u + L.xs;
+  // per-lane parts of the ldmatrix / stmatrix row addresses
+  const uint32_t st_off = (uint32_t)((mi & 1) * Dk * 16 + ((mi >> 1) * 8 + mr) * 16);   // S staging
+  const uint32_t su_off = (uint32_t)((mi & 1) * kSlab64 + ((mi >> 1) * 8 + mr) * 16);   // U staging, U~, W
+  const uint32_t kt_off = (uint32_t)((mi >> 1) * kSlab64 + ((mi & 1) * 8 + mr) * 16);   // K~ (trans)
+
+  // Own state rows -> bf16 A fragments, dumped to the S^T exchange and, as a
+  // chunk-start state, to staging buffer sbuf (none after the last chunk).
+  auto publish_state = [&](uint32_t sbuf, bool stage_it) {
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      *reinterpret_cast<uint32_t*>(Sop + nt * nslab_bytes + rA * 16 + cA * 2) =
-          pack_bf16x2(S[nt][0], S[nt][1]);
-      *reinterpret_cast<uint32_t*>(Sop + nt * nslab_bytes + (rA + 8) * 16 + cA * 2) =
-          pack_bf16x2(S[nt][2], S[nt][3]);
+    for (int k = 0; k < KPW; ++k) {
+      const int kb = kb_lo + k;
+      if (kb < kb_hi) {
+        uint32_t a[4];
+        a[0] = pack_bf16x2(S[2 * k][0], S[2 * k][1]);
+        a[1] = pack_bf16x2(S[2 * k][2], S[2 * k][3]);
+        a[2] = pack_bf16x2(S[2 * k + 1][0], S[2 * k + 1][1]);
+        a[3] = pack_bf16x2(S[2 * k + 1][2], S[2 * k + 1][3]);
+        if (stage_it) stmatrix_x4_trans(sbuf + kb * 256 + st_off, a);
+        st_shared_v4(xs_u + kb * 512 + lane * 16, a);
+      }
     }
   };
-  const int storer = blockDim.x > 64 ? 64 : 0;
-  publish(0);
+  publish_state(grp_u, true);
+  named_barrier(bar_id, bar_n);
 
-  // ldmatrix row addresses (bytes in shared space) for this thread
-  const int mi = lane >> 3, mr = lane & 7;
-  // A: matrices (rows 0-7 | 8-15) x (k 0-7 | 8-15) of this warp's 16 rows
-  const uint32_t a_off = (uint32_t)((mi >> 1) * Dk * 16 + (16 * warp + (mi & 1) * 8 + mr) * 16);
-  // B (trans): matrices (k 0-7 | 8-15) x (n-slab 0 | 1)
-  const uint32_t b_off = (uint32_t)((mi >> 1) * nslab_bytes + ((mi & 1) * 8 + mr) * 16);
-  const uint32_t sop_u32 = smem_u32(Sop0), stage_u32 = smem_u32(stage0);
-
-  // Software pipeline: the A fragments of Qc, the decay and the Rc slice of
-  // chunk c + 1 are read into registers while chunk c's MMAs run, and
-  // X = e^{gamma_C} S + Rc is formed before the product arrives, so the
-  // dependent path per chunk is: barrier, B fragments, MMA, S = X - Qc S,
-  // operand write.
-  uint32_t af[NKS][4];
-  float X[2][4];
-  // wait for chunk c's stage (every thread), then read its A fragments and
-  // form X from the current S
-  auto prefetch = [&](int cc) -> bool {
-    const int st = cc % nst;
-    const bool okw = mbar_wait(&hd.full[st], (cc / nst) & 1, limit);
-    const uint32_t qa = stage_u32 + st * stage_bytes + a_off;
-#pragma unroll
-    for (int ks = 0; ks < NKS; ++ks) ldmatrix_x4(qa + ks * 2 * Dk * 16, af[ks]);
-    const uint8_t* stp = stage0 + st * stage_bytes;
-    const float a = *reinterpret_cast<const float*>(stp + qbytes);
-    const __nv_bfloat16* R = reinterpret_cast<const __nv_bfloat16*>(stp + qbytes + 16);
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      const __nv_bfloat162 r0 = *reinterpret_cast<const __nv_bfloat162*>(R + rA * 16 + 8 * nt + cA);
-      const __nv_bfloat162 r1 = *reinterpret_cast<const __nv_bfloat162*>(R + (rA + 8) * 16 + 8 * nt + cA);
-      X[nt][0] = fmaf(a, S[nt][0], __low2float(r0));
-      X[nt][1] = fmaf(a, S[nt][1], __high2float(r0));
-      X[nt][2] = fmaf(a, S[nt][2], __low2float(r1));
-      X[nt][3] = fmaf(a, S[nt][3], __high2float(r1));
-    }
-    return okw;
-  };
-
-  bool ok = prefetch(0);
+  bool ok = true, okp = true;
   int c = 0;
+  int st = 0, bi = 0;  // load stage and staging buffer of chunk c
+  uint32_t ph = 0;     // parity of stage st's current fill
+  bool ready = false;  // chunk c's stage was seen full ahead of time
+  volatile int* fail = &bars.fail[gw];
   for (; c < nC; ++c) {
-    if (tid == storer) bulk_wait_read();  // last store done reading the buffer we reuse
-    fence_proxy_async_smem();             // operand writes -> the bulk store
-    if (!__syncthreads_and(ok)) break;  // S operand written, stage data visible
-    if (tid == storer)
-      bulk_store(ws.blk(ws.tile(dir, bh, dir ? nC - 1 - c : c)) + ws.off_s +
-                     (size_t)slice * 2 * nslab_bytes,
-                 Sop0 + (c & 1) * kRecSBytes, 2 * nslab_bytes);
-    if (tid == 32 % blockDim.x && c >= 1 && c - 1 + nst < nC) issue(c - 1 + nst);
-    if (c >= 1 && c - 1 + nst < nC) issued = c - 1 + nst + 1;
-    const uint32_t sb = sop_u32 + (c & 1) * kRecSBytes + b_off;
-    uint32_t bfr[NKS][4];
+    const uint32_t buf = grp_u + bi * L.stg;  // staging of chunk c
+    // the whole chunk-start state S^T, as A fragments over k = state rows
+    uint32_t sa[NKB][4];
 #pragma unroll
-    for (int ks = 0; ks < NKS; ++ks) ldmatrix_x4_trans(sb + ks * 256, bfr[ks]);
-    // two independent accumulator chains per n-tile (even / odd k-steps)
-    float acc[2][2][4];
+    for (int kb = 0; kb < NKB; ++kb) ld_shared_v4(xs_u + kb * 512 + lane * 16, sa[kb]);
+
+    bool okw = (ready || __all_sync(0xffffffffu, mbar_wait(&bars.full[st], ph, limit))) && okp;
+    const uint32_t sw = stage0 + st * L.stage;         // W
+    const uint32_t sk = sw + 64u * Dk * 2;             // K~
+    float u[2 * TPW][4];
+    uint32_t ua_mine[TPW][4];
+    if (okw) {
+      const uint32_t sut = sw + L.wk_bytes + 2u * gw * kSlab64;  // this slice's U~ slabs
+      // U^T = U~^T - S^T W^T over this warp's tokens: every B fragment is
+      // loaded before the MMAs that use them, so the loads overlap
+      uint32_t bw[NKB][TPW][4];
 #pragma unroll
-    for (int h = 0; h < 2; ++h)
+      for (int kb = 0; kb < NKB; ++kb)
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+        for (int t = 0; t < TPW; ++t) ldmatrix_x4(sw + 2 * kb * kSlab64 + (tb0 + t) * 256 + su_off, bw[kb][t]);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[h][nt][i] = 0.f;
+      for (int t = 0; t < TPW; ++t) {
+        uint32_t r[4];
+        ldmatrix_x4_trans(sut + (tb0 + t) * 256 + su_off, r);
+        unpack_bf16x2(r[0], u[2 * t][0], u[2 * t][1]);
+        unpack_bf16x2(r[1], u[2 * t][2], u[2 * t][3]);
+        unpack_bf16x2(r[2], u[2 * t + 1][0], u[2 * t + 1][1]);
+        unpack_bf16x2(r[3], u[2 * t + 1][2], u[2 * t + 1][3]);
+      }
 #pragma unroll
-    for (int ks = 0; ks < NKS; ++ks) {
-      mma_16816(acc[ks & 1][0], af[ks], bfr[ks][0], bfr[ks][1]);
-      mma_16816(acc[ks & 1][1], af[ks], bfr[ks][2], bfr[ks][3]);
+      for (int kb = 0; kb < NKB; ++kb) {
+        uint32_t na[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) na[e] = sa[kb][e] ^ 0x80008000u;  // -S^T
+#pragma unroll
+        for (int t = 0; t < TPW; ++t) {
+          mma_16816(u[2 * t], na, bw[kb][t][0], bw[kb][t][1]);
+          mma_16816(u[2 * t + 1], na, bw[kb][t][2], bw[kb][t][3]);
+        }
+      }
+      // this warp's U^T block(s): staged for stage C and dumped for the group
+#pragma unroll
+      for (int t = 0; t < TPW; ++t) {
+        ua_mine[t][0] = pack_bf16x2(u[2 * t][0], u[2 * t][1]);
+        ua_mine[t][1] = pack_bf16x2(u[2 * t][2], u[2 * t][3]);
+        ua_mine[t][2] = pack_bf16x2(u[2 * t + 1][0], u[2 * t + 1][1]);
+        ua_mine[t][3] = pack_bf16x2(u[2 * t + 1][2], u[2 * t + 1][3]);
+        stmatrix_x4_trans(buf + L.stg_s + (tb0 + t) * 256 + su_off, ua_mine[t]);
+        st_shared_v4(xu_u + (tb0 + t) * 512 + lane * 16, ua_mine[t]);
+      }
+      fence_proxy_async_smem();  // staging writes -> the producer's bulk stores
     }
-    // S <- (e^{gamma_C} S + Rc) - Qc S
+    if (!okw && lane == 0) *fail = 1;
+    named_barrier(bar_id, bar_n);
+    ok = *fail == 0;
+    if (!ok) break;
+    // chunk c's staging (its start state and U) is complete
+    if (q == 0 && lane == 0) mbar_arrive(&bars.staged[bi]);
+    // S^T <- e^{gamma_C} S^T + U^T K~ over this warp's state rows (B
+    // fragments first, then the MMAs)
+    uint32_t bk[4][KPW][4];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int kt = 0; kt < 4; ++kt)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) S[nt][i] = X[nt][i] - (acc[0][nt][i] + acc[1][nt][i]);
-    if (c + 1 < nC) {
-      publish((c + 1) & 1);
-      ok = prefetch(c + 1);
+      for (int k = 0; k < KPW; ++k)
+        if (kb_lo + k < kb_hi) ldmatrix_x4_trans(sk + 2 * (kb_lo + k) * kSlab64 + kt * 256 + kt_off, bk[kt][k]);
+    uint32_t ua[4][4];
+#pragma unroll
+    for (int kt = 0; kt < 4; ++kt) ld_shared_v4(xu_u + kt * 512 + lane * 16, ua[kt]);
+    float decay;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(decay) : "r"(sk + 64u * Dk * 2));
+#pragma unroll
+    for (int k = 0; k < 2 * KPW; ++k)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) S[k][e] *= decay;
+#pragma unroll
+    for (int kt = 0; kt < 4; ++kt) {
+#pragma unroll
+      for (int k = 0; k < KPW; ++k) {
+        if (kb_lo + k < kb_hi) {
+          mma_16816(S[2 * k], ua[kt], bk[kt][k][0], bk[kt][k][1]);
+          mma_16816(S[2 * k + 1], ua[kt], bk[kt][k][2], bk[kt][k][3]);
+        }
+      }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars.empty[st]);  // this warp's reads of the stage are done
+    if (++st == nst) {
+      st = 0;
+      ph ^= 1;
+    }
+    // probe the next chunk's stage while the MMAs above run
+    ready = __all_sync(0xffffffffu, mbar_test_wait(&bars.full[st], ph));
+    // the next chunk's start state goes to buffer (c + 1) % 3, which the
+    // producer's stores of chunk c - 2 must have finished reading
+    const bool more = c + 1 < nC;
+    const int bn = bi == kChainBufs - 1 ? 0 : bi + 1;
+    if (more && c >= 2)
+      okp = __all_sync(0xffffffffu, mbar_wait(&bars.freed[bn], ((c - 2) / kChainBufs) & 1, limit));
+    publish_state(grp_u + bn * L.stg, more && okp);
+    named_barrier(bar_id, bar_n);
+    bi = bn;
   }
-  if (tid == storer) bulk_wait_all();
-  if (c < nC) {  // a bounded wait expired: drain every load still in flight
-    if (tid == 0) atomicOr(err, kErrTimeout);
-    for (int p = c; p < issued; ++p)
-      mbar_wait(&hd.full[p % nst], (p / nst) & 1, kDrainPolls);
-    __syncthreads();
+  if (!ok) {
+    if (lane == 0) atomicOr(err, kErrTimeout);
     return false;
   }
   if (dir == 0 && state_out) {
-    float* base = state_out + (size_t)bh * Dk * Dv + 16 * slice;
+    float* base = state_out + (size_t)bh * Dk * Dv + 16 * s + g;
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      *reinterpret_cast<float2*>(base + (size_t)rA * Dv + 8 * nt + cA) = make_float2(S[nt][0], S[nt][1]);
-      *reinterpret_cast<float2*>(base + (size_t)(rA + 8) * Dv + 8 * nt + cA) = make_float2(S[nt][2], S[nt][3]);
+    for (int k = 0; k < 2 * KPW; ++k) {
+      if (kb_lo + k / 2 < kb_hi) {
+        const int i0 = 8 * (2 * kb_lo + k) + 2 * tq;
+        base[(size_t)i0 * Dv] = S[k][0];
+        base[(size_t)(i0 + 1) * Dv] = S[k][1];
+        base[(size_t)i0 * Dv + 8] = S[k][2];
+        base[(size_t)(i0 + 1) * Dv + 8] = S[k][3];
+      }
     }
   }
   return true;
 }
 
-template <int NKS, int NST>
-__global__ void __launch_bounds__(256, 1)
-gdn_recur_kernel(const float* state_in, float* state_out, Workspace ws, long long limit,
-                 unsigned* err) {
+// The producer (one thread): loads chunk c into stage c % nst once the chain
+// warps have released that stage's previous chunk, and publishes each
+// chunk's staged S and U for the CTA's groups with bulk stores.
+__device__ void chain_producer(uint8_t* smem, const ChainLayout& L, int nst, int active, int s0,
+                               const Workspace& ws, long long limit, unsigned* err) {
+  ChainBars& bars = *reinterpret_cast<ChainBars*>(smem);
+  const int bh = blockIdx.y, dir = blockIdx.z, nC = ws.nC, Dk = ws.Dk;
+  uint8_t* stage0 = smem + kChainHeadBytes;
+  const uint32_t ut_bytes = (uint32_t)active * 2 * kSlab64;
+  auto block_of = [&](int c) { return ws.blk(ws.tile(dir, bh, dir ? nC - 1 - c : c)); };
+  auto load = [&](int c) -> bool {
+    const int st = c % nst;
+    if (c >= nst && !mbar_wait(&bars.empty[st], ((c / nst) - 1) & 1, limit)) return false;
+    const uint8_t* blk = block_of(c);
+    uint8_t* dst = stage0 + st * L.stage;
+    mbar_arrive_expect_tx(&bars.full[st], L.wk_bytes + ut_bytes);
+    bulk_load(dst, blk + ws.off_w, L.wk_bytes, &bars.full[st]);
+    bulk_load(dst + L.wk_bytes, blk + ws.off_ut + (size_t)s0 * 2 * kSlab64, ut_bytes, &bars.full[st]);
+    return true;
+  };
+  int issued = 0;
+  bool ok = true;
+  for (; issued < nC && issued < nst; ++issued) load(issued);
+  for (int c = 0; c < nC && ok; ++c) {
+    const int b = c % kChainBufs;
+    // chunk c - 1's stores have read their buffer: the chain may reuse it
+    // (for chunk c + 2's start state, at the end of its chunk c + 1)
+    if (c >= 1) {
+      bulk_wait_read();
+      mbar_arrive(&bars.freed[(c - 1) % kChainBufs]);
+    }
+    // publish chunk c once every group has staged it
+    if (!mbar_wait(&bars.staged[b], (c / kChainBufs) & 1, limit)) {
+      ok = false;
+      break;
+    }
+    uint8_t* blk = block_of(c);
+    for (int gw = 0; gw < active; ++gw) {
+      const uint8_t* sb = smem + L.groups + gw * L.group + b * L.stg;
+      bulk_store_nc(blk + ws.off_s + (size_t)(s0 + gw) * 2 * Dk * 16, sb, L.stg_s);
+      bulk_store_nc(blk + ws.off_u + (size_t)(s0 + gw) * 2 * kSlab64, sb + L.stg_s, 2 * kSlab64);
+    }
+    bulk_commit();
+    // refill the stage chunk c used with chunk c + nst
+    if (issued < nC) {
+      if (!load(issued)) {
+        ok = false;
+        break;
+      }
+      ++issued;
+    }
+  }
+  bulk_wait_all();
+  if (!ok) atomicOr(err, kErrTimeout);
+  // nothing may still be landing in shared memory when the CTA leaves:
+  // wait for the last load issued into each stage (bounded by the timer)
+  for (int st = 0; st < nst && st < issued; ++st) {
+    const int last = st + ((issued - 1 - st) / nst) * nst;
+    mbar_wait(&bars.full[st], (last / nst) & 1, kDrainPolls);
+  }
+}
+
+template <int NKB>
+__global__ void __launch_bounds__(32 * (kChainMaxGroups * 4 + 1), 1)
+gdn_recur_kernel(const float* state_in, float* state_out, Workspace ws, int ns, int nst,
+                 long long limit, unsigned* err) {
+  constexpr int P = chain_group_warps(NKB);
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  RecSmemHead& hd = *reinterpret_cast<RecSmemHead*>(smem_raw);
+  ChainBars& bars = *reinterpret_cast<ChainBars*>(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int s0 = blockIdx.x * ns;
+  const int active = min(ns, ws.Dv / 16 - s0);  // slice groups with a slice
+  const ChainLayout L(ws.Dk, ns, nst);
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NST; ++i) mbar_init(&hd.full[i], 1);
+    for (int i = 0; i < nst; ++i) {
+      mbar_init(&bars.full[i], 1);
+      mbar_init(&bars.empty[i], active * P);
+    }
+    for (int i = 0; i < kChainBufs; ++i) {
+      mbar_init(&bars.staged[i], active);
+      mbar_init(&bars.freed[i], 1);
+    }
+    for (int i = 0; i < kChainMaxGroups; ++i) bars.fail[i] = 0;
     fence_mbar_init();
   }
   __syncthreads();
-  pdl_wait();  // stage A's summaries are complete and visible
+  pdl_wait();  // stage A's W, K~, U~ are complete and visible
   pdl_trigger();
-  recur_body<NKS, NST>(smem_raw, state_in, state_out, ws, limit, err);
+  const int gw = warp / P, q = warp - gw * P;
+  if (gw < active)
+    chain_warp<NKB>(smem_raw, L, nst, gw, q, s0 + gw, state_in, state_out, ws, limit, err);
+  else if (warp == ns * P && lane == 0)
+    chain_producer(smem_raw, L, nst, active, s0, ws, limit, err);
+  __syncthreads();
 }
 
-// The recurrence kernel for Dk = 16 * nks with an nst-stage load ring.
-using RecurKernel = void (*)(const float*, float*, Workspace, long long, unsigned*);
-template <int NST>
-RecurKernel recur_kernel_st(int nks) {
-  switch (nks) {
-    case 1: return gdn_recur_kernel<1, NST>;
-    case 2: return gdn_recur_kernel<2, NST>;
-    case 3: return gdn_recur_kernel<3, NST>;
-    case 4: return gdn_recur_kernel<4, NST>;
-    case 5: return gdn_recur_kernel<5, NST>;
-    case 6: return gdn_recur_kernel<6, NST>;
-    case 7: return gdn_recur_kernel<7, NST>;
-    default: return gdn_recur_kernel<8, NST>;
+// The recurrence kernel for Dk = 16 * nkb.
+using RecurKernel = void (*)(const float*, float*, Workspace, int, int, long long, unsigned*);
+RecurKernel recur_kernel(int nkb) {
+  switch (nkb) {
+    case 1: return gdn_recur_kernel<1>;
+    case 2: return gdn_recur_kernel<2>;
+    case 3: return gdn_recur_kernel<3>;
+    case 4: return gdn_recur_kernel<4>;
+    case 5: return gdn_recur_kernel<5>;
+    case 6: return gdn_recur_kernel<6>;
+    case 7: return gdn_recur_kernel<7>;
+    default: return gdn_recur_kernel<8>;
   }
-}
-RecurKernel recur_kernel(int nks, int nst) {
-  return nst >= 4 ? recur_kernel_st<4>(nks) : nst == 3 ? recur_kernel_st<3>(nks) : recur_kernel_st<2>(nks);
 }
 
 // ========================================================== stage C: output
@@ -793,27 +886,25 @@ RecurKernel recur_kernel(int nks, int nst) {
 // land while the current tile computes.  Per set (offsets from Dk, Dv):
 //   Q   [Dk/8][64][8]  raw q tile (TMA)
 //   K   [Dk/8][64][8]  raw k tile (TMA); after P = Q K^T it holds Qs = diag(e^g) Q
-//   W   [Dk/8][64][8]  W of the current direction     } one contiguous block,
-//   Ut  [Dv/8][64][8]  U~, then U in place            } as in the workspace:
-//   S   [Dv/8][Dk][8]  state at the chunk's start     } a single bulk copy
+//   U   [Dv/8][64][8]  U = U~ - W S0 of the current direction } one block, as in
+//   S   [Dv/8][Dk][8]  state at the chunk's start             } the workspace
 // then P [8][64][8] (masked, gated Q K^T, K-major A) and the scalar block.
 struct OutSmall {
   float g[2][64];
   float gam[64], rnq[2][64], rnk[2][64], arow[64];  // norms per tile set
   float bcol[8][64];
-  uint64_t tma_bar[2], ld_bar[2], mma_bar;
+  uint64_t tma_bar[2], ld_bar[2], mma_bar, p_bar;
   uint64_t fin_bar;  // one commit on a failed wait: every MMA issued has landed
   uint32_t tmem;
 };
 struct OutLayout {
-  uint32_t q, k, w, ut, s, set_bytes, p, small, total;
+  uint32_t q, k, u, s, set_bytes, p, small, total;
   __host__ __device__ OutLayout(int Dk, int Dv) {
     auto al = [](uint32_t x) { return (x + 127u) & ~127u; };
     q = 0;
     k = al(q + 64u * Dk * 2);
-    w = al(k + 64u * Dk * 2);
-    ut = w + 64u * Dk * 2;
-    s = ut + 64u * Dv * 2;
+    u = al(k + 64u * Dk * 2);
+    s = u + 64u * Dv * 2;
     set_bytes = al(s + (uint32_t)Dk * Dv * 2);
     p = 2 * set_bytes;
     small = al(p + 8u * kSlab64);
@@ -840,19 +931,19 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
   uint8_t* sP = smem + L.p;
   const uint32_t tm = sm.tmem;
   const uint32_t tmP = tm, tmO = tm + 64;
-  const uint32_t wbytes = kC * Dk * 2, ubytes = kC * Dv * 2, sbytes = Dk * Dv * 2;
+  const uint32_t ubytes = kC * Dv * 2, sbytes = Dk * Dv * 2;
   // warps w, w + 4, w + 8, w + 12 share TMEM lane quadrant w % 4 and split
   // the column blocks four ways
   const int quad = warp & 3, part = warp >> 2;
   const int r = 16 * quad + (lane & 15);
   const uint32_t lane_base = static_cast<uint32_t>(32 * quad) << 16;
 
-  auto issue_dir = [&](int set, int tile_t, int dir) {  // thread 0: W | U~ | S
+  auto issue_dir = [&](int set, int tile_t, int dir) {  // thread 0: U | S
     uint8_t* base = smem + set * L.set_bytes;
     const int bh = tile_t / nC, j = tile_t - bh * nC;
     const size_t tile = ws.tile(dir, bh, j);
-    mbar_arrive_expect_tx(&sm.ld_bar[set], wbytes + ubytes + sbytes);
-    bulk_load(base + L.w, ws.blk(tile) + ws.off_w, wbytes + ubytes + sbytes, &sm.ld_bar[set]);
+    mbar_arrive_expect_tx(&sm.ld_bar[set], ubytes + sbytes);
+    bulk_load(base + L.u, ws.blk(tile) + ws.off_u, ubytes + sbytes, &sm.ld_bar[set]);
   };
   // all threads: start loading tile `tile_t` into `set`
   auto issue_tile = [&](int set, int tile_t) {
@@ -873,11 +964,11 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
   };
 
   // mbarrier phase parities: bit `set` of tma_ph / ld_ph
-  uint32_t tma_ph = 0, ld_ph = 0, mma_ph = 0;
+  uint32_t tma_ph = 0, ld_ph = 0, mma_ph = 0, p_ph = 0;
   // Head of the tile in `set`: wait for its q/k tile and gates, issue
-  // P = Q K^T (shared by both directions), then the row norms, which overlap
-  // it.  `one_more`: a later tile's gates are in flight too.  The head of
-  // tile t + 1 runs while tile t's last MMA round executes.
+  // P = Q K^T (shared by both directions) and commit it, then the row norms,
+  // which overlap it.  `one_more`: a later tile's gates are in flight too.
+  // The head of tile t + 1 runs while tile t's last MMA round executes.
   auto head = [&](int set, bool one_more) -> bool {
     uint8_t* base = smem + set * L.set_bytes;
     uint8_t* sQ = base + L.q;
@@ -894,6 +985,7 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
       for (int ks = 0; ks < Dk / 16; ++ks)
         mma_bf16(tmP, sdesc(smem_u32(sQ) + ks * 2 * kSlab64, kSlab64, 128),
                  sdesc(smem_u32(sK) + ks * 2 * kSlab64, kSlab64, 128), idP, ks > 0);
+      mma_commit(&sm.p_bar);
     }
     {  // 1 / |q|, 1 / |k| per row: four threads per row and tensor
       const int row = tid >> 3, part = tid & 3;
@@ -905,8 +997,7 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
   };
 
   // On a failed wait, before leaving: one commit covering every MMA this
-  // CTA issued (P = Q K^T is issued ahead of its commit), so none is still
-  // writing TMEM when the accumulators are freed.
+  // CTA issued, so none is still writing TMEM when the accumulators are freed.
   auto drain_mma = [&]() {
     if (tid == 0) mma_commit(&sm.fin_bar);
     mbar_wait(&sm.fin_bar, 0, kDrainPolls);
@@ -939,18 +1030,13 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
     uint8_t* base = smem + set * L.set_bytes;
     uint8_t* sQ = base + L.q;
     uint8_t* sK = base + L.k;   // then Qs
-    uint8_t* sW = base + L.w;
-    uint8_t* sUt = base + L.ut;  // then U
+    uint8_t* sU = base + L.u;
     uint8_t* sS = base + L.s;
     const int bh = t / nC, j = t - bh * nC;
     const int b = bh / H, h = bh - b * H, t0 = j * kC;
     const int nvalid = min(kC, T - t0);
 
     for (int dir = 0; dir < ndir; ++dir) {
-      // D_U: direction 0 borrows D_O's columns (D_O is first written after
-      // D_U is consumed); direction 1 needs its own, [192, 320) of a
-      // 512-column allocation, because D_O then holds direction 0's sum.
-      const uint32_t tmU = tm + (dir == 0 ? 64u : 192u);
       __syncthreads();
       if (warp == 0) warp_gamma(sm.g[set], sm.gam, dir);
       __syncthreads();
@@ -967,50 +1053,25 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
         const float mb = sm.gam[dir ? 63 - 8 * (p >> 3) : 8 * (p >> 3)];
         sm.arow[tid] = exp2f((sm.gam[tid] - mb) * kLog2e);
       }
+      if (dir == 0) {
+        if (!block_wait(&sm.p_bar, p_ph, limit, err)) {
+          mbar_wait(&sm.ld_bar[set], (ld_ph >> set) & 1, kDrainPolls);
+          drain_other();
+          return false;
+        }
+        p_ph ^= 1;
+      }
       if (!block_wait(&sm.ld_bar[set], (ld_ph >> set) & 1, limit, err)) {
         drain_other();
         return false;
       }
       ld_ph ^= 1u << set;
-      if (tid == 0) {
-        tc_fence_after_sync();
-        // D_U = W S  (M = 64, N = Dv, K = Dk); S read MN-major (N = value column)
-        const uint32_t idU = idesc_bf16(64, Dv, 0, 1);
-        for (int ks = 0; ks < Dk / 16; ++ks)
-          mma_bf16(tmU, sdesc(smem_u32(sW) + ks * 2 * kSlab64, kSlab64, 128),
-                   sdesc(smem_u32(sS) + ks * 256, 128, Dk * 16), idU, ks > 0);
-        mma_commit(&sm.mma_bar);
-      }
-      if (!block_wait(&sm.mma_bar, mma_ph, limit, err)) {
-        drain_other();
-        return false;
-      }
-      mma_ph ^= 1;
       tc_fence_after_sync();
-      // U = U~ - W S, in place of U~ (MN-major B: [slab][64 tokens][8]);
-      // column blocks part and part + 4 of D_U and block part of P are
-      // loaded from TMEM together
+      // P'_ri = (q_r . k_i) / |k_i| * e^{gam_r - gam_i} for i at or before r
       {
-        float u0[16], u1[16], v[16];
-        const bool has1 = part + 4 < Dv / 16;
-        if (part < Dv / 16) tmem_ld16(tmU + lane_base + 16 * part, u0);
-        if (has1) tmem_ld16(tmU + lane_base + 16 * (part + 4), u1);
+        float v[16];
         tmem_ld16(tmP + lane_base + 16 * part, v);
         tmem_wait_ld();
-        auto sub = [&](int c, const float* d) {
-          float ut[16];
-          unpack8_bf16(reinterpret_cast<const uint4*>(sUt + (2 * c) * kSlab64)[r], ut);
-          unpack8_bf16(reinterpret_cast<const uint4*>(sUt + (2 * c + 1) * kSlab64)[r], ut + 8);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) ut[e] -= d[e];
-          reinterpret_cast<uint4*>(sUt + (2 * c) * kSlab64)[r] = pack8_bf16(ut);
-          reinterpret_cast<uint4*>(sUt + (2 * c + 1) * kSlab64)[r] = pack8_bf16(ut + 8);
-        };
-        if (lane < 16) {
-          if (part < Dv / 16) sub(part, u0);
-          if (has1) sub(part + 4, u1);
-        }
-        // P'_ri = (q_r . k_i) / |k_i| * e^{gam_r - gam_i} for i at or before r
         const int c = part;
         if (lane < 16) {
           const float ar = sm.arow[r];
@@ -1038,16 +1099,18 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
       }
       block_sync_async();
       if (tid == 0) {
+        // D_O (+)= Qs S0 (K = Dk) + P' U (K = 64 tokens); S and U read MN-major
         const uint32_t idO = idesc_bf16(64, Dv, 0, 1);
         for (int ks = 0; ks < Dk / 16; ++ks)
           mma_bf16(tmO, sdesc(smem_u32(sK) + ks * 2 * kSlab64, kSlab64, 128),
                    sdesc(smem_u32(sS) + ks * 256, 128, Dk * 16), idO, (dir > 0) || (ks > 0));
         for (int ks = 0; ks < kC / 16; ++ks)
           mma_bf16(tmO, sdesc(smem_u32(sP) + ks * 2 * kSlab64, kSlab64, 128),
-                   sdesc(smem_u32(sUt) + ks * 256, 128, kSlab64), idO, 1);
+                   sdesc(smem_u32(sU) + ks * 256, 128, kSlab64), idO, 1);
         mma_commit(&sm.mma_bar);
       }
       if (dir + 1 < ndir) {
+        // the next direction rewrites P', Qs and this set's U | S
         if (!block_wait(&sm.mma_bar, mma_ph, limit, err)) {
           drain_other();
           return false;
@@ -1056,10 +1119,10 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
         if (tid == 0) issue_dir(set, t, dir + 1);
       }
     }
-    // the last direction's second round is in flight: the next tile's head
+    // the last direction's MMA round is in flight: the next tile's head
     // (its loads, P = Q K^T and norms) runs meanwhile
     if (next_issued && !head(set ^ 1, false)) {
-      // head drained the next tile's q/k; its W | U~ | S and this round remain
+      // head drained the next tile's q/k; its U | S and this round remain
       mbar_wait(&sm.ld_bar[set ^ 1], (ld_ph >> (set ^ 1)) & 1, kDrainPolls);
       drain_mma();
       return false;
@@ -1107,13 +1170,14 @@ gdn_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const OutLayout L(ws.Dk, ws.Dv);
   OutSmall& sm = *reinterpret_cast<OutSmall*>(smem_raw + L.small);
   const int tid = threadIdx.x;
-  const uint32_t ncols = ndir > 1 ? 512u : 256u;
+  const uint32_t ncols = 256u;  // P [0, 64), D_O [64, 64 + Dv)
   if (tid == 0) {
     mbar_init(&sm.tma_bar[0], 1);
     mbar_init(&sm.tma_bar[1], 1);
     mbar_init(&sm.ld_bar[0], 1);
     mbar_init(&sm.ld_bar[1], 1);
     mbar_init(&sm.mma_bar, 1);
+    mbar_init(&sm.p_bar, 1);
     mbar_init(&sm.fin_bar, 1);
     fence_mbar_init();
   }
@@ -1179,23 +1243,6 @@ int num_sms() {
   return cached[dev];
 }
 
-int recur_smem_bytes(int Dk, int nst) {
-  const int stage = ((Dk * Dk * 2 + Dk * 32 + 16) + 127) & ~127;
-  return kRecHeadBytes + 2 * kRecSBytes + nst * stage;
-}
-
-// Stages of stage B's load ring: the full kRecStages while the grid fits one
-// CTA per SM; otherwise the deepest ring (at least 2) that lets two CTAs
-// share an SM, so a grid of more CTAs than SMs (both directions, many heads)
-// still runs in one wave instead of two chained ones.
-int recur_stages(int Dk, int ctas, int sms) {
-  if (ctas <= sms) return kRecStages;
-  constexpr int kHalfSm = 113 * 1024;  // per-CTA share of an SM's shared memory, two CTAs
-  int nst = kRecStages;
-  while (nst > 2 && recur_smem_bytes(Dk, nst) > kHalfSm) --nst;
-  return nst;
-}
-
 // Opt the kernels into their dynamic shared memory, once per device.
 cudaError_t set_smem_attrs() {
   constexpr int kMaxDev = 64;
@@ -1209,16 +1256,66 @@ cudaError_t set_smem_attrs() {
   if (done[dev]) return cudaSuccess;
   e = cudaFuncSetAttribute(gdn_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)sizeof(PrepSmem));
-  if (e == cudaSuccess)
-    for (int nks = 1; nks <= 8 && e == cudaSuccess; ++nks)
-      for (int nst = 2; nst <= kRecStages && e == cudaSuccess; ++nst)
-        e = cudaFuncSetAttribute(recur_kernel(nks, nst), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 recur_smem_bytes(128, nst));
+  for (int nkb = 1; nkb <= 8 && e == cudaSuccess; ++nkb)
+    e = cudaFuncSetAttribute(recur_kernel(nkb), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             227 * 1024);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(gdn_output_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)OutLayout(128, 128).total);
   if (e == cudaSuccess) done[dev] = true;
   return e;
+}
+
+// Stage B's shape: slices (16 state columns, one warp group each) per CTA
+// and load-ring stages, chosen for the fewest waves of CTAs (the occupancy
+// API counts how many fit an SM); among equals, one slice per CTA (its
+// groups then share no issue slots), then the deepest ring.  Cached per
+// (device, Dk, Dv, heads x directions).
+struct ChainShape {
+  int ns, nst;
+};
+ChainShape chain_shape(int Dk, int Dv, int heads_dirs, int sms) {
+  struct Entry {
+    int dev, Dk, Dv, hd;
+    ChainShape shape;
+  };
+  static std::mutex mu;
+  static Entry cache[64];
+  static int used = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i)
+      if (cache[i].dev == dev && cache[i].Dk == Dk && cache[i].Dv == Dv && cache[i].hd == heads_dirs)
+        return cache[i].shape;
+  }
+  const int nslices = Dv / 16;
+  const int P = chain_group_warps(Dk / 16);
+  ChainShape best = {1, 2};
+  long long best_waves = -1;
+  for (int ns = 1; ns <= kChainMaxGroups && ns <= nslices; ns *= 2) {
+    for (int nst = kChainMaxStages; nst >= 2; --nst) {
+      const int smem = (int)ChainLayout(Dk, ns, nst).total;
+      if (smem > 227 * 1024) continue;
+      int per_sm = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, recur_kernel(Dk / 16), 32 * (ns * P + 1),
+                                                        smem) != cudaSuccess) {
+        cudaGetLastError();
+        per_sm = 1;
+      }
+      per_sm = std::max(per_sm, 1);
+      const long long ctas = (long long)((nslices + ns - 1) / ns) * heads_dirs;
+      const long long waves = (ctas + (long long)sms * per_sm - 1) / ((long long)sms * per_sm);
+      if (best_waves < 0 || waves < best_waves) {
+        best_waves = waves;
+        best = {ns, nst};
+      }
+    }
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (used < 64) cache[used++] = {dev, Dk, Dv, heads_dirs, best};
+  return best;
 }
 
 // Launch with programmatic stream serialisation: the kernel may start while
@@ -1274,10 +1371,12 @@ cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
   if (e != cudaSuccess) return e;
   {
     ProfileScope ps(a.stream, kKernRecur);
-    const int nst = recur_stages(a.Dk, (a.Dv / 16) * NBH * ndir, num_sms());
-    e = launch_pdl(recur_kernel(a.Dk / 16, nst), dim3(a.Dv / 16, NBH, ndir), 32 * (a.Dk / 16),
-                   recur_smem_bytes(a.Dk, nst), a.stream, a.state_in, a.state_out, ws,
-                   a.wait_limit, a.err);
+    const ChainShape cs = chain_shape(a.Dk, a.Dv, NBH * ndir, num_sms());
+    const int nslices = a.Dv / 16;
+    e = launch_pdl(recur_kernel(a.Dk / 16), dim3((nslices + cs.ns - 1) / cs.ns, NBH, ndir),
+                   32 * (cs.ns * chain_group_warps(a.Dk / 16) + 1),
+                   ChainLayout(a.Dk, cs.ns, cs.nst).total, a.stream, a.state_in,
+                   a.state_out, ws, cs.ns, cs.nst, a.wait_limit, a.err);
   }
   if (e != cudaSuccess) return e;
   {

@@ -93,7 +93,7 @@ def test_small_sweep_unnormalised_qk(T, D, mode, dtype):
     check(w, xh, out, S, per_head=True)
 
 
-@pytest.mark.parametrize("Dk,Dv", [(32, 96), (128, 16), (64, 128)])
+@pytest.mark.parametrize("Dk,Dv", [(32, 96), (128, 16), (64, 128), (48, 64), (80, 32), (96, 112)])
 def test_rectangular_state(Dk, Dv):
     """Dk != Dv (the state is Dk x Dv; outputs are Dv wide)."""
     w = wl.Workload("rect", 1, 130, 2, Dk, Dv, "bf16", 64, "fwd",
