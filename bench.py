@@ -71,11 +71,17 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def gate_keys(w):
+    """Input names of the gates: g and beta, or the gate layer's logits for
+    the fused-prologue workloads."""
+    return ("g_logit", "beta_logit") if w.gate[0] == "logit_normal" else ("g", "beta")
+
+
 def algorithmic_bytes(w) -> int:
-    """q, k, v, out (dtype) + g, beta (fp32) per token-head, plus the fp32
-    state read and written once per (b, h)."""
+    """q, k, v, out (dtype) + g, beta (fp32; gate logits in the dtype) per
+    token-head, plus the fp32 state read and written once per (b, h)."""
     es = 2 if w.dtype == "bf16" else 4
-    per_tok = (2 * w.Dk + 2 * w.Dv) * es + 8
+    per_tok = (2 * w.Dk + 2 * w.Dv) * es + (2 * es if w.gate[0] == "logit_normal" else 8)
     return w.head_tokens * per_tok + 2 * w.B * w.H * w.Dk * w.Dv * 4
 
 
@@ -313,8 +319,9 @@ def make_sets(w, xh, dev, n):
     state_out, so consecutive steps read different buffers."""
     import torch
     dt = torch.bfloat16
-    base = {k: torch.from_numpy(xh[k]).to(dev) for k in ("q", "k", "v", "g", "beta")}
-    for k in ("q", "k", "v"):
+    gk = gate_keys(w)
+    base = {k: torch.from_numpy(xh[k]).to(dev) for k in ("q", "k", "v", *gk)}
+    for k in ("q", "k", "v") + (gk if gk[0] == "g_logit" else ()):
         base[k] = base[k].to(dt)
     base["state_in"] = torch.from_numpy(xh["state_in"]).to(dev)
     sets = []
@@ -332,9 +339,9 @@ class Stepper:
     stream comes first, so the library's per-stream scratch exists before any
     capture and the graphs hold kernel nodes only (no memory nodes)."""
 
-    def __init__(self, fn, sets, stream, chunk, use_graph):
+    def __init__(self, fn, sets, stream, chunk, use_graph, gates=("g", "beta")):
         import torch
-        self.fn, self.sets, self.stream, self.chunk = fn, sets, stream, chunk
+        self.fn, self.sets, self.stream, self.chunk, self.gates = fn, sets, stream, chunk, gates
         self.graphs = []
         with torch.cuda.stream(stream):
             self.call(0)
@@ -349,8 +356,8 @@ class Stepper:
 
     def call(self, i):
         s = self.sets[i % len(self.sets)]
-        self.fn(s["q"], s["k"], s["v"], s["g"], s["beta"], s["state_in"], state_out=s["state_out"],
-                out=s["out"], chunk=self.chunk, stream=self.stream)
+        self.fn(s["q"], s["k"], s["v"], s[self.gates[0]], s[self.gates[1]], s["state_in"],
+                state_out=s["state_out"], out=s["out"], chunk=self.chunk, stream=self.stream)
 
     def run(self, n, offset=0):
         import torch
@@ -641,6 +648,31 @@ def main():
             res["bound_latent_frames_per_s"] = frames / (res["calls"] * max(
                 roofline_times(ws, smode == "bidir", peaks)))
             extras[f"stack_32x15_{smode}"] = res
+        # the fused gate prologue: the causal chunk with the gate layer's bf16
+        # logits as inputs (own input sets, graph-timed like the main figure)
+        wlg = wl.stream_chunk_logits("fwd", seed=w_r.seed)
+        _, lsets = make_sets(wlg, wl.make_inputs(wlg), dev, N_SETS)
+        with nvtx("fwd_logits_chunk"):
+            lg = Stepper(gdn.chunk_fwd_logits, lsets, stream, w.chunk, use_graph, gate_keys(wlg))
+            lg.warm(max(3, args.warmup))
+            barrier()
+            a0.record(stream)
+            lg.run(n_side)
+            a1.record(stream)
+            barrier()
+            lg.release()
+        lg_ms = a0.elapsed_time(a1) / n_side
+
+        def lg_direct(i):
+            with torch.cuda.stream(stream):
+                lg.call(i)
+        extras["fwd_logits_chunk"] = {
+            "workload": wlg.name, "ms_per_step": lg_ms,
+            "head_tokens_per_s": w.head_tokens / (lg_ms / 1000.0), "steps": n_side,
+            "timing": "CUDA graph replays" if use_graph else "direct calls",
+            "roofline": roofline_of(wlg, kernel_times(lib, lg_direct, n_prof, launches_per_step),
+                                    lg_ms, peaks, peak_kind, False)}
+        del lsets
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -30,6 +30,8 @@ SIGNATURES = {
     "gdn_chunk_fwd": (ctypes.c_int, _SCAN_ARGS),
     "gdn_chunk_bidir": (ctypes.c_int, _SCAN_ARGS),
     "gdn_chunk_fwd_noalloc": (ctypes.c_int, _SCAN_ARGS),
+    "gdn_chunk_fwd_logits": (ctypes.c_int, _SCAN_ARGS),
+    "gdn_chunk_bidir_logits": (ctypes.c_int, _SCAN_ARGS),
     "gdn_state_reset": (ctypes.c_int, [_fp, _i, _i, _i, _i, _vp]),
     "gdn_device_error": (ctypes.c_int, [_vp]),
     "gdn_workspace_release": (ctypes.c_int, []),

@@ -41,7 +41,7 @@ def _check_tensor(t, name, dtype=None, shape=None):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
-def _scan(entry, q, k, v, g, beta, state_in, state_out, out, chunk, stream):
+def _scan(entry, q, k, v, g, beta, state_in, state_out, out, chunk, stream, logits=False):
     if q.dim() != 4 or v.dim() != 4:
         raise ValueError("q, k must be [B,T,H,Dk] and v [B,T,H,Dv]")
     B, T, H, Dk = q.shape
@@ -52,8 +52,9 @@ def _scan(entry, q, k, v, g, beta, state_in, state_out, out, chunk, stream):
     _check_tensor(q, "q", dt)
     _check_tensor(k, "k", dt, (B, T, H, Dk))
     _check_tensor(v, "v", dt, (B, T, H, Dv))
-    _check_tensor(g, "g", torch.float32, (B, T, H))
-    _check_tensor(beta, "beta", torch.float32, (B, T, H))
+    gdt = dt if logits else torch.float32  # gate logits come in the I/O dtype
+    _check_tensor(g, "g_logit" if logits else "g", gdt, (B, T, H))
+    _check_tensor(beta, "beta_logit" if logits else "beta", gdt, (B, T, H))
     if state_in is not None:
         _check_tensor(state_in, "state_in", torch.float32, (B, H, Dk, Dv))
     if state_out is None:
@@ -84,6 +85,22 @@ def chunk_bidir(q, k, v, g, beta, state_in=None, state_out=None, out=None, chunk
     """Forward scan from ``state_in`` plus the in-chunk reverse scan from zero,
     summed.  ``state_out`` is the forward scan's final state."""
     return _scan("gdn_chunk_bidir", q, k, v, g, beta, state_in, state_out, out, chunk, stream)
+
+
+def chunk_fwd_logits(q, k, v, g_logit, beta_logit, state_in=None, state_out=None, out=None,
+                     chunk=0, stream=None):
+    """Causal scan with the fused gate prologue: ``g_logit`` and ``beta_logit``
+    [B,T,H] (same dtype as q) are the gate layer's logits; the library forms
+    g = -softplus(g_logit) and beta = sigmoid(beta_logit) itself."""
+    return _scan("gdn_chunk_fwd_logits", q, k, v, g_logit, beta_logit, state_in, state_out, out,
+                 chunk, stream, logits=True)
+
+
+def chunk_bidir_logits(q, k, v, g_logit, beta_logit, state_in=None, state_out=None, out=None,
+                       chunk=0, stream=None):
+    """Bidirectional scan with the fused gate prologue (see chunk_fwd_logits)."""
+    return _scan("gdn_chunk_bidir_logits", q, k, v, g_logit, beta_logit, state_in, state_out, out,
+                 chunk, stream, logits=True)
 
 
 def state_reset(state, stream=None):

@@ -48,6 +48,7 @@
 #include <mutex>
 #include <utility>
 
+#include "gates.cuh"
 #include "gdn_internal.h"
 #include "sm100.cuh"
 
@@ -68,13 +69,14 @@ constexpr long long kDrainPolls = 1LL << 40;  // drains are bounded by the 2 s t
 //   W     [Dk/8][64][8]   bf16                        (A writes, B reads)
 //   Kt    [Dk/8][64][8]   bf16  K~                    (A writes, B reads)
 //   decay {e^{gamma_C}, 0, 0, 0} fp32                 (A writes, B reads)
+//   g     [64]            fp32  the tile's gates      (A writes, C reads)
 //   Ut    [Dv/8][64][8]   bf16  U~                    (A writes, B reads)
 //   U     [Dv/8][64][8]   bf16  U = U~ - W S0         (B writes, C reads)
 //   S     [Dv/8][Dk][8]   bf16  state at chunk start  (B writes, C reads)
 struct Workspace {
   uint8_t* base;
   size_t block_bytes;
-  uint32_t off_w, off_kt, off_decay, off_ut, off_u, off_s;
+  uint32_t off_w, off_kt, off_decay, off_g, off_ut, off_u, off_s;
   int NBH, nC, Dk, Dv;
 
   __host__ __device__ void layout(int dk, int dv) {
@@ -83,7 +85,8 @@ struct Workspace {
     off_w = 0;
     off_kt = off_w + 64u * Dk * 2;
     off_decay = off_kt + 64u * Dk * 2;
-    off_ut = off_decay + 16;
+    off_g = off_decay + 16;
+    off_ut = off_g + 64u * 4;
     off_u = off_ut + 64u * Dv * 2;
     off_s = off_u + 64u * Dv * 2;
     block_bytes = ((size_t)off_s + (size_t)Dk * Dv * 2 + 255) & ~size_t(255);
@@ -168,6 +171,7 @@ struct PrepSmem {
   float g[64], beta[64], gam[64], rn[64], csW[64], csU[64];
   float arow[64];      // beta_r |k_r|^-1 e^{gam_r - m_b(r)}       (scan order)
   float bcol[8][64];   // |k_q|^-1 e^{m_b - gam_q}, b = 8-row block (scan order)
+  float dg[64][8];     // A's factor inside p's own 8-row block       (scan order)
   uint64_t tma_bar, v_bar, mma_bar;  // K tile, V tile, MMA completion
   uint32_t tmem;
 };
@@ -276,7 +280,7 @@ __device__ __forceinline__ int scan_pos(int r) { return REV ? 63 - r : r; }
 
 template <int REV>
 __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
-                          const float* __restrict__ g, const float* __restrict__ beta,
+                          const void* __restrict__ g, const void* __restrict__ beta, int logits,
                           const Workspace& ws, int T, int H, long long limit, unsigned* err) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int j = blockIdx.x, bh = blockIdx.y, dir = REV;
@@ -296,11 +300,18 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
     float gv = 0.f, bv = 0.f;  // padding rows: a = 1, beta = 0 (no effect)
     if (tid < nvalid) {
       const size_t row = ((size_t)b * T + t0 + tid) * H + h;
-      gv = __ldg(g + row);
-      bv = __ldg(beta + row);
+      if (logits) {  // the fused prologue: the gate layer's bf16 logits
+        gv = gate_g_from_logit(__bfloat162float(static_cast<const __nv_bfloat16*>(g)[row]));
+        bv = gate_beta_from_logit(__bfloat162float(static_cast<const __nv_bfloat16*>(beta)[row]));
+      } else {
+        gv = __ldg(static_cast<const float*>(g) + row);
+        bv = __ldg(static_cast<const float*>(beta) + row);
+      }
     }
     s.g[tid] = gv;
     s.beta[tid] = bv;
+    // stage C takes the tile's gates from here, in both modes
+    if (dir == 0) reinterpret_cast<float*>(ws.blk(ws.tile(0, bh, j)) + ws.off_g)[tid] = gv;
   }
   __syncthreads();
   if (warp == 0) warp_gamma(s.g, s.gam, REV);
@@ -339,16 +350,22 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
   tc_fence_after_sync();
 
   // A[p][q] = beta_r e^{gam_r - gam_i} G_ri / (|k_r| |k_i|) for scan positions
-  // q < p, formed as arow[p] G bcol[b(p)][q]: the gate factor is split at
-  // m_b = gam at the first scan position of p's 8-row block b, so both factors
-  // are bounded (|gam_r - m_b| and, inside the block, |m_b - gam_i| span at
-  // most 7 tokens) and only 8 x 64 + 64 exponentials are taken per tile.
+  // q < p.  For q in an earlier 8-row block than p's block b the gate factor
+  // is split at m_b = gam at b's first scan position, A = arow[p] G bcol[b][q]:
+  // both exponents are <= 0, so the factors are exact (one underflows only
+  // when the product does).  Inside the diagonal block the whole factor
+  // beta_r e^{gam_r - gam_i} / (|k_r| |k_i|) <= 1 comes from dg[p] (the split
+  // would put e^{m_b - gam_i}, up to e^{7 |g|}, in one factor).
   {
     for (int e = tid; e < 8 * 64; e += kWideThreads) {
       const int blk = e >> 6, q = e & 63;
       const int i = REV ? 63 - q : q;
       const float mb = s.gam[REV ? 63 - 8 * blk : 8 * blk];
-      s.bcol[blk][q] = (q < 8 * blk + 8) ? s.rn[i] * exp2f((mb - s.gam[i]) * kLog2e) : 0.f;
+      s.bcol[blk][q] = q < 8 * blk ? s.rn[i] * exp2f((mb - s.gam[i]) * kLog2e) : 0.f;
+      const int p = e >> 3, qd = (p & ~7) + (e & 7);  // row p, column qd of its block
+      const int r = REV ? 63 - p : p, id = REV ? 63 - qd : qd;
+      s.dg[p][e & 7] = qd < p ? s.beta[r] * s.rn[r] * s.rn[id] * exp2f((s.gam[r] - s.gam[id]) * kLog2e)
+                              : 0.f;
     }
     if (tid < 64) {
       const int p = tid, r = REV ? 63 - p : p;
@@ -368,20 +385,22 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
     tmem_ld16(tm + lane_base + i0 + 16, *reinterpret_cast<float(*)[16]>(v + 16));
     tmem_wait_ld();
     if (lane < 16) {
-      const float ap = s.arow[p];
       const float* bc = s.bcol[p >> 3];
+      const int pb = p & ~7;  // first column of p's own block
       float* Arow = s.u.A[p];
 #pragma unroll
       for (int q4 = 0; q4 < 8; ++q4) {
         const int qb = 32 * half + 4 * q4;
-        const float4 b4 = *reinterpret_cast<const float4*>(bc + qb);
+        // earlier blocks: arow[p] bcol[b][q]; own block: dg[p][q - pb]; later: 0
+        const bool own = (qb & ~7) == pb;
+        const float sc = own ? 1.f : s.arow[p];
+        const float4 b4 = *reinterpret_cast<const float4*>(own ? &s.dg[p][qb - pb] : bc + qb);
         const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
         float o[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int q = qb + e;
           const int iv = REV ? 31 - (4 * q4 + e) : 4 * q4 + e;  // index into v
-          o[e] = (q < p) ? ap * v[iv] * bb[e] : 0.f;
+          o[e] = sc * v[iv] * bb[e];
         }
         *reinterpret_cast<float4*>(Arow + qb) = make_float4(o[0], o[1], o[2], o[3]);
       }
@@ -473,8 +492,8 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
 
 __global__ void __launch_bounds__(kWideThreads, 2)
 gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                const float* __restrict__ g, const float* __restrict__ beta, Workspace ws, int T,
-                int H, long long limit, unsigned* err) {
+                const void* __restrict__ g, const void* __restrict__ beta, int logits, Workspace ws,
+                int T, int H, long long limit, unsigned* err) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   PrepSmem& s = *reinterpret_cast<PrepSmem*>(smem_raw);
   const int tid = threadIdx.x;
@@ -494,9 +513,9 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
   pdl_wait();
   pdl_trigger();
   if (blockIdx.z == 0)
-    prep_body<0>(s, &tm_k, &tm_v, g, beta, ws, T, H, limit, err);
+    prep_body<0>(s, &tm_k, &tm_v, g, beta, logits, ws, T, H, limit, err);
   else
-    prep_body<1>(s, &tm_k, &tm_v, g, beta, ws, T, H, limit, err);
+    prep_body<1>(s, &tm_k, &tm_v, g, beta, logits, ws, T, H, limit, err);
   tc_fence_before_sync();
   __syncthreads();
   if ((tid >> 5) == 0) tmem_dealloc(s.tmem, 256);
@@ -893,6 +912,7 @@ struct OutSmall {
   float g[2][64];
   float gam[64], rnq[2][64], rnk[2][64], arow[64];  // norms per tile set
   float bcol[8][64];
+  float dg[64][8];  // P's gate factor inside row r's own 8-row block (memory order)
   uint64_t tma_bar[2], ld_bar[2], mma_bar, p_bar;
   uint64_t fin_bar;  // one commit on a failed wait: every MMA issued has landed
   uint32_t tmem;
@@ -920,9 +940,8 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
-                            const float* __restrict__ g, __nv_bfloat16* __restrict__ out,
-                            const Workspace& ws, int T, int H, int ndir, long long limit,
-                            unsigned* err) {
+                            __nv_bfloat16* __restrict__ out, const Workspace& ws, int T, int H,
+                            int ndir, long long limit, unsigned* err) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Dk = ws.Dk, Dv = ws.Dv, nC = ws.nC;
   const int ntiles = nC * ws.NBH;
@@ -956,9 +975,8 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
       tma_load_tile(base + L.k, tm_k, &sm.tma_bar[set], t0, h, b);
       issue_dir(set, tile_t, 0);
     }
-    if (tid < kC) {
-      if (tid < T - t0) cp_async4(&sm.g[set][tid], g + ((size_t)b * T + t0 + tid) * H + h);
-      else sm.g[set][tid] = 0.f;
+    if (tid < kC) {  // the tile's gates, as stage A formed them (0 past T)
+      cp_async4(&sm.g[set][tid], ws.blk(ws.tile(0, bh, j)) + ws.off_g + 4 * tid);
       cp_async_commit();
     }
   };
@@ -1040,13 +1058,18 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
       __syncthreads();
       if (warp == 0) warp_gamma(sm.g[set], sm.gam, dir);
       __syncthreads();
-      // Gate factors split at m_b = gam at the first scan position of each
-      // 8-row block (as in stage A): P'_ri = arow_r P_ri bcol[b(r)][i].
+      // Gate factors as in stage A: for i in an earlier 8-row block than r's
+      // block b, split at m_b = gam at b's first scan position,
+      // P'_ri = arow_r P_ri bcol[b][i] (both factors <= 1); inside the
+      // diagonal block e^{gam_r - gam_i} is taken whole.
       for (int e = tid; e < 8 * 64; e += kOutThreads) {
         const int blk = e >> 6, i = e & 63;
         const int qpos = dir ? 63 - i : i;
         const float mb = sm.gam[dir ? 63 - 8 * blk : 8 * blk];
-        sm.bcol[blk][i] = (qpos < 8 * blk + 8) ? sm.rnk[set][i] * exp2f((mb - sm.gam[i]) * kLog2e) : 0.f;
+        sm.bcol[blk][i] = qpos < 8 * blk ? sm.rnk[set][i] * exp2f((mb - sm.gam[i]) * kLog2e) : 0.f;
+        const int r = e >> 3, id = (r & ~7) + (e & 7);  // row r, column id of its block
+        const bool incl = dir ? (id >= r) : (id <= r);
+        sm.dg[r][e & 7] = incl ? sm.rnk[set][id] * exp2f((sm.gam[r] - sm.gam[id]) * kLog2e) : 0.f;
       }
       if (tid < 64) {
         const int p = dir ? 63 - tid : tid;
@@ -1076,11 +1099,13 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
         if (lane < 16) {
           const float ar = sm.arow[r];
           const float* bc = sm.bcol[(dir ? 63 - r : r) >> 3];
+          const int rb = r & ~7;  // first column of r's own block
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int i = 16 * c + e;
-            const bool incl = dir ? (i >= r) : (i <= r);
-            v[e] = incl ? ar * v[e] * bc[i] : 0.f;
+            // own block: dg (gate factor taken whole); elsewhere the split
+            // factors (zero for columns the mask excludes)
+            v[e] = (i & ~7) == rb ? v[e] * sm.dg[r][i - rb] : ar * v[e] * bc[i];
           }
           reinterpret_cast<uint4*>(sP + (2 * c) * kSlab64)[r] = pack8_bf16(v);
           reinterpret_cast<uint4*>(sP + (2 * c + 1) * kSlab64)[r] = pack8_bf16(v + 8);
@@ -1164,8 +1189,8 @@ __device__ bool output_body(uint8_t* smem, const CUtensorMap* tm_q, const CUtens
 
 __global__ void __launch_bounds__(kOutThreads, 1)
 gdn_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const float* __restrict__ g, __nv_bfloat16* __restrict__ out, Workspace ws, int T,
-                  int H, int ndir, long long limit, unsigned* err) {
+                  __nv_bfloat16* __restrict__ out, Workspace ws, int T, int H, int ndir,
+                  long long limit, unsigned* err) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const OutLayout L(ws.Dk, ws.Dv);
   OutSmall& sm = *reinterpret_cast<OutSmall*>(smem_raw + L.small);
@@ -1188,7 +1213,7 @@ gdn_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   block_sync_async();
   pdl_wait();  // stage B's chunk-start states are complete and visible
   pdl_trigger();
-  output_body(smem_raw, &tm_q, &tm_k, g, out, ws, T, H, ndir, limit, err);
+  output_body(smem_raw, &tm_q, &tm_k, out, ws, T, H, ndir, limit, err);
   tc_fence_before_sync();
   __syncthreads();
   if ((tid >> 5) == 0) tmem_dealloc(sm.tmem, ncols);
@@ -1366,7 +1391,7 @@ cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
   {
     ProfileScope ps(a.stream, kKernPrep);
     e = launch_pdl(gdn_prep_kernel, dim3(nC, NBH, ndir), kWideThreads, sizeof(PrepSmem), a.stream,
-                   mk, mv, a.g, a.beta, ws, a.T, a.H, a.wait_limit, a.err);
+                   mk, mv, a.g, a.beta, a.gate_logits ? 1 : 0, ws, a.T, a.H, a.wait_limit, a.err);
   }
   if (e != cudaSuccess) return e;
   {
@@ -1382,7 +1407,7 @@ cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
   {
     ProfileScope ps(a.stream, kKernOutput);
     e = launch_pdl(gdn_output_kernel, dim3(std::min(nC * NBH, num_sms())), kOutThreads,
-                   OutLayout(a.Dk, a.Dv).total, a.stream, mq, mk, a.g,
+                   OutLayout(a.Dk, a.Dv).total, a.stream, mq, mk,
                    static_cast<__nv_bfloat16*>(a.out), ws, a.T, a.H, ndir, a.wait_limit, a.err);
   }
   if (e == cudaSuccess) count_launches(3);

@@ -203,14 +203,14 @@ gdn_status stream_context(int dev, cudaStream_t s, size_t bytes, unsigned int** 
   return GDN_OK;
 }
 
-gdn_status scan(const void* q, const void* k, const void* v, const float* g,
-                const float* beta, const float* state_in, float* state_out,
+gdn_status scan(const void* q, const void* k, const void* v, const void* g,
+                const void* beta, const float* state_in, float* state_out,
                 void* out, int B, int T, int H, int Dk, int Dv, gdn_dtype dtype,
-                int chunk, void* stream, bool bidir) {
+                int chunk, void* stream, bool bidir, bool gate_logits) {
   ScanArgs a;
   int dev = 0;
   gdn_status st = prepare_scan(q, k, v, g, beta, state_in, state_out, out, B, T, H, Dk, Dv,
-                               dtype, chunk, stream, bidir, &a, &dev);
+                               dtype, chunk, stream, bidir, gate_logits, &a, &dev);
   if (st != GDN_OK) return st;
   if (a.B == 0 || a.H == 0) return GDN_OK;
   if (a.T == 0) return trivial_state_copy(a);
@@ -246,10 +246,11 @@ gdn_status scan(const void* q, const void* k, const void* v, const float* g,
 
 }  // namespace
 
-gdn_status prepare_scan(const void* q, const void* k, const void* v, const float* g,
-                        const float* beta, const float* state_in, float* state_out,
+gdn_status prepare_scan(const void* q, const void* k, const void* v, const void* g,
+                        const void* beta, const float* state_in, float* state_out,
                         void* out, int B, int T, int H, int Dk, int Dv, gdn_dtype dtype,
-                        int chunk, void* stream, bool bidir, ScanArgs* a, int* dev_out) {
+                        int chunk, void* stream, bool bidir, bool gate_logits, ScanArgs* a,
+                        int* dev_out) {
   // ---- pure host checks (no CUDA call)
   if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
   if (B < 0 || T < 0 || H < 0 || Dk < 0 || Dv < 0) return GDN_ERR_INVALID_ARG;
@@ -261,7 +262,7 @@ gdn_status prepare_scan(const void* q, const void* k, const void* v, const float
   a->q = q; a->k = k; a->v = v; a->g = g; a->beta = beta;
   a->state_in = state_in; a->state_out = state_out; a->out = out;
   a->B = B; a->T = T; a->H = H; a->Dk = Dk; a->Dv = Dv;
-  a->dtype = dtype; a->chunk = chunk; a->bidir = bidir;
+  a->dtype = dtype; a->chunk = chunk; a->bidir = bidir; a->gate_logits = gate_logits;
   a->stream = static_cast<cudaStream_t>(stream);
   a->err = nullptr;
   a->wait_limit = 0;
@@ -273,7 +274,8 @@ gdn_status prepare_scan(const void* q, const void* k, const void* v, const float
   const size_t state_bytes = (size_t)B * H * Dk * Dv * sizeof(float);
   const Range rq = range_of(q, rows * Dk * es), rk = range_of(k, rows * Dk * es);
   const Range rv = range_of(v, rows * Dv * es), ro = range_of(out, rows * Dv * es);
-  const Range rg = range_of(g, rows * 4), rb = range_of(beta, rows * 4);
+  const size_t gs = gate_logits ? es : 4;  // logits come in the I/O dtype
+  const Range rg = range_of(g, rows * gs), rb = range_of(beta, rows * gs);
   const Range rsi = range_of(state_in, state_in ? state_bytes : 0);
   const Range rso = range_of(state_out, state_out ? state_bytes : 0);
 
@@ -371,7 +373,7 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v,
                          int B, int T, int H, int Dk, int Dv, gdn_dtype dtype,
                          int chunk, void* stream) {
   return gdn::scan(q, k, v, g, beta, state_in, state_out, out, B, T, H, Dk, Dv,
-                   dtype, chunk, stream, false);
+                   dtype, chunk, stream, false, false);
 }
 
 gdn_status gdn_chunk_bidir(const void* q, const void* k, const void* v,
@@ -380,7 +382,25 @@ gdn_status gdn_chunk_bidir(const void* q, const void* k, const void* v,
                            int B, int T, int H, int Dk, int Dv,
                            gdn_dtype dtype, int chunk, void* stream) {
   return gdn::scan(q, k, v, g, beta, state_in, state_out, out, B, T, H, Dk, Dv,
-                   dtype, chunk, stream, true);
+                   dtype, chunk, stream, true, false);
+}
+
+gdn_status gdn_chunk_fwd_logits(const void* q, const void* k, const void* v,
+                                const void* g_logit, const void* beta_logit,
+                                const float* state_in, float* state_out, void* out, int B,
+                                int T, int H, int Dk, int Dv, gdn_dtype dtype, int chunk,
+                                void* stream) {
+  return gdn::scan(q, k, v, g_logit, beta_logit, state_in, state_out, out, B, T, H, Dk, Dv,
+                   dtype, chunk, stream, false, true);
+}
+
+gdn_status gdn_chunk_bidir_logits(const void* q, const void* k, const void* v,
+                                  const void* g_logit, const void* beta_logit,
+                                  const float* state_in, float* state_out, void* out, int B,
+                                  int T, int H, int Dk, int Dv, gdn_dtype dtype, int chunk,
+                                  void* stream) {
+  return gdn::scan(q, k, v, g_logit, beta_logit, state_in, state_out, out, B, T, H, Dk, Dv,
+                   dtype, chunk, stream, true, true);
 }
 
 gdn_status gdn_state_reset(float* state, int B, int H, int Dk, int Dv,

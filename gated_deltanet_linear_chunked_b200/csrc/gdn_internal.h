@@ -14,8 +14,8 @@ struct ScanArgs {
   const void* q;
   const void* k;
   const void* v;
-  const float* g;
-  const float* beta;
+  const void* g;           // fp32 g, or the decay logits (dtype) when gate_logits
+  const void* beta;        // fp32 beta, or the write-strength logits (dtype)
   const float* state_in;   // nullptr => zero state
   float* state_out;        // nullptr => not written
   void* out;
@@ -23,6 +23,7 @@ struct ScanArgs {
   gdn_dtype dtype;
   int chunk;               // sub-chunk length (already defaulted)
   bool bidir;
+  bool gate_logits;        // g and beta hold the gate layer's logits
   cudaStream_t stream;
   unsigned int* err;       // device error word (bounded waits report here)
   long long wait_limit;    // polls before a bounded wait gives up
@@ -52,10 +53,11 @@ class ProfileScope {
 // validated call (chunk defaulted; err and wait_limit not yet set) and `*dev`
 // the current device.  B == 0 or H == 0 returns GDN_OK with a->B or a->H
 // zero: the caller has nothing to do.
-gdn_status prepare_scan(const void* q, const void* k, const void* v, const float* g,
-                        const float* beta, const float* state_in, float* state_out,
+gdn_status prepare_scan(const void* q, const void* k, const void* v, const void* g,
+                        const void* beta, const float* state_in, float* state_out,
                         void* out, int B, int T, int H, int Dk, int Dv, gdn_dtype dtype,
-                        int chunk, void* stream, bool bidir, ScanArgs* a, int* dev);
+                        int chunk, void* stream, bool bidir, bool gate_logits, ScanArgs* a,
+                        int* dev);
 
 // T == 0: state_out = state_in (or zero); out untouched.
 gdn_status trivial_state_copy(const ScanArgs& a);

@@ -50,7 +50,7 @@ extern "C" gdn_status gdn_chunk_fwd_noalloc(const void* q, const void* k, const 
   ScanArgs a;
   int dev = 0;
   gdn_status st = prepare_scan(q, k, v, g, beta, state_in, state_out, out, B, T, H, Dk, Dv,
-                               dtype, chunk, stream, false, &a, &dev);
+                               dtype, chunk, stream, false, false, &a, &dev);
   if (st != GDN_OK) return st;
   if (dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;  // the scratch-using path is bf16
   if (a.B == 0 || a.H == 0) return GDN_OK;

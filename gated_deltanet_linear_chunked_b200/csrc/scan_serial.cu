@@ -23,6 +23,7 @@
 // q/k norms and k^.q^ are computed in parallel before the serial walk.
 #include <cuda_bf16.h>
 
+#include "gates.cuh"
 #include "gdn_internal.h"
 
 namespace gdn {
@@ -66,8 +67,8 @@ template <typename IO>
 __device__ void scan_direction(SerialSmem& sm, float (&S)[kRows][kColsPerWarp],
                                const IO* __restrict__ q, const IO* __restrict__ k,
                                const IO* __restrict__ v,
-                               const float* __restrict__ g,
-                               const float* __restrict__ beta, IO* out,
+                               const void* __restrict__ g,
+                               const void* __restrict__ beta, int logits, IO* out,
                                float* acc, int b, int h, int j0, int T, int H,
                                int Dk, int Dv, bool reverse) {
   const int tid = threadIdx.x;
@@ -91,8 +92,13 @@ __device__ void scan_direction(SerialSmem& sm, float (&S)[kRows][kColsPerWarp],
     if (tid < n) {
       const int t = reverse ? T - 1 - (p0 + tid) : p0 + tid;
       const size_t row = ((size_t)b * T + t) * H + h;
-      sm.a[tid] = expf(__ldg(g + row));
-      sm.beta[tid] = __ldg(beta + row);
+      if (logits) {  // the fused prologue: gates from the gate layer's logits
+        sm.a[tid] = expf(gate_g_from_logit(ld_in(static_cast<const IO*>(g) + row)));
+        sm.beta[tid] = gate_beta_from_logit(ld_in(static_cast<const IO*>(beta) + row));
+      } else {
+        sm.a[tid] = expf(__ldg(static_cast<const float*>(g) + row));
+        sm.beta[tid] = __ldg(static_cast<const float*>(beta) + row);
+      }
     }
     __syncthreads();
     // ---- per-token norms and k^.q^ (one warp per token)
@@ -177,8 +183,8 @@ __device__ void scan_direction(SerialSmem& sm, float (&S)[kRows][kColsPerWarp],
 template <typename IO>
 __global__ void __launch_bounds__(kThreads)
 gdn_scan_serial_kernel(const IO* __restrict__ q, const IO* __restrict__ k,
-                       const IO* __restrict__ v, const float* __restrict__ g,
-                       const float* __restrict__ beta,
+                       const IO* __restrict__ v, const void* __restrict__ g,
+                       const void* __restrict__ beta, int logits,
                        const float* state_in, float* state_out, IO* out,
                        float* acc, int T, int H, int Dk, int Dv, int bidir) {
   __shared__ SerialSmem sm;
@@ -201,7 +207,7 @@ gdn_scan_serial_kernel(const IO* __restrict__ q, const IO* __restrict__ k,
   // state_out (they may alias; slices are disjoint across CTAs).
   __syncthreads();
 
-  scan_direction<IO>(sm, S, q, k, v, g, beta, out, bidir ? acc : nullptr, b, h,
+  scan_direction<IO>(sm, S, q, k, v, g, beta, logits, out, bidir ? acc : nullptr, b, h,
                      j0, T, H, Dk, Dv, false);
 
   if (state_out) {
@@ -218,7 +224,7 @@ gdn_scan_serial_kernel(const IO* __restrict__ q, const IO* __restrict__ k,
   for (int r = 0; r < kRows; ++r)
 #pragma unroll
     for (int c = 0; c < kColsPerWarp; ++c) S[r][c] = 0.f;
-  scan_direction<IO>(sm, S, q, k, v, g, beta, out, acc, b, h, j0, T, H, Dk, Dv,
+  scan_direction<IO>(sm, S, q, k, v, g, beta, logits, out, acc, b, h, j0, T, H, Dk, Dv,
                      true);
 }
 
@@ -239,13 +245,13 @@ cudaError_t launch_scan_serial(const ScanArgs& a) {
   if (a.dtype == GDN_F32) {
     gdn_scan_serial_kernel<float><<<grid, kThreads, 0, a.stream>>>(
         static_cast<const float*>(a.q), static_cast<const float*>(a.k),
-        static_cast<const float*>(a.v), a.g, a.beta, a.state_in, a.state_out,
+        static_cast<const float*>(a.v), a.g, a.beta, a.gate_logits ? 1 : 0, a.state_in, a.state_out,
         static_cast<float*>(a.out), nullptr, a.T, a.H, a.Dk, a.Dv, a.bidir);
   } else {
     gdn_scan_serial_kernel<__nv_bfloat16><<<grid, kThreads, 0, a.stream>>>(
         static_cast<const __nv_bfloat16*>(a.q),
         static_cast<const __nv_bfloat16*>(a.k),
-        static_cast<const __nv_bfloat16*>(a.v), a.g, a.beta, a.state_in,
+        static_cast<const __nv_bfloat16*>(a.v), a.g, a.beta, a.gate_logits ? 1 : 0, a.state_in,
         a.state_out, static_cast<__nv_bfloat16*>(a.out), acc, a.T, a.H, a.Dk,
         a.Dv, a.bidir);
   }

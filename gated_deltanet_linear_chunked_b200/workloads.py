@@ -44,8 +44,9 @@ class Workload:
     dtype: str            # "f32" or "bf16": dtype of q, k, v and out
     chunk: int            # sub-chunk length handed to the library
     mode: str             # "fwd" or "bidir"
-    gate: tuple           # ("neg_softplus",) or ("uniform", lo, hi): g = log decay
-    beta: tuple           # ("sigmoid",) or ("const", value)
+    gate: tuple           # ("neg_softplus",), ("uniform", lo, hi): g = log decay;
+                          # ("logit_normal",): the gate layer's decay logit ~ N(0,1)
+    beta: tuple           # ("sigmoid",), ("const", value); ("logit_normal",): logit ~ N(0,1)
     state: tuple          # ("zero",) or ("normal", std)
     seed: int
     qk: tuple = ("unit",)  # ("unit",): rows L2-normalised; ("raw",): N(0,1) rows;
@@ -70,6 +71,16 @@ def stream_chunk(mode: str = "fwd", seed: int | None = None) -> Workload:
     name = "stream_chunk_causal" if mode == "fwd" else "stream_chunk_bidir"
     return Workload(name, 1, CHUNK_TOKENS, 20, 112, 112, "bf16", 64, mode,
                     ("uniform", -0.5, 0.0), ("sigmoid",), ("normal", 0.02), seed)
+
+
+def stream_chunk_logits(mode: str = "fwd", seed: int | None = None) -> Workload:
+    """The streaming chunk with the gate layer's logits as inputs (fused
+    prologue): decay and write-strength logits ~ N(0,1) rounded to bf16, so
+    g = -softplus(logit) and beta = sigmoid(logit) have the tiny workload's
+    stated gate distributions."""
+    w = stream_chunk(mode, seed)
+    return dataclasses.replace(w, name=w.name + "_logits", gate=("logit_normal",),
+                               beta=("logit_normal",))
 
 
 def stack_call(layer: int, chunk_index: int, mode: str = "bidir") -> Workload:
@@ -159,6 +170,14 @@ def make_head(w: Workload, b: int, h: int) -> dict:
     q = _shape_qk(rng.standard_normal((w.T, w.Dk), dtype=np.float32), w.qk, True)
     k = _shape_qk(rng.standard_normal((w.T, w.Dk), dtype=np.float32), w.qk, False)
     v = rng.standard_normal((w.T, w.Dv), dtype=np.float32)
+    if w.gate[0] == "logit_normal":
+        # the gate layer's raw outputs: the library forms g and beta itself
+        g_logit = rng.standard_normal(w.T, dtype=np.float32)
+        beta_logit = rng.standard_normal(w.T, dtype=np.float32)
+        if w.dtype == "bf16":
+            q, k, v = round_bf16(q), round_bf16(k), round_bf16(v)
+            g_logit, beta_logit = round_bf16(g_logit), round_bf16(beta_logit)
+        return {"q": q, "k": k, "v": v, "g_logit": g_logit, "beta_logit": beta_logit}
     if w.gate[0] == "neg_softplus":
         z = rng.standard_normal(w.T, dtype=np.float32).astype(np.float64)
         g = -np.logaddexp(0.0, z)
@@ -200,12 +219,13 @@ def make_inputs(w: Workload) -> dict:
     q = np.empty((w.B, w.T, w.H, w.Dk), np.float32)
     k = np.empty_like(q)
     v = np.empty((w.B, w.T, w.H, w.Dv), np.float32)
-    g = np.empty((w.B, w.T, w.H), np.float32)
-    beta = np.empty_like(g)
+    gates = ("g_logit", "beta_logit") if w.gate[0] == "logit_normal" else ("g", "beta")
+    ga = {n: np.empty((w.B, w.T, w.H), np.float32) for n in gates}
     for b, h, d in iter_heads(w):
         q[b, :, h], k[b, :, h], v[b, :, h] = d["q"], d["k"], d["v"]
-        g[b, :, h], beta[b, :, h] = d["g"], d["beta"]
-    return {"q": q, "k": k, "v": v, "g": g, "beta": beta, "state_in": make_state(w)}
+        for n in gates:
+            ga[n][b, :, h] = d[n]
+    return {"q": q, "k": k, "v": v, **ga, "state_in": make_state(w)}
 
 
 def slice_head(inputs: dict, b: int, h: int) -> dict:

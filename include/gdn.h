@@ -121,6 +121,32 @@ GDN_API gdn_status gdn_chunk_bidir(const void* q, const void* k, const void* v,
                            gdn_dtype dtype, int chunk, void* stream);
 
 /*
+ * The same two scans with the fused GDN prologue for the gates: instead of g
+ * and beta the caller passes the gate layer's two logits per (token, head),
+ * g_logit and beta_logit [B, T, H] in `dtype` (bf16 for the tensor-core path,
+ * which is how the gate layer runs under mixed precision), and the library
+ * forms
+ *     g_t = -softplus(g_logit_t) = -log(1 + e^{g_logit_t})     (so g_t <= 0)
+ *     beta_t = sigmoid(beta_logit_t)                           (in (0, 1))
+ * inside its kernels.  The pages name the gate layer and keep it in BF16
+ * ("SANA-Streaming：基于混合扩散Transformer的实时流式视频编辑系统", 实验结果)
+ * but do not write its activations; these are the plainest maps onto the
+ * scan's ranges.  q and k are L2-normalised inside the library as for every
+ * call.  Arguments, layouts and errors are otherwise those of gdn_chunk_fwd /
+ * gdn_chunk_bidir.
+ */
+GDN_API gdn_status gdn_chunk_fwd_logits(const void* q, const void* k, const void* v,
+                                        const void* g_logit, const void* beta_logit,
+                                        const float* state_in, float* state_out, void* out,
+                                        int B, int T, int H, int Dk, int Dv, gdn_dtype dtype,
+                                        int chunk, void* stream);
+GDN_API gdn_status gdn_chunk_bidir_logits(const void* q, const void* k, const void* v,
+                                          const void* g_logit, const void* beta_logit,
+                                          const float* state_in, float* state_out, void* out,
+                                          int B, int T, int H, int Dk, int Dv,
+                                          gdn_dtype dtype, int chunk, void* stream);
+
+/*
  * gdn_chunk_fwd for callers that cannot allocate device memory (no
  * counterpart on the pages).  Some callers cannot let a library allocate: a
  * streaming server that has already handed all remaining HBM to its caches
@@ -136,9 +162,9 @@ GDN_API gdn_status gdn_chunk_bidir(const void* q, const void* k, const void* v,
  * Arguments and layouts are those of gdn_chunk_fwd, with dtype GDN_BF16
  * only (other dtypes: GDN_ERR_UNSUPPORTED).  A problem whose scratch exceeds
  * the array returns GDN_ERR_SCRATCH_LIMIT and launches nothing.  The scratch
- * is about 104 KB per 64-token chunk of one head at Dk = Dv = 112, so about
- * 960 chunk-heads (B * H * ceil(T / 64)) fit: the 2640-token x 20-head
- * streaming chunk (840) does, two of them in one call do not.
+ * is about 81 KB per 64-token chunk of one head at Dk = Dv = 112, so about
+ * 1200 chunk-heads (B * H * ceil(T / 64)) fit: the 2640-token x 20-head
+ * streaming chunk (840) does, two of them in one call (1680) do not.
  *
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress, once per device, with that device current); make

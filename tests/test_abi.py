@@ -123,3 +123,13 @@ def test_wait_limit_hook_round_trips():
     old = lib.gdn_set_wait_limit(1234)
     assert lib.gdn_set_wait_limit(0) == 1234
     assert lib.gdn_set_wait_limit(old) > 0
+
+
+@pytest.mark.parametrize("entry", ["gdn_chunk_fwd_logits", "gdn_chunk_bidir_logits"])
+def test_logit_entry_points_validate_like_the_others(entry):
+    for name in ("q", "k", "v", "g", "beta", "out"):
+        assert call(entry, **{name: None}) == _lib.GDN_ERR_INVALID_ARG, name
+    assert call(entry, Dk=24) == _lib.GDN_ERR_UNSUPPORTED
+    assert call(entry, g=fake(7) + 64) == _lib.GDN_ERR_ALIAS       # logits overlap out
+    assert call(entry, beta=fake(3) + 8) == _lib.GDN_ERR_INVALID_ARG  # misaligned
+    assert call(entry) in (_lib.GDN_ERR_CUDA, _lib.GDN_ERR_INVALID_ARG)

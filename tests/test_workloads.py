@@ -146,3 +146,23 @@ def test_raw_and_mixed_qk_recipes():
     # the special row sets are disjoint from one another
     sets = [set(rows[n].tolist()) for n in ("small", "large", "subclamp")]
     assert not (sets[0] & sets[1]) and not (sets[0] & sets[2]) and not (sets[1] & sets[2])
+
+
+def test_logit_recipe_has_the_stated_gate_distributions():
+    """The fused-prologue workload passes the gate layer's logits: decay and
+    write-strength logits ~ N(0,1), bf16-exact, so that -softplus and sigmoid
+    of them have the tiny workload's stated gate distributions; q, k, v are
+    drawn exactly as in the streaming chunk."""
+    w = wl.stream_chunk_logits()
+    d = wl.make_head(w, 0, 4)
+    assert set(d) == {"q", "k", "v", "g_logit", "beta_logit"}
+    for n in ("g_logit", "beta_logit"):
+        x = d[n].astype(np.float64)
+        assert abs(x.mean()) < 0.05 and abs(x.std() - 1.0) < 0.05
+        assert np.array_equal(d[n], wl.round_bf16(d[n]))
+    plain = wl.make_head(wl.stream_chunk(), 0, 4)
+    for n in ("q", "k", "v"):
+        assert np.array_equal(d[n], plain[n])
+    x = wl.make_inputs(wl.Workload("lg", 2, 33, 3, 16, 16, "f32", 16, "fwd", ("logit_normal",),
+                                   ("logit_normal",), ("zero",), 3))
+    assert x["g_logit"].shape == (2, 33, 3) and "g" not in x
