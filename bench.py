@@ -384,17 +384,107 @@ def kernel_times(lib, step_fn, n, launches_per_step):
     _lib.check(lib.gdn_profile_begin(int(n * max(1, launches_per_step) + 8)), "gdn_profile_begin")
     for i in range(n):
         step_fn(i)
-    kms = (ctypes.c_float * 4)()
-    kn = (ctypes.c_int * 4)()
-    _lib.check(lib.gdn_profile_end(ctypes.addressof(kms), ctypes.addressof(kn), 4), "gdn_profile_end")
+    kms = (ctypes.c_float * 5)()
+    kn = (ctypes.c_int * 5)()
+    _lib.check(lib.gdn_profile_end(ctypes.addressof(kms), ctypes.addressof(kn), 5), "gdn_profile_end")
     kernels = {}
-    for i in range(4):
+    for i in range(5):
         if kn[i]:
             kernels[lib.gdn_kernel_name(i).decode()] = {"launches": kn[i], "ms_per_launch": kms[i] / kn[i]}
     tot = sum(v["ms_per_launch"] for v in kernels.values())
     for v in kernels.values():
         v["share"] = v["ms_per_launch"] / tot if tot else None
     return kernels
+
+
+def device_stream_inputs(w, dev, seed):
+    """Inputs of a long stream drawn on the device (torch generator, seeded)
+    with the workload's distributions -- q, k ~ N(0,1) rows L2-normalised, v
+    ~ N(0,1), g ~ U[lo, hi], beta constant, state_in ~ N(0, 0.02^2) -- so a
+    multi-GB stream needs no host round trip.  Timing only."""
+    import torch
+    gen = torch.Generator(device=dev).manual_seed(seed)
+    bf = torch.bfloat16
+
+    def rows(D):
+        x = torch.randn((w.B, w.T, w.H, D), generator=gen, device=dev)
+        return x / x.norm(dim=-1, keepdim=True)
+    x = {"q": rows(w.Dk).to(bf), "k": rows(w.Dk).to(bf),
+         "v": torch.randn((w.B, w.T, w.H, w.Dv), generator=gen, device=dev).to(bf)}
+    lo, hi = w.gate[1], w.gate[2]
+    x["g"] = lo + (hi - lo) * torch.rand((w.B, w.T, w.H), generator=gen, device=dev)
+    x["beta"] = torch.full((w.B, w.T, w.H), float(w.beta[1]), device=dev)
+    x["state_in"] = w.state[1] * torch.randn((w.B, w.H, w.Dk, w.Dv), generator=gen, device=dev)
+    x["out"] = torch.empty((w.B, w.T, w.H, w.Dv), dtype=bf, device=dev)
+    x["state_out"] = torch.empty_like(x["state_in"])
+    return x
+
+
+def time_calls(fn, x, stream, barrier, reps=3, warm=2):
+    """Mean ms of `reps` direct calls after `warm` (CUDA events)."""
+    import torch
+    call = lambda: fn(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state_in"],  # noqa: E731
+                      state_out=x["state_out"], out=x["out"], stream=stream)
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            call()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(reps):
+            call()
+    e1.record(stream)
+    barrier()
+    return e0.elapsed_time(e1) / reps
+
+
+def long_stream_figures(gdn, lib, w, stream, dev, peaks, peak_kind, barrier):
+    """The stress workload's longest case (B4 H16 d128 T65536, fast decay,
+    beta 0.99) against its HBM roofline, and one head of it (B1 H1) with and
+    without time segments: 1024 dependent chunk steps against the
+    segmented scan's 2 ceil(1024 / G) + G."""
+    import dataclasses
+    from gated_deltanet_linear_chunked_b200 import workloads as wl
+    res = {}
+    ws = [c for c in wl.stress_cases() if c.T == 65536 and c.Dk == 128][-1]
+    x = device_stream_inputs(ws, dev, 5)
+    ms = time_calls(gdn.chunk_fwd, x, stream, barrier)
+    t_hbm, t_tc = roofline_times(ws, False, peaks)
+    res["stress_B4_H16_d128_T65536"] = {
+        "workload": ws.name, "ms_per_call": ms, "head_tokens_per_s": ws.head_tokens / (ms / 1000.0),
+        "roofline": {"bound": "hbm", "roofline_us": 1e6 * max(t_hbm, t_tc),
+                     "algorithmic_bytes": algorithmic_bytes(ws),
+                     "achieved_gbs": algorithmic_bytes(ws) / (ms / 1000.0) / 1e9,
+                     "frac": (algorithmic_bytes(ws) / (ms / 1000.0) / 1e9) / peaks["hbm_gbs"],
+                     "peak_source": f"{peak_kind} hbm_gbs"}}
+    del x
+    import torch
+    torch.cuda.empty_cache()
+    w1 = dataclasses.replace(ws, B=1, H=1, name="long_stream_B1_H1_d128_T65536")
+    x = device_stream_inputs(w1, dev, 6)
+    nC = (w1.T + 63) // 64
+    old = lib.gdn_set_time_segments(1)
+    try:
+        ms_serial = time_calls(gdn.chunk_fwd, x, stream, barrier)
+    finally:
+        lib.gdn_set_time_segments(old)
+    ms_seg = time_calls(gdn.chunk_fwd, x, stream, barrier)
+
+    def seg_call(i):
+        with torch.cuda.stream(stream):
+            gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state_in"],
+                          state_out=x["state_out"], out=x["out"], stream=stream)
+    split = kernel_times(lib, seg_call, 2, 5)
+    G = int(round(nC ** 0.5))
+    res["long_stream_time_segments"] = {
+        "workload": w1.name, "chunks": nC,
+        "unsegmented": {"ms_per_call": ms_serial, "serial_chunk_steps": nC},
+        "segmented": {"ms_per_call": ms_seg, "segments_automatic": "about sqrt(chunks)",
+                      "kernels": split,
+                      "serial_chunk_steps_if_G_is_sqrt": 2 * ((nC + G - 1) // G) + G},
+        "speedup": ms_serial / ms_seg}
+    return res
 
 
 def roofline_times(w, bidir, peaks):
@@ -673,6 +763,7 @@ def main():
             "roofline": roofline_of(wlg, kernel_times(lib, lg_direct, n_prof, launches_per_step),
                                     lg_ms, peaks, peak_kind, False)}
         del lsets
+        extras.update(long_stream_figures(gdn, lib, w, stream, dev, peaks, peak_kind, barrier))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -8,7 +8,7 @@ is loaded on the first call.
 from . import workloads  # noqa: F401
 
 _API = ("chunk_fwd", "chunk_bidir", "chunk_fwd_logits", "chunk_bidir_logits", "state_reset",
-        "device_error", "set_wait_limit", "workspace_release")
+        "device_error", "set_wait_limit", "set_time_segments", "workspace_release")
 __all__ = [*_API, "GDNError", "workloads"]
 
 

@@ -36,6 +36,7 @@ SIGNATURES = {
     "gdn_device_error": (ctypes.c_int, [_vp]),
     "gdn_workspace_release": (ctypes.c_int, []),
     "gdn_set_wait_limit": (ctypes.c_longlong, [_ll]),
+    "gdn_set_time_segments": (ctypes.c_int, [_i]),
     "gdn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "gdn_version": (ctypes.c_int, []),
     "gdn_launch_count": (ctypes.c_ulonglong, []),

@@ -126,6 +126,12 @@ def workspace_release() -> None:
     _lib.check(_lib.load().gdn_workspace_release(), "gdn_workspace_release")
 
 
+def set_time_segments(segments: int) -> int:
+    """Time segments of the bf16 path's recurrence: 0 = automatic, 1 = never,
+    G >= 2 = exactly G.  Process-wide; returns the previous setting."""
+    return int(_lib.load().gdn_set_time_segments(int(segments)))
+
+
 def set_wait_limit(polls: int) -> int:
     """Polls a kernel's bounded wait makes before giving up (0 = default)."""
     return int(_lib.load().gdn_set_wait_limit(int(polls)))

@@ -45,6 +45,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <mutex>
 #include <utility>
 
@@ -593,12 +594,33 @@ __device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t (&r)[4]) {
                : "memory");
 }
 
+// What one launch of the chain kernel does (one pass of stage B):
+//  * publish pass: walk each time segment of the chunk sequence from its
+//    start state and publish every chunk's start state and U for stage C
+//    (unsegmented: one segment, started from state_in or zero);
+//  * summary pass (time-segmented scan only): walk each segment from zero
+//    and, beside the Dv/16 state slices, p_slices = Dk/16 more slices that
+//    start from the identity with U~ = 0: their final columns are the
+//    segment's transition P (S_out = P S_in + R), the others its offset R.
+struct ChainArgs {
+  const float* init;   // start states [dir][seg][b*h][Dk][Dv] (dir 0 only if
+                       // init_dir_stride == 0), or nullptr for zero
+  size_t init_seg_stride, init_dir_stride;  // floats between segments / directions
+  float* fin;          // final states, rows of fin_ld floats, or nullptr
+  size_t fin_seg_stride, fin_dir_stride;
+  int fin_ld;
+  int fin_last_seg_only;  // publish pass: only the last segment ends the scan
+  int nseg, seg_len;   // segments of seg_len chunks (the last may be shorter)
+  int publish;         // 1: publish pass, 0: summary pass
+  int p_slices;        // summary pass: slices past Dv/16 carry P's columns
+};
+
 // Warp q of the group walking slice s (16 state columns); gw = group index in
 // the CTA.  NKB = Dk / 16.  Returns false if a bounded wait expired.
-template <int NKB>
+template <int NKB, bool SUMMARY>
 __device__ bool chain_warp(uint8_t* smem, const ChainLayout& L, int nst, int gw, int q, int s,
-                           const float* state_in, float* state_out, const Workspace& ws,
-                           long long limit, unsigned* err) {
+                           const ChainArgs& A, const Workspace& ws, long long limit,
+                           unsigned* err) {
   constexpr int P = chain_group_warps(NKB);
   constexpr int KPW = (NKB + P - 1) / P;  // most state-row k-blocks of one warp
   constexpr int TPW = 4 / P;              // 16-token blocks of one warp
@@ -606,18 +628,34 @@ __device__ bool chain_warp(uint8_t* smem, const ChainLayout& L, int nst, int gw,
   const int lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
   const int mi = lane >> 3, mr = lane & 7;  // ldmatrix / stmatrix: matrix, row
   const int Dk = ws.Dk, Dv = ws.Dv, nC = ws.nC;
-  const int bh = blockIdx.y, dir = blockIdx.z;
+  const int bh = blockIdx.y, dir = blockIdx.z / A.nseg, seg = blockIdx.z - dir * A.nseg;
+  const int c_begin = seg * A.seg_len, n = min(A.seg_len, nC - c_begin);
   const int kb_lo = q * NKB / P, kb_hi = (q + 1) * NKB / P;  // this warp's state rows
   const int tb0 = q * TPW;                                    // this warp's tokens
   const int bar_id = 1 + gw, bar_n = 32 * P;
+  const bool pcol = SUMMARY && s >= Dv / 16;       // a transition slice (summary pass)
+  const int sj = pcol ? s - Dv / 16 : s;           // its 16 columns among P's or S's
+  constexpr bool publish = !SUMMARY;
 
-  // this warp's part of S^T: rows j = 16 s + g (regs 0, 1) and + 8 (2, 3),
+  // this warp's part of S^T: rows j = 16 sj + g (regs 0, 1) and + 8 (2, 3),
   // columns i = 8 nt + 2 tq (+1) for n-tiles nt of k-blocks [kb_lo, kb_hi)
   float S[2 * KPW][4];
 #pragma unroll
-  for (int k = 0; k < 2 * KPW; ++k) S[k][0] = S[k][1] = S[k][2] = S[k][3] = 0.f;
-  if (dir == 0 && state_in) {
-    const float* base = state_in + (size_t)bh * Dk * Dv + 16 * s + g;
+  for (int k = 0; k < 2 * KPW; ++k) {
+    const int i0 = 8 * (2 * kb_lo + k) + 2 * tq, j0 = 16 * sj + g;
+    S[k][0] = S[k][1] = S[k][2] = S[k][3] = 0.f;
+    if (pcol) {  // identity columns
+      S[k][0] = i0 == j0 ? 1.f : 0.f;
+      S[k][1] = i0 + 1 == j0 ? 1.f : 0.f;
+      S[k][2] = i0 == j0 + 8 ? 1.f : 0.f;
+      S[k][3] = i0 + 1 == j0 + 8 ? 1.f : 0.f;
+    }
+  }
+  const float* init = A.init && (A.init_dir_stride || dir == 0)
+                          ? A.init + dir * A.init_dir_stride + seg * A.init_seg_stride
+                          : nullptr;
+  if (init && !pcol) {
+    const float* base = init + (size_t)bh * Dk * Dv + 16 * sj + g;
 #pragma unroll
     for (int k = 0; k < 2 * KPW; ++k) {
       if (kb_lo + k / 2 < kb_hi) {
@@ -655,17 +693,17 @@ __device__ bool chain_warp(uint8_t* smem, const ChainLayout& L, int nst, int gw,
       }
     }
   };
-  publish_state(grp_u, true);
+  publish_state(grp_u, publish);
   named_barrier(bar_id, bar_n);
 
   bool ok = true, okp = true;
-  int c = 0;
-  int st = 0, bi = 0;  // load stage and staging buffer of chunk c
+  int lc = 0;          // chunk of this segment (its scan index is c_begin + lc)
+  int st = 0, bi = 0;  // load stage and staging buffer of chunk lc
   uint32_t ph = 0;     // parity of stage st's current fill
-  bool ready = false;  // chunk c's stage was seen full ahead of time
+  bool ready = false;  // chunk lc's stage was seen full ahead of time
   volatile int* fail = &bars.fail[gw];
-  for (; c < nC; ++c) {
-    const uint32_t buf = grp_u + bi * L.stg;  // staging of chunk c
+  for (; lc < n; ++lc) {
+    const uint32_t buf = grp_u + bi * L.stg;  // staging of chunk lc
     // the whole chunk-start state S^T, as A fragments over k = state rows
     uint32_t sa[NKB][4];
 #pragma unroll
@@ -687,6 +725,11 @@ __device__ bool chain_warp(uint8_t* smem, const ChainLayout& L, int nst, int gw,
         for (int t = 0; t < TPW; ++t) ldmatrix_x4(sw + 2 * kb * kSlab64 + (tb0 + t) * 256 + su_off, bw[kb][t]);
 #pragma unroll
       for (int t = 0; t < TPW; ++t) {
+        if (pcol) {  // transition columns: U~ = 0
+          u[2 * t][0] = u[2 * t][1] = u[2 * t][2] = u[2 * t][3] = 0.f;
+          u[2 * t + 1][0] = u[2 * t + 1][1] = u[2 * t + 1][2] = u[2 * t + 1][3] = 0.f;
+          continue;
+        }
         uint32_t r[4];
         ldmatrix_x4_trans(sut + (tb0 + t) * 256 + su_off, r);
         unpack_bf16x2(r[0], u[2 * t][0], u[2 * t][1]);
@@ -712,17 +755,17 @@ __device__ bool chain_warp(uint8_t* smem, const ChainLayout& L, int nst, int gw,
         ua_mine[t][1] = pack_bf16x2(u[2 * t][2], u[2 * t][3]);
         ua_mine[t][2] = pack_bf16x2(u[2 * t + 1][0], u[2 * t + 1][1]);
         ua_mine[t][3] = pack_bf16x2(u[2 * t + 1][2], u[2 * t + 1][3]);
-        stmatrix_x4_trans(buf + L.stg_s + (tb0 + t) * 256 + su_off, ua_mine[t]);
+        if (publish) stmatrix_x4_trans(buf + L.stg_s + (tb0 + t) * 256 + su_off, ua_mine[t]);
         st_shared_v4(xu_u + (tb0 + t) * 512 + lane * 16, ua_mine[t]);
       }
-      fence_proxy_async_smem();  // staging writes -> the producer's bulk stores
+      if (publish) fence_proxy_async_smem();  // staging writes -> the producer's bulk stores
     }
     if (!okw && lane == 0) *fail = 1;
     named_barrier(bar_id, bar_n);
     ok = *fail == 0;
     if (!ok) break;
-    // chunk c's staging (its start state and U) is complete
-    if (q == 0 && lane == 0) mbar_arrive(&bars.staged[bi]);
+    // chunk lc's staging (its start state and U) is complete
+    if (publish && q == 0 && lane == 0) mbar_arrive(&bars.staged[bi]);
     // S^T <- e^{gamma_C} S^T + U^T K~ over this warp's state rows (B
     // fragments first, then the MMAs)
     uint32_t bk[4][KPW][4];
@@ -758,13 +801,13 @@ __device__ bool chain_warp(uint8_t* smem, const ChainLayout& L, int nst, int gw,
     }
     // probe the next chunk's stage while the MMAs above run
     ready = __all_sync(0xffffffffu, mbar_test_wait(&bars.full[st], ph));
-    // the next chunk's start state goes to buffer (c + 1) % 3, which the
-    // producer's stores of chunk c - 2 must have finished reading
-    const bool more = c + 1 < nC;
+    // the next chunk's start state goes to buffer (lc + 1) % 3, which the
+    // producer's stores of chunk lc - 2 must have finished reading
+    const bool more = lc + 1 < n;
     const int bn = bi == kChainBufs - 1 ? 0 : bi + 1;
-    if (more && c >= 2)
-      okp = __all_sync(0xffffffffu, mbar_wait(&bars.freed[bn], ((c - 2) / kChainBufs) & 1, limit));
-    publish_state(grp_u + bn * L.stg, more && okp);
+    if (publish && more && lc >= 2)
+      okp = __all_sync(0xffffffffu, mbar_wait(&bars.freed[bn], ((lc - 2) / kChainBufs) & 1, limit));
+    publish_state(grp_u + bn * L.stg, publish && more && okp);
     named_barrier(bar_id, bar_n);
     bi = bn;
   }
@@ -772,67 +815,82 @@ __device__ bool chain_warp(uint8_t* smem, const ChainLayout& L, int nst, int gw,
     if (lane == 0) atomicOr(err, kErrTimeout);
     return false;
   }
-  if (dir == 0 && state_out) {
-    float* base = state_out + (size_t)bh * Dk * Dv + 16 * s + g;
+  const bool ends = !A.fin_last_seg_only || seg == A.nseg - 1;
+  float* fin = A.fin && ends && (A.fin_dir_stride || dir == 0)
+                   ? A.fin + dir * A.fin_dir_stride + seg * A.fin_seg_stride
+                   : nullptr;
+  if (fin) {
+    float* base = fin + (size_t)bh * Dk * A.fin_ld + (pcol ? Dv : 0) + 16 * sj + g;
 #pragma unroll
     for (int k = 0; k < 2 * KPW; ++k) {
       if (kb_lo + k / 2 < kb_hi) {
         const int i0 = 8 * (2 * kb_lo + k) + 2 * tq;
-        base[(size_t)i0 * Dv] = S[k][0];
-        base[(size_t)(i0 + 1) * Dv] = S[k][1];
-        base[(size_t)i0 * Dv + 8] = S[k][2];
-        base[(size_t)(i0 + 1) * Dv + 8] = S[k][3];
+        base[(size_t)i0 * A.fin_ld] = S[k][0];
+        base[(size_t)(i0 + 1) * A.fin_ld] = S[k][1];
+        base[(size_t)i0 * A.fin_ld + 8] = S[k][2];
+        base[(size_t)(i0 + 1) * A.fin_ld + 8] = S[k][3];
       }
     }
   }
   return true;
 }
 
-// The producer (one thread): loads chunk c into stage c % nst once the chain
-// warps have released that stage's previous chunk, and publishes each
-// chunk's staged S and U for the CTA's groups with bulk stores.
+// The producer (one thread): loads the segment's chunk lc into stage lc % nst
+// once the chain warps have released that stage's previous chunk and, in the
+// publish pass, stores each chunk's staged S and U for the CTA's groups.
 __device__ void chain_producer(uint8_t* smem, const ChainLayout& L, int nst, int active, int s0,
-                               const Workspace& ws, long long limit, unsigned* err) {
+                               const ChainArgs& A, const Workspace& ws, long long limit,
+                               unsigned* err) {
   ChainBars& bars = *reinterpret_cast<ChainBars*>(smem);
-  const int bh = blockIdx.y, dir = blockIdx.z, nC = ws.nC, Dk = ws.Dk;
+  const int bh = blockIdx.y, dir = blockIdx.z / A.nseg, seg = blockIdx.z - dir * A.nseg;
+  const int nC = ws.nC, Dk = ws.Dk;
+  const int c_begin = seg * A.seg_len, n = min(A.seg_len, nC - c_begin);
   uint8_t* stage0 = smem + kChainHeadBytes;
-  const uint32_t ut_bytes = (uint32_t)active * 2 * kSlab64;
-  auto block_of = [&](int c) { return ws.blk(ws.tile(dir, bh, dir ? nC - 1 - c : c)); };
-  auto load = [&](int c) -> bool {
-    const int st = c % nst;
-    if (c >= nst && !mbar_wait(&bars.empty[st], ((c / nst) - 1) & 1, limit)) return false;
-    const uint8_t* blk = block_of(c);
+  // U~ slabs of the state slices among the CTA's (transition slices need none)
+  const int ut_slices = max(0, min(s0 + active, ws.Dv / 16) - s0);
+  const uint32_t ut_bytes = (uint32_t)ut_slices * 2 * kSlab64;
+  auto block_of = [&](int lc) {
+    const int c = c_begin + lc;
+    return ws.blk(ws.tile(dir, bh, dir ? nC - 1 - c : c));
+  };
+  auto load = [&](int lc) -> bool {
+    const int st = lc % nst;
+    if (lc >= nst && !mbar_wait(&bars.empty[st], ((lc / nst) - 1) & 1, limit)) return false;
+    const uint8_t* blk = block_of(lc);
     uint8_t* dst = stage0 + st * L.stage;
     mbar_arrive_expect_tx(&bars.full[st], L.wk_bytes + ut_bytes);
     bulk_load(dst, blk + ws.off_w, L.wk_bytes, &bars.full[st]);
-    bulk_load(dst + L.wk_bytes, blk + ws.off_ut + (size_t)s0 * 2 * kSlab64, ut_bytes, &bars.full[st]);
+    if (ut_bytes)
+      bulk_load(dst + L.wk_bytes, blk + ws.off_ut + (size_t)s0 * 2 * kSlab64, ut_bytes, &bars.full[st]);
     return true;
   };
   int issued = 0;
   bool ok = true;
-  for (; issued < nC && issued < nst; ++issued) load(issued);
-  for (int c = 0; c < nC && ok; ++c) {
-    const int b = c % kChainBufs;
-    // chunk c - 1's stores have read their buffer: the chain may reuse it
-    // (for chunk c + 2's start state, at the end of its chunk c + 1)
-    if (c >= 1) {
-      bulk_wait_read();
-      mbar_arrive(&bars.freed[(c - 1) % kChainBufs]);
+  for (; issued < n && issued < nst; ++issued) load(issued);
+  for (int lc = 0; lc < n && ok; ++lc) {
+    if (A.publish) {
+      const int b = lc % kChainBufs;
+      // chunk lc - 1's stores have read their buffer: the chain may reuse it
+      // (for chunk lc + 2's start state, at the end of its chunk lc + 1)
+      if (lc >= 1) {
+        bulk_wait_read();
+        mbar_arrive(&bars.freed[(lc - 1) % kChainBufs]);
+      }
+      // publish chunk lc once every group has staged it
+      if (!mbar_wait(&bars.staged[b], (lc / kChainBufs) & 1, limit)) {
+        ok = false;
+        break;
+      }
+      uint8_t* blk = block_of(lc);
+      for (int gw = 0; gw < active; ++gw) {
+        const uint8_t* sb = smem + L.groups + gw * L.group + b * L.stg;
+        bulk_store_nc(blk + ws.off_s + (size_t)(s0 + gw) * 2 * Dk * 16, sb, L.stg_s);
+        bulk_store_nc(blk + ws.off_u + (size_t)(s0 + gw) * 2 * kSlab64, sb + L.stg_s, 2 * kSlab64);
+      }
+      bulk_commit();
     }
-    // publish chunk c once every group has staged it
-    if (!mbar_wait(&bars.staged[b], (c / kChainBufs) & 1, limit)) {
-      ok = false;
-      break;
-    }
-    uint8_t* blk = block_of(c);
-    for (int gw = 0; gw < active; ++gw) {
-      const uint8_t* sb = smem + L.groups + gw * L.group + b * L.stg;
-      bulk_store_nc(blk + ws.off_s + (size_t)(s0 + gw) * 2 * Dk * 16, sb, L.stg_s);
-      bulk_store_nc(blk + ws.off_u + (size_t)(s0 + gw) * 2 * kSlab64, sb + L.stg_s, 2 * kSlab64);
-    }
-    bulk_commit();
-    // refill the stage chunk c used with chunk c + nst
-    if (issued < nC) {
+    // refill the stage chunk lc used with chunk lc + nst
+    if (issued < n) {
       if (!load(issued)) {
         ok = false;
         break;
@@ -850,16 +908,16 @@ __device__ void chain_producer(uint8_t* smem, const ChainLayout& L, int nst, int
   }
 }
 
-template <int NKB>
+template <int NKB, bool SUMMARY>
 __global__ void __launch_bounds__(32 * (kChainMaxGroups * 4 + 1), 1)
-gdn_recur_kernel(const float* state_in, float* state_out, Workspace ws, int ns, int nst,
-                 long long limit, unsigned* err) {
+gdn_recur_kernel(ChainArgs A, Workspace ws, int ns, int nst, long long limit, unsigned* err) {
   constexpr int P = chain_group_warps(NKB);
   extern __shared__ __align__(128) uint8_t smem_raw[];
   ChainBars& bars = *reinterpret_cast<ChainBars*>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int s0 = blockIdx.x * ns;
-  const int active = min(ns, ws.Dv / 16 - s0);  // slice groups with a slice
+  const int nslices = ws.Dv / 16 + A.p_slices;
+  const int active = min(ns, nslices - s0);  // slice groups with a slice
   const ChainLayout L(ws.Dk, ns, nst);
   if (threadIdx.x == 0) {
     for (int i = 0; i < nst; ++i) {
@@ -874,29 +932,109 @@ gdn_recur_kernel(const float* state_in, float* state_out, Workspace ws, int ns, 
     fence_mbar_init();
   }
   __syncthreads();
-  pdl_wait();  // stage A's W, K~, U~ are complete and visible
+  pdl_wait();  // stage A's W, K~, U~ (or the previous pass) are complete and visible
   pdl_trigger();
   const int gw = warp / P, q = warp - gw * P;
   if (gw < active)
-    chain_warp<NKB>(smem_raw, L, nst, gw, q, s0 + gw, state_in, state_out, ws, limit, err);
+    chain_warp<NKB, SUMMARY>(smem_raw, L, nst, gw, q, s0 + gw, A, ws, limit, err);
   else if (warp == ns * P && lane == 0)
-    chain_producer(smem_raw, L, nst, active, s0, ws, limit, err);
+    chain_producer(smem_raw, L, nst, active, s0, A, ws, limit, err);
   __syncthreads();
 }
 
-// The recurrence kernel for Dk = 16 * nkb.
-using RecurKernel = void (*)(const float*, float*, Workspace, int, int, long long, unsigned*);
-RecurKernel recur_kernel(int nkb) {
-  switch (nkb) {
-    case 1: return gdn_recur_kernel<1>;
-    case 2: return gdn_recur_kernel<2>;
-    case 3: return gdn_recur_kernel<3>;
-    case 4: return gdn_recur_kernel<4>;
-    case 5: return gdn_recur_kernel<5>;
-    case 6: return gdn_recur_kernel<6>;
-    case 7: return gdn_recur_kernel<7>;
-    default: return gdn_recur_kernel<8>;
+// The time-segmented scan's prefix over segments (one CTA per 4 state
+// columns, b*h and direction): S_0 = the scan's start state, S_{g+1} = P_g S_g
+// + R_g, with the summary pass's maps [dir][seg][b*h][Dk][Dv + Dk] (row i:
+// R's row i, then P's row i); writes every segment's start state S_g to
+// seg_state [dir][seg][b*h][Dk][Dv].  fp32 on CUDA cores: nseg dependent
+// steps of a Dk x Dk by Dk x 4 product per CTA, with P and R staged in shared
+// memory by 16-byte cp.async copies (the next segment's land while this one
+// computes); each thread keeps one column and Dk / 64 rows.
+constexpr int kPrefixThreads = 256;
+constexpr int kPrefixCols = 4;
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+struct PrefixSmem {
+  float P[2][128][132];          // P_g, padded rows (double-buffered over segments)
+  float R[2][128][kPrefixCols];  // this CTA's columns of R_g
+  float S[128][kPrefixCols];     // this CTA's columns of the current start state
+};
+__global__ void __launch_bounds__(kPrefixThreads)
+gdn_segment_prefix_kernel(const float* maps, const float* state_in, float* seg_state, int Dk,
+                          int Dv, int NBH, int nseg) {
+  extern __shared__ __align__(16) uint8_t prefix_raw[];
+  PrefixSmem& sm = *reinterpret_cast<PrefixSmem*>(prefix_raw);
+  constexpr int kRowGroups = kPrefixThreads / kPrefixCols;  // 64
+  const int j0 = kPrefixCols * blockIdx.x, bh = blockIdx.y, dir = blockIdx.z;
+  const int tid = threadIdx.x, jj = tid % kPrefixCols, rg = tid / kPrefixCols;
+  const int ld = Dk + Dv;
+  pdl_wait();  // the summary pass is complete and visible
+  pdl_trigger();
+  auto stage = [&](int sg, int buf) {  // P_g and R_g's columns -> buffer buf
+    const float* M = maps + (((size_t)dir * nseg + sg) * NBH + bh) * Dk * ld;
+    const int q4 = Dk / 4;  // 16-byte pieces of a P row
+    for (int e = tid; e < Dk * q4; e += kPrefixThreads) {
+      const int i = e / q4, c = e - i * q4;
+      cp_async16(&sm.P[buf][i][4 * c], M + (size_t)i * ld + Dv + 4 * c);
+    }
+    for (int i = tid; i < Dk; i += kPrefixThreads) cp_async16(&sm.R[buf][i][0], M + (size_t)i * ld + j0);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  for (int e = tid; e < Dk * kPrefixCols; e += kPrefixThreads) {
+    const int i = e / kPrefixCols, j = e % kPrefixCols;
+    sm.S[i][j] = (dir == 0 && state_in) ? state_in[((size_t)bh * Dk + i) * Dv + j0 + j] : 0.f;
   }
+  if (nseg > 1) stage(0, 0);
+  for (int sg = 0; sg < nseg; ++sg) {
+    float* dst = seg_state + (((size_t)dir * nseg + sg) * NBH + bh) * Dk * Dv;
+    for (int e = tid; e < Dk * kPrefixCols; e += kPrefixThreads) {
+      const int i = e / kPrefixCols, j = e % kPrefixCols;
+      dst[(size_t)i * Dv + j0 + j] = sm.S[i][j];
+    }
+    if (sg + 1 == nseg) break;
+    const int buf = sg & 1;
+    // this segment's copies have landed (the next segment's may still fly)
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+    if (sg + 2 < nseg) stage(sg + 1, buf ^ 1);  // lands while this step computes
+    // rows rg, rg + 64 (Dk <= 128): acc = R + P S, S's column loaded once per k
+    const int nr = rg + kRowGroups < Dk ? 2 : (rg < Dk ? 1 : 0);
+    float acc0 = rg < Dk ? sm.R[buf][rg][jj] : 0.f;
+    float acc1 = nr == 2 ? sm.R[buf][rg + kRowGroups][jj] : 0.f;
+    const float* P0 = sm.P[buf][rg < Dk ? rg : 0];
+    const float* P1 = sm.P[buf][nr == 2 ? rg + kRowGroups : 0];
+    for (int k = 0; k < Dk; k += 4) {
+      const float s0 = sm.S[k][jj], s1 = sm.S[k + 1][jj], s2 = sm.S[k + 2][jj], s3 = sm.S[k + 3][jj];
+      const float4 p = *reinterpret_cast<const float4*>(P0 + k);
+      acc0 = fmaf(p.x, s0, fmaf(p.y, s1, fmaf(p.z, s2, fmaf(p.w, s3, acc0))));
+      const float4 p1 = *reinterpret_cast<const float4*>(P1 + k);
+      acc1 = fmaf(p1.x, s0, fmaf(p1.y, s1, fmaf(p1.z, s2, fmaf(p1.w, s3, acc1))));
+    }
+    __syncthreads();
+    if (nr >= 1) sm.S[rg][jj] = acc0;
+    if (nr == 2) sm.S[rg + kRowGroups][jj] = acc1;
+    __syncthreads();
+  }
+}
+
+// The recurrence kernel for Dk = 16 * nkb.
+using RecurKernel = void (*)(ChainArgs, Workspace, int, int, long long, unsigned*);
+template <bool SUMMARY>
+RecurKernel recur_kernel_pass(int nkb) {
+  switch (nkb) {
+    case 1: return gdn_recur_kernel<1, SUMMARY>;
+    case 2: return gdn_recur_kernel<2, SUMMARY>;
+    case 3: return gdn_recur_kernel<3, SUMMARY>;
+    case 4: return gdn_recur_kernel<4, SUMMARY>;
+    case 5: return gdn_recur_kernel<5, SUMMARY>;
+    case 6: return gdn_recur_kernel<6, SUMMARY>;
+    case 7: return gdn_recur_kernel<7, SUMMARY>;
+    default: return gdn_recur_kernel<8, SUMMARY>;
+  }
+}
+RecurKernel recur_kernel(int nkb, bool summary = false) {
+  return summary ? recur_kernel_pass<true>(nkb) : recur_kernel_pass<false>(nkb);
 }
 
 // ========================================================== stage C: output
@@ -1282,11 +1420,15 @@ cudaError_t set_smem_attrs() {
   e = cudaFuncSetAttribute(gdn_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)sizeof(PrepSmem));
   for (int nkb = 1; nkb <= 8 && e == cudaSuccess; ++nkb)
-    e = cudaFuncSetAttribute(recur_kernel(nkb), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             227 * 1024);
+    for (int sm = 0; sm < 2 && e == cudaSuccess; ++sm)
+      e = cudaFuncSetAttribute(recur_kernel(nkb, sm == 1), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               227 * 1024);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(gdn_output_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)OutLayout(128, 128).total);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gdn_segment_prefix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sizeof(PrefixSmem));
   if (e == cudaSuccess) done[dev] = true;
   return e;
 }
@@ -1364,11 +1506,41 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 
 }  // namespace
 
+// Time segments of the chunked scan.  Segmenting pays only when a call has
+// too few (head, state-slice) chains to fill the GPU and many chunks: its
+// three passes do about three times the chain work, with a serial depth of
+// about 2 nC / G + G chunk steps instead of nC.  A setting > 0 from
+// gdn_set_time_segments forces the count (1: never segment).
+int time_segments(int B, int T, int H, int Dk, int Dv, bool bidir) {
+  const int nC = (T + kC - 1) / kC;
+  const int forced = current_time_segments();
+  int G = 1;
+  if (forced > 0) {
+    G = forced;
+  } else {
+    const long long chains = (long long)(Dv / 16) * B * H * (bidir ? 2 : 1);
+    const int sms = num_sms();
+    if (nC >= 64 && chains * 4 <= sms) {
+      G = (int)std::lround(std::sqrt((double)nC));
+      const long long per_seg = (long long)((Dv + Dk) / 16 + 1) / 2 * B * H * (bidir ? 2 : 1);
+      G = (int)std::min<long long>(G, std::max<long long>(2, 2LL * sms / std::max<long long>(per_seg, 1)));
+    }
+  }
+  G = std::max(1, std::min(G, nC / 2));
+  const int seg_len = (nC + G - 1) / G;
+  return (nC + seg_len - 1) / seg_len;  // no empty segment
+}
+
 size_t chunk_tc_workspace_bytes(int B, int T, int H, int Dk, int Dv, bool bidir) {
-  const size_t tiles = (size_t)(bidir ? 2 : 1) * B * H * ((T + kC - 1) / kC);
+  const int ndir = bidir ? 2 : 1;
+  const size_t tiles = (size_t)ndir * B * H * ((T + kC - 1) / kC);
   Workspace ws;
   ws.layout(Dk, Dv);
-  return tiles * ws.block_bytes;
+  size_t bytes = tiles * ws.block_bytes;
+  const int G = time_segments(B, T, H, Dk, Dv, bidir);
+  if (G > 1)  // segment maps [dir][seg][b*h][Dk][Dv + Dk] and start states [..][Dk][Dv]
+    bytes += (size_t)ndir * G * B * H * Dk * ((Dv + Dk) + Dv) * sizeof(float);
+  return bytes;
 }
 
 cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
@@ -1394,14 +1566,58 @@ cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
                    mk, mv, a.g, a.beta, a.gate_logits ? 1 : 0, ws, a.T, a.H, a.wait_limit, a.err);
   }
   if (e != cudaSuccess) return e;
-  {
+  unsigned launches = 3;
+  const int nsl = a.Dv / 16, nkb = a.Dk / 16;
+  const int G = time_segments(a.B, a.T, a.H, a.Dk, a.Dv, a.bidir);
+  auto chain = [&](const ChainArgs& A, int slices, int groups_z) {
     ProfileScope ps(a.stream, kKernRecur);
-    const ChainShape cs = chain_shape(a.Dk, a.Dv, NBH * ndir, num_sms());
-    const int nslices = a.Dv / 16;
-    e = launch_pdl(recur_kernel(a.Dk / 16), dim3((nslices + cs.ns - 1) / cs.ns, NBH, ndir),
-                   32 * (cs.ns * chain_group_warps(a.Dk / 16) + 1),
-                   ChainLayout(a.Dk, cs.ns, cs.nst).total, a.stream, a.state_in,
-                   a.state_out, ws, cs.ns, cs.nst, a.wait_limit, a.err);
+    const ChainShape cs = chain_shape(a.Dk, 16 * slices, NBH * groups_z, num_sms());
+    return launch_pdl(recur_kernel(nkb, A.publish == 0), dim3((slices + cs.ns - 1) / cs.ns, NBH, groups_z),
+                      32 * (cs.ns * chain_group_warps(nkb) + 1), ChainLayout(a.Dk, cs.ns, cs.nst).total,
+                      a.stream, A, ws, cs.ns, cs.nst, a.wait_limit, a.err);
+  };
+  ChainArgs A = {};
+  A.fin_last_seg_only = 1;
+  A.publish = 1;
+  if (G <= 1) {  // one walk over the whole chunk sequence
+    A.init = a.state_in;
+    A.fin = a.state_out;
+    A.fin_ld = a.Dv;
+    A.nseg = 1;
+    A.seg_len = nC;
+    e = chain(A, nsl, ndir);
+  } else {  // time-segmented: segment maps, their prefix, then every segment
+    const int seg_len = (nC + G - 1) / G;
+    const size_t ld = (size_t)a.Dv + a.Dk;
+    float* maps = reinterpret_cast<float*>(ws.base + (size_t)ndir * NBH * nC * ws.block_bytes);
+    float* seg_state = maps + (size_t)ndir * G * NBH * a.Dk * ld;
+    ChainArgs S1 = {};
+    S1.fin = maps;
+    S1.fin_seg_stride = (size_t)NBH * a.Dk * ld;
+    S1.fin_dir_stride = (size_t)G * S1.fin_seg_stride;
+    S1.fin_ld = (int)ld;
+    S1.nseg = G;
+    S1.seg_len = seg_len;
+    S1.publish = 0;
+    S1.p_slices = nkb;
+    e = chain(S1, nsl + nkb, ndir * G);
+    if (e == cudaSuccess) {
+      ProfileScope ps(a.stream, kKernSegPrefix);
+      e = launch_pdl(gdn_segment_prefix_kernel, dim3(a.Dv / kPrefixCols, NBH, ndir), kPrefixThreads,
+                     sizeof(PrefixSmem), a.stream, (const float*)maps, a.state_in, seg_state, a.Dk,
+                     a.Dv, NBH, G);
+    }
+    if (e == cudaSuccess) {
+      A.init = seg_state;
+      A.init_seg_stride = (size_t)NBH * a.Dk * a.Dv;
+      A.init_dir_stride = (size_t)G * A.init_seg_stride;
+      A.fin = a.state_out;
+      A.fin_ld = a.Dv;
+      A.nseg = G;
+      A.seg_len = seg_len;
+      e = chain(A, nsl, ndir * G);
+    }
+    launches = 5;
   }
   if (e != cudaSuccess) return e;
   {
@@ -1410,7 +1626,7 @@ cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
                    OutLayout(a.Dk, a.Dv).total, a.stream, mq, mk,
                    static_cast<__nv_bfloat16*>(a.out), ws, a.T, a.H, ndir, a.wait_limit, a.err);
   }
-  if (e == cudaSuccess) count_launches(3);
+  if (e == cudaSuccess) count_launches(launches);
   return e;
 }
 

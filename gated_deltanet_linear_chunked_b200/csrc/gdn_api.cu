@@ -42,6 +42,7 @@ constexpr long long kDefaultWaitLimit = 1LL << 26;
 std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
 
 std::atomic<unsigned long long> g_launches{0};
+std::atomic<int> g_time_segments{0};
 
 constexpr int kMaxDevices = 64;
 std::mutex g_err_mu;
@@ -337,6 +338,7 @@ void count_launches(unsigned n) { g_launches.fetch_add(n); }
 
 cudaError_t current_error_word(unsigned int** out) { return error_word(out); }
 long long current_wait_limit() { return g_wait_limit.load(); }
+int current_time_segments() { return g_time_segments.load(); }
 
 // ------------------------------------------------------------- profiling
 namespace {
@@ -485,6 +487,11 @@ gdn_status gdn_workspace_release(void) {
   return st;
 }
 
+int gdn_set_time_segments(int segments) {
+  if (segments < 0) segments = 0;
+  return gdn::g_time_segments.exchange(segments);
+}
+
 long long gdn_set_wait_limit(long long polls) {
   if (polls <= 0) polls = gdn::kDefaultWaitLimit;
   return gdn::g_wait_limit.exchange(polls);
@@ -571,6 +578,7 @@ const char* gdn_kernel_name(int id) {
     case gdn::kKernPrep: return "gdn_prep_kernel";
     case gdn::kKernRecur: return "gdn_recur_kernel";
     case gdn::kKernOutput: return "gdn_output_kernel";
+    case gdn::kKernSegPrefix: return "gdn_segment_prefix_kernel";
   }
   return "unknown";
 }

@@ -35,7 +35,8 @@ enum KernelId : int {
   kKernPrep = 1,
   kKernRecur = 2,
   kKernOutput = 3,
-  kNumKernelIds = 4,
+  kKernSegPrefix = 4,
+  kNumKernelIds = 5,
 };
 
 // While profiling is armed, records CUDA events around one launch.
@@ -72,6 +73,9 @@ gdn_status finish(cudaStream_t s, cudaError_t launch_err, unsigned int* err);
 // bounded waits.
 cudaError_t current_error_word(unsigned int** out);
 long long current_wait_limit();
+
+// The time-segment setting of gdn_set_time_segments (0: automatic).
+int current_time_segments();
 
 // Adds n to the process-wide count of kernels the library has enqueued.
 void count_launches(unsigned n);

@@ -221,6 +221,25 @@ GDN_API gdn_status gdn_workspace_release(void);
 GDN_API long long gdn_set_wait_limit(long long polls);
 
 /*
+ * Time segments of the bf16 path's recurrence.  The stage that walks the
+ * chunks is a dependent chain of ceil(T / 64) steps per (head, 16 state
+ * columns).  When a call has too few such chains to fill the GPU and many
+ * chunks, the library splits time into G segments: each segment's affine
+ * map (S_out = P S_in + R) is formed in parallel, an exclusive prefix over
+ * the segments gives every segment its start state, and the segments are
+ * walked again in parallel from there -- a serial depth of about
+ * 2 ceil(T / 64) / G + G chunk steps for three times the chain's work.  The
+ * stream's carry is a forward scan that starts from the previous chunk's
+ * cache ("SANA-Streaming：基于混合扩散Transformer的实时流式视频编辑系统",
+ * 方法步骤详情), so the prefix runs over the same affine maps in time order.
+ * 0 (the default) lets the library choose G; 1 never segments; G >= 2 forces
+ * G segments (at most ceil(T / 64) / 2).  One process-wide setting, read
+ * when a call is made; meant for tests and benchmarks.  Returns the previous
+ * value.
+ */
+GDN_API int gdn_set_time_segments(int segments);
+
+/*
  * Instrumentation (no counterpart on the pages): the number of kernels this
  * process has enqueued through the library so far, on all devices and
  * streams (launches captured into a CUDA graph count once, at capture).
@@ -234,8 +253,8 @@ GDN_API unsigned long long gdn_launch_count(void);
  * launches, current device); gdn_profile_end synchronises the recorded
  * events, disarms, and writes for each kernel id i < nids the total
  * milliseconds ms[i] and launch count n[i].  Kernel ids: 0 token-serial scan,
- * 1 stage A (prep), 2 stage B (recurrence), 3 stage C (output); names from
- * gdn_kernel_name.  Not thread-safe against concurrent calls on other
+ * 1 stage A (prep), 2 stage B (recurrence, every pass), 3 stage C (output),
+ * 4 the time-segment prefix; names from gdn_kernel_name.  Not thread-safe against concurrent calls on other
  * threads; meant for benchmarks.
  */
 GDN_API gdn_status gdn_profile_begin(int max_launches);

@@ -133,3 +133,11 @@ def test_logit_entry_points_validate_like_the_others(entry):
     assert call(entry, g=fake(7) + 64) == _lib.GDN_ERR_ALIAS       # logits overlap out
     assert call(entry, beta=fake(3) + 8) == _lib.GDN_ERR_INVALID_ARG  # misaligned
     assert call(entry) in (_lib.GDN_ERR_CUDA, _lib.GDN_ERR_INVALID_ARG)
+
+
+def test_time_segment_hook_round_trips():
+    lib = _lib.load()
+    old = lib.gdn_set_time_segments(7)
+    assert lib.gdn_set_time_segments(-3) == 7      # negative means automatic
+    assert lib.gdn_set_time_segments(old) == 0
+    assert lib.gdn_kernel_name(4).decode() == "gdn_segment_prefix_kernel"
