@@ -17,6 +17,9 @@ Contents
                       form of the scan in fp64, used only to pin that the
                       chunked algebra reaches the recurrence exactly; and
                       ``gates_from_logits``, the gate activations in numpy.
+  * ``backward``   -- the forward definition in plain PyTorch CPU float64,
+                      differentiated by autograd: the reference gradients of
+                      the scan.
 
 Parity is pinned, not assumed: ``tests/test_oracle_pins.py`` checks these
 functions against closed forms, invariants, a hand-derived example and brute
@@ -30,6 +33,7 @@ from .cpu import (  # noqa: F401
     oracle_fwd,
     oracle_fwd_logits,
 )
+from . import backward  # noqa: F401
 from .numpy_ref import (  # noqa: F401
     chunked_bidir,
     chunked_fwd,

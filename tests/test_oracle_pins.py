@@ -527,3 +527,86 @@ def test_planted_gate_slip_fails_the_decay_pin():
     _, S = oracle.recurrence_fwd(q, k, v, g_wrong, np.zeros((B, T, H)), s)
     dec = np.prod(1.0 / (1.0 + np.exp(x.astype(np.float64))), axis=1)
     assert not np.allclose(S, s * dec[:, :, None, None], rtol=1e-6)
+
+
+# ---------------------------------------------------------------------------
+# Reference gradients (oracle/backward.py): autograd of the definition
+# ---------------------------------------------------------------------------
+
+
+def _fd_inputs(rng, B=1, T=5, H=2, Dk=3, Dv=2):
+    q = rng.standard_normal((B, T, H, Dk))
+    k = rng.standard_normal((B, T, H, Dk))
+    v = rng.standard_normal((B, T, H, Dv))
+    g = rng.uniform(-1.0, -0.05, (B, T, H))
+    beta = rng.uniform(0.1, 0.9, (B, T, H))
+    s = 0.5 * rng.standard_normal((B, H, Dk, Dv))
+    return q, k, v, g, beta, s
+
+
+@pytest.mark.parametrize("bidir", [False, True])
+def test_backward_matches_central_differences(bidir):
+    """Every gradient of L = <out, W1> + <state_out, W2> against central
+    differences of the token recurrence (fp64, step 1e-6), element by
+    element, for all six inputs."""
+    rng = np.random.default_rng(21)
+    q, k, v, g, beta, s = _fd_inputs(rng)
+    W1 = rng.standard_normal(v.shape)
+    W2 = rng.standard_normal(s.shape)
+    gr = oracle.backward.grads(q, k, v, g, beta, s, W1, W2, bidir=bidir)
+
+    def loss(xs):
+        o, S = oracle.recurrence_bidir(*xs) if bidir else oracle.recurrence_fwd(*xs)
+        return float(np.sum(o * W1) + np.sum(S * W2))
+    base = [q, k, v, g, beta, s]
+    h = 1e-6
+    for idx, name in enumerate(["dq", "dk", "dv", "dg", "dbeta", "dstate_in"]):
+        x = base[idx]
+        fd = np.zeros_like(x)
+        for e in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[e] += h
+            xm[e] -= h
+            bp, bm = list(base), list(base)
+            bp[idx], bm[idx] = xp, xm
+            fd[e] = (loss(bp) - loss(bm)) / (2 * h)
+        np.testing.assert_allclose(gr[name], fd, rtol=1e-5, atol=1e-7, err_msg=name)
+
+
+def test_backward_pure_decay_closed_form():
+    """beta = 0: o_t = (prod_{s<=t} a_s) S_in^T q^_t and S_T = (prod a) S_in,
+    so dv = 0 and dstate_in = sum_t (prod_{s<=t} a_s) q^_t do_t^T +
+    (prod a) dS_T, in closed form."""
+    rng = np.random.default_rng(22)
+    q, k, v, g, _, s = _fd_inputs(rng, T=7, Dk=4, Dv=3)
+    beta = np.zeros(g.shape)
+    do = rng.standard_normal(v.shape)
+    dS = rng.standard_normal(s.shape)
+    gr = oracle.backward.grads(q, k, v, g, beta, s, do, dS)
+    assert np.all(gr["dv"] == 0)
+    dec = np.cumprod(np.exp(g), axis=1)                      # [B,T,H]
+    qn = q / np.linalg.norm(q, axis=-1, keepdims=True)
+    want = np.einsum("bth,bthi,bthj->bhij", dec, qn, do) + dec[:, -1][..., None, None] * dS
+    np.testing.assert_allclose(gr["dstate_in"], want, rtol=1e-12, atol=1e-13)
+
+
+def test_backward_is_linear_in_the_upstream_gradients():
+    rng = np.random.default_rng(23)
+    q, k, v, g, beta, s = _fd_inputs(rng, T=6)
+    d1, d2 = rng.standard_normal(v.shape), rng.standard_normal(v.shape)
+    e1, e2 = rng.standard_normal(s.shape), rng.standard_normal(s.shape)
+    g1 = oracle.backward.grads(q, k, v, g, beta, s, d1, e1, bidir=True)
+    g2 = oracle.backward.grads(q, k, v, g, beta, s, d2, e2, bidir=True)
+    g12 = oracle.backward.grads(q, k, v, g, beta, s, 2 * d1 - 3 * d2, 2 * e1 - 3 * e2, bidir=True)
+    for n in ("dq", "dk", "dv", "dg", "dbeta", "dstate_in"):
+        np.testing.assert_allclose(g12[n], 2 * g1[n] - 3 * g2[n], rtol=1e-10, atol=1e-12, err_msg=n)
+
+
+@pytest.mark.parametrize("bidir", [False, True])
+def test_backward_forward_matches_c_oracle(bidir):
+    """The torch transcription's forward is the C oracle's (both fp64)."""
+    rng = np.random.default_rng(24)
+    q, k, v, g, beta, s = rand_inputs(rng, T=19)
+    o1, S1 = oracle.backward.forward_np(q, k, v, g, beta, s, bidir)
+    o2, S2 = (c_bidir if bidir else c_fwd)(q, k, v, g, beta, s)
+    assert rel(o1, o2) < 1e-12 and rel(S1, S2) < 1e-12
