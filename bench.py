@@ -384,11 +384,11 @@ def kernel_times(lib, step_fn, n, launches_per_step):
     _lib.check(lib.gdn_profile_begin(int(n * max(1, launches_per_step) + 8)), "gdn_profile_begin")
     for i in range(n):
         step_fn(i)
-    kms = (ctypes.c_float * 5)()
-    kn = (ctypes.c_int * 5)()
-    _lib.check(lib.gdn_profile_end(ctypes.addressof(kms), ctypes.addressof(kn), 5), "gdn_profile_end")
+    kms = (ctypes.c_float * 7)()
+    kn = (ctypes.c_int * 7)()
+    _lib.check(lib.gdn_profile_end(ctypes.addressof(kms), ctypes.addressof(kn), 7), "gdn_profile_end")
     kernels = {}
-    for i in range(5):
+    for i in range(7):
         if kn[i]:
             kernels[lib.gdn_kernel_name(i).decode()] = {"launches": kn[i], "ms_per_launch": kms[i] / kn[i]}
     tot = sum(v["ms_per_launch"] for v in kernels.values())
@@ -485,6 +485,48 @@ def long_stream_figures(gdn, lib, w, stream, dev, peaks, peak_kind, barrier):
                       "serial_chunk_steps_if_G_is_sqrt": 2 * ((nC + G - 1) // G) + G},
         "speedup": ms_serial / ms_seg}
     return res
+
+
+def backward_figure(gdn, lib, base, w, stream, peaks, peak_kind, barrier):
+    """The gradients of the bidirectional streaming chunk (the pages' short
+    bidirectional training) with respect to q, k, v, g, beta and the carried
+    state, given d_out and d_state_out.  Algorithmic bytes per token-head:
+    q, k, v, d_out in and dq, dk, dv out (bf16), g, beta in and dg, dbeta out
+    (fp32); plus three fp32 states per (b, h)."""
+    import torch
+    d_out = torch.randn_like(base["q"][..., :w.Dv].float()).to(base["q"].dtype)
+    d_S = torch.randn_like(base["state_in"])
+
+    def call():
+        return gdn.chunk_bidir_backward(base["q"], base["k"], base["v"], base["g"], base["beta"],
+                                        base["state_in"], d_out, d_S, stream=stream)
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            call()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 3
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(reps):
+            call()
+    e1.record(stream)
+    barrier()
+    ms = e0.elapsed_time(e1) / reps
+
+    def direct(i):
+        with torch.cuda.stream(stream):
+            call()
+    split = kernel_times(lib, direct, 2, 2)
+    per_tok = (4 * w.Dk + 3 * w.Dv) * 2 + 16
+    nbytes = w.head_tokens * per_tok + 3 * w.B * w.H * w.Dk * w.Dv * 4
+    gbs = nbytes / (ms / 1000.0) / 1e9
+    return {"workload": "stream_chunk_bidir (gradients)", "ms_per_call": ms,
+            "head_tokens_per_s": w.head_tokens / (ms / 1000.0), "kernels": split,
+            "roofline": {"bound": "hbm", "algorithmic_bytes": nbytes, "achieved_gbs": gbs,
+                         "peak": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"],
+                         "roofline_us": 1e6 * nbytes / (peaks["hbm_gbs"] * 1e9),
+                         "peak_source": f"{peak_kind} hbm_gbs"}}
 
 
 def roofline_times(w, bidir, peaks):
@@ -764,6 +806,8 @@ def main():
                                     lg_ms, peaks, peak_kind, False)}
         del lsets
         extras.update(long_stream_figures(gdn, lib, w, stream, dev, peaks, peak_kind, barrier))
+        extras["bidir_backward_chunk"] = backward_figure(gdn, lib, base, w, stream, peaks, peak_kind,
+                                                         barrier)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -7,7 +7,8 @@ is loaded on the first call.
 """
 from . import workloads  # noqa: F401
 
-_API = ("chunk_fwd", "chunk_bidir", "chunk_fwd_logits", "chunk_bidir_logits", "state_reset",
+_API = ("chunk_fwd", "chunk_bidir", "chunk_fwd_logits", "chunk_bidir_logits",
+        "chunk_fwd_backward", "chunk_bidir_backward", "state_reset",
         "device_error", "set_wait_limit", "set_time_segments", "workspace_release")
 __all__ = [*_API, "GDNError", "workloads"]
 

@@ -26,7 +26,10 @@ GDN_BF16 = 1
 # name -> (restype, argtypes), mirroring include/gdn.h
 _vp, _fp, _i, _ll = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong
 _SCAN_ARGS = [_vp, _vp, _vp, _fp, _fp, _fp, _fp, _vp] + [_i] * 5 + [_i, _i, _vp]
+_BWD_ARGS = [_vp] * 6 + [_vp, _vp] + [_vp] * 6 + [_i] * 5 + [_i, _vp]
 SIGNATURES = {
+    "gdn_chunk_fwd_backward": (ctypes.c_int, _BWD_ARGS),
+    "gdn_chunk_bidir_backward": (ctypes.c_int, _BWD_ARGS),
     "gdn_chunk_fwd": (ctypes.c_int, _SCAN_ARGS),
     "gdn_chunk_bidir": (ctypes.c_int, _SCAN_ARGS),
     "gdn_chunk_fwd_noalloc": (ctypes.c_int, _SCAN_ARGS),

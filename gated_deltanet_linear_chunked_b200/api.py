@@ -103,6 +103,49 @@ def chunk_bidir_logits(q, k, v, g_logit, beta_logit, state_in=None, state_out=No
                  chunk, stream, logits=True)
 
 
+def _backward(entry, q, k, v, g, beta, state_in, d_out, d_state_out, stream):
+    if q.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k must be [B,T,H,Dk] and v [B,T,H,Dv]")
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    if q.dtype not in _DTYPES:
+        raise TypeError(f"q/k/v must be bfloat16 or float32, got {q.dtype}")
+    dt = q.dtype
+    _check_tensor(q, "q", dt)
+    _check_tensor(k, "k", dt, (B, T, H, Dk))
+    _check_tensor(v, "v", dt, (B, T, H, Dv))
+    _check_tensor(g, "g", torch.float32, (B, T, H))
+    _check_tensor(beta, "beta", torch.float32, (B, T, H))
+    _check_tensor(d_out, "d_out", dt, (B, T, H, Dv))
+    if state_in is not None:
+        _check_tensor(state_in, "state_in", torch.float32, (B, H, Dk, Dv))
+    if d_state_out is not None:
+        _check_tensor(d_state_out, "d_state_out", torch.float32, (B, H, Dk, Dv))
+    dev = q.device
+    res = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
+           "dg": torch.empty_like(g), "dbeta": torch.empty_like(beta),
+           "dstate_in": torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=dev)}
+    st = getattr(_lib.load(), entry)(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in), _ptr(d_out),
+        _ptr(d_state_out), _ptr(res["dq"]), _ptr(res["dk"]), _ptr(res["dv"]), _ptr(res["dg"]),
+        _ptr(res["dbeta"]), _ptr(res["dstate_in"]), B, T, H, Dk, Dv, _DTYPES[dt], _stream(stream))
+    _lib.check(st, entry)
+    return res
+
+
+def chunk_fwd_backward(q, k, v, g, beta, state_in, d_out, d_state_out=None, stream=None):
+    """Gradients of the causal scan: returns a dict with dq, dk, dv (q's dtype),
+    dg, dbeta and dstate_in (fp32), given d_out and optionally d_state_out."""
+    return _backward("gdn_chunk_fwd_backward", q, k, v, g, beta, state_in, d_out, d_state_out,
+                     stream)
+
+
+def chunk_bidir_backward(q, k, v, g, beta, state_in, d_out, d_state_out=None, stream=None):
+    """Gradients of the bidirectional scan (see chunk_fwd_backward)."""
+    return _backward("gdn_chunk_bidir_backward", q, k, v, g, beta, state_in, d_out, d_state_out,
+                     stream)
+
+
 def state_reset(state, stream=None):
     """Zero a state tensor [B,H,Dk,Dv] in place (streaming restart)."""
     _check_tensor(state, "state", torch.float32)

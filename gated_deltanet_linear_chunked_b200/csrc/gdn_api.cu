@@ -336,6 +336,85 @@ gdn_status finish(cudaStream_t s, cudaError_t launch_err, unsigned int* err) {
 
 void count_launches(unsigned n) { g_launches.fetch_add(n); }
 
+gdn_status stream_scratch(int dev, cudaStream_t s, size_t bytes, unsigned int** err, void** ws) {
+  return stream_context(dev, s, bytes, err, ws);
+}
+
+namespace {
+gdn_status backward(const void* q, const void* k, const void* v, const float* g,
+                    const float* beta, const float* state_in, const void* d_out,
+                    const float* d_state_out, void* dq, void* dk, void* dv, float* dg,
+                    float* dbeta, float* d_state_in, int B, int T, int H, int Dk, int Dv,
+                    gdn_dtype dtype, void* stream, bool bidir) {
+  // the forward's checks on the forward's arguments (out := d_out, which is
+  // only read here; state_out := d_state_in, written)
+  ScanArgs a;
+  int dev = 0;
+  gdn_status st = prepare_scan(q, k, v, g, beta, state_in, d_state_in, const_cast<void*>(d_out), B,
+                               T, H, Dk, Dv, dtype, 0, stream, bidir, false, &a, &dev);
+  if (st != GDN_OK) return st;
+  if (B == 0 || H == 0) return GDN_OK;
+  const size_t es = dtype == GDN_BF16 ? 2 : 4;
+  const size_t rows = (size_t)B * T * H;
+  const size_t sbytes = (size_t)B * H * Dk * Dv * 4;
+  if (T > 0 && (!dq || !dk || !dv || !dg || !dbeta)) return GDN_ERR_INVALID_ARG;
+  const void* outs[] = {dq, dk, dv, dg, dbeta, d_out, d_state_out};
+  for (const void* p : outs)
+    if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+  // the gradients written must not overlap anything else of the call
+  const Range w[] = {range_of(dq, rows * Dk * es), range_of(dk, rows * Dk * es),
+                     range_of(dv, rows * Dv * es), range_of(dg, rows * 4),
+                     range_of(dbeta, rows * 4), range_of(d_state_in, d_state_in ? sbytes : 0)};
+  const Range r[] = {range_of(q, rows * Dk * es), range_of(k, rows * Dk * es),
+                     range_of(v, rows * Dv * es), range_of(g, rows * 4), range_of(beta, rows * 4),
+                     range_of(state_in, state_in ? sbytes : 0), range_of(d_out, rows * Dv * es),
+                     range_of(d_state_out, d_state_out ? sbytes : 0)};
+  if (T > 0) {
+    for (int i = 0; i < 6; ++i) {
+      for (const Range& x : r)
+        if (overlaps(w[i], x)) return GDN_ERR_ALIAS;
+      for (int j = i + 1; j < 6; ++j)
+        if (overlaps(w[i], w[j])) return GDN_ERR_ALIAS;
+    }
+  }
+  for (const void* p : outs) {
+    if (!p || (T == 0 && p != d_state_out)) continue;
+    st = check_device_pointer(p, dev);
+    if (st != GDN_OK) return st;
+  }
+  cudaStream_t s = a.stream;
+  if (T == 0) {  // state_out = state_in: d_state_in = d_state_out (or zero)
+    if (!d_state_in) return GDN_OK;
+    cudaError_t e = d_state_out
+                        ? cudaMemcpyAsync(d_state_in, d_state_out, sbytes, cudaMemcpyDeviceToDevice, s)
+                        : cudaMemsetAsync(d_state_in, 0, sbytes, s);
+    return finish(s, e, nullptr);
+  }
+  unsigned int* err = nullptr;
+  void* ws = nullptr;
+  const size_t bytes = bwd_workspace_bytes(B, T, H, Dk, Dv, bidir);
+  st = stream_context(dev, s, bytes, &err, &ws);
+  if (st != GDN_OK) return st;
+  BwdCall c;
+  c.q = q; c.k = k; c.v = v; c.g = g; c.beta = beta; c.state_in = state_in;
+  c.d_out = d_out; c.d_state_out = d_state_out;
+  c.dq = dq; c.dk = dk; c.dv = dv; c.dg = dg; c.dbeta = dbeta; c.d_state_in = d_state_in;
+  c.B = B; c.T = T; c.H = H; c.Dk = Dk; c.Dv = Dv; c.dtype = dtype; c.bidir = bidir; c.stream = s;
+  cudaError_t e;
+  if (ws) {
+    e = launch_backward(c, ws);
+  } else {  // under capture without a large enough cached scratch
+    e = cudaMallocAsync(&ws, bytes, s);
+    if (e == cudaSuccess) {
+      e = launch_backward(c, ws);
+      const cudaError_t f = cudaFreeAsync(ws, s);
+      if (e == cudaSuccess) e = f;
+    }
+  }
+  return finish(s, e, nullptr);
+}
+}  // namespace
+
 cudaError_t current_error_word(unsigned int** out) { return error_word(out); }
 long long current_wait_limit() { return g_wait_limit.load(); }
 int current_time_segments() { return g_time_segments.load(); }
@@ -403,6 +482,26 @@ gdn_status gdn_chunk_bidir_logits(const void* q, const void* k, const void* v,
                                   void* stream) {
   return gdn::scan(q, k, v, g_logit, beta_logit, state_in, state_out, out, B, T, H, Dk, Dv,
                    dtype, chunk, stream, true, true);
+}
+
+gdn_status gdn_chunk_fwd_backward(const void* q, const void* k, const void* v,
+                                  const float* g, const float* beta, const float* state_in,
+                                  const void* d_out, const float* d_state_out, void* dq,
+                                  void* dk, void* dv, float* dg, float* dbeta,
+                                  float* d_state_in, int B, int T, int H, int Dk, int Dv,
+                                  gdn_dtype dtype, void* stream) {
+  return gdn::backward(q, k, v, g, beta, state_in, d_out, d_state_out, dq, dk, dv, dg, dbeta,
+                       d_state_in, B, T, H, Dk, Dv, dtype, stream, false);
+}
+
+gdn_status gdn_chunk_bidir_backward(const void* q, const void* k, const void* v,
+                                    const float* g, const float* beta, const float* state_in,
+                                    const void* d_out, const float* d_state_out, void* dq,
+                                    void* dk, void* dv, float* dg, float* dbeta,
+                                    float* d_state_in, int B, int T, int H, int Dk, int Dv,
+                                    gdn_dtype dtype, void* stream) {
+  return gdn::backward(q, k, v, g, beta, state_in, d_out, d_state_out, dq, dk, dv, dg, dbeta,
+                       d_state_in, B, T, H, Dk, Dv, dtype, stream, true);
 }
 
 gdn_status gdn_state_reset(float* state, int B, int H, int Dk, int Dv,
@@ -579,6 +678,8 @@ const char* gdn_kernel_name(int id) {
     case gdn::kKernRecur: return "gdn_recur_kernel";
     case gdn::kKernOutput: return "gdn_output_kernel";
     case gdn::kKernSegPrefix: return "gdn_segment_prefix_kernel";
+    case gdn::kKernBwdScan: return "gdn_bwd_scan_kernel";
+    case gdn::kKernBwdReduce: return "gdn_bwd_reduce_kernel";
   }
   return "unknown";
 }

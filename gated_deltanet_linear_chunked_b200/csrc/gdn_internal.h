@@ -36,7 +36,9 @@ enum KernelId : int {
   kKernRecur = 2,
   kKernOutput = 3,
   kKernSegPrefix = 4,
-  kNumKernelIds = 5,
+  kKernBwdScan = 5,
+  kKernBwdReduce = 6,
+  kNumKernelIds = 7,
 };
 
 // While profiling is armed, records CUDA events around one launch.
@@ -87,6 +89,26 @@ cudaError_t launch_scan_serial(const ScanArgs& a);
 // output.  `workspace` must hold chunk_tc_workspace_bytes(...) bytes.
 size_t chunk_tc_workspace_bytes(int B, int T, int H, int Dk, int Dv, bool bidir);
 cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace);
+
+// One backward call, after validation (device pointers).
+struct BwdCall {
+  const void *q, *k, *v;
+  const float *g, *beta, *state_in;   // state_in may be nullptr (zero state)
+  const void* d_out;                  // [B,T,H,Dv] dtype
+  const float* d_state_out;           // may be nullptr (no gradient on state_out)
+  void *dq, *dk, *dv;                 // dtype
+  float *dg, *dbeta, *d_state_in;     // d_state_in may be nullptr
+  int B, T, H, Dk, Dv;
+  gdn_dtype dtype;
+  bool bidir;
+  cudaStream_t stream;
+};
+size_t bwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, bool bidir);
+cudaError_t launch_backward(const BwdCall& c, void* workspace);
+
+// The per-(device, stream) scratch of at least `bytes` (nullptr under stream
+// capture when it cannot be provided); GDN_OK or GDN_ERR_CUDA.
+gdn_status stream_scratch(int dev, cudaStream_t s, size_t bytes, unsigned int** err, void** ws);
 
 // Device error word values.
 enum : unsigned int {

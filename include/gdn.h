@@ -147,6 +147,37 @@ GDN_API gdn_status gdn_chunk_bidir_logits(const void* q, const void* k, const vo
                                           gdn_dtype dtype, int chunk, void* stream);
 
 /*
+ * Gradients of the two scans (the pages train the bidirectional GDN:
+ * "SANA-Streaming：基于混合扩散Transformer的实时流式视频编辑系统", 方法步骤详情,
+ * second step).  Given the forward call's inputs and the gradients of a loss
+ * with respect to its results -- d_out [B, T, H, Dv] (dtype) and, optionally,
+ * d_state_out [B, H, Dk, Dv] (fp32; NULL: the final state is unused) -- they
+ * write the gradients with respect to the inputs:
+ *   dq, dk [B, T, H, Dk] and dv [B, T, H, Dv] in dtype; dg, dbeta [B, T, H]
+ *   fp32; d_state_in [B, H, Dk, Dv] fp32 (may be NULL; zero-state calls pass
+ *   state_in = NULL and get the gradient of a zero start state).
+ * The recurrence is walked in fp32 on CUDA cores (token-serial, like the fp32
+ * forward path), with checkpoints every 64 tokens; scratch comes from the
+ * stream's context.  g and beta are taken as given (no gate-logit form).
+ * The gradient outputs may not overlap each other or any input.  Errors as
+ * for gdn_chunk_fwd.
+ */
+GDN_API gdn_status gdn_chunk_fwd_backward(const void* q, const void* k, const void* v,
+                                          const float* g, const float* beta,
+                                          const float* state_in, const void* d_out,
+                                          const float* d_state_out, void* dq, void* dk, void* dv,
+                                          float* dg, float* dbeta, float* d_state_in, int B,
+                                          int T, int H, int Dk, int Dv, gdn_dtype dtype,
+                                          void* stream);
+GDN_API gdn_status gdn_chunk_bidir_backward(const void* q, const void* k, const void* v,
+                                            const float* g, const float* beta,
+                                            const float* state_in, const void* d_out,
+                                            const float* d_state_out, void* dq, void* dk,
+                                            void* dv, float* dg, float* dbeta, float* d_state_in,
+                                            int B, int T, int H, int Dk, int Dv, gdn_dtype dtype,
+                                            void* stream);
+
+/*
  * gdn_chunk_fwd for callers that cannot allocate device memory (no
  * counterpart on the pages).  Some callers cannot let a library allocate: a
  * streaming server that has already handed all remaining HBM to its caches
@@ -254,7 +285,8 @@ GDN_API unsigned long long gdn_launch_count(void);
  * events, disarms, and writes for each kernel id i < nids the total
  * milliseconds ms[i] and launch count n[i].  Kernel ids: 0 token-serial scan,
  * 1 stage A (prep), 2 stage B (recurrence, every pass), 3 stage C (output),
- * 4 the time-segment prefix; names from gdn_kernel_name.  Not thread-safe against concurrent calls on other
+ * 4 the time-segment prefix, 5 the backward scan, 6 the backward reduction;
+ * names from gdn_kernel_name.  Not thread-safe against concurrent calls on other
  * threads; meant for benchmarks.
  */
 GDN_API gdn_status gdn_profile_begin(int max_launches);
