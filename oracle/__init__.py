@@ -20,8 +20,11 @@ Contents
   * ``backward``   -- the forward definition in plain PyTorch CPU float64,
                       differentiated by autograd: the reference gradients of
                       the scan.
+  * ``sink_window_attn`` -- the softmax blocks' attention over a persistent
+                      sink and a sliding window of chunks, in numpy float64.
 
-Parity is pinned, not assumed: ``tests/test_oracle_pins.py`` checks these
+Parity is pinned, not assumed: ``tests/test_oracle_pins.py`` and
+``tests/test_oracle_sink_window.py`` check these
 functions against closed forms, invariants, a hand-derived example and brute
 force (see each test's docstring).
 """
@@ -34,6 +37,7 @@ from .cpu import (  # noqa: F401
     oracle_fwd_logits,
 )
 from . import backward  # noqa: F401
+from . import sink_window_attn  # noqa: F401
 from .numpy_ref import (  # noqa: F401
     chunked_bidir,
     chunked_fwd,
