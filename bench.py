@@ -57,7 +57,10 @@ def parse():
     p.add_argument("--no-graph", action="store_true", help="time direct calls instead of CUDA-graph replays")
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle CPU baseline")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--no-extras", action="store_true", help="skip the bidir / stacked-stream side figures")
+    p.add_argument("--no-extras", action="store_true", help="skip every side figure")
+    p.add_argument("--extras", default="all",
+                   help="comma list of side figures: side (the other mode, the 32x15 stack, "
+                        "gate logits), long (long streams), backward, sink_window; or all")
     return p.parse_args()
 
 
@@ -384,11 +387,11 @@ def kernel_times(lib, step_fn, n, launches_per_step):
     _lib.check(lib.gdn_profile_begin(int(n * max(1, launches_per_step) + 8)), "gdn_profile_begin")
     for i in range(n):
         step_fn(i)
-    kms = (ctypes.c_float * 7)()
-    kn = (ctypes.c_int * 7)()
-    _lib.check(lib.gdn_profile_end(ctypes.addressof(kms), ctypes.addressof(kn), 7), "gdn_profile_end")
+    kms = (ctypes.c_float * 8)()
+    kn = (ctypes.c_int * 8)()
+    _lib.check(lib.gdn_profile_end(ctypes.addressof(kms), ctypes.addressof(kn), 8), "gdn_profile_end")
     kernels = {}
-    for i in range(7):
+    for i in range(8):
         if kn[i]:
             kernels[lib.gdn_kernel_name(i).decode()] = {"launches": kn[i], "ms_per_launch": kms[i] / kn[i]}
     tot = sum(v["ms_per_launch"] for v in kernels.values())
@@ -527,6 +530,69 @@ def backward_figure(gdn, lib, base, w, stream, peaks, peak_kind, barrier):
                          "peak": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"],
                          "roofline_us": 1e6 * nbytes / (peaks["hbm_gbs"] * 1e9),
                          "peak_source": f"{peak_kind} hbm_gbs"}}
+
+
+def sink_window_figure(gdn, lib, stream, dev, peaks, peak_kind, barrier):
+    """The softmax blocks' attention on the streaming chunk: B1 H20 D112
+    Tc2640, one sink chunk and a window of two, at a steady-state chunk
+    (index 5: the sink, chunk 4 and its own, 7920 keys per query).  Inputs
+    and caches rotate over three sets (each about 94 MB of reads and writes,
+    together more than L2).  Tensor-bound: 4 B H Tc L D flops per call."""
+    import torch
+    from gated_deltanet_linear_chunked_b200 import workloads as wl
+    w = wl.sink_window_stream()
+    gen = torch.Generator(device=dev).manual_seed(17)
+    shape = (w.B, w.Tc, w.H, w.D)
+    cshape = (w.B, w.n_sink + w.window, w.Tc, w.H, w.D)
+    sets = []
+    for _ in range(3):
+        x = {n: torch.randn(shape, generator=gen, device=dev).to(torch.bfloat16) for n in "qkv"}
+        x["kc"] = torch.randn(cshape, generator=gen, device=dev).to(torch.bfloat16)
+        x["vc"] = torch.randn(cshape, generator=gen, device=dev).to(torch.bfloat16)
+        x["out"] = torch.empty(shape, dtype=torch.bfloat16, device=dev)
+        sets.append(x)
+    c = 5
+    nkeys = len([m for m in range(c + 1) if m < w.n_sink or m > c - w.window]) * w.Tc
+
+    def call(i):
+        x = sets[i % len(sets)]
+        gdn.sink_window_attention(x["q"], x["k"], x["v"], x["kc"], x["vc"], c, w.n_sink, w.window,
+                                  out=x["out"], stream=stream)
+    with torch.cuda.stream(stream):
+        for i in range(6):
+            call(i)
+    barrier()
+    reps = 30
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for i in range(reps):
+            call(i)
+    e1.record(stream)
+    barrier()
+    ms = e0.elapsed_time(e1) / reps
+
+    def direct(i):
+        with torch.cuda.stream(stream):
+            call(i)
+    split = kernel_times(lib, direct, 6, 1)
+    flops = 4 * w.B * w.H * w.Tc * nkeys * w.D
+    chunk_bytes = w.B * w.Tc * w.H * w.D * 2
+    nbytes = chunk_bytes * (4 + 2 * (nkeys // w.Tc - 1) + 2)   # q k v out, cache reads, cache writes
+    tf = flops / (ms / 1000.0) / 1e12
+    kms = split.get("gdn_sink_window_kernel", {}).get("ms_per_launch", ms)
+    return {"workload": f"{w.name} (B{w.B} H{w.H} D{w.D} Tc{w.Tc}, n_sink {w.n_sink}, "
+                        f"window {w.window}, chunk {c}: {nkeys} keys)",
+            "ms_per_call": ms, "head_tokens_per_s": w.B * w.H * w.Tc / (ms / 1000.0),
+            "kernels": split,
+            "roofline": {"bound": "tensor", "achieved": tf, "unit": "TFLOP/s",
+                         "peak": peaks["bf16_tflops"], "frac": tf / peaks["bf16_tflops"],
+                         "kernel_tflops": flops / (kms / 1000.0) / 1e12,
+                         "kernel_frac": flops / (kms / 1000.0) / 1e12 / peaks["bf16_tflops"],
+                         "algorithmic_flops": flops, "algorithmic_bytes": nbytes,
+                         "hbm_floor_us": 1e6 * nbytes / (peaks["hbm_gbs"] * 1e9),
+                         "tensor_floor_us": 1e6 * flops / (peaks["bf16_tflops"] * 1e12),
+                         "peak_source": f"{peak_kind} bf16_tflops (burst: the kernel is timed alone)"}}
 
 
 def roofline_times(w, bidir, peaks):
@@ -706,7 +772,10 @@ def main():
     # ---- side figures: the other mode (its own roofline), and the 15-layer
     # stacked stream (direct calls and one captured graph)
     extras = {}
-    if not args.no_extras:
+    chosen = set() if args.no_extras else (
+        {"side", "long", "backward", "sink_window"} if args.extras == "all"
+        else {x.strip() for x in args.extras.split(",") if x.strip()})
+    if "side" in chosen:
         other = "bidir" if w.mode == "fwd" else "fwd"
         fo = gdn.chunk_bidir if other == "bidir" else gdn.chunk_fwd
         n_side = max(3, min(args.steps, 200))
@@ -805,8 +874,13 @@ def main():
             "roofline": roofline_of(wlg, kernel_times(lib, lg_direct, n_prof, launches_per_step),
                                     lg_ms, peaks, peak_kind, False)}
         del lsets
+    if "long" in chosen:
         extras.update(long_stream_figures(gdn, lib, w, stream, dev, peaks, peak_kind, barrier))
+    if "backward" in chosen:
         extras["bidir_backward_chunk"] = backward_figure(gdn, lib, base, w, stream, peaks, peak_kind,
+                                                         barrier)
+    if "sink_window" in chosen:
+        extras["sink_window_chunk"] = sink_window_figure(gdn, lib, stream, dev, peaks, peak_kind,
                                                          barrier)
 
     cpu = None

@@ -35,6 +35,8 @@ SIGNATURES = {
     "gdn_chunk_fwd_noalloc": (ctypes.c_int, _SCAN_ARGS),
     "gdn_chunk_fwd_logits": (ctypes.c_int, _SCAN_ARGS),
     "gdn_chunk_bidir_logits": (ctypes.c_int, _SCAN_ARGS),
+    "gdn_sink_window_attention": (ctypes.c_int, [_vp] * 6 + [_i] * 8 + [_vp]),
+    "gdn_sink_window_slot": (ctypes.c_int, [_i, _i, _i]),
     "gdn_state_reset": (ctypes.c_int, [_fp, _i, _i, _i, _i, _vp]),
     "gdn_device_error": (ctypes.c_int, [_vp]),
     "gdn_workspace_release": (ctypes.c_int, []),

@@ -146,6 +146,46 @@ def chunk_bidir_backward(q, k, v, g, beta, state_in, d_out, d_state_out=None, st
                      stream)
 
 
+def sink_window_cache(B, Tc, H, D, n_sink, window, device=None):
+    """An empty (zeroed) KV cache pair for ``sink_window_attention``:
+    two bf16 tensors [B, n_sink + window, Tc, H, D]."""
+    shape = (B, n_sink + window, Tc, H, D)
+    return (torch.zeros(shape, dtype=torch.bfloat16, device=device or "cuda"),
+            torch.zeros(shape, dtype=torch.bfloat16, device=device or "cuda"))
+
+
+def sink_window_slot(chunk_index, n_sink, window) -> int:
+    """Cache slot that holds stream chunk ``chunk_index`` (-1: invalid)."""
+    return int(_lib.load().gdn_sink_window_slot(int(chunk_index), int(n_sink), int(window)))
+
+
+def sink_window_attention(q, k, v, k_cache, v_cache, chunk_index, n_sink, window, out=None,
+                          stream=None):
+    """Softmax attention of one streaming chunk over the sink chunks and the
+    sliding window of chunks (its own included) held in ``k_cache`` /
+    ``v_cache``; writes the chunk's k, v into its cache slot on the way.
+    q, k, v [B, Tc, H, D] bf16; caches [B, n_sink + window, Tc, H, D] bf16.
+    Returns ``out`` [B, Tc, H, D] bf16."""
+    if q.dim() != 4:
+        raise ValueError("q, k, v must be [B, Tc, H, D]")
+    B, Tc, H, D = q.shape
+    _check_tensor(q, "q", torch.bfloat16)
+    _check_tensor(k, "k", torch.bfloat16, (B, Tc, H, D))
+    _check_tensor(v, "v", torch.bfloat16, (B, Tc, H, D))
+    cshape = (B, n_sink + window, Tc, H, D)
+    _check_tensor(k_cache, "k_cache", torch.bfloat16, cshape)
+    _check_tensor(v_cache, "v_cache", torch.bfloat16, cshape)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check_tensor(out, "out", torch.bfloat16, (B, Tc, H, D))
+    st = _lib.load().gdn_sink_window_attention(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(out), B, Tc, H, D,
+        int(n_sink), int(window), int(chunk_index), _lib.GDN_BF16, _stream(stream))
+    _lib.check(st, "gdn_sink_window_attention")
+    return out
+
+
 def state_reset(state, stream=None):
     """Zero a state tensor [B,H,Dk,Dv] in place (streaming restart)."""
     _check_tensor(state, "state", torch.float32)

@@ -1376,20 +1376,9 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// A [B, T, H, D] bf16 tensor viewed as 5-D (8 features, T, D/8 feature slabs,
-// H, B) so that one box (8 x 64 tokens x D/8 slabs x 1 x 1) lands in shared
-// memory exactly in the [slab][token][8] core-matrix layout of a tile.
+// A 64-token tile map of a [B, T, H, D] bf16 tensor.
 bool make_map(CUtensorMap* m, const void* base, int B, int T, int H, int D) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[5] = {8, (cuuint64_t)T, (cuuint64_t)(D / 8), (cuuint64_t)H, (cuuint64_t)B};
-  const cuuint64_t strides[4] = {(cuuint64_t)H * D * 2, 16, (cuuint64_t)D * 2,
-                                 (cuuint64_t)T * H * D * 2};
-  const cuuint32_t box[5] = {8, (cuuint32_t)kC, (cuuint32_t)(D / 8), 1, 1};
-  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return make_tile_map(m, base, B, T, H, D, kC);
 }
 
 // Streaming multiprocessors of the current device (persistent grids).
@@ -1529,6 +1518,19 @@ int time_segments(int B, int T, int H, int Dk, int Dv, bool bidir) {
   G = std::max(1, std::min(G, nC / 2));
   const int seg_len = (nC + G - 1) / G;
   return (nC + seg_len - 1) / seg_len;  // no empty segment
+}
+
+bool make_tile_map(CUtensorMap* m, const void* base, int nb, int T, int H, int D, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[5] = {8, (cuuint64_t)T, (cuuint64_t)(D / 8), (cuuint64_t)H, (cuuint64_t)nb};
+  const cuuint64_t strides[4] = {(cuuint64_t)H * D * 2, 16, (cuuint64_t)D * 2,
+                                 (cuuint64_t)T * H * D * 2};
+  const cuuint32_t box[5] = {8, (cuuint32_t)box_rows, (cuuint32_t)(D / 8), 1, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 size_t chunk_tc_workspace_bytes(int B, int T, int H, int Dk, int Dv, bool bidir) {

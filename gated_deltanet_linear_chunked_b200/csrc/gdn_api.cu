@@ -413,6 +413,64 @@ gdn_status backward(const void* q, const void* k, const void* v, const float* g,
   }
   return finish(s, e, nullptr);
 }
+gdn_status sink_window(const void* q, const void* k, const void* v, void* k_cache,
+                       void* v_cache, void* out, int B, int Tc, int H, int D, int n_sink,
+                       int window, int chunk, gdn_dtype dtype, void* stream) {
+  // ---- pure host checks
+  if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+  if (B < 0 || Tc < 0 || H < 0 || D < 0) return GDN_ERR_INVALID_ARG;
+  if (n_sink < 0 || window < 1 || n_sink + window > kSwaMaxSeg || chunk < 0)
+    return GDN_ERR_INVALID_ARG;
+  if (dtype != GDN_BF16 || !supported_dim(D)) return GDN_ERR_UNSUPPORTED;
+  if ((long long)B * H > 65535) return GDN_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || Tc == 0) return GDN_OK;
+  const void* ptrs[] = {q, k, v, k_cache, v_cache, out};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return GDN_ERR_INVALID_ARG;
+  const size_t chunk_bytes = (size_t)B * Tc * H * D * 2;
+  const int nslot = n_sink + window;
+  const size_t cache_bytes = chunk_bytes * nslot;
+  const Range rq = range_of(q, chunk_bytes), rk = range_of(k, chunk_bytes);
+  const Range rv = range_of(v, chunk_bytes), ro = range_of(out, chunk_bytes);
+  const Range rkc = range_of(k_cache, cache_bytes), rvc = range_of(v_cache, cache_bytes);
+  for (Range r : {rq, rk, rv, rkc, rvc})
+    if (overlaps(ro, r)) return GDN_ERR_ALIAS;
+  if (overlaps(rkc, rvc) || overlaps(rkc, rq) || overlaps(rvc, rq)) return GDN_ERR_ALIAS;
+  // k (v) may be exactly this chunk's slot of its own cache: with B > 1 a
+  // slot is strided over the batch, so only B == 1 makes it one block
+  const int slot = sink_window_slot(chunk, n_sink, window);
+  const uint8_t* kslot = static_cast<const uint8_t*>(k_cache) + (size_t)slot * Tc * H * D * 2;
+  const uint8_t* vslot = static_cast<const uint8_t*>(v_cache) + (size_t)slot * Tc * H * D * 2;
+  if (overlaps(rk, rkc) && !(B == 1 && k == kslot)) return GDN_ERR_ALIAS;
+  if (overlaps(rv, rvc) && !(B == 1 && v == vslot)) return GDN_ERR_ALIAS;
+  if (overlaps(rk, rvc) || overlaps(rv, rkc)) return GDN_ERR_ALIAS;
+
+  // ---- device checks
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return GDN_ERR_CUDA;
+  }
+  for (const void* p : ptrs) {
+    const gdn_status st = check_device_pointer(p, dev);
+    if (st != GDN_OK) return st;
+  }
+  cudaGetLastError();
+  SwaCall c;
+  c.q = q; c.k = k; c.v = v; c.k_cache = k_cache; c.v_cache = v_cache; c.out = out;
+  c.B = B; c.Tc = Tc; c.H = H; c.D = D; c.n_sink = n_sink; c.window = window; c.chunk = chunk;
+  c.stream = static_cast<cudaStream_t>(stream);
+  void* ws = nullptr;
+  gdn_status st = stream_context(dev, c.stream, 0, &c.err, &ws);
+  if (st != GDN_OK) return st;
+  if (!c.err && error_word(&c.err) != cudaSuccess) {
+    cudaGetLastError();
+    return GDN_ERR_CUDA;
+  }
+  c.limit = g_wait_limit.load();
+  return finish(c.stream, launch_sink_window(c), c.err);
+}
+
 }  // namespace
 
 cudaError_t current_error_word(unsigned int** out) { return error_word(out); }
@@ -502,6 +560,19 @@ gdn_status gdn_chunk_bidir_backward(const void* q, const void* k, const void* v,
                                     gdn_dtype dtype, void* stream) {
   return gdn::backward(q, k, v, g, beta, state_in, d_out, d_state_out, dq, dk, dv, dg, dbeta,
                        d_state_in, B, T, H, Dk, Dv, dtype, stream, true);
+}
+
+gdn_status gdn_sink_window_attention(const void* q, const void* k, const void* v, void* k_cache,
+                                     void* v_cache, void* out, int B, int Tc, int H, int D,
+                                     int n_sink, int window, int chunk_index, gdn_dtype dtype,
+                                     void* stream) {
+  return gdn::sink_window(q, k, v, k_cache, v_cache, out, B, Tc, H, D, n_sink, window,
+                          chunk_index, dtype, stream);
+}
+
+int gdn_sink_window_slot(int chunk_index, int n_sink, int window) {
+  if (chunk_index < 0 || n_sink < 0 || window < 1) return -1;
+  return gdn::sink_window_slot(chunk_index, n_sink, window);
 }
 
 gdn_status gdn_state_reset(float* state, int B, int H, int Dk, int Dv,
@@ -680,6 +751,7 @@ const char* gdn_kernel_name(int id) {
     case gdn::kKernSegPrefix: return "gdn_segment_prefix_kernel";
     case gdn::kKernBwdScan: return "gdn_bwd_scan_kernel";
     case gdn::kKernBwdReduce: return "gdn_bwd_reduce_kernel";
+    case gdn::kKernSinkWindow: return "gdn_sink_window_kernel";
   }
   return "unknown";
 }

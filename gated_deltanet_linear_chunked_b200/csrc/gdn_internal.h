@@ -2,6 +2,7 @@
 // translation units.  Not installed; callers use include/gdn.h.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -38,7 +39,8 @@ enum KernelId : int {
   kKernSegPrefix = 4,
   kKernBwdScan = 5,
   kKernBwdReduce = 6,
-  kNumKernelIds = 7,
+  kKernSinkWindow = 7,
+  kNumKernelIds = 8,
 };
 
 // While profiling is armed, records CUDA events around one launch.
@@ -105,6 +107,27 @@ struct BwdCall {
 };
 size_t bwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, bool bidir);
 cudaError_t launch_backward(const BwdCall& c, void* workspace);
+
+// A [nb, T, H, D] bf16 tensor viewed as 5-D (8 features, T, D/8 feature
+// slabs, H, nb) so that one box (8 x box_rows tokens x D/8 slabs x 1 x 1)
+// lands in shared memory in the [slab][token][8] core-matrix layout.
+bool make_tile_map(CUtensorMap* m, const void* base, int nb, int T, int H, int D, int box_rows);
+
+// One sink + sliding-window attention call, after validation.
+constexpr int kSwaMaxSeg = 16;  // n_sink + window at most
+struct SwaCall {
+  const void *q, *k, *v;       // [B, Tc, H, D] bf16: this chunk
+  void *k_cache, *v_cache;     // [B, n_sink + window, Tc, H, D] bf16
+  void* out;                   // [B, Tc, H, D] bf16
+  int B, Tc, H, D, n_sink, window, chunk;
+  cudaStream_t stream;
+  unsigned int* err;
+  long long limit;
+};
+// Cache slot of stream chunk `chunk`: sink chunks keep their own slots, the
+// rest share `window` ring slots.
+int sink_window_slot(int chunk, int n_sink, int window);
+cudaError_t launch_sink_window(const SwaCall& c);
 
 // The per-(device, stream) scratch of at least `bytes` (nullptr under stream
 // capture when it cannot be provided); GDN_OK or GDN_ERR_CUDA.

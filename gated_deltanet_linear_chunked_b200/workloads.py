@@ -234,3 +234,48 @@ def slice_head(inputs: dict, b: int, h: int) -> dict:
     s = inputs.get("state_in")
     out["state_in"] = None if s is None else np.ascontiguousarray(s[b:b + 1, h:h + 1])
     return out
+
+
+# --------------------------------------------------------------------------
+# The softmax blocks' sink + sliding-window attention
+
+
+@dataclasses.dataclass(frozen=True)
+class AttnStream:
+    """A stream of chunks through one softmax block: per chunk q, k, v
+    [B, Tc, H, D] bf16, drawn N(0, 1) (k, v) and N(0, q_scale^2) (q), rounded
+    to bf16; the block keeps ``n_sink`` sink chunks and a ``window`` of chunks
+    (its own included)."""
+    name: str
+    B: int
+    Tc: int
+    H: int
+    D: int
+    n_sink: int
+    window: int
+    chunks: int           # chunks 0 .. chunks-1 of the stream
+    seed: int
+    q_scale: float = 1.0  # > 1 sharpens the softmax (scores ~ N(0, q_scale^2))
+
+    @property
+    def steady_chunk(self) -> int:
+        """The first chunk whose query sees the full key set (sink + window)."""
+        return self.n_sink + self.window - 1
+
+
+def sink_window_stream(seed: int = 5, chunks: int = 4) -> AttnStream:
+    """The streaming chunk through a softmax block: B1 H20 D112 Tc2640 (the
+    GDN blocks' head layout), one sink chunk and a window of two chunks, so
+    from chunk 2 on a query sees 3 x 2640 = 7920 keys."""
+    return AttnStream("sink_window_chunk", 1, CHUNK_TOKENS, 20, 112, 1, 2, chunks, seed)
+
+
+def attn_chunk(w: AttnStream, c: int) -> dict:
+    """q, k, v of stream chunk c (fp32 arrays holding bf16 values), drawn from
+    the generator seeded with [seed, c] in the order q, k, v."""
+    rng = np.random.default_rng([w.seed, c])
+    shape = (w.B, w.Tc, w.H, w.D)
+    q = rng.standard_normal(shape, dtype=np.float32) * np.float32(w.q_scale)
+    k = rng.standard_normal(shape, dtype=np.float32)
+    v = rng.standard_normal(shape, dtype=np.float32)
+    return {"q": round_bf16(q), "k": round_bf16(k), "v": round_bf16(v)}

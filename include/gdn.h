@@ -252,6 +252,53 @@ GDN_API gdn_status gdn_workspace_release(void);
 GDN_API long long gdn_set_wait_limit(long long polls);
 
 /*
+ * The softmax blocks' attention: sink + sliding window over a streaming KV
+ * cache.  The hybrid DiT places softmax attention blocks among the GDN blocks
+ * at even intervals; each keeps a persistent sink and a sliding window, so
+ * its memory is fixed by the window while it still sees fine correspondences
+ * across chunk boundaries ("SANA-Streaming：基于混合扩散Transformer的实时流式
+ * 视频编辑系统", 核心方法; softmax attention is the dot-product, softmax-
+ * normalised token interaction of the same page's 线性注意力 vs Softmax注意力).
+ * The pages give neither size nor unit; here both count whole chunks.  A
+ * query of stream chunk c (chunk_index, from 0) attends to every token of
+ * chunk m iff m <= c and (m < n_sink or m > c - window):
+ *
+ *     out = softmax(q K^T / sqrt(D)) V      per (b, h), fp32 softmax and
+ *                                           accumulation, bf16 P and out
+ *
+ * over those keys, its own chunk's in both directions.  During the same call
+ * the chunk's k and v are written into the cache slot
+ * gdn_sink_window_slot(c, n_sink, window); the chunks read come from their
+ * slots, so a stream is a sequence of calls with c = 0, 1, 2, ... on one
+ * cache (chunks that left the window are overwritten, sink chunks never).
+ *
+ *   q, k, v, out   [B, Tc, H, D]                      bf16 (this chunk)
+ *   k_cache,       [B, n_sink + window, Tc, H, D]     bf16, caller-owned;
+ *   v_cache         a slot holds one chunk
+ *
+ * Requirements: dtype GDN_BF16 (else GDN_ERR_UNSUPPORTED); D a multiple of
+ * 16 in [16, 128] (else GDN_ERR_UNSUPPORTED); n_sink >= 0, window >= 1,
+ * n_sink + window <= 16, chunk_index >= 0 (else GDN_ERR_INVALID_ARG);
+ * B * H <= 65535 (else GDN_ERR_UNSUPPORTED); all six pointers device memory,
+ * 16-byte aligned.  out must not overlap anything; the two caches must not
+ * overlap each other, q or out; k (v) may overlap k_cache (v_cache) only by
+ * being exactly this chunk's slot in it (the projection wrote there).
+ * Otherwise GDN_ERR_ALIAS.  Tc, B or H zero: nothing to do, GDN_OK.  Errors
+ * and the per-stream error word as for the scan.
+ */
+GDN_API gdn_status gdn_sink_window_attention(const void* q, const void* k, const void* v,
+                                             void* k_cache, void* v_cache, void* out, int B,
+                                             int Tc, int H, int D, int n_sink, int window,
+                                             int chunk_index, gdn_dtype dtype, void* stream);
+
+/*
+ * Cache slot that holds stream chunk `chunk_index` (host-only arithmetic):
+ * chunk_index itself for a sink chunk (chunk_index < n_sink), else
+ * n_sink + (chunk_index - n_sink) mod window.  -1 for invalid arguments.
+ */
+GDN_API int gdn_sink_window_slot(int chunk_index, int n_sink, int window);
+
+/*
  * Time segments of the bf16 path's recurrence.  The stage that walks the
  * chunks is a dependent chain of ceil(T / 64) steps per (head, 16 state
  * columns).  When a call has too few such chains to fill the GPU and many
@@ -285,8 +332,8 @@ GDN_API unsigned long long gdn_launch_count(void);
  * events, disarms, and writes for each kernel id i < nids the total
  * milliseconds ms[i] and launch count n[i].  Kernel ids: 0 token-serial scan,
  * 1 stage A (prep), 2 stage B (recurrence, every pass), 3 stage C (output),
- * 4 the time-segment prefix, 5 the backward scan, 6 the backward reduction;
- * names from gdn_kernel_name.  Not thread-safe against concurrent calls on other
+ * 4 the time-segment prefix, 5 the backward scan, 6 the backward reduction,
+ * 7 the sink + window attention; names from gdn_kernel_name.  Not thread-safe against concurrent calls on other
  * threads; meant for benchmarks.
  */
 GDN_API gdn_status gdn_profile_begin(int max_launches);

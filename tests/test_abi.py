@@ -141,3 +141,57 @@ def test_time_segment_hook_round_trips():
     assert lib.gdn_set_time_segments(-3) == 7      # negative means automatic
     assert lib.gdn_set_time_segments(old) == 0
     assert lib.gdn_kernel_name(4).decode() == "gdn_segment_prefix_kernel"
+
+
+def swa(q=fake(0), k=fake(1), v=fake(2), kc=fake(3), vc=fake(4), out=fake(5), B=1, Tc=64, H=2,
+        D=64, n_sink=1, window=2, c=3, dtype=_lib.GDN_BF16):
+    return _lib.load().gdn_sink_window_attention(q, k, v, kc, vc, out, B, Tc, H, D, n_sink,
+                                                 window, c, dtype, None)
+
+
+def test_sink_window_slots_by_hand():
+    lib = _lib.load()
+    # one sink chunk, window 2: chunk 0 in the sink slot, then the ring 1, 2, 1, 2, ...
+    assert [lib.gdn_sink_window_slot(c, 1, 2) for c in range(7)] == [0, 1, 2, 1, 2, 1, 2]
+    # two sink chunks, window 3: ring slots 2, 3, 4
+    assert [lib.gdn_sink_window_slot(c, 2, 3) for c in range(8)] == [0, 1, 2, 3, 4, 2, 3, 4]
+    assert [lib.gdn_sink_window_slot(c, 0, 1) for c in range(3)] == [0, 0, 0]
+    assert lib.gdn_sink_window_slot(-1, 1, 2) == -1
+    assert lib.gdn_sink_window_slot(0, -1, 2) == -1
+    assert lib.gdn_sink_window_slot(0, 1, 0) == -1
+
+
+def test_sink_window_host_checks():
+    assert swa(window=0) == _lib.GDN_ERR_INVALID_ARG
+    assert swa(n_sink=-1) == _lib.GDN_ERR_INVALID_ARG
+    assert swa(n_sink=9, window=8) == _lib.GDN_ERR_INVALID_ARG
+    assert swa(c=-1) == _lib.GDN_ERR_INVALID_ARG
+    assert swa(B=-1) == _lib.GDN_ERR_INVALID_ARG
+    assert swa(Tc=-1) == _lib.GDN_ERR_INVALID_ARG
+    assert swa(dtype=7) == _lib.GDN_ERR_INVALID_ARG
+    assert swa(dtype=_lib.GDN_F32) == _lib.GDN_ERR_UNSUPPORTED
+    for d in (0, 8, 100, 144):
+        assert swa(D=d) == _lib.GDN_ERR_UNSUPPORTED, d
+    assert swa(B=2, H=40000) == _lib.GDN_ERR_UNSUPPORTED
+    # nothing to do
+    assert swa(Tc=0, q=None, k=None, v=None, kc=None, vc=None, out=None) == _lib.GDN_OK
+    assert swa(B=0, q=None) == _lib.GDN_OK
+    for name in ("q", "k", "v", "kc", "vc", "out"):
+        assert swa(**{name: None}) == _lib.GDN_ERR_INVALID_ARG, name
+        assert swa(**{name: fake(0 if name != "q" else 9) + 8}) == _lib.GDN_ERR_INVALID_ARG, name
+
+
+def test_sink_window_overlaps():
+    chunk = 64 * 2 * 64 * 2          # bytes of one chunk (B1 Tc64 H2 D64 bf16)
+    for name in ("q", "k", "v", "kc", "vc"):
+        assert swa(**{name: fake(5) + 1024}) == _lib.GDN_ERR_ALIAS, name   # out overlaps it
+    assert swa(vc=fake(3) + chunk) == _lib.GDN_ERR_ALIAS                  # the caches overlap
+    assert swa(q=fake(3) + chunk) == _lib.GDN_ERR_ALIAS                   # q inside k_cache
+    slot = _lib.load().gdn_sink_window_slot(3, 1, 2)
+    assert swa(k=fake(3) + (slot ^ 3) * chunk) == _lib.GDN_ERR_ALIAS      # k in another slot
+    assert swa(k=fake(4) + slot * chunk) == _lib.GDN_ERR_ALIAS            # k inside v_cache
+    assert swa(k=fake(3) + slot * chunk, B=2) == _lib.GDN_ERR_ALIAS       # a slot is strided for B > 1
+    # k, v exactly this chunk's slots (B = 1): the host checks pass; with no
+    # usable device the device checks report it, and nothing is launched
+    st = swa(k=fake(3) + slot * chunk, v=fake(4) + slot * chunk)
+    assert st in (_lib.GDN_ERR_CUDA, _lib.GDN_ERR_INVALID_ARG)
