@@ -9,25 +9,33 @@
 //
 //   out = softmax(Q K^T / sqrt(D)) V   over the visible keys, per (b, h)
 //
-// One CTA per 128 query rows of one (b, h), two CTAs per SM.  The work is a
-// dense contraction, so it runs on tcgen05 with TMEM accumulators, online
-// softmax between the two products (the streaming form of softmax that keeps
-// a running maximum and sum per row):
-//   warp 4 (one lane)  TMA producer: the Q tile, then 64-key K and V tiles of
-//                      every visible chunk through two 2-stage rings; it also
+// One CTA per 256 query rows of one (b, h): two 128-row query tiles that
+// share every K and V tile loaded (halving the K/V traffic per flop), one CTA
+// per SM holding all 512 TMEM columns.  The work is a dense contraction, so
+// it runs on tcgen05 with TMEM accumulators, online softmax between the two
+// products (the streaming form of softmax that keeps a running maximum and
+// sum per row):
+//   warp 8 (one lane)  TMA producer: the Q tiles, then 64-key K and V tiles of
+//                      every visible chunk through two 4-stage rings; it also
 //                      stores the current chunk's K and V tiles that match
 //                      this CTA's query rows into the cache slot of chunk c.
-//   warp 5 (one lane)  MMA issuer: S_j = Q K_j^T (M 128, N 64) into one of two
-//                      TMEM S buffers, then O += P_{j-1} V_{j-1} (M 128, N D).
-//   warps 0-3          softmax, one query row per thread (its TMEM lane): row
-//                      maximum, p = 2^(s log2e / sqrt(D) - m), row sum, P as
-//                      bf16 to shared memory; O is rescaled in TMEM only when
-//                      the running maximum grows by more than 2^8 (otherwise
-//                      p may reach 2^8, which fp32 sums and bf16 P hold
-//                      exactly as well); at the end O / l goes out through
-//                      shared memory and one TMA store.
-// Every wait is bounded; a wait that gives up sets the error word, and the
-// CTA drains its copies and MMAs before it frees TMEM and leaves.
+//   warps 9, 10        MMA issue, one lane per query tile g: per key tile j,
+//                      S_gj = Q_g K_j^T (M 128, N 64) into one of two TMEM S
+//                      buffers of tile g, then O_g += P_g,j-1 V_j-1 (M 128, N D).
+//                      Two issuing threads, because each bounded wait costs
+//                      the issuing thread about as long as an MMA takes; the
+//                      tensor pipe interleaves their MMAs.
+//   warps 0-3, 4-7     softmax of query tiles 0 and 1, one row per thread (its
+//                      TMEM lane): row maximum, p = 2^(s log2e / sqrt(D) - m),
+//                      row sum, P as bf16 to shared memory; O is rescaled in
+//                      TMEM only when the running maximum grows by more than
+//                      2^8 (otherwise p may reach 2^8, which fp32 sums and bf16
+//                      P hold as well as 1); at the end O / l goes out through
+//                      shared memory and one TMA store per tile.
+// The two warpgroups alternate on the tensor pipe: while one computes its
+// softmax the MMAs of the other run.  Every wait is bounded; a wait that gives
+// up sets the error word, and the CTA drains its copies and MMAs before it
+// frees TMEM and leaves.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -43,13 +51,19 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kQRows = 128;          // query rows per CTA = TMEM lanes
-constexpr int kKRows = 64;           // keys per tile
-constexpr int kStages = 2;           // K/V ring depth
-constexpr int kThreads = 192;        // softmax warps 0-3, producer 4, MMA 5
-constexpr uint32_t kTmemCols = 256;  // S0 [0, 64) | S1 [64, 128) | O [128, 128 + D)
-constexpr float kRescaleLog2 = 8.f;  // headroom of the running maximum
-constexpr long long kDrainPolls = 1LL << 40;  // drains are bounded by the 2 s timer
+constexpr int kQTiles = 2;                     // 128-row query tiles per CTA
+constexpr int kQRows = 128;                    // rows per query tile = TMEM lanes
+constexpr int kKRows = 64;                     // keys per tile
+constexpr int kStages = 4;                     // K and V ring depth
+constexpr int kSoftmaxWarps = 4 * kQTiles;
+constexpr int kProducerWarp = kSoftmaxWarps;
+constexpr int kMmaWarp = kSoftmaxWarps + 1;    // first MMA warp: one per query tile
+constexpr int kThreads = 32 * (kSoftmaxWarps + 1 + kQTiles);
+constexpr uint32_t kTileCols = 256;            // per query tile: S0 [0,64) | S1 [64,128) | O [128, 128+D)
+constexpr uint32_t kTmemCols = kTileCols * kQTiles;
+constexpr uint32_t kMinSmem = 116 * 1024;      // more than half an SM: one CTA per SM
+constexpr float kRescaleLog2 = 8.f;            // headroom of the running maximum
+constexpr long long kDrainPolls = 1LL << 40;   // drains are bounded by the 2 s timer
 
 struct SwaParams {
   int Tc, H, D, nslot;
@@ -64,31 +78,37 @@ struct SwaParams {
 struct SwaBars {
   uint64_t q_full;
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], s_free[2];
-  uint64_t p_full, pv_done, drain;
+  uint64_t s_full[kQTiles][2], s_free[kQTiles][2];
+  uint64_t p_full[kQTiles], pv_done[kQTiles];
+  uint64_t drain[kQTiles];
   uint32_t tmem;
   int abort;
 };
 
-// Shared memory: Q [D/8][128][8] (later the output tile), the K/V ring
-// (per stage K [D/8][64][8] | V [D/8][64][8]), P [8][128][8], barriers.
+// Shared memory: Q tiles [g][D/8][128][8] (later the output tiles), the K and
+// V rings (per stage K [D/8][64][8] | V [D/8][64][8]), P [g][8][128][8],
+// barriers.
 struct SwaLayout {
-  uint32_t q, kv, kv_stage, v_off, p, bars, total;
+  uint32_t q, q_tile, kv, kv_stage, v_off, p, p_tile, bars, total;
 };
 __host__ __device__ inline SwaLayout swa_layout(int D) {
   SwaLayout L;
   L.q = 0;
-  L.kv = kQRows * D * 2;
+  L.q_tile = kQRows * D * 2;
+  L.kv = kQTiles * L.q_tile;
   L.v_off = kKRows * D * 2;
   L.kv_stage = 2 * L.v_off;
   L.p = L.kv + kStages * L.kv_stage;
-  L.bars = L.p + kQRows * kKRows * 2;
+  L.p_tile = kQRows * kKRows * 2;
+  L.bars = L.p + kQTiles * L.p_tile;
   L.total = L.bars + 256;
+  if (L.total < kMinSmem) L.total = kMinSmem;
   return L;
 }
 static_assert(sizeof(SwaBars) <= 256, "barrier block");
 
-__global__ void __launch_bounds__(kThreads, 2)
+template <int NK>  // D / 16
+__global__ void __launch_bounds__(kThreads, 1)
 gdn_sink_window_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v,
@@ -97,11 +117,13 @@ gdn_sink_window_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_out,
                        const __grid_constant__ SwaParams P) {
   extern __shared__ __align__(128) uint8_t smem[];
-  const SwaLayout L = swa_layout(P.D);
+  constexpr int D = 16 * NK;
+  const SwaLayout L = swa_layout(D);
   SwaBars& bar = *reinterpret_cast<SwaBars*>(smem + L.bars);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qt = blockIdx.x, bh = blockIdx.y, b = bh / P.H, h = bh - b * P.H;
-  const int q0 = qt * kQRows, D = P.D, tps = P.tiles_per_seg;
+  const int pair = blockIdx.x, bh = blockIdx.y, b = bh / P.H, h = bh - b * P.H;
+  const int q0 = pair * kQTiles * kQRows, tps = P.tiles_per_seg;
+  const int nq = min(kQTiles, (P.Tc - q0 + kQRows - 1) / kQRows);  // query tiles present
   const int ntiles = P.nseg * tps;
   volatile int* abort_flag = &bar.abort;
 
@@ -109,21 +131,23 @@ gdn_sink_window_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(&bar.q_full, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bar.k_full[s], 1);
-      mbar_init(&bar.k_empty[s], 1);
+      mbar_init(&bar.k_empty[s], nq);  // one release per MMA warp in use
       mbar_init(&bar.v_full[s], 1);
-      mbar_init(&bar.v_empty[s], 1);
+      mbar_init(&bar.v_empty[s], nq);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bar.s_full[s], 1);
-      mbar_init(&bar.s_free[s], 128);
+    for (int g = 0; g < kQTiles; ++g) {
+      for (int s = 0; s < 2; ++s) {
+        mbar_init(&bar.s_full[g][s], 1);
+        mbar_init(&bar.s_free[g][s], 128);
+      }
+      mbar_init(&bar.p_full[g], 128);
+      mbar_init(&bar.pv_done[g], 1);
+      mbar_init(&bar.drain[g], 1);
     }
-    mbar_init(&bar.p_full, 128);
-    mbar_init(&bar.pv_done, 1);
-    mbar_init(&bar.drain, 1);
     bar.abort = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&bar.tmem, kTmemCols);
     tmem_relinquish();
   }
@@ -136,14 +160,14 @@ gdn_sink_window_kernel(const __grid_constant__ CUtensorMap tm_q,
     atomicOr(P.err, kErrTimeout);
   };
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
-    // K runs one tile ahead of V: K_j is free once S_j is done, V_j only
-    // once P_j V_j is, so the two rings refill independently.
+    // K runs one tile ahead of V: K_j is free once the S MMAs of tile j are
+    // done, V_j only once the P V MMAs are, so the rings refill independently.
     if (lane == 0) {
-      uint8_t* sq = smem + L.q;
-      mbar_arrive_expect_tx(&bar.q_full, kQRows * D * 2);
-      tma_load_tile(sq, &tm_q, &bar.q_full, q0, h, b);
+      mbar_arrive_expect_tx(&bar.q_full, nq * L.q_tile);
+      for (int g = 0; g < nq; ++g)
+        tma_load_tile(smem + L.q + g * L.q_tile, &tm_q, &bar.q_full, q0 + g * kQRows, h, b);
       const int cache_bs = b * P.nslot;
       // per ring (0: K, 1: V): loads issued into each stage, and the first
       // row of a tile still to be stored from the stage into the cache (-1)
@@ -187,7 +211,7 @@ gdn_sink_window_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_arrive_expect_tx(full(x, st), kKRows * D * 2);
         if (slot < 0) {
           tma_load_tile(stage_ptr(x, st), x ? &tm_v : &tm_k, full(x, st), r0, h, b);
-          if (P.append_slot >= 0 && r0 / kQRows == qt) append_row[x][st] = r0;
+          if (P.append_slot >= 0 && r0 / (kQTiles * kQRows) == pair) append_row[x][st] = r0;
         } else {
           tma_load_tile(stage_ptr(x, st), x ? &tm_vc : &tm_kc, full(x, st), r0, h, cache_bs + slot);
         }
@@ -208,13 +232,21 @@ gdn_sink_window_kernel(const __grid_constant__ CUtensorMap tm_q,
           if (loads[x][st]) mbar_wait(full(x, st), (loads[x][st] - 1) & 1, kDrainPolls);
       bulk_wait_all();
     }
-  } else if (warp == 5) {
+  } else if (warp >= kMmaWarp) {
     // ----------------------------------------------------------- MMA issue
-    if (lane == 0) {
+    const int g = warp - kMmaWarp;
+    if (lane == 0 && g < nq) {
+      constexpr uint32_t kQSlab = kQRows * 16, kKSlab = kKRows * 16;
       const uint32_t idS = idesc_bf16(kQRows, kKRows, 0, 0);
       const uint32_t idO = idesc_bf16(kQRows, D, 0, 1);
-      const uint32_t qa = smem_u32(smem + L.q), pa = smem_u32(smem + L.p);
-      constexpr uint32_t kQSlab = kQRows * 16, kKSlab = kKRows * 16;
+      const uint32_t tS = tm + g * kTileCols, tOg = tS + 2 * kKRows;
+      // descriptors of stage 0 / this tile; a stage or a K step moves only
+      // the start-address field (addresses >> 4)
+      const uint64_t dq = sdesc(smem_u32(smem + L.q + g * L.q_tile), kQSlab, 128);
+      const uint64_t dp = sdesc(smem_u32(smem + L.p + g * L.p_tile), kQSlab, 128);
+      const uint64_t dk = sdesc(smem_u32(smem + L.kv), kKSlab, 128);
+      const uint64_t dv = sdesc(smem_u32(smem + L.kv + L.v_off), 128, kKSlab);
+      const uint64_t dstage = L.kv_stage >> 4;
       bool ok = mbar_wait(&bar.q_full, 0, P.limit);
       if (!ok) fail();
       tc_fence_after_sync();
@@ -223,46 +255,49 @@ gdn_sink_window_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (j < ntiles) {
           const int s = j % kStages, sb = j & 1;
           if (!mbar_wait(&bar.k_full[s], (j / kStages) & 1, P.limit) ||
-              (j >= 2 && !mbar_wait(&bar.s_free[sb], ((j >> 1) - 1) & 1, P.limit))) {
+              (j >= 2 && !mbar_wait(&bar.s_free[g][sb], ((j >> 1) - 1) & 1, P.limit))) {
             fail();
             break;
           }
           tc_fence_after_sync();
-          const uint32_t ka = smem_u32(smem + L.kv + s * L.kv_stage);
-          // S_j = Q K_j^T: both K-major, K = D in steps of 16
-          for (int ks = 0; ks < D / 16; ++ks)
-            mma_bf16(tm + sb * kKRows, sdesc(qa + ks * 2 * kQSlab, kQSlab, 128),
-                     sdesc(ka + ks * 2 * kKSlab, kKSlab, 128), idS, ks > 0);
-          mma_commit(&bar.s_full[sb]);
+          // S_gj = Q_g K_j^T: both K-major, K = D in steps of 16
+          const uint64_t dks = dk + s * dstage;
+#pragma unroll
+          for (int ks = 0; ks < NK; ++ks)
+            mma_bf16(tS + sb * kKRows, dq + ks * (2 * kQSlab >> 4), dks + ks * (2 * kKSlab >> 4), idS,
+                     ks > 0);
+          mma_commit(&bar.s_full[g][sb]);
           mma_commit(&bar.k_empty[s]);
         }
         if (j >= 1) {
           const int jp = j - 1, s = jp % kStages;
           if (!mbar_wait(&bar.v_full[s], (jp / kStages) & 1, P.limit) ||
-              !mbar_wait(&bar.p_full, jp & 1, P.limit)) {
+              !mbar_wait(&bar.p_full[g], jp & 1, P.limit)) {
             fail();
             break;
           }
           tc_fence_after_sync();
-          const uint32_t va = smem_u32(smem + L.kv + s * L.kv_stage + L.v_off);
-          // O += P V: P K-major (K = 64 keys), V MN-major (N = D)
+          // O_g += P_g V: P K-major (K = 64 keys), V MN-major (N = D)
+          const uint64_t dvs = dv + s * dstage;
+#pragma unroll
           for (int ks = 0; ks < kKRows / 16; ++ks)
-            mma_bf16(tm + 2 * kKRows, sdesc(pa + ks * 2 * kQSlab, kQSlab, 128),
-                     sdesc(va + ks * 256, 128, kKSlab), idO, (jp > 0) || (ks > 0));
-          mma_commit(&bar.pv_done);
+            mma_bf16(tOg, dp + ks * (2 * kQSlab >> 4), dvs + ks * (256 >> 4), idO,
+                     (jp > 0) || (ks > 0));
+          mma_commit(&bar.pv_done[g]);
           mma_commit(&bar.v_empty[s]);
         }
       }
       // every MMA issued has completed before TMEM and shared memory go
-      mma_commit(&bar.drain);
-      mbar_wait(&bar.drain, 0, kDrainPolls);
+      mma_commit(&bar.drain[g]);
+      mbar_wait(&bar.drain[g], 0, kDrainPolls);
     }
-  } else {
+  } else if ((warp >> 2) < nq) {
     // ------------------------------------------------------------- softmax
-    const int r = tid;  // query row within the tile = TMEM lane
-    const uint32_t lrow = tm + ((uint32_t)(warp * 32) << 16);
+    const int g = warp >> 2;
+    const int r = tid & (kQRows - 1);  // query row within the tile = TMEM lane
+    const uint32_t lrow = tm + g * kTileCols + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t tO = lrow + 2 * kKRows;
-    uint8_t* sp = smem + L.p;
+    uint8_t* sp = smem + L.p + g * L.p_tile;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
@@ -271,7 +306,7 @@ gdn_sink_window_kernel(const __grid_constant__ CUtensorMap tm_q,
         ok = false;
         break;
       }
-      if (!__all_sync(~0u, mbar_wait(&bar.s_full[sb], (j >> 1) & 1, P.limit))) {
+      if (!__all_sync(~0u, mbar_wait(&bar.s_full[g][sb], (j >> 1) & 1, P.limit))) {
         if (lane == 0) fail();
         ok = false;
         break;
@@ -283,7 +318,7 @@ gdn_sink_window_kernel(const __grid_constant__ CUtensorMap tm_q,
         tmem_ld16(lrow + sb * kKRows + 16 * c, *reinterpret_cast<float(*)[16]>(s + 16 * c));
       tmem_wait_ld();
       tc_fence_before_sync();
-      mbar_arrive(&bar.s_free[sb]);
+      mbar_arrive(&bar.s_free[g][sb]);
 
       const int t = j % tps;
       const int nvalid = min(kKRows, P.Tc - t * kKRows);
@@ -320,7 +355,7 @@ gdn_sink_window_kernel(const __grid_constant__ CUtensorMap tm_q,
       const float rs = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
       // P and O belong to the previous tile's P V until it completes
       if (j > 0) {
-        if (!__all_sync(~0u, mbar_wait(&bar.pv_done, (j - 1) & 1, P.limit))) {
+        if (!__all_sync(~0u, mbar_wait(&bar.pv_done[g], (j - 1) & 1, P.limit))) {
           if (lane == 0) fail();
           ok = false;
           break;
@@ -346,19 +381,19 @@ gdn_sink_window_kernel(const __grid_constant__ CUtensorMap tm_q,
         reinterpret_cast<uint4*>(sp + sl * kQRows * 16)[r] = pack8_bf16(s + 8 * sl);
       fence_proxy_async_smem();
       tc_fence_before_sync();
-      mbar_arrive(&bar.p_full);
+      mbar_arrive(&bar.p_full[g]);
     }
     if (ok && ntiles > 0 &&
-        !__all_sync(~0u, mbar_wait(&bar.pv_done, (ntiles - 1) & 1, P.limit))) {
+        !__all_sync(~0u, mbar_wait(&bar.pv_done[g], (ntiles - 1) & 1, P.limit))) {
       if (lane == 0) fail();
       ok = false;
     }
-    // all 128 rows agree before the tile is stored
-    ok = named_barrier_and(1, 128, ok);
+    // all 128 rows of the tile agree before it is stored
+    ok = named_barrier_and(1 + g, kQRows, ok);
     if (ok) {
       tc_fence_after_sync();
-      // every S MMA has completed, so the Q buffer takes the output tile
-      uint8_t* so = smem + L.q;
+      // every S MMA has completed, so the tile's Q buffer takes its output
+      uint8_t* so = smem + L.q + g * L.q_tile;
       const float inv = 1.f / l_run;
       for (int c0 = 0; c0 < D; c0 += 16) {
         float o[16];
@@ -370,9 +405,9 @@ gdn_sink_window_kernel(const __grid_constant__ CUtensorMap tm_q,
         reinterpret_cast<uint4*>(so + (c0 / 8 + 1) * kQRows * 16)[r] = pack8_bf16(o + 8);
       }
       fence_proxy_async_smem();
-      named_barrier(1, 128);
-      if (tid == 0) {
-        tma_store_tile(&tm_out, so, q0, h, b);
+      named_barrier(1 + g, kQRows);
+      if (r == 0) {
+        tma_store_tile(&tm_out, so, q0 + g * kQRows, h, b);
         bulk_commit();
         bulk_wait_all();
       }
@@ -380,27 +415,36 @@ gdn_sink_window_kernel(const __grid_constant__ CUtensorMap tm_q,
   }
   tc_fence_before_sync();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after_sync();
     tmem_dealloc(tm, kTmemCols);
   }
 }
 
-cudaError_t set_attr_once(int smem_bytes) {
+template <int NK>
+cudaError_t launch_nk(dim3 grid, cudaStream_t stream, const CUtensorMap& mq, const CUtensorMap& mk,
+                      const CUtensorMap& mv, const CUtensorMap& mkc, const CUtensorMap& mvc,
+                      const CUtensorMap& mo, const SwaParams& P) {
+  // opt in to the dynamic shared memory once per device
   constexpr int kMaxDev = 64;
   static std::mutex mu;
-  static int done[kMaxDev] = {};
+  static bool done[kMaxDev] = {};
+  const int bytes = (int)swa_layout(16 * NK).total;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  std::lock_guard<std::mutex> lock(mu);
-  if (dev >= 0 && dev < kMaxDev && done[dev] >= smem_bytes) return cudaSuccess;
-  // the largest layout (D = 128) once, so every D after it is covered
-  const int bytes = (int)swa_layout(128).total;
-  e = cudaFuncSetAttribute(gdn_sink_window_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess && dev >= 0 && dev < kMaxDev) done[dev] = bytes;
-  (void)smem_bytes;
-  return e;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 0 || dev >= kMaxDev || !done[dev]) {
+      e = cudaFuncSetAttribute(gdn_sink_window_kernel<NK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               bytes);
+      if (e != cudaSuccess) return e;
+      if (dev >= 0 && dev < kMaxDev) done[dev] = true;
+    }
+  }
+  ProfileScope ps(stream, kKernSinkWindow);
+  gdn_sink_window_kernel<NK><<<grid, kThreads, bytes, stream>>>(mq, mk, mv, mkc, mvc, mo, P);
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -435,14 +479,20 @@ cudaError_t launch_sink_window(const SwaCall& c) {
       !make_tile_map(&mvc, c.v_cache, c.B * P.nslot, c.Tc, c.H, c.D, kKRows) ||
       !make_tile_map(&mo, c.out, c.B, c.Tc, c.H, c.D, kQRows))
     return cudaErrorInvalidValue;
-  const SwaLayout L = swa_layout(c.D);
-  cudaError_t e = set_attr_once((int)L.total);
-  if (e != cudaSuccess) return e;
-  const dim3 grid((c.Tc + kQRows - 1) / kQRows, c.B * c.H);
-  {
-    ProfileScope ps(c.stream, kKernSinkWindow);
-    gdn_sink_window_kernel<<<grid, kThreads, L.total, c.stream>>>(mq, mk, mv, mkc, mvc, mo, P);
+  const dim3 grid((c.Tc + kQTiles * kQRows - 1) / (kQTiles * kQRows), c.B * c.H);
+  cudaError_t e = cudaSuccess;
+  switch (c.D / 16) {
+    case 1: e = launch_nk<1>(grid, c.stream, mq, mk, mv, mkc, mvc, mo, P); break;
+    case 2: e = launch_nk<2>(grid, c.stream, mq, mk, mv, mkc, mvc, mo, P); break;
+    case 3: e = launch_nk<3>(grid, c.stream, mq, mk, mv, mkc, mvc, mo, P); break;
+    case 4: e = launch_nk<4>(grid, c.stream, mq, mk, mv, mkc, mvc, mo, P); break;
+    case 5: e = launch_nk<5>(grid, c.stream, mq, mk, mv, mkc, mvc, mo, P); break;
+    case 6: e = launch_nk<6>(grid, c.stream, mq, mk, mv, mkc, mvc, mo, P); break;
+    case 7: e = launch_nk<7>(grid, c.stream, mq, mk, mv, mkc, mvc, mo, P); break;
+    case 8: e = launch_nk<8>(grid, c.stream, mq, mk, mv, mkc, mvc, mo, P); break;
+    default: return cudaErrorInvalidValue;
   }
+  if (e != cudaSuccess) return e;
   e = cudaGetLastError();
   if (e == cudaSuccess) count_launches(1);
   return e;
