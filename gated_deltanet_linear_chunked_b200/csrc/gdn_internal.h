@@ -113,6 +113,9 @@ cudaError_t launch_backward(const BwdCall& c, void* workspace);
 // lands in shared memory in the [slab][token][8] core-matrix layout.
 bool make_tile_map(CUtensorMap* m, const void* base, int nb, int T, int H, int D, int box_rows);
 
+// Streaming multiprocessors of the current device (cached per device).
+int num_sms();
+
 // One sink + sliding-window attention call, after validation.
 constexpr int kSwaMaxSeg = 16;  // n_sink + window at most
 struct SwaCall {

@@ -65,8 +65,39 @@ constexpr uint32_t kMinSmem = 116 * 1024;      // more than half an SM: one CTA 
 constexpr float kRescaleLog2 = 8.f;            // headroom of the running maximum
 constexpr long long kDrainPolls = 1LL << 40;   // drains are bounded by the 2 s timer
 
+// 2^x for a pair of x <= 2^8 on the FMA pipe, so that the special-function
+// unit's ex2 is not the only source of exponentials: Cody and Waite's range
+// reduction x = n + f (n = round(x) by adding and subtracting 1.5 * 2^23, f in
+// [-1/2, 1/2]) with 2^f from a degree-3 polynomial whose coefficients were
+// fitted here to 2^f on [-1/2, 1/2] by weighted least squares in relative
+// error (Lawson's iteration); its largest relative error is 7.5e-5, far under
+// the bf16 rounding of P.  2^n enters by adding n to the exponent field.
+// Inputs are clamped at -125 (2^-125 stands for 0, as ex2 gives for -inf).
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  const uint64_t xc = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t magic = f2_pack(12582912.f, 12582912.f);
+  const uint64_t t = f2_add(xc, magic);                        // n in the low bits
+  const uint64_t n = f2_add(t, f2_pack(-12582912.f, -12582912.f));
+  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), xc);       // x - n
+  uint64_t p = f2_fma(f2_pack(0.0551716648f, 0.0551716648f), f,
+                      f2_pack(0.2426111251f, 0.2426111251f));
+  p = f2_fma(p, f, f2_pack(0.6932609677f, 0.6932609677f));
+  p = f2_fma(p, f, f2_pack(0.9999280572f, 0.9999280572f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  return f2_pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
+                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
+}
+
 struct SwaParams {
   int Tc, H, D, nslot;
+  // work units: blockIdx.x < pair_units is the pair of query tiles
+  // (bh, blockIdx.x % pairs_per_bh); beyond, each later pair is split into
+  // two single-tile units (fewer query rows in the last wave of CTAs)
+  int pairs_per_bh, pair_units;
   int nseg, tiles_per_seg;
   int seg_slot[kSwaMaxSeg];  // cache slot of each visible chunk; -1: this chunk (the inputs)
   int append_slot;           // cache slot this chunk is written to
@@ -121,9 +152,20 @@ gdn_sink_window_kernel(const __grid_constant__ CUtensorMap tm_q,
   const SwaLayout L = swa_layout(D);
   SwaBars& bar = *reinterpret_cast<SwaBars*>(smem + L.bars);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int pair = blockIdx.x, bh = blockIdx.y, b = bh / P.H, h = bh - b * P.H;
-  const int q0 = pair * kQTiles * kQRows, tps = P.tiles_per_seg;
-  const int nq = min(kQTiles, (P.Tc - q0 + kQRows - 1) / kQRows);  // query tiles present
+  int pair_index, q0, nq;  // query tiles present: nq of 128 rows from row q0
+  if ((int)blockIdx.x < P.pair_units) {
+    pair_index = blockIdx.x;
+    q0 = (pair_index % P.pairs_per_bh) * kQTiles * kQRows;
+    nq = min(kQTiles, (P.Tc - q0 + kQRows - 1) / kQRows);
+  } else {
+    const int u = blockIdx.x - P.pair_units;
+    pair_index = P.pair_units + u / kQTiles;
+    q0 = (pair_index % P.pairs_per_bh) * kQTiles * kQRows + (u % kQTiles) * kQRows;
+    nq = q0 < P.Tc ? 1 : 0;
+  }
+  if (nq == 0) return;  // the missing half of a ragged pair (uniform over the CTA)
+  const int bh = pair_index / P.pairs_per_bh, b = bh / P.H, h = bh - b * P.H;
+  const int tps = P.tiles_per_seg;
   const int ntiles = P.nseg * tps;
   volatile int* abort_flag = &bar.abort;
 
@@ -211,7 +253,7 @@ gdn_sink_window_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_arrive_expect_tx(full(x, st), kKRows * D * 2);
         if (slot < 0) {
           tma_load_tile(stage_ptr(x, st), x ? &tm_v : &tm_k, full(x, st), r0, h, b);
-          if (P.append_slot >= 0 && r0 / (kQTiles * kQRows) == pair) append_row[x][st] = r0;
+          if (P.append_slot >= 0 && r0 >= q0 && r0 < q0 + nq * kQRows) append_row[x][st] = r0;
         } else {
           tma_load_tile(stage_ptr(x, st), x ? &tm_vc : &tm_kc, full(x, st), r0, h, cache_bs + slot);
         }
@@ -345,14 +387,31 @@ gdn_sink_window_kernel(const __grid_constant__ CUtensorMap tm_q,
         alpha = ex2_approx(m_run - m_new);  // 0 on the first tile
         resc = j > 0;
       }
+      // p = 2^(s c - m), two at a time: one pair in four on the FMA pipe,
+      // the rest on the special-function unit; P packed to bf16 as it goes
+      const uint64_t c2 = f2_pack(P.scale_log2, P.scale_log2), nm2 = f2_pack(-m_new, -m_new);
+      uint64_t sum2[4] = {0, 0, 0, 0};  // packed +0.0f pairs
+      uint32_t pk[kKRows / 2];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll
-      for (int i = 0; i < kKRows; ++i) {
-        s[i] = ex2_approx(fmaf(s[i], P.scale_log2, -m_new));
-        acc[i & 7] += s[i];
+      for (int i = 0; i < kKRows; i += 2) {
+        const uint64_t x = f2_fma(f2_pack(s[i], s[i + 1]), c2, nm2);
+        uint64_t p2;
+        if ((i & 7) == 6) {
+          p2 = exp2_poly2(x);
+        } else {
+          float a, c;
+          f2_unpack(x, a, c);
+          p2 = f2_pack(ex2_approx(a), ex2_approx(c));
+        }
+        sum2[(i >> 1) & 3] = f2_add(sum2[(i >> 1) & 3], p2);
+        float a, c;
+        f2_unpack(p2, a, c);
+        pk[i >> 1] = pack_bf16x2(a, c);
       }
-      const float rs = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+      const uint64_t sa = f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3]));
+      float rs0, rs1;
+      f2_unpack(sa, rs0, rs1);
+      const float rs = rs0 + rs1;
       // P and O belong to the previous tile's P V until it completes
       if (j > 0) {
         if (!__all_sync(~0u, mbar_wait(&bar.pv_done[g], (j - 1) & 1, P.limit))) {
@@ -378,7 +437,8 @@ gdn_sink_window_kernel(const __grid_constant__ CUtensorMap tm_q,
       m_run = m_new;
 #pragma unroll
       for (int sl = 0; sl < kKRows / 8; ++sl)
-        reinterpret_cast<uint4*>(sp + sl * kQRows * 16)[r] = pack8_bf16(s + 8 * sl);
+        reinterpret_cast<uint4*>(sp + sl * kQRows * 16)[r] =
+            make_uint4(pk[4 * sl], pk[4 * sl + 1], pk[4 * sl + 2], pk[4 * sl + 3]);
       fence_proxy_async_smem();
       tc_fence_before_sync();
       mbar_arrive(&bar.p_full[g]);
@@ -479,7 +539,16 @@ cudaError_t launch_sink_window(const SwaCall& c) {
       !make_tile_map(&mvc, c.v_cache, c.B * P.nslot, c.Tc, c.H, c.D, kKRows) ||
       !make_tile_map(&mo, c.out, c.B, c.Tc, c.H, c.D, kQRows))
     return cudaErrorInvalidValue;
-  const dim3 grid((c.Tc + kQTiles * kQRows - 1) / (kQTiles * kQRows), c.B * c.H);
+  // one CTA per SM: a pair of query tiles per CTA, except that when the
+  // pairs overfill the first wave by less than half, the overflow's worth of
+  // pairs run as single tiles so that the second wave is half as long
+  P.pairs_per_bh = (c.Tc + kQTiles * kQRows - 1) / (kQTiles * kQRows);
+  const int pairs = P.pairs_per_bh * c.B * c.H;
+  const int sms = num_sms();
+  int split = 0;
+  if (pairs > sms && 2 * (pairs - sms) <= sms) split = pairs - sms;
+  P.pair_units = pairs - split;
+  const dim3 grid(P.pair_units + kQTiles * split);
   cudaError_t e = cudaSuccess;
   switch (c.D / 16) {
     case 1: e = launch_nk<1>(grid, c.stream, mq, mk, mv, mkc, mvc, mo, P); break;

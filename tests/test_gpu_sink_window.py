@@ -10,7 +10,8 @@ exactly as a softmax block does, and after every call checks:
 * that the chunk's k and v landed in its cache slot bit for bit (byte work).
 
 Shapes cover ragged tiles (Tc not a multiple of 64 or 128, Tc = 1), every
-supported head width class, several (n_sink, window) pairs including no sink
+supported head width class, grids whose last pairs of query tiles run as
+single tiles, several (n_sink, window) pairs including no sink
 and a one-chunk window, the full streaming chunk (B1 H20 D112 Tc2640, one
 sink chunk, window 2: 7920 keys from chunk 2 on), a sharp softmax that makes
 the running maximum grow (the rescale path), inputs that are the cache slot
@@ -62,6 +63,11 @@ SMALL = [
     (1, 300, 4, 112, 0, 4, 6),
     (1, 257, 2, 48, 3, 1, 5),
     (2, 640, 2, 96, 1, 3, 5),
+    # pairs of query tiles just above a B200's 148 SMs: the last pairs run as
+    # single tiles (a ragged pair of 128 + 72 rows; a pair whose second tile
+    # is missing)
+    (1, 200, 150, 32, 1, 2, 3),
+    (1, 100, 160, 16, 0, 2, 3),
 ]
 
 
