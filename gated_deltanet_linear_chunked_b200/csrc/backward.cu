@@ -359,9 +359,12 @@ __device__ __forceinline__ void st_io(__nv_bfloat16* p, float x) { *p = __float2
 
 // Sum the partials of every slice and direction for one (b, t, h) row, apply
 // the normalisation's Jacobian, and write dq, dk, dv, dg, dbeta.
+// pab[..][0] holds dL/da (token-serial path: dg = e^g da) or dL/dg itself
+// (chunked path, `pab_is_dg`).
 template <typename IO>
 __global__ void __launch_bounds__(128)
-gdn_bwd_reduce_kernel(BwdArgs A, int ndir, void* dq_, void* dk_, void* dv_, float* dg, float* dbeta) {
+gdn_bwd_reduce_kernel(BwdArgs A, int ndir, void* dq_, void* dk_, void* dv_, float* dg, float* dbeta,
+                      int pab_is_dg) {
   const size_t rows_bth = (size_t)A.B * A.T * A.H;
   const size_t row = blockIdx.x;
   const int tid = threadIdx.x, Dk = A.Dk, Dv = A.Dv;
@@ -417,14 +420,15 @@ gdn_bwd_reduce_kernel(BwdArgs A, int ndir, void* dq_, void* dk_, void* dv_, floa
         da += A.pab[(base + row) * 2];
         db += A.pab[(base + row) * 2 + 1];
       }
-    dg[row] = expf(__ldg(A.g + row)) * da;
+    dg[row] = pab_is_dg ? da : expf(__ldg(A.g + row)) * da;
     dbeta[row] = db;
   }
 }
 
 }  // namespace
 
-size_t bwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, bool bidir) {
+size_t bwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, gdn_dtype dtype, bool bidir) {
+  if (dtype == GDN_BF16 && bwd_chunked_fits(Dk, Dv)) return bwd_chunked_workspace_bytes(B, T, H, Dk, Dv, bidir);
   const size_t ndir = bidir ? 2 : 1, nslice = Dv / kBCols, nblk = (T + kBBlock - 1) / kBBlock;
   const size_t rows = (size_t)B * T * H, ctas = ndir * B * H * nslice;
   return sizeof(float) * (ctas * (nblk + 1) * kBState + ctas * kBBlock * kBState +
@@ -432,6 +436,22 @@ size_t bwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, bool bidir) {
 }
 
 cudaError_t launch_backward(const BwdCall& c, void* workspace) {
+  if (c.dtype == GDN_BF16 && bwd_chunked_fits(c.Dk, c.Dv)) {
+    BwdArgs A = {};
+    A.q = c.q; A.k = c.k; A.v = c.v; A.g = c.g; A.beta = c.beta;
+    A.B = c.B; A.T = c.T; A.H = c.H; A.Dk = c.Dk; A.Dv = c.Dv; A.nslice = 1;
+    cudaError_t e = launch_backward_chunked(c, workspace, &A.pq, &A.pk, &A.pab, &A.dvb);
+    if (e != cudaSuccess) return e;
+    const size_t rows = (size_t)c.B * c.T * c.H;
+    {
+      ProfileScope ps(c.stream, kKernBwdReduce);
+      gdn_bwd_reduce_kernel<__nv_bfloat16><<<(unsigned)rows, 128, 0, c.stream>>>(
+          A, c.bidir ? 2 : 1, c.dq, c.dk, c.dv, c.dg, c.dbeta, 1);
+    }
+    e = cudaGetLastError();
+    if (e == cudaSuccess) count_launches(1);
+    return e;
+  }
   const int ndir = c.bidir ? 2 : 1, nslice = c.Dv / kBCols, nblk = (c.T + kBBlock - 1) / kBBlock;
   const size_t rows = (size_t)c.B * c.T * c.H, ctas = (size_t)ndir * c.B * c.H * nslice;
   BwdArgs A;
@@ -464,7 +484,7 @@ cudaError_t launch_backward(const BwdCall& c, void* workspace) {
     if (e != cudaSuccess) return e;
     ProfileScope ps(c.stream, kKernBwdReduce);
     gdn_bwd_reduce_kernel<float><<<(unsigned)rows, 128, 0, c.stream>>>(A, ndir, c.dq, c.dk, c.dv, c.dg,
-                                                                       c.dbeta);
+                                                                       c.dbeta, 0);
   } else {
     e = cudaFuncSetAttribute(gdn_bwd_scan_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem);
@@ -477,7 +497,7 @@ cudaError_t launch_backward(const BwdCall& c, void* workspace) {
     if (e != cudaSuccess) return e;
     ProfileScope ps(c.stream, kKernBwdReduce);
     gdn_bwd_reduce_kernel<__nv_bfloat16><<<(unsigned)rows, 128, 0, c.stream>>>(A, ndir, c.dq, c.dk, c.dv,
-                                                                               c.dg, c.dbeta);
+                                                                               c.dg, c.dbeta, 0);
   }
   e = cudaGetLastError();
   if (e == cudaSuccess) count_launches(2);

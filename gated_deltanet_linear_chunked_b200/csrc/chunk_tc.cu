@@ -1533,6 +1533,21 @@ int num_sms() {
   return cached[dev];
 }
 
+WsLayout chunk_tc_ws_layout(int Dk, int Dv) {
+  Workspace w;
+  w.layout(Dk, Dv);
+  WsLayout L;
+  L.block_bytes = w.block_bytes;
+  L.off_w = w.off_w;
+  L.off_kt = w.off_kt;
+  L.off_decay = w.off_decay;
+  L.off_g = w.off_g;
+  L.off_ut = w.off_ut;
+  L.off_u = w.off_u;
+  L.off_s = w.off_s;
+  return L;
+}
+
 size_t chunk_tc_workspace_bytes(int B, int T, int H, int Dk, int Dv, bool bidir) {
   const int ndir = bidir ? 2 : 1;
   const size_t tiles = (size_t)ndir * B * H * ((T + kC - 1) / kC);
@@ -1622,6 +1637,10 @@ cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
     launches = 5;
   }
   if (e != cudaSuccess) return e;
+  if (a.skip_output) {
+    count_launches(launches - 1);
+    return e;
+  }
   {
     ProfileScope ps(a.stream, kKernOutput);
     e = launch_pdl(gdn_output_kernel, dim3(std::min(nC * NBH, num_sms())), kOutThreads,

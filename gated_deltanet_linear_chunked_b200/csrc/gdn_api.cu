@@ -392,14 +392,20 @@ gdn_status backward(const void* q, const void* k, const void* v, const float* g,
   }
   unsigned int* err = nullptr;
   void* ws = nullptr;
-  const size_t bytes = bwd_workspace_bytes(B, T, H, Dk, Dv, bidir);
+  const size_t bytes = bwd_workspace_bytes(B, T, H, Dk, Dv, dtype, bidir);
   st = stream_context(dev, s, bytes, &err, &ws);
   if (st != GDN_OK) return st;
+  if (!err && error_word(&err) != cudaSuccess) {
+    cudaGetLastError();
+    return GDN_ERR_CUDA;
+  }
   BwdCall c;
   c.q = q; c.k = k; c.v = v; c.g = g; c.beta = beta; c.state_in = state_in;
   c.d_out = d_out; c.d_state_out = d_state_out;
   c.dq = dq; c.dk = dk; c.dv = dv; c.dg = dg; c.dbeta = dbeta; c.d_state_in = d_state_in;
   c.B = B; c.T = T; c.H = H; c.Dk = Dk; c.Dv = Dv; c.dtype = dtype; c.bidir = bidir; c.stream = s;
+  c.err = err;
+  c.wait_limit = g_wait_limit.load();
   cudaError_t e;
   if (ws) {
     e = launch_backward(c, ws);
@@ -411,7 +417,7 @@ gdn_status backward(const void* q, const void* k, const void* v, const float* g,
       if (e == cudaSuccess) e = f;
     }
   }
-  return finish(s, e, nullptr);
+  return finish(s, e, err);
 }
 gdn_status sink_window(const void* q, const void* k, const void* v, void* k_cache,
                        void* v_cache, void* out, int B, int Tc, int H, int D, int n_sink,
@@ -752,6 +758,7 @@ const char* gdn_kernel_name(int id) {
     case gdn::kKernBwdScan: return "gdn_bwd_scan_kernel";
     case gdn::kKernBwdReduce: return "gdn_bwd_reduce_kernel";
     case gdn::kKernSinkWindow: return "gdn_sink_window_kernel";
+    case gdn::kKernBwdChunk: return "gdn_bwd_chunk_kernel";
   }
   return "unknown";
 }

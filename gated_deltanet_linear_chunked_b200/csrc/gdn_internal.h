@@ -28,6 +28,7 @@ struct ScanArgs {
   cudaStream_t stream;
   unsigned int* err;       // device error word (bounded waits report here)
   long long wait_limit;    // polls before a bounded wait gives up
+  bool skip_output = false;  // chunked path: stages A and B only (workspace filled, out untouched)
 };
 
 // Kernel ids for the profiling hook.
@@ -40,7 +41,8 @@ enum KernelId : int {
   kKernBwdScan = 5,
   kKernBwdReduce = 6,
   kKernSinkWindow = 7,
-  kNumKernelIds = 8,
+  kKernBwdChunk = 8,
+  kNumKernelIds = 9,
 };
 
 // While profiling is armed, records CUDA events around one launch.
@@ -91,6 +93,15 @@ cudaError_t launch_scan_serial(const ScanArgs& a);
 // output.  `workspace` must hold chunk_tc_workspace_bytes(...) bytes.
 size_t chunk_tc_workspace_bytes(int B, int T, int H, int Dk, int Dv, bool bidir);
 cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace);
+// Layout of one (direction, b*h, chunk) block of the chunked path's
+// workspace (block index ((dir * B*H) + bh) * nC + chunk; rows in time order):
+//   W, K~ [Dk/8][64][8] bf16, decay (fp32 e^{gamma_C}), g [64] fp32,
+//   U~, U [Dv/8][64][8] bf16, S (chunk-start state) [Dv/8][Dk][8] bf16.
+struct WsLayout {
+  size_t block_bytes;
+  uint32_t off_w, off_kt, off_decay, off_g, off_ut, off_u, off_s;
+};
+WsLayout chunk_tc_ws_layout(int Dk, int Dv);
 
 // One backward call, after validation (device pointers).
 struct BwdCall {
@@ -104,9 +115,18 @@ struct BwdCall {
   gdn_dtype dtype;
   bool bidir;
   cudaStream_t stream;
+  unsigned int* err;     // error word of the forward stages' bounded waits
+  long long wait_limit;
 };
-size_t bwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, bool bidir);
+size_t bwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, gdn_dtype dtype, bool bidir);
 cudaError_t launch_backward(const BwdCall& c, void* workspace);
+// bf16 I/O: the chunked backward (forward stages A and B, then one CTA per
+// (b*h, direction) walking the chunks in reverse); returns the partials'
+// addresses in the workspace for the reduction.
+bool bwd_chunked_fits(int Dk, int Dv);  // its shared-memory layout fits (Dk, Dv <= 112)
+size_t bwd_chunked_workspace_bytes(int B, int T, int H, int Dk, int Dv, bool bidir);
+cudaError_t launch_backward_chunked(const BwdCall& c, void* workspace, float** pq, float** pk,
+                                    float** pab, float** dvb);
 
 // A [nb, T, H, D] bf16 tensor viewed as 5-D (8 features, T, D/8 feature
 // slabs, H, nb) so that one box (8 x box_rows tokens x D/8 slabs x 1 x 1)

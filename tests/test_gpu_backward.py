@@ -1,8 +1,9 @@
 """GPU parity of the backward pass: every gradient (q, k, v, g, beta,
 state_in) of L = <out, d_out> + <state_out, d_state_out> against autograd of
 the fp64 definition (oracle/backward.py), at the forward's bar applied to
-each gradient tensor: max |x - ref| / max |ref| <= 1e-4 with fp32 I/O and
-<= 2e-2 with bf16 I/O."""
+each gradient tensor: max |x - ref| / max |ref| <= 1e-4 with fp32 I/O (the
+token-serial kernel) and <= 2e-2 with bf16 I/O (the chunked tensor-core
+kernel)."""
 import numpy as np
 import pytest
 import torch
@@ -69,17 +70,29 @@ def test_backward_sweep(T, D, mode, dtype):
     run_and_check(w, seed=T + D)
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("Dk,Dv", [(32, 96), (128, 16), (48, 64)])
-def test_backward_rectangular(Dk, Dv):
-    w = wl.Workload("bwd_rect", 1, 100, 2, Dk, Dv, "f32", 64, "bidir", ("uniform", -0.5, 0.0),
+def test_backward_rectangular(Dk, Dv, dtype):
+    w = wl.Workload("bwd_rect", 1, 100, 2, Dk, Dv, dtype, 64, "bidir", ("uniform", -0.5, 0.0),
                     ("sigmoid",), ("normal", 0.3), 92000 + Dk + Dv)
     run_and_check(w)
 
 
-def test_backward_zero_state_no_final_gradient():
-    w = wl.Workload("bwd_zero", 1, 90, 3, 64, 64, "f32", 64, "fwd", ("neg_softplus",),
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_backward_zero_state_no_final_gradient(dtype):
+    w = wl.Workload("bwd_zero", 1, 90, 3, 64, 64, dtype, 64, "fwd", ("neg_softplus",),
                     ("sigmoid",), ("zero",), 93000)
     run_and_check(w, with_state=False, with_dS=False)
+
+
+@pytest.mark.parametrize("mode", ["fwd", "bidir"])
+def test_backward_unnormalised_rows_bf16(mode):
+    """q, k rows not unit-norm (N(0,1) rows with rows at 1e-3 and 1e3, rows
+    under the 1e-12 clamp, an all-zero q row and k row): the chunked bf16
+    backward's normalisation and the reduction's Jacobian."""
+    w = wl.Workload("bwd_mixed", 1, 200, 2, 64, 64, "bf16", 64, mode, ("uniform", -0.5, 0.0),
+                    ("sigmoid",), ("normal", 0.3), 94000, qk=("mixed",))
+    run_and_check(w, seed=5)
 
 
 def test_backward_empty_sequence():
