@@ -369,16 +369,19 @@ gdn_sink_window_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int i = 0; i < kKRows; ++i)
           if (i >= nvalid) s[i] = -INFINITY;
       }
-      // row maximum and, below, row sum as eight independent chains each
+      // row maximum: eight independent chains of three-input maxima over
+      // columns 0-23, 24-39, 40-55, then 56-63
+      static_assert(kKRows == 64, "the maximum's column pattern");
       float acc[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] = fmaxf(s[e], s[e + 8]);
+      for (int e = 0; e < 8; ++e) acc[e] = fmax3(s[e], s[e + 8], s[e + 16]);
 #pragma unroll
-      for (int i = 16; i < kKRows; i += 8)
+      for (int i = 24; i + 16 <= 56; i += 16)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = fmaxf(acc[e], s[i + e]);
-      float mx = fmaxf(fmaxf(fmaxf(acc[0], acc[1]), fmaxf(acc[2], acc[3])),
-                       fmaxf(fmaxf(acc[4], acc[5]), fmaxf(acc[6], acc[7])));
+        for (int e = 0; e < 8; ++e) acc[e] = fmax3(acc[e], s[i + e], s[i + 8 + e]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = fmaxf(acc[e], s[56 + e]);
+      float mx = fmax3(fmax3(acc[0], acc[1], acc[2]), fmax3(acc[3], acc[4], acc[5]), fmaxf(acc[6], acc[7]));
       mx *= P.scale_log2;
       float m_new = m_run, alpha = 1.f;
       bool resc = false;

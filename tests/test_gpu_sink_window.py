@@ -98,6 +98,16 @@ def test_sharp_softmax_matches_oracle():
         assert err <= TOL["bf16"], (c, err)
 
 
+def test_extremely_sharp_softmax_matches_oracle():
+    """q ~ N(0, 40^2): scores span hundreds of units of log2, so a row maximum
+    that missed any column would overflow or underflow 2^(s - m)."""
+    w = wl.AttnStream("swa_extreme", 1, 700, 2, 64, 1, 2, 3, seed=78, q_scale=40.0)
+    for c, got, ref in _stream(w):
+        assert np.isfinite(got).all(), c
+        err = max_rel_per_head(got, ref, (0, 2))
+        assert err <= TOL["bf16"], (c, err)
+
+
 def test_inputs_that_are_the_cache_slot():
     """A projection may write k, v straight into the chunk's slot: the call
     then stores the same bytes over themselves and the result is the same."""
