@@ -387,11 +387,11 @@ def kernel_times(lib, step_fn, n, launches_per_step):
     _lib.check(lib.gdn_profile_begin(int(n * max(1, launches_per_step) + 8)), "gdn_profile_begin")
     for i in range(n):
         step_fn(i)
-    kms = (ctypes.c_float * 9)()
-    kn = (ctypes.c_int * 9)()
-    _lib.check(lib.gdn_profile_end(ctypes.addressof(kms), ctypes.addressof(kn), 9), "gdn_profile_end")
+    kms = (ctypes.c_float * 11)()
+    kn = (ctypes.c_int * 11)()
+    _lib.check(lib.gdn_profile_end(ctypes.addressof(kms), ctypes.addressof(kn), 11), "gdn_profile_end")
     kernels = {}
-    for i in range(9):
+    for i in range(11):
         if kn[i]:
             kernels[lib.gdn_kernel_name(i).decode()] = {"launches": kn[i], "ms_per_launch": kms[i] / kn[i]}
     tot = sum(v["ms_per_launch"] for v in kernels.values())

@@ -25,12 +25,18 @@
 // and beta and gam collect the matching row sums (each exponent gam_p - gam_i
 // sends +c to row p and -c to row i); dg_p is the suffix sum of dgam over the
 // chunk in scan order plus dgam_C.  The forward's stages A and B provide W,
-// K~, U~, U and S0 of every chunk (their workspace); this kernel, one CTA per
-// (b, h, direction), walks the chunks in reverse, recomputes Q^ K^T, K^ K^T
-// and the gates, and runs every product above on tf32 mma.sync (fp32
-// accumulate).  dq^ and dk^ (before the normalisation's Jacobian), dv, dg and
-// dbeta of each direction go to per-direction partials that the reduction
-// kernel of backward.cu sums.
+// K~, U~, U and S0 of every chunk (their workspace).  Only dU and dS0 depend
+// on the chunks after this one, so three kernels share the work:
+//   gdn_bwd_pre_kernel    every chunk at once: X = P^T dO, Y = Q^^T diag(e^gam) dO
+//   gdn_bwd_chain_kernel  per (16 columns of dS, b*h, direction), the chunks in
+//                         reverse: dU = X + K~ dS_e, dS0 = e^{gam_C} dS_e + Y - W^T dU
+//                         (the columns of dS evolve independently; fp32), each
+//                         chunk's dU and dS_e stored
+//   gdn_bwd_grad_kernel   every chunk at once: the other products, from that
+//                         chunk's dU and dS_e
+// all on tf32 mma.sync (fp32 accumulate).  dq^ and dk^ (before the
+// normalisation's Jacobian), dv, dg and dbeta of each direction go to
+// per-direction partials that the reduction kernel of backward.cu sums.
 #include <cuda_bf16.h>
 
 #include "gdn_internal.h"
@@ -91,9 +97,14 @@ struct BcArgs {
   float* d_state_in;         // dL/dS0 of the forward scan, or null
   const uint8_t* ws;         // the forward's workspace
   WsLayout wl;
-  float* dS;                 // [dir][bh][Dk][Dv] running dS_e
+  // per (direction, b*h, time chunk), rows in scan order:
+  float* X;                  // [64][Dv]  P^T dO
+  float* Y;                  // [Dk][Dv]  Q^^T diag(e^gam) dO
+  float* dU;                 // [64][Dv]  dU
+  __nv_bfloat16* dSe;        // [Dk][Dv]  dS_e, the gradient of the chunk's end state
   float *pq, *pk, *pab, *dvb;  // [dir][rows][Dk], [dir][rows][Dk], [dir][rows][2], [dir][rows][Dv]
   int B, T, H, Dk, Dv, nC, NBH;
+  __device__ size_t blk(int dir, int bh, int j) const { return ((size_t)dir * NBH + bh) * nC + j; }
 };
 
 // tf32 operands are fp32 bit patterns whose low 13 mantissa bits the tensor
@@ -141,9 +152,9 @@ __device__ __forceinline__ int tile_col(int e) { return 2 * (threadIdx.x & 3) + 
 // each element to epi(m, n, value).  M % 16 == N % 8 == K % 8 == 0.
 template <class FA, class FB, class FE>
 __device__ __forceinline__ void gemm(int M, int N, int K, FA A, FB B, FE epi) {
-  const int warp = threadIdx.x >> 5;
+  const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const int tn = N >> 4, nt = (M >> 4) * tn;  // 16 x 16 blocks
-  for (int t = warp; t < nt; t += kBcWarps) {
+  for (int t = warp; t < nt; t += nw) {
     const int m0 = (t / tn) << 4, n0 = (t % tn) << 4;
     float d[2][4];
     tile_mma(m0, n0, K, A, B, d);
@@ -236,7 +247,240 @@ __device__ __forceinline__ void solve_upper(const float* A, float (&x)[64]) {
   }
 }
 
-__global__ void __launch_bounds__(kBcThreads, 1) gdn_bwd_chunk_kernel(BcArgs a) {
+// Stage chunk j of (b, h) in direction dir, rows in scan order: gates (zero
+// past T), q^ = q / |q|, k^ likewise (bf16), dO; gam (inclusive prefix sum of
+// g) and e^gam.  Every thread of the CTA takes part; ends with a barrier.
+__device__ void stage_rows(const BcArgs& a, BcSmall& sm, __nv_bfloat16* sQ, __nv_bfloat16* sK,
+                           __nv_bfloat16* sO, int lbk, int lbv, int b, int h, int dir, int j) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
+  const int Dk = a.Dk, Dv = a.Dv, t0 = 64 * j;
+  if (tid < 64) {
+    const int p = tid, t = t0 + (dir == 0 ? p : 63 - p);
+    const bool valid = t < a.T;
+    const size_t r = ((size_t)b * a.T + t) * a.H + h;
+    sm.row[p] = valid ? (int)r : -1;
+    sm.g[p] = valid ? __ldg(a.g + r) : 0.f;
+    sm.beta[p] = valid ? __ldg(a.beta + r) : 0.f;
+    sm.dgam[p] = 0.f;
+    sm.dbeta[p] = 0.f;
+    sm.cK[p] = 0.f;
+  }
+  __syncthreads();
+  const int ck = Dk / 8, cv = Dv / 8;
+  for (int e = tid; e < 64 * (2 * ck + cv); e += blockDim.x) {
+    const int p = e / (2 * ck + cv), c = e - p * (2 * ck + cv), r = sm.row[p];
+    __nv_bfloat16* dst;
+    const __nv_bfloat16* src;
+    if (c < ck) {
+      dst = sQ + p * lbk + 8 * c;
+      src = a.q + (size_t)r * Dk + 8 * c;
+    } else if (c < 2 * ck) {
+      dst = sK + p * lbk + 8 * (c - ck);
+      src = a.k + (size_t)r * Dk + 8 * (c - ck);
+    } else {
+      dst = sO + p * lbv + 8 * (c - 2 * ck);
+      src = a.dout + (size_t)r * Dv + 8 * (c - 2 * ck);
+    }
+    if (r >= 0) cp16(dst, src);
+    else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+  }
+  if (warp == 0) {
+    const float a0 = sm.g[2 * lane], a1 = sm.g[2 * lane + 1];
+    float incl = a0 + a1;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    const float excl = incl - (a0 + a1);
+    sm.gam[2 * lane] = excl + a0;
+    sm.gam[2 * lane + 1] = incl;
+    sm.eg[2 * lane] = expf(excl + a0);
+    sm.eg[2 * lane + 1] = expf(incl);
+  }
+  cp_wait_all();
+  __syncthreads();
+  for (int p = warp; p < 64; p += nw) {
+    float qq = 0.f, kk = 0.f;
+    for (int d = lane; d < Dk; d += 32) {
+      const float qv = bf(sQ[p * lbk + d]), kv = bf(sK[p * lbk + d]);
+      qq = fmaf(qv, qv, qq);
+      kk = fmaf(kv, kv, kk);
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) {
+      qq += __shfl_xor_sync(0xffffffffu, qq, off);
+      kk += __shfl_xor_sync(0xffffffffu, kk, off);
+    }
+    const float rq = 1.f / sqrtf(fmaxf(qq, 1e-12f)), rk = 1.f / sqrtf(fmaxf(kk, 1e-12f));
+    for (int d = lane; d < Dk; d += 32) {
+      sQ[p * lbk + d] = __float2bfloat16_rn(bf(sQ[p * lbk + d]) * rq);
+      sK[p * lbk + d] = __float2bfloat16_rn(bf(sK[p * lbk + d]) * rk);
+    }
+  }
+  __syncthreads();
+}
+
+// ---------------------------------------------------------------- pre pass
+// Every chunk at once: X = P^T dO and Y = Q^^T diag(e^gam) dO, which do not
+// depend on the later chunks.  Shared memory: q^, k^, dO (bf16), P (fp32).
+struct PreLayout {
+  int lbk, lbv;
+  uint32_t q, k, dout, P, small, total;
+  __host__ __device__ PreLayout(int Dk, int Dv) {
+    lbk = Dk + 8;
+    lbv = Dv + 8;
+    uint32_t o = 0;
+    q = o;    o += 64 * lbk * 2;
+    k = o;    o += 64 * lbk * 2;
+    dout = o; o += 64 * lbv * 2;
+    P = o;    o += 64 * kLd64 * 4;
+    small = o; o += sizeof(BcSmall);
+    total = (o + 15) & ~15u;
+  }
+};
+
+__global__ void __launch_bounds__(kBcThreads) gdn_bwd_pre_kernel(BcArgs a) {
+  extern __shared__ __align__(16) uint8_t bp_raw[];
+  const int Dk = a.Dk, Dv = a.Dv;
+  const PreLayout L(Dk, Dv);
+  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(bp_raw + L.q);
+  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(bp_raw + L.k);
+  __nv_bfloat16* sO = reinterpret_cast<__nv_bfloat16*>(bp_raw + L.dout);
+  float* sP = reinterpret_cast<float*>(bp_raw + L.P);
+  BcSmall& sm = *reinterpret_cast<BcSmall*>(bp_raw + L.small);
+  const int j = blockIdx.x, bh = blockIdx.y, dir = blockIdx.z;
+  const int b = bh / a.H, h = bh - b * a.H;
+  const int lbk = L.lbk, lbv = L.lbv;
+  stage_rows(a, sm, sQ, sK, sO, lbk, lbv, b, h, dir, j);
+  auto Qh = [&](int p, int d) { return bf(sQ[p * lbk + d]); };
+  auto Kh = [&](int p, int d) { return bf(sK[p * lbk + d]); };
+  auto dO = [&](int p, int c) { return bf(sO[p * lbv + c]); };
+  gemm(64, 64, Dk, Qh, [&](int kk, int n) { return Kh(n, kk); },
+       [&](int m, int n, float v) { sP[m * kLd64 + n] = n <= m ? expf(sm.gam[m] - sm.gam[n]) * v : 0.f; });
+  __syncthreads();
+  const size_t blk = a.blk(dir, bh, j);
+  float* X = a.X + blk * 64 * Dv;
+  float* Y = a.Y + blk * Dk * Dv;
+  gemm(64, Dv, 64, [&](int m, int kk) { return sP[kk * kLd64 + m]; }, dO,
+       [&](int m, int n, float v) { X[m * Dv + n] = v; });
+  gemm(Dk, Dv, 64, [&](int m, int kk) { return Qh(kk, m) * sm.eg[kk]; }, dO,
+       [&](int m, int n, float v) { Y[m * Dv + n] = v; });
+}
+
+// -------------------------------------------------------------- chain pass
+// One CTA per (16 columns of dS, b*h, direction), 128 threads, the chunks in
+// reverse scan order with the next chunk's tiles prefetched (cp.async, two
+// sets): dU = X + K~ dS_e, then dS0 = e^{gam_C} dS_e + Y - W^T dU.  Stores
+// each chunk's dS_e (bf16) and dU (fp32) for the gradient pass.
+constexpr int kChThreads = 128;
+constexpr int kChCols = 16;
+constexpr int kChLd = kChCols + 4;  // fp32 row stride of the 16-column tiles
+struct ChainLayout2 {
+  int lbk;
+  uint32_t kt, w, x, y, set, dS, dU, total;
+  __host__ __device__ ChainLayout2(int Dk) {
+    lbk = Dk + 8;
+    uint32_t o = 0;
+    kt = o; o += 64 * lbk * 2;        // K~ (bf16, scan rows)
+    w = o;  o += 64 * lbk * 2;        // W
+    x = o;  o += 64 * kChLd * 4;      // X columns
+    y = o;  o += Dk * kChLd * 4;      // Y columns
+    set = o;                          // one prefetch set
+    o *= 2;
+    dS = o; o += Dk * kChLd * 4;      // the running dS columns (fp32)
+    dU = o; o += 64 * kChLd * 4;
+    total = o;
+  }
+};
+
+__global__ void __launch_bounds__(kChThreads) gdn_bwd_chain_kernel(BcArgs a) {
+  extern __shared__ __align__(16) uint8_t bch_raw[];
+  const int Dk = a.Dk, Dv = a.Dv;
+  const ChainLayout2 L(Dk);
+  const int sl = blockIdx.x, bh = blockIdx.y, dir = blockIdx.z, c0 = kChCols * sl;
+  const int tid = threadIdx.x, lbk = L.lbk;
+  float* sdS = reinterpret_cast<float*>(bch_raw + L.dS);
+  float* sdU = reinterpret_cast<float*>(bch_raw + L.dU);
+  for (int e = tid; e < Dk * kChCols; e += kChThreads) {
+    const int d = e / kChCols, c = e - d * kChCols;
+    sdS[d * kChLd + c] = (dir == 0 && a.d_state_out)
+                             ? a.d_state_out[((size_t)bh * Dk + d) * Dv + c0 + c]
+                             : 0.f;
+  }
+  auto chunk_of = [&](int step) { return dir == 0 ? a.nC - 1 - step : step; };
+  auto prefetch = [&](int step, int set) {
+    uint8_t* base = bch_raw + set * L.set;
+    const int j = chunk_of(step);
+    const size_t blk = a.blk(dir, bh, j);
+    const uint8_t* wsb = a.ws + blk * a.wl.block_bytes;
+    const int ck = Dk / 8;
+    for (int e = tid; e < 64 * 2 * ck; e += kChThreads) {  // K~, W: [slab][time row][8] -> [scan row]
+      const int s2 = e >> 6, t = e & 63, p = dir == 0 ? t : 63 - t;
+      if (s2 < ck) cp16(base + L.kt + 2 * (p * lbk + 8 * s2), wsb + a.wl.off_kt + 16 * (s2 * 64 + t));
+      else cp16(base + L.w + 2 * (p * lbk + 8 * (s2 - ck)), wsb + a.wl.off_w + 16 * ((s2 - ck) * 64 + t));
+    }
+    const float* X = a.X + blk * 64 * Dv + c0;
+    const float* Y = a.Y + blk * Dk * Dv + c0;
+    for (int e = tid; e < (64 + Dk) * 4; e += kChThreads) {  // 16 fp32 columns = 4 x 16 B per row
+      const int r = e >> 2, q4 = e & 3;
+      if (r < 64) cp16(base + L.x + 4 * (r * kChLd + 4 * q4), X + (size_t)r * Dv + 4 * q4);
+      else cp16(base + L.y + 4 * ((r - 64) * kChLd + 4 * q4), Y + (size_t)(r - 64) * Dv + 4 * q4);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  prefetch(0, 0);
+  for (int step = 0; step < a.nC; ++step) {
+    const int set = step & 1, j = chunk_of(step);
+    if (step + 1 < a.nC) {
+      prefetch(step + 1, set ^ 1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      cp_wait_all();
+    }
+    __syncthreads();
+    uint8_t* base = bch_raw + set * L.set;
+    const __nv_bfloat16* sKt = reinterpret_cast<const __nv_bfloat16*>(base + L.kt);
+    const __nv_bfloat16* sW = reinterpret_cast<const __nv_bfloat16*>(base + L.w);
+    const float* sX = reinterpret_cast<const float*>(base + L.x);
+    const float* sY = reinterpret_cast<const float*>(base + L.y);
+    const size_t blk = a.blk(dir, bh, j);
+    const float eC =
+        *reinterpret_cast<const float*>(a.ws + blk * a.wl.block_bytes + a.wl.off_decay);
+    // dS_e of this chunk, for the gradient pass
+    __nv_bfloat16* dSe = a.dSe + blk * Dk * Dv + c0;
+    for (int e = tid; e < Dk * kChCols / 2; e += kChThreads) {
+      const int d = e / (kChCols / 2), c = 2 * (e - d * (kChCols / 2));
+      *reinterpret_cast<__nv_bfloat162*>(dSe + (size_t)d * Dv + c) =
+          __floats2bfloat162_rn(sdS[d * kChLd + c], sdS[d * kChLd + c + 1]);
+    }
+    // dU = X + K~ dS_e
+    gemm(64, kChCols, Dk, [&](int m, int kk) { return bf(sKt[m * lbk + kk]); },
+         [&](int kk, int n) { return sdS[kk * kChLd + n]; },
+         [&](int m, int n, float v) { sdU[m * kChLd + n] = sX[m * kChLd + n] + v; });
+    __syncthreads();
+    float* dUg = a.dU + blk * 64 * Dv + c0;
+    for (int e = tid; e < 64 * kChCols; e += kChThreads) {
+      const int m = e / kChCols, c = e - m * kChCols;
+      dUg[(size_t)m * Dv + c] = sdU[m * kChLd + c];
+    }
+    // dS0 = e^{gam_C} dS_e + Y - W^T dU  (in place: each element by its owner)
+    gemm(Dk, kChCols, 64, [&](int m, int kk) { return -bf(sW[kk * lbk + m]); },
+         [&](int kk, int n) { return sdU[kk * kChLd + n]; },
+         [&](int m, int n, float v) { sdS[m * kChLd + n] = fmaf(eC, sdS[m * kChLd + n], sY[m * kChLd + n] + v); });
+    __syncthreads();
+  }
+  if (dir == 0 && a.d_state_in)
+    for (int e = tid; e < Dk * kChCols; e += kChThreads) {
+      const int d = e / kChCols, c = e - d * kChCols;
+      a.d_state_in[((size_t)bh * Dk + d) * Dv + c0 + c] = sdS[d * kChLd + c];
+    }
+}
+
+// ----------------------------------------------------------- gradient pass
+// Every chunk at once (one CTA per (chunk, b*h, direction)), from the
+// chunk's dU and dS_e: every product but the chain's.
+__global__ void __launch_bounds__(kBcThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   extern __shared__ __align__(16) uint8_t bc_raw[];
   const int Dk = a.Dk, Dv = a.Dv;
   const BcLayout L(Dk, Dv);
@@ -256,119 +500,49 @@ __global__ void __launch_bounds__(kBcThreads, 1) gdn_bwd_chunk_kernel(BcArgs a) 
   BcSmall& sm = *reinterpret_cast<BcSmall*>(bc_raw + L.small);
   const int lbk = L.lbk, lbv = L.lbv, ldk = L.ldk, ldv = L.ldv;
 
-  const int bh = blockIdx.x, dir = blockIdx.y;
+  const int j = blockIdx.x, bh = blockIdx.y, dir = blockIdx.z;
   const int b = bh / a.H, h = bh - b * a.H;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const size_t rows_bth = (size_t)a.B * a.T * a.H;
-  float* dS = a.dS + ((size_t)dir * a.NBH + bh) * Dk * Dv;
   float* pq = a.pq + (size_t)dir * rows_bth * Dk;
   float* pk = a.pk + (size_t)dir * rows_bth * Dk;
   float* pab = a.pab + (size_t)dir * rows_bth * 2;
   float* dvb = a.dvb + (size_t)dir * rows_bth * Dv;
 
-  // dS_e of the last chunk walked first: the final state's gradient (forward
-  // scan) or zero (the reverse scan's final state is not an output)
-  for (int e = tid; e < Dk * Dv; e += kBcThreads)
-    dS[e] = (dir == 0 && a.d_state_out) ? a.d_state_out[(size_t)bh * Dk * Dv + e] : 0.f;
-  __syncthreads();
+  {
+    // scan position p is time row p (forward) or 63 - p (reverse) of the tile
+    const size_t bi = a.blk(dir, bh, j);
+    const uint8_t* blk = a.ws + bi * a.wl.block_bytes;
 
-  for (int step = 0; step < a.nC; ++step) {
-    // chunks in reverse scan order: time chunk j; scan position p is time
-    // row p (forward) or 63 - p (reverse) of the tile
-    const int j = dir == 0 ? a.nC - 1 - step : step;
-    const int t0 = 64 * j;
-    const uint8_t* blk = a.ws + (((size_t)dir * a.NBH + bh) * a.nC + j) * a.wl.block_bytes;
-
-    // ---- stage the chunk
-    if (tid < 64) {
-      const int p = tid, t = t0 + (dir == 0 ? p : 63 - p);
-      const bool valid = t < a.T;
-      const size_t r = ((size_t)b * a.T + t) * a.H + h;
-      sm.row[p] = valid ? (int)r : -1;
-      sm.g[p] = valid ? __ldg(a.g + r) : 0.f;
-      sm.beta[p] = valid ? __ldg(a.beta + r) : 0.f;
-      sm.dgam[p] = 0.f;
-      sm.dbeta[p] = 0.f;
-      sm.cK[p] = 0.f;
-    }
-    __syncthreads();
+    // ---- stage the chunk: rows, then W, U~, U, S0 (workspace), dU and dS_e
+    stage_rows(a, sm, sQ, sK, sO, lbk, lbv, b, h, dir, j);
     {
-      // q, k, dO rows (zero past T); W, K~, U tiles and S0 from the workspace
       const int ck = Dk / 8, cv = Dv / 8;
-      for (int e = tid; e < 64 * (2 * ck + cv); e += kBcThreads) {
-        const int p = e / (2 * ck + cv), c = e - p * (2 * ck + cv), r = sm.row[p];
-        __nv_bfloat16* dst;
-        const __nv_bfloat16* src;
-        if (c < ck) {
-          dst = sQ + p * lbk + 8 * c;
-          src = a.q + (size_t)r * Dk + 8 * c;
-        } else if (c < 2 * ck) {
-          dst = sK + p * lbk + 8 * (c - ck);
-          src = a.k + (size_t)r * Dk + 8 * (c - ck);
+      for (int e = tid; e < 64 * (ck + 2 * cv); e += kBcThreads) {  // [slab][time row][8] -> [scan row]
+        const int s2 = e >> 6, t = e & 63, p = dir == 0 ? t : 63 - t;
+        if (s2 < ck) {
+          cp16(sW + p * lbk + 8 * s2, blk + a.wl.off_w + 16 * (s2 * 64 + t));
+        } else if (s2 < ck + cv) {
+          cp16(sKU + p * lbv + 8 * (s2 - ck), blk + a.wl.off_ut + 16 * ((s2 - ck) * 64 + t));
         } else {
-          dst = sO + p * lbv + 8 * (c - 2 * ck);
-          src = a.dout + (size_t)r * Dv + 8 * (c - 2 * ck);
-        }
-        if (r >= 0) cp16(dst, src);
-        else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-      }
-      // [slab][time row][8] -> [scan row][8 slab ..]
-      for (int e = tid; e < 64 * (2 * ck + cv); e += kBcThreads) {
-        const int sl = e >> 6, t = e & 63, p = dir == 0 ? t : 63 - t;
-        if (sl < ck) {
-          cp16(sW + p * lbk + 8 * sl, blk + a.wl.off_w + 16 * (sl * 64 + t));
-        } else if (sl < 2 * ck) {
-          cp16(sKU + p * lbk + 8 * (sl - ck), blk + a.wl.off_kt + 16 * ((sl - ck) * 64 + t));
-        } else {
-          cp16(sU + p * lbv + 8 * (sl - 2 * ck), blk + a.wl.off_u + 16 * ((sl - 2 * ck) * 64 + t));
+          cp16(sU + p * lbv + 8 * (s2 - ck - cv), blk + a.wl.off_u + 16 * ((s2 - ck - cv) * 64 + t));
         }
       }
       for (int e = tid; e < cv * Dk; e += kBcThreads) {  // S0: [Dv/8][Dk][8] -> [Dk][Dv]
-        const int sl = e / Dk, d = e - sl * Dk;
-        cp16(sS0 + d * lbv + 8 * sl, blk + a.wl.off_s + 16 * (sl * Dk + d));
+        const int s2 = e / Dk, d = e - s2 * Dk;
+        cp16(sS0 + d * lbv + 8 * s2, blk + a.wl.off_s + 16 * (s2 * Dk + d));
       }
-      // dS_e rounded to bf16 for the two products that read it
-      for (int e = tid; e < Dk * Dv / 4; e += kBcThreads) {
-        const int d = (4 * e) / Dv, c = 4 * e - d * Dv;
-        const float4 x = *reinterpret_cast<const float4*>(dS + 4 * e);
-        __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(sdS + d * lbv + c);
-        o[0] = __floats2bfloat162_rn(x.x, x.y);
-        o[1] = __floats2bfloat162_rn(x.z, x.w);
+      const __nv_bfloat16* dSe = a.dSe + bi * Dk * Dv;
+      for (int e = tid; e < Dk * cv; e += kBcThreads) {  // dS_e (bf16) [Dk][Dv]
+        const int d = e / cv, c = e - d * cv;
+        cp16(sdS + d * lbv + 8 * c, dSe + (size_t)d * Dv + 8 * c);
+      }
+      const float* dUg = a.dU + bi * 64 * Dv;
+      for (int e = tid; e < 64 * (Dv / 4); e += kBcThreads) {  // dU (fp32) [64][Dv]
+        const int p = e / (Dv / 4), c = e - p * (Dv / 4);
+        cp16(sdU + p * ldv + 4 * c, dUg + (size_t)p * Dv + 4 * c);
       }
       cp_wait_all();
-    }
-    if (warp == 0) {  // gam = inclusive prefix sum of g in scan order
-      const float a0 = sm.g[2 * lane], a1 = sm.g[2 * lane + 1];
-      float incl = a0 + a1;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += y;
-      }
-      const float excl = incl - (a0 + a1);
-      sm.gam[2 * lane] = excl + a0;
-      sm.gam[2 * lane + 1] = incl;
-      sm.eg[2 * lane] = expf(excl + a0);
-      sm.eg[2 * lane + 1] = expf(incl);
-    }
-    __syncthreads();
-    for (int p = warp; p < 64; p += kBcWarps) {  // q^ = q / |q|, k^ likewise, in place
-      float qq = 0.f, kk = 0.f;
-      for (int d = lane; d < Dk; d += 32) {
-        const float qv = bf(sQ[p * lbk + d]), kv = bf(sK[p * lbk + d]);
-        qq = fmaf(qv, qv, qq);
-        kk = fmaf(kv, kv, kk);
-      }
-#pragma unroll
-      for (int off = 16; off; off >>= 1) {
-        qq += __shfl_xor_sync(0xffffffffu, qq, off);
-        kk += __shfl_xor_sync(0xffffffffu, kk, off);
-      }
-      const float rq = 1.f / sqrtf(fmaxf(qq, 1e-12f)), rk = 1.f / sqrtf(fmaxf(kk, 1e-12f));
-      for (int d = lane; d < Dk; d += 32) {
-        sQ[p * lbk + d] = __float2bfloat16_rn(bf(sQ[p * lbk + d]) * rq);
-        sK[p * lbk + d] = __float2bfloat16_rn(bf(sK[p * lbk + d]) * rk);
-      }
     }
     __syncthreads();
     const float gamC = sm.gam[63], eC = expf(gamC);
@@ -386,11 +560,6 @@ __global__ void __launch_bounds__(kBcThreads, 1) gdn_bwd_chunk_kernel(BcArgs a) 
     });
     __syncthreads();
 
-    // ---- 2. dU = P^T dO + K~ dS_e
-    gemm(64, Dv, 64 + Dk,
-         [&](int m, int kk) { return kk < 64 ? sP[kk * kLd64 + m] : bf(sKU[m * lbk + kk - 64]); },
-         [&](int kk, int n) { return kk < 64 ? dO(kk, n) : bf(sdS[(kk - 64) * lbv + n]); },
-         [&](int m, int n, float v) { sdU[m * ldv + n] = v; });
     // ---- 3. dK~ = U dS_e^T: dk^ starts as e^{gam_C - gam} dK~; c_i = K~_i . dK~_i
     float dk[kMaxBlocks][2][4];
 #pragma unroll
@@ -428,34 +597,19 @@ __global__ void __launch_bounds__(kBcThreads, 1) gdn_bwd_chunk_kernel(BcArgs a) 
     }
     {  // <dS_e, S0> -> dgam_C
       float dot = 0.f;
-      for (int e = tid; e < Dk * Dv / 4; e += kBcThreads) {
-        const int d = (4 * e) / Dv, c = 4 * e - d * Dv;
-        const float4 x = *reinterpret_cast<const float4*>(dS + 4 * e);
-        const __nv_bfloat16* s0 = sS0 + d * lbv + c;
-        dot = fmaf(x.x, bf(s0[0]), fmaf(x.y, bf(s0[1]), fmaf(x.z, bf(s0[2]), fmaf(x.w, bf(s0[3]), dot))));
+      for (int e = tid; e < Dk * Dv; e += kBcThreads) {
+        const int d = e / Dv, c = e - d * Dv;
+        dot = fmaf(bf(sdS[d * lbv + c]), bf(sS0[d * lbv + c]), dot);
       }
 #pragma unroll
       for (int off = 16; off; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
       if (lane == 0) sm.red[warp] = dot;
     }
-    __syncthreads();  // every read of dS_e and of K~ is done
+    __syncthreads();  // every read of dS_e is done
     float dgamC = 0.f;
 #pragma unroll
     for (int w = 0; w < kBcWarps; ++w) dgamC += sm.red[w];
     dgamC *= eC;
-    {  // U~ into K~'s buffer (read in step 12)
-      const int cv = Dv / 8;
-      for (int e = tid; e < 64 * cv; e += kBcThreads) {
-        const int sl = e >> 6, t = e & 63, p = dir == 0 ? t : 63 - t;
-        cp16(sKU + p * lbv + 8 * sl, blk + a.wl.off_ut + 16 * (sl * 64 + t));
-      }
-    }
-
-    // ---- 4. dS0 = e^{gam_C} dS_e + Q^^T diag(e^gam) dO - W^T dU  (in place, fp32)
-    gemm(Dk, Dv, 128,
-         [&](int m, int kk) { return kk < 64 ? Qh(kk, m) * sm.eg[kk] : -bf(sW[(kk - 64) * lbk + m]); },
-         [&](int kk, int n) { return kk < 64 ? dO(kk, n) : sdU[(kk - 64) * ldv + n]; },
-         [&](int m, int n, float v) { dS[m * Dv + n] = fmaf(eC, dS[m * Dv + n], v); });
     // ---- 5. dP = dO U^T -> dQK = M o dP; gam gets dP o P
     gemm_rc(64, 64, Dv, dO, [&](int kk, int n) { return bf(sU[n * lbv + kk]); },
             [&](int m, int n, float v) { return n <= m ? v * sP[m * kLd64 + n] : 0.f; },
@@ -497,7 +651,6 @@ __global__ void __launch_bounds__(kBcThreads, 1) gdn_bwd_chunk_kernel(BcArgs a) 
 #pragma unroll
       for (int p = 0; p < 64; ++p) col[p * ld] = x[p];
     }
-    cp_wait_all();  // U~
     __syncthreads();
     // ---- 11. dk^ += diag(beta e^gam) dX_w;  dv = diag(beta) dX_u;  beta and gam
     //          from the rows of X_w = diag(beta e^gam) K^ and X_u = diag(beta) V
@@ -608,10 +761,7 @@ __global__ void __launch_bounds__(kBcThreads, 1) gdn_bwd_chunk_kernel(BcArgs a) 
         pab[(size_t)r1 * 2 + 1] = sm.dbeta[2 * lane + 1];
       }
     }
-    __syncthreads();
   }
-  if (dir == 0 && a.d_state_in)
-    for (int e = tid; e < Dk * Dv; e += kBcThreads) a.d_state_in[(size_t)bh * Dk * Dv + e] = dS[e];
 }
 
 }  // namespace
@@ -620,18 +770,39 @@ bool bwd_chunked_fits(int Dk, int Dv) {
   return Dk <= 112 && Dv <= 112 && BcLayout(Dk, Dv).total <= 227u * 1024u;
 }
 
+namespace {
+struct BwdScratch {
+  size_t fwd, x, y, du, dse, pq, pk, pab, dvb, total;
+  BwdScratch(int B, int T, int H, int Dk, int Dv, bool bidir) {
+    const size_t ndir = bidir ? 2 : 1, rows = (size_t)B * T * H, NBH = (size_t)B * H;
+    const size_t blocks = ndir * NBH * ((T + 63) / 64);
+    auto al = [](size_t n) { return (n + 255) & ~size_t(255); };
+    size_t o = 0;
+    fwd = o; o += al(chunk_tc_workspace_bytes(B, T, H, Dk, Dv, bidir));
+    x = o;   o += al(blocks * 64 * Dv * 4);
+    y = o;   o += al(blocks * (size_t)Dk * Dv * 4);
+    du = o;  o += al(blocks * 64 * Dv * 4);
+    dse = o; o += al(blocks * (size_t)Dk * Dv * 2);
+    pq = o;  o += al(ndir * rows * Dk * 4);
+    pk = o;  o += al(ndir * rows * Dk * 4);
+    pab = o; o += al(ndir * rows * 2 * 4);
+    dvb = o; o += al(ndir * rows * Dv * 4);
+    total = o;
+  }
+};
+}  // namespace
+
 size_t bwd_chunked_workspace_bytes(int B, int T, int H, int Dk, int Dv, bool bidir) {
-  const size_t ndir = bidir ? 2 : 1, rows = (size_t)B * T * H, NBH = (size_t)B * H;
-  const size_t fwd = (chunk_tc_workspace_bytes(B, T, H, Dk, Dv, bidir) + 255) & ~size_t(255);
-  return fwd + sizeof(float) * ndir * (NBH * Dk * Dv + rows * (2 * Dk + 2 + Dv));
+  return BwdScratch(B, T, H, Dk, Dv, bidir).total;
 }
 
 cudaError_t launch_backward_chunked(const BwdCall& c, void* workspace, float** pq, float** pk,
                                     float** pab, float** dvb) {
   const int ndir = c.bidir ? 2 : 1;
-  const size_t rows = (size_t)c.B * c.T * c.H, NBH = (size_t)c.B * c.H;
+  const size_t NBH = (size_t)c.B * c.H;
+  const int nC = (c.T + 63) / 64;
   uint8_t* base = static_cast<uint8_t*>(workspace);
-  const size_t fwd = (chunk_tc_workspace_bytes(c.B, c.T, c.H, c.Dk, c.Dv, c.bidir) + 255) & ~size_t(255);
+  const BwdScratch W(c.B, c.T, c.H, c.Dk, c.Dv, c.bidir);
   // the forward's stages A and B fill the workspace (W, K~, U~, U, S per chunk)
   ScanArgs f;
   f.q = c.q; f.k = c.k; f.v = c.v; f.g = c.g; f.beta = c.beta;
@@ -639,7 +810,7 @@ cudaError_t launch_backward_chunked(const BwdCall& c, void* workspace, float** p
   f.B = c.B; f.T = c.T; f.H = c.H; f.Dk = c.Dk; f.Dv = c.Dv;
   f.dtype = GDN_BF16; f.chunk = 64; f.bidir = c.bidir; f.gate_logits = false;
   f.stream = c.stream; f.err = c.err; f.wait_limit = c.wait_limit; f.skip_output = true;
-  cudaError_t e = launch_chunk_tc(f, base);
+  cudaError_t e = launch_chunk_tc(f, base + W.fwd);
   if (e != cudaSuccess) return e;
 
   BcArgs a;
@@ -649,31 +820,47 @@ cudaError_t launch_backward_chunked(const BwdCall& c, void* workspace, float** p
   a.dout = static_cast<const __nv_bfloat16*>(c.d_out);
   a.g = c.g; a.beta = c.beta;
   a.d_state_out = c.d_state_out; a.d_state_in = c.d_state_in;
-  a.ws = base;
+  a.ws = base + W.fwd;
   a.wl = chunk_tc_ws_layout(c.Dk, c.Dv);
-  float* w = reinterpret_cast<float*>(base + fwd);
-  a.dS = w;
-  w += ndir * NBH * c.Dk * c.Dv;
-  a.pq = w;
-  w += ndir * rows * c.Dk;
-  a.pk = w;
-  w += ndir * rows * c.Dk;
-  a.pab = w;
-  w += ndir * rows * 2;
-  a.dvb = w;
+  a.X = reinterpret_cast<float*>(base + W.x);
+  a.Y = reinterpret_cast<float*>(base + W.y);
+  a.dU = reinterpret_cast<float*>(base + W.du);
+  a.dSe = reinterpret_cast<__nv_bfloat16*>(base + W.dse);
+  a.pq = reinterpret_cast<float*>(base + W.pq);
+  a.pk = reinterpret_cast<float*>(base + W.pk);
+  a.pab = reinterpret_cast<float*>(base + W.pab);
+  a.dvb = reinterpret_cast<float*>(base + W.dvb);
   a.B = c.B; a.T = c.T; a.H = c.H; a.Dk = c.Dk; a.Dv = c.Dv;
-  a.nC = (c.T + 63) / 64;
+  a.nC = nC;
   a.NBH = (int)NBH;
   *pq = a.pq; *pk = a.pk; *pab = a.pab; *dvb = a.dvb;
-  const int smem = (int)BcLayout(c.Dk, c.Dv).total;
-  e = cudaFuncSetAttribute(gdn_bwd_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
+  const int smem_pre = (int)PreLayout(c.Dk, c.Dv).total;
+  const int smem_chain = (int)ChainLayout2(c.Dk).total;
+  const int smem_grad = (int)BcLayout(c.Dk, c.Dv).total;
+  if ((e = cudaFuncSetAttribute(gdn_bwd_pre_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                smem_pre)) != cudaSuccess ||
+      (e = cudaFuncSetAttribute(gdn_bwd_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                smem_chain)) != cudaSuccess ||
+      (e = cudaFuncSetAttribute(gdn_bwd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                smem_grad)) != cudaSuccess)
+    return e;
+  const dim3 per_chunk((unsigned)nC, (unsigned)NBH, ndir);
   {
     ProfileScope ps(c.stream, kKernBwdChunk);
-    gdn_bwd_chunk_kernel<<<dim3((unsigned)NBH, ndir), kBcThreads, smem, c.stream>>>(a);
+    gdn_bwd_pre_kernel<<<per_chunk, kBcThreads, smem_pre, c.stream>>>(a);
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  {
+    ProfileScope ps(c.stream, kKernBwdChain);
+    gdn_bwd_chain_kernel<<<dim3(c.Dv / kChCols, (unsigned)NBH, ndir), kChThreads, smem_chain, c.stream>>>(a);
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  {
+    ProfileScope ps(c.stream, kKernBwdGrad);
+    gdn_bwd_grad_kernel<<<per_chunk, kBcThreads, smem_grad, c.stream>>>(a);
   }
   e = cudaGetLastError();
-  if (e == cudaSuccess) count_launches(1);
+  if (e == cudaSuccess) count_launches(3);
   return e;
 }
 

@@ -758,7 +758,9 @@ const char* gdn_kernel_name(int id) {
     case gdn::kKernBwdScan: return "gdn_bwd_scan_kernel";
     case gdn::kKernBwdReduce: return "gdn_bwd_reduce_kernel";
     case gdn::kKernSinkWindow: return "gdn_sink_window_kernel";
-    case gdn::kKernBwdChunk: return "gdn_bwd_chunk_kernel";
+    case gdn::kKernBwdChunk: return "gdn_bwd_pre_kernel";
+    case gdn::kKernBwdChain: return "gdn_bwd_chain_kernel";
+    case gdn::kKernBwdGrad: return "gdn_bwd_grad_kernel";
   }
   return "unknown";
 }

@@ -41,8 +41,10 @@ enum KernelId : int {
   kKernBwdScan = 5,
   kKernBwdReduce = 6,
   kKernSinkWindow = 7,
-  kKernBwdChunk = 8,
-  kNumKernelIds = 9,
+  kKernBwdChunk = 8,   // the chunked backward's pre pass
+  kKernBwdChain = 9,
+  kKernBwdGrad = 10,
+  kNumKernelIds = 11,
 };
 
 // While profiling is armed, records CUDA events around one launch.

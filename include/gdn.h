@@ -332,8 +332,9 @@ GDN_API unsigned long long gdn_launch_count(void);
  * events, disarms, and writes for each kernel id i < nids the total
  * milliseconds ms[i] and launch count n[i].  Kernel ids: 0 token-serial scan,
  * 1 stage A (prep), 2 stage B (recurrence, every pass), 3 stage C (output),
- * 4 the time-segment prefix, 5 the backward scan, 6 the backward reduction,
- * 7 the sink + window attention; names from gdn_kernel_name.  Not thread-safe against concurrent calls on other
+ * 4 the time-segment prefix, 5 the token-serial backward, 6 the backward
+ * reduction, 7 the sink + window attention, 8 / 9 / 10 the chunked
+ * backward's pre, chain and gradient passes; names from gdn_kernel_name.  Not thread-safe against concurrent calls on other
  * threads; meant for benchmarks.
  */
 GDN_API gdn_status gdn_profile_begin(int max_launches);
