@@ -40,49 +40,21 @@
 #include <cuda_bf16.h>
 
 #include "gdn_internal.h"
+#include "sm100.cuh"
 
 namespace gdn {
 namespace {
+
+using sm100::ldmatrix_x4;
+using sm100::ldmatrix_x4_trans;
+using sm100::mma_16816;
+using sm100::smem_u32;
 
 constexpr int kBcThreads = 256;
 constexpr int kBcWarps = kBcThreads / 32;
 constexpr int kLd64 = 68;   // fp32 row stride of the 64 x 64 tiles
 constexpr int kLdE = 72;    // bf16 row stride of the 64 x 64 E tile
 constexpr int kMaxBlocks = 4;  // 16 x 16 output blocks per warp of a 64 x Dk product, Dk <= 112
-
-// Shared memory of one CTA, laid out by (Dk, Dv) (byte offsets; all 16-byte
-// aligned).  bf16 tiles have row strides Dk + 8 or Dv + 8, fp32 ones Dk + 4,
-// Dv + 4 or 68.  Rows are scan positions.
-struct BcLayout {
-  int lbk, lbv, ldk, ldv;  // strides: bf16 Dk / Dv tiles, fp32 Dk / Dv tiles
-  uint32_t q, k, dout, w, ktut, u, s0, P, A, E, dU, dW, small, total;
-  __host__ __device__ BcLayout(int Dk, int Dv) {
-    lbk = Dk + 8;
-    lbv = Dv + 8;
-    ldk = Dk + 4;
-    ldv = Dv + 4;
-    const int lbmax = lbk > lbv ? lbk : lbv;
-    uint32_t o = 0;
-    q = o;    o += 64 * lbk * 2;    // q^
-    k = o;    o += 64 * lbk * 2;    // k^
-    dout = o; o += 64 * lbv * 2;    // dO
-    w = o;    o += 64 * lbk * 2;    // W
-    ktut = o; o += 64 * lbmax * 2;  // K~, then U~
-    u = o;    o += 64 * lbv * 2;    // U
-    s0 = o;   o += Dk * lbv * 2;    // S0 [Dk][Dv]
-    P = o;    o += 64 * kLd64 * 4;  // P, then dQK, then dG
-    A = o;    o += 64 * kLd64 * 4;  // A
-    E = o;    o += 64 * kLdE * 2;   // e^{gam_p - gam_i} K^ K^T (i < p), bf16
-    dU = o;   o += 64 * ldv * 4;    // dU, then dX_u
-    dW = o;                          // dS_e (bf16 [Dk][Dv]), then dq^, then dW, then dX_w
-    {
-      const uint32_t a = 64u * ldk * 4, b = (uint32_t)Dk * lbv * 2;
-      o += a > b ? a : b;
-    }
-    small = o; o += 8 * 64 * 4 + 64;
-    total = o;
-  }
-};
 
 struct BcSmall {
   float g[64], beta[64], gam[64], eg[64], dgam[64], dbeta[64], cK[64];
@@ -164,86 +136,17 @@ __device__ __forceinline__ void gemm(int M, int N, int K, FA A, FB B, FE epi) {
       for (int e = 0; e < 4; ++e) epi(m0 + tile_row(e), n0 + 8 * h + tile_col(e), d[h][e]);
   }
 }
-// Row and column sums of a per-element contribution c(m, n, value) over each
-// output tile, reduced across the tile's lanes with shuffles and added to
-// rsum[m] (+) and csum[n] (-) with one shared atomic per row / column; epi
-// runs on every element as in gemm.
-template <class FA, class FB, class FC, class FE>
-__device__ __forceinline__ void gemm_rc(int M, int N, int K, FA A, FB B, FC contrib, FE epi,
-                                        float* rsum, float* csum) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tn = N >> 4, nt = (M >> 4) * tn;  // 16 x 16 blocks
-  for (int t = warp; t < nt; t += kBcWarps) {
-    const int m0 = (t / tn) << 4, nb = (t % tn) << 4;
-    float dd[2][4];
-    tile_mma(m0, nb, K, A, B, dd);
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-    const int n0 = nb + 8 * hh;
-    float d[4], c[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      d[e] = dd[hh][e];
-      c[e] = contrib(m0 + tile_row(e), n0 + tile_col(e), d[e]);
-      epi(m0 + tile_row(e), n0 + tile_col(e), d[e]);
-    }
-    float r0 = c[0] + c[1], r1 = c[2] + c[3];  // rows gq, gq + 8: sum over the 4 lanes of a row
-    r0 += __shfl_xor_sync(0xffffffffu, r0, 1);
-    r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
-    r0 += __shfl_xor_sync(0xffffffffu, r0, 2);
-    r1 += __shfl_xor_sync(0xffffffffu, r1, 2);
-    if (rsum && (lane & 3) == 0) {
-      atomicAdd(&rsum[m0 + tile_row(0)], r0);
-      atomicAdd(&rsum[m0 + tile_row(2)], r1);
-    }
-    if (csum) {
-      float c0 = c[0] + c[2], c1 = c[1] + c[3];  // columns 2 tq, 2 tq + 1: sum over the 8 rows
-#pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        c0 += __shfl_xor_sync(0xffffffffu, c0, off);
-        c1 += __shfl_xor_sync(0xffffffffu, c1, off);
-      }
-      if (lane < 4) {
-        atomicAdd(&csum[n0 + tile_col(0)], -c0);
-        atomicAdd(&csum[n0 + tile_col(1)], -c1);
-      }
-    }
-    }
-  }
-}
-
-// The same for a 64 x N product accumulated in registers: block i of warp w
-// is output block w + 8 i, acc[i][h][e] += epi(m, n, value).
-template <class FA, class FB, class FE>
-__device__ __forceinline__ void gemm_acc(int N, int K, FA A, FB B, float (&acc)[kMaxBlocks][2][4], FE epi) {
-  const int warp = threadIdx.x >> 5;
-  const int tn = N >> 4, nt = 4 * tn;  // 16 x 16 blocks of a 64-row product
-#pragma unroll
-  for (int i = 0; i < kMaxBlocks; ++i) {
-    const int t = warp + kBcWarps * i;
-    if (t < nt) {
-      const int m0 = (t / tn) << 4, n0 = (t % tn) << 4;
-      float d[2][4];
-      tile_mma(m0, n0, K, A, B, d);
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          acc[i][h][e] += epi(m0 + tile_row(e), n0 + 8 * h + tile_col(e), d[h][e]);
-    }
-  }
-}
-
 // x_p = r_p - sum_{t > p} A[t][p] x_t for p = 63 .. 0: (I + A)^T x = r for
-// one column held in registers.  Each sum takes the newest x_t (t = p + 1)
-// last, so row p's accumulation overlaps rows p + 1, p + 2, ...
+// one column held in registers.  Each sum runs in four interleaved
+// accumulators (a warp issues in order, so independent chains are what hides
+// the FMA latency) and takes the newest x_t (t = p + 1) last.
 __device__ __forceinline__ void solve_upper(const float* A, float (&x)[64]) {
 #pragma unroll
   for (int p = 62; p >= 0; --p) {
-    float s = x[p];
+    float s[4] = {x[p], 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int t = 63; t > p; --t) s = fmaf(-A[t * kLd64 + p], x[t], s);
-    x[p] = s;
+    for (int t = 63; t > p; --t) s[(63 - t) & 3] = fmaf(-A[t * kLd64 + p], x[t], s[(63 - t) & 3]);
+    x[p] = (s[0] + s[1]) + (s[2] + s[3]);
   }
 }
 
@@ -479,26 +382,207 @@ __global__ void __launch_bounds__(kChThreads) gdn_bwd_chain_kernel(BcArgs a) {
 
 // ----------------------------------------------------------- gradient pass
 // Every chunk at once (one CTA per (chunk, b*h, direction)), from the
-// chunk's dU and dS_e: every product but the chain's.
+// chunk's dU and dS_e: every product but the chain's.  All product operands
+// are bf16 tiles in shared memory fed to mma.sync.m16n8k16 by ldmatrix (the
+// .trans form where a tile is read transposed); dq^ and dk^ accumulate in
+// registers; the triangular solve runs in fp32 registers per column.
+struct GradLayout {
+  int lbk, lbv;
+  uint32_t q, k, dout, w, ut, u, s0, dse, P, A, E, dU, dW, small, total;
+  __host__ __device__ GradLayout(int Dk, int Dv) {
+    lbk = Dk + 8;
+    lbv = Dv + 8;
+    uint32_t o = 0;
+    q = o;    o += 64 * lbk * 2;    // q^
+    k = o;    o += 64 * lbk * 2;    // k^
+    dout = o; o += 64 * lbv * 2;    // dO
+    w = o;    o += 64 * lbk * 2;    // W
+    ut = o;   o += 64 * lbv * 2;    // U~
+    u = o;    o += 64 * lbv * 2;    // U
+    s0 = o;   o += Dk * lbv * 2;    // S0 [Dk][Dv]
+    dse = o;  o += Dk * lbv * 2;    // dS_e [Dk][Dv]
+    P = o;    o += 64 * kLdE * 2;   // P, then dQK, then dA / dG (bf16)
+    A = o;    o += 64 * kLd64 * 4;  // A (fp32, the solve's matrix)
+    E = o;    o += 64 * kLdE * 2;   // e^{gam_p - gam_i} K^ K^T (i < p), bf16
+    dU = o;   o += 64 * lbv * 2;    // dU, then dX_u (bf16)
+    dW = o;   o += 64 * lbk * 2;    // dW, then dX_w (bf16)
+    small = o; o += sizeof(BcSmall);
+    total = (o + 15) & ~15u;
+  }
+};
+
+// A bf16 matrix in shared memory, row-major with row stride ld (a multiple
+// of 8).  As the A operand (m x k): element (m, k) = p[m ld + k], or
+// p[k ld + m] when read transposed.  As the B operand (k x n): element
+// (k, n) = p[k ld + n], or p[n ld + k] when read transposed.
+struct BMat {
+  const __nv_bfloat16* p;
+  int ld;
+};
+
+// 16 x 16 output block (m0, n0) += A B over k < K (K % 16 == 0).
+template <bool TA, bool TB>
+__device__ __forceinline__ void blk16(int m0, int n0, int K, BMat A, BMat B, float (&d)[2][4]) {
+  const int l = threadIdx.x & 31;
+#pragma unroll 2
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    uint32_t a[4], bb[4];
+    if (TA)
+      ldmatrix_x4_trans(smem_u32(A.p + (k0 + (l & 7) + 8 * (l >> 4)) * A.ld + m0 + 8 * ((l >> 3) & 1)), a);
+    else
+      ldmatrix_x4(smem_u32(A.p + (m0 + (l & 15)) * A.ld + k0 + 8 * (l >> 4)), a);
+    if (TB)
+      ldmatrix_x4(smem_u32(B.p + (n0 + (l & 7) + 8 * (l >> 4)) * B.ld + k0 + 8 * ((l >> 3) & 1)), bb);
+    else
+      ldmatrix_x4_trans(smem_u32(B.p + (k0 + (l & 7) + 8 * ((l >> 3) & 1)) * B.ld + n0 + 8 * (l >> 4)), bb);
+    mma_16816(d[0], a, bb[0], bb[1]);
+    mma_16816(d[1], a, bb[2], bb[3]);
+  }
+}
+__device__ __forceinline__ void zero2(float (&d)[2][4]) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) d[h][0] = d[h][1] = d[h][2] = d[h][3] = 0.f;
+}
+
+// Out (M x N) = A1 B1 (+ A2 B2): warps take 16 x 16 blocks in turn; epi(m, n,
+// value) per element; with rsum / csum, the row / column sums of contrib(m,
+// n, value) over each block are added to rsum[m] (+) and csum[n] (-) with one
+// shared atomic per row / column.
+template <bool TA1, bool TB1, bool TA2, bool TB2, class FC, class FE>
+__device__ __forceinline__ void gemm2(int M, int N, BMat A1, BMat B1, int K1, BMat A2, BMat B2, int K2,
+                                      FC contrib, FE epi, float* rsum, float* csum) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int tn = N >> 4, nt = (M >> 4) * tn;
+  for (int t = warp; t < nt; t += nw) {
+    const int m0 = (t / tn) << 4, nb = (t % tn) << 4;
+    float dd[2][4];
+    zero2(dd);
+    blk16<TA1, TB1>(m0, nb, K1, A1, B1, dd);
+    if (K2) blk16<TA2, TB2>(m0, nb, K2, A2, B2, dd);
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int n0 = nb + 8 * hh;
+      float c[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        c[e] = rsum || csum ? contrib(m0 + tile_row(e), n0 + tile_col(e), dd[hh][e]) : 0.f;
+        epi(m0 + tile_row(e), n0 + tile_col(e), dd[hh][e]);
+      }
+      if (rsum) {
+        float r0 = c[0] + c[1], r1 = c[2] + c[3];
+        r0 += __shfl_xor_sync(0xffffffffu, r0, 1);
+        r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
+        r0 += __shfl_xor_sync(0xffffffffu, r0, 2);
+        r1 += __shfl_xor_sync(0xffffffffu, r1, 2);
+        if ((lane & 3) == 0) {
+          atomicAdd(&rsum[m0 + tile_row(0)], r0);
+          atomicAdd(&rsum[m0 + tile_row(2)], r1);
+        }
+      }
+      if (csum) {
+        float c0 = c[0] + c[2], c1 = c[1] + c[3];
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+          c0 += __shfl_xor_sync(0xffffffffu, c0, off);
+          c1 += __shfl_xor_sync(0xffffffffu, c1, off);
+        }
+        if (lane < 4) {
+          atomicAdd(&csum[n0 + tile_col(0)], -c0);
+          atomicAdd(&csum[n0 + tile_col(1)], -c1);
+        }
+      }
+    }
+  }
+}
+// A 64 x N product accumulated in registers: block i of warp w is output
+// block w + 8 i; acc[i][h][e] += scale(m) * value.
+template <bool TA, bool TB, class FS>
+__device__ __forceinline__ void gemm_acc2(int N, int K, BMat A, BMat B, float (&acc)[kMaxBlocks][2][4],
+                                          FS scale) {
+  const int warp = threadIdx.x >> 5;
+  const int tn = N >> 4, nt = 4 * tn;
+#pragma unroll
+  for (int i = 0; i < kMaxBlocks; ++i) {
+    const int t = warp + kBcWarps * i;
+    if (t < nt) {
+      const int m0 = (t / tn) << 4, n0 = (t % tn) << 4;
+      float d[2][4];
+      zero2(d);
+      blk16<TA, TB>(m0, n0, K, A, B, d);
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[i][h][e] += scale(m0 + tile_row(e)) * d[h][e];
+    }
+  }
+}
+// The register blocks' elements: f(i, h, e, m, n) for every one this thread holds.
+template <class F>
+__device__ __forceinline__ void for_acc(int N, F f) {
+  const int warp = threadIdx.x >> 5;
+  const int tn = N >> 4, nt = 4 * tn;
+#pragma unroll
+  for (int i = 0; i < kMaxBlocks; ++i) {
+    const int t = warp + kBcWarps * i;
+    if (t < nt) {
+      const int m0 = (t / tn) << 4, n0 = (t % tn) << 4;
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) f(i, h, e, m0 + tile_row(e), n0 + 8 * h + tile_col(e));
+    }
+  }
+}
+// Row sums of f(i, h, e, m, n) over the register blocks, added to dst[m].
+template <class F>
+__device__ __forceinline__ void acc_row_sums(int N, float* dst, F f) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tn = N >> 4, nt = 4 * tn;
+#pragma unroll
+  for (int i = 0; i < kMaxBlocks; ++i) {
+    const int t = warp + kBcWarps * i;
+    if (t < nt) {
+      const int m0 = (t / tn) << 4, n0 = (t % tn) << 4;
+      float r0 = 0.f, r1 = 0.f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        r0 += f(i, h, 0, m0 + tile_row(0), n0 + 8 * h + tile_col(0)) +
+              f(i, h, 1, m0 + tile_row(1), n0 + 8 * h + tile_col(1));
+        r1 += f(i, h, 2, m0 + tile_row(2), n0 + 8 * h + tile_col(2)) +
+              f(i, h, 3, m0 + tile_row(3), n0 + 8 * h + tile_col(3));
+      }
+      r0 += __shfl_xor_sync(0xffffffffu, r0, 1);
+      r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
+      r0 += __shfl_xor_sync(0xffffffffu, r0, 2);
+      r1 += __shfl_xor_sync(0xffffffffu, r1, 2);
+      if ((lane & 3) == 0) {
+        atomicAdd(&dst[m0 + tile_row(0)], r0);
+        atomicAdd(&dst[m0 + tile_row(2)], r1);
+      }
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kBcThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
-  extern __shared__ __align__(16) uint8_t bc_raw[];
+  extern __shared__ __align__(16) uint8_t bg_raw[];
   const int Dk = a.Dk, Dv = a.Dv;
-  const BcLayout L(Dk, Dv);
-  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(bc_raw + L.q);
-  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(bc_raw + L.k);
-  __nv_bfloat16* sO = reinterpret_cast<__nv_bfloat16*>(bc_raw + L.dout);
-  __nv_bfloat16* sW = reinterpret_cast<__nv_bfloat16*>(bc_raw + L.w);
-  __nv_bfloat16* sKU = reinterpret_cast<__nv_bfloat16*>(bc_raw + L.ktut);
-  __nv_bfloat16* sU = reinterpret_cast<__nv_bfloat16*>(bc_raw + L.u);
-  __nv_bfloat16* sS0 = reinterpret_cast<__nv_bfloat16*>(bc_raw + L.s0);
-  float* sP = reinterpret_cast<float*>(bc_raw + L.P);
-  float* sA = reinterpret_cast<float*>(bc_raw + L.A);
-  __nv_bfloat16* sE = reinterpret_cast<__nv_bfloat16*>(bc_raw + L.E);
-  float* sdU = reinterpret_cast<float*>(bc_raw + L.dU);
-  float* sdW = reinterpret_cast<float*>(bc_raw + L.dW);
-  __nv_bfloat16* sdS = reinterpret_cast<__nv_bfloat16*>(bc_raw + L.dW);  // steps 2-3 only
-  BcSmall& sm = *reinterpret_cast<BcSmall*>(bc_raw + L.small);
-  const int lbk = L.lbk, lbv = L.lbv, ldk = L.ldk, ldv = L.ldv;
+  const GradLayout L(Dk, Dv);
+  using bf16 = __nv_bfloat16;
+  bf16* sQ = reinterpret_cast<bf16*>(bg_raw + L.q);
+  bf16* sK = reinterpret_cast<bf16*>(bg_raw + L.k);
+  bf16* sO = reinterpret_cast<bf16*>(bg_raw + L.dout);
+  bf16* sW = reinterpret_cast<bf16*>(bg_raw + L.w);
+  bf16* sUt = reinterpret_cast<bf16*>(bg_raw + L.ut);
+  bf16* sU = reinterpret_cast<bf16*>(bg_raw + L.u);
+  bf16* sS0 = reinterpret_cast<bf16*>(bg_raw + L.s0);
+  bf16* sdS = reinterpret_cast<bf16*>(bg_raw + L.dse);
+  bf16* sP = reinterpret_cast<bf16*>(bg_raw + L.P);
+  float* sA = reinterpret_cast<float*>(bg_raw + L.A);
+  bf16* sE = reinterpret_cast<bf16*>(bg_raw + L.E);
+  bf16* sdU = reinterpret_cast<bf16*>(bg_raw + L.dU);
+  bf16* sdW = reinterpret_cast<bf16*>(bg_raw + L.dW);
+  BcSmall& sm = *reinterpret_cast<BcSmall*>(bg_raw + L.small);
+  const int lbk = L.lbk, lbv = L.lbv;
 
   const int j = blockIdx.x, bh = blockIdx.y, dir = blockIdx.z;
   const int b = bh / a.H, h = bh - b * a.H;
@@ -508,258 +592,201 @@ __global__ void __launch_bounds__(kBcThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   float* pk = a.pk + (size_t)dir * rows_bth * Dk;
   float* pab = a.pab + (size_t)dir * rows_bth * 2;
   float* dvb = a.dvb + (size_t)dir * rows_bth * Dv;
+  const size_t bi = a.blk(dir, bh, j);
+  const uint8_t* blk = a.ws + bi * a.wl.block_bytes;
 
+  // ---- stage: rows (q^, k^, dO, gates), then W, U~, U, S0 (workspace),
+  //      dS_e, and dU rounded to bf16
+  stage_rows(a, sm, sQ, sK, sO, lbk, lbv, b, h, dir, j);
   {
-    // scan position p is time row p (forward) or 63 - p (reverse) of the tile
-    const size_t bi = a.blk(dir, bh, j);
-    const uint8_t* blk = a.ws + bi * a.wl.block_bytes;
+    const int ck = Dk / 8, cv = Dv / 8;
+    for (int e = tid; e < 64 * (ck + 2 * cv); e += kBcThreads) {  // [slab][time row][8] -> [scan row]
+      const int s2 = e >> 6, t = e & 63, p = dir == 0 ? t : 63 - t;
+      if (s2 < ck) cp16(sW + p * lbk + 8 * s2, blk + a.wl.off_w + 16 * (s2 * 64 + t));
+      else if (s2 < ck + cv) cp16(sUt + p * lbv + 8 * (s2 - ck), blk + a.wl.off_ut + 16 * ((s2 - ck) * 64 + t));
+      else cp16(sU + p * lbv + 8 * (s2 - ck - cv), blk + a.wl.off_u + 16 * ((s2 - ck - cv) * 64 + t));
+    }
+    for (int e = tid; e < cv * Dk; e += kBcThreads) {  // S0: [Dv/8][Dk][8] -> [Dk][Dv]
+      const int s2 = e / Dk, d = e - s2 * Dk;
+      cp16(sS0 + d * lbv + 8 * s2, blk + a.wl.off_s + 16 * (s2 * Dk + d));
+    }
+    const bf16* dSe = a.dSe + bi * Dk * Dv;
+    for (int e = tid; e < Dk * cv; e += kBcThreads) {
+      const int d = e / cv, c = e - d * cv;
+      cp16(sdS + d * lbv + 8 * c, dSe + (size_t)d * Dv + 8 * c);
+    }
+    const float* dUg = a.dU + bi * 64 * Dv;
+    for (int e = tid; e < 64 * (Dv / 4); e += kBcThreads) {
+      const int p = e / (Dv / 4), c = 4 * (e - p * (Dv / 4));
+      const float4 x = *reinterpret_cast<const float4*>(dUg + (size_t)p * Dv + c);
+      __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(sdU + p * lbv + c);
+      o[0] = __floats2bfloat162_rn(x.x, x.y);
+      o[1] = __floats2bfloat162_rn(x.z, x.w);
+    }
+    cp_wait_all();
+  }
+  __syncthreads();
+  const float gamC = sm.gam[63], eC = expf(gamC);
+  const BMat Q{sQ, lbk}, K{sK, lbk}, O{sO, lbv}, Wm{sW, lbk}, Ut{sUt, lbv}, Um{sU, lbv};
+  const BMat S0{sS0, lbv}, dSm{sdS, lbv}, Pm{sP, kLdE}, dUm{sdU, lbv}, dWm{sdW, lbk};
+  auto none = [](int, int, float) { return 0.f; };
 
-    // ---- stage the chunk: rows, then W, U~, U, S0 (workspace), dU and dS_e
-    stage_rows(a, sm, sQ, sK, sO, lbk, lbv, b, h, dir, j);
-    {
-      const int ck = Dk / 8, cv = Dv / 8;
-      for (int e = tid; e < 64 * (ck + 2 * cv); e += kBcThreads) {  // [slab][time row][8] -> [scan row]
-        const int s2 = e >> 6, t = e & 63, p = dir == 0 ? t : 63 - t;
-        if (s2 < ck) {
-          cp16(sW + p * lbk + 8 * s2, blk + a.wl.off_w + 16 * (s2 * 64 + t));
-        } else if (s2 < ck + cv) {
-          cp16(sKU + p * lbv + 8 * (s2 - ck), blk + a.wl.off_ut + 16 * ((s2 - ck) * 64 + t));
-        } else {
-          cp16(sU + p * lbv + 8 * (s2 - ck - cv), blk + a.wl.off_u + 16 * ((s2 - ck - cv) * 64 + t));
-        }
-      }
-      for (int e = tid; e < cv * Dk; e += kBcThreads) {  // S0: [Dv/8][Dk][8] -> [Dk][Dv]
-        const int s2 = e / Dk, d = e - s2 * Dk;
-        cp16(sS0 + d * lbv + 8 * s2, blk + a.wl.off_s + 16 * (s2 * Dk + d));
-      }
-      const __nv_bfloat16* dSe = a.dSe + bi * Dk * Dv;
-      for (int e = tid; e < Dk * cv; e += kBcThreads) {  // dS_e (bf16) [Dk][Dv]
-        const int d = e / cv, c = e - d * cv;
-        cp16(sdS + d * lbv + 8 * c, dSe + (size_t)d * Dv + 8 * c);
-      }
-      const float* dUg = a.dU + bi * 64 * Dv;
-      for (int e = tid; e < 64 * (Dv / 4); e += kBcThreads) {  // dU (fp32) [64][Dv]
-        const int p = e / (Dv / 4), c = e - p * (Dv / 4);
-        cp16(sdU + p * ldv + 4 * c, dUg + (size_t)p * Dv + 4 * c);
-      }
-      cp_wait_all();
+  // ---- 1. P = M o (Q^ K^T);  A = beta_p E, E = e^{gam_p - gam_i} K^ K^T (i < p)
+  gemm2<false, true, false, true>(64, 64, Q, K, Dk, Q, K, 0, none, [&](int m, int n, float v) {
+    sP[m * kLdE + n] = __float2bfloat16_rn(n <= m ? expf(sm.gam[m] - sm.gam[n]) * v : 0.f);
+  }, nullptr, nullptr);
+  gemm2<false, true, false, true>(64, 64, K, K, Dk, K, K, 0, none, [&](int m, int n, float v) {
+    const float e = n < m ? expf(sm.gam[m] - sm.gam[n]) * v : 0.f;
+    sE[m * kLdE + n] = __float2bfloat16_rn(e);
+    sA[m * kLd64 + n] = sm.beta[m] * e;
+  }, nullptr, nullptr);
+  // ---- 3. dK~ = U dS_e^T: dk^ starts as e^{gam_C - gam} dK~; c_m = k^_m . dk^_m
+  float dk[kMaxBlocks][2][4], dq[kMaxBlocks][2][4];
+#pragma unroll
+  for (int i = 0; i < kMaxBlocks; ++i) {
+    zero2(dk[i]);
+    zero2(dq[i]);
+  }
+  gemm_acc2<false, true>(Dk, Dv, Um, dSm, dk, [&](int m) { return expf(gamC - sm.gam[m]); });
+  acc_row_sums(Dk, sm.cK, [&](int i, int hh, int e, int m, int n) { return bf(sK[m * lbk + n]) * dk[i][hh][e]; });
+  {  // <dS_e, S0> -> dgam_C
+    float dot = 0.f;
+    for (int e = tid; e < Dk * Dv; e += kBcThreads) {
+      const int d = e / Dv, c = e - d * Dv;
+      dot = fmaf(bf(sdS[d * lbv + c]), bf(sS0[d * lbv + c]), dot);
     }
-    __syncthreads();
-    const float gamC = sm.gam[63], eC = expf(gamC);
-    auto Qh = [&](int p, int d) { return bf(sQ[p * lbk + d]); };
-    auto Kh = [&](int p, int d) { return bf(sK[p * lbk + d]); };
-    auto dO = [&](int p, int c) { return bf(sO[p * lbv + c]); };
-
-    // ---- 1. P = M o (Q^ K^T); A = beta_p E, E = e^{gam_p - gam_i} K^ K^T (i < p)
-    gemm(64, 64, Dk, Qh, [&](int kk, int n) { return Kh(n, kk); },
-         [&](int m, int n, float v) { sP[m * kLd64 + n] = n <= m ? expf(sm.gam[m] - sm.gam[n]) * v : 0.f; });
-    gemm(64, 64, Dk, Kh, [&](int kk, int n) { return Kh(n, kk); }, [&](int m, int n, float v) {
-      const float e = n < m ? expf(sm.gam[m] - sm.gam[n]) * v : 0.f;
-      sE[m * kLdE + n] = __float2bfloat16_rn(e);
-      sA[m * kLd64 + n] = sm.beta[m] * e;
-    });
-    __syncthreads();
-
-    // ---- 3. dK~ = U dS_e^T: dk^ starts as e^{gam_C - gam} dK~; c_i = K~_i . dK~_i
-    float dk[kMaxBlocks][2][4];
 #pragma unroll
-    for (int i = 0; i < kMaxBlocks; ++i)
+    for (int off = 16; off; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+    if (lane == 0) sm.red[warp] = dot;
+  }
+  __syncthreads();  // P and A, E complete; every read of dS_e done
+  float dgamC = 0.f;
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) dk[i][hh][0] = dk[i][hh][1] = dk[i][hh][2] = dk[i][hh][3] = 0.f;
-    gemm_acc(Dk, Dv, [&](int m, int kk) { return bf(sU[m * lbv + kk]); },
-             [&](int kk, int n) { return bf(sdS[n * lbv + kk]); }, dk,
-             [&](int m, int, float v) { return expf(gamC - sm.gam[m]) * v; });
-    {  // c_m = K~_m . dK~_m = k^_m . dk^_m so far (K~ = e^{gam_C - gam} K^), per block row
-      const int tn = Dk >> 4, nt = 4 * tn;
+  for (int w = 0; w < kBcWarps; ++w) dgamC += sm.red[w];
+  dgamC *= eC;
+  // ---- 5. dP = dO U^T -> dQK = M o dP (in place of P); gam gets dP o P
+  gemm2<false, true, false, true>(64, 64, O, Um, Dv, O, Um, 0,
+      [&](int m, int n, float v) { return n <= m ? v * bf(sP[m * kLdE + n]) : 0.f; },
+      [&](int m, int n, float v) {
+        sP[m * kLdE + n] = __float2bfloat16_rn(n <= m ? expf(sm.gam[m] - sm.gam[n]) * v : 0.f);
+      },
+      sm.dgam, sm.dgam);
+  // ---- 6. Z = diag(e^gam) dO S0^T -> dq^; gam_p gets q^_p . Z_p
+  gemm_acc2<false, true>(Dk, Dv, O, S0, dq, [&](int m) { return sm.eg[m]; });
+  acc_row_sums(Dk, sm.dgam, [&](int i, int hh, int e, int m, int n) { return bf(sQ[m * lbk + n]) * dq[i][hh][e]; });
+  __syncthreads();  // dQK complete
+  // ---- 7. dq^ += dQK K^;  8. dk^ += dQK^T Q^
+  gemm_acc2<false, false>(Dk, 64, Pm, K, dq, [](int) { return 1.f; });
+  gemm_acc2<true, false>(Dk, 64, Pm, Q, dk, [](int) { return 1.f; });
+  for_acc(Dk, [&](int i, int hh, int e, int m, int n) {
+    if (sm.row[m] >= 0) pq[(size_t)sm.row[m] * Dk + n] = dq[i][hh][e];
+  });
+  // ---- 9. dW = -dU S0^T
+  gemm2<false, true, false, true>(64, Dk, dUm, S0, Dv, dUm, S0, 0, none,
+      [&](int m, int n, float v) { sdW[m * lbk + n] = __float2bfloat16_rn(-v); }, nullptr, nullptr);
+  __syncthreads();
+  // ---- 10. [dX_w | dX_u] solves (I + A)^T X = [dW | dU], a column per thread
+  for (int c = tid; c < Dk + Dv; c += kBcThreads) {
+    bf16* col = c < Dk ? sdW + c : sdU + (c - Dk);
+    const int ld = c < Dk ? lbk : lbv;
+    float x[64];
 #pragma unroll
-      for (int i = 0; i < kMaxBlocks; ++i) {
-        const int t = warp + kBcWarps * i;
-        if (t < nt) {
-          const int m0 = (t / tn) << 4, n0 = (t % tn) << 4;
-          float r0 = 0.f, r1 = 0.f;
+    for (int p = 0; p < 64; ++p) x[p] = bf(col[p * ld]);
+    solve_upper(sA, x);
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            r0 += Kh(m0 + tile_row(0), n0 + 8 * hh + tile_col(0)) * dk[i][hh][0] +
-                  Kh(m0 + tile_row(1), n0 + 8 * hh + tile_col(1)) * dk[i][hh][1];
-            r1 += Kh(m0 + tile_row(2), n0 + 8 * hh + tile_col(2)) * dk[i][hh][2] +
-                  Kh(m0 + tile_row(3), n0 + 8 * hh + tile_col(3)) * dk[i][hh][3];
-          }
-          r0 += __shfl_xor_sync(0xffffffffu, r0, 1);
-          r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
-          r0 += __shfl_xor_sync(0xffffffffu, r0, 2);
-          r1 += __shfl_xor_sync(0xffffffffu, r1, 2);
-          if ((lane & 3) == 0) {
-            atomicAdd(&sm.cK[m0 + tile_row(0)], r0);
-            atomicAdd(&sm.cK[m0 + tile_row(2)], r1);
-          }
-        }
-      }
+    for (int p = 0; p < 64; ++p) col[p * ld] = __float2bfloat16_rn(x[p]);
+  }
+  __syncthreads();
+  // ---- 11. dk^ += diag(beta e^gam) dX_w;  dv = diag(beta) dX_u;  beta and gam
+  //          from the rows of X_w = diag(beta e^gam) K^ and X_u = diag(beta) V
+  for_acc(Dk, [&](int i, int hh, int e, int m, int n) {
+    dk[i][hh][e] = fmaf(sm.beta[m] * sm.eg[m], bf(sdW[m * lbk + n]), dk[i][hh][e]);
+  });
+  // v of this warp's rows, every load issued before any is used
+  float vreg[64 / kBcWarps][4];
+#pragma unroll
+  for (int i = 0; i < 64 / kBcWarps; ++i) {
+    const int r = sm.row[warp + kBcWarps * i];
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+      const int c = lane + 32 * q4;
+      vreg[i][q4] = (r >= 0 && c < Dv) ? __bfloat162float(__ldg(a.v + (size_t)r * Dv + c)) : 0.f;
     }
-    {  // <dS_e, S0> -> dgam_C
-      float dot = 0.f;
-      for (int e = tid; e < Dk * Dv; e += kBcThreads) {
-        const int d = e / Dv, c = e - d * Dv;
-        dot = fmaf(bf(sdS[d * lbv + c]), bf(sS0[d * lbv + c]), dot);
-      }
+  }
 #pragma unroll
-      for (int off = 16; off; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-      if (lane == 0) sm.red[warp] = dot;
-    }
-    __syncthreads();  // every read of dS_e is done
-    float dgamC = 0.f;
+  for (int i = 0; i < 64 / kBcWarps; ++i) {
+    const int p = warp + kBcWarps * i, r = sm.row[p];
+    float sw = 0.f, su = 0.f;
+    for (int d = lane; d < Dk; d += 32) sw = fmaf(bf(sK[p * lbk + d]), bf(sdW[p * lbk + d]), sw);
 #pragma unroll
-    for (int w = 0; w < kBcWarps; ++w) dgamC += sm.red[w];
-    dgamC *= eC;
-    // ---- 5. dP = dO U^T -> dQK = M o dP; gam gets dP o P
-    gemm_rc(64, 64, Dv, dO, [&](int kk, int n) { return bf(sU[n * lbv + kk]); },
-            [&](int m, int n, float v) { return n <= m ? v * sP[m * kLd64 + n] : 0.f; },
-            [&](int m, int n, float v) {
-              sP[m * kLd64 + n] = n <= m ? expf(sm.gam[m] - sm.gam[n]) * v : 0.f;
-            },
-            sm.dgam, sm.dgam);
-    // ---- 6. Z = diag(e^gam) dO S0^T: dq^ = Z, gam_p gets q^_p . Z_p
-    gemm_rc(64, Dk, Dv, [&](int m, int kk) { return sm.eg[m] * dO(m, kk); },
-            [&](int kk, int n) { return bf(sS0[n * lbv + kk]); },
-            [&](int m, int n, float v) { return Qh(m, n) * v; },
-            [&](int m, int n, float v) { sdW[m * ldk + n] = v; }, sm.dgam, nullptr);
-    __syncthreads();
-    // ---- 7. dq^ += dQK K^ (same tile owners as step 6)
-    gemm(64, Dk, 64, [&](int m, int kk) { return sP[m * kLd64 + kk]; }, Kh,
-         [&](int m, int n, float v) { sdW[m * ldk + n] += v; });
-    // ---- 8. dk^ += dQK^T Q^
-    gemm_acc(Dk, 64, [&](int m, int kk) { return sP[kk * kLd64 + m]; }, Qh, dk,
-             [&](int, int, float v) { return v; });
-    __syncthreads();
-    for (int e = tid; e < 64 * Dk; e += kBcThreads) {  // dq^ out
-      const int p = e / Dk, d = e - p * Dk;
-      if (sm.row[p] >= 0) pq[(size_t)sm.row[p] * Dk + d] = sdW[p * ldk + d];
-    }
-    __syncthreads();
-    // ---- 9. dW = -dU S0^T
-    gemm(64, Dk, Dv, [&](int m, int kk) { return sdU[m * ldv + kk]; },
-         [&](int kk, int n) { return bf(sS0[n * lbv + kk]); },
-         [&](int m, int n, float v) { sdW[m * ldk + n] = -v; });
-    __syncthreads();
-    // ---- 10. [dX_w | dX_u] solves (I + A)^T X = [dW | dU], a column per thread
-    for (int c = tid; c < Dk + Dv; c += kBcThreads) {
-      float* col = c < Dk ? sdW + c : sdU + (c - Dk);
-      const int ld = c < Dk ? ldk : ldv;
-      float x[64];
-#pragma unroll
-      for (int p = 0; p < 64; ++p) x[p] = col[p * ld];
-      solve_upper(sA, x);
-#pragma unroll
-      for (int p = 0; p < 64; ++p) col[p * ld] = x[p];
-    }
-    __syncthreads();
-    // ---- 11. dk^ += diag(beta e^gam) dX_w;  dv = diag(beta) dX_u;  beta and gam
-    //          from the rows of X_w = diag(beta e^gam) K^ and X_u = diag(beta) V
-    {
-      const int tn = Dk >> 4, nt = 4 * tn;
-#pragma unroll
-      for (int i = 0; i < kMaxBlocks; ++i) {
-        const int t = warp + kBcWarps * i;
-        if (t < nt) {
-          const int m0 = (t / tn) << 4, n0 = (t % tn) << 4;
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int m = m0 + tile_row(e), n = n0 + 8 * hh + tile_col(e);
-              dk[i][hh][e] = fmaf(sm.beta[m] * sm.eg[m], sdW[m * ldk + n], dk[i][hh][e]);
-            }
-        }
+    for (int q4 = 0; q4 < 4; ++q4) {
+      const int c = lane + 32 * q4;
+      if (c < Dv) {
+        const float xu = bf(sdU[p * lbv + c]);
+        if (r >= 0) dvb[(size_t)r * Dv + c] = sm.beta[p] * xu;
+        su = fmaf(vreg[i][q4], xu, su);
       }
     }
-    for (int p = warp; p < 64; p += kBcWarps) {
-      const int r = sm.row[p];
-      float sw = 0.f, su = 0.f;
-      for (int d = lane; d < Dk; d += 32) sw = fmaf(Kh(p, d), sdW[p * ldk + d], sw);
-      if (r >= 0) {
-        for (int c = lane; c < Dv; c += 32) {
-          const float xu = sdU[p * ldv + c];
-          dvb[(size_t)r * Dv + c] = sm.beta[p] * xu;
-          su = fmaf(bf(a.v[(size_t)r * Dv + c]), xu, su);
-        }
-      }
 #pragma unroll
-      for (int off = 16; off; off >>= 1) {
-        sw += __shfl_xor_sync(0xffffffffu, sw, off);
-        su += __shfl_xor_sync(0xffffffffu, su, off);
-      }
-      if (lane == 0) {  // step 12's epilogues may already be adding to these rows
-        atomicAdd(&sm.dbeta[p], sm.eg[p] * sw + su);
-        atomicAdd(&sm.dgam[p], sm.beta[p] * sm.eg[p] * sw);
-      }
+    for (int off = 16; off; off >>= 1) {
+      sw += __shfl_xor_sync(0xffffffffu, sw, off);
+      su += __shfl_xor_sync(0xffffffffu, su, off);
     }
-    // ---- 12. dA = -(dX_w W^T + dX_u U~^T) on i < p -> dG; gam and beta from A
-    // (dA o E) into sP first: its row sums feed beta, then it becomes dG
-    gemm_rc(64, 64, Dk + Dv,
-            [&](int m, int kk) { return kk < Dk ? sdW[m * ldk + kk] : sdU[m * ldv + kk - Dk]; },
-            [&](int kk, int n) { return kk < Dk ? bf(sW[n * lbk + kk]) : bf(sKU[n * lbv + kk - Dk]); },
-            [&](int m, int n, float v) { return n < m ? -v * sA[m * kLd64 + n] : 0.f; },
-            [&](int m, int n, float v) { sP[m * kLd64 + n] = n < m ? -v : 0.f; }, sm.dgam, sm.dgam);
-    __syncthreads();
-    for (int p = warp; p < 64; p += kBcWarps) {  // dbeta_p += sum_i dA_pi E_pi; dG = dA beta_p e^{..}
-      float sb = 0.f;
-      for (int i = lane; i < p; i += 32) {
-        const float dA = sP[p * kLd64 + i];
-        sb = fmaf(dA, bf(sE[p * kLdE + i]), sb);
-        sP[p * kLd64 + i] = dA * sm.beta[p] * expf(sm.gam[p] - sm.gam[i]);
-      }
-#pragma unroll
-      for (int off = 16; off; off >>= 1) sb += __shfl_xor_sync(0xffffffffu, sb, off);
-      if (lane == 0) atomicAdd(&sm.dbeta[p], sb);
+    if (lane == 0) {  // step 12's epilogues may already be adding to these rows
+      atomicAdd(&sm.dbeta[p], sm.eg[p] * sw + su);
+      atomicAdd(&sm.dgam[p], sm.beta[p] * sm.eg[p] * sw);
     }
-    __syncthreads();
-    // ---- 13. dk^ += (dG + dG^T) K^
-    gemm_acc(Dk, 64, [&](int m, int kk) { return sP[m * kLd64 + kk] + sP[kk * kLd64 + m]; }, Kh, dk,
-             [&](int, int, float v) { return v; });
-    // ---- 14. outputs: dk^, dbeta, dg = suffix sum of dgam + dgam_C
-    {
-      const int tn = Dk >> 4, nt = 4 * tn;
-#pragma unroll
-      for (int i = 0; i < kMaxBlocks; ++i) {
-        const int t = warp + kBcWarps * i;
-        if (t < nt) {
-          const int m0 = (t / tn) << 4, n0 = (t % tn) << 4;
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int m = m0 + tile_row(e), n = n0 + 8 * hh + tile_col(e);
-              if (sm.row[m] >= 0) pk[(size_t)sm.row[m] * Dk + n] = dk[i][hh][e];
-            }
-        }
-      }
+  }
+  // ---- 12. dA = -(dX_w W^T + dX_u U~^T) on i < p (into P); gam from A
+  gemm2<false, true, false, true>(64, 64, dWm, Wm, Dk, dUm, Ut, Dv,
+      [&](int m, int n, float v) { return n < m ? -v * sA[m * kLd64 + n] : 0.f; },
+      [&](int m, int n, float v) { sP[m * kLdE + n] = __float2bfloat16_rn(n < m ? -v : 0.f); },
+      sm.dgam, sm.dgam);
+  __syncthreads();
+  for (int p = warp; p < 64; p += kBcWarps) {  // dbeta_p += sum_i dA_pi E_pi; dG = dA beta_p e^{..}
+    float sb = 0.f;
+    for (int i = lane; i < p; i += 32) {
+      const float dA = bf(sP[p * kLdE + i]);
+      sb = fmaf(dA, bf(sE[p * kLdE + i]), sb);
+      sP[p * kLdE + i] = __float2bfloat16_rn(dA * sm.beta[p] * expf(sm.gam[p] - sm.gam[i]));
     }
-    __syncthreads();  // every addition to dgam and dbeta is done
-    if (warp == 0) {
-      // K~ = diag(e^{gam_C - gam}) K^: row p's exponent gives -c_p to gam_p
-      // and +c_p to gam_C
-      float cs = sm.cK[2 * lane] + sm.cK[2 * lane + 1];
 #pragma unroll
-      for (int off = 16; off; off >>= 1) cs += __shfl_xor_sync(0xffffffffu, cs, off);
-      const float dC = dgamC + cs;
-      const float d0 = sm.dgam[2 * lane] - sm.cK[2 * lane];
-      const float d1 = sm.dgam[2 * lane + 1] - sm.cK[2 * lane + 1];
-      // suffix sums over scan positions 2 lane, 2 lane + 1 .. 63
-      float incl = d0 + d1;
+    for (int off = 16; off; off >>= 1) sb += __shfl_xor_sync(0xffffffffu, sb, off);
+    if (lane == 0) atomicAdd(&sm.dbeta[p], sb);
+  }
+  __syncthreads();
+  // ---- 13. dk^ += (dG + dG^T) K^
+  gemm_acc2<false, false>(Dk, 64, Pm, K, dk, [](int) { return 1.f; });
+  gemm_acc2<true, false>(Dk, 64, Pm, K, dk, [](int) { return 1.f; });
+  // ---- 14. outputs: dk^, dbeta, dg = suffix sum of dgam + dgam_C
+  for_acc(Dk, [&](int i, int hh, int e, int m, int n) {
+    if (sm.row[m] >= 0) pk[(size_t)sm.row[m] * Dk + n] = dk[i][hh][e];
+  });
+  __syncthreads();  // every addition to dgam and dbeta is done
+  if (warp == 0) {
+    // K~ = diag(e^{gam_C - gam}) K^: row p's exponent gives -c_p to gam_p
+    // and +c_p to gam_C
+    float cs = sm.cK[2 * lane] + sm.cK[2 * lane + 1];
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const float y = __shfl_down_sync(0xffffffffu, incl, off);
-        if (lane + off < 32) incl += y;
-      }
-      const float g0 = incl + dC, g1 = incl - d0 + dC;
-      const int r0 = sm.row[2 * lane], r1 = sm.row[2 * lane + 1];
-      if (r0 >= 0) {
-        pab[(size_t)r0 * 2] = g0;
-        pab[(size_t)r0 * 2 + 1] = sm.dbeta[2 * lane];
-      }
-      if (r1 >= 0) {
-        pab[(size_t)r1 * 2] = g1;
-        pab[(size_t)r1 * 2 + 1] = sm.dbeta[2 * lane + 1];
-      }
+    for (int off = 16; off; off >>= 1) cs += __shfl_xor_sync(0xffffffffu, cs, off);
+    const float dC = dgamC + cs;
+    const float d0 = sm.dgam[2 * lane] - sm.cK[2 * lane];
+    const float d1 = sm.dgam[2 * lane + 1] - sm.cK[2 * lane + 1];
+    float incl = d0 + d1;  // suffix sums over scan positions 2 lane, 2 lane + 1 .. 63
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float y = __shfl_down_sync(0xffffffffu, incl, off);
+      if (lane + off < 32) incl += y;
+    }
+    const float g0 = incl + dC, g1 = incl - d0 + dC;
+    const int r0 = sm.row[2 * lane], r1 = sm.row[2 * lane + 1];
+    if (r0 >= 0) {
+      pab[(size_t)r0 * 2] = g0;
+      pab[(size_t)r0 * 2 + 1] = sm.dbeta[2 * lane];
+    }
+    if (r1 >= 0) {
+      pab[(size_t)r1 * 2] = g1;
+      pab[(size_t)r1 * 2 + 1] = sm.dbeta[2 * lane + 1];
     }
   }
 }
@@ -767,7 +794,7 @@ __global__ void __launch_bounds__(kBcThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
 }  // namespace
 
 bool bwd_chunked_fits(int Dk, int Dv) {
-  return Dk <= 112 && Dv <= 112 && BcLayout(Dk, Dv).total <= 227u * 1024u;
+  return Dk <= 112 && Dv <= 112 && GradLayout(Dk, Dv).total <= 227u * 1024u;
 }
 
 namespace {
@@ -836,7 +863,7 @@ cudaError_t launch_backward_chunked(const BwdCall& c, void* workspace, float** p
   *pq = a.pq; *pk = a.pk; *pab = a.pab; *dvb = a.dvb;
   const int smem_pre = (int)PreLayout(c.Dk, c.Dv).total;
   const int smem_chain = (int)ChainLayout2(c.Dk).total;
-  const int smem_grad = (int)BcLayout(c.Dk, c.Dv).total;
+  const int smem_grad = (int)GradLayout(c.Dk, c.Dv).total;
   if ((e = cudaFuncSetAttribute(gdn_bwd_pre_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 smem_pre)) != cudaSuccess ||
       (e = cudaFuncSetAttribute(gdn_bwd_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
