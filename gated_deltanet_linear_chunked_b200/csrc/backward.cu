@@ -360,59 +360,97 @@ __device__ __forceinline__ void st_io(__nv_bfloat16* p, float x) { *p = __float2
 // Sum the partials of every slice and direction for one (b, t, h) row, apply
 // the normalisation's Jacobian, and write dq, dk, dv, dg, dbeta.
 // pab[..][0] holds dL/da (token-serial path: dg = e^g da) or dL/dg itself
-// (chunked path, `pab_is_dg`).
+// (chunked path, `pab_is_dg`).  One warp per (b, t, h) row, four rows per
+// block; lane l holds elements 4 l .. 4 l + 3 (D <= 128), read 16 bytes at a
+// time from the fp32 partials.
+constexpr int kRedRows = 4;
+
+__device__ __forceinline__ void ld4_io(const float* p, float (&x)[4]) {
+  const float4 v = *reinterpret_cast<const float4*>(p);
+  x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+}
+__device__ __forceinline__ void ld4_io(const __nv_bfloat16* p, float (&x)[4]) {
+  const uint2 v = *reinterpret_cast<const uint2*>(p);
+  x[0] = __uint_as_float(v.x << 16); x[1] = __uint_as_float(v.x & 0xFFFF0000u);
+  x[2] = __uint_as_float(v.y << 16); x[3] = __uint_as_float(v.y & 0xFFFF0000u);
+}
+__device__ __forceinline__ void st4_io(float* p, const float (&x)[4]) {
+  *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
+}
+__device__ __forceinline__ void st4_io(__nv_bfloat16* p, const float (&x)[4]) {
+  const __nv_bfloat162 a = __floats2bfloat162_rn(x[0], x[1]), b = __floats2bfloat162_rn(x[2], x[3]);
+  *reinterpret_cast<uint2*>(p) = make_uint2(*reinterpret_cast<const uint32_t*>(&a),
+                                            *reinterpret_cast<const uint32_t*>(&b));
+}
+
 template <typename IO>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(32 * kRedRows)
 gdn_bwd_reduce_kernel(BwdArgs A, int ndir, void* dq_, void* dk_, void* dv_, float* dg, float* dbeta,
                       int pab_is_dg) {
   const size_t rows_bth = (size_t)A.B * A.T * A.H;
-  const size_t row = blockIdx.x;
-  const int tid = threadIdx.x, Dk = A.Dk, Dv = A.Dv;
+  const size_t row = (size_t)blockIdx.x * kRedRows + (threadIdx.x >> 5);
+  if (row >= rows_bth) return;  // whole warps
+  const int lane = threadIdx.x & 31, Dk = A.Dk, Dv = A.Dv, c = 4 * lane;
   const IO* q = static_cast<const IO*>(A.q);
   const IO* k = static_cast<const IO*>(A.k);
   IO* dq = static_cast<IO*>(dq_);
   IO* dk = static_cast<IO*>(dk_);
   IO* dv = static_cast<IO*>(dv_);
-  // dq^, dk^ (this thread's element i = tid), their dot products with q^, k^
-  float gq = 0.f, gk = 0.f, qi = 0.f, ki = 0.f;
-  if (tid < Dk) {
+  float gq[4] = {0.f, 0.f, 0.f, 0.f}, gk[4] = {0.f, 0.f, 0.f, 0.f};
+  float qi[4] = {0.f, 0.f, 0.f, 0.f}, ki[4] = {0.f, 0.f, 0.f, 0.f};
+  if (c < Dk) {
     for (int d = 0; d < ndir; ++d)
       for (int s = 0; s < A.nslice; ++s) {
-        const size_t base = ((size_t)d * A.nslice + s) * rows_bth;
-        gq += A.pq[(base + row) * Dk + tid];
-        gk += A.pk[(base + row) * Dk + tid];
+        const size_t base = ((size_t)d * A.nslice + s) * rows_bth + row;
+        float x[4], y[4];
+        ld4_io(A.pq + base * Dk + c, x);
+        ld4_io(A.pk + base * Dk + c, y);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          gq[e] += x[e];
+          gk[e] += y[e];
+        }
       }
-    qi = ld_io(q + row * Dk + tid);
-    ki = ld_io(k + row * Dk + tid);
+    ld4_io(q + row * Dk + c, qi);
+    ld4_io(k + row * Dk + c, ki);
   }
-  float v4[4] = {qi * qi, ki * ki, qi * gq, ki * gk};
+  // |q|^2, |k|^2, q . dq^, k . dk^ over the row
+  float t4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    t4[0] = fmaf(qi[e], qi[e], t4[0]);
+    t4[1] = fmaf(ki[e], ki[e], t4[1]);
+    t4[2] = fmaf(qi[e], gq[e], t4[2]);
+    t4[3] = fmaf(ki[e], gk[e], t4[3]);
+  }
 #pragma unroll
   for (int off = 16; off; off >>= 1)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) v4[e] += __shfl_xor_sync(0xffffffffu, v4[e], off);
-  __shared__ float wsum[4][4];
-  if ((tid & 31) == 0)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) wsum[tid >> 5][e] = v4[e];
-  __syncthreads();
-  float tot[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) tot[e] = wsum[0][e] + wsum[1][e] + wsum[2][e] + wsum[3][e];
-  if (tid < Dk) {
+    for (int e = 0; e < 4; ++e) t4[e] += __shfl_xor_sync(0xffffffffu, t4[e], off);
+  if (c < Dk) {
     // x^ = x r with r = 1 / max(|x|, 1e-6): dx = r (dx^ - x^ (x^ . dx^)) when
     // |x|^2 > 1e-12, else r dx^ (the clamp makes r constant)
-    const float rq = 1.0f / sqrtf(fmaxf(tot[0], 1e-12f)), rk = 1.0f / sqrtf(fmaxf(tot[1], 1e-12f));
-    const float dq_i = tot[0] > 1e-12f ? rq * (gq - qi * rq * rq * tot[2]) : rq * gq;
-    const float dk_i = tot[1] > 1e-12f ? rk * (gk - ki * rk * rk * tot[3]) : rk * gk;
-    st_io(dq + row * Dk + tid, dq_i);
-    st_io(dk + row * Dk + tid, dk_i);
+    const float rq = 1.0f / sqrtf(fmaxf(t4[0], 1e-12f)), rk = 1.0f / sqrtf(fmaxf(t4[1], 1e-12f));
+    float oq[4], ok[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      oq[e] = t4[0] > 1e-12f ? rq * (gq[e] - qi[e] * rq * rq * t4[2]) : rq * gq[e];
+      ok[e] = t4[1] > 1e-12f ? rk * (gk[e] - ki[e] * rk * rk * t4[3]) : rk * gk[e];
+    }
+    st4_io(dq + row * Dk + c, oq);
+    st4_io(dk + row * Dk + c, ok);
   }
-  for (int j = tid; j < Dv; j += 128) {
-    float s = 0.f;
-    for (int d = 0; d < ndir; ++d) s += A.dvb[((size_t)d * rows_bth + row) * Dv + j];
-    st_io(dv + row * Dv + j, s);
+  if (c < Dv) {
+    float sv[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int d = 0; d < ndir; ++d) {
+      float x[4];
+      ld4_io(A.dvb + ((size_t)d * rows_bth + row) * Dv + c, x);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sv[e] += x[e];
+    }
+    st4_io(dv + row * Dv + c, sv);
   }
-  if (tid == 0) {
+  if (lane == 0) {
     float da = 0.f, db = 0.f;
     for (int d = 0; d < ndir; ++d)
       for (int s = 0; s < A.nslice; ++s) {
@@ -431,8 +469,11 @@ size_t bwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, gdn_dtype dtype,
   if (dtype == GDN_BF16 && bwd_chunked_fits(Dk, Dv)) return bwd_chunked_workspace_bytes(B, T, H, Dk, Dv, bidir);
   const size_t ndir = bidir ? 2 : 1, nslice = Dv / kBCols, nblk = (T + kBBlock - 1) / kBBlock;
   const size_t rows = (size_t)B * T * H, ctas = ndir * B * H * nslice;
+  // the (da, dbeta) partials are rounded up to 4 floats so that dv's start
+  // stays 16-byte aligned for the reduction's vector loads
   return sizeof(float) * (ctas * (nblk + 1) * kBState + ctas * kBBlock * kBState +
-                          2 * ndir * nslice * rows * Dk + ndir * nslice * rows * 2 + ndir * rows * Dv);
+                          2 * ndir * nslice * rows * Dk + ((ndir * nslice * rows * 2 + 3) & ~size_t(3)) +
+                          ndir * rows * Dv);
 }
 
 cudaError_t launch_backward(const BwdCall& c, void* workspace) {
@@ -445,7 +486,7 @@ cudaError_t launch_backward(const BwdCall& c, void* workspace) {
     const size_t rows = (size_t)c.B * c.T * c.H;
     {
       ProfileScope ps(c.stream, kKernBwdReduce);
-      gdn_bwd_reduce_kernel<__nv_bfloat16><<<(unsigned)rows, 128, 0, c.stream>>>(
+      gdn_bwd_reduce_kernel<__nv_bfloat16><<<(unsigned)((rows + kRedRows - 1) / kRedRows), 32 * kRedRows, 0, c.stream>>>(
           A, c.bidir ? 2 : 1, c.dq, c.dk, c.dv, c.dg, c.dbeta, 1);
     }
     e = cudaGetLastError();
@@ -468,7 +509,7 @@ cudaError_t launch_backward(const BwdCall& c, void* workspace) {
   A.pk = w;
   w += (size_t)ndir * nslice * rows * c.Dk;
   A.pab = w;
-  w += (size_t)ndir * nslice * rows * 2;
+  w += ((size_t)ndir * nslice * rows * 2 + 3) & ~size_t(3);
   A.dvb = w;
   const int smem = (int)sizeof(BwdSmem);
   cudaError_t e;
@@ -483,7 +524,7 @@ cudaError_t launch_backward(const BwdCall& c, void* workspace) {
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     ProfileScope ps(c.stream, kKernBwdReduce);
-    gdn_bwd_reduce_kernel<float><<<(unsigned)rows, 128, 0, c.stream>>>(A, ndir, c.dq, c.dk, c.dv, c.dg,
+    gdn_bwd_reduce_kernel<float><<<(unsigned)((rows + kRedRows - 1) / kRedRows), 32 * kRedRows, 0, c.stream>>>(A, ndir, c.dq, c.dk, c.dv, c.dg,
                                                                        c.dbeta, 0);
   } else {
     e = cudaFuncSetAttribute(gdn_bwd_scan_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -496,7 +537,7 @@ cudaError_t launch_backward(const BwdCall& c, void* workspace) {
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     ProfileScope ps(c.stream, kKernBwdReduce);
-    gdn_bwd_reduce_kernel<__nv_bfloat16><<<(unsigned)rows, 128, 0, c.stream>>>(A, ndir, c.dq, c.dk, c.dv,
+    gdn_bwd_reduce_kernel<__nv_bfloat16><<<(unsigned)((rows + kRedRows - 1) / kRedRows), 32 * kRedRows, 0, c.stream>>>(A, ndir, c.dq, c.dk, c.dv,
                                                                                c.dg, c.dbeta, 0);
   }
   e = cudaGetLastError();
