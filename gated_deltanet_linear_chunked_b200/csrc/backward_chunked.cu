@@ -54,12 +54,16 @@ constexpr int kBcThreads = 256;
 constexpr int kBcWarps = kBcThreads / 32;
 constexpr int kLd64 = 68;   // fp32 row stride of the 64 x 64 tiles
 constexpr int kLdE = 72;    // bf16 row stride of the 64 x 64 E tile
-constexpr int kMaxBlocks = 4;  // 16 x 16 output blocks per warp of a 64 x Dk product, Dk <= 112
+// The gradient pass runs 16 warps: every phase has many independent 16 x 16
+// tiles, and with one CTA per SM the extra warps hide their latencies.
+constexpr int kGrThreads = 512;
+constexpr int kGrWarps = kGrThreads / 32;
+constexpr int kMaxBlocks = 2;  // 16 x 16 output blocks per warp of a 64 x Dk product, Dk <= 128
 
 struct BcSmall {
   float g[64], beta[64], gam[64], eg[64], dgam[64], dbeta[64], cK[64];
   int row[64];  // (b, t, h) row of scan position p, -1 past T
-  float red[kBcWarps];
+  float red[kGrWarps];
 };
 
 struct BcArgs {
@@ -136,20 +140,6 @@ __device__ __forceinline__ void gemm(int M, int N, int K, FA A, FB B, FE epi) {
       for (int e = 0; e < 4; ++e) epi(m0 + tile_row(e), n0 + 8 * h + tile_col(e), d[h][e]);
   }
 }
-// x_p = r_p - sum_{t > p} A[t][p] x_t for p = 63 .. 0: (I + A)^T x = r for
-// one column held in registers.  Each sum runs in four interleaved
-// accumulators (a warp issues in order, so independent chains are what hides
-// the FMA latency) and takes the newest x_t (t = p + 1) last.
-__device__ __forceinline__ void solve_upper(const float* A, float (&x)[64]) {
-#pragma unroll
-  for (int p = 62; p >= 0; --p) {
-    float s[4] = {x[p], 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int t = 63; t > p; --t) s[(63 - t) & 3] = fmaf(-A[t * kLd64 + p], x[t], s[(63 - t) & 3]);
-    x[p] = (s[0] + s[1]) + (s[2] + s[3]);
-  }
-}
-
 // Stage chunk j of (b, h) in direction dir, rows in scan order: gates (zero
 // past T), q^ = q / |q|, k^ likewise (bf16), dO; gam (inclusive prefix sum of
 // g) and e^gam.  Every thread of the CTA takes part; ends with a barrier.
@@ -388,7 +378,7 @@ __global__ void __launch_bounds__(kChThreads) gdn_bwd_chain_kernel(BcArgs a) {
 // registers; the triangular solve runs in fp32 registers per column.
 struct GradLayout {
   int lbk, lbv;
-  uint32_t q, k, dout, w, ut, u, s0, dse, P, A, E, dU, dW, small, total;
+  uint32_t q, k, dout, w, ut, u, s0, dse, P, A, Ab, E, dU, dW, small, total;
   __host__ __device__ GradLayout(int Dk, int Dv) {
     lbk = Dk + 8;
     lbv = Dv + 8;
@@ -403,6 +393,7 @@ struct GradLayout {
     dse = o;  o += Dk * lbv * 2;    // dS_e [Dk][Dv]
     P = o;    o += 64 * kLdE * 2;   // P, then dQK, then dA / dG (bf16)
     A = o;    o += 64 * kLd64 * 4;  // A (fp32, the solve's matrix)
+    Ab = o;   o += 64 * kLdE * 2;   // A in bf16 (the solve's block updates)
     E = o;    o += 64 * kLdE * 2;   // e^{gam_p - gam_i} K^ K^T (i < p), bf16
     dU = o;   o += 64 * lbv * 2;    // dU, then dX_u (bf16)
     dW = o;   o += 64 * lbk * 2;    // dW, then dX_w (bf16)
@@ -503,7 +494,7 @@ __device__ __forceinline__ void gemm_acc2(int N, int K, BMat A, BMat B, float (&
   const int tn = N >> 4, nt = 4 * tn;
 #pragma unroll
   for (int i = 0; i < kMaxBlocks; ++i) {
-    const int t = warp + kBcWarps * i;
+    const int t = warp + kGrWarps * i;
     if (t < nt) {
       const int m0 = (t / tn) << 4, n0 = (t % tn) << 4;
       float d[2][4];
@@ -523,7 +514,7 @@ __device__ __forceinline__ void for_acc(int N, F f) {
   const int tn = N >> 4, nt = 4 * tn;
 #pragma unroll
   for (int i = 0; i < kMaxBlocks; ++i) {
-    const int t = warp + kBcWarps * i;
+    const int t = warp + kGrWarps * i;
     if (t < nt) {
       const int m0 = (t / tn) << 4, n0 = (t % tn) << 4;
 #pragma unroll
@@ -540,7 +531,7 @@ __device__ __forceinline__ void acc_row_sums(int N, float* dst, F f) {
   const int tn = N >> 4, nt = 4 * tn;
 #pragma unroll
   for (int i = 0; i < kMaxBlocks; ++i) {
-    const int t = warp + kBcWarps * i;
+    const int t = warp + kGrWarps * i;
     if (t < nt) {
       const int m0 = (t / tn) << 4, n0 = (t % tn) << 4;
       float r0 = 0.f, r1 = 0.f;
@@ -563,7 +554,7 @@ __device__ __forceinline__ void acc_row_sums(int N, float* dst, F f) {
   }
 }
 
-__global__ void __launch_bounds__(kBcThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
+__global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   extern __shared__ __align__(16) uint8_t bg_raw[];
   const int Dk = a.Dk, Dv = a.Dv;
   const GradLayout L(Dk, Dv);
@@ -578,6 +569,7 @@ __global__ void __launch_bounds__(kBcThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   bf16* sdS = reinterpret_cast<bf16*>(bg_raw + L.dse);
   bf16* sP = reinterpret_cast<bf16*>(bg_raw + L.P);
   float* sA = reinterpret_cast<float*>(bg_raw + L.A);
+  bf16* sAb = reinterpret_cast<bf16*>(bg_raw + L.Ab);
   bf16* sE = reinterpret_cast<bf16*>(bg_raw + L.E);
   bf16* sdU = reinterpret_cast<bf16*>(bg_raw + L.dU);
   bf16* sdW = reinterpret_cast<bf16*>(bg_raw + L.dW);
@@ -600,23 +592,23 @@ __global__ void __launch_bounds__(kBcThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   stage_rows(a, sm, sQ, sK, sO, lbk, lbv, b, h, dir, j);
   {
     const int ck = Dk / 8, cv = Dv / 8;
-    for (int e = tid; e < 64 * (ck + 2 * cv); e += kBcThreads) {  // [slab][time row][8] -> [scan row]
+    for (int e = tid; e < 64 * (ck + 2 * cv); e += kGrThreads) {  // [slab][time row][8] -> [scan row]
       const int s2 = e >> 6, t = e & 63, p = dir == 0 ? t : 63 - t;
       if (s2 < ck) cp16(sW + p * lbk + 8 * s2, blk + a.wl.off_w + 16 * (s2 * 64 + t));
       else if (s2 < ck + cv) cp16(sUt + p * lbv + 8 * (s2 - ck), blk + a.wl.off_ut + 16 * ((s2 - ck) * 64 + t));
       else cp16(sU + p * lbv + 8 * (s2 - ck - cv), blk + a.wl.off_u + 16 * ((s2 - ck - cv) * 64 + t));
     }
-    for (int e = tid; e < cv * Dk; e += kBcThreads) {  // S0: [Dv/8][Dk][8] -> [Dk][Dv]
+    for (int e = tid; e < cv * Dk; e += kGrThreads) {  // S0: [Dv/8][Dk][8] -> [Dk][Dv]
       const int s2 = e / Dk, d = e - s2 * Dk;
       cp16(sS0 + d * lbv + 8 * s2, blk + a.wl.off_s + 16 * (s2 * Dk + d));
     }
     const bf16* dSe = a.dSe + bi * Dk * Dv;
-    for (int e = tid; e < Dk * cv; e += kBcThreads) {
+    for (int e = tid; e < Dk * cv; e += kGrThreads) {
       const int d = e / cv, c = e - d * cv;
       cp16(sdS + d * lbv + 8 * c, dSe + (size_t)d * Dv + 8 * c);
     }
     const float* dUg = a.dU + bi * 64 * Dv;
-    for (int e = tid; e < 64 * (Dv / 4); e += kBcThreads) {
+    for (int e = tid; e < 64 * (Dv / 4); e += kGrThreads) {
       const int p = e / (Dv / 4), c = 4 * (e - p * (Dv / 4));
       const float4 x = *reinterpret_cast<const float4*>(dUg + (size_t)p * Dv + c);
       __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(sdU + p * lbv + c);
@@ -639,6 +631,7 @@ __global__ void __launch_bounds__(kBcThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
     const float e = n < m ? expf(sm.gam[m] - sm.gam[n]) * v : 0.f;
     sE[m * kLdE + n] = __float2bfloat16_rn(e);
     sA[m * kLd64 + n] = sm.beta[m] * e;
+    sAb[m * kLdE + n] = __float2bfloat16_rn(sm.beta[m] * e);
   }, nullptr, nullptr);
   // ---- 3. dK~ = U dS_e^T: dk^ starts as e^{gam_C - gam} dK~; c_m = k^_m . dk^_m
   float dk[kMaxBlocks][2][4], dq[kMaxBlocks][2][4];
@@ -651,7 +644,7 @@ __global__ void __launch_bounds__(kBcThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   acc_row_sums(Dk, sm.cK, [&](int i, int hh, int e, int m, int n) { return bf(sK[m * lbk + n]) * dk[i][hh][e]; });
   {  // <dS_e, S0> -> dgam_C
     float dot = 0.f;
-    for (int e = tid; e < Dk * Dv; e += kBcThreads) {
+    for (int e = tid; e < Dk * Dv; e += kGrThreads) {
       const int d = e / Dv, c = e - d * Dv;
       dot = fmaf(bf(sdS[d * lbv + c]), bf(sS0[d * lbv + c]), dot);
     }
@@ -662,7 +655,7 @@ __global__ void __launch_bounds__(kBcThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   __syncthreads();  // P and A, E complete; every read of dS_e done
   float dgamC = 0.f;
 #pragma unroll
-  for (int w = 0; w < kBcWarps; ++w) dgamC += sm.red[w];
+  for (int w = 0; w < kGrWarps; ++w) dgamC += sm.red[w];
   dgamC *= eC;
   // ---- 5. dP = dO U^T -> dQK = M o dP (in place of P); gam gets dP o P
   gemm2<false, true, false, true>(64, 64, O, Um, Dv, O, Um, 0,
@@ -685,28 +678,54 @@ __global__ void __launch_bounds__(kBcThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   gemm2<false, true, false, true>(64, Dk, dUm, S0, Dv, dUm, S0, 0, none,
       [&](int m, int n, float v) { sdW[m * lbk + n] = __float2bfloat16_rn(-v); }, nullptr, nullptr);
   __syncthreads();
-  // ---- 10. [dX_w | dX_u] solves (I + A)^T X = [dW | dU], a column per thread
-  for (int c = tid; c < Dk + Dv; c += kBcThreads) {
-    bf16* col = c < Dk ? sdW + c : sdU + (c - Dk);
-    const int ld = c < Dk ? lbk : lbv;
-    float x[64];
+  // ---- 10. [dX_w | dX_u] solves (I + A)^T X = [dW | dU], blocked by 16 rows
+  //          from the last: each diagonal block by back-substitution (a
+  //          column per thread, in registers), then the rows above it lose
+  //          A[block rows][above]^T X_block (tensor cores, in place)
+  for (int blk16r = 3; blk16r >= 0; --blk16r) {
+    const int r0 = 16 * blk16r;
+    for (int c = tid; c < Dk + Dv; c += kGrThreads) {
+      bf16* col = (c < Dk ? sdW + c : sdU + (c - Dk)) + r0 * (c < Dk ? lbk : lbv);
+      const int ld = c < Dk ? lbk : lbv;
+      float x[16];
 #pragma unroll
-    for (int p = 0; p < 64; ++p) x[p] = bf(col[p * ld]);
-    solve_upper(sA, x);
+      for (int p = 0; p < 16; ++p) x[p] = bf(col[p * ld]);
 #pragma unroll
-    for (int p = 0; p < 64; ++p) col[p * ld] = __float2bfloat16_rn(x[p]);
+      for (int p = 14; p >= 0; --p) {
+        float s4[4] = {x[p], 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int t = 15; t > p; --t)
+          s4[(15 - t) & 3] = fmaf(-sA[(r0 + t) * kLd64 + r0 + p], x[t], s4[(15 - t) & 3]);
+        x[p] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+      }
+#pragma unroll
+      for (int p = 0; p < 16; ++p) col[p * ld] = __float2bfloat16_rn(x[p]);
+    }
+    __syncthreads();
+    if (r0 > 0) {
+      // rows [0, r0) -= A[r0 .. r0+15][rows]^T X[r0 .. r0+15]
+      const BMat Ablk{sAb + r0 * kLdE, kLdE};
+      gemm2<true, false, true, false>(r0, Dk, Ablk, BMat{sdW + r0 * lbk, lbk}, 16, Ablk, Ablk, 0, none,
+          [&](int m, int n, float v) {
+            sdW[m * lbk + n] = __float2bfloat16_rn(bf(sdW[m * lbk + n]) - v);
+          }, nullptr, nullptr);
+      gemm2<true, false, true, false>(r0, Dv, Ablk, BMat{sdU + r0 * lbv, lbv}, 16, Ablk, Ablk, 0, none,
+          [&](int m, int n, float v) {
+            sdU[m * lbv + n] = __float2bfloat16_rn(bf(sdU[m * lbv + n]) - v);
+          }, nullptr, nullptr);
+      __syncthreads();
+    }
   }
-  __syncthreads();
   // ---- 11. dk^ += diag(beta e^gam) dX_w;  dv = diag(beta) dX_u;  beta and gam
   //          from the rows of X_w = diag(beta e^gam) K^ and X_u = diag(beta) V
   for_acc(Dk, [&](int i, int hh, int e, int m, int n) {
     dk[i][hh][e] = fmaf(sm.beta[m] * sm.eg[m], bf(sdW[m * lbk + n]), dk[i][hh][e]);
   });
   // v of this warp's rows, every load issued before any is used
-  float vreg[64 / kBcWarps][4];
+  float vreg[64 / kGrWarps][4];
 #pragma unroll
-  for (int i = 0; i < 64 / kBcWarps; ++i) {
-    const int r = sm.row[warp + kBcWarps * i];
+  for (int i = 0; i < 64 / kGrWarps; ++i) {
+    const int r = sm.row[warp + kGrWarps * i];
 #pragma unroll
     for (int q4 = 0; q4 < 4; ++q4) {
       const int c = lane + 32 * q4;
@@ -714,8 +733,8 @@ __global__ void __launch_bounds__(kBcThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
     }
   }
 #pragma unroll
-  for (int i = 0; i < 64 / kBcWarps; ++i) {
-    const int p = warp + kBcWarps * i, r = sm.row[p];
+  for (int i = 0; i < 64 / kGrWarps; ++i) {
+    const int p = warp + kGrWarps * i, r = sm.row[p];
     float sw = 0.f, su = 0.f;
     for (int d = lane; d < Dk; d += 32) sw = fmaf(bf(sK[p * lbk + d]), bf(sdW[p * lbk + d]), sw);
 #pragma unroll
@@ -743,7 +762,7 @@ __global__ void __launch_bounds__(kBcThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
       [&](int m, int n, float v) { sP[m * kLdE + n] = __float2bfloat16_rn(n < m ? -v : 0.f); },
       sm.dgam, sm.dgam);
   __syncthreads();
-  for (int p = warp; p < 64; p += kBcWarps) {  // dbeta_p += sum_i dA_pi E_pi; dG = dA beta_p e^{..}
+  for (int p = warp; p < 64; p += kGrWarps) {  // dbeta_p += sum_i dA_pi E_pi; dG = dA beta_p e^{..}
     float sb = 0.f;
     for (int i = lane; i < p; i += 32) {
       const float dA = bf(sP[p * kLdE + i]);
@@ -884,7 +903,7 @@ cudaError_t launch_backward_chunked(const BwdCall& c, void* workspace, float** p
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   {
     ProfileScope ps(c.stream, kKernBwdGrad);
-    gdn_bwd_grad_kernel<<<per_chunk, kBcThreads, smem_grad, c.stream>>>(a);
+    gdn_bwd_grad_kernel<<<per_chunk, kGrThreads, smem_grad, c.stream>>>(a);
   }
   e = cudaGetLastError();
   if (e == cudaSuccess) count_launches(3);
