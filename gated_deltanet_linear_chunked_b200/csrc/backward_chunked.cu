@@ -45,10 +45,7 @@
 namespace gdn {
 namespace {
 
-using sm100::ldmatrix_x4;
-using sm100::ldmatrix_x4_trans;
-using sm100::mma_16816;
-using sm100::smem_u32;
+using namespace sm100;
 
 constexpr int kBcThreads = 256;
 constexpr int kBcWarps = kBcThreads / 32;
@@ -74,12 +71,15 @@ struct BcArgs {
   const uint8_t* ws;         // the forward's workspace
   WsLayout wl;
   // per (direction, b*h, time chunk), rows in scan order:
-  float* X;                  // [64][Dv]  P^T dO
-  float* Y;                  // [Dk][Dv]  Q^^T diag(e^gam) dO
-  float* dU;                 // [64][Dv]  dU
-  __nv_bfloat16* dSe;        // [Dk][Dv]  dS_e, the gradient of the chunk's end state
+  // (all bf16, transposed so that a slice of 16 columns is contiguous):
+  __nv_bfloat16* XT;         // [Dv][64]  (P^T dO)^T
+  __nv_bfloat16* YT;         // [Dv][Dk]  (Q^^T diag(e^gam) dO)^T
+  __nv_bfloat16* dUT;        // [Dv][64]  dU^T
+  __nv_bfloat16* dSeT;       // [Dv][Dk]  dS_e^T, dS_e the gradient of the chunk's end state
   float *pq, *pk, *pab, *dvb;  // [dir][rows][Dk], [dir][rows][Dk], [dir][rows][2], [dir][rows][Dv]
   int B, T, H, Dk, Dv, nC, NBH;
+  unsigned* err;             // device error word (the chain's bounded waits)
+  long long limit;           // polls before a bounded wait gives up
   __device__ size_t blk(int dir, int bh, int j) const { return ((size_t)dir * NBH + bh) * nC + j; }
 };
 
@@ -140,268 +140,6 @@ __device__ __forceinline__ void gemm(int M, int N, int K, FA A, FB B, FE epi) {
       for (int e = 0; e < 4; ++e) epi(m0 + tile_row(e), n0 + 8 * h + tile_col(e), d[h][e]);
   }
 }
-// Stage chunk j of (b, h) in direction dir, rows in scan order: gates (zero
-// past T), q^ = q / |q|, k^ likewise (bf16), dO; gam (inclusive prefix sum of
-// g) and e^gam.  Every thread of the CTA takes part; ends with a barrier.
-__device__ void stage_rows(const BcArgs& a, BcSmall& sm, __nv_bfloat16* sQ, __nv_bfloat16* sK,
-                           __nv_bfloat16* sO, int lbk, int lbv, int b, int h, int dir, int j) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
-  const int Dk = a.Dk, Dv = a.Dv, t0 = 64 * j;
-  if (tid < 64) {
-    const int p = tid, t = t0 + (dir == 0 ? p : 63 - p);
-    const bool valid = t < a.T;
-    const size_t r = ((size_t)b * a.T + t) * a.H + h;
-    sm.row[p] = valid ? (int)r : -1;
-    sm.g[p] = valid ? __ldg(a.g + r) : 0.f;
-    sm.beta[p] = valid ? __ldg(a.beta + r) : 0.f;
-    sm.dgam[p] = 0.f;
-    sm.dbeta[p] = 0.f;
-    sm.cK[p] = 0.f;
-  }
-  __syncthreads();
-  const int ck = Dk / 8, cv = Dv / 8;
-  for (int e = tid; e < 64 * (2 * ck + cv); e += blockDim.x) {
-    const int p = e / (2 * ck + cv), c = e - p * (2 * ck + cv), r = sm.row[p];
-    __nv_bfloat16* dst;
-    const __nv_bfloat16* src;
-    if (c < ck) {
-      dst = sQ + p * lbk + 8 * c;
-      src = a.q + (size_t)r * Dk + 8 * c;
-    } else if (c < 2 * ck) {
-      dst = sK + p * lbk + 8 * (c - ck);
-      src = a.k + (size_t)r * Dk + 8 * (c - ck);
-    } else {
-      dst = sO + p * lbv + 8 * (c - 2 * ck);
-      src = a.dout + (size_t)r * Dv + 8 * (c - 2 * ck);
-    }
-    if (r >= 0) cp16(dst, src);
-    else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-  }
-  if (warp == 0) {
-    const float a0 = sm.g[2 * lane], a1 = sm.g[2 * lane + 1];
-    float incl = a0 + a1;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const float y = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += y;
-    }
-    const float excl = incl - (a0 + a1);
-    sm.gam[2 * lane] = excl + a0;
-    sm.gam[2 * lane + 1] = incl;
-    sm.eg[2 * lane] = expf(excl + a0);
-    sm.eg[2 * lane + 1] = expf(incl);
-  }
-  cp_wait_all();
-  __syncthreads();
-  for (int p = warp; p < 64; p += nw) {
-    float qq = 0.f, kk = 0.f;
-    for (int d = lane; d < Dk; d += 32) {
-      const float qv = bf(sQ[p * lbk + d]), kv = bf(sK[p * lbk + d]);
-      qq = fmaf(qv, qv, qq);
-      kk = fmaf(kv, kv, kk);
-    }
-#pragma unroll
-    for (int off = 16; off; off >>= 1) {
-      qq += __shfl_xor_sync(0xffffffffu, qq, off);
-      kk += __shfl_xor_sync(0xffffffffu, kk, off);
-    }
-    const float rq = 1.f / sqrtf(fmaxf(qq, 1e-12f)), rk = 1.f / sqrtf(fmaxf(kk, 1e-12f));
-    for (int d = lane; d < Dk; d += 32) {
-      sQ[p * lbk + d] = __float2bfloat16_rn(bf(sQ[p * lbk + d]) * rq);
-      sK[p * lbk + d] = __float2bfloat16_rn(bf(sK[p * lbk + d]) * rk);
-    }
-  }
-  __syncthreads();
-}
-
-// ---------------------------------------------------------------- pre pass
-// Every chunk at once: X = P^T dO and Y = Q^^T diag(e^gam) dO, which do not
-// depend on the later chunks.  Shared memory: q^, k^, dO (bf16), P (fp32).
-struct PreLayout {
-  int lbk, lbv;
-  uint32_t q, k, dout, P, small, total;
-  __host__ __device__ PreLayout(int Dk, int Dv) {
-    lbk = Dk + 8;
-    lbv = Dv + 8;
-    uint32_t o = 0;
-    q = o;    o += 64 * lbk * 2;
-    k = o;    o += 64 * lbk * 2;
-    dout = o; o += 64 * lbv * 2;
-    P = o;    o += 64 * kLd64 * 4;
-    small = o; o += sizeof(BcSmall);
-    total = (o + 15) & ~15u;
-  }
-};
-
-__global__ void __launch_bounds__(kBcThreads) gdn_bwd_pre_kernel(BcArgs a) {
-  extern __shared__ __align__(16) uint8_t bp_raw[];
-  const int Dk = a.Dk, Dv = a.Dv;
-  const PreLayout L(Dk, Dv);
-  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(bp_raw + L.q);
-  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(bp_raw + L.k);
-  __nv_bfloat16* sO = reinterpret_cast<__nv_bfloat16*>(bp_raw + L.dout);
-  float* sP = reinterpret_cast<float*>(bp_raw + L.P);
-  BcSmall& sm = *reinterpret_cast<BcSmall*>(bp_raw + L.small);
-  const int j = blockIdx.x, bh = blockIdx.y, dir = blockIdx.z;
-  const int b = bh / a.H, h = bh - b * a.H;
-  const int lbk = L.lbk, lbv = L.lbv;
-  stage_rows(a, sm, sQ, sK, sO, lbk, lbv, b, h, dir, j);
-  auto Qh = [&](int p, int d) { return bf(sQ[p * lbk + d]); };
-  auto Kh = [&](int p, int d) { return bf(sK[p * lbk + d]); };
-  auto dO = [&](int p, int c) { return bf(sO[p * lbv + c]); };
-  gemm(64, 64, Dk, Qh, [&](int kk, int n) { return Kh(n, kk); },
-       [&](int m, int n, float v) { sP[m * kLd64 + n] = n <= m ? expf(sm.gam[m] - sm.gam[n]) * v : 0.f; });
-  __syncthreads();
-  const size_t blk = a.blk(dir, bh, j);
-  float* X = a.X + blk * 64 * Dv;
-  float* Y = a.Y + blk * Dk * Dv;
-  gemm(64, Dv, 64, [&](int m, int kk) { return sP[kk * kLd64 + m]; }, dO,
-       [&](int m, int n, float v) { X[m * Dv + n] = v; });
-  gemm(Dk, Dv, 64, [&](int m, int kk) { return Qh(kk, m) * sm.eg[kk]; }, dO,
-       [&](int m, int n, float v) { Y[m * Dv + n] = v; });
-}
-
-// -------------------------------------------------------------- chain pass
-// One CTA per (16 columns of dS, b*h, direction), 128 threads, the chunks in
-// reverse scan order with the next chunk's tiles prefetched (cp.async, two
-// sets): dU = X + K~ dS_e, then dS0 = e^{gam_C} dS_e + Y - W^T dU.  Stores
-// each chunk's dS_e (bf16) and dU (fp32) for the gradient pass.
-constexpr int kChThreads = 128;
-constexpr int kChCols = 16;
-constexpr int kChLd = kChCols + 4;  // fp32 row stride of the 16-column tiles
-struct ChainLayout2 {
-  int lbk;
-  uint32_t kt, w, x, y, set, dS, dU, total;
-  __host__ __device__ ChainLayout2(int Dk) {
-    lbk = Dk + 8;
-    uint32_t o = 0;
-    kt = o; o += 64 * lbk * 2;        // K~ (bf16, scan rows)
-    w = o;  o += 64 * lbk * 2;        // W
-    x = o;  o += 64 * kChLd * 4;      // X columns
-    y = o;  o += Dk * kChLd * 4;      // Y columns
-    set = o;                          // one prefetch set
-    o *= 2;
-    dS = o; o += Dk * kChLd * 4;      // the running dS columns (fp32)
-    dU = o; o += 64 * kChLd * 4;
-    total = o;
-  }
-};
-
-__global__ void __launch_bounds__(kChThreads) gdn_bwd_chain_kernel(BcArgs a) {
-  extern __shared__ __align__(16) uint8_t bch_raw[];
-  const int Dk = a.Dk, Dv = a.Dv;
-  const ChainLayout2 L(Dk);
-  const int sl = blockIdx.x, bh = blockIdx.y, dir = blockIdx.z, c0 = kChCols * sl;
-  const int tid = threadIdx.x, lbk = L.lbk;
-  float* sdS = reinterpret_cast<float*>(bch_raw + L.dS);
-  float* sdU = reinterpret_cast<float*>(bch_raw + L.dU);
-  for (int e = tid; e < Dk * kChCols; e += kChThreads) {
-    const int d = e / kChCols, c = e - d * kChCols;
-    sdS[d * kChLd + c] = (dir == 0 && a.d_state_out)
-                             ? a.d_state_out[((size_t)bh * Dk + d) * Dv + c0 + c]
-                             : 0.f;
-  }
-  auto chunk_of = [&](int step) { return dir == 0 ? a.nC - 1 - step : step; };
-  auto prefetch = [&](int step, int set) {
-    uint8_t* base = bch_raw + set * L.set;
-    const int j = chunk_of(step);
-    const size_t blk = a.blk(dir, bh, j);
-    const uint8_t* wsb = a.ws + blk * a.wl.block_bytes;
-    const int ck = Dk / 8;
-    for (int e = tid; e < 64 * 2 * ck; e += kChThreads) {  // K~, W: [slab][time row][8] -> [scan row]
-      const int s2 = e >> 6, t = e & 63, p = dir == 0 ? t : 63 - t;
-      if (s2 < ck) cp16(base + L.kt + 2 * (p * lbk + 8 * s2), wsb + a.wl.off_kt + 16 * (s2 * 64 + t));
-      else cp16(base + L.w + 2 * (p * lbk + 8 * (s2 - ck)), wsb + a.wl.off_w + 16 * ((s2 - ck) * 64 + t));
-    }
-    const float* X = a.X + blk * 64 * Dv + c0;
-    const float* Y = a.Y + blk * Dk * Dv + c0;
-    for (int e = tid; e < (64 + Dk) * 4; e += kChThreads) {  // 16 fp32 columns = 4 x 16 B per row
-      const int r = e >> 2, q4 = e & 3;
-      if (r < 64) cp16(base + L.x + 4 * (r * kChLd + 4 * q4), X + (size_t)r * Dv + 4 * q4);
-      else cp16(base + L.y + 4 * ((r - 64) * kChLd + 4 * q4), Y + (size_t)(r - 64) * Dv + 4 * q4);
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-  };
-  prefetch(0, 0);
-  for (int step = 0; step < a.nC; ++step) {
-    const int set = step & 1, j = chunk_of(step);
-    if (step + 1 < a.nC) {
-      prefetch(step + 1, set ^ 1);
-      asm volatile("cp.async.wait_group 1;" ::: "memory");
-    } else {
-      cp_wait_all();
-    }
-    __syncthreads();
-    uint8_t* base = bch_raw + set * L.set;
-    const __nv_bfloat16* sKt = reinterpret_cast<const __nv_bfloat16*>(base + L.kt);
-    const __nv_bfloat16* sW = reinterpret_cast<const __nv_bfloat16*>(base + L.w);
-    const float* sX = reinterpret_cast<const float*>(base + L.x);
-    const float* sY = reinterpret_cast<const float*>(base + L.y);
-    const size_t blk = a.blk(dir, bh, j);
-    const float eC =
-        *reinterpret_cast<const float*>(a.ws + blk * a.wl.block_bytes + a.wl.off_decay);
-    // dS_e of this chunk, for the gradient pass
-    __nv_bfloat16* dSe = a.dSe + blk * Dk * Dv + c0;
-    for (int e = tid; e < Dk * kChCols / 2; e += kChThreads) {
-      const int d = e / (kChCols / 2), c = 2 * (e - d * (kChCols / 2));
-      *reinterpret_cast<__nv_bfloat162*>(dSe + (size_t)d * Dv + c) =
-          __floats2bfloat162_rn(sdS[d * kChLd + c], sdS[d * kChLd + c + 1]);
-    }
-    // dU = X + K~ dS_e
-    gemm(64, kChCols, Dk, [&](int m, int kk) { return bf(sKt[m * lbk + kk]); },
-         [&](int kk, int n) { return sdS[kk * kChLd + n]; },
-         [&](int m, int n, float v) { sdU[m * kChLd + n] = sX[m * kChLd + n] + v; });
-    __syncthreads();
-    float* dUg = a.dU + blk * 64 * Dv + c0;
-    for (int e = tid; e < 64 * kChCols; e += kChThreads) {
-      const int m = e / kChCols, c = e - m * kChCols;
-      dUg[(size_t)m * Dv + c] = sdU[m * kChLd + c];
-    }
-    // dS0 = e^{gam_C} dS_e + Y - W^T dU  (in place: each element by its owner)
-    gemm(Dk, kChCols, 64, [&](int m, int kk) { return -bf(sW[kk * lbk + m]); },
-         [&](int kk, int n) { return sdU[kk * kChLd + n]; },
-         [&](int m, int n, float v) { sdS[m * kChLd + n] = fmaf(eC, sdS[m * kChLd + n], sY[m * kChLd + n] + v); });
-    __syncthreads();
-  }
-  if (dir == 0 && a.d_state_in)
-    for (int e = tid; e < Dk * kChCols; e += kChThreads) {
-      const int d = e / kChCols, c = e - d * kChCols;
-      a.d_state_in[((size_t)bh * Dk + d) * Dv + c0 + c] = sdS[d * kChLd + c];
-    }
-}
-
-// ----------------------------------------------------------- gradient pass
-// Every chunk at once (one CTA per (chunk, b*h, direction)), from the
-// chunk's dU and dS_e: every product but the chain's.  All product operands
-// are bf16 tiles in shared memory fed to mma.sync.m16n8k16 by ldmatrix (the
-// .trans form where a tile is read transposed); dq^ and dk^ accumulate in
-// registers; the triangular solve runs in fp32 registers per column.
-struct GradLayout {
-  int lbk, lbv;
-  uint32_t q, k, dout, w, ut, u, s0, dse, P, A, Ab, E, dU, dW, small, total;
-  __host__ __device__ GradLayout(int Dk, int Dv) {
-    lbk = Dk + 8;
-    lbv = Dv + 8;
-    uint32_t o = 0;
-    q = o;    o += 64 * lbk * 2;    // q^
-    k = o;    o += 64 * lbk * 2;    // k^
-    dout = o; o += 64 * lbv * 2;    // dO
-    w = o;    o += 64 * lbk * 2;    // W
-    ut = o;   o += 64 * lbv * 2;    // U~
-    u = o;    o += 64 * lbv * 2;    // U
-    s0 = o;   o += Dk * lbv * 2;    // S0 [Dk][Dv]
-    dse = o;  o += Dk * lbv * 2;    // dS_e [Dk][Dv]
-    P = o;    o += 64 * kLdE * 2;   // P, then dQK, then dA / dG (bf16)
-    A = o;    o += 64 * kLd64 * 4;  // A (fp32, the solve's matrix)
-    Ab = o;   o += 64 * kLdE * 2;   // A in bf16 (the solve's block updates)
-    E = o;    o += 64 * kLdE * 2;   // e^{gam_p - gam_i} K^ K^T (i < p), bf16
-    dU = o;   o += 64 * lbv * 2;    // dU, then dX_u (bf16)
-    dW = o;   o += 64 * lbk * 2;    // dW, then dX_w (bf16)
-    small = o; o += sizeof(BcSmall);
-    total = (o + 15) & ~15u;
-  }
-};
-
 // A bf16 matrix in shared memory, row-major with row stride ld (a multiple
 // of 8).  As the A operand (m x k): element (m, k) = p[m ld + k], or
 // p[k ld + m] when read transposed.  As the B operand (k x n): element
@@ -485,6 +223,458 @@ __device__ __forceinline__ void gemm2(int M, int N, BMat A1, BMat B1, int K1, BM
     }
   }
 }
+// Out (M x N) = A B, stored to global memory as bf16: dst[m ld + n], the two
+// neighbouring columns a thread holds in one 4-byte store.
+template <bool TA, bool TB>
+__device__ __forceinline__ void gemm_store_bf16(int M, int N, BMat A, BMat B, int K,
+                                                __nv_bfloat16* dst, int ld) {
+  const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int tn = N >> 4, nt = (M >> 4) * tn;
+  for (int t = warp; t < nt; t += nw) {
+    const int m0 = (t / tn) << 4, nb = (t % tn) << 4;
+    float dd[2][4];
+    zero2(dd);
+    blk16<TA, TB>(m0, nb, K, A, B, dd);
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int n = nb + 8 * hh + tile_col(0);
+      *reinterpret_cast<uint32_t*>(dst + (size_t)(m0 + tile_row(0)) * ld + n) = pack_bf16x2(dd[hh][0], dd[hh][1]);
+      *reinterpret_cast<uint32_t*>(dst + (size_t)(m0 + tile_row(2)) * ld + n) = pack_bf16x2(dd[hh][2], dd[hh][3]);
+    }
+  }
+}
+
+// Stage chunk j of (b, h) in direction dir, rows in scan order: gates (zero
+// past T), q^ = q / |q|, k^ likewise (bf16), dO; gam (inclusive prefix sum of
+// g) and e^gam.  Every thread of the CTA takes part; ends with a barrier.
+__device__ void stage_rows(const BcArgs& a, BcSmall& sm, __nv_bfloat16* sQ, __nv_bfloat16* sK,
+                           __nv_bfloat16* sO, int lbk, int lbv, int b, int h, int dir, int j) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
+  const int Dk = a.Dk, Dv = a.Dv, t0 = 64 * j;
+  if (tid < 64) {
+    const int p = tid, t = t0 + (dir == 0 ? p : 63 - p);
+    const bool valid = t < a.T;
+    const size_t r = ((size_t)b * a.T + t) * a.H + h;
+    sm.row[p] = valid ? (int)r : -1;
+    sm.g[p] = valid ? __ldg(a.g + r) : 0.f;
+    sm.beta[p] = valid ? __ldg(a.beta + r) : 0.f;
+    sm.dgam[p] = 0.f;
+    sm.dbeta[p] = 0.f;
+    sm.cK[p] = 0.f;
+  }
+  __syncthreads();
+  const int ck = Dk / 8, cv = Dv / 8;
+  for (int e = tid; e < 64 * (2 * ck + cv); e += blockDim.x) {
+    const int p = e / (2 * ck + cv), c = e - p * (2 * ck + cv), r = sm.row[p];
+    __nv_bfloat16* dst;
+    const __nv_bfloat16* src;
+    if (c < ck) {
+      dst = sQ + p * lbk + 8 * c;
+      src = a.q + (size_t)r * Dk + 8 * c;
+    } else if (c < 2 * ck) {
+      dst = sK + p * lbk + 8 * (c - ck);
+      src = a.k + (size_t)r * Dk + 8 * (c - ck);
+    } else {
+      dst = sO + p * lbv + 8 * (c - 2 * ck);
+      src = a.dout + (size_t)r * Dv + 8 * (c - 2 * ck);
+    }
+    if (r >= 0) cp16(dst, src);
+    else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+  }
+  if (warp == 0) {
+    const float a0 = sm.g[2 * lane], a1 = sm.g[2 * lane + 1];
+    float incl = a0 + a1;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    const float excl = incl - (a0 + a1);
+    sm.gam[2 * lane] = excl + a0;
+    sm.gam[2 * lane + 1] = incl;
+    sm.eg[2 * lane] = expf(excl + a0);
+    sm.eg[2 * lane + 1] = expf(incl);
+  }
+  cp_wait_all();
+  __syncthreads();
+  for (int p = warp; p < 64; p += nw) {
+    float qq = 0.f, kk = 0.f;
+    for (int d = lane; d < Dk; d += 32) {
+      const float qv = bf(sQ[p * lbk + d]), kv = bf(sK[p * lbk + d]);
+      qq = fmaf(qv, qv, qq);
+      kk = fmaf(kv, kv, kk);
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) {
+      qq += __shfl_xor_sync(0xffffffffu, qq, off);
+      kk += __shfl_xor_sync(0xffffffffu, kk, off);
+    }
+    const float rq = 1.f / sqrtf(fmaxf(qq, 1e-12f)), rk = 1.f / sqrtf(fmaxf(kk, 1e-12f));
+    for (int d = lane; d < Dk; d += 32) {
+      sQ[p * lbk + d] = __float2bfloat16_rn(bf(sQ[p * lbk + d]) * rq);
+      sK[p * lbk + d] = __float2bfloat16_rn(bf(sK[p * lbk + d]) * rk);
+    }
+  }
+  __syncthreads();
+}
+
+// ---------------------------------------------------------------- pre pass
+// Every chunk at once: X = P^T dO and Y = Q^^T diag(e^gam) dO, which do not
+// depend on the later chunks, stored transposed (X^T = dO^T P, Y^T = dO^T
+// diag(e^gam) Q^) in bf16.  Shared memory: q^, k^, dO, diag(e^gam) Q^, P (bf16).
+struct PreLayout {
+  int lbk, lbv;
+  uint32_t q, k, dout, qs, P, small, total;
+  __host__ __device__ PreLayout(int Dk, int Dv) {
+    lbk = Dk + 8;
+    lbv = Dv + 8;
+    uint32_t o = 0;
+    q = o;    o += 64 * lbk * 2;
+    k = o;    o += 64 * lbk * 2;
+    dout = o; o += 64 * lbv * 2;
+    qs = o;   o += 64 * lbk * 2;    // diag(e^gam) Q^ (bf16)
+    P = o;    o += 64 * kLdE * 2;   // M o (Q^ K^^T) (bf16)
+    small = o; o += sizeof(BcSmall);
+    total = (o + 15) & ~15u;
+  }
+};
+
+__global__ void __launch_bounds__(kBcThreads) gdn_bwd_pre_kernel(BcArgs a) {
+  extern __shared__ __align__(16) uint8_t bp_raw[];
+  using bf16 = __nv_bfloat16;
+  const int Dk = a.Dk, Dv = a.Dv;
+  const PreLayout L(Dk, Dv);
+  bf16* sQ = reinterpret_cast<bf16*>(bp_raw + L.q);
+  bf16* sK = reinterpret_cast<bf16*>(bp_raw + L.k);
+  bf16* sO = reinterpret_cast<bf16*>(bp_raw + L.dout);
+  bf16* sQs = reinterpret_cast<bf16*>(bp_raw + L.qs);
+  bf16* sP = reinterpret_cast<bf16*>(bp_raw + L.P);
+  BcSmall& sm = *reinterpret_cast<BcSmall*>(bp_raw + L.small);
+  const int j = blockIdx.x, bh = blockIdx.y, dir = blockIdx.z;
+  const int b = bh / a.H, h = bh - b * a.H;
+  const int lbk = L.lbk, lbv = L.lbv;
+  stage_rows(a, sm, sQ, sK, sO, lbk, lbv, b, h, dir, j);
+  for (int e = threadIdx.x; e < 64 * Dk / 2; e += blockDim.x) {
+    const int p = e / (Dk / 2), d = 2 * (e - p * (Dk / 2));
+    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(sQ + p * lbk + d);
+    *reinterpret_cast<__nv_bfloat162*>(sQs + p * lbk + d) =
+        __floats2bfloat162_rn(__low2float(x) * sm.eg[p], __high2float(x) * sm.eg[p]);
+  }
+  auto none = [](int, int, float) { return 0.f; };
+  const BMat Q{sQ, lbk}, K{sK, lbk}, O{sO, lbv}, Qs{sQs, lbk}, Pm{sP, kLdE};
+  gemm2<false, true, false, true>(64, 64, Q, K, Dk, Q, K, 0, none, [&](int m, int n, float v) {
+    sP[m * kLdE + n] = __float2bfloat16_rn(n <= m ? expf(sm.gam[m] - sm.gam[n]) * v : 0.f);
+  }, nullptr, nullptr);
+  __syncthreads();
+  const size_t blk = a.blk(dir, bh, j);
+  gemm_store_bf16<true, false>(Dv, 64, O, Pm, 64, a.XT + blk * Dv * 64, 64);
+  gemm_store_bf16<true, false>(Dv, Dk, O, Qs, 64, a.YT + blk * Dv * Dk, Dk);
+}
+
+// -------------------------------------------------------------- chain pass
+// One CTA per (kChSlices slices of 16 columns of dS, b*h, direction): four
+// warps per slice and one producer warp, the chunks in reverse scan order.
+// A slice runs on the transposed gradient state dS^T (16 x Dk) held in
+// mma.sync accumulators.  An accumulator block of dS^T, packed to bf16, is
+// the A fragment of the same block, so the slice's warps trade their blocks
+// through shared memory in fragment order and nothing is transposed:
+//   dU^T  = X^T + dS_e^T K~^T                  (16 x 64, K = Dk; warp w: tokens 16w ..)
+//   dS0^T = e^{gam_C} dS_e^T + Y^T - dU^T W    (16 x Dk, K = 64; warp w: k16 blocks w, w + 4)
+// B fragments come from the staged W and K~ tiles by ldmatrix (the
+// workspace's [slab][time row][8] layout; a lane's row address picks the
+// scan-order token).  W, K~ and e^{gam_C} arrive by one bulk copy per chunk
+// and the slices' X^T and Y^T columns by one each, into kChStages stages
+// that the producer refills as the slices release them.  Each step writes
+// the chunk's dS_e^T and dU^T (bf16) for the gradient pass.
+constexpr int kChSlices = 2;  // slices per CTA (they share one W, K~ stage)
+constexpr int kChStages = 2;
+constexpr int kChThreads = 32 * (4 * kChSlices + 1);
+constexpr long long kChDrainPolls = 1LL << 40;  // drains are bounded by the 2 s timer
+
+struct ChainBarsBwd {
+  uint64_t full[kChStages], empty[kChStages];
+  int fail[kChSlices];  // a bounded wait of the slice's warps expired
+};
+static_assert(sizeof(ChainBarsBwd) <= 128, "the chain's barriers fit their slot");
+
+struct ChainSmem {
+  uint32_t xs, xu, stage0, stage, xt, yt, total;
+  __host__ __device__ explicit ChainSmem(int Dk) {
+    xs = 128;                                   // dS_e^T A fragments: [slice][Dk/16][32 lanes][16 B]
+    xu = xs + kChSlices * (Dk / 16) * 512;      // dU^T A fragments: [slice][4][32 lanes][16 B]
+    stage0 = (xu + kChSlices * 2048 + 127) & ~127u;
+    xt = (Dk * 256 + 16 + 127) & ~127u;         // after W, K~ and e^{gam_C}
+    yt = xt + kChSlices * 16 * 64 * 2;
+    stage = (yt + kChSlices * 16 * Dk * 2 + 127) & ~127u;
+    total = stage0 + kChStages * stage;
+  }
+};
+
+// The producer (one thread): chunk step s into stage s % kChStages once
+// every active slice has released the stage's previous chunk.
+__device__ void bwd_chain_loads(const BcArgs& a, uint8_t* smem, const ChainSmem& L, int active,
+                                int s0, int bh, int dir) {
+  ChainBarsBwd& bars = *reinterpret_cast<ChainBarsBwd*>(smem);
+  const int Dk = a.Dk, Dv = a.Dv, nC = a.nC;
+  const uint32_t wk_bytes = Dk * 256 + 16;
+  const uint32_t xt_bytes = active * 16 * 64 * 2, yt_bytes = active * 16 * Dk * 2;
+  int issued = 0;
+  bool ok = true;
+  for (; issued < nC; ++issued) {
+    const int st = issued % kChStages;
+    if (issued >= kChStages &&
+        !mbar_wait(&bars.empty[st], ((issued / kChStages) - 1) & 1, a.limit)) {
+      ok = false;
+      break;
+    }
+    const size_t blk = a.blk(dir, bh, dir == 0 ? nC - 1 - issued : issued);
+    uint8_t* dst = smem + L.stage0 + st * L.stage;
+    mbar_arrive_expect_tx(&bars.full[st], wk_bytes + xt_bytes + yt_bytes);
+    bulk_load(dst, a.ws + blk * a.wl.block_bytes + a.wl.off_w, wk_bytes, &bars.full[st]);
+    bulk_load(dst + L.xt, a.XT + (blk * Dv + 16 * s0) * 64, xt_bytes, &bars.full[st]);
+    bulk_load(dst + L.yt, a.YT + (blk * Dv + 16 * s0) * Dk, yt_bytes, &bars.full[st]);
+  }
+  if (!ok) atomicOr(a.err, kErrTimeout);
+  // nothing may still be landing in shared memory when the CTA leaves
+  for (int st = 0; st < kChStages && st < issued; ++st) {
+    const int last = st + ((issued - 1 - st) / kChStages) * kChStages;
+    mbar_wait(&bars.full[st], (last / kChStages) & 1, kChDrainPolls);
+  }
+}
+
+template <int NKB>
+__global__ void __launch_bounds__(kChThreads, 2) gdn_bwd_chain_kernel(BcArgs a) {
+  extern __shared__ __align__(128) uint8_t bch_raw[];
+  ChainBarsBwd& bars = *reinterpret_cast<ChainBarsBwd*>(bch_raw);
+  constexpr int Dk = 16 * NKB;
+  constexpr int KPW = (NKB + 3) / 4;  // k16 blocks of dS^T per warp
+  const int Dv = a.Dv;
+  const ChainSmem L(Dk);
+  const int bh = blockIdx.y, dir = blockIdx.z, s0 = blockIdx.x * kChSlices;
+  const int active = min(kChSlices, Dv / 16 - s0);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kChStages; ++i) {
+      mbar_init(&bars.full[i], 1);
+      mbar_init(&bars.empty[i], 4 * active);
+    }
+    for (int i = 0; i < kChSlices; ++i) bars.fail[i] = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == 4 * kChSlices) {
+    if (lane == 0) bwd_chain_loads(a, bch_raw, L, active, s0, bh, dir);
+    return;
+  }
+  const int g = warp >> 2, q = warp & 3;
+  if (g >= active) return;
+  const int c0 = 16 * (s0 + g), gq = lane >> 2, tq = lane & 3;
+  const uint32_t xs_u = smem_u32(bch_raw + L.xs + g * NKB * 512) + lane * 16;
+  const uint32_t xu_u = smem_u32(bch_raw + L.xu + g * 2048) + lane * 16;
+  volatile int* fail = &bars.fail[g];
+  // the lane's ldmatrix row addresses in a W / K~ tile (time rows; scan row
+  // p is time row p, or 63 - p in the reverse direction)
+  const int mi = lane >> 3, r8 = lane & 7;
+  auto trow = [&](int p) { return dir == 0 ? p : 63 - p; };
+  const uint32_t k_off = (mi & 1) * 1024 + trow(16 * q + 8 * (mi >> 1) + r8) * 16;
+  uint32_t w_off[4];
+#pragma unroll
+  for (int kt = 0; kt < 4; ++kt) w_off[kt] = (mi >> 1) * 1024 + trow(16 * kt + 8 * (mi & 1) + r8) * 16;
+
+  // dS^T blocks kb = q + 4 i: S[i][h][e] is (column gq + 8 (e >> 1), row d =
+  // 16 kb + 8 h + 2 tq + (e & 1)) of dS
+  float S[KPW][2][4];
+#pragma unroll
+  for (int i = 0; i < KPW; ++i)
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int kb = q + 4 * i, col = gq + 8 * (e >> 1), d = 16 * kb + 8 * h + 2 * tq + (e & 1);
+        S[i][h][e] = (kb < NKB && dir == 0 && a.d_state_out)
+                         ? a.d_state_out[((size_t)bh * Dk + d) * Dv + c0 + col]
+                         : 0.f;
+      }
+  int st = 0;
+  uint32_t ph = 0;
+  bool ok = true;
+  for (int s = 0; s < a.nC; ++s) {
+    const size_t blk = a.blk(dir, bh, dir == 0 ? a.nC - 1 - s : s);
+    // dS_e^T (the state entering this chunk) to the slice's warps, in
+    // fragment order, and to the gradient pass
+    uint32_t* dse = reinterpret_cast<uint32_t*>(a.dSeT + (blk * Dv + c0) * Dk);
+#pragma unroll
+    for (int i = 0; i < KPW; ++i) {
+      const int kb = q + 4 * i;
+      if (kb < NKB) {
+        const uint32_t f[4] = {pack_bf16x2(S[i][0][0], S[i][0][1]), pack_bf16x2(S[i][0][2], S[i][0][3]),
+                               pack_bf16x2(S[i][1][0], S[i][1][1]), pack_bf16x2(S[i][1][2], S[i][1][3])};
+        st_shared_v4(xs_u + kb * 512, f);
+        const int d = 16 * kb + 2 * tq;
+        dse[(gq * Dk + d) >> 1] = f[0];
+        dse[((gq + 8) * Dk + d) >> 1] = f[1];
+        dse[(gq * Dk + d + 8) >> 1] = f[2];
+        dse[((gq + 8) * Dk + d + 8) >> 1] = f[3];
+      }
+    }
+    const bool okw = __all_sync(0xffffffffu, mbar_wait(&bars.full[st], ph, a.limit));
+    uint8_t* sb = bch_raw + L.stage0 + st * L.stage;
+    float u[2][4];
+    if (okw) {
+      // X^T starts dU^T, and e^{gam_C} dS_e^T + Y^T starts dS0^T
+      const __nv_bfloat16* xt = reinterpret_cast<const __nv_bfloat16*>(sb + L.xt) + g * 16 * 64;
+      const __nv_bfloat16* yt = reinterpret_cast<const __nv_bfloat16*>(sb + L.yt) + g * 16 * Dk;
+      const float decay = *reinterpret_cast<const float*>(sb + Dk * 256);
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr)
+          unpack_bf16x2(*reinterpret_cast<const uint32_t*>(xt + (gq + 8 * rr) * 64 + 16 * q + 8 * h + 2 * tq),
+                        u[h][2 * rr], u[h][2 * rr + 1]);
+#pragma unroll
+      for (int i = 0; i < KPW; ++i) {
+        const int kb = q + 4 * i;
+        if (kb < NKB) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+              float y0, y1;
+              unpack_bf16x2(*reinterpret_cast<const uint32_t*>(yt + (gq + 8 * rr) * Dk + 16 * kb + 8 * h + 2 * tq),
+                            y0, y1);
+              S[i][h][2 * rr] = fmaf(decay, S[i][h][2 * rr], y0);
+              S[i][h][2 * rr + 1] = fmaf(decay, S[i][h][2 * rr + 1], y1);
+            }
+        }
+      }
+    } else if (lane == 0) {
+      *fail = 1;
+    }
+    named_barrier(1 + g, 128);
+    if (*fail) {
+      ok = false;
+      break;
+    }
+    const uint32_t sw = smem_u32(sb), sk = sw + Dk * 128;
+    // ---- dU^T (+)= dS_e^T K~^T over tokens 16 q .. 16 q + 15
+    {
+      uint32_t af[NKB][4], bk[NKB][4];
+#pragma unroll
+      for (int kb = 0; kb < NKB; ++kb) {
+        ld_shared_v4(xs_u + kb * 512, af[kb]);
+        ldmatrix_x4(sk + 2 * kb * 1024 + k_off, bk[kb]);
+      }
+#pragma unroll
+      for (int kb = 0; kb < NKB; ++kb) {
+        mma_16816(u[0], af[kb], bk[kb][0], bk[kb][1]);
+        mma_16816(u[1], af[kb], bk[kb][2], bk[kb][3]);
+      }
+    }
+    {
+      const uint32_t f[4] = {pack_bf16x2(u[0][0], u[0][1]), pack_bf16x2(u[0][2], u[0][3]),
+                             pack_bf16x2(u[1][0], u[1][1]), pack_bf16x2(u[1][2], u[1][3])};
+      st_shared_v4(xu_u + q * 512, f);
+      uint32_t* du = reinterpret_cast<uint32_t*>(a.dUT + (blk * Dv + c0) * 64);
+      const int p = 16 * q + 2 * tq;
+      du[(gq * 64 + p) >> 1] = f[0];
+      du[((gq + 8) * 64 + p) >> 1] = f[1];
+      du[(gq * 64 + p + 8) >> 1] = f[2];
+      du[((gq + 8) * 64 + p + 8) >> 1] = f[3];
+    }
+    named_barrier(1 + g, 128);
+    // ---- dS0^T (+)= -dU^T W over this warp's blocks
+    {
+      uint32_t ua[4][4];
+#pragma unroll
+      for (int kt = 0; kt < 4; ++kt) {
+        ld_shared_v4(xu_u + kt * 512, ua[kt]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) ua[kt][e] ^= 0x80008000u;  // -dU^T
+      }
+#pragma unroll
+      for (int i = 0; i < KPW; ++i) {
+        const int kb = q + 4 * i;
+        if (kb < NKB) {
+          uint32_t bw[4][4];
+#pragma unroll
+          for (int kt = 0; kt < 4; ++kt) ldmatrix_x4_trans(sw + 2 * kb * 1024 + w_off[kt], bw[kt]);
+#pragma unroll
+          for (int kt = 0; kt < 4; ++kt) {
+            mma_16816(S[i][0], ua[kt], bw[kt][0], bw[kt][1]);
+            mma_16816(S[i][1], ua[kt], bw[kt][2], bw[kt][3]);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars.empty[st]);  // this warp's reads of the stage are done
+    if (++st == kChStages) {
+      st = 0;
+      ph ^= 1;
+    }
+  }
+  if (!ok) {
+    if (lane == 0) atomicOr(a.err, kErrTimeout);
+    return;
+  }
+  if (dir == 0 && a.d_state_in) {
+#pragma unroll
+    for (int i = 0; i < KPW; ++i)
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int kb = q + 4 * i, col = gq + 8 * (e >> 1), d = 16 * kb + 8 * h + 2 * tq + (e & 1);
+          if (kb < NKB) a.d_state_in[((size_t)bh * Dk + d) * Dv + c0 + col] = S[i][h][e];
+        }
+  }
+}
+
+using ChainKernel = void (*)(BcArgs);
+ChainKernel chain_kernel_for(int nkb) {
+  switch (nkb) {
+    case 1: return gdn_bwd_chain_kernel<1>;
+    case 2: return gdn_bwd_chain_kernel<2>;
+    case 3: return gdn_bwd_chain_kernel<3>;
+    case 4: return gdn_bwd_chain_kernel<4>;
+    case 5: return gdn_bwd_chain_kernel<5>;
+    case 6: return gdn_bwd_chain_kernel<6>;
+    default: return gdn_bwd_chain_kernel<7>;
+  }
+}
+
+// ----------------------------------------------------------- gradient pass
+// Every chunk at once (one CTA per (chunk, b*h, direction)), from the
+// chunk's dU and dS_e: every product but the chain's.  All product operands
+// are bf16 tiles in shared memory fed to mma.sync.m16n8k16 by ldmatrix (the
+// .trans form where a tile is read transposed); dq^ and dk^ accumulate in
+// registers; the triangular solve runs in fp32 registers per column.
+struct GradLayout {
+  int lbk, lbv;
+  uint32_t q, k, dout, w, ut, u, s0, dse, P, A, Ab, E, dU, dW, small, total;
+  __host__ __device__ GradLayout(int Dk, int Dv) {
+    lbk = Dk + 8;
+    lbv = Dv + 8;
+    uint32_t o = 0;
+    q = o;    o += 64 * lbk * 2;    // q^
+    k = o;    o += 64 * lbk * 2;    // k^
+    dout = o; o += 64 * lbv * 2;    // dO
+    w = o;    o += 64 * lbk * 2;    // W
+    ut = o;   o += 64 * lbv * 2;    // U~
+    u = o;    o += 64 * lbv * 2;    // U
+    s0 = o;   o += Dk * lbv * 2;    // S0 [Dk][Dv]
+    dse = o;  o += Dv * lbk * 2;    // dS_e^T [Dv][Dk]
+    P = o;    o += 64 * kLdE * 2;   // P, then dQK, then dA / dG (bf16)
+    A = o;    o += 64 * kLd64 * 4;  // A (fp32, the solve's matrix)
+    Ab = o;   o += 64 * kLdE * 2;   // A in bf16 (the solve's block updates)
+    E = o;    o += 64 * kLdE * 2;   // e^{gam_p - gam_i} K^ K^T (i < p), bf16
+    dU = o;   o += 64 * lbv * 2;    // dU, then dX_u (bf16)
+    dW = o;   o += 64 * lbk * 2;    // dW, then dX_w (bf16)
+    small = o; o += sizeof(BcSmall);
+    total = (o + 15) & ~15u;
+  }
+};
+
 // A 64 x N product accumulated in registers: block i of warp w is output
 // block w + 8 i; acc[i][h][e] += scale(m) * value.
 template <bool TA, bool TB, class FS>
@@ -566,7 +756,7 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   bf16* sUt = reinterpret_cast<bf16*>(bg_raw + L.ut);
   bf16* sU = reinterpret_cast<bf16*>(bg_raw + L.u);
   bf16* sS0 = reinterpret_cast<bf16*>(bg_raw + L.s0);
-  bf16* sdS = reinterpret_cast<bf16*>(bg_raw + L.dse);
+  bf16* sdST = reinterpret_cast<bf16*>(bg_raw + L.dse);
   bf16* sP = reinterpret_cast<bf16*>(bg_raw + L.P);
   float* sA = reinterpret_cast<float*>(bg_raw + L.A);
   bf16* sAb = reinterpret_cast<bf16*>(bg_raw + L.Ab);
@@ -588,7 +778,7 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   const uint8_t* blk = a.ws + bi * a.wl.block_bytes;
 
   // ---- stage: rows (q^, k^, dO, gates), then W, U~, U, S0 (workspace),
-  //      dS_e, and dU rounded to bf16
+  //      dS_e^T and dU (from dU^T)
   stage_rows(a, sm, sQ, sK, sO, lbk, lbv, b, h, dir, j);
   {
     const int ck = Dk / 8, cv = Dv / 8;
@@ -602,25 +792,28 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
       const int s2 = e / Dk, d = e - s2 * Dk;
       cp16(sS0 + d * lbv + 8 * s2, blk + a.wl.off_s + 16 * (s2 * Dk + d));
     }
-    const bf16* dSe = a.dSe + bi * Dk * Dv;
-    for (int e = tid; e < Dk * cv; e += kGrThreads) {
-      const int d = e / cv, c = e - d * cv;
-      cp16(sdS + d * lbv + 8 * c, dSe + (size_t)d * Dv + 8 * c);
+    const bf16* dSeT = a.dSeT + bi * Dv * Dk;
+    for (int e = tid; e < Dv * ck; e += kGrThreads) {
+      const int c = e / ck, d8 = e - c * ck;
+      cp16(sdST + c * lbk + 8 * d8, dSeT + (size_t)c * Dk + 8 * d8);
     }
-    const float* dUg = a.dU + bi * 64 * Dv;
-    for (int e = tid; e < 64 * (Dv / 4); e += kGrThreads) {
-      const int p = e / (Dv / 4), c = 4 * (e - p * (Dv / 4));
-      const float4 x = *reinterpret_cast<const float4*>(dUg + (size_t)p * Dv + c);
-      __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(sdU + p * lbv + c);
-      o[0] = __floats2bfloat162_rn(x.x, x.y);
-      o[1] = __floats2bfloat162_rn(x.z, x.w);
+    const bf16* dUT = a.dUT + bi * Dv * 64;
+    for (int e = tid; e < Dv * 8; e += kGrThreads) {  // 8 tokens of a column per 16-byte load
+      const int c = e % Dv, p8 = e / Dv;
+      const uint4 x = __ldg(reinterpret_cast<const uint4*>(dUT + (size_t)c * 64 + 8 * p8));
+      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        sdU[(8 * p8 + 2 * i) * lbv + c] = __ushort_as_bfloat16((unsigned short)(w[i] & 0xFFFFu));
+        sdU[(8 * p8 + 2 * i + 1) * lbv + c] = __ushort_as_bfloat16((unsigned short)(w[i] >> 16));
+      }
     }
     cp_wait_all();
   }
   __syncthreads();
   const float gamC = sm.gam[63], eC = expf(gamC);
   const BMat Q{sQ, lbk}, K{sK, lbk}, O{sO, lbv}, Wm{sW, lbk}, Ut{sUt, lbv}, Um{sU, lbv};
-  const BMat S0{sS0, lbv}, dSm{sdS, lbv}, Pm{sP, kLdE}, dUm{sdU, lbv}, dWm{sdW, lbk};
+  const BMat S0{sS0, lbv}, dSTm{sdST, lbk}, Pm{sP, kLdE}, dUm{sdU, lbv}, dWm{sdW, lbk};
   auto none = [](int, int, float) { return 0.f; };
 
   // ---- 1. P = M o (Q^ K^T);  A = beta_p E, E = e^{gam_p - gam_i} K^ K^T (i < p)
@@ -640,13 +833,13 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
     zero2(dk[i]);
     zero2(dq[i]);
   }
-  gemm_acc2<false, true>(Dk, Dv, Um, dSm, dk, [&](int m) { return expf(gamC - sm.gam[m]); });
+  gemm_acc2<false, false>(Dk, Dv, Um, dSTm, dk, [&](int m) { return expf(gamC - sm.gam[m]); });
   acc_row_sums(Dk, sm.cK, [&](int i, int hh, int e, int m, int n) { return bf(sK[m * lbk + n]) * dk[i][hh][e]; });
   {  // <dS_e, S0> -> dgam_C
     float dot = 0.f;
     for (int e = tid; e < Dk * Dv; e += kGrThreads) {
-      const int d = e / Dv, c = e - d * Dv;
-      dot = fmaf(bf(sdS[d * lbv + c]), bf(sS0[d * lbv + c]), dot);
+      const int c = e / Dk, d = e - c * Dk;
+      dot = fmaf(bf(sdST[c * lbk + d]), bf(sS0[d * lbv + c]), dot);
     }
 #pragma unroll
     for (int off = 16; off; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
@@ -818,17 +1011,17 @@ bool bwd_chunked_fits(int Dk, int Dv) {
 
 namespace {
 struct BwdScratch {
-  size_t fwd, x, y, du, dse, pq, pk, pab, dvb, total;
+  size_t fwd, xt, yt, dut, dset, pq, pk, pab, dvb, total;
   BwdScratch(int B, int T, int H, int Dk, int Dv, bool bidir) {
     const size_t ndir = bidir ? 2 : 1, rows = (size_t)B * T * H, NBH = (size_t)B * H;
     const size_t blocks = ndir * NBH * ((T + 63) / 64);
     auto al = [](size_t n) { return (n + 255) & ~size_t(255); };
     size_t o = 0;
     fwd = o; o += al(chunk_tc_workspace_bytes(B, T, H, Dk, Dv, bidir));
-    x = o;   o += al(blocks * 64 * Dv * 4);
-    y = o;   o += al(blocks * (size_t)Dk * Dv * 4);
-    du = o;  o += al(blocks * 64 * Dv * 4);
-    dse = o; o += al(blocks * (size_t)Dk * Dv * 2);
+    xt = o;   o += al(blocks * 64 * Dv * 2);
+    yt = o;   o += al(blocks * (size_t)Dk * Dv * 2);
+    dut = o;  o += al(blocks * 64 * Dv * 2);
+    dset = o; o += al(blocks * (size_t)Dk * Dv * 2);
     pq = o;  o += al(ndir * rows * Dk * 4);
     pk = o;  o += al(ndir * rows * Dk * 4);
     pab = o; o += al(ndir * rows * 2 * 4);
@@ -868,10 +1061,12 @@ cudaError_t launch_backward_chunked(const BwdCall& c, void* workspace, float** p
   a.d_state_out = c.d_state_out; a.d_state_in = c.d_state_in;
   a.ws = base + W.fwd;
   a.wl = chunk_tc_ws_layout(c.Dk, c.Dv);
-  a.X = reinterpret_cast<float*>(base + W.x);
-  a.Y = reinterpret_cast<float*>(base + W.y);
-  a.dU = reinterpret_cast<float*>(base + W.du);
-  a.dSe = reinterpret_cast<__nv_bfloat16*>(base + W.dse);
+  a.XT = reinterpret_cast<__nv_bfloat16*>(base + W.xt);
+  a.YT = reinterpret_cast<__nv_bfloat16*>(base + W.yt);
+  a.dUT = reinterpret_cast<__nv_bfloat16*>(base + W.dut);
+  a.dSeT = reinterpret_cast<__nv_bfloat16*>(base + W.dset);
+  a.err = c.err;
+  a.limit = c.wait_limit;
   a.pq = reinterpret_cast<float*>(base + W.pq);
   a.pk = reinterpret_cast<float*>(base + W.pk);
   a.pab = reinterpret_cast<float*>(base + W.pab);
@@ -881,11 +1076,16 @@ cudaError_t launch_backward_chunked(const BwdCall& c, void* workspace, float** p
   a.NBH = (int)NBH;
   *pq = a.pq; *pk = a.pk; *pab = a.pab; *dvb = a.dvb;
   const int smem_pre = (int)PreLayout(c.Dk, c.Dv).total;
-  const int smem_chain = (int)ChainLayout2(c.Dk).total;
+  const int smem_chain = (int)ChainSmem(c.Dk).total;
+  const ChainKernel chain = chain_kernel_for(c.Dk / 16);
+  // the chain copies W, K~ and e^{gam_C} of a chunk as one span
+  if (a.wl.off_kt != a.wl.off_w + 128u * c.Dk || a.wl.off_decay != a.wl.off_kt + 128u * c.Dk ||
+      a.wl.off_w % 16 != 0)
+    return cudaErrorInvalidValue;
   const int smem_grad = (int)GradLayout(c.Dk, c.Dv).total;
   if ((e = cudaFuncSetAttribute(gdn_bwd_pre_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 smem_pre)) != cudaSuccess ||
-      (e = cudaFuncSetAttribute(gdn_bwd_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      (e = cudaFuncSetAttribute(chain, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 smem_chain)) != cudaSuccess ||
       (e = cudaFuncSetAttribute(gdn_bwd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 smem_grad)) != cudaSuccess)
@@ -898,7 +1098,8 @@ cudaError_t launch_backward_chunked(const BwdCall& c, void* workspace, float** p
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   {
     ProfileScope ps(c.stream, kKernBwdChain);
-    gdn_bwd_chain_kernel<<<dim3(c.Dv / kChCols, (unsigned)NBH, ndir), kChThreads, smem_chain, c.stream>>>(a);
+    const unsigned groups = (unsigned)((c.Dv / 16 + kChSlices - 1) / kChSlices);
+    chain<<<dim3(groups, (unsigned)NBH, ndir), kChThreads, smem_chain, c.stream>>>(a);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   {

@@ -578,21 +578,6 @@ struct ChainBars {
   int fail[kChainMaxGroups];                       // a bounded wait of the group expired
 };
 
-__device__ __forceinline__ void unpack_bf16x2(uint32_t u, float& lo, float& hi) {
-  lo = __uint_as_float(u << 16);
-  hi = __uint_as_float(u & 0xFFFF0000u);
-}
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint32_t (&r)[4]) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(r[0]), "r"(r[1]),
-               "r"(r[2]), "r"(r[3])
-               : "memory");
-}
-__device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr)
-               : "memory");
-}
 
 // What one launch of the chain kernel does (one pass of stage B):
 //  * publish pass: walk each time segment of the chunk sequence from its
