@@ -360,7 +360,9 @@ __device__ __forceinline__ void st_io(__nv_bfloat16* p, float x) { *p = __float2
 // Sum the partials of every slice and direction for one (b, t, h) row, apply
 // the normalisation's Jacobian, and write dq, dk, dv, dg, dbeta.
 // pab[..][0] holds dL/da (token-serial path: dg = e^g da) or dL/dg itself
-// (chunked path, `pab_is_dg`).  One warp per (b, t, h) row, four rows per
+// (chunked path, `chunked`).  dvb holds dv itself, or (chunked path) the
+// gradient of the rows of X_u = diag(beta) V: then dv = beta dX_u and beta
+// gains v . dX_u.  One warp per (b, t, h) row, four rows per
 // block; lane l holds elements 4 l .. 4 l + 3 (D <= 128), read 16 bytes at a
 // time from the fp32 partials.
 constexpr int kRedRows = 4;
@@ -386,7 +388,7 @@ __device__ __forceinline__ void st4_io(__nv_bfloat16* p, const float (&x)[4]) {
 template <typename IO>
 __global__ void __launch_bounds__(32 * kRedRows)
 gdn_bwd_reduce_kernel(BwdArgs A, int ndir, void* dq_, void* dk_, void* dv_, float* dg, float* dbeta,
-                      int pab_is_dg) {
+                      int chunked) {
   const size_t rows_bth = (size_t)A.B * A.T * A.H;
   const size_t row = (size_t)blockIdx.x * kRedRows + (threadIdx.x >> 5);
   if (row >= rows_bth) return;  // whole warps
@@ -440,6 +442,7 @@ gdn_bwd_reduce_kernel(BwdArgs A, int ndir, void* dq_, void* dk_, void* dv_, floa
     st4_io(dq + row * Dk + c, oq);
     st4_io(dk + row * Dk + c, ok);
   }
+  float vdx = 0.f;  // v . dX_u (chunked path)
   if (c < Dv) {
     float sv[4] = {0.f, 0.f, 0.f, 0.f};
     for (int d = 0; d < ndir; ++d) {
@@ -448,8 +451,21 @@ gdn_bwd_reduce_kernel(BwdArgs A, int ndir, void* dq_, void* dk_, void* dv_, floa
 #pragma unroll
       for (int e = 0; e < 4; ++e) sv[e] += x[e];
     }
+    if (chunked) {
+      float vi[4];
+      ld4_io(static_cast<const IO*>(A.v) + row * Dv + c, vi);
+      const float bt = __ldg(A.beta + row);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        vdx = fmaf(vi[e], sv[e], vdx);
+        sv[e] *= bt;
+      }
+    }
     st4_io(dv + row * Dv + c, sv);
   }
+  if (chunked)
+#pragma unroll
+    for (int off = 16; off; off >>= 1) vdx += __shfl_xor_sync(0xffffffffu, vdx, off);
   if (lane == 0) {
     float da = 0.f, db = 0.f;
     for (int d = 0; d < ndir; ++d)
@@ -458,8 +474,8 @@ gdn_bwd_reduce_kernel(BwdArgs A, int ndir, void* dq_, void* dk_, void* dv_, floa
         da += A.pab[(base + row) * 2];
         db += A.pab[(base + row) * 2 + 1];
       }
-    dg[row] = pab_is_dg ? da : expf(__ldg(A.g + row)) * da;
-    dbeta[row] = db;
+    dg[row] = chunked ? da : expf(__ldg(A.g + row)) * da;
+    dbeta[row] = db + vdx;
   }
 }
 

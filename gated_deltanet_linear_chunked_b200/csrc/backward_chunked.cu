@@ -28,15 +28,18 @@
 // K~, U~, U and S0 of every chunk (their workspace).  Only dU and dS0 depend
 // on the chunks after this one, so three kernels share the work:
 //   gdn_bwd_pre_kernel    every chunk at once: X = P^T dO, Y = Q^^T diag(e^gam) dO
+//                         (stored transposed, bf16)
 //   gdn_bwd_chain_kernel  per (16 columns of dS, b*h, direction), the chunks in
 //                         reverse: dU = X + K~ dS_e, dS0 = e^{gam_C} dS_e + Y - W^T dU
-//                         (the columns of dS evolve independently; fp32), each
-//                         chunk's dU and dS_e stored
+//                         (the columns of dS evolve independently; the state in
+//                         fp32 accumulators), each chunk's dU and dS_e stored (bf16)
 //   gdn_bwd_grad_kernel   every chunk at once: the other products, from that
 //                         chunk's dU and dS_e
-// all on tf32 mma.sync (fp32 accumulate).  dq^ and dk^ (before the
-// normalisation's Jacobian), dv, dg and dbeta of each direction go to
-// per-direction partials that the reduction kernel of backward.cu sums.
+// all on bf16 mma.sync.m16n8k16 (fp32 accumulate) fed by ldmatrix or by
+// fragments held in registers.  dq^ and dk^ (before the normalisation's
+// Jacobian), dX_u, dg and dbeta of each direction go to per-direction
+// partials that the reduction kernel of backward.cu sums (forming dv =
+// diag(beta) dX_u and beta's share v . dX_u there).
 #include <cuda_bf16.h>
 
 #include "gdn_internal.h"
@@ -48,7 +51,6 @@ namespace {
 using namespace sm100;
 
 constexpr int kBcThreads = 256;
-constexpr int kBcWarps = kBcThreads / 32;
 constexpr int kLd64 = 68;   // fp32 row stride of the 64 x 64 tiles
 constexpr int kLdE = 72;    // bf16 row stride of the 64 x 64 E tile
 // The gradient pass runs 16 warps: every phase has many independent 16 x 16
@@ -72,21 +74,17 @@ struct BcArgs {
   WsLayout wl;
   // per (direction, b*h, time chunk), rows in scan order:
   // (all bf16, transposed so that a slice of 16 columns is contiguous):
-  __nv_bfloat16* XT;         // [Dv][64]  (P^T dO)^T
-  __nv_bfloat16* YT;         // [Dv][Dk]  (Q^^T diag(e^gam) dO)^T
+  __nv_bfloat16* XT;         // (P^T dO)^T, Dv x 64 in fragment order [Dv/16][4][32 lanes][8]
+  __nv_bfloat16* YT;         // (Q^^T diag(e^gam) dO)^T, Dv x Dk, [Dv/16][Dk/16][32][8]
   __nv_bfloat16* dUT;        // [Dv][64]  dU^T
   __nv_bfloat16* dSeT;       // [Dv][Dk]  dS_e^T, dS_e the gradient of the chunk's end state
-  float *pq, *pk, *pab, *dvb;  // [dir][rows][Dk], [dir][rows][Dk], [dir][rows][2], [dir][rows][Dv]
+  float *pq, *pk, *pab, *dvb;  // [dir][rows][Dk], [dir][rows][Dk], [dir][rows][2], [dir][rows][Dv] (dX_u)
   int B, T, H, Dk, Dv, nC, NBH;
   unsigned* err;             // device error word (the chain's bounded waits)
   long long limit;           // polls before a bounded wait gives up
   __device__ size_t blk(int dir, int bh, int j) const { return ((size_t)dir * NBH + bh) * nC + j; }
 };
 
-// tf32 operands are fp32 bit patterns whose low 13 mantissa bits the tensor
-// core ignores: bf16-sourced values are exact, fp32 intermediates are
-// truncated (relative error below 2^-10).
-__device__ __forceinline__ uint32_t tf32(float x) { return __float_as_uint(x); }
 __device__ __forceinline__ float bf(const __nv_bfloat16& x) { return __bfloat162float(x); }
 __device__ __forceinline__ void cp16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
@@ -95,51 +93,15 @@ __device__ __forceinline__ void cp16(void* dst, const void* src) {
                : "memory");
 }
 __device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's committed cp.async groups are pending.
+template <int N>
+__device__ __forceinline__ void cp_wait_group() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// The 16 x 8 tile product D = sum_k A(m0 + i, k) B(k, n0 + j), k < K, on
-// tf32 mma.sync.m16n8k8 (fp32 accumulate).
-// Two neighbouring 16 x 8 tiles (columns n0 and n0 + 8) at once: the A
-// fragment is shared and the two accumulator chains are independent.
-template <class FA, class FB>
-__device__ __forceinline__ void tile_mma(int m0, int n0, int K, FA A, FB B, float (&d)[2][4]) {
-  const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) d[h][0] = d[h][1] = d[h][2] = d[h][3] = 0.f;
-#pragma unroll 2
-  for (int k0 = 0; k0 < K; k0 += 8) {
-    const uint32_t a0 = tf32(A(m0 + gq, k0 + tq)), a1 = tf32(A(m0 + gq + 8, k0 + tq));
-    const uint32_t a2 = tf32(A(m0 + gq, k0 + tq + 4)), a3 = tf32(A(m0 + gq + 8, k0 + tq + 4));
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint32_t b0 = tf32(B(k0 + tq, n0 + 8 * h + gq)), b1 = tf32(B(k0 + tq + 4, n0 + 8 * h + gq));
-      asm volatile(
-          "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
-          "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-          : "+f"(d[h][0]), "+f"(d[h][1]), "+f"(d[h][2]), "+f"(d[h][3])
-          : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-    }
-  }
-}
 // Element e (0..3) of a thread's accumulator tile: row and column offsets.
 __device__ __forceinline__ int tile_row(int e) { return ((threadIdx.x & 31) >> 2) + (e >= 2 ? 8 : 0); }
 __device__ __forceinline__ int tile_col(int e) { return 2 * (threadIdx.x & 3) + (e & 1); }
 
-// Out (M x N) = A B: warps take the 16 x 8 output tiles in turn and hand
-// each element to epi(m, n, value).  M % 16 == N % 8 == K % 8 == 0.
-template <class FA, class FB, class FE>
-__device__ __forceinline__ void gemm(int M, int N, int K, FA A, FB B, FE epi) {
-  const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  const int tn = N >> 4, nt = (M >> 4) * tn;  // 16 x 16 blocks
-  for (int t = warp; t < nt; t += nw) {
-    const int m0 = (t / tn) << 4, n0 = (t % tn) << 4;
-    float d[2][4];
-    tile_mma(m0, n0, K, A, B, d);
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) epi(m0 + tile_row(e), n0 + 8 * h + tile_col(e), d[h][e]);
-  }
-}
 // A bf16 matrix in shared memory, row-major with row stride ld (a multiple
 // of 8).  As the A operand (m x k): element (m, k) = p[m ld + k], or
 // p[k ld + m] when read transposed.  As the B operand (k x n): element
@@ -223,32 +185,36 @@ __device__ __forceinline__ void gemm2(int M, int N, BMat A1, BMat B1, int K1, BM
     }
   }
 }
-// Out (M x N) = A B, stored to global memory as bf16: dst[m ld + n], the two
-// neighbouring columns a thread holds in one 4-byte store.
+// Out (M x N) = A B, stored to global memory as bf16 in mma fragment order:
+// 16 x 16 block (bm, bn) at dst + ((bm (N / 16) + bn) 32 + lane) 8, a lane's
+// eight values being its accumulator pairs (rows gq, gq + 8 of columns
+// 2 tq, 2 tq + 1, then the same of columns 8 + 2 tq, 9 + 2 tq) -- what a warp
+// using the block as its accumulator start, or as an A fragment, loads with
+// one 16-byte access per lane.
 template <bool TA, bool TB>
-__device__ __forceinline__ void gemm_store_bf16(int M, int N, BMat A, BMat B, int K,
-                                                __nv_bfloat16* dst, int ld) {
-  const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+__device__ __forceinline__ void gemm_store_frag(int M, int N, BMat A, BMat B, int K,
+                                                __nv_bfloat16* dst) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   const int tn = N >> 4, nt = (M >> 4) * tn;
   for (int t = warp; t < nt; t += nw) {
     const int m0 = (t / tn) << 4, nb = (t % tn) << 4;
     float dd[2][4];
     zero2(dd);
     blk16<TA, TB>(m0, nb, K, A, B, dd);
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int n = nb + 8 * hh + tile_col(0);
-      *reinterpret_cast<uint32_t*>(dst + (size_t)(m0 + tile_row(0)) * ld + n) = pack_bf16x2(dd[hh][0], dd[hh][1]);
-      *reinterpret_cast<uint32_t*>(dst + (size_t)(m0 + tile_row(2)) * ld + n) = pack_bf16x2(dd[hh][2], dd[hh][3]);
-    }
+    *reinterpret_cast<uint4*>(dst + ((size_t)t * 32 + lane) * 8) =
+        make_uint4(pack_bf16x2(dd[0][0], dd[0][1]), pack_bf16x2(dd[0][2], dd[0][3]),
+                   pack_bf16x2(dd[1][0], dd[1][1]), pack_bf16x2(dd[1][2], dd[1][3]));
   }
 }
 
 // Stage chunk j of (b, h) in direction dir, rows in scan order: gates (zero
 // past T), q^ = q / |q|, k^ likewise (bf16), dO; gam (inclusive prefix sum of
-// g) and e^gam.  Every thread of the CTA takes part; ends with a barrier.
-__device__ void stage_rows(const BcArgs& a, BcSmall& sm, __nv_bfloat16* sQ, __nv_bfloat16* sK,
-                           __nv_bfloat16* sO, int lbk, int lbv, int b, int h, int dir, int j) {
+// g) and e^gam; with sQs, also diag(e^gam) q^ there.  Every thread of the
+// CTA takes part.  stage_rows_issue starts the row copies (one cp.async
+// group); stage_rows_finish<N> waits for them with N later groups still
+// pending, normalises, and ends with a barrier.
+__device__ void stage_rows_issue(const BcArgs& a, BcSmall& sm, __nv_bfloat16* sQ, __nv_bfloat16* sK,
+                                 __nv_bfloat16* sO, int lbk, int lbv, int b, int h, int dir, int j) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
   const int Dk = a.Dk, Dv = a.Dv, t0 = 64 * j;
   if (tid < 64) {
@@ -264,23 +230,26 @@ __device__ void stage_rows(const BcArgs& a, BcSmall& sm, __nv_bfloat16* sQ, __nv
   }
   __syncthreads();
   const int ck = Dk / 8, cv = Dv / 8;
-  for (int e = tid; e < 64 * (2 * ck + cv); e += blockDim.x) {
-    const int p = e / (2 * ck + cv), c = e - p * (2 * ck + cv), r = sm.row[p];
-    __nv_bfloat16* dst;
-    const __nv_bfloat16* src;
-    if (c < ck) {
-      dst = sQ + p * lbk + 8 * c;
-      src = a.q + (size_t)r * Dk + 8 * c;
-    } else if (c < 2 * ck) {
-      dst = sK + p * lbk + 8 * (c - ck);
-      src = a.k + (size_t)r * Dk + 8 * (c - ck);
-    } else {
-      dst = sO + p * lbv + 8 * (c - 2 * ck);
-      src = a.dout + (size_t)r * Dv + 8 * (c - 2 * ck);
+  for (int p = warp; p < 64; p += nw) {  // a row's 16-byte pieces of q, k and dO across the lanes
+    const int r = sm.row[p];
+    for (int c = lane; c < 2 * ck + cv; c += 32) {
+      __nv_bfloat16* dst;
+      const __nv_bfloat16* src;
+      if (c < ck) {
+        dst = sQ + p * lbk + 8 * c;
+        src = a.q + (size_t)r * Dk + 8 * c;
+      } else if (c < 2 * ck) {
+        dst = sK + p * lbk + 8 * (c - ck);
+        src = a.k + (size_t)r * Dk + 8 * (c - ck);
+      } else {
+        dst = sO + p * lbv + 8 * (c - 2 * ck);
+        src = a.dout + (size_t)r * Dv + 8 * (c - 2 * ck);
+      }
+      if (r >= 0) cp16(dst, src);
+      else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
     }
-    if (r >= 0) cp16(dst, src);
-    else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
   }
+  cp_commit();
   if (warp == 0) {
     const float a0 = sm.g[2 * lane], a1 = sm.g[2 * lane + 1];
     float incl = a0 + a1;
@@ -295,14 +264,28 @@ __device__ void stage_rows(const BcArgs& a, BcSmall& sm, __nv_bfloat16* sQ, __nv
     sm.eg[2 * lane] = expf(excl + a0);
     sm.eg[2 * lane + 1] = expf(incl);
   }
-  cp_wait_all();
+}
+template <int N>
+__device__ void stage_rows_finish(const BcArgs& a, BcSmall& sm, __nv_bfloat16* sQ, __nv_bfloat16* sK,
+                                  int lbk, __nv_bfloat16* sQs = nullptr) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int Dk = a.Dk;
+  cp_wait_group<N>();
   __syncthreads();
-  for (int p = warp; p < 64; p += nw) {
+  for (int p = warp; p < 64; p += nw) {  // bf16 pairs: Dk / 2 <= 64, two per lane at most
+    uint32_t* q2 = reinterpret_cast<uint32_t*>(sQ + p * lbk);
+    uint32_t* k2 = reinterpret_cast<uint32_t*>(sK + p * lbk);
+    float qv[2][2] = {}, kv[2][2] = {};
     float qq = 0.f, kk = 0.f;
-    for (int d = lane; d < Dk; d += 32) {
-      const float qv = bf(sQ[p * lbk + d]), kv = bf(sK[p * lbk + d]);
-      qq = fmaf(qv, qv, qq);
-      kk = fmaf(kv, kv, kk);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int d2 = lane + 32 * i;
+      if (d2 < Dk / 2) {
+        unpack_bf16x2(q2[d2], qv[i][0], qv[i][1]);
+        unpack_bf16x2(k2[d2], kv[i][0], kv[i][1]);
+        qq = fmaf(qv[i][0], qv[i][0], fmaf(qv[i][1], qv[i][1], qq));
+        kk = fmaf(kv[i][0], kv[i][0], fmaf(kv[i][1], kv[i][1], kk));
+      }
     }
 #pragma unroll
     for (int off = 16; off; off >>= 1) {
@@ -310,9 +293,19 @@ __device__ void stage_rows(const BcArgs& a, BcSmall& sm, __nv_bfloat16* sQ, __nv
       kk += __shfl_xor_sync(0xffffffffu, kk, off);
     }
     const float rq = 1.f / sqrtf(fmaxf(qq, 1e-12f)), rk = 1.f / sqrtf(fmaxf(kk, 1e-12f));
-    for (int d = lane; d < Dk; d += 32) {
-      sQ[p * lbk + d] = __float2bfloat16_rn(bf(sQ[p * lbk + d]) * rq);
-      sK[p * lbk + d] = __float2bfloat16_rn(bf(sK[p * lbk + d]) * rk);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int d2 = lane + 32 * i;
+      if (d2 < Dk / 2) {
+        const uint32_t qn = pack_bf16x2(qv[i][0] * rq, qv[i][1] * rq);
+        q2[d2] = qn;
+        k2[d2] = pack_bf16x2(kv[i][0] * rk, kv[i][1] * rk);
+        if (sQs) {  // e^gam times the rounded q^
+          float x0, x1;
+          unpack_bf16x2(qn, x0, x1);
+          reinterpret_cast<uint32_t*>(sQs + p * lbk)[d2] = pack_bf16x2(x0 * sm.eg[p], x1 * sm.eg[p]);
+        }
+      }
     }
   }
   __syncthreads();
@@ -353,13 +346,8 @@ __global__ void __launch_bounds__(kBcThreads) gdn_bwd_pre_kernel(BcArgs a) {
   const int j = blockIdx.x, bh = blockIdx.y, dir = blockIdx.z;
   const int b = bh / a.H, h = bh - b * a.H;
   const int lbk = L.lbk, lbv = L.lbv;
-  stage_rows(a, sm, sQ, sK, sO, lbk, lbv, b, h, dir, j);
-  for (int e = threadIdx.x; e < 64 * Dk / 2; e += blockDim.x) {
-    const int p = e / (Dk / 2), d = 2 * (e - p * (Dk / 2));
-    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(sQ + p * lbk + d);
-    *reinterpret_cast<__nv_bfloat162*>(sQs + p * lbk + d) =
-        __floats2bfloat162_rn(__low2float(x) * sm.eg[p], __high2float(x) * sm.eg[p]);
-  }
+  stage_rows_issue(a, sm, sQ, sK, sO, lbk, lbv, b, h, dir, j);
+  stage_rows_finish<0>(a, sm, sQ, sK, lbk, sQs);
   auto none = [](int, int, float) { return 0.f; };
   const BMat Q{sQ, lbk}, K{sK, lbk}, O{sO, lbv}, Qs{sQs, lbk}, Pm{sP, kLdE};
   gemm2<false, true, false, true>(64, 64, Q, K, Dk, Q, K, 0, none, [&](int m, int n, float v) {
@@ -367,8 +355,8 @@ __global__ void __launch_bounds__(kBcThreads) gdn_bwd_pre_kernel(BcArgs a) {
   }, nullptr, nullptr);
   __syncthreads();
   const size_t blk = a.blk(dir, bh, j);
-  gemm_store_bf16<true, false>(Dv, 64, O, Pm, 64, a.XT + blk * Dv * 64, 64);
-  gemm_store_bf16<true, false>(Dv, Dk, O, Qs, 64, a.YT + blk * Dv * Dk, Dk);
+  gemm_store_frag<true, false>(Dv, 64, O, Pm, 64, a.XT + blk * Dv * 64);
+  gemm_store_frag<true, false>(Dv, Dk, O, Qs, 64, a.YT + blk * Dv * Dk);
 }
 
 // -------------------------------------------------------------- chain pass
@@ -521,27 +509,29 @@ __global__ void __launch_bounds__(kChThreads, 2) gdn_bwd_chain_kernel(BcArgs a) 
     uint8_t* sb = bch_raw + L.stage0 + st * L.stage;
     float u[2][4];
     if (okw) {
-      // X^T starts dU^T, and e^{gam_C} dS_e^T + Y^T starts dS0^T
-      const __nv_bfloat16* xt = reinterpret_cast<const __nv_bfloat16*>(sb + L.xt) + g * 16 * 64;
-      const __nv_bfloat16* yt = reinterpret_cast<const __nv_bfloat16*>(sb + L.yt) + g * 16 * Dk;
+      // X^T starts dU^T, and e^{gam_C} dS_e^T + Y^T starts dS0^T (both
+      // stored in fragment order: one 16-byte load per block)
+      const uint32_t xt = smem_u32(sb + L.xt) + g * 2048 + lane * 16;
+      const uint32_t yt = smem_u32(sb + L.yt) + g * NKB * 512 + lane * 16;
       const float decay = *reinterpret_cast<const float*>(sb + Dk * 256);
+      uint32_t xf[4];
+      ld_shared_v4(xt + q * 512, xf);
 #pragma unroll
       for (int h = 0; h < 2; ++h)
 #pragma unroll
-        for (int rr = 0; rr < 2; ++rr)
-          unpack_bf16x2(*reinterpret_cast<const uint32_t*>(xt + (gq + 8 * rr) * 64 + 16 * q + 8 * h + 2 * tq),
-                        u[h][2 * rr], u[h][2 * rr + 1]);
+        for (int rr = 0; rr < 2; ++rr) unpack_bf16x2(xf[2 * h + rr], u[h][2 * rr], u[h][2 * rr + 1]);
 #pragma unroll
       for (int i = 0; i < KPW; ++i) {
         const int kb = q + 4 * i;
         if (kb < NKB) {
+          uint32_t yf[4];
+          ld_shared_v4(yt + kb * 512, yf);
 #pragma unroll
           for (int h = 0; h < 2; ++h)
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr) {
               float y0, y1;
-              unpack_bf16x2(*reinterpret_cast<const uint32_t*>(yt + (gq + 8 * rr) * Dk + 16 * kb + 8 * h + 2 * tq),
-                            y0, y1);
+              unpack_bf16x2(yf[2 * h + rr], y0, y1);
               S[i][h][2 * rr] = fmaf(decay, S[i][h][2 * rr], y0);
               S[i][h][2 * rr + 1] = fmaf(decay, S[i][h][2 * rr + 1], y1);
             }
@@ -744,6 +734,28 @@ __device__ __forceinline__ void acc_row_sums(int N, float* dst, F f) {
   }
 }
 
+// The register blocks to fp32 rows of global memory: dst[rows[m] ld + n] for
+// rows[m] >= 0, a thread's two neighbouring columns per 8-byte store.
+__device__ __forceinline__ void store_acc(int N, const float (&acc)[kMaxBlocks][2][4], float* dst,
+                                          int ld, const int* rows) {
+  const int warp = threadIdx.x >> 5;
+  const int tn = N >> 4, nt = 4 * tn;
+#pragma unroll
+  for (int i = 0; i < kMaxBlocks; ++i) {
+    const int t = warp + kGrWarps * i;
+    if (t < nt) {
+      const int m0 = (t / tn) << 4, n0 = (t % tn) << 4;
+      const int r0 = rows[m0 + tile_row(0)], r1 = rows[m0 + tile_row(2)];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int n = n0 + 8 * hh + tile_col(0);
+        if (r0 >= 0) *reinterpret_cast<float2*>(dst + (size_t)r0 * ld + n) = make_float2(acc[i][hh][0], acc[i][hh][1]);
+        if (r1 >= 0) *reinterpret_cast<float2*>(dst + (size_t)r1 * ld + n) = make_float2(acc[i][hh][2], acc[i][hh][3]);
+      }
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   extern __shared__ __align__(16) uint8_t bg_raw[];
   const int Dk = a.Dk, Dv = a.Dv;
@@ -777,40 +789,36 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   const size_t bi = a.blk(dir, bh, j);
   const uint8_t* blk = a.ws + bi * a.wl.block_bytes;
 
-  // ---- stage: rows (q^, k^, dO, gates), then W, U~, U, S0 (workspace),
-  //      dS_e^T and dU (from dU^T)
-  stage_rows(a, sm, sQ, sK, sO, lbk, lbv, b, h, dir, j);
-  {
-    const int ck = Dk / 8, cv = Dv / 8;
-    for (int e = tid; e < 64 * (ck + 2 * cv); e += kGrThreads) {  // [slab][time row][8] -> [scan row]
-      const int s2 = e >> 6, t = e & 63, p = dir == 0 ? t : 63 - t;
-      if (s2 < ck) cp16(sW + p * lbk + 8 * s2, blk + a.wl.off_w + 16 * (s2 * 64 + t));
-      else if (s2 < ck + cv) cp16(sUt + p * lbv + 8 * (s2 - ck), blk + a.wl.off_ut + 16 * ((s2 - ck) * 64 + t));
-      else cp16(sU + p * lbv + 8 * (s2 - ck - cv), blk + a.wl.off_u + 16 * ((s2 - ck - cv) * 64 + t));
-    }
-    for (int e = tid; e < cv * Dk; e += kGrThreads) {  // S0: [Dv/8][Dk][8] -> [Dk][Dv]
-      const int s2 = e / Dk, d = e - s2 * Dk;
-      cp16(sS0 + d * lbv + 8 * s2, blk + a.wl.off_s + 16 * (s2 * Dk + d));
-    }
-    const bf16* dSeT = a.dSeT + bi * Dv * Dk;
-    for (int e = tid; e < Dv * ck; e += kGrThreads) {
-      const int c = e / ck, d8 = e - c * ck;
-      cp16(sdST + c * lbk + 8 * d8, dSeT + (size_t)c * Dk + 8 * d8);
-    }
-    const bf16* dUT = a.dUT + bi * Dv * 64;
-    for (int e = tid; e < Dv * 8; e += kGrThreads) {  // 8 tokens of a column per 16-byte load
-      const int c = e % Dv, p8 = e / Dv;
-      const uint4 x = __ldg(reinterpret_cast<const uint4*>(dUT + (size_t)c * 64 + 8 * p8));
-      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        sdU[(8 * p8 + 2 * i) * lbv + c] = __ushort_as_bfloat16((unsigned short)(w[i] & 0xFFFFu));
-        sdU[(8 * p8 + 2 * i + 1) * lbv + c] = __ushort_as_bfloat16((unsigned short)(w[i] >> 16));
-      }
-    }
-    cp_wait_all();
+  // ---- stage: rows (q^, k^, dO, gates), then W, U~, U, S0 (workspace) and
+  //      dS_e^T, which land while step 1 runs; dU (from dU^T) after step 1
+  stage_rows_issue(a, sm, sQ, sK, sO, lbk, lbv, b, h, dir, j);
+  const int ck = Dk / 8, cv = Dv / 8;
+  for (int e = tid; e < 64 * (ck + 2 * cv); e += kGrThreads) {  // [slab][time row][8] -> [scan row]
+    const int s2 = e >> 6, t = e & 63, p = dir == 0 ? t : 63 - t;
+    if (s2 < ck) cp16(sW + p * lbk + 8 * s2, blk + a.wl.off_w + 16 * (s2 * 64 + t));
+    else if (s2 < ck + cv) cp16(sUt + p * lbv + 8 * (s2 - ck), blk + a.wl.off_ut + 16 * ((s2 - ck) * 64 + t));
+    else cp16(sU + p * lbv + 8 * (s2 - ck - cv), blk + a.wl.off_u + 16 * ((s2 - ck - cv) * 64 + t));
   }
-  __syncthreads();
+  for (int s2 = warp; s2 < cv; s2 += kGrWarps)  // S0: [Dv/8][Dk][8] -> [Dk][Dv]
+    for (int d = lane; d < Dk; d += 32) cp16(sS0 + d * lbv + 8 * s2, blk + a.wl.off_s + 16 * (s2 * Dk + d));
+  const bf16* dSeT = a.dSeT + bi * Dv * Dk;
+  for (int e = tid; e < Dv * 16; e += kGrThreads) {  // Dk / 8 <= 16 pieces a row
+    const int c = e >> 4, d8 = e & 15;
+    if (d8 < ck) cp16(sdST + c * lbk + 8 * d8, dSeT + (size_t)c * Dk + 8 * d8);
+  }
+  cp_commit();
+  // dU^T: 8 tokens of a column per 16-byte load (Dv <= 128), held in
+  // registers until step 1 is done
+  constexpr int kDuLoads = 128 * 8 / kGrThreads;
+  uint4 du_raw[kDuLoads];
+  const bf16* dUT = a.dUT + bi * Dv * 64;
+#pragma unroll
+  for (int i = 0; i < kDuLoads; ++i) {
+    const int e = tid + kGrThreads * i, c = e & 127, p8 = e >> 7;
+    du_raw[i] = c < Dv ? __ldg(reinterpret_cast<const uint4*>(dUT + (size_t)c * 64 + 8 * p8))
+                       : make_uint4(0, 0, 0, 0);
+  }
+  stage_rows_finish<1>(a, sm, sQ, sK, lbk);
   const float gamC = sm.gam[63], eC = expf(gamC);
   const BMat Q{sQ, lbk}, K{sK, lbk}, O{sO, lbv}, Wm{sW, lbk}, Ut{sUt, lbv}, Um{sU, lbv};
   const BMat S0{sS0, lbv}, dSTm{sdST, lbk}, Pm{sP, kLdE}, dUm{sdU, lbv}, dWm{sdW, lbk};
@@ -826,6 +834,21 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
     sA[m * kLd64 + n] = sm.beta[m] * e;
     sAb[m * kLdE + n] = __float2bfloat16_rn(sm.beta[m] * e);
   }, nullptr, nullptr);
+  // dU rows from the registers, then every staged tile
+#pragma unroll
+  for (int i = 0; i < kDuLoads; ++i) {
+    const int e = tid + kGrThreads * i, c = e & 127, p8 = e >> 7;
+    if (c < Dv) {
+      const uint32_t w[4] = {du_raw[i].x, du_raw[i].y, du_raw[i].z, du_raw[i].w};
+#pragma unroll
+      for (int k2 = 0; k2 < 4; ++k2) {
+        sdU[(8 * p8 + 2 * k2) * lbv + c] = __ushort_as_bfloat16((unsigned short)(w[k2] & 0xFFFFu));
+        sdU[(8 * p8 + 2 * k2 + 1) * lbv + c] = __ushort_as_bfloat16((unsigned short)(w[k2] >> 16));
+      }
+    }
+  }
+  cp_wait_all();
+  __syncthreads();
   // ---- 3. dK~ = U dS_e^T: dk^ starts as e^{gam_C - gam} dK~; c_m = k^_m . dk^_m
   float dk[kMaxBlocks][2][4], dq[kMaxBlocks][2][4];
 #pragma unroll
@@ -837,10 +860,8 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   acc_row_sums(Dk, sm.cK, [&](int i, int hh, int e, int m, int n) { return bf(sK[m * lbk + n]) * dk[i][hh][e]; });
   {  // <dS_e, S0> -> dgam_C
     float dot = 0.f;
-    for (int e = tid; e < Dk * Dv; e += kGrThreads) {
-      const int c = e / Dk, d = e - c * Dk;
-      dot = fmaf(bf(sdST[c * lbk + d]), bf(sS0[d * lbv + c]), dot);
-    }
+    for (int c = warp; c < Dv; c += kGrWarps)
+      for (int d = lane; d < Dk; d += 32) dot = fmaf(bf(sdST[c * lbk + d]), bf(sS0[d * lbv + c]), dot);
 #pragma unroll
     for (int off = 16; off; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
     if (lane == 0) sm.red[warp] = dot;
@@ -864,9 +885,7 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   // ---- 7. dq^ += dQK K^;  8. dk^ += dQK^T Q^
   gemm_acc2<false, false>(Dk, 64, Pm, K, dq, [](int) { return 1.f; });
   gemm_acc2<true, false>(Dk, 64, Pm, Q, dk, [](int) { return 1.f; });
-  for_acc(Dk, [&](int i, int hh, int e, int m, int n) {
-    if (sm.row[m] >= 0) pq[(size_t)sm.row[m] * Dk + n] = dq[i][hh][e];
-  });
+  store_acc(Dk, dq, pq, Dk, sm.row);
   // ---- 9. dW = -dU S0^T
   gemm2<false, true, false, true>(64, Dk, dUm, S0, Dv, dUm, S0, 0, none,
       [&](int m, int n, float v) { sdW[m * lbk + n] = __float2bfloat16_rn(-v); }, nullptr, nullptr);
@@ -884,12 +903,16 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
 #pragma unroll
       for (int p = 0; p < 16; ++p) x[p] = bf(col[p * ld]);
 #pragma unroll
-      for (int p = 14; p >= 0; --p) {
-        float s4[4] = {x[p], 0.f, 0.f, 0.f};
+      for (int t = 15; t > 0; --t) {  // x_t is final: take A[t][p] x_t from the rows p < t
+        const float* arow = sA + (r0 + t) * kLd64 + r0;
 #pragma unroll
-        for (int t = 15; t > p; --t)
-          s4[(15 - t) & 3] = fmaf(-sA[(r0 + t) * kLd64 + r0 + p], x[t], s4[(15 - t) & 3]);
-        x[p] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+        for (int p4 = 0; p4 < t; p4 += 4) {
+          const float4 a4 = *reinterpret_cast<const float4*>(arow + p4);
+          x[p4] = fmaf(-a4.x, x[t], x[p4]);
+          if (p4 + 1 < t) x[p4 + 1] = fmaf(-a4.y, x[t], x[p4 + 1]);
+          if (p4 + 2 < t) x[p4 + 2] = fmaf(-a4.z, x[t], x[p4 + 2]);
+          if (p4 + 3 < t) x[p4 + 3] = fmaf(-a4.w, x[t], x[p4 + 3]);
+        }
       }
 #pragma unroll
       for (int p = 0; p < 16; ++p) col[p * ld] = __float2bfloat16_rn(x[p]);
@@ -909,43 +932,31 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
       __syncthreads();
     }
   }
-  // ---- 11. dk^ += diag(beta e^gam) dX_w;  dv = diag(beta) dX_u;  beta and gam
-  //          from the rows of X_w = diag(beta e^gam) K^ and X_u = diag(beta) V
+  // ---- 11. dk^ += diag(beta e^gam) dX_w; dX_u goes out as it is (the
+  //          reduction forms dv = beta dX_u and beta's share v . dX_u);
+  //          beta and gam from the rows of X_w = diag(beta e^gam) K^
   for_acc(Dk, [&](int i, int hh, int e, int m, int n) {
     dk[i][hh][e] = fmaf(sm.beta[m] * sm.eg[m], bf(sdW[m * lbk + n]), dk[i][hh][e]);
   });
-  // v of this warp's rows, every load issued before any is used
-  float vreg[64 / kGrWarps][4];
-#pragma unroll
-  for (int i = 0; i < 64 / kGrWarps; ++i) {
-    const int r = sm.row[warp + kGrWarps * i];
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-      const int c = lane + 32 * q4;
-      vreg[i][q4] = (r >= 0 && c < Dv) ? __bfloat162float(__ldg(a.v + (size_t)r * Dv + c)) : 0.f;
+  for (int p = warp; p < 64; p += kGrWarps) {
+    const int r = sm.row[p];
+    float sw = 0.f;
+    for (int d2 = lane; d2 < Dk / 2; d2 += 32) {
+      float k0, k1, w0, w1;
+      unpack_bf16x2(reinterpret_cast<const uint32_t*>(sK + p * lbk)[d2], k0, k1);
+      unpack_bf16x2(reinterpret_cast<const uint32_t*>(sdW + p * lbk)[d2], w0, w1);
+      sw = fmaf(k0, w0, fmaf(k1, w1, sw));
     }
-  }
-#pragma unroll
-  for (int i = 0; i < 64 / kGrWarps; ++i) {
-    const int p = warp + kGrWarps * i, r = sm.row[p];
-    float sw = 0.f, su = 0.f;
-    for (int d = lane; d < Dk; d += 32) sw = fmaf(bf(sK[p * lbk + d]), bf(sdW[p * lbk + d]), sw);
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-      const int c = lane + 32 * q4;
-      if (c < Dv) {
-        const float xu = bf(sdU[p * lbv + c]);
-        if (r >= 0) dvb[(size_t)r * Dv + c] = sm.beta[p] * xu;
-        su = fmaf(vreg[i][q4], xu, su);
+    if (r >= 0)
+      for (int c2 = lane; c2 < Dv / 2; c2 += 32) {
+        float x0, x1;
+        unpack_bf16x2(reinterpret_cast<const uint32_t*>(sdU + p * lbv)[c2], x0, x1);
+        *reinterpret_cast<float2*>(dvb + (size_t)r * Dv + 2 * c2) = make_float2(x0, x1);
       }
-    }
 #pragma unroll
-    for (int off = 16; off; off >>= 1) {
-      sw += __shfl_xor_sync(0xffffffffu, sw, off);
-      su += __shfl_xor_sync(0xffffffffu, su, off);
-    }
+    for (int off = 16; off; off >>= 1) sw += __shfl_xor_sync(0xffffffffu, sw, off);
     if (lane == 0) {  // step 12's epilogues may already be adding to these rows
-      atomicAdd(&sm.dbeta[p], sm.eg[p] * sw + su);
+      atomicAdd(&sm.dbeta[p], sm.eg[p] * sw);
       atomicAdd(&sm.dgam[p], sm.beta[p] * sm.eg[p] * sw);
     }
   }
@@ -971,9 +982,7 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   gemm_acc2<false, false>(Dk, 64, Pm, K, dk, [](int) { return 1.f; });
   gemm_acc2<true, false>(Dk, 64, Pm, K, dk, [](int) { return 1.f; });
   // ---- 14. outputs: dk^, dbeta, dg = suffix sum of dgam + dgam_C
-  for_acc(Dk, [&](int i, int hh, int e, int m, int n) {
-    if (sm.row[m] >= 0) pk[(size_t)sm.row[m] * Dk + n] = dk[i][hh][e];
-  });
+  store_acc(Dk, dk, pk, Dk, sm.row);
   __syncthreads();  // every addition to dgam and dbeta is done
   if (warp == 0) {
     // K~ = diag(e^{gam_C - gam}) K^: row p's exponent gives -c_p to gam_p

@@ -122,9 +122,10 @@ struct BwdCall {
 };
 size_t bwd_workspace_bytes(int B, int T, int H, int Dk, int Dv, gdn_dtype dtype, bool bidir);
 cudaError_t launch_backward(const BwdCall& c, void* workspace);
-// bf16 I/O: the chunked backward (forward stages A and B, then one CTA per
-// (b*h, direction) walking the chunks in reverse); returns the partials'
-// addresses in the workspace for the reduction.
+// bf16 I/O: the chunked backward (forward stages A and B, then a pre pass,
+// the reverse chain over the chunks and a chunk-parallel gradient pass);
+// returns the partials' addresses in the workspace for the reduction (dvb
+// holds the gradient of diag(beta) V's rows, not dv).
 bool bwd_chunked_fits(int Dk, int Dv);  // its shared-memory layout fits (Dk, Dv <= 112)
 size_t bwd_chunked_workspace_bytes(int B, int T, int H, int Dk, int Dv, bool bidir);
 cudaError_t launch_backward_chunked(const BwdCall& c, void* workspace, float** pq, float** pk,
