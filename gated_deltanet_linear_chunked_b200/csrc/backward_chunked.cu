@@ -374,7 +374,9 @@ __global__ void __launch_bounds__(kBcThreads) gdn_bwd_pre_kernel(BcArgs a) {
 // and the slices' X^T and Y^T columns by one each, into kChStages stages
 // that the producer refills as the slices release them.  Each step writes
 // the chunk's dS_e^T and dU^T (bf16) for the gradient pass.
-constexpr int kChSlices = 2;  // slices per CTA (they share one W, K~ stage)
+// One slice per CTA: slices sharing a stage would wait for one another, and
+// the step is bound by its dependent MMAs and exchanges, not by the loads.
+constexpr int kChSlices = 1;
 constexpr int kChStages = 2;
 constexpr int kChThreads = 32 * (4 * kChSlices + 1);
 constexpr long long kChDrainPolls = 1LL << 40;  // drains are bounded by the 2 s timer
@@ -546,7 +548,8 @@ __global__ void __launch_bounds__(kChThreads, 2) gdn_bwd_chain_kernel(BcArgs a) 
       break;
     }
     const uint32_t sw = smem_u32(sb), sk = sw + Dk * 128;
-    // ---- dU^T (+)= dS_e^T K~^T over tokens 16 q .. 16 q + 15
+    // ---- dU^T (+)= dS_e^T K~^T over tokens 16 q .. 16 q + 15 (the odd
+    //      k16 blocks in a second accumulator: shorter dependent chains)
     {
       uint32_t af[NKB][4], bk[NKB][4];
 #pragma unroll
@@ -554,11 +557,17 @@ __global__ void __launch_bounds__(kChThreads, 2) gdn_bwd_chain_kernel(BcArgs a) 
         ld_shared_v4(xs_u + kb * 512, af[kb]);
         ldmatrix_x4(sk + 2 * kb * 1024 + k_off, bk[kb]);
       }
+      float u2[2][4] = {};
 #pragma unroll
       for (int kb = 0; kb < NKB; ++kb) {
-        mma_16816(u[0], af[kb], bk[kb][0], bk[kb][1]);
-        mma_16816(u[1], af[kb], bk[kb][2], bk[kb][3]);
+        float (&acc)[2][4] = (kb & 1) ? u2 : u;
+        mma_16816(acc[0], af[kb], bk[kb][0], bk[kb][1]);
+        mma_16816(acc[1], af[kb], bk[kb][2], bk[kb][3]);
       }
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) u[h][e] += u2[h][e];
     }
     {
       const uint32_t f[4] = {pack_bf16x2(u[0][0], u[0][1]), pack_bf16x2(u[0][2], u[0][3]),
@@ -588,11 +597,17 @@ __global__ void __launch_bounds__(kChThreads, 2) gdn_bwd_chain_kernel(BcArgs a) 
           uint32_t bw[4][4];
 #pragma unroll
           for (int kt = 0; kt < 4; ++kt) ldmatrix_x4_trans(sw + 2 * kb * 1024 + w_off[kt], bw[kt]);
+          float s2[2][4] = {};  // token blocks 2, 3 (shorter dependent chains)
 #pragma unroll
           for (int kt = 0; kt < 4; ++kt) {
-            mma_16816(S[i][0], ua[kt], bw[kt][0], bw[kt][1]);
-            mma_16816(S[i][1], ua[kt], bw[kt][2], bw[kt][3]);
+            float (&acc)[2][4] = kt < 2 ? S[i] : s2;
+            mma_16816(acc[0], ua[kt], bw[kt][0], bw[kt][1]);
+            mma_16816(acc[1], ua[kt], bw[kt][2], bw[kt][3]);
           }
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) S[i][h][e] += s2[h][e];
         }
       }
     }
