@@ -51,7 +51,6 @@ namespace {
 using namespace sm100;
 
 constexpr int kBcThreads = 256;
-constexpr int kLd64 = 68;   // fp32 row stride of the 64 x 64 tiles
 constexpr int kLdE = 72;    // bf16 row stride of the 64 x 64 E tile
 // The gradient pass runs 16 warps: every phase has many independent 16 x 16
 // tiles, and with one CTA per SM the extra warps hide their latencies.
@@ -78,6 +77,7 @@ struct BcArgs {
   __nv_bfloat16* YT;         // (Q^^T diag(e^gam) dO)^T, Dv x Dk, [Dv/16][Dk/16][32][8]
   __nv_bfloat16* dUT;        // [Dv][64]  dU^T
   __nv_bfloat16* dSeT;       // [Dv][Dk]  dS_e^T, dS_e the gradient of the chunk's end state
+  const __nv_bfloat16* tinv; // [64][64]  (I + A)^-1 from the forward's stage A (scan order)
   float *pq, *pk, *pab, *dvb;  // [dir][rows][Dk], [dir][rows][Dk], [dir][rows][2], [dir][rows][Dv] (dX_u)
   int B, T, H, Dk, Dv, nC, NBH;
   unsigned* err;             // device error word (the chain's bounded waits)
@@ -111,24 +111,38 @@ struct BMat {
   int ld;
 };
 
-// 16 x 16 output block (m0, n0) += A B over k < K (K % 16 == 0).
+// One k16 step of a 16 x 16 output block (m0, n0): d += A[m0.., k0..] B[k0.., n0..].
+template <bool TA, bool TB>
+__device__ __forceinline__ void step16(int m0, int n0, int k0, BMat A, BMat B, float (&d)[2][4]) {
+  const int l = threadIdx.x & 31;
+  uint32_t a[4], bb[4];
+  if (TA)
+    ldmatrix_x4_trans(smem_u32(A.p + (k0 + (l & 7) + 8 * (l >> 4)) * A.ld + m0 + 8 * ((l >> 3) & 1)), a);
+  else
+    ldmatrix_x4(smem_u32(A.p + (m0 + (l & 15)) * A.ld + k0 + 8 * (l >> 4)), a);
+  if (TB)
+    ldmatrix_x4(smem_u32(B.p + (n0 + (l & 7) + 8 * (l >> 4)) * B.ld + k0 + 8 * ((l >> 3) & 1)), bb);
+  else
+    ldmatrix_x4_trans(smem_u32(B.p + (k0 + (l & 7) + 8 * ((l >> 3) & 1)) * B.ld + n0 + 8 * (l >> 4)), bb);
+  mma_16816(d[0], a, bb[0], bb[1]);
+  mma_16816(d[1], a, bb[2], bb[3]);
+}
+// 16 x 16 output block (m0, n0) += A B over k < K (K % 16 == 0); odd k16
+// steps go to a second accumulator, which halves the dependent MMA chains.
 template <bool TA, bool TB>
 __device__ __forceinline__ void blk16(int m0, int n0, int K, BMat A, BMat B, float (&d)[2][4]) {
-  const int l = threadIdx.x & 31;
-#pragma unroll 2
-  for (int k0 = 0; k0 < K; k0 += 16) {
-    uint32_t a[4], bb[4];
-    if (TA)
-      ldmatrix_x4_trans(smem_u32(A.p + (k0 + (l & 7) + 8 * (l >> 4)) * A.ld + m0 + 8 * ((l >> 3) & 1)), a);
-    else
-      ldmatrix_x4(smem_u32(A.p + (m0 + (l & 15)) * A.ld + k0 + 8 * (l >> 4)), a);
-    if (TB)
-      ldmatrix_x4(smem_u32(B.p + (n0 + (l & 7) + 8 * (l >> 4)) * B.ld + k0 + 8 * ((l >> 3) & 1)), bb);
-    else
-      ldmatrix_x4_trans(smem_u32(B.p + (k0 + (l & 7) + 8 * ((l >> 3) & 1)) * B.ld + n0 + 8 * (l >> 4)), bb);
-    mma_16816(d[0], a, bb[0], bb[1]);
-    mma_16816(d[1], a, bb[2], bb[3]);
+  float e[2][4] = {};
+  int k0 = 0;
+#pragma unroll 1
+  for (; k0 + 32 <= K; k0 += 32) {
+    step16<TA, TB>(m0, n0, k0, A, B, d);
+    step16<TA, TB>(m0, n0, k0 + 16, A, B, e);
   }
+  if (k0 < K) step16<TA, TB>(m0, n0, k0, A, B, d);
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d[h][i] += e[h][i];
 }
 __device__ __forceinline__ void zero2(float (&d)[2][4]) {
 #pragma unroll
@@ -653,28 +667,28 @@ ChainKernel chain_kernel_for(int nkb) {
 // chunk's dU and dS_e: every product but the chain's.  All product operands
 // are bf16 tiles in shared memory fed to mma.sync.m16n8k16 by ldmatrix (the
 // .trans form where a tile is read transposed); dq^ and dk^ accumulate in
-// registers; the triangular solve runs in fp32 registers per column.
+// registers; the triangular solve is the product with the forward's own
+// T = (I + A)^-1, which its stage A leaves in the workspace.
 struct GradLayout {
   int lbk, lbv;
-  uint32_t q, k, dout, w, ut, u, s0, dse, P, A, Ab, E, dU, dW, small, total;
+  uint32_t q, k, dout, w, ut, u, s0, dse, P, Tb, E, dU, dW, small, total;
   __host__ __device__ GradLayout(int Dk, int Dv) {
     lbk = Dk + 8;
     lbv = Dv + 8;
     uint32_t o = 0;
-    q = o;    o += 64 * lbk * 2;    // q^
+    q = o;    o += 64 * lbk * 2;    // q^, then dX_w
     k = o;    o += 64 * lbk * 2;    // k^
-    dout = o; o += 64 * lbv * 2;    // dO
+    dout = o; o += 64 * lbv * 2;    // dO, then dX_u
     w = o;    o += 64 * lbk * 2;    // W
     ut = o;   o += 64 * lbv * 2;    // U~
     u = o;    o += 64 * lbv * 2;    // U
     s0 = o;   o += Dk * lbv * 2;    // S0 [Dk][Dv]
     dse = o;  o += Dv * lbk * 2;    // dS_e^T [Dv][Dk]
     P = o;    o += 64 * kLdE * 2;   // P, then dQK, then dA / dG (bf16)
-    A = o;    o += 64 * kLd64 * 4;  // A (fp32, the solve's matrix)
-    Ab = o;   o += 64 * kLdE * 2;   // A in bf16 (the solve's block updates)
+    Tb = o;   o += 64 * kLdE * 2;   // T = (I + A)^-1 (bf16)
     E = o;    o += 64 * kLdE * 2;   // e^{gam_p - gam_i} K^ K^T (i < p), bf16
-    dU = o;   o += 64 * lbv * 2;    // dU, then dX_u (bf16)
-    dW = o;   o += 64 * lbk * 2;    // dW, then dX_w (bf16)
+    dU = o;   o += 64 * lbv * 2;    // dU (bf16)
+    dW = o;   o += 64 * lbk * 2;    // dW (bf16)
     small = o; o += sizeof(BcSmall);
     total = (o + 15) & ~15u;
   }
@@ -785,8 +799,7 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   bf16* sS0 = reinterpret_cast<bf16*>(bg_raw + L.s0);
   bf16* sdST = reinterpret_cast<bf16*>(bg_raw + L.dse);
   bf16* sP = reinterpret_cast<bf16*>(bg_raw + L.P);
-  float* sA = reinterpret_cast<float*>(bg_raw + L.A);
-  bf16* sAb = reinterpret_cast<bf16*>(bg_raw + L.Ab);
+  bf16* sT = reinterpret_cast<bf16*>(bg_raw + L.Tb);
   bf16* sE = reinterpret_cast<bf16*>(bg_raw + L.E);
   bf16* sdU = reinterpret_cast<bf16*>(bg_raw + L.dU);
   bf16* sdW = reinterpret_cast<bf16*>(bg_raw + L.dW);
@@ -821,6 +834,8 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
     const int c = e >> 4, d8 = e & 15;
     if (d8 < ck) cp16(sdST + c * lbk + 8 * d8, dSeT + (size_t)c * Dk + 8 * d8);
   }
+  const bf16* Tg = a.tinv + bi * 64 * 64;
+  for (int e = tid; e < 64 * 8; e += kGrThreads) cp16(sT + (e >> 3) * kLdE + 8 * (e & 7), Tg + 8 * e);
   cp_commit();
   // dU^T: 8 tokens of a column per 16-byte load (Dv <= 128), held in
   // registers until step 1 is done
@@ -839,15 +854,12 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   const BMat S0{sS0, lbv}, dSTm{sdST, lbk}, Pm{sP, kLdE}, dUm{sdU, lbv}, dWm{sdW, lbk};
   auto none = [](int, int, float) { return 0.f; };
 
-  // ---- 1. P = M o (Q^ K^T);  A = beta_p E, E = e^{gam_p - gam_i} K^ K^T (i < p)
+  // ---- 1. P = M o (Q^ K^T);  E = e^{gam_p - gam_i} K^ K^T (i < p), A = diag(beta) E
   gemm2<false, true, false, true>(64, 64, Q, K, Dk, Q, K, 0, none, [&](int m, int n, float v) {
     sP[m * kLdE + n] = __float2bfloat16_rn(n <= m ? expf(sm.gam[m] - sm.gam[n]) * v : 0.f);
   }, nullptr, nullptr);
   gemm2<false, true, false, true>(64, 64, K, K, Dk, K, K, 0, none, [&](int m, int n, float v) {
-    const float e = n < m ? expf(sm.gam[m] - sm.gam[n]) * v : 0.f;
-    sE[m * kLdE + n] = __float2bfloat16_rn(e);
-    sA[m * kLd64 + n] = sm.beta[m] * e;
-    sAb[m * kLdE + n] = __float2bfloat16_rn(sm.beta[m] * e);
+    sE[m * kLdE + n] = __float2bfloat16_rn(n < m ? expf(sm.gam[m] - sm.gam[n]) * v : 0.f);
   }, nullptr, nullptr);
   // dU rows from the registers, then every staged tile
 #pragma unroll
@@ -879,13 +891,8 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
       for (int d = lane; d < Dk; d += 32) dot = fmaf(bf(sdST[c * lbk + d]), bf(sS0[d * lbv + c]), dot);
 #pragma unroll
     for (int off = 16; off; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-    if (lane == 0) sm.red[warp] = dot;
+    if (lane == 0) sm.red[warp] = dot;  // summed after the last barrier
   }
-  __syncthreads();  // P and A, E complete; every read of dS_e done
-  float dgamC = 0.f;
-#pragma unroll
-  for (int w = 0; w < kGrWarps; ++w) dgamC += sm.red[w];
-  dgamC *= eC;
   // ---- 5. dP = dO U^T -> dQK = M o dP (in place of P); gam gets dP o P
   gemm2<false, true, false, true>(64, 64, O, Um, Dv, O, Um, 0,
       [&](int m, int n, float v) { return n <= m ? v * bf(sP[m * kLdE + n]) : 0.f; },
@@ -905,53 +912,25 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   gemm2<false, true, false, true>(64, Dk, dUm, S0, Dv, dUm, S0, 0, none,
       [&](int m, int n, float v) { sdW[m * lbk + n] = __float2bfloat16_rn(-v); }, nullptr, nullptr);
   __syncthreads();
-  // ---- 10. [dX_w | dX_u] solves (I + A)^T X = [dW | dU], blocked by 16 rows
-  //          from the last: each diagonal block by back-substitution (a
-  //          column per thread, in registers), then the rows above it lose
-  //          A[block rows][above]^T X_block (tensor cores, in place)
-  for (int blk16r = 3; blk16r >= 0; --blk16r) {
-    const int r0 = 16 * blk16r;
-    for (int c = tid; c < Dk + Dv; c += kGrThreads) {
-      bf16* col = (c < Dk ? sdW + c : sdU + (c - Dk)) + r0 * (c < Dk ? lbk : lbv);
-      const int ld = c < Dk ? lbk : lbv;
-      float x[16];
-#pragma unroll
-      for (int p = 0; p < 16; ++p) x[p] = bf(col[p * ld]);
-#pragma unroll
-      for (int t = 15; t > 0; --t) {  // x_t is final: take A[t][p] x_t from the rows p < t
-        const float* arow = sA + (r0 + t) * kLd64 + r0;
-#pragma unroll
-        for (int p4 = 0; p4 < t; p4 += 4) {
-          const float4 a4 = *reinterpret_cast<const float4*>(arow + p4);
-          x[p4] = fmaf(-a4.x, x[t], x[p4]);
-          if (p4 + 1 < t) x[p4 + 1] = fmaf(-a4.y, x[t], x[p4 + 1]);
-          if (p4 + 2 < t) x[p4 + 2] = fmaf(-a4.z, x[t], x[p4 + 2]);
-          if (p4 + 3 < t) x[p4 + 3] = fmaf(-a4.w, x[t], x[p4 + 3]);
-        }
-      }
-#pragma unroll
-      for (int p = 0; p < 16; ++p) col[p * ld] = __float2bfloat16_rn(x[p]);
-    }
-    __syncthreads();
-    if (r0 > 0) {
-      // rows [0, r0) -= A[r0 .. r0+15][rows]^T X[r0 .. r0+15]
-      const BMat Ablk{sAb + r0 * kLdE, kLdE};
-      gemm2<true, false, true, false>(r0, Dk, Ablk, BMat{sdW + r0 * lbk, lbk}, 16, Ablk, Ablk, 0, none,
-          [&](int m, int n, float v) {
-            sdW[m * lbk + n] = __float2bfloat16_rn(bf(sdW[m * lbk + n]) - v);
-          }, nullptr, nullptr);
-      gemm2<true, false, true, false>(r0, Dv, Ablk, BMat{sdU + r0 * lbv, lbv}, 16, Ablk, Ablk, 0, none,
-          [&](int m, int n, float v) {
-            sdU[m * lbv + n] = __float2bfloat16_rn(bf(sdU[m * lbv + n]) - v);
-          }, nullptr, nullptr);
-      __syncthreads();
-    }
+  // ---- 10. [dX_w | dX_u] solves (I + A)^T X = [dW | dU]: X = T^T [dW | dU]
+  //          with the forward's own T, into the tiles of q^ and dO (neither
+  //          is read again)
+  bf16* sXw = sQ;
+  bf16* sXu = sO;
+  {
+    const BMat Tt{sT, kLdE};
+    gemm2<true, false, true, false>(64, Dk, Tt, dWm, 64, Tt, Tt, 0, none,
+        [&](int m, int n, float v) { sXw[m * lbk + n] = __float2bfloat16_rn(v); }, nullptr, nullptr);
+    gemm2<true, false, true, false>(64, Dv, Tt, dUm, 64, Tt, Tt, 0, none,
+        [&](int m, int n, float v) { sXu[m * lbv + n] = __float2bfloat16_rn(v); }, nullptr, nullptr);
   }
+  __syncthreads();
+  const BMat Xw{sXw, lbk}, Xu{sXu, lbv};
   // ---- 11. dk^ += diag(beta e^gam) dX_w; dX_u goes out as it is (the
   //          reduction forms dv = beta dX_u and beta's share v . dX_u);
   //          beta and gam from the rows of X_w = diag(beta e^gam) K^
   for_acc(Dk, [&](int i, int hh, int e, int m, int n) {
-    dk[i][hh][e] = fmaf(sm.beta[m] * sm.eg[m], bf(sdW[m * lbk + n]), dk[i][hh][e]);
+    dk[i][hh][e] = fmaf(sm.beta[m] * sm.eg[m], bf(sXw[m * lbk + n]), dk[i][hh][e]);
   });
   for (int p = warp; p < 64; p += kGrWarps) {
     const int r = sm.row[p];
@@ -959,13 +938,13 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
     for (int d2 = lane; d2 < Dk / 2; d2 += 32) {
       float k0, k1, w0, w1;
       unpack_bf16x2(reinterpret_cast<const uint32_t*>(sK + p * lbk)[d2], k0, k1);
-      unpack_bf16x2(reinterpret_cast<const uint32_t*>(sdW + p * lbk)[d2], w0, w1);
+      unpack_bf16x2(reinterpret_cast<const uint32_t*>(sXw + p * lbk)[d2], w0, w1);
       sw = fmaf(k0, w0, fmaf(k1, w1, sw));
     }
     if (r >= 0)
       for (int c2 = lane; c2 < Dv / 2; c2 += 32) {
         float x0, x1;
-        unpack_bf16x2(reinterpret_cast<const uint32_t*>(sdU + p * lbv)[c2], x0, x1);
+        unpack_bf16x2(reinterpret_cast<const uint32_t*>(sXu + p * lbv)[c2], x0, x1);
         *reinterpret_cast<float2*>(dvb + (size_t)r * Dv + 2 * c2) = make_float2(x0, x1);
       }
 #pragma unroll
@@ -976,8 +955,8 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
     }
   }
   // ---- 12. dA = -(dX_w W^T + dX_u U~^T) on i < p (into P); gam from A
-  gemm2<false, true, false, true>(64, 64, dWm, Wm, Dk, dUm, Ut, Dv,
-      [&](int m, int n, float v) { return n < m ? -v * sA[m * kLd64 + n] : 0.f; },
+  gemm2<false, true, false, true>(64, 64, Xw, Wm, Dk, Xu, Ut, Dv,
+      [&](int m, int n, float v) { return n < m ? -v * sm.beta[m] * bf(sE[m * kLdE + n]) : 0.f; },
       [&](int m, int n, float v) { sP[m * kLdE + n] = __float2bfloat16_rn(n < m ? -v : 0.f); },
       sm.dgam, sm.dgam);
   __syncthreads();
@@ -1005,7 +984,10 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
     float cs = sm.cK[2 * lane] + sm.cK[2 * lane + 1];
 #pragma unroll
     for (int off = 16; off; off >>= 1) cs += __shfl_xor_sync(0xffffffffu, cs, off);
-    const float dC = dgamC + cs;
+    float dgamC = 0.f;  // e^{gam_C} <dS_e, S0>
+#pragma unroll
+    for (int w = 0; w < kGrWarps; ++w) dgamC += sm.red[w];
+    const float dC = eC * dgamC + cs;
     const float d0 = sm.dgam[2 * lane] - sm.cK[2 * lane];
     const float d1 = sm.dgam[2 * lane + 1] - sm.cK[2 * lane + 1];
     float incl = d0 + d1;  // suffix sums over scan positions 2 lane, 2 lane + 1 .. 63
@@ -1035,13 +1017,14 @@ bool bwd_chunked_fits(int Dk, int Dv) {
 
 namespace {
 struct BwdScratch {
-  size_t fwd, xt, yt, dut, dset, pq, pk, pab, dvb, total;
+  size_t fwd, tinv, xt, yt, dut, dset, pq, pk, pab, dvb, total;
   BwdScratch(int B, int T, int H, int Dk, int Dv, bool bidir) {
     const size_t ndir = bidir ? 2 : 1, rows = (size_t)B * T * H, NBH = (size_t)B * H;
     const size_t blocks = ndir * NBH * ((T + 63) / 64);
     auto al = [](size_t n) { return (n + 255) & ~size_t(255); };
     size_t o = 0;
     fwd = o; o += al(chunk_tc_workspace_bytes(B, T, H, Dk, Dv, bidir));
+    tinv = o; o += al(blocks * 64 * 64 * 2);
     xt = o;   o += al(blocks * 64 * Dv * 2);
     yt = o;   o += al(blocks * (size_t)Dk * Dv * 2);
     dut = o;  o += al(blocks * 64 * Dv * 2);
@@ -1073,6 +1056,7 @@ cudaError_t launch_backward_chunked(const BwdCall& c, void* workspace, float** p
   f.B = c.B; f.T = c.T; f.H = c.H; f.Dk = c.Dk; f.Dv = c.Dv;
   f.dtype = GDN_BF16; f.chunk = 64; f.bidir = c.bidir; f.gate_logits = false;
   f.stream = c.stream; f.err = c.err; f.wait_limit = c.wait_limit; f.skip_output = true;
+  f.t_out = base + W.tinv;
   cudaError_t e = launch_chunk_tc(f, base + W.fwd);
   if (e != cudaSuccess) return e;
 
@@ -1085,6 +1069,7 @@ cudaError_t launch_backward_chunked(const BwdCall& c, void* workspace, float** p
   a.d_state_out = c.d_state_out; a.d_state_in = c.d_state_in;
   a.ws = base + W.fwd;
   a.wl = chunk_tc_ws_layout(c.Dk, c.Dv);
+  a.tinv = reinterpret_cast<const __nv_bfloat16*>(base + W.tinv);
   a.XT = reinterpret_cast<__nv_bfloat16*>(base + W.xt);
   a.YT = reinterpret_cast<__nv_bfloat16*>(base + W.yt);
   a.dUT = reinterpret_cast<__nv_bfloat16*>(base + W.dut);

@@ -76,6 +76,7 @@ constexpr long long kDrainPolls = 1LL << 40;  // drains are bounded by the 2 s t
 //   S     [Dv/8][Dk][8]   bf16  state at chunk start  (B writes, C reads)
 struct Workspace {
   uint8_t* base;
+  uint8_t* tinv = nullptr;  // optional: each tile's (I + A)^-1, bf16 [64][64] in scan order
   size_t block_bytes;
   uint32_t off_w, off_kt, off_decay, off_g, off_ut, off_u, off_s;
   int NBH, nC, Dk, Dv;
@@ -409,6 +410,13 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
   }
   __syncthreads();
   unit_lower_inverse(s.u);
+  if (ws.tinv) {  // a bf16 copy of T for the backward pass, rows and columns in scan order
+    uint4* dst = reinterpret_cast<uint4*>(ws.tinv + ws.tile(dir, bh, j) * (64 * 64 * 2));
+    for (int idx = tid; idx < 64 * 8; idx += kWideThreads) {
+      const int r = idx >> 3, ks = idx & 7;
+      dst[idx] = pack8_bf16(&s.u.T[r][8 * ks]);
+    }
+  }
 
   // TW[r][i] = T[pos r][pos i] beta_i e^{gam_i} / |k_i|, TU[r][i] = T[..] beta_i,
   // as bf16 K-major A operands in memory order
@@ -1553,6 +1561,7 @@ cudaError_t launch_chunk_tc(const ScanArgs& a, void* workspace) {
   const int NBH = a.B * a.H;
   Workspace ws;
   ws.base = static_cast<uint8_t*>(workspace);
+  ws.tinv = static_cast<uint8_t*>(a.t_out);
   ws.layout(a.Dk, a.Dv);
   ws.NBH = NBH;
   ws.nC = nC;
