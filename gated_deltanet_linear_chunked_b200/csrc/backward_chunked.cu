@@ -151,8 +151,9 @@ __device__ __forceinline__ void zero2(float (&d)[2][4]) {
 
 // Out (M x N) = A1 B1 (+ A2 B2): warps take 16 x 16 blocks in turn; epi(m, n,
 // value) per element; with rsum / csum, the row / column sums of contrib(m,
-// n, value) over each block are added to rsum[m] (+) and csum[n] (-) with one
-// shared atomic per row / column.
+// n, value) over each block are added to rsum[m] (+) and csum[n] (-).
+// rsum and csum belong to the calling warp alone (plain read-modify-writes:
+// shared-memory float atomics cost more than the products here).
 template <bool TA1, bool TB1, bool TA2, bool TB2, class FC, class FE>
 __device__ __forceinline__ void gemm2(int M, int N, BMat A1, BMat B1, int K1, BMat A2, BMat B2, int K2,
                                       FC contrib, FE epi, float* rsum, float* csum) {
@@ -180,8 +181,8 @@ __device__ __forceinline__ void gemm2(int M, int N, BMat A1, BMat B1, int K1, BM
         r0 += __shfl_xor_sync(0xffffffffu, r0, 2);
         r1 += __shfl_xor_sync(0xffffffffu, r1, 2);
         if ((lane & 3) == 0) {
-          atomicAdd(&rsum[m0 + tile_row(0)], r0);
-          atomicAdd(&rsum[m0 + tile_row(2)], r1);
+          rsum[m0 + tile_row(0)] += r0;
+          rsum[m0 + tile_row(2)] += r1;
         }
       }
       if (csum) {
@@ -192,8 +193,8 @@ __device__ __forceinline__ void gemm2(int M, int N, BMat A1, BMat B1, int K1, BM
           c1 += __shfl_xor_sync(0xffffffffu, c1, off);
         }
         if (lane < 4) {
-          atomicAdd(&csum[n0 + tile_col(0)], -c0);
-          atomicAdd(&csum[n0 + tile_col(1)], -c1);
+          csum[n0 + tile_col(0)] -= c0;
+          csum[n0 + tile_col(1)] -= c1;
         }
       }
     }
@@ -671,7 +672,7 @@ ChainKernel chain_kernel_for(int nkb) {
 // T = (I + A)^-1, which its stage A leaves in the workspace.
 struct GradLayout {
   int lbk, lbv;
-  uint32_t q, k, dout, w, ut, u, s0, dse, P, Tb, E, dU, dW, small, total;
+  uint32_t q, k, dout, w, ut, u, s0, dse, P, Tb, E, dU, dW, part, small, total;
   __host__ __device__ GradLayout(int Dk, int Dv) {
     lbk = Dk + 8;
     lbv = Dv + 8;
@@ -689,6 +690,7 @@ struct GradLayout {
     E = o;    o += 64 * kLdE * 2;   // e^{gam_p - gam_i} K^ K^T (i < p), bf16
     dU = o;   o += 64 * lbv * 2;    // dU (bf16)
     dW = o;   o += 64 * lbk * 2;    // dW (bf16)
+    part = o; o += 3 * kGrWarps * 64 * 4;  // per-warp partial row sums of dgam, dbeta, c
     small = o; o += sizeof(BcSmall);
     total = (o + 15) & ~15u;
   }
@@ -733,7 +735,8 @@ __device__ __forceinline__ void for_acc(int N, F f) {
     }
   }
 }
-// Row sums of f(i, h, e, m, n) over the register blocks, added to dst[m].
+// Row sums of f(i, h, e, m, n) over the register blocks, added to dst[m]
+// (dst belongs to the calling warp alone).
 template <class F>
 __device__ __forceinline__ void acc_row_sums(int N, float* dst, F f) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -756,8 +759,8 @@ __device__ __forceinline__ void acc_row_sums(int N, float* dst, F f) {
       r0 += __shfl_xor_sync(0xffffffffu, r0, 2);
       r1 += __shfl_xor_sync(0xffffffffu, r1, 2);
       if ((lane & 3) == 0) {
-        atomicAdd(&dst[m0 + tile_row(0)], r0);
-        atomicAdd(&dst[m0 + tile_row(2)], r1);
+        dst[m0 + tile_row(0)] += r0;
+        dst[m0 + tile_row(2)] += r1;
       }
     }
   }
@@ -805,6 +808,11 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   bf16* sdW = reinterpret_cast<bf16*>(bg_raw + L.dW);
   BcSmall& sm = *reinterpret_cast<BcSmall*>(bg_raw + L.small);
   const int lbk = L.lbk, lbv = L.lbv;
+  // this warp's partial row sums: gam's, beta's, and c_m = k^_m . dk^_m
+  float* const part = reinterpret_cast<float*>(bg_raw + L.part);
+  float* const wg = part + (threadIdx.x >> 5) * 64;
+  float* const wb = wg + kGrWarps * 64;
+  float* const wc = wb + kGrWarps * 64;
 
   const int j = blockIdx.x, bh = blockIdx.y, dir = blockIdx.z;
   const int b = bh / a.H, h = bh - b * a.H;
@@ -820,6 +828,7 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   // ---- stage: rows (q^, k^, dO, gates), then W, U~, U, S0 (workspace) and
   //      dS_e^T, which land while step 1 runs; dU (from dU^T) after step 1
   stage_rows_issue(a, sm, sQ, sK, sO, lbk, lbv, b, h, dir, j);
+  for (int e = tid; e < 3 * kGrWarps * 64; e += kGrThreads) part[e] = 0.f;
   const int ck = Dk / 8, cv = Dv / 8;
   for (int e = tid; e < 64 * (ck + 2 * cv); e += kGrThreads) {  // [slab][time row][8] -> [scan row]
     const int s2 = e >> 6, t = e & 63, p = dir == 0 ? t : 63 - t;
@@ -884,7 +893,7 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
     zero2(dq[i]);
   }
   gemm_acc2<false, false>(Dk, Dv, Um, dSTm, dk, [&](int m) { return expf(gamC - sm.gam[m]); });
-  acc_row_sums(Dk, sm.cK, [&](int i, int hh, int e, int m, int n) { return bf(sK[m * lbk + n]) * dk[i][hh][e]; });
+  acc_row_sums(Dk, wc, [&](int i, int hh, int e, int m, int n) { return bf(sK[m * lbk + n]) * dk[i][hh][e]; });
   {  // <dS_e, S0> -> dgam_C
     float dot = 0.f;
     for (int c = warp; c < Dv; c += kGrWarps)
@@ -899,10 +908,10 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
       [&](int m, int n, float v) {
         sP[m * kLdE + n] = __float2bfloat16_rn(n <= m ? expf(sm.gam[m] - sm.gam[n]) * v : 0.f);
       },
-      sm.dgam, sm.dgam);
+      wg, wg);
   // ---- 6. Z = diag(e^gam) dO S0^T -> dq^; gam_p gets q^_p . Z_p
   gemm_acc2<false, true>(Dk, Dv, O, S0, dq, [&](int m) { return sm.eg[m]; });
-  acc_row_sums(Dk, sm.dgam, [&](int i, int hh, int e, int m, int n) { return bf(sQ[m * lbk + n]) * dq[i][hh][e]; });
+  acc_row_sums(Dk, wg, [&](int i, int hh, int e, int m, int n) { return bf(sQ[m * lbk + n]) * dq[i][hh][e]; });
   __syncthreads();  // dQK complete
   // ---- 7. dq^ += dQK K^;  8. dk^ += dQK^T Q^
   gemm_acc2<false, false>(Dk, 64, Pm, K, dq, [](int) { return 1.f; });
@@ -949,16 +958,16 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
       }
 #pragma unroll
     for (int off = 16; off; off >>= 1) sw += __shfl_xor_sync(0xffffffffu, sw, off);
-    if (lane == 0) {  // step 12's epilogues may already be adding to these rows
-      atomicAdd(&sm.dbeta[p], sm.eg[p] * sw);
-      atomicAdd(&sm.dgam[p], sm.beta[p] * sm.eg[p] * sw);
+    if (lane == 0) {
+      wb[p] += sm.eg[p] * sw;
+      wg[p] += sm.beta[p] * sm.eg[p] * sw;
     }
   }
   // ---- 12. dA = -(dX_w W^T + dX_u U~^T) on i < p (into P); gam from A
   gemm2<false, true, false, true>(64, 64, Xw, Wm, Dk, Xu, Ut, Dv,
       [&](int m, int n, float v) { return n < m ? -v * sm.beta[m] * bf(sE[m * kLdE + n]) : 0.f; },
       [&](int m, int n, float v) { sP[m * kLdE + n] = __float2bfloat16_rn(n < m ? -v : 0.f); },
-      sm.dgam, sm.dgam);
+      wg, wg);
   __syncthreads();
   for (int p = warp; p < 64; p += kGrWarps) {  // dbeta_p += sum_i dA_pi E_pi; dG = dA beta_p e^{..}
     float sb = 0.f;
@@ -969,7 +978,7 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
     }
 #pragma unroll
     for (int off = 16; off; off >>= 1) sb += __shfl_xor_sync(0xffffffffu, sb, off);
-    if (lane == 0) atomicAdd(&sm.dbeta[p], sb);
+    if (lane == 0) wb[p] += sb;
   }
   __syncthreads();
   // ---- 13. dk^ += (dG + dG^T) K^
@@ -977,7 +986,15 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   gemm_acc2<true, false>(Dk, 64, Pm, K, dk, [](int) { return 1.f; });
   // ---- 14. outputs: dk^, dbeta, dg = suffix sum of dgam + dgam_C
   store_acc(Dk, dk, pk, Dk, sm.row);
-  __syncthreads();  // every addition to dgam and dbeta is done
+  __syncthreads();  // every partial row sum is done
+  if (tid < 3 * 64) {  // the warps' partials: dgam, dbeta, c
+    const float* src = part + (tid >> 6) * kGrWarps * 64 + (tid & 63);
+    float acc = 0.f;
+#pragma unroll
+    for (int w = 0; w < kGrWarps; ++w) acc += src[w * 64];
+    (tid < 64 ? sm.dgam : tid < 128 ? sm.dbeta : sm.cK)[tid & 63] = acc;
+  }
+  __syncthreads();
   if (warp == 0) {
     // K~ = diag(e^{gam_C - gam}) K^: row p's exponent gives -c_p to gam_p
     // and +c_p to gam_C
