@@ -42,6 +42,8 @@
 // diag(beta) dX_u and beta's share v . dX_u there).
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "gdn_internal.h"
 #include "sm100.cuh"
 
@@ -62,6 +64,7 @@ struct BcSmall {
   float g[64], beta[64], gam[64], eg[64], dgam[64], dbeta[64], cK[64];
   int row[64];  // (b, t, h) row of scan position p, -1 past T
   float red[kGrWarps];
+  uint64_t full[5];  // the gradient pass's staged tile groups have landed
 };
 
 struct BcArgs {
@@ -75,9 +78,9 @@ struct BcArgs {
   // (all bf16, transposed so that a slice of 16 columns is contiguous):
   __nv_bfloat16* XT;         // (P^T dO)^T, Dv x 64 in fragment order [Dv/16][4][32 lanes][8]
   __nv_bfloat16* YT;         // (Q^^T diag(e^gam) dO)^T, Dv x Dk, [Dv/16][Dk/16][32][8]
-  __nv_bfloat16* dUT;        // [Dv][64]  dU^T
-  __nv_bfloat16* dSeT;       // [Dv][Dk]  dS_e^T, dS_e the gradient of the chunk's end state
-  const __nv_bfloat16* tinv; // [64][64]  (I + A)^-1 from the forward's stage A (scan order)
+  __nv_bfloat16* dUT;        // dU^T, Dv x 64, core-matrix [64/8][Dv][8]
+  __nv_bfloat16* dSeT;       // dS_e^T, Dv x Dk, [Dk/8][Dv][8] (dS_e: gradient of the chunk's end state)
+  const __nv_bfloat16* tinv; // (I + A)^-1 from the forward's stage A, [64/8][64][8] (scan order)
   float *pq, *pk, *pab, *dvb;  // [dir][rows][Dk], [dir][rows][Dk], [dir][rows][2], [dir][rows][Dv] (dX_u)
   int B, T, H, Dk, Dv, nC, NBH;
   unsigned* err;             // device error word (the chain's bounded waits)
@@ -102,43 +105,74 @@ __device__ __forceinline__ void cp_wait_group() { asm volatile("cp.async.wait_gr
 __device__ __forceinline__ int tile_row(int e) { return ((threadIdx.x & 31) >> 2) + (e >= 2 ? 8 : 0); }
 __device__ __forceinline__ int tile_col(int e) { return 2 * (threadIdx.x & 3) + (e & 1); }
 
-// A bf16 matrix in shared memory, row-major with row stride ld (a multiple
-// of 8).  As the A operand (m x k): element (m, k) = p[m ld + k], or
-// p[k ld + m] when read transposed.  As the B operand (k x n): element
-// (k, n) = p[k ld + n], or p[n ld + k] when read transposed.
+// A bf16 matrix in shared memory.  Element (r, c) sits at byte
+//   base + (c / 8) slab + row(r) rs + 2 (c % 8),  row(r) = r, or rrev - r
+// for a tile whose rows are stored in reverse.  Row-major with row stride ld
+// elements: slab = 16, rs = 2 ld.  The core-matrix layout [c/8][rows][8]
+// (each 8-column slab a run of 16-byte rows, as the workspace and TMA tiles
+// store them): slab = 16 rows, rs = 16.  As the A operand (m x k): element
+// (m, k) = (m, k), or (k, m) when read transposed; as the B operand (k x n):
+// element (k, n) = (k, n), or (n, k) when read transposed.
 struct BMat {
-  const __nv_bfloat16* p;
-  int ld;
+  uint32_t base;
+  int slab, rs;
+  int rrev;  // 0: rows in order
 };
-
-// One k16 step of a 16 x 16 output block (m0, n0): d += A[m0.., k0..] B[k0.., n0..].
-template <bool TA, bool TB>
-__device__ __forceinline__ void step16(int m0, int n0, int k0, BMat A, BMat B, float (&d)[2][4]) {
-  const int l = threadIdx.x & 31;
-  uint32_t a[4], bb[4];
-  if (TA)
-    ldmatrix_x4_trans(smem_u32(A.p + (k0 + (l & 7) + 8 * (l >> 4)) * A.ld + m0 + 8 * ((l >> 3) & 1)), a);
-  else
-    ldmatrix_x4(smem_u32(A.p + (m0 + (l & 15)) * A.ld + k0 + 8 * (l >> 4)), a);
-  if (TB)
-    ldmatrix_x4(smem_u32(B.p + (n0 + (l & 7) + 8 * (l >> 4)) * B.ld + k0 + 8 * ((l >> 3) & 1)), bb);
-  else
-    ldmatrix_x4_trans(smem_u32(B.p + (k0 + (l & 7) + 8 * ((l >> 3) & 1)) * B.ld + n0 + 8 * (l >> 4)), bb);
-  mma_16816(d[0], a, bb[0], bb[1]);
-  mma_16816(d[1], a, bb[2], bb[3]);
+__device__ __forceinline__ BMat row_major(const void* p, int ld) { return {smem_u32(p), 16, 2 * ld, 0}; }
+__device__ __forceinline__ BMat core_mat(const void* p, int rows, bool rev) {
+  return {smem_u32(p), 16 * rows, 16, rev ? rows - 1 : 0};
 }
-// 16 x 16 output block (m0, n0) += A B over k < K (K % 16 == 0); odd k16
-// steps go to a second accumulator, which halves the dependent MMA chains.
+__device__ __forceinline__ uint32_t bm_at(const BMat& M, int r, int c8) {
+  return M.base + c8 * M.slab + (M.rrev ? M.rrev - r : r) * M.rs;
+}
+// Element index (in bf16 units) of (r, c) in a core-matrix tile of `rows`
+// rows, rows stored reversed when rev.
+__device__ __forceinline__ int cidx(int r, int c, int rows, bool rev) {
+  return ((c >> 3) * rows + (rev ? rows - 1 - r : r)) * 8 + (c & 7);
+}
+
+// 16 x 16 output block (m0, n0) += A B over k < K (K % 16 == 0): per k16
+// step one ldmatrix.x4 of each operand and two MMAs; odd steps go to a
+// second accumulator, which halves the dependent MMA chains.
 template <bool TA, bool TB>
-__device__ __forceinline__ void blk16(int m0, int n0, int K, BMat A, BMat B, float (&d)[2][4]) {
+__device__ __forceinline__ void blk16(int m0, int n0, int K, const BMat& A, const BMat& B,
+                                      float (&d)[2][4]) {
+  const int l = threadIdx.x & 31;
+  uint32_t pa, pb;
+  int da, db;  // address steps per k16
+  if (TA) {
+    pa = bm_at(A, (l & 7) + 8 * (l >> 4), (m0 >> 3) + ((l >> 3) & 1));
+    da = A.rrev ? -16 * A.rs : 16 * A.rs;
+  } else {
+    pa = bm_at(A, m0 + (l & 15), l >> 4);
+    da = 2 * A.slab;
+  }
+  if (TB) {
+    pb = bm_at(B, n0 + (l & 7) + 8 * (l >> 4), (l >> 3) & 1);
+    db = 2 * B.slab;
+  } else {
+    pb = bm_at(B, (l & 7) + 8 * ((l >> 3) & 1), (n0 >> 3) + (l >> 4));
+    db = B.rrev ? -16 * B.rs : 16 * B.rs;
+  }
+  auto step = [&](float (&acc)[2][4]) {
+    uint32_t a[4], bb[4];
+    if (TA) ldmatrix_x4_trans(pa, a);
+    else ldmatrix_x4(pa, a);
+    if (TB) ldmatrix_x4(pb, bb);
+    else ldmatrix_x4_trans(pb, bb);
+    mma_16816(acc[0], a, bb[0], bb[1]);
+    mma_16816(acc[1], a, bb[2], bb[3]);
+    pa += da;
+    pb += db;
+  };
   float e[2][4] = {};
   int k0 = 0;
 #pragma unroll 1
   for (; k0 + 32 <= K; k0 += 32) {
-    step16<TA, TB>(m0, n0, k0, A, B, d);
-    step16<TA, TB>(m0, n0, k0 + 16, A, B, e);
+    step(d);
+    step(e);
   }
-  if (k0 < K) step16<TA, TB>(m0, n0, k0, A, B, d);
+  if (k0 < K) step(d);
 #pragma unroll
   for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -155,7 +189,8 @@ __device__ __forceinline__ void zero2(float (&d)[2][4]) {
 // rsum and csum belong to the calling warp alone (plain read-modify-writes:
 // shared-memory float atomics cost more than the products here).
 template <bool TA1, bool TB1, bool TA2, bool TB2, class FC, class FE>
-__device__ __forceinline__ void gemm2(int M, int N, BMat A1, BMat B1, int K1, BMat A2, BMat B2, int K2,
+__device__ __forceinline__ void gemm2(int M, int N, const BMat& A1, const BMat& B1, int K1, const BMat& A2,
+                                      const BMat& B2, int K2,
                                       FC contrib, FE epi, float* rsum, float* csum) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   const int tn = N >> 4, nt = (M >> 4) * tn;
@@ -207,7 +242,7 @@ __device__ __forceinline__ void gemm2(int M, int N, BMat A1, BMat B1, int K1, BM
 // using the block as its accumulator start, or as an A fragment, loads with
 // one 16-byte access per lane.
 template <bool TA, bool TB>
-__device__ __forceinline__ void gemm_store_frag(int M, int N, BMat A, BMat B, int K,
+__device__ __forceinline__ void gemm_store_frag(int M, int N, const BMat& A, const BMat& B, int K,
                                                 __nv_bfloat16* dst) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   const int tn = N >> 4, nt = (M >> 4) * tn;
@@ -219,6 +254,60 @@ __device__ __forceinline__ void gemm_store_frag(int M, int N, BMat A, BMat B, in
     *reinterpret_cast<uint4*>(dst + ((size_t)t * 32 + lane) * 8) =
         make_uint4(pack_bf16x2(dd[0][0], dd[0][1]), pack_bf16x2(dd[0][2], dd[0][3]),
                    pack_bf16x2(dd[1][0], dd[1][1]), pack_bf16x2(dd[1][2], dd[1][3]));
+  }
+}
+
+// gam (inclusive prefix sum of the gates in scan order) and e^gam from sm.g;
+// one warp.
+__device__ void gate_prefix(BcSmall& sm) {
+  const int lane = threadIdx.x & 31;
+  const float a0 = sm.g[2 * lane], a1 = sm.g[2 * lane + 1];
+  float incl = a0 + a1;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const float y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  const float excl = incl - (a0 + a1);
+  sm.gam[2 * lane] = excl + a0;
+  sm.gam[2 * lane + 1] = incl;
+  sm.eg[2 * lane] = expf(excl + a0);
+  sm.eg[2 * lane + 1] = expf(incl);
+}
+// q^ = q / |q| and k^ = k / |k| in place, row by row, for two core-matrix
+// [Dk/8][64][8] tiles (a warp per row; rows of zeros stay zero).  No barrier.
+__device__ void normalize_rows_core(const BcArgs& a, __nv_bfloat16* sQ, __nv_bfloat16* sK) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int Dk = a.Dk;
+  uint32_t* q2 = reinterpret_cast<uint32_t*>(sQ);
+  uint32_t* k2 = reinterpret_cast<uint32_t*>(sK);
+  for (int r = warp; r < 64; r += nw) {
+    float qv[2][2] = {}, kv[2][2] = {};
+    float qq = 0.f, kk = 0.f;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int d2 = lane + 32 * i, at = cidx(r, 2 * d2, 64, false) / 2;
+      if (d2 < Dk / 2) {
+        unpack_bf16x2(q2[at], qv[i][0], qv[i][1]);
+        unpack_bf16x2(k2[at], kv[i][0], kv[i][1]);
+        qq = fmaf(qv[i][0], qv[i][0], fmaf(qv[i][1], qv[i][1], qq));
+        kk = fmaf(kv[i][0], kv[i][0], fmaf(kv[i][1], kv[i][1], kk));
+      }
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) {
+      qq += __shfl_xor_sync(0xffffffffu, qq, off);
+      kk += __shfl_xor_sync(0xffffffffu, kk, off);
+    }
+    const float rq = 1.f / sqrtf(fmaxf(qq, 1e-12f)), rk = 1.f / sqrtf(fmaxf(kk, 1e-12f));
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int d2 = lane + 32 * i, at = cidx(r, 2 * d2, 64, false) / 2;
+      if (d2 < Dk / 2) {
+        q2[at] = pack_bf16x2(qv[i][0] * rq, qv[i][1] * rq);
+        k2[at] = pack_bf16x2(kv[i][0] * rk, kv[i][1] * rk);
+      }
+    }
   }
 }
 
@@ -250,14 +339,15 @@ __device__ void stage_rows_issue(const BcArgs& a, BcSmall& sm, __nv_bfloat16* sQ
     for (int c = lane; c < 2 * ck + cv; c += 32) {
       __nv_bfloat16* dst;
       const __nv_bfloat16* src;
+      // row-major with strides lbk / lbv, or (lbk == 0) core-matrix [D/8][64][8]
       if (c < ck) {
-        dst = sQ + p * lbk + 8 * c;
+        dst = sQ + (lbk ? p * lbk + 8 * c : (c * 64 + p) * 8);
         src = a.q + (size_t)r * Dk + 8 * c;
       } else if (c < 2 * ck) {
-        dst = sK + p * lbk + 8 * (c - ck);
+        dst = sK + (lbk ? p * lbk + 8 * (c - ck) : ((c - ck) * 64 + p) * 8);
         src = a.k + (size_t)r * Dk + 8 * (c - ck);
       } else {
-        dst = sO + p * lbv + 8 * (c - 2 * ck);
+        dst = sO + (lbk ? p * lbv + 8 * (c - 2 * ck) : ((c - 2 * ck) * 64 + p) * 8);
         src = a.dout + (size_t)r * Dv + 8 * (c - 2 * ck);
       }
       if (r >= 0) cp16(dst, src);
@@ -265,20 +355,7 @@ __device__ void stage_rows_issue(const BcArgs& a, BcSmall& sm, __nv_bfloat16* sQ
     }
   }
   cp_commit();
-  if (warp == 0) {
-    const float a0 = sm.g[2 * lane], a1 = sm.g[2 * lane + 1];
-    float incl = a0 + a1;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const float y = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += y;
-    }
-    const float excl = incl - (a0 + a1);
-    sm.gam[2 * lane] = excl + a0;
-    sm.gam[2 * lane + 1] = incl;
-    sm.eg[2 * lane] = expf(excl + a0);
-    sm.eg[2 * lane + 1] = expf(incl);
-  }
+  if (warp == 0) gate_prefix(sm);
 }
 template <int N>
 __device__ void stage_rows_finish(const BcArgs& a, BcSmall& sm, __nv_bfloat16* sQ, __nv_bfloat16* sK,
@@ -288,16 +365,19 @@ __device__ void stage_rows_finish(const BcArgs& a, BcSmall& sm, __nv_bfloat16* s
   cp_wait_group<N>();
   __syncthreads();
   for (int p = warp; p < 64; p += nw) {  // bf16 pairs: Dk / 2 <= 64, two per lane at most
-    uint32_t* q2 = reinterpret_cast<uint32_t*>(sQ + p * lbk);
-    uint32_t* k2 = reinterpret_cast<uint32_t*>(sK + p * lbk);
+    // pair d2 of row p, in pairs: row-major with stride lbk, or (lbk == 0)
+    // core-matrix [Dk/8][64][8]
+    auto at2 = [&](int d2) { return lbk ? (p * lbk) / 2 + d2 : cidx(p, 2 * d2, 64, false) / 2; };
+    uint32_t* q2 = reinterpret_cast<uint32_t*>(sQ);
+    uint32_t* k2 = reinterpret_cast<uint32_t*>(sK);
     float qv[2][2] = {}, kv[2][2] = {};
     float qq = 0.f, kk = 0.f;
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const int d2 = lane + 32 * i;
       if (d2 < Dk / 2) {
-        unpack_bf16x2(q2[d2], qv[i][0], qv[i][1]);
-        unpack_bf16x2(k2[d2], kv[i][0], kv[i][1]);
+        unpack_bf16x2(q2[at2(d2)], qv[i][0], qv[i][1]);
+        unpack_bf16x2(k2[at2(d2)], kv[i][0], kv[i][1]);
         qq = fmaf(qv[i][0], qv[i][0], fmaf(qv[i][1], qv[i][1], qq));
         kk = fmaf(kv[i][0], kv[i][0], fmaf(kv[i][1], kv[i][1], kk));
       }
@@ -313,12 +393,12 @@ __device__ void stage_rows_finish(const BcArgs& a, BcSmall& sm, __nv_bfloat16* s
       const int d2 = lane + 32 * i;
       if (d2 < Dk / 2) {
         const uint32_t qn = pack_bf16x2(qv[i][0] * rq, qv[i][1] * rq);
-        q2[d2] = qn;
-        k2[d2] = pack_bf16x2(kv[i][0] * rk, kv[i][1] * rk);
+        q2[at2(d2)] = qn;
+        k2[at2(d2)] = pack_bf16x2(kv[i][0] * rk, kv[i][1] * rk);
         if (sQs) {  // e^gam times the rounded q^
           float x0, x1;
           unpack_bf16x2(qn, x0, x1);
-          reinterpret_cast<uint32_t*>(sQs + p * lbk)[d2] = pack_bf16x2(x0 * sm.eg[p], x1 * sm.eg[p]);
+          reinterpret_cast<uint32_t*>(sQs)[at2(d2)] = pack_bf16x2(x0 * sm.eg[p], x1 * sm.eg[p]);
         }
       }
     }
@@ -364,7 +444,8 @@ __global__ void __launch_bounds__(kBcThreads) gdn_bwd_pre_kernel(BcArgs a) {
   stage_rows_issue(a, sm, sQ, sK, sO, lbk, lbv, b, h, dir, j);
   stage_rows_finish<0>(a, sm, sQ, sK, lbk, sQs);
   auto none = [](int, int, float) { return 0.f; };
-  const BMat Q{sQ, lbk}, K{sK, lbk}, O{sO, lbv}, Qs{sQs, lbk}, Pm{sP, kLdE};
+  const BMat Q = row_major(sQ, lbk), K = row_major(sK, lbk), O = row_major(sO, lbv);
+  const BMat Qs = row_major(sQs, lbk), Pm = row_major(sP, kLdE);
   gemm2<false, true, false, true>(64, 64, Q, K, Dk, Q, K, 0, none, [&](int m, int n, float v) {
     sP[m * kLdE + n] = __float2bfloat16_rn(n <= m ? expf(sm.gam[m] - sm.gam[n]) * v : 0.f);
   }, nullptr, nullptr);
@@ -507,7 +588,8 @@ __global__ void __launch_bounds__(kChThreads, 2) gdn_bwd_chain_kernel(BcArgs a) 
     const size_t blk = a.blk(dir, bh, dir == 0 ? a.nC - 1 - s : s);
     // dS_e^T (the state entering this chunk) to the slice's warps, in
     // fragment order, and to the gradient pass
-    uint32_t* dse = reinterpret_cast<uint32_t*>(a.dSeT + (blk * Dv + c0) * Dk);
+    // (dS_e^T of the block: core-matrix [Dk/8][Dv][8], rows c, columns d)
+    uint32_t* dse = reinterpret_cast<uint32_t*>(a.dSeT + blk * Dv * Dk);
 #pragma unroll
     for (int i = 0; i < KPW; ++i) {
       const int kb = q + 4 * i;
@@ -515,11 +597,11 @@ __global__ void __launch_bounds__(kChThreads, 2) gdn_bwd_chain_kernel(BcArgs a) 
         const uint32_t f[4] = {pack_bf16x2(S[i][0][0], S[i][0][1]), pack_bf16x2(S[i][0][2], S[i][0][3]),
                                pack_bf16x2(S[i][1][0], S[i][1][1]), pack_bf16x2(S[i][1][2], S[i][1][3])};
         st_shared_v4(xs_u + kb * 512, f);
-        const int d = 16 * kb + 2 * tq;
-        dse[(gq * Dk + d) >> 1] = f[0];
-        dse[((gq + 8) * Dk + d) >> 1] = f[1];
-        dse[(gq * Dk + d + 8) >> 1] = f[2];
-        dse[((gq + 8) * Dk + d + 8) >> 1] = f[3];
+        const int c = c0 + gq, d = 16 * kb + 2 * tq;
+        dse[(((d >> 3) * Dv + c) * 8 + (d & 7)) >> 1] = f[0];
+        dse[(((d >> 3) * Dv + c + 8) * 8 + (d & 7)) >> 1] = f[1];
+        dse[((((d + 8) >> 3) * Dv + c) * 8 + (d & 7)) >> 1] = f[2];
+        dse[((((d + 8) >> 3) * Dv + c + 8) * 8 + (d & 7)) >> 1] = f[3];
       }
     }
     const bool okw = __all_sync(0xffffffffu, mbar_wait(&bars.full[st], ph, a.limit));
@@ -588,12 +670,13 @@ __global__ void __launch_bounds__(kChThreads, 2) gdn_bwd_chain_kernel(BcArgs a) 
       const uint32_t f[4] = {pack_bf16x2(u[0][0], u[0][1]), pack_bf16x2(u[0][2], u[0][3]),
                              pack_bf16x2(u[1][0], u[1][1]), pack_bf16x2(u[1][2], u[1][3])};
       st_shared_v4(xu_u + q * 512, f);
-      uint32_t* du = reinterpret_cast<uint32_t*>(a.dUT + (blk * Dv + c0) * 64);
-      const int p = 16 * q + 2 * tq;
-      du[(gq * 64 + p) >> 1] = f[0];
-      du[((gq + 8) * 64 + p) >> 1] = f[1];
-      du[(gq * 64 + p + 8) >> 1] = f[2];
-      du[((gq + 8) * 64 + p + 8) >> 1] = f[3];
+      // dU^T of the block: core-matrix [64/8][Dv][8] (rows c, columns p)
+      uint32_t* du = reinterpret_cast<uint32_t*>(a.dUT + blk * Dv * 64);
+      const int c = c0 + gq, p = 16 * q + 2 * tq;
+      du[(((p >> 3) * Dv + c) * 8 + (p & 7)) >> 1] = f[0];
+      du[(((p >> 3) * Dv + c + 8) * 8 + (p & 7)) >> 1] = f[1];
+      du[((((p + 8) >> 3) * Dv + c) * 8 + (p & 7)) >> 1] = f[2];
+      du[((((p + 8) >> 3) * Dv + c + 8) * 8 + (p & 7)) >> 1] = f[3];
     }
     named_barrier(1 + g, 128);
     // ---- dS0^T (+)= -dU^T W over this warp's blocks
@@ -677,18 +760,20 @@ struct GradLayout {
     lbk = Dk + 8;
     lbv = Dv + 8;
     uint32_t o = 0;
-    q = o;    o += 64 * lbk * 2;    // q^, then dX_w
-    k = o;    o += 64 * lbk * 2;    // k^
-    dout = o; o += 64 * lbv * 2;    // dO, then dX_u
-    w = o;    o += 64 * lbk * 2;    // W
-    ut = o;   o += 64 * lbv * 2;    // U~
-    u = o;    o += 64 * lbv * 2;    // U
-    s0 = o;   o += Dk * lbv * 2;    // S0 [Dk][Dv]
-    dse = o;  o += Dv * lbk * 2;    // dS_e^T [Dv][Dk]
+    // core-matrix tiles [cols/8][rows][8], as their sources store them
+    q = o;    o += 64 * Dk * 2;     // q^ (scan rows), then dX_w
+    k = o;    o += 64 * Dk * 2;     // k^ (scan rows)
+    dout = o; o += 64 * Dv * 2;     // dO (scan rows), then dX_u
+    w = o;    o += 64 * Dk * 2;     // W  (time rows)
+    ut = o;   o += 64 * Dv * 2;     // U~ (time rows)
+    u = o;    o += 64 * Dv * 2;     // U  (time rows)
+    s0 = o;   o += Dk * Dv * 2;     // S0: rows d, columns c
+    dse = o;  o += Dv * Dk * 2;     // dS_e^T: rows c, columns d
+    Tb = o;   o += 64 * 64 * 2;     // T = (I + A)^-1 (scan rows)
+    dU = o;   o += 64 * Dv * 2;     // dU^T: rows c, columns p
+    // row-major tiles the pass writes itself
     P = o;    o += 64 * kLdE * 2;   // P, then dQK, then dA / dG (bf16)
-    Tb = o;   o += 64 * kLdE * 2;   // T = (I + A)^-1 (bf16)
     E = o;    o += 64 * kLdE * 2;   // e^{gam_p - gam_i} K^ K^T (i < p), bf16
-    dU = o;   o += 64 * lbv * 2;    // dU (bf16)
     dW = o;   o += 64 * lbk * 2;    // dW (bf16)
     part = o; o += 3 * kGrWarps * 64 * 4;  // per-warp partial row sums of dgam, dbeta, c
     small = o; o += sizeof(BcSmall);
@@ -699,7 +784,7 @@ struct GradLayout {
 // A 64 x N product accumulated in registers: block i of warp w is output
 // block w + 8 i; acc[i][h][e] += scale(m) * value.
 template <bool TA, bool TB, class FS>
-__device__ __forceinline__ void gemm_acc2(int N, int K, BMat A, BMat B, float (&acc)[kMaxBlocks][2][4],
+__device__ __forceinline__ void gemm_acc2(int N, int K, const BMat& A, const BMat& B, float (&acc)[kMaxBlocks][2][4],
                                           FS scale) {
   const int warp = threadIdx.x >> 5;
   const int tn = N >> 4, nt = 4 * tn;
@@ -788,8 +873,30 @@ __device__ __forceinline__ void store_acc(int N, const float (&acc)[kMaxBlocks][
   }
 }
 
-__global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
-  extern __shared__ __align__(16) uint8_t bg_raw[];
+// Gradient-pass tile t: chunk j fastest, then b*h, then direction.
+struct GrTile {
+  int j, bh, dir, b, h;
+  size_t bi;  // block index in the per-chunk buffers
+};
+__device__ __forceinline__ GrTile gr_tile(const BcArgs& a, int t) {
+  GrTile c;
+  c.j = t % a.nC;
+  const int rest = t / a.nC;
+  c.bh = rest % a.NBH;
+  c.dir = rest / a.NBH;
+  c.b = c.bh / a.H;
+  c.h = c.bh - c.b * a.H;
+  c.bi = a.blk(c.dir, c.bh, c.j);
+  return c;
+}
+
+// Persistent: CTA x walks tiles x, x + gridDim.x, ...; each group of the
+// next tile's inputs is fetched by one thread as soon as this tile has done
+// with the buffers it lands in, so the next tile starts with its data on chip.
+__global__ void __launch_bounds__(kGrThreads, 1)
+gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_o, BcArgs a, int ntiles) {
+  extern __shared__ __align__(128) uint8_t bg_raw[];
   const int Dk = a.Dk, Dv = a.Dv;
   const GradLayout L(Dk, Dv);
   using bf16 = __nv_bfloat16;
@@ -807,60 +914,113 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   bf16* sdU = reinterpret_cast<bf16*>(bg_raw + L.dU);
   bf16* sdW = reinterpret_cast<bf16*>(bg_raw + L.dW);
   BcSmall& sm = *reinterpret_cast<BcSmall*>(bg_raw + L.small);
-  const int lbk = L.lbk, lbv = L.lbv;
+  const int lbk = L.lbk;
   // this warp's partial row sums: gam's, beta's, and c_m = k^_m . dk^_m
   float* const part = reinterpret_cast<float*>(bg_raw + L.part);
   float* const wg = part + (threadIdx.x >> 5) * 64;
   float* const wb = wg + kGrWarps * 64;
   float* const wc = wb + kGrWarps * 64;
 
-  const int j = blockIdx.x, bh = blockIdx.y, dir = blockIdx.z;
-  const int b = bh / a.H, h = bh - b * a.H;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const size_t rows_bth = (size_t)a.B * a.T * a.H;
+  // Tile groups, each landing on its own mbarrier (one phase per tile):
+  //   0: U, dS_e^T   1: S0   2: T, dU^T   3: q, dO, W, U~   4: k
+  // Group g of the next tile is issued (by one thread) right after the
+  // barrier behind which this tile last reads group g's buffers.
+  uint64_t* full = sm.full;
+  auto issue = [&](int g, const GrTile& c) {
+    const uint8_t* blk = a.ws + c.bi * a.wl.block_bytes;
+    fence_proxy_async_smem();  // the buffers' last generic accesses come first
+    switch (g) {
+      case 0:
+        mbar_arrive_expect_tx(&full[0], 64 * Dv * 2 + Dv * Dk * 2);
+        bulk_load(sU, blk + a.wl.off_u, 64 * Dv * 2, &full[0]);
+        bulk_load(sdST, a.dSeT + c.bi * Dv * Dk, Dv * Dk * 2, &full[0]);
+        break;
+      case 1:
+        mbar_arrive_expect_tx(&full[1], Dk * Dv * 2);
+        bulk_load(sS0, blk + a.wl.off_s, Dk * Dv * 2, &full[1]);
+        break;
+      case 2:
+        mbar_arrive_expect_tx(&full[2], 64 * 64 * 2 + 64 * Dv * 2);
+        bulk_load(sT, a.tinv + c.bi * 64 * 64, 64 * 64 * 2, &full[2]);
+        bulk_load(sdU, a.dUT + c.bi * Dv * 64, 64 * Dv * 2, &full[2]);
+        break;
+      case 3:
+        mbar_arrive_expect_tx(&full[3], 2 * 64 * Dk * 2 + 2 * 64 * Dv * 2);
+        tma_load_tile(sQ, &tm_q, &full[3], 64 * c.j, c.h, c.b);
+        tma_load_tile(sO, &tm_o, &full[3], 64 * c.j, c.h, c.b);
+        bulk_load(sW, blk + a.wl.off_w, 64 * Dk * 2, &full[3]);
+        bulk_load(sUt, blk + a.wl.off_ut, 64 * Dv * 2, &full[3]);
+        break;
+      default:
+        mbar_arrive_expect_tx(&full[4], 64 * Dk * 2);
+        tma_load_tile(sK, &tm_k, &full[4], 64 * c.j, c.h, c.b);
+        break;
+    }
+  };
+  float gate_g = 0.f, gate_b = 0.f;  // row tid (< 64) of the next tile
+  int gate_row = -1;
+  auto load_gates = [&](const GrTile& c) {
+    if (tid < 64) {
+      const int t = 64 * c.j + (c.dir == 0 ? tid : 63 - tid);
+      const bool valid = t < a.T;
+      const size_t r = ((size_t)c.b * a.T + t) * a.H + c.h;
+      gate_row = valid ? (int)r : -1;
+      gate_g = valid ? __ldg(a.g + r) : 0.f;
+      gate_b = valid ? __ldg(a.beta + r) : 0.f;
+    }
+  };
+
+  int t = blockIdx.x;
+  if (t >= ntiles) return;
+  if (tid == 0) {
+    for (int g = 0; g < 5; ++g) mbar_init(&full[g], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  {
+    const GrTile c = gr_tile(a, t);
+    load_gates(c);
+    if (tid == 0)
+      for (int g = 0; g < 5; ++g) issue(g, c);
+  }
+  for (int it = 0; t < ntiles; t += gridDim.x, ++it) {
+  const GrTile cur = gr_tile(a, t);
+  const bool more = t + (int)gridDim.x < ntiles;
+  const GrTile nxt = gr_tile(a, more ? t + (int)gridDim.x : t);
+  const int dir = cur.dir;
   float* pq = a.pq + (size_t)dir * rows_bth * Dk;
   float* pk = a.pk + (size_t)dir * rows_bth * Dk;
   float* pab = a.pab + (size_t)dir * rows_bth * 2;
   float* dvb = a.dvb + (size_t)dir * rows_bth * Dv;
-  const size_t bi = a.blk(dir, bh, j);
-  const uint8_t* blk = a.ws + bi * a.wl.block_bytes;
 
-  // ---- stage: rows (q^, k^, dO, gates), then W, U~, U, S0 (workspace) and
-  //      dS_e^T, which land while step 1 runs; dU (from dU^T) after step 1
-  stage_rows_issue(a, sm, sQ, sK, sO, lbk, lbv, b, h, dir, j);
+  // ---- this tile's gates and zeroed partial sums; every group landed
+  if (tid < 64) {
+    sm.row[tid] = gate_row;
+    sm.g[tid] = gate_g;
+    sm.beta[tid] = gate_b;
+  }
   for (int e = tid; e < 3 * kGrWarps * 64; e += kGrThreads) part[e] = 0.f;
-  const int ck = Dk / 8, cv = Dv / 8;
-  for (int e = tid; e < 64 * (ck + 2 * cv); e += kGrThreads) {  // [slab][time row][8] -> [scan row]
-    const int s2 = e >> 6, t = e & 63, p = dir == 0 ? t : 63 - t;
-    if (s2 < ck) cp16(sW + p * lbk + 8 * s2, blk + a.wl.off_w + 16 * (s2 * 64 + t));
-    else if (s2 < ck + cv) cp16(sUt + p * lbv + 8 * (s2 - ck), blk + a.wl.off_ut + 16 * ((s2 - ck) * 64 + t));
-    else cp16(sU + p * lbv + 8 * (s2 - ck - cv), blk + a.wl.off_u + 16 * ((s2 - ck - cv) * 64 + t));
+  __syncthreads();
+  if (warp == 0) gate_prefix(sm);
+  {
+    bool ok = true;
+    for (int g = 0; g < 5; ++g) ok = mbar_wait(&full[g], it & 1, a.limit) && ok;
+    if (!__syncthreads_and(ok)) {
+      if (tid == 0) atomicOr(a.err, kErrTimeout);
+      for (int g = 0; g < 5; ++g) mbar_wait(&full[g], it & 1, kChDrainPolls);  // nothing may land after exit
+      return;
+    }
   }
-  for (int s2 = warp; s2 < cv; s2 += kGrWarps)  // S0: [Dv/8][Dk][8] -> [Dk][Dv]
-    for (int d = lane; d < Dk; d += 32) cp16(sS0 + d * lbv + 8 * s2, blk + a.wl.off_s + 16 * (s2 * Dk + d));
-  const bf16* dSeT = a.dSeT + bi * Dv * Dk;
-  for (int e = tid; e < Dv * 16; e += kGrThreads) {  // Dk / 8 <= 16 pieces a row
-    const int c = e >> 4, d8 = e & 15;
-    if (d8 < ck) cp16(sdST + c * lbk + 8 * d8, dSeT + (size_t)c * Dk + 8 * d8);
-  }
-  const bf16* Tg = a.tinv + bi * 64 * 64;
-  for (int e = tid; e < 64 * 8; e += kGrThreads) cp16(sT + (e >> 3) * kLdE + 8 * (e & 7), Tg + 8 * e);
-  cp_commit();
-  // dU^T: 8 tokens of a column per 16-byte load (Dv <= 128), held in
-  // registers until step 1 is done
-  constexpr int kDuLoads = 128 * 8 / kGrThreads;
-  uint4 du_raw[kDuLoads];
-  const bf16* dUT = a.dUT + bi * Dv * 64;
-#pragma unroll
-  for (int i = 0; i < kDuLoads; ++i) {
-    const int e = tid + kGrThreads * i, c = e & 127, p8 = e >> 7;
-    du_raw[i] = c < Dv ? __ldg(reinterpret_cast<const uint4*>(dUT + (size_t)c * 64 + 8 * p8))
-                       : make_uint4(0, 0, 0, 0);
-  }
-  stage_rows_finish<1>(a, sm, sQ, sK, lbk);
+  normalize_rows_core(a, sQ, sK);  // per memory row: the order of the rows does not matter
+  __syncthreads();
   const float gamC = sm.gam[63], eC = expf(gamC);
-  const BMat Q{sQ, lbk}, K{sK, lbk}, O{sO, lbv}, Wm{sW, lbk}, Ut{sUt, lbv}, Um{sU, lbv};
-  const BMat S0{sS0, lbv}, dSTm{sdST, lbk}, Pm{sP, kLdE}, dUm{sdU, lbv}, dWm{sdW, lbk};
+  const bool rev = dir != 0;  // the tiles' time rows run against the scan
+  const BMat Q = core_mat(sQ, 64, rev), K = core_mat(sK, 64, rev), O = core_mat(sO, 64, rev);
+  const BMat Wm = core_mat(sW, 64, rev), Ut = core_mat(sUt, 64, rev), Um = core_mat(sU, 64, rev);
+  const BMat S0 = core_mat(sS0, Dk, false), dSTm = core_mat(sdST, Dv, false);
+  const BMat dUTm = core_mat(sdU, Dv, false), Pm = row_major(sP, kLdE), dWm = row_major(sdW, lbk);
   auto none = [](int, int, float) { return 0.f; };
 
   // ---- 1. P = M o (Q^ K^T);  E = e^{gam_p - gam_i} K^ K^T (i < p), A = diag(beta) E
@@ -870,19 +1030,7 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   gemm2<false, true, false, true>(64, 64, K, K, Dk, K, K, 0, none, [&](int m, int n, float v) {
     sE[m * kLdE + n] = __float2bfloat16_rn(n < m ? expf(sm.gam[m] - sm.gam[n]) * v : 0.f);
   }, nullptr, nullptr);
-  // dU rows from the registers, then every staged tile
-#pragma unroll
-  for (int i = 0; i < kDuLoads; ++i) {
-    const int e = tid + kGrThreads * i, c = e & 127, p8 = e >> 7;
-    if (c < Dv) {
-      const uint32_t w[4] = {du_raw[i].x, du_raw[i].y, du_raw[i].z, du_raw[i].w};
-#pragma unroll
-      for (int k2 = 0; k2 < 4; ++k2) {
-        sdU[(8 * p8 + 2 * k2) * lbv + c] = __ushort_as_bfloat16((unsigned short)(w[k2] & 0xFFFFu));
-        sdU[(8 * p8 + 2 * k2 + 1) * lbv + c] = __ushort_as_bfloat16((unsigned short)(w[k2] >> 16));
-      }
-    }
-  }
+  // every staged tile
   cp_wait_all();
   __syncthreads();
   // ---- 3. dK~ = U dS_e^T: dk^ starts as e^{gam_C - gam} dK~; c_m = k^_m . dk^_m
@@ -893,11 +1041,12 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
     zero2(dq[i]);
   }
   gemm_acc2<false, false>(Dk, Dv, Um, dSTm, dk, [&](int m) { return expf(gamC - sm.gam[m]); });
-  acc_row_sums(Dk, wc, [&](int i, int hh, int e, int m, int n) { return bf(sK[m * lbk + n]) * dk[i][hh][e]; });
+  acc_row_sums(Dk, wc, [&](int i, int hh, int e, int m, int n) { return bf(sK[cidx(m, n, 64, rev)]) * dk[i][hh][e]; });
   {  // <dS_e, S0> -> dgam_C
     float dot = 0.f;
     for (int c = warp; c < Dv; c += kGrWarps)
-      for (int d = lane; d < Dk; d += 32) dot = fmaf(bf(sdST[c * lbk + d]), bf(sS0[d * lbv + c]), dot);
+      for (int d = lane; d < Dk; d += 32)
+        dot = fmaf(bf(sdST[cidx(c, d, Dv, false)]), bf(sS0[cidx(d, c, Dk, false)]), dot);
 #pragma unroll
     for (int off = 16; off; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
     if (lane == 0) sm.red[warp] = dot;  // summed after the last barrier
@@ -911,49 +1060,52 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
       wg, wg);
   // ---- 6. Z = diag(e^gam) dO S0^T -> dq^; gam_p gets q^_p . Z_p
   gemm_acc2<false, true>(Dk, Dv, O, S0, dq, [&](int m) { return sm.eg[m]; });
-  acc_row_sums(Dk, wg, [&](int i, int hh, int e, int m, int n) { return bf(sQ[m * lbk + n]) * dq[i][hh][e]; });
-  __syncthreads();  // dQK complete
+  acc_row_sums(Dk, wg, [&](int i, int hh, int e, int m, int n) { return bf(sQ[cidx(m, n, 64, rev)]) * dq[i][hh][e]; });
+  __syncthreads();  // dQK complete; U and dS_e^T are read no more
+  if (more && tid == 0) issue(0, nxt);
   // ---- 7. dq^ += dQK K^;  8. dk^ += dQK^T Q^
   gemm_acc2<false, false>(Dk, 64, Pm, K, dq, [](int) { return 1.f; });
   gemm_acc2<true, false>(Dk, 64, Pm, Q, dk, [](int) { return 1.f; });
   store_acc(Dk, dq, pq, Dk, sm.row);
   // ---- 9. dW = -dU S0^T
-  gemm2<false, true, false, true>(64, Dk, dUm, S0, Dv, dUm, S0, 0, none,
+  gemm2<true, true, true, true>(64, Dk, dUTm, S0, Dv, dUTm, S0, 0, none,
       [&](int m, int n, float v) { sdW[m * lbk + n] = __float2bfloat16_rn(-v); }, nullptr, nullptr);
-  __syncthreads();
+  __syncthreads();  // S0 is read no more
+  if (more && tid == 0) issue(1, nxt);
   // ---- 10. [dX_w | dX_u] solves (I + A)^T X = [dW | dU]: X = T^T [dW | dU]
   //          with the forward's own T, into the tiles of q^ and dO (neither
   //          is read again)
   bf16* sXw = sQ;
   bf16* sXu = sO;
   {
-    const BMat Tt{sT, kLdE};
+    const BMat Tt = core_mat(sT, 64, false);
     gemm2<true, false, true, false>(64, Dk, Tt, dWm, 64, Tt, Tt, 0, none,
-        [&](int m, int n, float v) { sXw[m * lbk + n] = __float2bfloat16_rn(v); }, nullptr, nullptr);
-    gemm2<true, false, true, false>(64, Dv, Tt, dUm, 64, Tt, Tt, 0, none,
-        [&](int m, int n, float v) { sXu[m * lbv + n] = __float2bfloat16_rn(v); }, nullptr, nullptr);
+        [&](int m, int n, float v) { sXw[cidx(m, n, 64, false)] = __float2bfloat16_rn(v); }, nullptr, nullptr);
+    gemm2<true, true, true, true>(64, Dv, Tt, dUTm, 64, Tt, Tt, 0, none,
+        [&](int m, int n, float v) { sXu[cidx(m, n, 64, false)] = __float2bfloat16_rn(v); }, nullptr, nullptr);
   }
-  __syncthreads();
-  const BMat Xw{sXw, lbk}, Xu{sXu, lbv};
+  __syncthreads();  // T and dU^T are read no more
+  if (more && tid == 0) issue(2, nxt);
+  const BMat Xw = core_mat(sXw, 64, false), Xu = core_mat(sXu, 64, false);
   // ---- 11. dk^ += diag(beta e^gam) dX_w; dX_u goes out as it is (the
   //          reduction forms dv = beta dX_u and beta's share v . dX_u);
   //          beta and gam from the rows of X_w = diag(beta e^gam) K^
   for_acc(Dk, [&](int i, int hh, int e, int m, int n) {
-    dk[i][hh][e] = fmaf(sm.beta[m] * sm.eg[m], bf(sXw[m * lbk + n]), dk[i][hh][e]);
+    dk[i][hh][e] = fmaf(sm.beta[m] * sm.eg[m], bf(sXw[cidx(m, n, 64, false)]), dk[i][hh][e]);
   });
   for (int p = warp; p < 64; p += kGrWarps) {
     const int r = sm.row[p];
     float sw = 0.f;
     for (int d2 = lane; d2 < Dk / 2; d2 += 32) {
       float k0, k1, w0, w1;
-      unpack_bf16x2(reinterpret_cast<const uint32_t*>(sK + p * lbk)[d2], k0, k1);
-      unpack_bf16x2(reinterpret_cast<const uint32_t*>(sXw + p * lbk)[d2], w0, w1);
+      unpack_bf16x2(*reinterpret_cast<const uint32_t*>(sK + cidx(p, 2 * d2, 64, rev)), k0, k1);
+      unpack_bf16x2(*reinterpret_cast<const uint32_t*>(sXw + cidx(p, 2 * d2, 64, false)), w0, w1);
       sw = fmaf(k0, w0, fmaf(k1, w1, sw));
     }
     if (r >= 0)
       for (int c2 = lane; c2 < Dv / 2; c2 += 32) {
         float x0, x1;
-        unpack_bf16x2(reinterpret_cast<const uint32_t*>(sXu + p * lbv)[c2], x0, x1);
+        unpack_bf16x2(*reinterpret_cast<const uint32_t*>(sXu + cidx(p, 2 * c2, 64, false)), x0, x1);
         *reinterpret_cast<float2*>(dvb + (size_t)r * Dv + 2 * c2) = make_float2(x0, x1);
       }
 #pragma unroll
@@ -968,7 +1120,8 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
       [&](int m, int n, float v) { return n < m ? -v * sm.beta[m] * bf(sE[m * kLdE + n]) : 0.f; },
       [&](int m, int n, float v) { sP[m * kLdE + n] = __float2bfloat16_rn(n < m ? -v : 0.f); },
       wg, wg);
-  __syncthreads();
+  __syncthreads();  // dX_w, dX_u (in the q^ and dO tiles), W and U~ are read no more
+  if (more && tid == 0) issue(3, nxt);
   for (int p = warp; p < 64; p += kGrWarps) {  // dbeta_p += sum_i dA_pi E_pi; dG = dA beta_p e^{..}
     float sb = 0.f;
     for (int i = lane; i < p; i += 32) {
@@ -986,7 +1139,11 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
   gemm_acc2<true, false>(Dk, 64, Pm, K, dk, [](int) { return 1.f; });
   // ---- 14. outputs: dk^, dbeta, dg = suffix sum of dgam + dgam_C
   store_acc(Dk, dk, pk, Dk, sm.row);
-  __syncthreads();  // every partial row sum is done
+  __syncthreads();  // every partial row sum is done; k^ is read no more
+  if (more) {
+    if (tid == 0) issue(4, nxt);
+    load_gates(nxt);
+  }
   if (tid < 3 * 64) {  // the warps' partials: dgam, dbeta, c
     const float* src = part + (tid >> 6) * kGrWarps * 64 + (tid & 63);
     float acc = 0.f;
@@ -1023,6 +1180,8 @@ __global__ void __launch_bounds__(kGrThreads, 1) gdn_bwd_grad_kernel(BcArgs a) {
       pab[(size_t)r1 * 2] = g1;
       pab[(size_t)r1 * 2 + 1] = sm.dbeta[2 * lane + 1];
     }
+  }
+  __syncthreads();  // the next tile rewrites sm
   }
 }
 
@@ -1109,6 +1268,13 @@ cudaError_t launch_backward_chunked(const BwdCall& c, void* workspace, float** p
       a.wl.off_w % 16 != 0)
     return cudaErrorInvalidValue;
   const int smem_grad = (int)GradLayout(c.Dk, c.Dv).total;
+  // the gradient pass copies U~, U and S0 of a chunk as one span
+  if (a.wl.off_u != a.wl.off_ut + 128u * c.Dv || a.wl.off_s != a.wl.off_u + 128u * c.Dv)
+    return cudaErrorInvalidValue;
+  CUtensorMap tq, tk, to;
+  if (!make_tile_map(&tq, c.q, c.B, c.T, c.H, c.Dk, 64) || !make_tile_map(&tk, c.k, c.B, c.T, c.H, c.Dk, 64) ||
+      !make_tile_map(&to, c.d_out, c.B, c.T, c.H, c.Dv, 64))
+    return cudaErrorInvalidValue;
   if ((e = cudaFuncSetAttribute(gdn_bwd_pre_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 smem_pre)) != cudaSuccess ||
       (e = cudaFuncSetAttribute(chain, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1130,7 +1296,9 @@ cudaError_t launch_backward_chunked(const BwdCall& c, void* workspace, float** p
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   {
     ProfileScope ps(c.stream, kKernBwdGrad);
-    gdn_bwd_grad_kernel<<<per_chunk, kGrThreads, smem_grad, c.stream>>>(a);
+    const int ntiles = nC * (int)NBH * ndir;
+    gdn_bwd_grad_kernel<<<std::min(ntiles, num_sms()), kGrThreads, smem_grad, c.stream>>>(tq, tk, to, a,
+                                                                                       ntiles);
   }
   e = cudaGetLastError();
   if (e == cudaSuccess) count_launches(3);

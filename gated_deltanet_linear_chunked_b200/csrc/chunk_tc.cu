@@ -76,7 +76,7 @@ constexpr long long kDrainPolls = 1LL << 40;  // drains are bounded by the 2 s t
 //   S     [Dv/8][Dk][8]   bf16  state at chunk start  (B writes, C reads)
 struct Workspace {
   uint8_t* base;
-  uint8_t* tinv = nullptr;  // optional: each tile's (I + A)^-1, bf16 [64][64] in scan order
+  uint8_t* tinv = nullptr;  // optional: each tile's (I + A)^-1, bf16 [8][64][8] in scan order
   size_t block_bytes;
   uint32_t off_w, off_kt, off_decay, off_g, off_ut, off_u, off_s;
   int NBH, nC, Dk, Dv;
@@ -410,10 +410,10 @@ __device__ bool prep_body(PrepSmem& s, const CUtensorMap* tm_k, const CUtensorMa
   }
   __syncthreads();
   unit_lower_inverse(s.u);
-  if (ws.tinv) {  // a bf16 copy of T for the backward pass, rows and columns in scan order
+  if (ws.tinv) {  // a bf16 copy of T for the backward pass: scan order, [8][64][8] core matrices
     uint4* dst = reinterpret_cast<uint4*>(ws.tinv + ws.tile(dir, bh, j) * (64 * 64 * 2));
     for (int idx = tid; idx < 64 * 8; idx += kWideThreads) {
-      const int r = idx >> 3, ks = idx & 7;
+      const int r = idx & 63, ks = idx >> 6;
       dst[idx] = pack8_bf16(&s.u.T[r][8 * ks]);
     }
   }

@@ -30,7 +30,8 @@ struct ScanArgs {
   long long wait_limit;    // polls before a bounded wait gives up
   bool skip_output = false;  // chunked path: stages A and B only (workspace filled, out untouched)
   void* t_out = nullptr;     // chunked path: stage A also writes each chunk's (I + A)^-1, bf16
-                             // [64][64] in scan order, one 8 KB block per (dir, b*h, chunk)
+                             // in scan order as core matrices [8 column slabs][64 rows][8],
+                             // one 8 KB block per (dir, b*h, chunk)
 };
 
 // Kernel ids for the profiling hook.
