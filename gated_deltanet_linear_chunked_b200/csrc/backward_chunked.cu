@@ -53,6 +53,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kBcThreads = 256;
+constexpr long long kDrainPolls = 1LL << 40;  // drains are bounded by the 2 s timer
 constexpr int kLdE = 72;    // bf16 row stride of the 64 x 64 E tile
 // The gradient pass runs 16 warps: every phase has many independent 16 x 16
 // tiles, and with one CTA per SM the extra warps hide their latencies.
@@ -89,17 +90,6 @@ struct BcArgs {
 };
 
 __device__ __forceinline__ float bf(const __nv_bfloat16& x) { return __bfloat162float(x); }
-__device__ __forceinline__ void cp16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                   static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
-               "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-// Wait until at most N of this thread's committed cp.async groups are pending.
-template <int N>
-__device__ __forceinline__ void cp_wait_group() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // Element e (0..3) of a thread's accumulator tile: row and column offsets.
 __device__ __forceinline__ int tile_row(int e) { return ((threadIdx.x & 31) >> 2) + (e >= 2 ? 8 : 0); }
@@ -275,8 +265,12 @@ __device__ void gate_prefix(BcSmall& sm) {
   sm.eg[2 * lane + 1] = expf(incl);
 }
 // q^ = q / |q| and k^ = k / |k| in place, row by row, for two core-matrix
-// [Dk/8][64][8] tiles (a warp per row; rows of zeros stay zero).  No barrier.
-__device__ void normalize_rows_core(const BcArgs& a, __nv_bfloat16* sQ, __nv_bfloat16* sK) {
+// [Dk/8][64][8] tiles (a warp per row; rows of zeros stay zero); with sQs,
+// also e^gam times the rounded q^ there (eg by scan row; memory row r is scan
+// row 63 - r when rev).  No barrier.
+__device__ void normalize_rows_core(const BcArgs& a, __nv_bfloat16* sQ, __nv_bfloat16* sK,
+                                    __nv_bfloat16* sQs = nullptr, const float* eg = nullptr,
+                                    bool rev = false) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   const int Dk = a.Dk;
   uint32_t* q2 = reinterpret_cast<uint32_t*>(sQ);
@@ -304,106 +298,35 @@ __device__ void normalize_rows_core(const BcArgs& a, __nv_bfloat16* sQ, __nv_bfl
     for (int i = 0; i < 2; ++i) {
       const int d2 = lane + 32 * i, at = cidx(r, 2 * d2, 64, false) / 2;
       if (d2 < Dk / 2) {
-        q2[at] = pack_bf16x2(qv[i][0] * rq, qv[i][1] * rq);
+        const uint32_t qn = pack_bf16x2(qv[i][0] * rq, qv[i][1] * rq);
+        q2[at] = qn;
         k2[at] = pack_bf16x2(kv[i][0] * rk, kv[i][1] * rk);
+        if (sQs) {
+          const float e = eg[rev ? 63 - r : r];
+          float x0, x1;
+          unpack_bf16x2(qn, x0, x1);
+          reinterpret_cast<uint32_t*>(sQs)[at] = pack_bf16x2(x0 * e, x1 * e);
+        }
       }
     }
   }
 }
 
-// Stage chunk j of (b, h) in direction dir, rows in scan order: gates (zero
-// past T), q^ = q / |q|, k^ likewise (bf16), dO; gam (inclusive prefix sum of
-// g) and e^gam; with sQs, also diag(e^gam) q^ there.  Every thread of the
-// CTA takes part.  stage_rows_issue starts the row copies (one cp.async
-// group); stage_rows_finish<N> waits for them with N later groups still
-// pending, normalises, and ends with a barrier.
-__device__ void stage_rows_issue(const BcArgs& a, BcSmall& sm, __nv_bfloat16* sQ, __nv_bfloat16* sK,
-                                 __nv_bfloat16* sO, int lbk, int lbv, int b, int h, int dir, int j) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
-  const int Dk = a.Dk, Dv = a.Dv, t0 = 64 * j;
-  if (tid < 64) {
-    const int p = tid, t = t0 + (dir == 0 ? p : 63 - p);
-    const bool valid = t < a.T;
-    const size_t r = ((size_t)b * a.T + t) * a.H + h;
-    sm.row[p] = valid ? (int)r : -1;
-    sm.g[p] = valid ? __ldg(a.g + r) : 0.f;
-    sm.beta[p] = valid ? __ldg(a.beta + r) : 0.f;
-    sm.dgam[p] = 0.f;
-    sm.dbeta[p] = 0.f;
-    sm.cK[p] = 0.f;
-  }
-  __syncthreads();
-  const int ck = Dk / 8, cv = Dv / 8;
-  for (int p = warp; p < 64; p += nw) {  // a row's 16-byte pieces of q, k and dO across the lanes
-    const int r = sm.row[p];
-    for (int c = lane; c < 2 * ck + cv; c += 32) {
-      __nv_bfloat16* dst;
-      const __nv_bfloat16* src;
-      // row-major with strides lbk / lbv, or (lbk == 0) core-matrix [D/8][64][8]
-      if (c < ck) {
-        dst = sQ + (lbk ? p * lbk + 8 * c : (c * 64 + p) * 8);
-        src = a.q + (size_t)r * Dk + 8 * c;
-      } else if (c < 2 * ck) {
-        dst = sK + (lbk ? p * lbk + 8 * (c - ck) : ((c - ck) * 64 + p) * 8);
-        src = a.k + (size_t)r * Dk + 8 * (c - ck);
-      } else {
-        dst = sO + (lbk ? p * lbv + 8 * (c - 2 * ck) : ((c - 2 * ck) * 64 + p) * 8);
-        src = a.dout + (size_t)r * Dv + 8 * (c - 2 * ck);
-      }
-      if (r >= 0) cp16(dst, src);
-      else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-    }
-  }
-  cp_commit();
-  if (warp == 0) gate_prefix(sm);
-}
-template <int N>
-__device__ void stage_rows_finish(const BcArgs& a, BcSmall& sm, __nv_bfloat16* sQ, __nv_bfloat16* sK,
-                                  int lbk, __nv_bfloat16* sQs = nullptr) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  const int Dk = a.Dk;
-  cp_wait_group<N>();
-  __syncthreads();
-  for (int p = warp; p < 64; p += nw) {  // bf16 pairs: Dk / 2 <= 64, two per lane at most
-    // pair d2 of row p, in pairs: row-major with stride lbk, or (lbk == 0)
-    // core-matrix [Dk/8][64][8]
-    auto at2 = [&](int d2) { return lbk ? (p * lbk) / 2 + d2 : cidx(p, 2 * d2, 64, false) / 2; };
-    uint32_t* q2 = reinterpret_cast<uint32_t*>(sQ);
-    uint32_t* k2 = reinterpret_cast<uint32_t*>(sK);
-    float qv[2][2] = {}, kv[2][2] = {};
-    float qq = 0.f, kk = 0.f;
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int d2 = lane + 32 * i;
-      if (d2 < Dk / 2) {
-        unpack_bf16x2(q2[at2(d2)], qv[i][0], qv[i][1]);
-        unpack_bf16x2(k2[at2(d2)], kv[i][0], kv[i][1]);
-        qq = fmaf(qv[i][0], qv[i][0], fmaf(qv[i][1], qv[i][1], qq));
-        kk = fmaf(kv[i][0], kv[i][0], fmaf(kv[i][1], kv[i][1], kk));
-      }
-    }
-#pragma unroll
-    for (int off = 16; off; off >>= 1) {
-      qq += __shfl_xor_sync(0xffffffffu, qq, off);
-      kk += __shfl_xor_sync(0xffffffffu, kk, off);
-    }
-    const float rq = 1.f / sqrtf(fmaxf(qq, 1e-12f)), rk = 1.f / sqrtf(fmaxf(kk, 1e-12f));
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int d2 = lane + 32 * i;
-      if (d2 < Dk / 2) {
-        const uint32_t qn = pack_bf16x2(qv[i][0] * rq, qv[i][1] * rq);
-        q2[at2(d2)] = qn;
-        k2[at2(d2)] = pack_bf16x2(kv[i][0] * rk, kv[i][1] * rk);
-        if (sQs) {  // e^gam times the rounded q^
-          float x0, x1;
-          unpack_bf16x2(qn, x0, x1);
-          reinterpret_cast<uint32_t*>(sQs)[at2(d2)] = pack_bf16x2(x0 * sm.eg[p], x1 * sm.eg[p]);
-        }
-      }
-    }
-  }
-  __syncthreads();
+// Tile t of the chunk-parallel passes: chunk j fastest, then b*h, then direction.
+struct GrTile {
+  int j, bh, dir, b, h;
+  size_t bi;  // block index in the per-chunk buffers
+};
+__device__ __forceinline__ GrTile gr_tile(const BcArgs& a, int t) {
+  GrTile c;
+  c.j = t % a.nC;
+  const int rest = t / a.nC;
+  c.bh = rest % a.NBH;
+  c.dir = rest / a.NBH;
+  c.b = c.bh / a.H;
+  c.h = c.bh - c.b * a.H;
+  c.bi = a.blk(c.dir, c.bh, c.j);
+  return c;
 }
 
 // ---------------------------------------------------------------- pre pass
@@ -411,24 +334,23 @@ __device__ void stage_rows_finish(const BcArgs& a, BcSmall& sm, __nv_bfloat16* s
 // depend on the later chunks, stored transposed (X^T = dO^T P, Y^T = dO^T
 // diag(e^gam) Q^) in bf16.  Shared memory: q^, k^, dO, diag(e^gam) Q^, P (bf16).
 struct PreLayout {
-  int lbk, lbv;
   uint32_t q, k, dout, qs, P, small, total;
   __host__ __device__ PreLayout(int Dk, int Dv) {
-    lbk = Dk + 8;
-    lbv = Dv + 8;
-    uint32_t o = 0;
-    q = o;    o += 64 * lbk * 2;
-    k = o;    o += 64 * lbk * 2;
-    dout = o; o += 64 * lbv * 2;
-    qs = o;   o += 64 * lbk * 2;    // diag(e^gam) Q^ (bf16)
-    P = o;    o += 64 * kLdE * 2;   // M o (Q^ K^^T) (bf16)
+    uint32_t o = 0;  // q, k, dO: TMA tiles, core-matrix [D/8][64][8] in time order
+    q = o;    o += 64 * Dk * 2;
+    k = o;    o += 64 * Dk * 2;
+    dout = o; o += 64 * Dv * 2;
+    qs = o;   o += 64 * Dk * 2;     // diag(e^gam) Q^ (bf16, the same layout)
+    P = o;    o += 64 * kLdE * 2;   // M o (Q^ K^^T) (bf16, row-major, scan order)
     small = o; o += sizeof(BcSmall);
     total = (o + 15) & ~15u;
   }
 };
 
-__global__ void __launch_bounds__(kBcThreads) gdn_bwd_pre_kernel(BcArgs a) {
-  extern __shared__ __align__(16) uint8_t bp_raw[];
+__global__ void __launch_bounds__(kBcThreads)
+gdn_bwd_pre_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_o, BcArgs a) {
+  extern __shared__ __align__(128) uint8_t bp_raw[];
   using bf16 = __nv_bfloat16;
   const int Dk = a.Dk, Dv = a.Dv;
   const PreLayout L(Dk, Dv);
@@ -440,12 +362,36 @@ __global__ void __launch_bounds__(kBcThreads) gdn_bwd_pre_kernel(BcArgs a) {
   BcSmall& sm = *reinterpret_cast<BcSmall*>(bp_raw + L.small);
   const int j = blockIdx.x, bh = blockIdx.y, dir = blockIdx.z;
   const int b = bh / a.H, h = bh - b * a.H;
-  const int lbk = L.lbk, lbv = L.lbv;
-  stage_rows_issue(a, sm, sQ, sK, sO, lbk, lbv, b, h, dir, j);
-  stage_rows_finish<0>(a, sm, sQ, sK, lbk, sQs);
+  const int tid = threadIdx.x;
+  const GrTile c = gr_tile(a, j + a.nC * (bh + a.NBH * dir));
+  // the gates by 64 threads; q, k, dO by TMA (one thread, one mbarrier)
+  if (tid < 64) {
+    const int t = 64 * j + (dir == 0 ? tid : 63 - tid);
+    const bool valid = t < a.T;
+    const size_t r = ((size_t)b * a.T + t) * a.H + h;
+    sm.g[tid] = valid ? __ldg(a.g + r) : 0.f;
+  }
+  if (tid == 0) {
+    mbar_init(&sm.full[0], 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(&sm.full[0], 64 * (2 * Dk + Dv) * 2);
+    tma_load_tile(sQ, &tm_q, &sm.full[0], 64 * c.j, c.h, c.b);
+    tma_load_tile(sK, &tm_k, &sm.full[0], 64 * c.j, c.h, c.b);
+    tma_load_tile(sO, &tm_o, &sm.full[0], 64 * c.j, c.h, c.b);
+  }
+  __syncthreads();
+  if ((tid >> 5) == 0) gate_prefix(sm);
+  if (!__syncthreads_and(mbar_wait(&sm.full[0], 0, a.limit))) {
+    if (tid == 0) atomicOr(a.err, kErrTimeout);
+    mbar_wait(&sm.full[0], 0, kDrainPolls);  // nothing may land after the CTA leaves
+    return;
+  }
+  const bool rev = dir != 0;  // the tiles' time rows run against the scan
+  normalize_rows_core(a, sQ, sK, sQs, sm.eg, rev);
+  __syncthreads();
   auto none = [](int, int, float) { return 0.f; };
-  const BMat Q = row_major(sQ, lbk), K = row_major(sK, lbk), O = row_major(sO, lbv);
-  const BMat Qs = row_major(sQs, lbk), Pm = row_major(sP, kLdE);
+  const BMat Q = core_mat(sQ, 64, rev), K = core_mat(sK, 64, rev), O = core_mat(sO, 64, rev);
+  const BMat Qs = core_mat(sQs, 64, rev), Pm = row_major(sP, kLdE);
   gemm2<false, true, false, true>(64, 64, Q, K, Dk, Q, K, 0, none, [&](int m, int n, float v) {
     sP[m * kLdE + n] = __float2bfloat16_rn(n <= m ? expf(sm.gam[m] - sm.gam[n]) * v : 0.f);
   }, nullptr, nullptr);
@@ -475,7 +421,6 @@ __global__ void __launch_bounds__(kBcThreads) gdn_bwd_pre_kernel(BcArgs a) {
 constexpr int kChSlices = 1;
 constexpr int kChStages = 2;
 constexpr int kChThreads = 32 * (4 * kChSlices + 1);
-constexpr long long kChDrainPolls = 1LL << 40;  // drains are bounded by the 2 s timer
 
 struct ChainBarsBwd {
   uint64_t full[kChStages], empty[kChStages];
@@ -524,7 +469,7 @@ __device__ void bwd_chain_loads(const BcArgs& a, uint8_t* smem, const ChainSmem&
   // nothing may still be landing in shared memory when the CTA leaves
   for (int st = 0; st < kChStages && st < issued; ++st) {
     const int last = st + ((issued - 1 - st) / kChStages) * kChStages;
-    mbar_wait(&bars.full[st], (last / kChStages) & 1, kChDrainPolls);
+    mbar_wait(&bars.full[st], (last / kChStages) & 1, kDrainPolls);
   }
 }
 
@@ -873,23 +818,6 @@ __device__ __forceinline__ void store_acc(int N, const float (&acc)[kMaxBlocks][
   }
 }
 
-// Gradient-pass tile t: chunk j fastest, then b*h, then direction.
-struct GrTile {
-  int j, bh, dir, b, h;
-  size_t bi;  // block index in the per-chunk buffers
-};
-__device__ __forceinline__ GrTile gr_tile(const BcArgs& a, int t) {
-  GrTile c;
-  c.j = t % a.nC;
-  const int rest = t / a.nC;
-  c.bh = rest % a.NBH;
-  c.dir = rest / a.NBH;
-  c.b = c.bh / a.H;
-  c.h = c.bh - c.b * a.H;
-  c.bi = a.blk(c.dir, c.bh, c.j);
-  return c;
-}
-
 // Persistent: CTA x walks tiles x, x + gridDim.x, ...; each group of the
 // next tile's inputs is fetched by one thread as soon as this tile has done
 // with the buffers it lands in, so the next tile starts with its data on chip.
@@ -1009,7 +937,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     for (int g = 0; g < 5; ++g) ok = mbar_wait(&full[g], it & 1, a.limit) && ok;
     if (!__syncthreads_and(ok)) {
       if (tid == 0) atomicOr(a.err, kErrTimeout);
-      for (int g = 0; g < 5; ++g) mbar_wait(&full[g], it & 1, kChDrainPolls);  // nothing may land after exit
+      for (int g = 0; g < 5; ++g) mbar_wait(&full[g], it & 1, kDrainPolls);  // nothing may land after exit
       return;
     }
   }
@@ -1030,9 +958,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   gemm2<false, true, false, true>(64, 64, K, K, Dk, K, K, 0, none, [&](int m, int n, float v) {
     sE[m * kLdE + n] = __float2bfloat16_rn(n < m ? expf(sm.gam[m] - sm.gam[n]) * v : 0.f);
   }, nullptr, nullptr);
-  // every staged tile
-  cp_wait_all();
-  __syncthreads();
+  __syncthreads();  // P and E complete
   // ---- 3. dK~ = U dS_e^T: dk^ starts as e^{gam_C - gam} dK~; c_m = k^_m . dk^_m
   float dk[kMaxBlocks][2][4], dq[kMaxBlocks][2][4];
 #pragma unroll
@@ -1285,7 +1211,7 @@ cudaError_t launch_backward_chunked(const BwdCall& c, void* workspace, float** p
   const dim3 per_chunk((unsigned)nC, (unsigned)NBH, ndir);
   {
     ProfileScope ps(c.stream, kKernBwdChunk);
-    gdn_bwd_pre_kernel<<<per_chunk, kBcThreads, smem_pre, c.stream>>>(a);
+    gdn_bwd_pre_kernel<<<per_chunk, kBcThreads, smem_pre, c.stream>>>(tq, tk, to, a);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   {
