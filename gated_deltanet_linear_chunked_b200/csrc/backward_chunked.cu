@@ -64,7 +64,6 @@ constexpr int kMaxBlocks = 2;  // 16 x 16 output blocks per warp of a 64 x Dk pr
 struct BcSmall {
   float g[64], beta[64], gam[64], eg[64], dgam[64], dbeta[64], cK[64];
   int row[64];  // (b, t, h) row of scan position p, -1 past T
-  float red[kGrWarps];
   uint64_t full[5];  // the gradient pass's staged tile groups have landed
 };
 
@@ -82,6 +81,7 @@ struct BcArgs {
   __nv_bfloat16* dUT;        // dU^T, Dv x 64, core-matrix [64/8][Dv][8]
   __nv_bfloat16* dSeT;       // dS_e^T, Dv x Dk, [Dk/8][Dv][8] (dS_e: gradient of the chunk's end state)
   const __nv_bfloat16* tinv; // (I + A)^-1 from the forward's stage A, [64/8][64][8] (scan order)
+  float* dot;                // <dS_e, S0> (bf16 operands): zeroed by the pre pass, summed by the chain
   float *pq, *pk, *pab, *dvb;  // [dir][rows][Dk], [dir][rows][Dk], [dir][rows][2], [dir][rows][Dv] (dX_u)
   int B, T, H, Dk, Dv, nC, NBH;
   unsigned* err;             // device error word (the chain's bounded waits)
@@ -397,6 +397,7 @@ gdn_bwd_pre_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   }, nullptr, nullptr);
   __syncthreads();
   const size_t blk = a.blk(dir, bh, j);
+  if (tid == 0) a.dot[blk] = 0.f;  // the chain pass adds into it
   gemm_store_frag<true, false>(Dv, 64, O, Pm, 64, a.XT + blk * Dv * 64);
   gemm_store_frag<true, false>(Dv, Dk, O, Qs, 64, a.YT + blk * Dv * Dk);
 }
@@ -429,14 +430,15 @@ struct ChainBarsBwd {
 static_assert(sizeof(ChainBarsBwd) <= 128, "the chain's barriers fit their slot");
 
 struct ChainSmem {
-  uint32_t xs, xu, stage0, stage, xt, yt, total;
+  uint32_t xs, xu, stage0, stage, xt, yt, s0, total;
   __host__ __device__ explicit ChainSmem(int Dk) {
     xs = 128;                                   // dS_e^T A fragments: [slice][Dk/16][32 lanes][16 B]
     xu = xs + kChSlices * (Dk / 16) * 512;      // dU^T A fragments: [slice][4][32 lanes][16 B]
     stage0 = (xu + kChSlices * 2048 + 127) & ~127u;
     xt = (Dk * 256 + 16 + 127) & ~127u;         // after W, K~ and e^{gam_C}
     yt = xt + kChSlices * 16 * 64 * 2;
-    stage = (yt + kChSlices * 16 * Dk * 2 + 127) & ~127u;
+    s0 = yt + kChSlices * 16 * Dk * 2;          // the slices' columns of S0: [2 slice][Dk][8]
+    stage = (s0 + kChSlices * 16 * Dk * 2 + 127) & ~127u;
     total = stage0 + kChStages * stage;
   }
 };
@@ -449,6 +451,7 @@ __device__ void bwd_chain_loads(const BcArgs& a, uint8_t* smem, const ChainSmem&
   const int Dk = a.Dk, Dv = a.Dv, nC = a.nC;
   const uint32_t wk_bytes = Dk * 256 + 16;
   const uint32_t xt_bytes = active * 16 * 64 * 2, yt_bytes = active * 16 * Dk * 2;
+  const uint32_t s0_bytes = active * 16 * Dk * 2;
   int issued = 0;
   bool ok = true;
   for (; issued < nC; ++issued) {
@@ -460,8 +463,10 @@ __device__ void bwd_chain_loads(const BcArgs& a, uint8_t* smem, const ChainSmem&
     }
     const size_t blk = a.blk(dir, bh, dir == 0 ? nC - 1 - issued : issued);
     uint8_t* dst = smem + L.stage0 + st * L.stage;
-    mbar_arrive_expect_tx(&bars.full[st], wk_bytes + xt_bytes + yt_bytes);
+    mbar_arrive_expect_tx(&bars.full[st], wk_bytes + xt_bytes + yt_bytes + s0_bytes);
     bulk_load(dst, a.ws + blk * a.wl.block_bytes + a.wl.off_w, wk_bytes, &bars.full[st]);
+    bulk_load(dst + L.s0, a.ws + blk * a.wl.block_bytes + a.wl.off_s + (size_t)s0 * 2 * Dk * 16, s0_bytes,
+              &bars.full[st]);
     bulk_load(dst + L.xt, a.XT + (blk * Dv + 16 * s0) * 64, xt_bytes, &bars.full[st]);
     bulk_load(dst + L.yt, a.YT + (blk * Dv + 16 * s0) * Dk, yt_bytes, &bars.full[st]);
   }
@@ -535,12 +540,16 @@ __global__ void __launch_bounds__(kChThreads, 2) gdn_bwd_chain_kernel(BcArgs a) 
     // fragment order, and to the gradient pass
     // (dS_e^T of the block: core-matrix [Dk/8][Dv][8], rows c, columns d)
     uint32_t* dse = reinterpret_cast<uint32_t*>(a.dSeT + blk * Dv * Dk);
+    uint32_t fse[KPW][4];  // this warp's dS_e^T blocks in bf16 (kept for <dS_e, S0>)
 #pragma unroll
     for (int i = 0; i < KPW; ++i) {
       const int kb = q + 4 * i;
       if (kb < NKB) {
-        const uint32_t f[4] = {pack_bf16x2(S[i][0][0], S[i][0][1]), pack_bf16x2(S[i][0][2], S[i][0][3]),
-                               pack_bf16x2(S[i][1][0], S[i][1][1]), pack_bf16x2(S[i][1][2], S[i][1][3])};
+        uint32_t (&f)[4] = fse[i];
+        f[0] = pack_bf16x2(S[i][0][0], S[i][0][1]);
+        f[1] = pack_bf16x2(S[i][0][2], S[i][0][3]);
+        f[2] = pack_bf16x2(S[i][1][0], S[i][1][1]);
+        f[3] = pack_bf16x2(S[i][1][2], S[i][1][3]);
         st_shared_v4(xs_u + kb * 512, f);
         const int c = c0 + gq, d = 16 * kb + 2 * tq;
         dse[(((d >> 3) * Dv + c) * 8 + (d & 7)) >> 1] = f[0];
@@ -653,6 +662,32 @@ __global__ void __launch_bounds__(kChThreads, 2) gdn_bwd_chain_kernel(BcArgs a) 
             for (int e = 0; e < 4; ++e) S[i][h][e] += s2[h][e];
         }
       }
+    }
+    {  // this warp's share of <dS_e, S0> (bf16 operands, as the gradient pass's
+       // products use them), while the MMAs above run: fse[i][2 h + rr] holds
+       // columns gq + 8 rr, rows d, d + 1 (d = 16 kb + 8 h + 2 tq); the staged
+       // slice of S0 is [2][Dk][8] (rows d)
+      const __nv_bfloat16* s0s = reinterpret_cast<const __nv_bfloat16*>(sb + L.s0) + g * 16 * Dk;
+      float dot = 0.f;
+#pragma unroll
+      for (int i = 0; i < KPW; ++i) {
+        const int kb = q + 4 * i;
+        if (kb < NKB) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+              const int d = 16 * kb + 8 * h + 2 * tq;
+              float x0, x1;
+              unpack_bf16x2(fse[i][2 * h + rr], x0, x1);
+              dot = fmaf(x0, bf(s0s[(rr * Dk + d) * 8 + gq]), dot);
+              dot = fmaf(x1, bf(s0s[(rr * Dk + d + 1) * 8 + gq]), dot);
+            }
+        }
+      }
+#pragma unroll
+      for (int off = 16; off; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+      if (lane == 0) atomicAdd(a.dot + blk, dot);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars.empty[st]);  // this warp's reads of the stage are done
@@ -968,15 +1003,6 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   }
   gemm_acc2<false, false>(Dk, Dv, Um, dSTm, dk, [&](int m) { return expf(gamC - sm.gam[m]); });
   acc_row_sums(Dk, wc, [&](int i, int hh, int e, int m, int n) { return bf(sK[cidx(m, n, 64, rev)]) * dk[i][hh][e]; });
-  {  // <dS_e, S0> -> dgam_C
-    float dot = 0.f;
-    for (int c = warp; c < Dv; c += kGrWarps)
-      for (int d = lane; d < Dk; d += 32)
-        dot = fmaf(bf(sdST[cidx(c, d, Dv, false)]), bf(sS0[cidx(d, c, Dk, false)]), dot);
-#pragma unroll
-    for (int off = 16; off; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-    if (lane == 0) sm.red[warp] = dot;  // summed after the last barrier
-  }
   // ---- 5. dP = dO U^T -> dQK = M o dP (in place of P); gam gets dP o P
   gemm2<false, true, false, true>(64, 64, O, Um, Dv, O, Um, 0,
       [&](int m, int n, float v) { return n <= m ? v * bf(sP[m * kLdE + n]) : 0.f; },
@@ -1084,10 +1110,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     float cs = sm.cK[2 * lane] + sm.cK[2 * lane + 1];
 #pragma unroll
     for (int off = 16; off; off >>= 1) cs += __shfl_xor_sync(0xffffffffu, cs, off);
-    float dgamC = 0.f;  // e^{gam_C} <dS_e, S0>
-#pragma unroll
-    for (int w = 0; w < kGrWarps; ++w) dgamC += sm.red[w];
-    const float dC = eC * dgamC + cs;
+    const float dC = eC * __ldg(a.dot + cur.bi) + cs;  // e^{gam_C} <dS_e, S0> (the chain's sum)
     const float d0 = sm.dgam[2 * lane] - sm.cK[2 * lane];
     const float d1 = sm.dgam[2 * lane + 1] - sm.cK[2 * lane + 1];
     float incl = d0 + d1;  // suffix sums over scan positions 2 lane, 2 lane + 1 .. 63
@@ -1119,7 +1142,7 @@ bool bwd_chunked_fits(int Dk, int Dv) {
 
 namespace {
 struct BwdScratch {
-  size_t fwd, tinv, xt, yt, dut, dset, pq, pk, pab, dvb, total;
+  size_t fwd, tinv, xt, yt, dut, dset, dot, pq, pk, pab, dvb, total;
   BwdScratch(int B, int T, int H, int Dk, int Dv, bool bidir) {
     const size_t ndir = bidir ? 2 : 1, rows = (size_t)B * T * H, NBH = (size_t)B * H;
     const size_t blocks = ndir * NBH * ((T + 63) / 64);
@@ -1131,6 +1154,7 @@ struct BwdScratch {
     yt = o;   o += al(blocks * (size_t)Dk * Dv * 2);
     dut = o;  o += al(blocks * 64 * Dv * 2);
     dset = o; o += al(blocks * (size_t)Dk * Dv * 2);
+    dot = o;  o += al(blocks * 4);
     pq = o;  o += al(ndir * rows * Dk * 4);
     pk = o;  o += al(ndir * rows * Dk * 4);
     pab = o; o += al(ndir * rows * 2 * 4);
@@ -1176,6 +1200,7 @@ cudaError_t launch_backward_chunked(const BwdCall& c, void* workspace, float** p
   a.YT = reinterpret_cast<__nv_bfloat16*>(base + W.yt);
   a.dUT = reinterpret_cast<__nv_bfloat16*>(base + W.dut);
   a.dSeT = reinterpret_cast<__nv_bfloat16*>(base + W.dset);
+  a.dot = reinterpret_cast<float*>(base + W.dot);
   a.err = c.err;
   a.limit = c.wait_limit;
   a.pq = reinterpret_cast<float*>(base + W.pq);
