@@ -735,26 +735,30 @@ ChainKernel chain_kernel_for(int nkb) {
 // T = (I + A)^-1, which its stage A leaves in the workspace.
 struct GradLayout {
   int lbk, lbv;
-  uint32_t q, k, dout, w, ut, u, s0, dse, P, Tb, E, dU, dW, part, small, total;
+  uint32_t q, k, dout, w, ut, u, s0, dse, P, Tb, E, dU, dW, xw, xu, part, small, total;
   __host__ __device__ GradLayout(int Dk, int Dv) {
     lbk = Dk + 8;
     lbv = Dv + 8;
     uint32_t o = 0;
     // core-matrix tiles [cols/8][rows][8], as their sources store them
-    q = o;    o += 64 * Dk * 2;     // q^ (scan rows), then dX_w
-    k = o;    o += 64 * Dk * 2;     // k^ (scan rows)
-    dout = o; o += 64 * Dv * 2;     // dO (scan rows), then dX_u
+    q = o;    o += 64 * Dk * 2;     // q^ (time rows)
+    k = o;    o += 2 * 64 * Dk * 2; // k^ (time rows), two buffers: this chunk's and the next's
+    dout = o; o += 64 * Dv * 2;     // dO (time rows)
     w = o;    o += 64 * Dk * 2;     // W  (time rows)
     ut = o;   o += 64 * Dv * 2;     // U~ (time rows)
     u = o;    o += 64 * Dv * 2;     // U  (time rows)
-    s0 = o;   o += Dk * Dv * 2;     // S0: rows d, columns c
-    dse = o;  o += Dv * Dk * 2;     // dS_e^T: rows c, columns d
+    s0 = o;   o += Dk * Dv * 2;     // S0: rows d, columns c; then dX_u (64 x Dv)
+    dse = o;  o += Dv * Dk * 2;     // dS_e^T: rows c, columns d; then dX_w (64 x Dk)
     Tb = o;   o += 64 * 64 * 2;     // T = (I + A)^-1 (scan rows)
     dU = o;   o += 64 * Dv * 2;     // dU^T: rows c, columns p
     // row-major tiles the pass writes itself
     P = o;    o += 64 * kLdE * 2;   // P, then dQK, then dA / dG (bf16)
     E = o;    o += 64 * kLdE * 2;   // e^{gam_p - gam_i} K^ K^T (i < p), bf16
     dW = o;   o += 64 * lbk * 2;    // dW (bf16)
+    // dX_w (64 x Dk) and dX_u (64 x Dv), core-matrix, in the dS_e^T and S0
+    // tiles where they fit (Dv >= 64, Dk >= 64), else tiles of their own
+    if (Dv >= 64) xw = dse; else { xw = o; o += 64 * Dk * 2; }
+    if (Dk >= 64) xu = s0; else { xu = o; o += 64 * Dv * 2; }
     part = o; o += 3 * kGrWarps * 64 * 4;  // per-warp partial row sums of dgam, dbeta, c
     small = o; o += sizeof(BcSmall);
     total = (o + 15) & ~15u;
@@ -887,22 +891,24 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const size_t rows_bth = (size_t)a.B * a.T * a.H;
   // Tile groups, each landing on its own mbarrier (one phase per tile):
-  //   0: U, dS_e^T   1: S0   2: T, dU^T   3: q, dO, W, U~   4: k
+  //   0: U, dO   1: q   2: T, dU^T   3: S0, dS_e^T, W, U~   4: k (two buffers)
   // Group g of the next tile is issued (by one thread) right after the
-  // barrier behind which this tile last reads group g's buffers.
+  // barrier behind which this tile last reads group g's buffers; k, double
+  // buffered, at the start of this tile.
   uint64_t* full = sm.full;
+  int kbuf = 1;  // the k buffer of the current tile (the first tile's k goes to buffer 0)
   auto issue = [&](int g, const GrTile& c) {
     const uint8_t* blk = a.ws + c.bi * a.wl.block_bytes;
     fence_proxy_async_smem();  // the buffers' last generic accesses come first
     switch (g) {
       case 0:
-        mbar_arrive_expect_tx(&full[0], 64 * Dv * 2 + Dv * Dk * 2);
+        mbar_arrive_expect_tx(&full[0], 64 * Dv * 2 + 64 * Dv * 2);
         bulk_load(sU, blk + a.wl.off_u, 64 * Dv * 2, &full[0]);
-        bulk_load(sdST, a.dSeT + c.bi * Dv * Dk, Dv * Dk * 2, &full[0]);
+        tma_load_tile(sO, &tm_o, &full[0], 64 * c.j, c.h, c.b);
         break;
       case 1:
-        mbar_arrive_expect_tx(&full[1], Dk * Dv * 2);
-        bulk_load(sS0, blk + a.wl.off_s, Dk * Dv * 2, &full[1]);
+        mbar_arrive_expect_tx(&full[1], 64 * Dk * 2);
+        tma_load_tile(sQ, &tm_q, &full[1], 64 * c.j, c.h, c.b);
         break;
       case 2:
         mbar_arrive_expect_tx(&full[2], 64 * 64 * 2 + 64 * Dv * 2);
@@ -910,15 +916,15 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         bulk_load(sdU, a.dUT + c.bi * Dv * 64, 64 * Dv * 2, &full[2]);
         break;
       case 3:
-        mbar_arrive_expect_tx(&full[3], 2 * 64 * Dk * 2 + 2 * 64 * Dv * 2);
-        tma_load_tile(sQ, &tm_q, &full[3], 64 * c.j, c.h, c.b);
-        tma_load_tile(sO, &tm_o, &full[3], 64 * c.j, c.h, c.b);
+        mbar_arrive_expect_tx(&full[3], 2 * Dk * Dv * 2 + 64 * Dk * 2 + 64 * Dv * 2);
+        bulk_load(sS0, blk + a.wl.off_s, Dk * Dv * 2, &full[3]);
+        bulk_load(sdST, a.dSeT + c.bi * Dv * Dk, Dv * Dk * 2, &full[3]);
         bulk_load(sW, blk + a.wl.off_w, 64 * Dk * 2, &full[3]);
         bulk_load(sUt, blk + a.wl.off_ut, 64 * Dv * 2, &full[3]);
         break;
-      default:
+      default:  // into the k buffer the tile after this one uses
         mbar_arrive_expect_tx(&full[4], 64 * Dk * 2);
-        tma_load_tile(sK, &tm_k, &full[4], 64 * c.j, c.h, c.b);
+        tma_load_tile(sK + (kbuf ^ 1) * 64 * Dk, &tm_k, &full[4], 64 * c.j, c.h, c.b);
         break;
     }
   };
@@ -948,6 +954,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     if (tid == 0)
       for (int g = 0; g < 5; ++g) issue(g, c);
   }
+  kbuf = 0;
   for (int it = 0; t < ntiles; t += gridDim.x, ++it) {
   const GrTile cur = gr_tile(a, t);
   const bool more = t + (int)gridDim.x < ntiles;
@@ -976,11 +983,13 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       return;
     }
   }
-  normalize_rows_core(a, sQ, sK);  // per memory row: the order of the rows does not matter
+  bf16* const sKc = sK + kbuf * 64 * Dk;  // this tile's k^
+  if (more && tid == 0) issue(4, nxt);  // the other k buffer was last read by the previous tile
+  normalize_rows_core(a, sQ, sKc);  // per memory row: the order of the rows does not matter
   __syncthreads();
   const float gamC = sm.gam[63], eC = expf(gamC);
   const bool rev = dir != 0;  // the tiles' time rows run against the scan
-  const BMat Q = core_mat(sQ, 64, rev), K = core_mat(sK, 64, rev), O = core_mat(sO, 64, rev);
+  const BMat Q = core_mat(sQ, 64, rev), K = core_mat(sKc, 64, rev), O = core_mat(sO, 64, rev);
   const BMat Wm = core_mat(sW, 64, rev), Ut = core_mat(sUt, 64, rev), Um = core_mat(sU, 64, rev);
   const BMat S0 = core_mat(sS0, Dk, false), dSTm = core_mat(sdST, Dv, false);
   const BMat dUTm = core_mat(sdU, Dv, false), Pm = row_major(sP, kLdE), dWm = row_major(sdW, lbk);
@@ -1002,7 +1011,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     zero2(dq[i]);
   }
   gemm_acc2<false, false>(Dk, Dv, Um, dSTm, dk, [&](int m) { return expf(gamC - sm.gam[m]); });
-  acc_row_sums(Dk, wc, [&](int i, int hh, int e, int m, int n) { return bf(sK[cidx(m, n, 64, rev)]) * dk[i][hh][e]; });
+  acc_row_sums(Dk, wc, [&](int i, int hh, int e, int m, int n) { return bf(sKc[cidx(m, n, 64, rev)]) * dk[i][hh][e]; });
   // ---- 5. dP = dO U^T -> dQK = M o dP (in place of P); gam gets dP o P
   gemm2<false, true, false, true>(64, 64, O, Um, Dv, O, Um, 0,
       [&](int m, int n, float v) { return n <= m ? v * bf(sP[m * kLdE + n]) : 0.f; },
@@ -1013,7 +1022,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   // ---- 6. Z = diag(e^gam) dO S0^T -> dq^; gam_p gets q^_p . Z_p
   gemm_acc2<false, true>(Dk, Dv, O, S0, dq, [&](int m) { return sm.eg[m]; });
   acc_row_sums(Dk, wg, [&](int i, int hh, int e, int m, int n) { return bf(sQ[cidx(m, n, 64, rev)]) * dq[i][hh][e]; });
-  __syncthreads();  // dQK complete; U and dS_e^T are read no more
+  __syncthreads();  // dQK complete; U and dO are read no more
   if (more && tid == 0) issue(0, nxt);
   // ---- 7. dq^ += dQK K^;  8. dk^ += dQK^T Q^
   gemm_acc2<false, false>(Dk, 64, Pm, K, dq, [](int) { return 1.f; });
@@ -1022,13 +1031,13 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   // ---- 9. dW = -dU S0^T
   gemm2<true, true, true, true>(64, Dk, dUTm, S0, Dv, dUTm, S0, 0, none,
       [&](int m, int n, float v) { sdW[m * lbk + n] = __float2bfloat16_rn(-v); }, nullptr, nullptr);
-  __syncthreads();  // S0 is read no more
+  __syncthreads();  // q^ is read no more
   if (more && tid == 0) issue(1, nxt);
   // ---- 10. [dX_w | dX_u] solves (I + A)^T X = [dW | dU]: X = T^T [dW | dU]
   //          with the forward's own T, into the tiles of q^ and dO (neither
   //          is read again)
-  bf16* sXw = sQ;
-  bf16* sXu = sO;
+  bf16* sXw = reinterpret_cast<bf16*>(bg_raw + L.xw);  // dS_e^T is read no more after step 3,
+  bf16* sXu = reinterpret_cast<bf16*>(bg_raw + L.xu);  // S0 after step 9
   {
     const BMat Tt = core_mat(sT, 64, false);
     gemm2<true, false, true, false>(64, Dk, Tt, dWm, 64, Tt, Tt, 0, none,
@@ -1039,32 +1048,28 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   __syncthreads();  // T and dU^T are read no more
   if (more && tid == 0) issue(2, nxt);
   const BMat Xw = core_mat(sXw, 64, false), Xu = core_mat(sXu, 64, false);
-  // ---- 11. dk^ += diag(beta e^gam) dX_w; dX_u goes out as it is (the
-  //          reduction forms dv = beta dX_u and beta's share v . dX_u);
-  //          beta and gam from the rows of X_w = diag(beta e^gam) K^
+  // ---- 11. dk^ += diag(beta e^gam) dX_w; beta and gam from the rows of
+  //          X_w = diag(beta e^gam) K^ (s_p = k^_p . dX_w_p gives e^gam_p s_p
+  //          to beta_p and beta_p e^gam_p s_p to gam_p); dX_u goes out as it
+  //          is (the reduction forms dv = beta dX_u and beta's v . dX_u)
   for_acc(Dk, [&](int i, int hh, int e, int m, int n) {
     dk[i][hh][e] = fmaf(sm.beta[m] * sm.eg[m], bf(sXw[cidx(m, n, 64, false)]), dk[i][hh][e]);
   });
-  for (int p = warp; p < 64; p += kGrWarps) {
+  acc_row_sums(Dk, wb, [&](int, int, int, int m, int n) {
+    return sm.eg[m] * bf(sKc[cidx(m, n, 64, rev)]) * bf(sXw[cidx(m, n, 64, false)]);
+  });
+  acc_row_sums(Dk, wg, [&](int, int, int, int m, int n) {
+    return sm.beta[m] * sm.eg[m] * bf(sKc[cidx(m, n, 64, rev)]) * bf(sXw[cidx(m, n, 64, false)]);
+  });
+  for (int p = warp; p < 64; p += kGrWarps) {  // dX_u rows: four columns (8 bytes) a lane
     const int r = sm.row[p];
-    float sw = 0.f;
-    for (int d2 = lane; d2 < Dk / 2; d2 += 32) {
-      float k0, k1, w0, w1;
-      unpack_bf16x2(*reinterpret_cast<const uint32_t*>(sK + cidx(p, 2 * d2, 64, rev)), k0, k1);
-      unpack_bf16x2(*reinterpret_cast<const uint32_t*>(sXw + cidx(p, 2 * d2, 64, false)), w0, w1);
-      sw = fmaf(k0, w0, fmaf(k1, w1, sw));
-    }
-    if (r >= 0)
-      for (int c2 = lane; c2 < Dv / 2; c2 += 32) {
-        float x0, x1;
-        unpack_bf16x2(*reinterpret_cast<const uint32_t*>(sXu + cidx(p, 2 * c2, 64, false)), x0, x1);
-        *reinterpret_cast<float2*>(dvb + (size_t)r * Dv + 2 * c2) = make_float2(x0, x1);
-      }
-#pragma unroll
-    for (int off = 16; off; off >>= 1) sw += __shfl_xor_sync(0xffffffffu, sw, off);
-    if (lane == 0) {
-      wb[p] += sm.eg[p] * sw;
-      wg[p] += sm.beta[p] * sm.eg[p] * sw;
+    if (r < 0) continue;
+    for (int c4 = lane; c4 < Dv / 4; c4 += 32) {
+      const uint2 x = *reinterpret_cast<const uint2*>(sXu + cidx(p, 4 * c4, 64, false));
+      float f0, f1, f2, f3;
+      unpack_bf16x2(x.x, f0, f1);
+      unpack_bf16x2(x.y, f2, f3);
+      *reinterpret_cast<float4*>(dvb + (size_t)r * Dv + 4 * c4) = make_float4(f0, f1, f2, f3);
     }
   }
   // ---- 12. dA = -(dX_w W^T + dX_u U~^T) on i < p (into P); gam from A
@@ -1072,7 +1077,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       [&](int m, int n, float v) { return n < m ? -v * sm.beta[m] * bf(sE[m * kLdE + n]) : 0.f; },
       [&](int m, int n, float v) { sP[m * kLdE + n] = __float2bfloat16_rn(n < m ? -v : 0.f); },
       wg, wg);
-  __syncthreads();  // dX_w, dX_u (in the q^ and dO tiles), W and U~ are read no more
+  __syncthreads();  // dX_w, dX_u (in the dS_e^T and S0 tiles), W and U~ are read no more
   if (more && tid == 0) issue(3, nxt);
   for (int p = warp; p < 64; p += kGrWarps) {  // dbeta_p += sum_i dA_pi E_pi; dG = dA beta_p e^{..}
     float sb = 0.f;
@@ -1091,11 +1096,8 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   gemm_acc2<true, false>(Dk, 64, Pm, K, dk, [](int) { return 1.f; });
   // ---- 14. outputs: dk^, dbeta, dg = suffix sum of dgam + dgam_C
   store_acc(Dk, dk, pk, Dk, sm.row);
-  __syncthreads();  // every partial row sum is done; k^ is read no more
-  if (more) {
-    if (tid == 0) issue(4, nxt);
-    load_gates(nxt);
-  }
+  __syncthreads();  // every partial row sum is done
+  if (more) load_gates(nxt);
   if (tid < 3 * 64) {  // the warps' partials: dgam, dbeta, c
     const float* src = part + (tid >> 6) * kGrWarps * 64 + (tid & 63);
     float acc = 0.f;
@@ -1131,6 +1133,7 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
   }
   __syncthreads();  // the next tile rewrites sm
+  kbuf ^= 1;
   }
 }
 
