@@ -265,48 +265,42 @@ __device__ void gate_prefix(BcSmall& sm) {
   sm.eg[2 * lane + 1] = expf(incl);
 }
 // q^ = q / |q| and k^ = k / |k| in place, row by row, for two core-matrix
-// [Dk/8][64][8] tiles (a warp per row; rows of zeros stay zero); with sQs,
-// also e^gam times the rounded q^ there (eg by scan row; memory row r is scan
-// row 63 - r when rev).  No barrier.
+// [Dk/8][64][8] tiles (rows of zeros stay zero); with sQs, also e^gam times
+// the rounded q^ there (eg by scan row; memory row r is scan row 63 - r when
+// rev).  Warp w takes rows 8 (w % 8) .. + 7 of q and k (with 16 warps, of
+// q for w < 8 and of k for the rest); lane l reads the 4-byte word l % 4 of
+// row l / 4 in every 8-column slab, so a warp's read of a slab is 128
+// contiguous bytes (a row's slabs are 1 KB apart: lanes spread along a row
+// would all hit the same four banks).  8 or 16 warps.  No barrier.
 __device__ void normalize_rows_core(const BcArgs& a, __nv_bfloat16* sQ, __nv_bfloat16* sK,
                                     __nv_bfloat16* sQs = nullptr, const float* eg = nullptr,
                                     bool rev = false) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  const int Dk = a.Dk;
-  uint32_t* q2 = reinterpret_cast<uint32_t*>(sQ);
-  uint32_t* k2 = reinterpret_cast<uint32_t*>(sK);
-  for (int r = warp; r < 64; r += nw) {
-    float qv[2][2] = {}, kv[2][2] = {};
-    float qq = 0.f, kk = 0.f;
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int d2 = lane + 32 * i, at = cidx(r, 2 * d2, 64, false) / 2;
-      if (d2 < Dk / 2) {
-        unpack_bf16x2(q2[at], qv[i][0], qv[i][1]);
-        unpack_bf16x2(k2[at], kv[i][0], kv[i][1]);
-        qq = fmaf(qv[i][0], qv[i][0], fmaf(qv[i][1], qv[i][1], qq));
-        kk = fmaf(kv[i][0], kv[i][0], fmaf(kv[i][1], kv[i][1], kk));
-      }
+  const int ns = a.Dk / 8;
+  const int r = 8 * (warp & 7) + (lane >> 2);
+  const int at0 = r * 4 + (lane & 3);  // word index in slab 0; + 256 words a slab
+  const int t0 = nw >= 16 ? (warp >> 3) : 0, tstep = nw >= 16 ? 2 : 1;
+  for (int ts = t0; ts < 2; ts += tstep) {
+    const bool is_q = ts == 0;
+    uint32_t* x2 = reinterpret_cast<uint32_t*>(is_q ? sQ : sK);
+    float ss = 0.f;
+    for (int sl = 0; sl < ns; ++sl) {
+      float x0, x1;
+      unpack_bf16x2(x2[at0 + 256 * sl], x0, x1);
+      ss = fmaf(x0, x0, fmaf(x1, x1, ss));
     }
-#pragma unroll
-    for (int off = 16; off; off >>= 1) {
-      qq += __shfl_xor_sync(0xffffffffu, qq, off);
-      kk += __shfl_xor_sync(0xffffffffu, kk, off);
-    }
-    const float rq = 1.f / sqrtf(fmaxf(qq, 1e-12f)), rk = 1.f / sqrtf(fmaxf(kk, 1e-12f));
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int d2 = lane + 32 * i, at = cidx(r, 2 * d2, 64, false) / 2;
-      if (d2 < Dk / 2) {
-        const uint32_t qn = pack_bf16x2(qv[i][0] * rq, qv[i][1] * rq);
-        q2[at] = qn;
-        k2[at] = pack_bf16x2(kv[i][0] * rk, kv[i][1] * rk);
-        if (sQs) {
-          const float e = eg[rev ? 63 - r : r];
-          float x0, x1;
-          unpack_bf16x2(qn, x0, x1);
-          reinterpret_cast<uint32_t*>(sQs)[at] = pack_bf16x2(x0 * e, x1 * e);
-        }
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+    const float rn = 1.f / sqrtf(fmaxf(ss, 1e-12f));
+    const float e = (sQs && is_q) ? eg[rev ? 63 - r : r] : 0.f;
+    for (int sl = 0; sl < ns; ++sl) {
+      float x0, x1;
+      unpack_bf16x2(x2[at0 + 256 * sl], x0, x1);
+      const uint32_t xn = pack_bf16x2(x0 * rn, x1 * rn);
+      x2[at0 + 256 * sl] = xn;
+      if (sQs && is_q) {  // e^gam times the rounded q^
+        unpack_bf16x2(xn, x0, x1);
+        reinterpret_cast<uint32_t*>(sQs)[at0 + 256 * sl] = pack_bf16x2(x0 * e, x1 * e);
       }
     }
   }
@@ -1061,16 +1055,16 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   acc_row_sums(Dk, wg, [&](int, int, int, int m, int n) {
     return sm.beta[m] * sm.eg[m] * bf(sKc[cidx(m, n, 64, rev)]) * bf(sXw[cidx(m, n, 64, false)]);
   });
-  for (int p = warp; p < 64; p += kGrWarps) {  // dX_u rows: four columns (8 bytes) a lane
-    const int r = sm.row[p];
-    if (r < 0) continue;
-    for (int c4 = lane; c4 < Dv / 4; c4 += 32) {
-      const uint2 x = *reinterpret_cast<const uint2*>(sXu + cidx(p, 4 * c4, 64, false));
-      float f0, f1, f2, f3;
-      unpack_bf16x2(x.x, f0, f1);
-      unpack_bf16x2(x.y, f2, f3);
-      *reinterpret_cast<float4*>(dvb + (size_t)r * Dv + 4 * c4) = make_float4(f0, f1, f2, f3);
-    }
+  {  // dX_u rows: warp w takes rows 8 (w % 8) .. + 7 and every other slab
+     // from w / 8; lane l the word l % 4 of row l / 4 (128 contiguous bytes a slab)
+    const int p = 8 * (warp & 7) + (lane >> 2), r = sm.row[p];
+    const uint32_t* x2 = reinterpret_cast<const uint32_t*>(sXu);
+    if (r >= 0)
+      for (int sl = warp >> 3; sl < Dv / 8; sl += 2) {
+        float f0, f1;
+        unpack_bf16x2(x2[(sl * 64 + p) * 4 + (lane & 3)], f0, f1);
+        *reinterpret_cast<float2*>(dvb + (size_t)r * Dv + 8 * sl + 2 * (lane & 3)) = make_float2(f0, f1);
+      }
   }
   // ---- 12. dA = -(dX_w W^T + dX_u U~^T) on i < p (into P); gam from A
   gemm2<false, true, false, true>(64, 64, Xw, Wm, Dk, Xu, Ut, Dv,
