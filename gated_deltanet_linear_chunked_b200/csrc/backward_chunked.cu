@@ -168,6 +168,40 @@ __device__ __forceinline__ void blk16(int m0, int n0, int K, const BMat& A, cons
 #pragma unroll
     for (int i = 0; i < 4; ++i) d[h][i] += e[h][i];
 }
+// Two 16 x 16 output blocks (m0[x], n0[x]) += A B over k < K, their k-steps
+// interleaved: two independent chains per block, four in flight.
+template <bool TA, bool TB>
+__device__ __forceinline__ void blk16x2(const int (&m0)[2], const int (&n0)[2], int K, const BMat& A,
+                                        const BMat& B, float (&d0)[2][4], float (&d1)[2][4]) {
+  const int l = threadIdx.x & 31;
+  uint32_t pa[2], pb[2];
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    pa[x] = TA ? bm_at(A, (l & 7) + 8 * (l >> 4), (m0[x] >> 3) + ((l >> 3) & 1))
+               : bm_at(A, m0[x] + (l & 15), l >> 4);
+    pb[x] = TB ? bm_at(B, n0[x] + (l & 7) + 8 * (l >> 4), (l >> 3) & 1)
+               : bm_at(B, (l & 7) + 8 * ((l >> 3) & 1), (n0[x] >> 3) + (l >> 4));
+  }
+  const int da = TA ? (A.rrev ? -16 * A.rs : 16 * A.rs) : 2 * A.slab;
+  const int db = TB ? 2 * B.slab : (B.rrev ? -16 * B.rs : 16 * B.rs);
+#pragma unroll 1
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    uint32_t a[2][4], bb[2][4];
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      if (TA) ldmatrix_x4_trans(pa[x], a[x]);
+      else ldmatrix_x4(pa[x], a[x]);
+      if (TB) ldmatrix_x4(pb[x], bb[x]);
+      else ldmatrix_x4_trans(pb[x], bb[x]);
+      pa[x] += da;
+      pb[x] += db;
+    }
+    mma_16816(d0[0], a[0], bb[0][0], bb[0][1]);
+    mma_16816(d0[1], a[0], bb[0][2], bb[0][3]);
+    mma_16816(d1[0], a[1], bb[1][0], bb[1][1]);
+    mma_16816(d1[1], a[1], bb[1][2], bb[1][3]);
+  }
+}
 __device__ __forceinline__ void zero2(float (&d)[2][4]) {
 #pragma unroll
   for (int h = 0; h < 2; ++h) d[h][0] = d[h][1] = d[h][2] = d[h][3] = 0.f;
@@ -184,12 +218,7 @@ __device__ __forceinline__ void gemm2(int M, int N, const BMat& A1, const BMat& 
                                       FC contrib, FE epi, float* rsum, float* csum) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   const int tn = N >> 4, nt = (M >> 4) * tn;
-  for (int t = warp; t < nt; t += nw) {
-    const int m0 = (t / tn) << 4, nb = (t % tn) << 4;
-    float dd[2][4];
-    zero2(dd);
-    blk16<TA1, TB1>(m0, nb, K1, A1, B1, dd);
-    if (K2) blk16<TA2, TB2>(m0, nb, K2, A2, B2, dd);
+  auto finish = [&](int m0, int nb, float (&dd)[2][4]) {
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       const int n0 = nb + 8 * hh;
@@ -222,6 +251,25 @@ __device__ __forceinline__ void gemm2(int M, int N, const BMat& A1, const BMat& 
           csum[n0 + tile_col(1)] -= c1;
         }
       }
+    }
+  };
+  for (int t = warp; t < nt; t += 2 * nw) {
+    const int m0[2] = {(t / tn) << 4, ((t + nw) / tn) << 4};
+    const int nb[2] = {(t % tn) << 4, ((t + nw) % tn) << 4};
+    if (t + nw < nt) {  // two blocks, interleaved
+      float d0[2][4], d1[2][4];
+      zero2(d0);
+      zero2(d1);
+      blk16x2<TA1, TB1>(m0, nb, K1, A1, B1, d0, d1);
+      if (K2) blk16x2<TA2, TB2>(m0, nb, K2, A2, B2, d0, d1);
+      finish(m0[0], nb[0], d0);
+      finish(m0[1], nb[1], d1);
+    } else {
+      float dd[2][4];
+      zero2(dd);
+      blk16<TA1, TB1>(m0[0], nb[0], K1, A1, B1, dd);
+      if (K2) blk16<TA2, TB2>(m0[0], nb[0], K2, A2, B2, dd);
+      finish(m0[0], nb[0], dd);
     }
   }
 }
@@ -764,22 +812,23 @@ struct GradLayout {
 template <bool TA, bool TB, class FS>
 __device__ __forceinline__ void gemm_acc2(int N, int K, const BMat& A, const BMat& B, float (&acc)[kMaxBlocks][2][4],
                                           FS scale) {
+  static_assert(kMaxBlocks == 2, "two register blocks per warp");
   const int warp = threadIdx.x >> 5;
   const int tn = N >> 4, nt = 4 * tn;
+  const int t1 = warp + kGrWarps;
+  const int m0[2] = {(warp / tn) << 4, (t1 / tn) << 4}, n0[2] = {(warp % tn) << 4, (t1 % tn) << 4};
+  float d[2][2][4];
+  zero2(d[0]);
+  zero2(d[1]);
+  if (t1 < nt) blk16x2<TA, TB>(m0, n0, K, A, B, d[0], d[1]);
+  else if (warp < nt) blk16<TA, TB>(m0[0], n0[0], K, A, B, d[0]);
 #pragma unroll
-  for (int i = 0; i < kMaxBlocks; ++i) {
-    const int t = warp + kGrWarps * i;
-    if (t < nt) {
-      const int m0 = (t / tn) << 4, n0 = (t % tn) << 4;
-      float d[2][4];
-      zero2(d);
-      blk16<TA, TB>(m0, n0, K, A, B, d);
+  for (int i = 0; i < 2; ++i)
+    if (warp + kGrWarps * i < nt)
 #pragma unroll
       for (int h = 0; h < 2; ++h)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[i][h][e] += scale(m0 + tile_row(e)) * d[h][e];
-    }
-  }
+        for (int e = 0; e < 4; ++e) acc[i][h][e] += scale(m0[i] + tile_row(e)) * d[i][h][e];
 }
 // The register blocks' elements: f(i, h, e, m, n) for every one this thread holds.
 template <class F>
