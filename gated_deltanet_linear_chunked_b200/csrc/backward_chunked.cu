@@ -168,38 +168,54 @@ __device__ __forceinline__ void blk16(int m0, int n0, int K, const BMat& A, cons
 #pragma unroll
     for (int i = 0; i < 4; ++i) d[h][i] += e[h][i];
 }
-// Two 16 x 16 output blocks (m0[x], n0[x]) += A B over k < K, their k-steps
-// interleaved: two independent chains per block, four in flight.
-template <bool TA, bool TB>
-__device__ __forceinline__ void blk16x2(const int (&m0)[2], const int (&n0)[2], int K, const BMat& A,
-                                        const BMat& B, float (&d0)[2][4], float (&d1)[2][4]) {
+// Two 16 x 16 output blocks, d0 = block (m0[0], n0[0]) of A0 B0 over k < K0
+// and d1 = block (m0[1], n0[1]) of A1 B1 over k < K1 (added to d0, d1), their
+// k-steps interleaved: independent chains hide each other's latency.
+template <bool TA0, bool TB0, bool TA1, bool TB1>
+__device__ __forceinline__ void blk16x2(const int (&m0)[2], const int (&n0)[2], const BMat& A0,
+                                        const BMat& B0, int K0, const BMat& A1, const BMat& B1, int K1,
+                                        float (&d0)[2][4], float (&d1)[2][4]) {
   const int l = threadIdx.x & 31;
-  uint32_t pa[2], pb[2];
-#pragma unroll
-  for (int x = 0; x < 2; ++x) {
-    pa[x] = TA ? bm_at(A, (l & 7) + 8 * (l >> 4), (m0[x] >> 3) + ((l >> 3) & 1))
-               : bm_at(A, m0[x] + (l & 15), l >> 4);
-    pb[x] = TB ? bm_at(B, n0[x] + (l & 7) + 8 * (l >> 4), (l >> 3) & 1)
-               : bm_at(B, (l & 7) + 8 * ((l >> 3) & 1), (n0[x] >> 3) + (l >> 4));
-  }
-  const int da = TA ? (A.rrev ? -16 * A.rs : 16 * A.rs) : 2 * A.slab;
-  const int db = TB ? 2 * B.slab : (B.rrev ? -16 * B.rs : 16 * B.rs);
+  auto a_at = [&](bool ta, const BMat& A, int m) {
+    return ta ? bm_at(A, (l & 7) + 8 * (l >> 4), (m >> 3) + ((l >> 3) & 1)) : bm_at(A, m + (l & 15), l >> 4);
+  };
+  auto b_at = [&](bool tb, const BMat& B, int n) {
+    return tb ? bm_at(B, n + (l & 7) + 8 * (l >> 4), (l >> 3) & 1)
+              : bm_at(B, (l & 7) + 8 * ((l >> 3) & 1), (n >> 3) + (l >> 4));
+  };
+  auto a_step = [](bool ta, const BMat& A) { return ta ? (A.rrev ? -16 * A.rs : 16 * A.rs) : 2 * A.slab; };
+  auto b_step = [](bool tb, const BMat& B) { return tb ? 2 * B.slab : (B.rrev ? -16 * B.rs : 16 * B.rs); };
+  uint32_t pa0 = a_at(TA0, A0, m0[0]), pb0 = b_at(TB0, B0, n0[0]);
+  uint32_t pa1 = a_at(TA1, A1, m0[1]), pb1 = b_at(TB1, B1, n0[1]);
+  const int da0 = a_step(TA0, A0), db0 = b_step(TB0, B0), da1 = a_step(TA1, A1), db1 = b_step(TB1, B1);
+  const int K = K0 > K1 ? K0 : K1;
 #pragma unroll 1
   for (int k0 = 0; k0 < K; k0 += 16) {
     uint32_t a[2][4], bb[2][4];
-#pragma unroll
-    for (int x = 0; x < 2; ++x) {
-      if (TA) ldmatrix_x4_trans(pa[x], a[x]);
-      else ldmatrix_x4(pa[x], a[x]);
-      if (TB) ldmatrix_x4(pb[x], bb[x]);
-      else ldmatrix_x4_trans(pb[x], bb[x]);
-      pa[x] += da;
-      pb[x] += db;
+    if (k0 < K0) {
+      if (TA0) ldmatrix_x4_trans(pa0, a[0]);
+      else ldmatrix_x4(pa0, a[0]);
+      if (TB0) ldmatrix_x4(pb0, bb[0]);
+      else ldmatrix_x4_trans(pb0, bb[0]);
+      pa0 += da0;
+      pb0 += db0;
     }
-    mma_16816(d0[0], a[0], bb[0][0], bb[0][1]);
-    mma_16816(d0[1], a[0], bb[0][2], bb[0][3]);
-    mma_16816(d1[0], a[1], bb[1][0], bb[1][1]);
-    mma_16816(d1[1], a[1], bb[1][2], bb[1][3]);
+    if (k0 < K1) {
+      if (TA1) ldmatrix_x4_trans(pa1, a[1]);
+      else ldmatrix_x4(pa1, a[1]);
+      if (TB1) ldmatrix_x4(pb1, bb[1]);
+      else ldmatrix_x4_trans(pb1, bb[1]);
+      pa1 += da1;
+      pb1 += db1;
+    }
+    if (k0 < K0) {
+      mma_16816(d0[0], a[0], bb[0][0], bb[0][1]);
+      mma_16816(d0[1], a[0], bb[0][2], bb[0][3]);
+    }
+    if (k0 < K1) {
+      mma_16816(d1[0], a[1], bb[1][0], bb[1][1]);
+      mma_16816(d1[1], a[1], bb[1][2], bb[1][3]);
+    }
   }
 }
 __device__ __forceinline__ void zero2(float (&d)[2][4]) {
@@ -260,15 +276,25 @@ __device__ __forceinline__ void gemm2(int M, int N, const BMat& A1, const BMat& 
       float d0[2][4], d1[2][4];
       zero2(d0);
       zero2(d1);
-      blk16x2<TA1, TB1>(m0, nb, K1, A1, B1, d0, d1);
-      if (K2) blk16x2<TA2, TB2>(m0, nb, K2, A2, B2, d0, d1);
+      blk16x2<TA1, TB1, TA1, TB1>(m0, nb, A1, B1, K1, A1, B1, K1, d0, d1);
+      if (K2) blk16x2<TA2, TB2, TA2, TB2>(m0, nb, A2, B2, K2, A2, B2, K2, d0, d1);
       finish(m0[0], nb[0], d0);
       finish(m0[1], nb[1], d1);
     } else {
       float dd[2][4];
       zero2(dd);
-      blk16<TA1, TB1>(m0[0], nb[0], K1, A1, B1, dd);
-      if (K2) blk16<TA2, TB2>(m0[0], nb[0], K2, A2, B2, dd);
+      if (K2) {  // the two operand pairs of the one block as two chains
+        float d2[2][4];
+        zero2(d2);
+        const int mm[2] = {m0[0], m0[0]}, nn[2] = {nb[0], nb[0]};
+        blk16x2<TA1, TB1, TA2, TB2>(mm, nn, A1, B1, K1, A2, B2, K2, dd, d2);
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dd[h][e] += d2[h][e];
+      } else {
+        blk16<TA1, TB1>(m0[0], nb[0], K1, A1, B1, dd);
+      }
       finish(m0[0], nb[0], dd);
     }
   }
@@ -820,7 +846,7 @@ __device__ __forceinline__ void gemm_acc2(int N, int K, const BMat& A, const BMa
   float d[2][2][4];
   zero2(d[0]);
   zero2(d[1]);
-  if (t1 < nt) blk16x2<TA, TB>(m0, n0, K, A, B, d[0], d[1]);
+  if (t1 < nt) blk16x2<TA, TB, TA, TB>(m0, n0, A, B, K, A, B, K, d[0], d[1]);
   else if (warp < nt) blk16<TA, TB>(m0[0], n0[0], K, A, B, d[0]);
 #pragma unroll
   for (int i = 0; i < 2; ++i)
@@ -1039,12 +1065,22 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   auto none = [](int, int, float) { return 0.f; };
 
   // ---- 1. P = M o (Q^ K^T);  E = e^{gam_p - gam_i} K^ K^T (i < p), A = diag(beta) E
-  gemm2<false, true, false, true>(64, 64, Q, K, Dk, Q, K, 0, none, [&](int m, int n, float v) {
-    sP[m * kLdE + n] = __float2bfloat16_rn(n <= m ? expf(sm.gam[m] - sm.gam[n]) * v : 0.f);
-  }, nullptr, nullptr);
-  gemm2<false, true, false, true>(64, 64, K, K, Dk, K, K, 0, none, [&](int m, int n, float v) {
-    sE[m * kLdE + n] = __float2bfloat16_rn(n < m ? expf(sm.gam[m] - sm.gam[n]) * v : 0.f);
-  }, nullptr, nullptr);
+  {  // block `warp` of P and of E, interleaved (16 blocks each, one a warp)
+    const int mm[2] = {(warp >> 2) << 4, (warp >> 2) << 4}, nn[2] = {(warp & 3) << 4, (warp & 3) << 4};
+    float dp[2][4], de[2][4];
+    zero2(dp);
+    zero2(de);
+    blk16x2<false, true, false, true>(mm, nn, Q, K, Dk, K, K, Dk, dp, de);
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int m = mm[0] + tile_row(e), n = nn[0] + 8 * hh + tile_col(e);
+        const float decay = n <= m ? expf(sm.gam[m] - sm.gam[n]) : 0.f;
+        sP[m * kLdE + n] = __float2bfloat16_rn(decay * dp[hh][e]);
+        sE[m * kLdE + n] = __float2bfloat16_rn(n < m ? decay * de[hh][e] : 0.f);
+      }
+  }
   __syncthreads();  // P and E complete
   // ---- 3. dK~ = U dS_e^T: dk^ starts as e^{gam_C - gam} dK~; c_m = k^_m . dk^_m
   float dk[kMaxBlocks][2][4], dq[kMaxBlocks][2][4];
