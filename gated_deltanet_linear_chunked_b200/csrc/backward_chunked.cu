@@ -602,6 +602,15 @@ __global__ void __launch_bounds__(kChThreads, 2) gdn_bwd_chain_kernel(BcArgs a) 
   int st = 0;
   uint32_t ph = 0;
   bool ok = true;
+  // <dS_e, S0> of the previous chunk: this lane's part, reduced over the warp
+  // and added to its block's sum one step later, off the chain's critical path
+  float dot_pend = 0.f;
+  size_t blk_pend = 0;
+  auto flush_dot = [&]() {
+#pragma unroll
+    for (int off = 16; off; off >>= 1) dot_pend += __shfl_xor_sync(0xffffffffu, dot_pend, off);
+    if (lane == 0) atomicAdd(a.dot + blk_pend, dot_pend);
+  };
   for (int s = 0; s < a.nC; ++s) {
     const size_t blk = a.blk(dir, bh, dir == 0 ? a.nC - 1 - s : s);
     // dS_e^T (the state entering this chunk) to the slice's warps, in
@@ -683,6 +692,7 @@ __global__ void __launch_bounds__(kChThreads, 2) gdn_bwd_chain_kernel(BcArgs a) 
         mma_16816(acc[0], af[kb], bk[kb][0], bk[kb][1]);
         mma_16816(acc[1], af[kb], bk[kb][2], bk[kb][3]);
       }
+      if (s > 0) flush_dot();  // while the MMAs above run
 #pragma unroll
       for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -731,7 +741,7 @@ __global__ void __launch_bounds__(kChThreads, 2) gdn_bwd_chain_kernel(BcArgs a) 
         }
       }
     }
-    {  // this warp's share of <dS_e, S0> (bf16 operands, as the gradient pass's
+    {  // this lane's part of <dS_e, S0> (bf16 operands, as the gradient pass's
        // products use them), while the MMAs above run: fse[i][2 h + rr] holds
        // columns gq + 8 rr, rows d, d + 1 (d = 16 kb + 8 h + 2 tq); the staged
        // slice of S0 is [2][Dk][8] (rows d)
@@ -753,9 +763,8 @@ __global__ void __launch_bounds__(kChThreads, 2) gdn_bwd_chain_kernel(BcArgs a) 
             }
         }
       }
-#pragma unroll
-      for (int off = 16; off; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-      if (lane == 0) atomicAdd(a.dot + blk, dot);
+      dot_pend = dot;
+      blk_pend = blk;
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars.empty[st]);  // this warp's reads of the stage are done
@@ -768,6 +777,7 @@ __global__ void __launch_bounds__(kChThreads, 2) gdn_bwd_chain_kernel(BcArgs a) 
     if (lane == 0) atomicOr(a.err, kErrTimeout);
     return;
   }
+  flush_dot();  // the last chunk's
   if (dir == 0 && a.d_state_in) {
 #pragma unroll
     for (int i = 0; i < KPW; ++i)
