@@ -310,14 +310,24 @@ __device__ __forceinline__ void gemm_store_frag(int M, int N, const BMat& A, con
                                                 __nv_bfloat16* dst) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   const int tn = N >> 4, nt = (M >> 4) * tn;
-  for (int t = warp; t < nt; t += nw) {
-    const int m0 = (t / tn) << 4, nb = (t % tn) << 4;
-    float dd[2][4];
-    zero2(dd);
-    blk16<TA, TB>(m0, nb, K, A, B, dd);
+  auto put = [&](int t, const float (&dd)[2][4]) {
     *reinterpret_cast<uint4*>(dst + ((size_t)t * 32 + lane) * 8) =
         make_uint4(pack_bf16x2(dd[0][0], dd[0][1]), pack_bf16x2(dd[0][2], dd[0][3]),
                    pack_bf16x2(dd[1][0], dd[1][1]), pack_bf16x2(dd[1][2], dd[1][3]));
+  };
+  for (int t = warp; t < nt; t += 2 * nw) {
+    const int m0[2] = {(t / tn) << 4, ((t + nw) / tn) << 4}, nb[2] = {(t % tn) << 4, ((t + nw) % tn) << 4};
+    float d0[2][4], d1[2][4];
+    zero2(d0);
+    zero2(d1);
+    if (t + nw < nt) {  // two blocks, interleaved
+      blk16x2<TA, TB, TA, TB>(m0, nb, A, B, K, A, B, K, d0, d1);
+      put(t, d0);
+      put(t + nw, d1);
+    } else {
+      blk16<TA, TB>(m0[0], nb[0], K, A, B, d0);
+      put(t, d0);
+    }
   }
 }
 
