@@ -47,7 +47,7 @@ def max_rel_per_head(x, ref, head_axes) -> float:
 def max_rel_rows(x, ref, rows) -> float:
     """Largest error over the given token rows of an output [B,T,H,D],
     relative to each (b, h, row)'s own largest reference value: rows whose
-    reference is tiny or huge are judged on their own scale."""
+    reference is tiny or huge are measured on their own scale."""
     x = np.asarray(x, np.float64)[:, rows]
     ref = np.asarray(ref, np.float64)[:, rows]
     den = np.max(np.abs(ref), axis=-1)
