@@ -111,3 +111,14 @@ def test_backward_stream_chunk_full_size(mode):
     """The 2640-token x 20-head x d112 streaming chunk, bf16 I/O; heads 0
     and 19 compared with the oracle (heads are independent)."""
     run_and_check(wl.stream_chunk(mode), seed=1, heads=[0, 19])
+
+
+@pytest.mark.parametrize("Dk,Dv", [(48, 80), (96, 32)])
+def test_backward_many_chunks_rectangular(Dk, Dv):
+    """Enough chunk tiles (2 x 24 chunks x 6 heads x 2 directions = 576) that
+    each CTA of the persistent gradient pass walks several and prefetches the
+    next; Dk or Dv below 64 gives the dX tiles buffers of their own.  Heads
+    0 and 5 of both batch rows compared with the oracle."""
+    w = wl.Workload(f"bwd_many_{Dk}_{Dv}", 2, 1500, 6, Dk, Dv, "bf16", 64, "bidir", ("uniform", -0.5, 0.0),
+                    ("sigmoid",), ("normal", 0.3), 93000 + Dk + Dv)
+    run_and_check(w, seed=4, heads=[0, 5])
