@@ -398,23 +398,62 @@ gdn_bwd_reduce_kernel(BwdArgs A, int ndir, void* dq_, void* dk_, void* dv_, floa
   IO* dq = static_cast<IO*>(dq_);
   IO* dk = static_cast<IO*>(dk_);
   IO* dv = static_cast<IO*>(dv_);
+  // Every load of the row first (two directions at most; with one slice per
+  // direction -- the chunked path -- nothing waits on another load), then the
+  // arithmetic and the stores.
   float gq[4] = {0.f, 0.f, 0.f, 0.f}, gk[4] = {0.f, 0.f, 0.f, 0.f};
-  float qi[4] = {0.f, 0.f, 0.f, 0.f}, ki[4] = {0.f, 0.f, 0.f, 0.f};
+  float qi[4] = {0.f, 0.f, 0.f, 0.f}, ki[4] = {0.f, 0.f, 0.f, 0.f}, vi[4] = {0.f, 0.f, 0.f, 0.f};
+  float pqv[2][4] = {}, pkv[2][4] = {}, dvv[2][4] = {};
+  const bool one_slice = A.nslice == 1;
   if (c < Dk) {
-    for (int d = 0; d < ndir; ++d)
-      for (int s = 0; s < A.nslice; ++s) {
-        const size_t base = ((size_t)d * A.nslice + s) * rows_bth + row;
-        float x[4], y[4];
-        ld4_io(A.pq + base * Dk + c, x);
-        ld4_io(A.pk + base * Dk + c, y);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          gq[e] += x[e];
-          gk[e] += y[e];
-        }
-      }
     ld4_io(q + row * Dk + c, qi);
     ld4_io(k + row * Dk + c, ki);
+    if (one_slice) {
+#pragma unroll
+      for (int d = 0; d < 2; ++d)
+        if (d < ndir) {
+          const size_t base = (size_t)d * rows_bth + row;
+          ld4_io(A.pq + base * Dk + c, pqv[d]);
+          ld4_io(A.pk + base * Dk + c, pkv[d]);
+        }
+    }
+  }
+  if (c < Dv) {
+#pragma unroll
+    for (int d = 0; d < 2; ++d)
+      if (d < ndir) ld4_io(A.dvb + ((size_t)d * rows_bth + row) * Dv + c, dvv[d]);
+    if (chunked) ld4_io(static_cast<const IO*>(A.v) + row * Dv + c, vi);
+  }
+  const float bt = chunked ? __ldg(A.beta + row) : 0.f;
+  float2 pab2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // (da, dbeta) per direction
+  if (one_slice && lane == 0) {
+#pragma unroll
+    for (int d = 0; d < 2; ++d)
+      if (d < ndir) pab2[d] = *reinterpret_cast<const float2*>(A.pab + ((size_t)d * rows_bth + row) * 2);
+  }
+  if (c < Dk) {
+    if (one_slice) {
+#pragma unroll
+      for (int d = 0; d < 2; ++d)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          gq[e] += pqv[d][e];
+          gk[e] += pkv[d][e];
+        }
+    } else {
+      for (int d = 0; d < ndir; ++d)
+        for (int s = 0; s < A.nslice; ++s) {
+          const size_t base = ((size_t)d * A.nslice + s) * rows_bth + row;
+          float x[4], y[4];
+          ld4_io(A.pq + base * Dk + c, x);
+          ld4_io(A.pk + base * Dk + c, y);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            gq[e] += x[e];
+            gk[e] += y[e];
+          }
+        }
+    }
   }
   // |q|^2, |k|^2, q . dq^, k . dk^ over the row
   float t4[4] = {0.f, 0.f, 0.f, 0.f};
@@ -444,17 +483,10 @@ gdn_bwd_reduce_kernel(BwdArgs A, int ndir, void* dq_, void* dk_, void* dv_, floa
   }
   float vdx = 0.f;  // v . dX_u (chunked path)
   if (c < Dv) {
-    float sv[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int d = 0; d < ndir; ++d) {
-      float x[4];
-      ld4_io(A.dvb + ((size_t)d * rows_bth + row) * Dv + c, x);
+    float sv[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sv[e] += x[e];
-    }
+    for (int e = 0; e < 4; ++e) sv[e] = dvv[0][e] + dvv[1][e];
     if (chunked) {
-      float vi[4];
-      ld4_io(static_cast<const IO*>(A.v) + row * Dv + c, vi);
-      const float bt = __ldg(A.beta + row);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         vdx = fmaf(vi[e], sv[e], vdx);
@@ -467,13 +499,14 @@ gdn_bwd_reduce_kernel(BwdArgs A, int ndir, void* dq_, void* dk_, void* dv_, floa
 #pragma unroll
     for (int off = 16; off; off >>= 1) vdx += __shfl_xor_sync(0xffffffffu, vdx, off);
   if (lane == 0) {
-    float da = 0.f, db = 0.f;
-    for (int d = 0; d < ndir; ++d)
-      for (int s = 0; s < A.nslice; ++s) {
-        const size_t base = ((size_t)d * A.nslice + s) * rows_bth;
-        da += A.pab[(base + row) * 2];
-        db += A.pab[(base + row) * 2 + 1];
-      }
+    float da = pab2[0].x + pab2[1].x, db = pab2[0].y + pab2[1].y;
+    if (!one_slice)
+      for (int d = 0; d < ndir; ++d)
+        for (int s = 0; s < A.nslice; ++s) {
+          const size_t base = ((size_t)d * A.nslice + s) * rows_bth;
+          da += A.pab[(base + row) * 2];
+          db += A.pab[(base + row) * 2 + 1];
+        }
     dg[row] = chunked ? da : expf(__ldg(A.g + row)) * da;
     dbeta[row] = db + vdx;
   }
