@@ -156,9 +156,13 @@ GDN_API gdn_status gdn_chunk_bidir_logits(const void* q, const void* k, const vo
  *   dq, dk [B, T, H, Dk] and dv [B, T, H, Dv] in dtype; dg, dbeta [B, T, H]
  *   fp32; d_state_in [B, H, Dk, Dv] fp32 (may be NULL; zero-state calls pass
  *   state_in = NULL and get the gradient of a zero start state).
- * The recurrence is walked in fp32 on CUDA cores (token-serial, like the fp32
- * forward path), with checkpoints every 64 tokens; scratch comes from the
- * stream's context.  g and beta are taken as given (no gate-logit form).
+ * bf16 I/O with Dk, Dv <= 112 runs the chunked reverse mode on tensor cores
+ * (the forward's stages A and B, then a pre pass, the reverse walk over the
+ * chunks and a chunk-parallel gradient pass; bf16 operands, fp32
+ * accumulation, within 2e-2 of the definition); fp32 I/O and wider heads
+ * walk the recurrence in fp32 on CUDA cores (token-serial, with checkpoints
+ * every 64 tokens, within 1e-4).  Scratch comes from the stream's context.
+ * g and beta are taken as given (no gate-logit form).
  * The gradient outputs may not overlap each other or any input.  Errors as
  * for gdn_chunk_fwd.
  */
