@@ -1171,25 +1171,58 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         *reinterpret_cast<float2*>(dvb + (size_t)r * Dv + 8 * sl + 2 * (lane & 3)) = make_float2(f0, f1);
       }
   }
-  // ---- 12. dA = -(dX_w W^T + dX_u U~^T) on i < p (into P); gam from A
-  gemm2<false, true, false, true>(64, 64, Xw, Wm, Dk, Xu, Ut, Dv,
-      [&](int m, int n, float v) { return n < m ? -v * sm.beta[m] * bf(sE[m * kLdE + n]) : 0.f; },
-      [&](int m, int n, float v) { sP[m * kLdE + n] = __float2bfloat16_rn(n < m ? -v : 0.f); },
-      wg, wg);
-  __syncthreads();  // dX_w, dX_u (in the dS_e^T and S0 tiles), W and U~ are read no more
-  if (more && tid == 0) issue(3, nxt);
-  for (int p = warp; p < 64; p += kGrWarps) {  // dbeta_p += sum_i dA_pi E_pi; dG = dA beta_p e^{..}
-    float sb = 0.f;
-    for (int i = lane; i < p; i += 32) {
-      const float dA = bf(sP[p * kLdE + i]);
-      sb = fmaf(dA, bf(sE[p * kLdE + i]), sb);
-      sP[p * kLdE + i] = __float2bfloat16_rn(dA * sm.beta[p] * expf(sm.gam[p] - sm.gam[i]));
-    }
+  // ---- 12. dA = -(dX_w W^T + dX_u U~^T) on i < p (warp w: block w of the
+  //          64 x 64, its two operand pairs as two chains), and from it in
+  //          the same pass: gam's share from A (dA o A: + to row p, - to
+  //          column i), beta_p += sum_i dA_pi E_pi, and dG = dA o (beta_p
+  //          e^{gam_p - gam_i}) into P
+  {
+    const int mm[2] = {(warp >> 2) << 4, (warp >> 2) << 4}, nn[2] = {(warp & 3) << 4, (warp & 3) << 4};
+    float d1[2][4], d2[2][4];
+    zero2(d1);
+    zero2(d2);
+    blk16x2<false, true, false, true>(mm, nn, Xw, Wm, Dk, Xu, Ut, Dv, d1, d2);
 #pragma unroll
-    for (int off = 16; off; off >>= 1) sb += __shfl_xor_sync(0xffffffffu, sb, off);
-    if (lane == 0) wb[p] += sb;
+    for (int hh = 0; hh < 2; ++hh) {
+      const int n0 = nn[0] + 8 * hh;
+      float cg[4], cb[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int m = mm[0] + tile_row(e), n = n0 + tile_col(e);
+        const float dA = n < m ? -(d1[hh][e] + d2[hh][e]) : 0.f;
+        const float E = bf(sE[m * kLdE + n]);  // zero on and above the diagonal
+        cg[e] = dA * sm.beta[m] * E;
+        cb[e] = dA * E;
+        sP[m * kLdE + n] = __float2bfloat16_rn(n < m ? dA * sm.beta[m] * expf(sm.gam[m] - sm.gam[n]) : 0.f);
+      }
+      float rg0 = cg[0] + cg[1], rg1 = cg[2] + cg[3], rb0 = cb[0] + cb[1], rb1 = cb[2] + cb[3];
+#pragma unroll
+      for (int off = 1; off < 4; off <<= 1) {
+        rg0 += __shfl_xor_sync(0xffffffffu, rg0, off);
+        rg1 += __shfl_xor_sync(0xffffffffu, rg1, off);
+        rb0 += __shfl_xor_sync(0xffffffffu, rb0, off);
+        rb1 += __shfl_xor_sync(0xffffffffu, rb1, off);
+      }
+      float c0 = cg[0] + cg[2], c1 = cg[1] + cg[3];
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        c0 += __shfl_xor_sync(0xffffffffu, c0, off);
+        c1 += __shfl_xor_sync(0xffffffffu, c1, off);
+      }
+      if ((lane & 3) == 0) {  // this warp's partial rows
+        wg[mm[0] + tile_row(0)] += rg0;
+        wg[mm[0] + tile_row(2)] += rg1;
+        wb[mm[0] + tile_row(0)] += rb0;
+        wb[mm[0] + tile_row(2)] += rb1;
+      }
+      if (lane < 4) {
+        wg[n0 + tile_col(0)] -= c0;
+        wg[n0 + tile_col(1)] -= c1;
+      }
+    }
   }
-  __syncthreads();
+  __syncthreads();  // dG complete; dX_w, dX_u (in the dS_e^T and S0 tiles), W and U~ are read no more
+  if (more && tid == 0) issue(3, nxt);
   // ---- 13. dk^ += (dG + dG^T) K^
   gemm_acc2<false, false>(Dk, 64, Pm, K, dk, [](int) { return 1.f; });
   gemm_acc2<true, false>(Dk, 64, Pm, K, dk, [](int) { return 1.f; });
