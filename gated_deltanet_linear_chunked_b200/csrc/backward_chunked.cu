@@ -492,9 +492,10 @@ gdn_bwd_pre_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 // B fragments come from the staged W and K~ tiles by ldmatrix (the
 // workspace's [slab][time row][8] layout; a lane's row address picks the
 // scan-order token).  W, K~ and e^{gam_C} arrive by one bulk copy per chunk
-// and the slices' X^T and Y^T columns by one each, into kChStages stages
+// and the slices' X^T, Y^T and S0 columns by one each, into kChStages stages
 // that the producer refills as the slices release them.  Each step writes
-// the chunk's dS_e^T and dU^T (bf16) for the gradient pass.
+// the chunk's dS_e^T and dU^T (bf16) for the gradient pass and adds the
+// slice's part of <dS_e, S0> to the chunk's sum.
 // One slice per CTA: slices sharing a stage would wait for one another, and
 // the step is bound by its dependent MMAs and exchanges, not by the loads.
 constexpr int kChSlices = 1;
@@ -815,11 +816,13 @@ ChainKernel chain_kernel_for(int nkb) {
 }
 
 // ----------------------------------------------------------- gradient pass
-// Every chunk at once (one CTA per (chunk, b*h, direction)), from the
-// chunk's dU and dS_e: every product but the chain's.  All product operands
-// are bf16 tiles in shared memory fed to mma.sync.m16n8k16 by ldmatrix (the
-// .trans form where a tile is read transposed); dq^ and dk^ accumulate in
-// registers; the triangular solve is the product with the forward's own
+// Every chunk (persistent CTAs, one per SM, walking the (chunk, b*h,
+// direction) tiles), from the chunk's dU and dS_e: every product but the
+// chain's.  All product operands are bf16 tiles in shared memory -- the
+// staged ones in their sources' core-matrix layouts, brought by one thread
+// a chunk ahead -- fed to mma.sync.m16n8k16 by ldmatrix (the .trans form
+// where a tile is read transposed); dq^ and dk^ accumulate in registers;
+// the triangular solve is the product with the forward's own
 // T = (I + A)^-1, which its stage A leaves in the workspace.
 struct GradLayout {
   int lbk, lbv;
