@@ -1154,15 +1154,38 @@ gdn_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   //          X_w = diag(beta e^gam) K^ (s_p = k^_p . dX_w_p gives e^gam_p s_p
   //          to beta_p and beta_p e^gam_p s_p to gam_p); dX_u goes out as it
   //          is (the reduction forms dv = beta dX_u and beta's v . dX_u)
-  for_acc(Dk, [&](int i, int hh, int e, int m, int n) {
-    dk[i][hh][e] = fmaf(sm.beta[m] * sm.eg[m], bf(sXw[cidx(m, n, 64, false)]), dk[i][hh][e]);
-  });
-  acc_row_sums(Dk, wb, [&](int, int, int, int m, int n) {
-    return sm.eg[m] * bf(sKc[cidx(m, n, 64, rev)]) * bf(sXw[cidx(m, n, 64, false)]);
-  });
-  acc_row_sums(Dk, wg, [&](int, int, int, int m, int n) {
-    return sm.beta[m] * sm.eg[m] * bf(sKc[cidx(m, n, 64, rev)]) * bf(sXw[cidx(m, n, 64, false)]);
-  });
+  {  // one pass over this thread's elements of the 64 x Dk register blocks
+    const int tn = Dk >> 4, nt = 4 * tn;
+#pragma unroll
+    for (int i = 0; i < kMaxBlocks; ++i) {
+      const int t = warp + kGrWarps * i;
+      if (t < nt) {
+        const int m0 = (t / tn) << 4, n0 = (t % tn) << 4;
+        float r[2] = {0.f, 0.f};  // s of rows m0 + gq and m0 + gq + 8
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int m = m0 + tile_row(e), n = n0 + 8 * hh + tile_col(e);
+            const float xw = bf(sXw[cidx(m, n, 64, false)]);
+            dk[i][hh][e] = fmaf(sm.beta[m] * sm.eg[m], xw, dk[i][hh][e]);
+            r[e >> 1] = fmaf(bf(sKc[cidx(m, n, 64, rev)]), xw, r[e >> 1]);
+          }
+#pragma unroll
+        for (int off = 1; off < 4; off <<= 1) {
+          r[0] += __shfl_xor_sync(0xffffffffu, r[0], off);
+          r[1] += __shfl_xor_sync(0xffffffffu, r[1], off);
+        }
+        if ((lane & 3) == 0) {  // this warp's partial rows: e^gam s to beta, beta e^gam s to gam
+          const int ma = m0 + tile_row(0), mb = m0 + tile_row(2);
+          wb[ma] += sm.eg[ma] * r[0];
+          wg[ma] += sm.beta[ma] * sm.eg[ma] * r[0];
+          wb[mb] += sm.eg[mb] * r[1];
+          wg[mb] += sm.beta[mb] * sm.eg[mb] * r[1];
+        }
+      }
+    }
+  }
   {  // dX_u rows: warp w takes rows 8 (w % 8) .. + 7 and every other slab
      // from w / 8; lane l the word l % 4 of row l / 4 (128 contiguous bytes a slab)
     const int p = 8 * (warp & 7) + (lane >> 2), r = sm.row[p];
