@@ -524,12 +524,21 @@ def backward_figure(gdn, lib, base, w, stream, peaks, peak_kind, barrier):
     per_tok = (4 * w.Dk + 3 * w.Dv) * 2 + 16
     nbytes = w.head_tokens * per_tok + 3 * w.B * w.H * w.Dk * w.Dv * 4
     gbs = nbytes / (ms / 1000.0) / 1e9
+    # the tensor pipe binds first: the forward's products recomputed, then
+    # twice them for the gradients
+    flops = 3 * algorithmic_flops(w, True)
+    tflops = flops / (ms / 1000.0) / 1e12
+    tpeak = peaks["bf16_tflops_sustained"]
     return {"workload": "stream_chunk_bidir (gradients)", "ms_per_call": ms,
             "head_tokens_per_s": w.head_tokens / (ms / 1000.0), "kernels": split,
             "roofline": {"bound": "hbm", "algorithmic_bytes": nbytes, "achieved_gbs": gbs,
                          "peak": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"],
                          "roofline_us": 1e6 * nbytes / (peaks["hbm_gbs"] * 1e9),
-                         "peak_source": f"{peak_kind} hbm_gbs"}}
+                         "peak_source": f"{peak_kind} hbm_gbs",
+                         "tensor": {"algorithmic_flops": flops, "achieved_tflops": tflops,
+                                    "peak": tpeak, "frac": tflops / tpeak,
+                                    "roofline_us": 1e6 * flops / (tpeak * 1e12),
+                                    "peak_source": f"{peak_kind} bf16_tflops_sustained"}}}
 
 
 def sink_window_figure(gdn, lib, stream, dev, peaks, peak_kind, barrier):
