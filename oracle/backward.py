@@ -16,8 +16,9 @@ a zero state; the state returned is the forward scan's.
 ``scan`` returns (out, state_out); ``grads`` returns the gradients of
 <out, d_out> + <state_out, d_state_out> with respect to q, k, v, g, beta and
 state_in.  ``tests/test_oracle_pins.py`` pins them to central finite
-differences of the recurrence, to the pure-decay closed form and to
-linearity, and checks the forward against the C oracle.
+differences of the recurrence, to the pure-decay closed form, to the
+single-token adjoint derived by hand and to linearity, and checks the forward
+against the C oracle.
 """
 from __future__ import annotations
 

@@ -610,3 +610,53 @@ def test_backward_forward_matches_c_oracle(bidir):
     o1, S1 = oracle.backward.forward_np(q, k, v, g, beta, s, bidir)
     o2, S2 = (c_bidir if bidir else c_fwd)(q, k, v, g, beta, s)
     assert rel(o1, o2) < 1e-12 and rel(S1, S2) < 1e-12
+
+
+@pytest.mark.parametrize("bidir", [False, True])
+def test_backward_single_token_adjoint_closed_form(bidir):
+    """T = 1, worked out by hand from one update step.  With M = q^ do^T + dS
+    (the gradient reaching S_1 = a (I - b k^k^T) S_0 + b k^ v^T):
+
+        dS_0 = a (I - b k^k^T) M          dv = b M^T k^
+        dg   = a <M, (I - b k^k^T) S_0>   db = <M, k^ v^T - a k^ k^T S_0>
+        dq^  = S_1 do                      dk^ = b M v - a b (M S_0^T + S_0 M^T) k^
+
+    and dx = (I - x^x^T) dx^ / |x| for the two normalised inputs.  The
+    reverse scan of a one-token chunk starts from zero, so bidirectional mode
+    adds o_r = b (k^.q^) v: dv += b (k^.q^) do, db += (k^.q^)(v.do),
+    dq^ += b (v.do) k^, dk^ += b (v.do) q^.  Each term is a separate
+    derivation, so a dropped term, a wrong sign or a transposed S_0 or M in
+    the oracle's gradient moves one of the six outputs."""
+    rng = np.random.default_rng(25)
+    Dk, Dv = 4, 3
+    q, k, v, g, beta, s = _fd_inputs(rng, B=1, T=1, H=1, Dk=Dk, Dv=Dv)
+    do = rng.standard_normal(v.shape)
+    dS = rng.standard_normal(s.shape)
+    gr = oracle.backward.grads(q, k, v, g, beta, s, do, dS, bidir=bidir)
+
+    qv, kv, vv, S0 = q[0, 0, 0], k[0, 0, 0], v[0, 0, 0], s[0, 0]
+    a, b, dov = np.exp(g[0, 0, 0]), beta[0, 0, 0], do[0, 0, 0]
+    nq, nk = np.linalg.norm(qv), np.linalg.norm(kv)
+    qh, kh = qv / nq, kv / nk
+    proj = np.eye(Dk) - b * np.outer(kh, kh)
+    S1 = a * proj @ S0 + b * np.outer(kh, vv)
+    M = np.outer(qh, dov) + dS[0, 0]
+    want = {
+        "dstate_in": a * proj @ M,
+        "dv": b * M.T @ kh,
+        "dg": a * np.sum(M * (proj @ S0)),
+        "dbeta": np.sum(M * (np.outer(kh, vv) - a * np.outer(kh, kh @ S0))),
+    }
+    dqh = S1 @ dov
+    dkh = b * M @ vv - a * b * (M @ S0.T + S0 @ M.T) @ kh
+    if bidir:
+        kq, vd = kh @ qh, vv @ dov
+        want["dv"] = want["dv"] + b * kq * dov
+        want["dbeta"] = want["dbeta"] + kq * vd
+        dqh = dqh + b * vd * kh
+        dkh = dkh + b * vd * qh
+    want["dq"] = (np.eye(Dk) - np.outer(qh, qh)) @ dqh / nq
+    want["dk"] = (np.eye(Dk) - np.outer(kh, kh)) @ dkh / nk
+    for name, w in want.items():
+        got = np.asarray(gr[name], np.float64).reshape(np.shape(w))
+        np.testing.assert_allclose(got, w, rtol=1e-12, atol=1e-14, err_msg=name)
