@@ -247,12 +247,10 @@ gdn_status scan(const void* q, const void* k, const void* v, const void* g,
 
 }  // namespace
 
-gdn_status prepare_scan(const void* q, const void* k, const void* v, const void* g,
-                        const void* beta, const float* state_in, float* state_out,
-                        void* out, int B, int T, int H, int Dk, int Dv, gdn_dtype dtype,
-                        int chunk, void* stream, bool bidir, bool gate_logits, ScanArgs* a,
-                        int* dev_out) {
-  // ---- pure host checks (no CUDA call)
+gdn_status check_scan_host(const void* q, const void* k, const void* v, const void* g,
+                           const void* beta, const float* state_in, float* state_out,
+                           void* out, int B, int T, int H, int Dk, int Dv, gdn_dtype dtype,
+                           int chunk, void* stream, bool bidir, bool gate_logits, ScanArgs* a) {
   if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
   if (B < 0 || T < 0 || H < 0 || Dk < 0 || Dv < 0) return GDN_ERR_INVALID_ARG;
   if (!supported_dim(Dk) || !supported_dim(Dv)) return GDN_ERR_UNSUPPORTED;
@@ -267,7 +265,6 @@ gdn_status prepare_scan(const void* q, const void* k, const void* v, const void*
   a->stream = static_cast<cudaStream_t>(stream);
   a->err = nullptr;
   a->wait_limit = 0;
-  *dev_out = 0;
   if (B == 0 || H == 0) return GDN_OK;
 
   const size_t es = dtype == GDN_BF16 ? 2 : 4;
@@ -292,22 +289,37 @@ gdn_status prepare_scan(const void* q, const void* k, const void* v, const void*
   }
   if (state_in && state_out && state_in != state_out && overlaps(rsi, rso))
     return GDN_ERR_ALIAS;
+  return GDN_OK;
+}
 
-  // ---- device checks
+gdn_status check_scan_device(const ScanArgs& a, int* dev_out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
     cudaGetLastError();
     return GDN_ERR_CUDA;
   }
+  const void* ptrs[] = {a.q, a.k, a.v, a.g, a.beta, a.state_in, a.state_out, a.out};
   for (const void* p : ptrs) {
     if (!p) continue;
-    if (T == 0 && p != state_in && p != state_out) continue;
+    if (a.T == 0 && p != a.state_in && p != a.state_out) continue;
     const gdn_status st = check_device_pointer(p, dev);
     if (st != GDN_OK) return st;
   }
   cudaGetLastError();  // start from a clean launch-error state
   *dev_out = dev;
   return GDN_OK;
+}
+
+gdn_status prepare_scan(const void* q, const void* k, const void* v, const void* g,
+                        const void* beta, const float* state_in, float* state_out,
+                        void* out, int B, int T, int H, int Dk, int Dv, gdn_dtype dtype,
+                        int chunk, void* stream, bool bidir, bool gate_logits, ScanArgs* a,
+                        int* dev_out) {
+  *dev_out = 0;
+  const gdn_status st = check_scan_host(q, k, v, g, beta, state_in, state_out, out, B, T, H, Dk,
+                                        Dv, dtype, chunk, stream, bidir, gate_logits, a);
+  if (st != GDN_OK || B == 0 || H == 0) return st;
+  return check_scan_device(*a, dev_out);
 }
 
 gdn_status trivial_state_copy(const ScanArgs& a) {
@@ -346,12 +358,15 @@ gdn_status backward(const void* q, const void* k, const void* v, const float* g,
                     const float* d_state_out, void* dq, void* dk, void* dv, float* dg,
                     float* dbeta, float* d_state_in, int B, int T, int H, int Dk, int Dv,
                     gdn_dtype dtype, void* stream, bool bidir) {
-  // the forward's checks on the forward's arguments (out := d_out, which is
-  // only read here; state_out := d_state_in, written)
+  // the forward's host checks on the forward's arguments (out := d_out, which
+  // is only read here; state_out := d_state_in, written), then the gradients'
+  // host checks, then the device checks of both: a bad argument is reported
+  // before any CUDA call
   ScanArgs a;
   int dev = 0;
-  gdn_status st = prepare_scan(q, k, v, g, beta, state_in, d_state_in, const_cast<void*>(d_out), B,
-                               T, H, Dk, Dv, dtype, 0, stream, bidir, false, &a, &dev);
+  gdn_status st = check_scan_host(q, k, v, g, beta, state_in, d_state_in,
+                                  const_cast<void*>(d_out), B, T, H, Dk, Dv, dtype, 0, stream,
+                                  bidir, false, &a);
   if (st != GDN_OK) return st;
   if (B == 0 || H == 0) return GDN_OK;
   const size_t es = dtype == GDN_BF16 ? 2 : 4;
@@ -377,6 +392,8 @@ gdn_status backward(const void* q, const void* k, const void* v, const float* g,
         if (overlaps(w[i], w[j])) return GDN_ERR_ALIAS;
     }
   }
+  st = check_scan_device(a, &dev);
+  if (st != GDN_OK) return st;
   for (const void* p : outs) {
     if (!p || (T == 0 && p != d_state_out)) continue;
     st = check_device_pointer(p, dev);

@@ -60,16 +60,28 @@ class ProfileScope {
   int slot_;
 };
 
-// Every check gdn.h lists for a scan call (host checks first, then device
-// residency of each pointer on the current device).  On GDN_OK `a` holds the
-// validated call (chunk defaulted; err and wait_limit not yet set) and `*dev`
-// the current device.  B == 0 or H == 0 returns GDN_OK with a->B or a->H
-// zero: the caller has nothing to do.
+// Every check gdn.h lists for a scan call: check_scan_host, then
+// check_scan_device.  On GDN_OK `a` holds the validated call (chunk defaulted;
+// err and wait_limit not yet set) and `*dev` the current device.  B == 0 or
+// H == 0 returns GDN_OK with a->B or a->H zero: the caller has nothing to do.
 gdn_status prepare_scan(const void* q, const void* k, const void* v, const void* g,
                         const void* beta, const float* state_in, float* state_out,
                         void* out, int B, int T, int H, int Dk, int Dv, gdn_dtype dtype,
                         int chunk, void* stream, bool bidir, bool gate_logits, ScanArgs* a,
                         int* dev);
+
+// The two halves of prepare_scan.  check_scan_host makes no CUDA call: dtype,
+// sizes, head dims, chunk, null pointers, 16-byte alignment and overlaps; on
+// GDN_OK it fills `a` (and stops there when B or H is zero).
+// check_scan_device checks that each pointer of a host-checked call is device
+// memory of the current device (with T == 0 only the states, the only buffers
+// touched); on GDN_OK `*dev` is that device.  Entry points with checks of
+// their own run all host checks before the device ones.
+gdn_status check_scan_host(const void* q, const void* k, const void* v, const void* g,
+                           const void* beta, const float* state_in, float* state_out,
+                           void* out, int B, int T, int H, int Dk, int Dv, gdn_dtype dtype,
+                           int chunk, void* stream, bool bidir, bool gate_logits, ScanArgs* a);
+gdn_status check_scan_device(const ScanArgs& a, int* dev);
 
 // T == 0: state_out = state_in (or zero); out untouched.
 gdn_status trivial_state_copy(const ScanArgs& a);

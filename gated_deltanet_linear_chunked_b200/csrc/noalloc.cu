@@ -49,11 +49,13 @@ extern "C" gdn_status gdn_chunk_fwd_noalloc(const void* q, const void* k, const 
   using namespace gdn;
   ScanArgs a;
   int dev = 0;
-  gdn_status st = prepare_scan(q, k, v, g, beta, state_in, state_out, out, B, T, H, Dk, Dv,
-                               dtype, chunk, stream, false, false, &a, &dev);
+  gdn_status st = check_scan_host(q, k, v, g, beta, state_in, state_out, out, B, T, H, Dk, Dv,
+                                  dtype, chunk, stream, false, false, &a);
   if (st != GDN_OK) return st;
   if (dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;  // the scratch-using path is bf16
   if (a.B == 0 || a.H == 0) return GDN_OK;
+  st = check_scan_device(a, &dev);
+  if (st != GDN_OK) return st;
   if (a.T == 0) return trivial_state_copy(a);
   if (chunk_tc_workspace_bytes(B, T, H, Dk, Dv, false) > kScratchBytes)
     return GDN_ERR_SCRATCH_LIMIT;

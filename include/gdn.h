@@ -45,7 +45,11 @@
  * come from several host threads at once.
  *
  * Errors.  Arguments are validated on the host before anything is enqueued;
- * on any error nothing is launched and a status is returned:
+ * on any error nothing is launched and a status is returned.  The checks that
+ * need no CUDA call (sizes, dims, dtype, chunk, null pointers, alignment,
+ * overlaps) all run before those that do (that each pointer is device memory
+ * of the current device), so a bad argument is reported as such even when no
+ * device is usable:
  *   GDN_ERR_INVALID_ARG  null pointer where data is needed, negative size,
  *                        pointer not 16-byte aligned, host (pageable or
  *                        pinned) pointer, unknown dtype, bad chunk value

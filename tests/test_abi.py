@@ -195,3 +195,79 @@ def test_sink_window_overlaps():
     # usable device the device checks report it, and nothing is launched
     st = swa(k=fake(3) + slot * chunk, v=fake(4) + slot * chunk)
     assert st in (_lib.GDN_ERR_CUDA, _lib.GDN_ERR_INVALID_ARG)
+
+
+# ---------------------------------------------------------------- backward
+# Gradient outputs at their own fake addresses, apart from the forward's.
+def bwd(entry="gdn_chunk_fwd_backward", q=fake(0), k=fake(1), v=fake(2), g=fake(3),
+        beta=fake(4), s_in=fake(5), d_out=fake(6), d_s_out=fake(7), dq=fake(8), dk=fake(9),
+        dv=fake(10), dg=fake(11), dbeta=fake(12), d_s_in=fake(13), B=1, T=64, H=2, Dk=64,
+        Dv=64, dtype=_lib.GDN_BF16):
+    lib = _lib.load()
+    return getattr(lib, entry)(q, k, v, g, beta, s_in, d_out, d_s_out, dq, dk, dv, dg, dbeta,
+                               d_s_in, B, T, H, Dk, Dv, dtype, None)
+
+
+BWD_ENTRIES = ["gdn_chunk_fwd_backward", "gdn_chunk_bidir_backward"]
+GRADS = ("dq", "dk", "dv", "dg", "dbeta", "d_s_in")
+
+
+@pytest.mark.parametrize("entry", BWD_ENTRIES)
+def test_backward_null_pointers_rejected(entry):
+    for name in ("q", "k", "v", "g", "beta", "d_out", "dq", "dk", "dv", "dg", "dbeta"):
+        assert bwd(entry, **{name: None}) == _lib.GDN_ERR_INVALID_ARG, name
+
+
+@pytest.mark.parametrize("entry", BWD_ENTRIES)
+def test_backward_sizes_dims_and_dtype(entry):
+    assert bwd(entry, B=-1) == _lib.GDN_ERR_INVALID_ARG
+    assert bwd(entry, T=-3) == _lib.GDN_ERR_INVALID_ARG
+    assert bwd(entry, dtype=5) == _lib.GDN_ERR_INVALID_ARG
+    for d in (0, 8, 40, 144):
+        assert bwd(entry, Dk=d) == _lib.GDN_ERR_UNSUPPORTED, d
+        assert bwd(entry, Dv=d) == _lib.GDN_ERR_UNSUPPORTED, d
+    # nothing to do: no pointer is looked at
+    nulls = {n: None for n in ("q", "k", "v", "g", "beta", "d_out") + GRADS}
+    assert bwd(entry, B=0, **nulls) == _lib.GDN_OK
+    assert bwd(entry, H=0, **nulls) == _lib.GDN_OK
+
+
+@pytest.mark.parametrize("entry", BWD_ENTRIES)
+def test_backward_misaligned_pointers_rejected(entry):
+    for i, name in enumerate(("q", "k", "v", "g", "beta", "s_in", "d_out", "d_s_out") + GRADS):
+        assert bwd(entry, **{name: fake(i) + 8}) == _lib.GDN_ERR_INVALID_ARG, name
+
+
+@pytest.mark.parametrize("entry", BWD_ENTRIES)
+def test_backward_gradients_may_not_overlap_anything(entry):
+    reads = {"q": 0, "k": 1, "v": 2, "g": 3, "beta": 4, "s_in": 5, "d_out": 6, "d_s_out": 7}
+    for grad in GRADS:
+        for name, i in reads.items():      # a gradient inside an input
+            assert bwd(entry, **{grad: fake(i) + 256}) == _lib.GDN_ERR_ALIAS, (grad, name)
+        for other in GRADS:                # two gradients sharing memory
+            if other != grad:
+                slot = 8 + GRADS.index(other)
+                assert bwd(entry, **{grad: fake(slot) + 256}) == _lib.GDN_ERR_ALIAS, (grad, other)
+    # d_state_in exactly on state_in is an overlap too (it is written while
+    # state_in is still read)
+    assert bwd(entry, d_s_in=fake(5)) == _lib.GDN_ERR_ALIAS
+
+
+@pytest.mark.parametrize("entry", BWD_ENTRIES)
+def test_backward_valid_arguments_reach_the_device_checks(entry):
+    # optional buffers absent or present: the host checks pass and, with no
+    # usable device, the device checks report it; nothing is launched
+    for extra in ({}, {"s_in": None}, {"d_s_out": None}, {"d_s_in": None}):
+        assert bwd(entry, **extra) in (_lib.GDN_ERR_CUDA, _lib.GDN_ERR_INVALID_ARG), extra
+
+
+def test_allocation_free_entry_host_checks():
+    entry = "gdn_chunk_fwd_noalloc"
+    for name in ("q", "k", "v", "g", "beta", "out"):
+        assert call(entry, **{name: None}) == _lib.GDN_ERR_INVALID_ARG, name
+    assert call(entry, Dk=24) == _lib.GDN_ERR_UNSUPPORTED
+    assert call(entry, dtype=_lib.GDN_F32) == _lib.GDN_ERR_UNSUPPORTED   # bf16 only
+    assert call(entry, s_out=fake(7) + 64) == _lib.GDN_ERR_ALIAS
+    assert call(entry, q=fake(0) + 8) == _lib.GDN_ERR_INVALID_ARG
+    assert call(entry, B=0, q=None, k=None, v=None, g=None, beta=None, out=None) == _lib.GDN_OK
+    assert call(entry) in (_lib.GDN_ERR_CUDA, _lib.GDN_ERR_INVALID_ARG)
