@@ -660,3 +660,37 @@ def test_backward_single_token_adjoint_closed_form(bidir):
     for name, w in want.items():
         got = np.asarray(gr[name], np.float64).reshape(np.shape(w))
         np.testing.assert_allclose(got, w, rtol=1e-12, atol=1e-14, err_msg=name)
+
+
+@pytest.mark.parametrize("impl", ["c", "numpy"])
+def test_time_segments_compose_to_the_recurrence(impl):
+    """The time-segmented scan's reading: the update is affine in the state,
+    S_t = a_t (I - b_t k^k^T) S_{t-1} + b_t k^ v_t^T, so a segment of tokens
+    maps its start state by S_out = P S_in + R.  P is the segment walked from
+    the identity (Dk columns) with zero values, R the segment walked from a
+    zero state; both come from the oracle itself.  Composing the maps in time
+    order must give every segment's start state and the final state of one
+    scan, and re-walking each segment from its start must give that scan's
+    outputs -- exactly, up to fp64 rounding, for ragged segments too."""
+    rng = np.random.default_rng(26)
+    Bn, Hn, Dk, Dv = 2, 2, 6, 5
+    q, k, v, g, beta, s = rand_inputs(rng, Bn, 41, Hn, Dk, Dv)
+    out, S_end = FWD[impl](q, k, v, g, beta, s)
+    cuts = [0, 9, 10, 27, 41]
+    eye = np.broadcast_to(np.eye(Dk), (Bn, Hn, Dk, Dk)).copy()
+    maps = []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        sl = (slice(None), slice(a, b))
+        zeros_v = np.zeros(q[sl].shape[:3] + (Dk,), np.float32)
+        _, P = FWD[impl](q[sl], k[sl], zeros_v, g[sl], beta[sl], eye)
+        _, R = FWD[impl](q[sl], k[sl], v[sl], g[sl], beta[sl], np.zeros_like(s))
+        maps.append((P, R))
+    St = s
+    for (a, b), (P, R) in zip(zip(cuts[:-1], cuts[1:]), maps):
+        o, _ = FWD[impl](q[:, a:b], k[:, a:b], v[:, a:b], g[:, a:b], beta[:, a:b], St)
+        np.testing.assert_allclose(o, out[:, a:b], rtol=1e-12, atol=1e-13)
+        St = np.einsum("bhij,bhjk->bhik", P, St) + R
+    np.testing.assert_allclose(St, S_end, rtol=1e-12, atol=1e-13)
+    # a map that skips its decay or its projection is visibly wrong
+    P0 = maps[0][0]
+    assert np.max(np.abs(P0 - eye)) > 1e-2
