@@ -15,7 +15,9 @@ Contents
   * ``numpy_ref``  -- the same recurrence in numpy (a second, independent
                       transcription for tiny cases) and the chunked (WY / UT)
                       form of the scan in fp64, used only to pin that the
-                      chunked algebra reaches the recurrence exactly; and
+                      chunked algebra reaches the recurrence exactly;
+                      reverse mode through that chunked form, pinned to the
+                      autograd gradients the same way; and
                       ``gates_from_logits``, the gate activations in numpy.
   * ``backward``   -- the forward definition in plain PyTorch CPU float64,
                       differentiated by autograd: the reference gradients of

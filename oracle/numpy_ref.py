@@ -37,6 +37,13 @@
     length including a ragged tail; ``tests/test_oracle_pins.py`` checks that
     by brute force.  Only differences of gamma are exponentiated where they
     can be positive, so fast decays do not overflow.
+
+``chunked_backward``
+    Reverse mode through that sub-chunked form (the derivation is in its
+    docstring): the gradients the pages' bidirectional short training needs
+    (same page, 方法步骤详情, second step), computed the way the chunked
+    backward kernels do, in fp64.  Pinned by brute force against autograd of
+    the recurrence (``oracle.backward``); it is not itself a reference.
 """
 from __future__ import annotations
 
@@ -134,3 +141,141 @@ def chunked_bidir(q, k, v, g, beta, state_in=None, chunk=64):
     flip = lambda x: np.flip(np.asarray(x), axis=1)  # noqa: E731
     out_r, _ = chunked_fwd(flip(q), flip(k), flip(v), flip(g), flip(beta), None, chunk)
     return out_f + np.flip(out_r, axis=1), S
+
+
+def _normalise_vjp(x, dxh):
+    """Gradient through x^ = x / sqrt(max(|x|^2, 1e-12)) on the last axis:
+    (dx^ - x^ (x^ . dx^)) / |x|, or dx^ / 1e-6 where the clamp holds."""
+    ss = np.sum(x * x, axis=-1, keepdims=True)
+    n = np.sqrt(np.maximum(ss, 1e-12))
+    xh = x / n
+    proj = np.where(ss > 1e-12, np.sum(xh * dxh, axis=-1, keepdims=True), 0.0)
+    return (dxh - xh * proj) / n
+
+
+def _chunked_reverse_one(q, k, v, g, beta, S_init, d_out, dS_end, chunk):
+    """One (batch, head, direction) in scan order: q, k [T,Dk], v, d_out
+    [T,Dv], g, beta [T], S_init, dS_end [Dk,Dv].  Returns the gradients with
+    respect to q^, k^ (before the normalisation), v, g, beta and S_init."""
+    T = q.shape[0]
+    Qh, Kh = _normalise(q), _normalise(k)
+    fwd = []
+    S = S_init.copy()
+    for c0 in range(0, T, chunk):
+        sl = slice(c0, min(c0 + chunk, T))
+        Q, K, V, bt = Qh[sl], Kh[sl], v[sl], beta[sl]
+        gam = np.cumsum(g[sl])
+        n = gam.shape[0]
+        diff = gam[:, None] - gam[None, :]
+        strict = np.tril(np.ones((n, n), dtype=bool), -1)
+        incl = np.tril(np.ones((n, n), dtype=bool), 0)
+        E = np.exp(np.where(strict, diff, -np.inf))
+        G = K @ K.T
+        A = bt[:, None] * E * G
+        Tm = np.linalg.inv(np.eye(n) + A)
+        W = Tm @ ((bt * np.exp(gam))[:, None] * K)
+        Ut = Tm @ (bt[:, None] * V)
+        U = Ut - W @ S
+        M = np.exp(np.where(incl, diff, -np.inf))
+        Kt = np.exp(gam[-1] - gam)[:, None] * K
+        fwd.append(dict(sl=sl, Q=Q, K=K, V=V, bt=bt, gam=gam, strict=strict, E=E, G=G, A=A,
+                        Tm=Tm, W=W, Ut=Ut, U=U, M=M, P=M * (Q @ K.T), Kt=Kt, S0=S))
+        S = np.exp(gam[-1]) * S + Kt.T @ U
+    dqh, dkh = np.zeros_like(Qh), np.zeros_like(Kh)
+    dv, dg, dbeta = np.zeros_like(v), np.zeros(T), np.zeros(T)
+    dSe = dS_end.copy()
+    for c in reversed(fwd):
+        sl, Q, K, V, bt, gam = c["sl"], c["Q"], c["K"], c["V"], c["bt"], c["gam"]
+        W, Ut, U, P, Kt, S0, Tm = c["W"], c["Ut"], c["U"], c["P"], c["Kt"], c["S0"], c["Tm"]
+        dO = d_out[sl]
+        e, eC = np.exp(gam), np.exp(gam[-1])
+        # O = diag(e^g) Q^ S0 + P U  and  S_e = e^{g_C} S0 + K~^T U
+        dU = P.T @ dO + Kt @ dSe
+        dP = dO @ U.T
+        dQK = c["M"] * dP
+        dQ = dQK @ K + e[:, None] * (dO @ S0.T)
+        dK = dQK.T @ Q
+        dKt = U @ dSe.T
+        dK += np.exp(gam[-1] - gam)[:, None] * dKt
+        # U = U~ - W S0
+        dS0 = eC * dSe + Q.T @ (e[:, None] * dO) - W.T @ dU
+        dW = -dU @ S0.T
+        # W = T diag(beta e^g) K^ and U~ = T diag(beta) V, T = (I + A)^-1:
+        # the transposed solve, then dA = -T^T dT T^T = -(X_w W^T + X_u U~^T)
+        Xw, Xu = Tm.T @ dW, Tm.T @ dU
+        dK += (bt * e)[:, None] * Xw
+        dv[sl] = bt[:, None] * Xu
+        xk = np.sum(Xw * K, axis=1)
+        dbt = e * xk + np.sum(Xu * V, axis=1)
+        dgam = bt * e * xk
+        dA = np.where(c["strict"], -(Xw @ W.T + Xu @ Ut.T), 0.0)
+        # A = diag(beta) (E o K^ K^^T), E_ti = e^{g_t - g_i} below the diagonal
+        dG = dA * bt[:, None] * c["E"]
+        dK += (dG + dG.T) @ K
+        dbt += np.sum(dA * c["E"] * c["G"], axis=1)
+        dAA = dA * c["A"]
+        dgam += dAA.sum(axis=1) - dAA.sum(axis=0)
+        # the decays inside O and S_e
+        dgam += np.sum(dO * (e[:, None] * (Q @ S0)), axis=1)
+        dPP = dP * P
+        dgam += dPP.sum(axis=1) - dPP.sum(axis=0)
+        dKK = np.sum(dKt * Kt, axis=1)
+        dgam -= dKK
+        dgam[-1] += dKK.sum() + eC * np.sum(dSe * S0)
+        # gamma_r = sum_{i<=r} g_i: dg is the suffix sum of dgamma
+        dg[sl] = np.cumsum(dgam[::-1])[::-1]
+        dbeta[sl] = dbt
+        dqh[sl], dkh[sl] = dQ, dK
+        dSe = dS0
+    return dqh, dkh, dv, dg, dbeta, dSe
+
+
+def chunked_backward(q, k, v, g, beta, state_in, d_out, d_state_out=None, bidir=False,
+                     chunk=64):
+    """Gradients of <out, d_out> + <state_out, d_state_out> by reverse mode
+    through the sub-chunked form above: the derivation the chunked backward
+    kernels compute, restated in fp64.  Per sub-chunk, walked in reverse
+    scan order with dS_e the gradient reaching its end state:
+
+      dU   = P^T dO + K~ dS_e                      (P = Mask o Q^ K^^T)
+      dS0  = e^{gamma_n} dS_e + Q^^T diag(e^gamma) dO - W^T dU   (-> dS_e of
+             the sub-chunk before)
+      dq^  = (Mask o dO U^T) K^ + diag(e^gamma) dO S0^T
+      dk^  = (Mask o dO U^T)^T Q^ + diag(e^{gamma_n - gamma}) U dS_e^T
+             + diag(beta e^gamma) X_w + (dG + dG^T) K^
+      [X_w | X_u] = T^T [-dU S0^T | dU],  dv = diag(beta) X_u
+      dA   = -(X_w W^T + X_u U~^T) below the diagonal,  dG = dA o diag(beta) E
+      dbeta, dgamma: row (and column) sums of the terms each factor enters;
+      dg   = suffix sum of dgamma over the sub-chunk.
+
+    q, k, v pass through the normalisation's Jacobian at the end; bidir adds
+    the reverse scan from zero (no state gradient) on the flipped sequence.
+    Returns the dict of ``oracle.backward.grads``."""
+    q, k, v, g, beta, d_out = _as64(q, k, v, g, beta, d_out)
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    S_in = np.zeros((B, H, Dk, Dv)) if state_in is None else np.asarray(state_in, np.float64)
+    dS_out = (np.zeros((B, H, Dk, Dv)) if d_state_out is None
+              else np.asarray(d_state_out, np.float64))
+    dqh, dkh = np.zeros_like(q), np.zeros_like(k)
+    dv, dg, dbeta = np.zeros_like(v), np.zeros_like(g), np.zeros_like(beta)
+    dstate = np.zeros((B, H, Dk, Dv))
+    fwd_order, rev_order = np.arange(T), np.arange(T)[::-1]
+    for b in range(B):
+        for h in range(H):
+            runs = [(fwd_order, S_in[b, h], dS_out[b, h])]
+            if bidir:
+                runs.append((rev_order, np.zeros((Dk, Dv)), np.zeros((Dk, Dv))))
+            for r, (idx, S0, dSe) in enumerate(runs):
+                res = _chunked_reverse_one(q[b, idx, h], k[b, idx, h], v[b, idx, h],
+                                           g[b, idx, h], beta[b, idx, h], S0, d_out[b, idx, h],
+                                           dSe, chunk)
+                dqh[b, idx, h] += res[0]
+                dkh[b, idx, h] += res[1]
+                dv[b, idx, h] += res[2]
+                dg[b, idx, h] += res[3]
+                dbeta[b, idx, h] += res[4]
+                if r == 0:
+                    dstate[b, h] = res[5]
+    return {"dq": _normalise_vjp(q, dqh), "dk": _normalise_vjp(k, dkh), "dv": dv, "dg": dg,
+            "dbeta": dbeta, "dstate_in": None if state_in is None else dstate}

@@ -694,3 +694,31 @@ def test_time_segments_compose_to_the_recurrence(impl):
     # a map that skips its decay or its projection is visibly wrong
     P0 = maps[0][0]
     assert np.max(np.abs(P0 - eye)) > 1e-2
+
+
+@pytest.mark.parametrize("bidir", [False, True])
+@pytest.mark.parametrize("chunk,with_state", [(4, True), (7, True), (64, True), (7, False)])
+def test_chunked_reverse_mode_reaches_the_reference_gradients(bidir, chunk, with_state):
+    """Brute force: reverse mode through the sub-chunked (WY / UT) form --
+    dU, dS0 carried backwards over the sub-chunks, the transposed solve
+    T^T [dW | dU], dA = -(X_w W^T + X_u U~^T), row and column sums for dbeta
+    and dgamma, dg as a suffix sum -- reaches autograd of the token
+    recurrence for every input, sub-chunks of 4, 7 (ragged) and 64 tokens,
+    with and without a start state; rows of zero and of tiny norm exercise
+    the normalisation's clamp."""
+    rng = np.random.default_rng(27)
+    q, k, v, g, beta, s = _fd_inputs(rng, B=2, T=23, H=2, Dk=6, Dv=5)
+    q[0, 3, 1] = 0.0
+    k[1, 11, 0] = 0.0
+    q[1, 5, 0] *= 1e-8
+    s = s if with_state else None
+    do = rng.standard_normal(v.shape)
+    dS = rng.standard_normal((2, 2, 6, 5))
+    want = oracle.backward.grads(q, k, v, g, beta, s, do, dS, bidir=bidir)
+    got = oracle.numpy_ref.chunked_backward(q, k, v, g, beta, s, do, dS, bidir=bidir, chunk=chunk)
+    for name in ("dq", "dk", "dv", "dg", "dbeta"):
+        np.testing.assert_allclose(got[name], want[name], rtol=1e-10, atol=1e-10, err_msg=name)
+    if with_state:
+        np.testing.assert_allclose(got["dstate_in"], want["dstate_in"], rtol=1e-10, atol=1e-12)
+    else:
+        assert got["dstate_in"] is None
