@@ -37,3 +37,33 @@ def test_path_flops_forms():
     d, c = 112, 64
     assert bench.algorithmic_flops(w) == 2640 * 20 * (6 * d * d + 8 * c * d)
     assert bench.algorithmic_flops(w, True) == 2 * bench.algorithmic_flops(w)
+
+
+@pytest.mark.parametrize("mode", ["fwd", "bidir"])
+def test_reference_arm_prints_one_contract_line(mode):
+    """``bench.py --impl reference`` (the fp64 oracle on this host's cores)
+    prints exactly one JSON line on the same metric, unit, direction and
+    workload as the native arm, with its own cpu_baseline and an e2e that
+    moves no bytes."""
+    import json
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--mode", mode, "--steps", "1", "--warmup", "0"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference"
+    assert d["metric"] == bench.METRIC and d["unit"] == bench.UNIT
+    assert d["higher_is_better"] is True and d["scaling"] == "weak"
+    assert d["steps"] == 1 and d["warmup"] == 0 and d["n_gpus"] == 1
+    assert d["config"]["workload"] == ("stream_chunk_causal" if mode == "fwd"
+                                       else "stream_chunk_bidir")
+    assert (d["config"]["T"], d["config"]["Dk"], d["config"]["Dv"]) == (2640, 112, 112)
+    assert d["value"] > 0 and d["ms_per_step"] > 0
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1
+    assert cb["unit"] == d["unit"] and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
