@@ -354,9 +354,6 @@ gdn_bwd_scan_kernel(BwdArgs A) {
   }
 }
 
-__device__ __forceinline__ void st_io(float* p, float x) { *p = x; }
-__device__ __forceinline__ void st_io(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
-
 // Sum the partials of every slice and direction for one (b, t, h) row, apply
 // the normalisation's Jacobian, and write dq, dk, dv, dg, dbeta.
 // pab[..][0] holds dL/da (token-serial path: dg = e^g da) or dL/dg itself
