@@ -722,3 +722,31 @@ def test_chunked_reverse_mode_reaches_the_reference_gradients(bidir, chunk, with
         np.testing.assert_allclose(got["dstate_in"], want["dstate_in"], rtol=1e-10, atol=1e-12)
     else:
         assert got["dstate_in"] is None
+
+
+def test_planted_gradient_slip_fails_both_gradient_pins(monkeypatch):
+    """The gradient pins have teeth: a copy of the gradient oracle's
+    recurrence with the decay applied after the delta correction (the slip
+    the forward's planted test uses) fails the hand-derived single-token
+    adjoint and the chunked reverse mode alike."""
+    import torch
+
+    def slipped(q, k, v, g, beta, S, reverse):
+        T = q.shape[1]
+        qn, kn = oracle.backward._normalise(q), oracle.backward._normalise(k)
+        outs = [None] * T
+        for t in (range(T - 1, -1, -1) if reverse else range(T)):
+            kt, qt, vt = kn[:, t], qn[:, t], v[:, t]
+            a = torch.exp(g[:, t])[..., None, None]
+            b = beta[:, t][..., None, None]
+            S = a * S
+            x = torch.einsum("bhi,bhij->bhj", kt, S)
+            S = S - b * kt[..., :, None] * x[..., None, :] + a * b * kt[..., :, None] * vt[..., None, :]
+            outs[t] = torch.einsum("bhi,bhij->bhj", qt, S)
+        return torch.stack(outs, dim=1), S
+
+    monkeypatch.setattr(oracle.backward, "_one_direction", slipped)
+    with pytest.raises(AssertionError):
+        test_backward_single_token_adjoint_closed_form(False)
+    with pytest.raises(AssertionError):
+        test_chunked_reverse_mode_reaches_the_reference_gradients(False, 7, True)
