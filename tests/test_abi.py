@@ -271,3 +271,59 @@ def test_allocation_free_entry_host_checks():
     assert call(entry, q=fake(0) + 8) == _lib.GDN_ERR_INVALID_ARG
     assert call(entry, B=0, q=None, k=None, v=None, g=None, beta=None, out=None) == _lib.GDN_OK
     assert call(entry) in (_lib.GDN_ERR_CUDA, _lib.GDN_ERR_INVALID_ARG)
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "gdn.h"
+
+#define CHECK(cond) do { if (!(cond)) { printf("failed: %s\n", #cond); return 1; } } while (0)
+
+int main(void) {
+    /* fake, aligned, disjoint addresses: every status below comes from the
+       host checks, before any CUDA call */
+    char* base = (char*)0x7f0000000000ULL;
+    const void* q = base;
+    const void* k = base + (1 << 24);
+    const void* v = base + (2 << 24);
+    const float* g = (const float*)(base + (3 << 24));
+    const float* beta = (const float*)(base + (4 << 24));
+    void* out = base + (5 << 24);
+    CHECK(gdn_version() >= 100);
+    CHECK(strcmp(gdn_status_string(GDN_ERR_ALIAS), "GDN_ERR_ALIAS") == 0);
+    CHECK(gdn_chunk_fwd(NULL, k, v, g, beta, NULL, NULL, out, 1, 64, 2, 64, 64, GDN_BF16, 0,
+                        NULL) == GDN_ERR_INVALID_ARG);
+    CHECK(gdn_chunk_bidir(q, k, v, g, beta, NULL, NULL, out, 1, 64, 2, 24, 64, GDN_BF16, 0,
+                          NULL) == GDN_ERR_UNSUPPORTED);
+    CHECK(gdn_chunk_fwd(q, k, v, g, beta, NULL, NULL, (void*)q, 1, 64, 2, 64, 64, GDN_BF16, 0,
+                        NULL) == GDN_ERR_ALIAS);
+    CHECK(gdn_chunk_fwd(q, k, v, g, beta, NULL, NULL, out, 0, 64, 2, 64, 64, GDN_BF16, 0,
+                        NULL) == GDN_OK);
+    CHECK(gdn_sink_window_slot(5, 1, 2) == 1);  /* 1 + (5 - 1) mod 2 */
+    printf("ok\n");
+    return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_the_library_links_from_c(tmp_path):
+    """A C99 program (no C++, no CUDA headers) includes gdn.h, links
+    libgdn.so and gets the documented statuses back from the host checks."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc") or shutil.which("cc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    lib_dir = os.path.dirname(_lib.library_path())
+    _lib.load()  # builds the library if it is missing
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    cc = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                         "-I", os.path.join(ROOT, "include"), str(src), "-L", lib_dir, "-lgdn",
+                         "-Wl,-rpath," + lib_dir, "-o", str(exe)],
+                        capture_output=True, text=True)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0 and run.stdout.strip() == "ok", run.stdout + run.stderr
