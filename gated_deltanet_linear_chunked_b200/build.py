@@ -5,7 +5,7 @@
 Compiles every ``csrc/*.cu`` into one shared library beside this file
 (``libgdn.so``), exporting the C ABI declared in ``include/gdn.h``.  The CUDA
 runtime is linked statically, so the library loads on a machine without a
-GPU (the ABI tests use that); the driver API (tensor maps) is reached at run
+GPU (the ABI tests use that); the CUDA driver API (tensor maps) is reached at run
 time through ``cudaGetDriverEntryPoint``.
 """
 from __future__ import annotations

@@ -104,7 +104,7 @@ def test_overlaps_rejected():
 
 def test_valid_arguments_reach_the_device_checks_without_a_gpu():
     # All host checks pass; with no usable device the call reports a CUDA
-    # error instead of crashing (on a GPU machine the fake pointers are rejected
+    # error instead of crashing (on a machine with a GPU the fake pointers are rejected
     # as not device memory).  Either way nothing is launched.
     st = call()
     assert st in (_lib.GDN_ERR_CUDA, _lib.GDN_ERR_INVALID_ARG)

@@ -82,7 +82,7 @@ def _noalloc(x, out, state_in, state_out, w):
 
 def test_noalloc_matches_allocating_entry_point_twice():
     """Two calls in a row.  The first call on a device may load the module
-    that holds the fixed array (the driver places it then, once), so free
+    that holds the fixed array (the CUDA driver places it then, once), so free
     device memory is compared across the second call; the default pool's
     high-water mark across both."""
     pool = DefaultPool()
