@@ -166,3 +166,25 @@ def test_logit_recipe_has_the_stated_gate_distributions():
     x = wl.make_inputs(wl.Workload("lg", 2, 33, 3, 16, 16, "f32", 16, "fwd", ("logit_normal",),
                                    ("logit_normal",), ("zero",), 3))
     assert x["g_logit"].shape == (2, 33, 3) and "g" not in x
+
+
+def test_attention_stream_recipe():
+    """The softmax blocks' stream: the GDN blocks' head layout, one sink
+    chunk and a window of two (7920 keys from chunk 2 on), bf16 values with
+    the stated distributions, each chunk seeded on its own."""
+    w = wl.sink_window_stream()
+    assert (w.B, w.Tc, w.H, w.D, w.n_sink, w.window) == (1, 2640, 20, 112, 1, 2)
+    assert w.steady_chunk == 2 and (w.n_sink + w.window) * w.Tc == 7920
+    small = wl.AttnStream("t", 1, 300, 2, 64, 1, 2, 3, 7)
+    a0, a1 = wl.attn_chunk(small, 0), wl.attn_chunk(small, 1)
+    for n in ("q", "k", "v"):
+        assert a0[n].shape == (1, 300, 2, 64)
+        assert np.all((a0[n].view(np.uint32) & 0xFFFF) == 0)          # bf16 values
+        x = a0[n].astype(np.float64)
+        assert abs(x.mean()) < 0.02 and abs(x.std() - 1.0) < 0.02      # N(0, 1)
+        assert not np.array_equal(a0[n], a1[n])                        # per-chunk seeds
+        assert np.array_equal(a0[n], wl.attn_chunk(small, 0)[n])       # reproducible
+    sharp = wl.AttnStream("t", 1, 300, 2, 64, 1, 2, 3, 7, q_scale=6.0)
+    qs = wl.attn_chunk(sharp, 0)["q"].astype(np.float64)
+    assert abs(qs.std() - 6.0) < 0.1                                   # N(0, q_scale^2)
+    np.testing.assert_array_equal(wl.attn_chunk(sharp, 0)["k"], a0["k"])  # k, v unscaled
