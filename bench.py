@@ -65,13 +65,36 @@ def parse():
 
 
 def load_peaks():
+    """The roofline denominators and where they came from.  Each of the three
+    peaks is taken from MEASURED_PEAKS.json when the file holds it as a
+    number, else from FALLBACK_PEAKS; an absent or unreadable file counts as
+    holding none.  The second value names the source for the peak_source
+    fields: "measured", "fallback", or "measured, with fallback for <keys>"."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        return d, "measured"
-    except OSError:
-        return dict(FALLBACK_PEAKS), "fallback"
+    except (OSError, ValueError):
+        d = {}
+    if not isinstance(d, dict):
+        d = {}
+    peaks, missing = {}, []
+    for key, fallback in FALLBACK_PEAKS.items():
+        v = d.get(key)
+        try:
+            v = float(v)
+        except (TypeError, ValueError):
+            v = None
+        if v is None or not v > 0:
+            peaks[key] = fallback
+            missing.append(key)
+        else:
+            peaks[key] = v
+    if not missing:
+        return peaks, "measured"
+    if len(missing) == len(FALLBACK_PEAKS):
+        return peaks, "fallback"
+    return peaks, "measured, with fallback for " + " and ".join(missing)
 
 
 def gate_keys(w):

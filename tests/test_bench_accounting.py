@@ -67,3 +67,53 @@ def test_reference_arm_prints_one_contract_line(mode):
     assert cb["unit"] == d["unit"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
+
+
+def test_peaks_file_is_read_key_by_key(monkeypatch, tmp_path):
+    """The roofline denominators: measured where the peaks file holds a
+    positive number, the fallback elsewhere, and the source said truthfully;
+    a missing or unreadable file means the fallback throughout."""
+    import json
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    f = tmp_path / "MEASURED_PEAKS.json"
+    assert bench.load_peaks() == (bench.FALLBACK_PEAKS, "fallback")           # absent
+    full = {"hbm_gbs": 6547.2, "bf16_tflops": 1646.1, "bf16_tflops_sustained": 1391.6,
+            "clocks": {"sm_mhz": 1965}}
+    f.write_text(json.dumps(full))
+    peaks, kind = bench.load_peaks()
+    assert kind == "measured" and peaks == {k: full[k] for k in bench.FALLBACK_PEAKS}
+    f.write_text(json.dumps({"hbm_gbs": "6547.2", "bf16_tflops": 1646.1}))
+    peaks, kind = bench.load_peaks()
+    assert peaks["hbm_gbs"] == 6547.2 and peaks["bf16_tflops"] == 1646.1
+    assert peaks["bf16_tflops_sustained"] == bench.FALLBACK_PEAKS["bf16_tflops_sustained"]
+    assert kind == "measured, with fallback for bf16_tflops_sustained"
+    for bad in ("{not json", "[1, 2]", json.dumps({"hbm_gbs": None, "bf16_tflops": -1})):
+        f.write_text(bad)
+        assert bench.load_peaks() == (bench.FALLBACK_PEAKS, "fallback"), bad
+
+
+@pytest.mark.parametrize("mode,bound", [("fwd", "hbm"), ("bidir", "tensor")])
+def test_roofline_object_arithmetic(mode, bound):
+    """The roofline object on made-up kernel times: the causal chunk is bound
+    by HBM and the bidirectional one by the tensor pipe; the dominant kernel
+    is the longest; achieved is the path's work per launch over that
+    kernel's time, the path figure the same work over the step."""
+    w = wl.stream_chunk(mode)
+    peaks = dict(bench.FALLBACK_PEAKS)
+    kernels = {"gdn_prep_kernel": {"ms_per_launch": 0.03},
+               "gdn_recur_kernel": {"ms_per_launch": 0.02},
+               "gdn_output_kernel": {"ms_per_launch": 0.04}}
+    r = bench.roofline_of(w, kernels, 0.1, peaks, "fallback", mode == "bidir")
+    assert r["bound"] == bound and r["kernel"] == "gdn_output_kernel"
+    if bound == "hbm":
+        work, peak, unit = bench.algorithmic_bytes(w) / 1e9, peaks["hbm_gbs"], "GB/s"
+    else:
+        work, peak = bench.algorithmic_flops(w, True) / 1e12, peaks["bf16_tflops_sustained"]
+        unit = "TFLOP/s"
+    assert r["unit"] == unit and r["peak"] == peak
+    assert r["achieved"] == pytest.approx(work / 0.04e-3)
+    assert r["frac"] == pytest.approx(work / 0.04e-3 / peak)
+    assert r["path"]["frac"] == pytest.approx(work / 0.1e-3 / peak)
+    assert r["peak_source"].startswith("fallback")
+    t_hbm, t_tc = bench.roofline_times(w, mode == "bidir", peaks)
+    assert r["path"]["roofline_us"] == pytest.approx(1e6 * max(t_hbm, t_tc))
