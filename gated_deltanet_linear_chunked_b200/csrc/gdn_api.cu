@@ -1,8 +1,10 @@
 // gdn_api.cu -- the C ABI (include/gdn.h): host-side validation and dispatch.
 //
 // Every entry point validates its arguments on the host before it enqueues
-// anything, then launches onto the caller's stream and returns without
-// synchronising.  Nothing here throws, aborts or prints.
+// anything -- first every check that needs no CUDA call, then that each
+// pointer is device memory of the current device -- then launches onto the
+// caller's stream and returns without synchronising.  Nothing here throws,
+// aborts or prints.
 //
 // Per-stream context.  The chunked path needs scratch between its kernels,
 // and every bounded wait needs a word to report an expiry in.  Both are kept
