@@ -1,0 +1,110 @@
+"""Property-based pins of the CPU oracle (no GPU): the fixed-case pins of
+test_oracle_pins.py, drawn over random small shapes instead.
+
+Each example draws its sizes (T, Dk, Dv, heads), a sub-chunk length, the
+mode, whether a start state is given, and a seed for the values; the
+properties are ones the mathematics fixes for every such draw:
+
+- the sub-chunked (WY / UT) forward form reaches the token recurrence;
+- reverse mode through that form reaches autograd of the recurrence;
+- streaming over arbitrary cut points equals one scan;
+- the C oracle and the numpy recurrence agree.
+"""
+import numpy as np
+from hypothesis import given, settings
+from hypothesis import strategies as st
+
+import oracle
+
+SETTINGS = settings(max_examples=25, deadline=None, derandomize=True)
+
+shapes = st.fixed_dictionaries({
+    "T": st.integers(1, 40),
+    "Dk": st.integers(1, 7),
+    "Dv": st.integers(1, 6),
+    "H": st.integers(1, 2),
+    "chunk": st.integers(1, 17),
+    "bidir": st.booleans(),
+    "state": st.booleans(),
+    "g_lo": st.sampled_from([-0.05, -1.0, -6.0]),
+    "seed": st.integers(0, 2 ** 31 - 1),
+})
+
+
+def draw(p):
+    rng = np.random.default_rng(p["seed"])
+    B, T, H, Dk, Dv = 1, p["T"], p["H"], p["Dk"], p["Dv"]
+    q = rng.standard_normal((B, T, H, Dk))
+    k = rng.standard_normal((B, T, H, Dk))
+    v = rng.standard_normal((B, T, H, Dv))
+    g = rng.uniform(p["g_lo"], 0.0, (B, T, H))
+    beta = rng.uniform(0.0, 1.0, (B, T, H))
+    s = rng.standard_normal((B, H, Dk, Dv)) if p["state"] else None
+    return rng, q, k, v, g, beta, s
+
+
+def rel(a, b):
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    return np.max(np.abs(a - b)) / max(np.max(np.abs(b)), 1e-300)
+
+
+@SETTINGS
+@given(shapes)
+def test_chunked_form_reaches_the_recurrence(p):
+    _, q, k, v, g, beta, s = draw(p)
+    if p["bidir"]:
+        want = oracle.recurrence_bidir(q, k, v, g, beta, s)
+        got = oracle.numpy_ref.chunked_bidir(q, k, v, g, beta, s, chunk=p["chunk"])
+    else:
+        want = oracle.recurrence_fwd(q, k, v, g, beta, s)
+        got = oracle.numpy_ref.chunked_fwd(q, k, v, g, beta, s, chunk=p["chunk"])
+    assert rel(got[0], want[0]) < 1e-10 and rel(got[1], want[1]) < 1e-10
+
+
+@SETTINGS
+@given(shapes)
+def test_chunked_reverse_mode_reaches_autograd(p):
+    rng, q, k, v, g, beta, s = draw(p)
+    do = rng.standard_normal(v.shape)
+    dS = rng.standard_normal((1, p["H"], p["Dk"], p["Dv"]))
+    want = oracle.backward.grads(q, k, v, g, beta, s, do, dS, bidir=p["bidir"])
+    got = oracle.numpy_ref.chunked_backward(q, k, v, g, beta, s, do, dS, bidir=p["bidir"],
+                                            chunk=p["chunk"])
+    # with Dk = 1 the normalised q, k are +-1 and dq, dk vanish: compare
+    # against a floor set by the largest gradient, not each tensor's own
+    names = ["dq", "dk", "dv", "dg", "dbeta"] + ([] if s is None else ["dstate_in"])
+    scale = max(np.max(np.abs(want[n])) for n in names)
+    for name in names:
+        np.testing.assert_allclose(got[name], want[name], rtol=1e-9, atol=1e-12 * scale,
+                                   err_msg=name)
+    if s is None:
+        assert got["dstate_in"] is None and want["dstate_in"] is None
+
+
+@SETTINGS
+@given(shapes, st.lists(st.integers(0, 40), max_size=4))
+def test_streaming_over_any_cuts_equals_one_scan(p, cuts):
+    _, q, k, v, g, beta, s = draw(p)
+    T = p["T"]
+    out, S = oracle.recurrence_fwd(q, k, v, g, beta, s)
+    edges = sorted({0, T, *[c for c in cuts if c <= T]})
+    St = s
+    for a, b in zip(edges[:-1], edges[1:]):
+        o, St = oracle.recurrence_fwd(q[:, a:b], k[:, a:b], v[:, a:b], g[:, a:b], beta[:, a:b], St)
+        assert rel(o, out[:, a:b]) < 1e-12 or np.max(np.abs(out[:, a:b])) == 0
+    assert rel(St, S) < 1e-12
+
+
+@SETTINGS
+@given(shapes)
+def test_c_and_numpy_recurrences_agree(p):
+    _, q, k, v, g, beta, s = draw(p)
+    q, k, v = (x.astype(np.float32) for x in (q, k, v))
+    g, beta = g.astype(np.float32), beta.astype(np.float32)
+    if p["bidir"]:
+        c = oracle.oracle_bidir(q, k, v, g, beta, s, nthreads=1)
+        n = oracle.recurrence_bidir(q, k, v, g, beta, s)
+    else:
+        c = oracle.oracle_fwd(q, k, v, g, beta, s, nthreads=1)
+        n = oracle.recurrence_fwd(q, k, v, g, beta, s)
+    assert rel(c[0], n[0]) < 1e-12 and rel(c[1], n[1]) < 1e-12
