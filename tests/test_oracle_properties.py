@@ -8,7 +8,9 @@ properties are ones the mathematics fixes for every such draw:
 - the sub-chunked (WY / UT) forward form reaches the token recurrence;
 - reverse mode through that form reaches autograd of the recurrence;
 - streaming over arbitrary cut points equals one scan;
-- the C oracle and the numpy recurrence agree.
+- the C oracle and the numpy recurrence agree;
+- the library's cache-slot rule keeps every chunk the attention oracle's
+  visibility rule shows a query in a slot of its own.
 """
 import numpy as np
 from hypothesis import given, settings
@@ -108,3 +110,24 @@ def test_c_and_numpy_recurrences_agree(p):
         c = oracle.oracle_fwd(q, k, v, g, beta, s, nthreads=1)
         n = oracle.recurrence_fwd(q, k, v, g, beta, s)
     assert rel(c[0], n[0]) < 1e-12 and rel(c[1], n[1]) < 1e-12
+
+
+@SETTINGS
+@given(st.integers(0, 6), st.integers(1, 8), st.integers(0, 60))
+def test_cache_slots_of_the_visible_chunks_are_distinct(n_sink, window, c):
+    """The library's cache-slot rule against the oracle's visibility rule:
+    every chunk a query of chunk c sees (its own included) still sits in its
+    own slot of the n_sink + window cache when chunk c runs, so no two visible
+    chunks share a slot, and each visible chunk's slot is the one it was
+    written to."""
+    from gated_deltanet_linear_chunked_b200 import _lib
+    lib = _lib.load()
+    seen = oracle.sink_window_attn.visible_chunks(c, n_sink, window)
+    assert len(seen) == min(c + 1, n_sink + window)
+    slots = [lib.gdn_sink_window_slot(m, n_sink, window) for m in seen]
+    assert all(0 <= x < n_sink + window for x in slots)
+    assert len(set(slots)) == len(slots)
+    # nothing written after chunk m (up to c) landed in m's slot
+    for m, x in zip(seen, slots):
+        later = [lib.gdn_sink_window_slot(j, n_sink, window) for j in range(m + 1, c + 1)]
+        assert x not in later, (m, later)
