@@ -164,7 +164,8 @@ def recorded_traffic(kernel):
 
 
 class ClockSampler:
-    """Samples SM clock and throttle reasons through NVML every ~20 ms."""
+    """Samples SM clock and throttle reasons through NVML every ~5 ms (a
+    timed region of 20-400 graph replays lasts only tens of milliseconds)."""
 
     def __init__(self, device_index: int):
         self.samples, self.reasons, self.max_mhz = [], set(), None
@@ -202,7 +203,7 @@ class ClockSampler:
                 self._sample()
             except Exception:
                 pass
-            self._stop.wait(0.02)
+            self._stop.wait(0.005)
 
     def __enter__(self):
         if self.nv is not None:
