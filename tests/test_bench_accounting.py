@@ -117,3 +117,32 @@ def test_roofline_object_arithmetic(mode, bound):
     assert r["peak_source"].startswith("fallback")
     t_hbm, t_tc = bench.roofline_times(w, mode == "bidir", peaks)
     assert r["path"]["roofline_us"] == pytest.approx(1e6 * max(t_hbm, t_tc))
+
+
+def test_clock_sampler_against_a_fake_nvml(monkeypatch):
+    """The clock record of the JSON line, on a fake NVML: clocks sampled
+    while the region runs, reason bits decoded by name (idle dropped), the
+    median taken; and no NVML at all gives an empty record, not an error."""
+    import time
+    import types
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=1,
+        nvmlInit=lambda: None,
+        nvmlDeviceGetHandleByIndex=lambda i: ("gpu", i),
+        nvmlDeviceGetMaxClockInfo=lambda h, c: 1965,
+        nvmlDeviceGetClockInfo=lambda h, c: 1965,
+        nvmlDeviceGetCurrentClocksEventReasons=lambda h: 0x1 | 0x4,   # idle, sw_power_cap
+    )
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    with bench.ClockSampler(0) as c:
+        time.sleep(0.1)
+    s = c.summary()
+    assert s["sm_mhz"] == 1965 and s["sm_max_mhz"] == 1965
+    assert s["reasons"] == ["sw_power_cap"] and s["samples"] >= 5
+
+    def no_nvml():
+        raise RuntimeError("NVML unavailable")
+    monkeypatch.setattr(fake, "nvmlInit", no_nvml)
+    with bench.ClockSampler(0) as c:
+        time.sleep(0.01)
+    assert c.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
