@@ -146,3 +146,26 @@ def test_clock_sampler_against_a_fake_nvml(monkeypatch):
     with bench.ClockSampler(0) as c:
         time.sleep(0.01)
     assert c.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+
+def test_recorded_traffic_only_while_the_source_matches(monkeypatch, tmp_path):
+    """roofline.traffic comes from the committed ncu table only while the
+    kernel's source still hashes to the value the capture was taken on;
+    after any edit of that source it is null."""
+    import hashlib
+    src = tmp_path / "k.cu"
+    src.write_text("kernel v1\n")
+    (tmp_path / "profiles").mkdir()
+    digest = hashlib.sha256(src.read_bytes()).hexdigest()
+    (tmp_path / "profiles" / "dram_traffic.txt").write_text(
+        "# kernel  sha256  bytes\n" f"gdn_output_kernel {digest} 57273344\n"
+        f"gdn_prep_kernel {'0' * 64} 1\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "KERNEL_SOURCES", {"gdn_output_kernel": "k.cu",
+                                                  "gdn_prep_kernel": "k.cu"})
+    assert bench.recorded_traffic("gdn_output_kernel") == 57273344
+    assert bench.recorded_traffic("gdn_prep_kernel") is None       # taken on another source
+    assert bench.recorded_traffic("gdn_recur_kernel") is None      # no source known
+    src.write_text("kernel v2\n")
+    assert bench.recorded_traffic("gdn_output_kernel") is None      # source changed since
+
