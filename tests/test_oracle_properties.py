@@ -10,7 +10,9 @@ properties are ones the mathematics fixes for every such draw:
 - streaming over arbitrary cut points equals one scan;
 - the C oracle and the numpy recurrence agree;
 - the library's cache-slot rule keeps every chunk the attention oracle's
-  visibility rule shows a query in a slot of its own.
+  visibility rule shows a query in a slot of its own;
+- gate logits up to +-60 give gates in range, and the C oracle's logit mode
+  equals the numpy recurrence on numpy's gates.
 """
 import numpy as np
 from hypothesis import given, settings
@@ -131,3 +133,28 @@ def test_cache_slots_of_the_visible_chunks_are_distinct(n_sink, window, c):
     for m, x in zip(seen, slots):
         later = [lib.gdn_sink_window_slot(j, n_sink, window) for j in range(m + 1, c + 1)]
         assert x not in later, (m, later)
+
+
+@SETTINGS
+@given(shapes, st.floats(0.1, 60.0))
+def test_gate_logits_stay_in_range_and_transcriptions_agree(p, spread):
+    """Gate logits anywhere in [-spread, spread] (up to +-60, far past what a
+    bf16 gate layer emits) give g <= 0 and beta in [0, 1] with no NaN or
+    overflow, and the C oracle's logit mode equals the numpy recurrence fed
+    numpy's gates."""
+    rng, q, k, v, _, _, s = draw(p)
+    shape = q.shape[:3]
+    x = rng.uniform(-spread, spread, shape).astype(np.float32)
+    y = rng.uniform(-spread, spread, shape).astype(np.float32)
+    g, beta = oracle.gates_from_logits(x, y)
+    assert np.all(np.isfinite(g)) and np.all(g <= 0.0)
+    assert np.all((beta >= 0.0) & (beta <= 1.0))
+    q, k, v = (t.astype(np.float32) for t in (q, k, v))
+    if p["bidir"]:
+        c = oracle.oracle_bidir_logits(q, k, v, x, y, s, nthreads=1)
+        n = oracle.recurrence_bidir(q, k, v, g, beta, s)
+    else:
+        c = oracle.oracle_fwd_logits(q, k, v, x, y, s, nthreads=1)
+        n = oracle.recurrence_fwd(q, k, v, g, beta, s)
+    assert np.all(np.isfinite(c[0])) and np.all(np.isfinite(c[1]))
+    assert rel(c[0], n[0]) < 1e-11 and rel(c[1], n[1]) < 1e-11
