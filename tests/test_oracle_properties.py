@@ -12,7 +12,9 @@ properties are ones the mathematics fixes for every such draw:
 - the library's cache-slot rule keeps every chunk the attention oracle's
   visibility rule shows a query in a slot of its own;
 - gate logits up to +-60 give gates in range, and the C oracle's logit mode
-  equals the numpy recurrence on numpy's gates.
+  equals the numpy recurrence on numpy's gates;
+- the attention oracle's outputs are convex combinations of the visible
+  values, unchanged by a common shift of the keys, linear in the values.
 """
 import numpy as np
 from hypothesis import given, settings
@@ -158,3 +160,43 @@ def test_gate_logits_stay_in_range_and_transcriptions_agree(p, spread):
         n = oracle.recurrence_fwd(q, k, v, g, beta, s)
     assert np.all(np.isfinite(c[0])) and np.all(np.isfinite(c[1]))
     assert rel(c[0], n[0]) < 1e-11 and rel(c[1], n[1]) < 1e-11
+
+
+attn = st.fixed_dictionaries({
+    "chunk": st.integers(1, 6),
+    "chunks": st.integers(1, 5),
+    "d": st.integers(1, 8),
+    "dv": st.integers(1, 5),
+    "n_sink": st.integers(0, 2),
+    "window": st.integers(1, 3),
+    "scale": st.sampled_from([0.1, 1.0, 4.0]),
+    "seed": st.integers(0, 2 ** 31 - 1),
+})
+
+
+@SETTINGS
+@given(attn)
+def test_attention_is_a_convex_combination_invariant_to_a_key_shift(p):
+    """Softmax attention over the visible chunks: every output row lies in
+    the per-coordinate range of the values it can see; adding one vector to
+    every key moves each query's scores by a constant and leaves the output
+    alone; scaling the values scales the output."""
+    rng = np.random.default_rng(p["seed"])
+    T = p["chunk"] * p["chunks"]
+    q = p["scale"] * rng.standard_normal((1, T, 1, p["d"]))
+    k = rng.standard_normal((1, T, 1, p["d"]))
+    v = rng.standard_normal((1, T, 1, p["dv"]))
+    args = (p["chunk"], p["n_sink"], p["window"])
+    out = oracle.sink_window_attn.stream_outputs(q, k, v, *args)
+    for c in range(p["chunks"]):
+        rows = np.concatenate([np.arange(m * p["chunk"], (m + 1) * p["chunk"])
+                               for m in oracle.sink_window_attn.visible_chunks(c, p["n_sink"],
+                                                                                p["window"])])
+        lo, hi = v[0, rows, 0].min(axis=0), v[0, rows, 0].max(axis=0)
+        o = out[0, c * p["chunk"]:(c + 1) * p["chunk"], 0]
+        assert np.all(o >= lo - 1e-12) and np.all(o <= hi + 1e-12)
+    shift = rng.standard_normal(p["d"])
+    out2 = oracle.sink_window_attn.stream_outputs(q, k + shift, v, *args)
+    np.testing.assert_allclose(out2, out, rtol=1e-9, atol=1e-12)
+    out3 = oracle.sink_window_attn.stream_outputs(q, k, -2.5 * v, *args)
+    np.testing.assert_allclose(out3, -2.5 * out, rtol=1e-12, atol=1e-12)
