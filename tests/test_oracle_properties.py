@@ -14,7 +14,9 @@ properties are ones the mathematics fixes for every such draw:
 - gate logits up to +-60 give gates in range, and the C oracle's logit mode
   equals the numpy recurrence on numpy's gates;
 - the attention oracle's outputs are convex combinations of the visible
-  values, unchanged by a common shift of the keys, linear in the values.
+  values, unchanged by a common shift of the keys, linear in the values;
+- the bidirectional gradients are the forward scan's plus the flipped
+  gradients of the flipped scan from zero.
 """
 import numpy as np
 from hypothesis import given, settings
@@ -200,3 +202,25 @@ def test_attention_is_a_convex_combination_invariant_to_a_key_shift(p):
     np.testing.assert_allclose(out2, out, rtol=1e-9, atol=1e-12)
     out3 = oracle.sink_window_attn.stream_outputs(q, k, -2.5 * v, *args)
     np.testing.assert_allclose(out3, -2.5 * out, rtol=1e-12, atol=1e-12)
+
+
+@SETTINGS
+@given(shapes)
+def test_bidirectional_gradients_are_the_two_scans_gradients(p):
+    """Bidirectional mode is the forward scan plus the forward scan of the
+    flipped chunk from zero, so its gradients are the forward scan's plus the
+    flipped gradients of the flipped scan (which has no state gradient)."""
+    rng, q, k, v, g, beta, s = draw(p)
+    do = rng.standard_normal(v.shape)
+    dS = rng.standard_normal((1, p["H"], p["Dk"], p["Dv"]))
+    both = oracle.backward.grads(q, k, v, g, beta, s, do, dS, bidir=True)
+    fwd = oracle.backward.grads(q, k, v, g, beta, s, do, dS, bidir=False)
+    f = lambda x: np.flip(x, axis=1).copy()  # noqa: E731
+    rev = oracle.backward.grads(f(q), f(k), f(v), f(g), f(beta), None, f(do), None, bidir=False)
+    names = ["dq", "dk", "dv", "dg", "dbeta"]
+    scale = max(np.max(np.abs(both[n])) for n in names)
+    for n in names:
+        np.testing.assert_allclose(both[n], fwd[n] + f(rev[n]), rtol=1e-10, atol=1e-13 * scale,
+                                   err_msg=n)
+    if s is not None:
+        np.testing.assert_allclose(both["dstate_in"], fwd["dstate_in"], rtol=1e-12, atol=1e-14)
