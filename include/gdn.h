@@ -37,7 +37,10 @@
  * a scratch, the call allocates stream-ordered (cudaMallocAsync /
  * cudaFreeAsync, captured as graph memory nodes) and reports through the
  * device-wide error word.  Make one call on a stream before capturing on it
- * to keep memory nodes out of the graph.
+ * to keep memory nodes out of the graph.  Contexts are found by the stream's
+ * handle, and cudaStreamDestroy returns before the stream's work is done: let
+ * a stream's calls finish before destroying it, since a stream created
+ * afterwards may get the same handle, and with it the same scratch.
  *
  * Execution.  Work is enqueued on `stream` (a cudaStream_t; NULL is the
  * legacy default stream) and the call returns without synchronising;
