@@ -40,6 +40,7 @@ def test_status_strings_and_version():
     names = [lib.gdn_status_string(i).decode() for i in range(6)]
     assert names == ["GDN_OK", "GDN_ERR_INVALID_ARG", "GDN_ERR_UNSUPPORTED",
                      "GDN_ERR_ALIAS", "GDN_ERR_CUDA", "GDN_ERR_TIMEOUT"]
+    assert lib.gdn_status_string(6).decode() == "GDN_ERR_SCRATCH_LIMIT"
     assert lib.gdn_status_string(99).decode() == "GDN_ERR_UNKNOWN"
     assert lib.gdn_version() >= 100
 
