@@ -6,7 +6,7 @@
 // reverse mode of the chunked forward the bf16 path computes.  Per 64-token
 // chunk, in scan order, entered with state S0 (Dk x Dv) and left with S_e:
 //
-//   A_pi = beta_p e^{g_p - g_i} k^_p . k^_i (i < p),  T = (I + A)^-1
+//   A_pi = beta_p e^{gam_p - gam_i} k^_p . k^_i (i < p),  T = (I + A)^-1
 //   X_w = diag(beta e^gam) K^,  X_u = diag(beta) V,  W = T X_w,  U~ = T X_u
 //   U = U~ - W S0,  P = M o (Q^ K^T) with M_pi = e^{gam_p - gam_i} (i <= p)
 //   O = diag(e^gam) Q^ S0 + P U,  S_e = e^{gam_C} S0 + K~^T U,  K~ = diag(e^{gam_C - gam}) K^
